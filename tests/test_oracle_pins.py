@@ -1,0 +1,389 @@
+"""Pins for the float64 oracle: closed forms, textbook special cases, brute
+force and LAPACK.  None of these re-types the oracle's own formula; each
+would fail on a dropped term, a wrong sign or index, or a transposed operand
+somewhere in the oracle."""
+import json
+import os
+from math import sqrt
+
+import numpy as np
+import pytest
+
+from oracle import prism_ref as o
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def rot(n, seed):
+    Q, Rq = np.linalg.qr(np.random.default_rng(seed).standard_normal((n, n)))
+    return Q * np.sign(np.diag(Rq))
+
+
+def spd(n, lam, seed):
+    Q = rot(n, seed)
+    return (Q * lam) @ Q.T, Q
+
+
+# ---------------------------------------------------------------- Gram EMA
+def test_ema_rank_one_closed_form():
+    m, n, i, j, s, beta, eps, e0 = 6, 4, 2, 3, 1.7, 0.95, 1e-3, 0.25
+    G = np.zeros((m, n)); G[i, j] = s
+    L, R = o.gram_ema_ref(G, e0 * np.eye(m), e0 * np.eye(n), beta, eps)
+    for k in range(m):
+        want = beta * e0 + eps + ((1 - beta) * s * s if k == i else 0.0)
+        assert L[k, k] == pytest.approx(want, rel=1e-15)
+    for k in range(n):
+        want = beta * e0 + eps + ((1 - beta) * s * s if k == j else 0.0)
+        assert R[k, k] == pytest.approx(want, rel=1e-15)
+    assert np.count_nonzero(L - np.diag(np.diag(L))) == 0
+    assert np.count_nonzero(R - np.diag(np.diag(R))) == 0
+
+
+def test_ema_orthogonal_gradient_closed_form():
+    n, s, beta, eps = 12, 0.3, 0.9, 1e-8
+    Q = rot(n, 1)
+    L = R = eps * np.eye(n)
+    ell = eps
+    for _ in range(7):
+        L, R = o.gram_ema_ref(s * Q, L, R, beta, eps)
+        ell = beta * ell + (1 - beta) * s * s + eps       # scalar recursion
+    np.testing.assert_allclose(L, ell * np.eye(n), atol=1e-15)
+    np.testing.assert_allclose(R, ell * np.eye(n), atol=1e-15)
+
+
+def test_ema_trace_symmetry_psd():
+    rng = np.random.default_rng(3)
+    m, n, beta, eps = 9, 5, 0.95, 1e-6
+    G = rng.standard_normal((m, n))
+    L0, R0 = eps * np.eye(m), eps * np.eye(n)
+    L, R = o.gram_ema_ref(G, L0, R0, beta, eps)
+    fro2 = np.sum(G * G)
+    assert np.trace(L - beta * L0) - m * eps == pytest.approx((1 - beta) * fro2, rel=1e-13)
+    assert np.trace(R - beta * R0) - n * eps == pytest.approx((1 - beta) * fro2, rel=1e-13)
+    assert np.array_equal(L, L.T) and np.array_equal(R, R.T)
+    assert np.linalg.eigvalsh(L).min() > 0 and np.linalg.eigvalsh(R).min() > 0
+
+
+def test_ema_row_vs_column_covariance():
+    # L is the row covariance (m x m) and R the column covariance (n x n):
+    # a gradient whose rows are identical has a rank-one R direction set by the row.
+    m, n = 5, 3
+    row = np.array([1.0, -2.0, 0.5])
+    G = np.tile(row, (m, 1))
+    L, R = o.gram_ema_ref(G, np.zeros((m, m)), np.zeros((n, n)), 0.0, 0.0)
+    np.testing.assert_allclose(R, m * np.outer(row, row), rtol=1e-15)
+    np.testing.assert_allclose(L, np.full((m, m), row @ row), rtol=1e-15)
+
+
+# ---------------------------------------------------------- polynomials
+def test_taylor_series_of_inverse_sqrt():
+    # (1 - x)^(-1/2) = 1 + x/2 + 3x^2/8 + 5x^3/16 + 35x^4/128 + ...
+    np.testing.assert_allclose(o.taylor_coeffs(4), [1, 0.5, 0.375, 0.3125, 35 / 128], rtol=0)
+
+
+def test_golden_interval_is_taylor_to_one():
+    page = json.load(open(os.path.join(HERE, "golden", "page_constants.json")))
+    lo, hi = page["alpha_interval_d1"]["value"]
+    # alpha = lo must reproduce the plain Taylor update (classic Newton-Schulz)
+    assert o.taylor_coeffs(1)[1] == lo
+    np.testing.assert_allclose(o.g_coeffs(1, lo), [1.0, 0.5])
+    assert hi == 1.0
+    assert page["root_exponent"]["value"] == -0.25
+
+
+def test_classic_newton_schulz_residual():
+    # d=1, alpha=1/2: g = (3 - x)/2 in terms of x = 1 - xi; textbook residual 3/4 xi^2 + 1/4 xi^3
+    np.testing.assert_allclose(o.residual_coeffs(1, 0.5), [0, 0, 0.75, 0.25], atol=1e-15)
+    # d=2, alpha=3/8 is the third-order Newton-Schulz (15 - 10 x + 3 x^2)/8: no xi^2 term
+    r = o.residual_coeffs(2, 0.375)
+    assert abs(r[2]) < 1e-15 and abs(r[0]) < 1e-15 and abs(r[1]) < 1e-15
+    x = np.linspace(-0.3, 1.0, 17)
+    g_textbook = (15 - 10 * x + 3 * x * x) / 8
+    np.testing.assert_allclose(np.polynomial.polynomial.polyval(1 - x, o.g_coeffs(2, 0.375)),
+                               g_textbook, rtol=1e-14)
+
+
+@pytest.mark.parametrize("d", [1, 2, 3])
+def test_residual_table_matches_polynomial(d):
+    T = o.residual_alpha_table(d)
+    for a in (0.0, 0.3, 0.5, 1.0, -0.7):
+        via_table = T[:, 0] + T[:, 1] * a + T[:, 2] * a * a
+        np.testing.assert_allclose(via_table, o.residual_coeffs(d, a), atol=1e-14)
+    # r vanishes below degree d for every alpha, and r(1; alpha) = 1 (X = 0 is a fixed point)
+    assert np.all(T[:d] == 0)
+    for a in (0.2, 0.9):
+        assert np.polynomial.polynomial.polyval(1.0, o.residual_coeffs(d, a)) == pytest.approx(1.0)
+
+
+def ideal_alpha(d, xi):
+    """alpha that makes (1 - xi) g(xi)^2 = 1 exactly for a scalar residual xi."""
+    f = sum(o.taylor_coeffs(d)[j] * xi ** j for j in range(d))
+    return (1 / sqrt(1 - xi) - f) / xi ** d
+
+
+@pytest.mark.parametrize("d,xi,want", [
+    (1, 0.5, 2 * sqrt(2) - 2),        # 0.828427...
+    (1, 0.75, 1.0),                   # ideal 4/3, clamped to the upper end
+    (1, -0.5, 0.5),                   # ideal 0.367, clamped to the lower end
+    (2, 0.5, (sqrt(2) - 1.25) * 4),   # 0.656854...
+    (2, 0.1, None),
+])
+def test_alpha_closed_form_scalar_residual(d, xi, want):
+    n, p = 8, 3
+    lo, hi = (0.5, 1.0) if d == 1 else (0.375, 1.0)
+    S = np.random.default_rng(7).standard_normal((n, p))
+    a, coef = o.prism_alpha_ref(xi * np.eye(n), S, d, lo, hi)
+    if want is None:
+        want = ideal_alpha(d, xi)
+        assert lo < want < hi
+    assert a == pytest.approx(want, abs=1e-9)
+
+
+def _grid_alpha(Rk, S, d, lo, hi, step=1e-6):
+    """Brute force: evaluate ||(I - (I - R) g(R)^2) S||_F^2 on a grid, from the
+    matrix identity itself (no coefficient table, no Gram matrix)."""
+    n = Rk.shape[0]
+    I = np.eye(n)
+    f = np.eye(n) if d == 1 else I + 0.5 * Rk
+    Rd = np.linalg.matrix_power(Rk, d)
+    F, Fd = f @ S, Rd @ S
+    # g(R) S = F + a Fd, and (I-R) g(R)^2 S = (I-R) g(R) (F + a Fd)
+    gF, gFd = f @ F, f @ Fd
+    RdF, RdFd = Rd @ F, Rd @ Fd
+    A0 = S - (I - Rk) @ gF
+    A1 = -(I - Rk) @ (gFd + RdF)
+    A2 = -(I - Rk) @ RdFd
+    grid = np.arange(lo, hi + step / 2, step)
+    best, besta = np.inf, None
+    for chunk in np.array_split(grid, 50):
+        a = chunk[:, None, None]
+        vals = np.sum((A0[None] + a * A1[None] + a * a * A2[None]) ** 2, axis=(1, 2))
+        k = int(np.argmin(vals))
+        if vals[k] < best:
+            best, besta = vals[k], chunk[k]
+    return besta
+
+
+@pytest.mark.parametrize("kind", ["diag", "rotated", "symmetric", "nonsymmetric"])
+@pytest.mark.parametrize("p", [1, 2, 4, 8])
+@pytest.mark.parametrize("d", [1, 2])
+def test_alpha_brute_force_8x8(kind, p, d):
+    rng = np.random.default_rng(100 * p + d + len(kind))
+    n = 8
+    lam = rng.uniform(0.05, 0.95, n)
+    if kind == "diag":
+        Rk = np.diag(lam)
+    elif kind == "rotated":
+        Q = rot(n, 5)
+        Rk = (Q * lam) @ Q.T
+    elif kind == "symmetric":
+        M = rng.standard_normal((n, n)); Rk = 0.15 * (M + M.T)
+    else:
+        Rk = np.diag(lam) + 0.05 * rng.standard_normal((n, n))
+    S = rng.standard_normal((n, p))
+    lo, hi = (0.5, 1.0) if d == 1 else (0.375, 1.0)
+    a, _ = o.prism_alpha_ref(Rk, S, d, lo, hi)
+    assert a == pytest.approx(_grid_alpha(Rk, S, d, lo, hi), abs=2e-6)
+
+
+@pytest.mark.parametrize("d", [1, 2])
+def test_alpha_exact_trace_objective(d):
+    # p = n with an orthogonal sketch: the sketched objective is the exact
+    # spectral least-squares objective sum_i r(lambda_i; alpha)^2.
+    n = 10
+    rng = np.random.default_rng(11)
+    M = rng.standard_normal((n, n)); Rk = 0.2 * (M + M.T)
+    S = rot(n, 12)
+    _, coef = o.prism_alpha_ref(Rk, S, d, 0.3, 1.0)
+    lam = np.linalg.eigvalsh(Rk)
+    P = np.polynomial.polynomial
+    for a in (0.1, 0.4, 0.8, 1.3):
+        r_of_lam = 1 - (1 - lam) * P.polyval(lam, o.g_coeffs(d, a)) ** 2
+        assert P.polyval(a, coef) == pytest.approx(np.sum(r_of_lam ** 2), rel=1e-10)
+
+
+def test_alpha_constant_objective_takes_lower_end():
+    a, coef = o.prism_alpha_ref(np.zeros((6, 6)), np.ones((6, 2)), 2, 0.375, 1.0)
+    assert a == 0.375
+
+
+# ------------------------------------------------------- Newton-Schulz passes
+def scalar_coupled(lam, alphas, d):
+    """Eigenvalue-domain recurrence: y <- y g(1 - z y), z <- g(1 - z y) z."""
+    y, z = lam.copy(), np.ones_like(lam)
+    for a in alphas:
+        xi = 1 - z * y
+        c = o.taylor_coeffs(d).copy(); c[d] = a
+        g = sum(c[j] * xi ** j for j in range(d + 1))
+        y, z = y * g, g * z
+    return y, z
+
+
+@pytest.mark.parametrize("d", [1, 2])
+@pytest.mark.parametrize("rotated", [False, True])
+def test_coupled_matches_scalar_recurrence(d, rotated):
+    n = 16
+    lam = np.exp(np.random.default_rng(2).uniform(np.log(1e-3), 0, n))
+    Q = rot(n, 4) if rotated else np.eye(n)
+    B = (Q * lam) @ Q.T
+    opts = o.PrismOpts(d=d, p=4, lo=0.5 if d == 1 else 0.375, tol=1e-13, max_iter=60,
+                       stall_below=0.0)
+    S = np.random.default_rng(5).standard_normal((200, n, 4))
+    Y, Z, info = o.coupled_ref(B, opts, S)
+    assert info.status == o.OK
+    y, z = scalar_coupled(lam, info.alpha, d)
+    np.testing.assert_allclose(Y, (Q * y) @ Q.T, atol=1e-12)
+    np.testing.assert_allclose(Z, (Q * z) @ Q.T, atol=1e-9 * np.max(z))
+    np.testing.assert_allclose(y, np.sqrt(lam), rtol=1e-11)
+    np.testing.assert_allclose(z, 1 / np.sqrt(lam), rtol=1e-11)
+
+
+def test_textbook_coupled_newton_schulz():
+    # d=1 with alpha fixed at 1/2:  Y <- Y (3I - ZY)/2,  Z <- (3I - ZY) Z / 2
+    n = 12
+    B, _ = spd(n, np.linspace(0.2, 0.9, n), 8)
+    opts = o.PrismOpts(d=1, p=2, lo=0.5, hi=1.0, tol=0.0, max_iter=6, fixed_alpha=True,
+                       stall_below=0.0)
+    Y, Z, info = o.coupled_ref(B, opts, None)
+    Yt, Zt = B.copy(), np.eye(n)
+    for _ in range(6):
+        T = 3 * np.eye(n) - Zt @ Yt
+        Yt, Zt = Yt @ T / 2, T @ Zt / 2
+    np.testing.assert_allclose(Y, Yt, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(Z, Zt, rtol=1e-14, atol=1e-15)
+    assert info.iters == 6 and info.status == o.ENOCONV
+
+
+@pytest.mark.parametrize("d", [1, 2])
+def test_inverse_roots_vs_eigh_and_identities(d):
+    n = 32
+    lam = np.exp(np.random.default_rng(9).uniform(np.log(1e-2), np.log(3.0), n))
+    A, Q = spd(n, lam, 10)
+    opts = o.PrismOpts(d=d, p=4, lo=0.5 if d == 1 else 0.375, tol=1e-13, max_iter=60,
+                       stall_below=0.0)
+    S = np.random.default_rng(6).standard_normal((200, n, 4))
+    X4, infos = o.inv_root_ref(A, o.POW_INV4, opts, S)
+    assert [i.status for i in infos] == [o.OK, o.OK]
+    np.testing.assert_allclose(X4, (Q * lam ** -0.25) @ Q.T, atol=1e-10)
+    np.testing.assert_allclose(X4 @ X4 @ X4 @ X4 @ A, np.eye(n), atol=1e-9)
+    np.testing.assert_allclose(X4 @ A, A @ X4, atol=1e-9)
+    np.testing.assert_allclose(X4, X4.T, atol=1e-10)
+    X2, _ = o.inv_root_ref(A, o.POW_INV2, opts, S)
+    np.testing.assert_allclose(X2 @ X2 @ A, np.eye(n), atol=1e-9)
+    Xs, _ = o.inv_root_ref(A, o.POW_SQRT, opts, S)
+    np.testing.assert_allclose(Xs @ Xs, A, atol=1e-10)
+
+
+def test_eigh_reference_on_diagonal():
+    lam = np.array([4.0, 1.0, 0.0625, 16.0])
+    np.testing.assert_allclose(o.spd_power_eigh(np.diag(lam), -0.25),
+                               np.diag([1 / sqrt(2), 1.0, 2.0, 0.5]), atol=1e-15)
+
+
+# ---------------------------------------------------------------- polar
+@pytest.mark.parametrize("shape", [(40, 12), (12, 40), (16, 16)])
+def test_polar_orthonormal_and_svd(shape):
+    rng = np.random.default_rng(sum(shape))
+    G = rng.standard_normal(shape)
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=60, stall_below=0.0)
+    S = rng.standard_normal((100, min(shape), 4))
+    X, infos = o.polar_ref(G, opts, S)
+    assert infos[0].status == o.OK
+    k = min(shape)
+    XtX = X.T @ X if shape[0] >= shape[1] else X @ X.T
+    np.testing.assert_allclose(XtX, np.eye(k), atol=1e-11)
+    np.testing.assert_allclose(X, o.polar_svd(G), atol=1e-10)
+
+
+def test_polar_error_bounded_by_residual():
+    rng = np.random.default_rng(21)
+    G = rng.standard_normal((30, 10))
+    U = o.polar_svd(G)
+    for it in (2, 4, 6):
+        opts = o.PrismOpts(d=1, p=3, lo=0.5, tol=0.0, max_iter=it, stall_below=0.0)
+        X, infos = o.polar_ref(G, opts, rng.standard_normal((10, 10, 3)))
+        resid = np.linalg.norm(np.eye(10) - X.T @ X)
+        assert np.linalg.norm(X - U) <= resid + 1e-14
+
+
+def test_polar_of_orthonormal_is_itself():
+    Q = rot(20, 30)[:, :8]
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=60, stall_below=0.0)
+    X, _ = o.polar_ref(Q, opts, np.random.default_rng(1).standard_normal((60, 8, 4)))
+    np.testing.assert_allclose(X, Q, atol=1e-12)
+
+
+def test_polar_textbook_and_singular_value_recurrence():
+    # d=1, alpha=1/2: X <- X (3I - X^T X)/2 ; on a diagonal input each singular
+    # value follows s <- s (3 - s^2)/2.
+    sig = np.array([3.0, 1.0, 0.2, 0.05])
+    G = np.zeros((6, 4)); G[:4, :4] = np.diag(sig)
+    opts = o.PrismOpts(d=1, p=2, lo=0.5, tol=0.0, max_iter=5, fixed_alpha=True, stall_below=0.0)
+    X, _ = o.polar_ref(G, opts, None)
+    s = sig / np.linalg.norm(sig)
+    for _ in range(5):
+        s = s * (3 - s * s) / 2
+    want = np.zeros((6, 4)); want[:4, :4] = np.diag(s)
+    np.testing.assert_allclose(X, want, atol=1e-15)
+
+
+# ---------------------------------------------------------------- apply / step
+def test_apply_closed_forms():
+    rng = np.random.default_rng(4)
+    W, G = rng.standard_normal((5, 3)), rng.standard_normal((5, 3))
+    np.testing.assert_allclose(o.apply_ref(W, G, np.eye(5), np.eye(3), 0.1), W - 0.1 * G)
+    a, b = rng.uniform(1, 2, 5), rng.uniform(1, 2, 3)
+    got = o.apply_ref(W, G, np.diag(a), np.diag(b), 0.01)
+    for i in range(5):
+        for j in range(3):
+            assert got[i, j] == pytest.approx(W[i, j] - 0.01 * a[i] * G[i, j] * b[j], rel=1e-15)
+
+
+def test_shampoo_step_vs_eigh():
+    rng = np.random.default_rng(8)
+    m, n, eps, beta, lr = 16, 8, 1e-6, 0.95, 1e-3
+    W = 0.02 * rng.standard_normal((m, n))
+    Gs = [0.02 * rng.standard_normal((m, n)) for _ in range(4)]
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=80, stall_below=0.0)
+    S = rng.standard_normal((200, n, 4))
+    # L is m x m and R is n x n, so each gets a sketch of its own size
+    L, R = eps * np.eye(m), eps * np.eye(n)
+    for G in Gs:
+        L = beta * L + (1 - beta) * G @ G.T + eps * np.eye(m)
+        R = beta * R + (1 - beta) * G.T @ G + eps * np.eye(n)
+    SL = rng.standard_normal((200, m, 4))
+    PL, _ = o.inv_root_ref(L, o.POW_INV4, opts, SL)
+    PR, _ = o.inv_root_ref(R, o.POW_INV4, opts, S)
+    np.testing.assert_allclose(PL, o.spd_power_eigh(L, -0.25), rtol=1e-8, atol=1e-8 * np.abs(PL).max())
+    np.testing.assert_allclose(PR, o.spd_power_eigh(R, -0.25), rtol=1e-8, atol=1e-8 * np.abs(PR).max())
+    Wn = o.apply_ref(W, Gs[-1], PL, PR, lr)
+    want = W - lr * o.spd_power_eigh(L, -0.25) @ Gs[-1] @ o.spd_power_eigh(R, -0.25)
+    np.testing.assert_allclose(Wn - W, want - W, rtol=1e-7, atol=1e-9 * np.abs(want - W).max())
+
+
+def test_shampoo_step_ref_square():
+    rng = np.random.default_rng(18)
+    n, eps, beta, lr = 12, 1e-6, 0.95, 1e-3
+    W = 0.02 * rng.standard_normal((n, n))
+    Gs = [0.02 * rng.standard_normal((n, n)) for _ in range(3)]
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=80, stall_below=0.0)
+    S = rng.standard_normal((200, n, 4))
+    W1, L, R, PL, PR, infos = o.shampoo_step_ref(W, Gs, eps * np.eye(n), eps * np.eye(n),
+                                                 beta, eps, lr, opts, S)
+    want = W - lr * o.spd_power_eigh(L, -0.25) @ Gs[-1] @ o.spd_power_eigh(R, -0.25)
+    np.testing.assert_allclose(W1 - W, want - W, rtol=1e-7, atol=1e-9 * np.abs(want - W).max())
+
+
+# ---------------------------------------------------------------- stop rules
+def test_stop_rules():
+    S = np.random.default_rng(0).standard_normal((10, 4, 2))
+    opts = o.PrismOpts(d=1, p=2, lo=0.5, tol=1e-12, max_iter=1)
+    B = np.diag([0.5, 0.2, 0.1, 0.9])
+    _, _, info = o.coupled_ref(B, opts, S)
+    assert info.status == o.ENOCONV and info.iters == 1 and len(info.res) == 2
+    Bn = B.copy(); Bn[1, 1] = np.nan
+    _, _, info = o.coupled_ref(Bn, opts, S)
+    assert info.status == o.ENONFINITE and info.iters == 0
+    Y, Z, info = o.coupled_ref(np.eye(4), opts, S)
+    assert info.status == o.OK and info.iters == 0 and info.res == [0.0]
+    np.testing.assert_array_equal(Y, np.eye(4))
