@@ -1,0 +1,181 @@
+/*
+ * shampoo_prism.h - C ABI of the B200 (sm_100a) Shampoo preconditioner step
+ * with PRISM-accelerated Newton-Schulz matrix functions.
+ *
+ * Sources of the operations (page title, section):
+ *   [Shampoo]  "深度学习中的优化器之Shampoo算法原理与二阶优化机制"
+ *              (algorithm.idocdown.com): 2.2-2.3 statistics and update,
+ *              3.1 matrix roots, 3.2 block-diagonal approximation,
+ *              6.3 shampoo_update(W, G, L, R, beta, epsilon, lr).
+ *   [PRISM]    "Sintesi Tecnica: PRISM" (gist.science): Parte I residual-form
+ *              iteration X_{k+1} = X_k f(R_k); Parte II.1 polynomial
+ *              g_d(xi; alpha) = f_{d-1}(xi) + alpha xi^d, alpha fitted by least
+ *              squares and constrained to [l, u]; Parte II.2 Gaussian sketch.
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are fp32 (or bf16 where stated), row-major, contiguous, and a
+ *     batch of B matrices is B consecutive matrices (stride rows*cols).
+ *   - Every pointer argument is DEVICE memory owned by the caller unless it is
+ *     documented as host memory.  The library never allocates, frees or keeps
+ *     a caller pointer after the call returns; scratch memory is the caller's
+ *     `ws` buffer of at least shp_workspace_bytes(...) bytes, 256-byte aligned.
+ *   - Column counts of fp32 matrices must be multiples of 4 and of bf16
+ *     matrices multiples of 8 (16-byte rows for the tensor-memory-access
+ *     unit); base pointers must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronise the host.
+ *   - The return value is decided before any launch: SHP_OK, SHP_EINVAL
+ *     (bad argument, nothing launched), SHP_EUNSUPPORTED, or SHP_ECUDA (a
+ *     CUDA runtime error at launch; the stream may hold partial work).
+ *     Numerical outcomes are per-block codes written to `report.status` on the
+ *     device; the caller reads them after synchronising the stream.
+ *   - No exceptions cross this boundary; the library keeps no state between
+ *     calls other than cached kernel attributes.
+ */
+#ifndef SHAMPOO_PRISM_H
+#define SHAMPOO_PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* shp_stream; /* cudaStream_t */
+
+typedef enum {
+  SHP_OK = 0,
+  SHP_EINVAL = 1,
+  SHP_EUNSUPPORTED = 2,
+  SHP_ECUDA = 3,
+  /* per-block outcomes, written to report.status */
+  SHP_ENOCONV = 16,    /* max_iter update steps taken, residual still above tol  */
+  SHP_ESTALL = 17,     /* residual stopped shrinking once small (precision floor) */
+  SHP_ENONFINITE = 18, /* residual became NaN or Inf                              */
+  SHP_ETIMEOUT = 19    /* a bounded wait inside a kernel ran out                  */
+} shp_status;
+
+typedef enum {
+  SHP_TF32 = 0,   /* fp32 storage, products on TF32 tensor cores                  */
+  SHP_3XTF32 = 1, /* fp32 storage split as hi (TF32) + lo; acc += hh + hl + lh     */
+  SHP_BF16 = 2    /* bf16 storage, fp32 accumulation (polar factor only)           */
+} shp_precision;
+
+typedef enum {
+  SHP_POW_INV4 = 0, /* A^(-1/4): the Shampoo preconditioner power ([Shampoo] 2.3) */
+  SHP_POW_INV2 = 1, /* A^(-1/2)                                                    */
+  SHP_POW_SQRT = 2  /* A^(1/2)                                                     */
+} shp_power;
+
+typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_OP_APPLY = 3,
+               SHP_OP_GRAM_EMA = 4 } shp_op;
+
+/* Knobs of a PRISM Newton-Schulz pass ([PRISM] Parte I-II).
+ *   d           degree of g_d; 1 or 2
+ *   p           sketch width, 1..32
+ *   lo, hi      alpha interval [l, u]; [1/2, 1] for d = 1 as printed, the
+ *               Taylor coefficient 3/8 and 1 for d = 2
+ *   tol         stop when ||R_k||_F / sqrt(n) <= tol (checked before an update)
+ *   max_iter    at most this many update steps per pass (<= 256)
+ *   prec        SHP_TF32 / SHP_3XTF32 (SHP_BF16 only for polar storage)
+ *   fixed_alpha 1: alpha = lo every step (plain Taylor Newton-Schulz)
+ *   stall_below, stall_ratio: stop with SHP_ESTALL when the previous residual
+ *               is below stall_below and the new one exceeds stall_ratio times it
+ */
+typedef struct {
+  int d;
+  int p;
+  float lo, hi;
+  float tol;
+  int max_iter;
+  int prec;
+  int fixed_alpha;
+  float stall_below;
+  float stall_ratio;
+} shp_prism_opts;
+
+/* Optional per-block trajectory, all device pointers, each may be NULL.
+ *   status [B]                      final shp_status of the block
+ *   iters  [B][2]                   update steps in pass 1 and pass 2
+ *   resid  [B][2][max_iter + 1]     ||R_k||_F / sqrt(n) at every k
+ *   alpha  [B][2][max_iter]         alpha_k used at every update
+ * Entries after a block stops are left untouched. */
+typedef struct {
+  int32_t* status;
+  int32_t* iters;
+  float* resid;
+  float* alpha;
+} shp_prism_report;
+
+/* Bytes of scratch the call `op` needs for these sizes (0 if none).  For
+ * SHP_OP_INV_ROOT / SHP_OP_ALPHA_FIT m is ignored (pass n); for SHP_OP_POLAR
+ * and SHP_OP_APPLY m x n is the matrix shape.  Returns 0 on bad arguments. */
+size_t shp_workspace_bytes(int op, int64_t m, int64_t n, int64_t batch,
+                           const shp_prism_opts* opts);
+
+/* Kronecker-factor statistics, one EMA step ([Shampoo] 2.2-2.3, step 2):
+ *   L <- beta L + (1 - beta) G G^T + eps I      (L: m x m, in place)
+ *   R <- beta R + (1 - beta) G^T G + eps I      (R: n x n, in place)
+ * G: [batch][m][n] fp32; L: [batch][m][m]; R: [batch][n][n].
+ * prec: SHP_TF32 or SHP_3XTF32 (the latter needs workspace for the split G).
+ * Either L or R may be NULL to skip that factor. */
+int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float* L, float* R,
+                     float beta, float eps, int prec, void* ws, size_t ws_bytes,
+                     shp_stream stream);
+
+/* Matrix power of a batch of SPD matrices by coupled Newton-Schulz with PRISM
+ * alpha ([PRISM] Parte I-II; [Shampoo] 2.3 step 3 and 3.1):
+ *   c = ||A||_F, B = A / c;  pass 1: Y_0 = B, Z_0 = I, for k = 0, 1, ...:
+ *   R_k = I - Z_k Y_k, stop test, alpha_k = argmin_{[lo,hi]} ||r(R_k;alpha) S_k||_F,
+ *   g = g_d(R_k; alpha_k), Y_{k+1} = Y_k g, Z_{k+1} = g Z_k.
+ *   SHP_POW_SQRT -> sqrt(c) Y;  SHP_POW_INV2 -> Z / sqrt(c);
+ *   SHP_POW_INV4 -> pass 2 on Y (same recurrence) and c^(-1/4) Z.
+ * A: [batch][n][n] fp32 SPD; X_out: [batch][n][n] fp32 (may not alias A).
+ * S: [S_count][n][p] fp32 Gaussian sketches shared by the batch; pass 1
+ *   iteration k uses S[k], pass 2 uses S[max_iter + k]; S_count must be
+ *   >= max_iter (one pass) or >= 2 * max_iter (SHP_POW_INV4).
+ * Output of a block that stopped without converging is its last iterate. */
+int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
+                   const shp_prism_opts* opts, const float* S, int64_t S_count, float* X_out,
+                   const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
+
+/* Polar factor U V^T of a batch of m x n matrices (the Muon orthogonalisation;
+ * [PRISM] Parte I with R_k = I - X_k^T X_k):
+ *   X_0 = G / ||G||_F; R_k = I - X_k^T X_k; stop test; alpha_k from S[k];
+ *   X_{k+1} = X_k g_d(R_k; alpha_k).  A wide G (m < n) is handled as G^T.
+ * G, X_out: [batch][m][n], bf16 (storage = SHP_BF16; the iterate is kept in
+ *   bf16 with fp32 accumulation) or fp32 (storage = SHP_TF32 / SHP_3XTF32).
+ * S: [S_count][min(m,n)][p] fp32, S_count >= max_iter. */
+int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
+                const shp_prism_opts* opts, const float* S, int64_t S_count, void* X_out,
+                const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
+
+/* One sketched alpha fit ([PRISM] Parte II.1-II.2) on given residuals:
+ *   V_0 = S, V_j = R V_{j-1} (j <= 2d+1), M_ij = <V_i, V_j>_F (i, j = d..2d+1),
+ *   J(alpha) = sum_ij r_i(alpha) r_j(alpha) M_ij,  alpha* = argmin_{[lo,hi]} J.
+ * R: [batch][n][n] fp32; S: [n][p] fp32 shared by the batch;
+ * alpha_out: [batch] fp32; J_coef_out: [batch][5] fp64 coefficients of
+ * alpha^0..alpha^4, or NULL. */
+int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, int p, int d,
+                    float lo, float hi, float* alpha_out, double* J_coef_out, void* ws,
+                    size_t ws_bytes, shp_stream stream);
+
+/* Preconditioned update ([Shampoo] 2.3 step 4; 6.3):
+ *   W <- W - lr * Lroot * G * Rroot        (in place)
+ * W, G: [batch][m][n]; Lroot: [batch][m][m]; Rroot: [batch][n][n]; fp32.
+ * prec: SHP_TF32 or SHP_3XTF32. */
+int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rroot, int64_t m,
+                  int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
+                  shp_stream stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* shp_status_string(int status);
+
+/* Library version, e.g. "0.1.0" (static storage). */
+const char* shp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHAMPOO_PRISM_H */

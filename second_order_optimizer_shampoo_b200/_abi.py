@@ -1,0 +1,77 @@
+"""ctypes view of the C ABI in include/shampoo_prism.h.
+
+Only marshalling lives here: structure layouts, argument types and the
+loader.  There is no fallback implementation; if the shared library is
+missing the import of any entry point raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libshampoo_prism.so")
+
+# status codes
+SHP_OK, SHP_EINVAL, SHP_EUNSUPPORTED, SHP_ECUDA = 0, 1, 2, 3
+SHP_ENOCONV, SHP_ESTALL, SHP_ENONFINITE, SHP_ETIMEOUT = 16, 17, 18, 19
+# precisions / storage
+SHP_TF32, SHP_3XTF32, SHP_BF16 = 0, 1, 2
+# powers
+SHP_POW_INV4, SHP_POW_INV2, SHP_POW_SQRT = 0, 1, 2
+# workspace queries
+SHP_OP_INV_ROOT, SHP_OP_POLAR, SHP_OP_ALPHA_FIT, SHP_OP_APPLY, SHP_OP_GRAM_EMA = 0, 1, 2, 3, 4
+
+EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar",
+           "prism_alpha_fit", "shampoo_apply", "shp_status_string", "shp_version")
+
+
+class PrismOpts(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("p", ctypes.c_int), ("lo", ctypes.c_float),
+                ("hi", ctypes.c_float), ("tol", ctypes.c_float), ("max_iter", ctypes.c_int),
+                ("prec", ctypes.c_int), ("fixed_alpha", ctypes.c_int),
+                ("stall_below", ctypes.c_float), ("stall_ratio", ctypes.c_float)]
+
+
+class PrismReport(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_void_p), ("iters", ctypes.c_void_p),
+                ("resid", ctypes.c_void_p), ("alpha", ctypes.c_void_p)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+_INT = ctypes.c_int
+
+_SIGS = {
+    "shp_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64, ctypes.POINTER(PrismOpts)]),
+    "shampoo_gram_ema": (_INT, [_P, _I64, _I64, _I64, _P, _P, _F, _F, _INT, _P, _SZ, _P]),
+    "matfn_inv_root": (_INT, [_P, _I64, _I64, _INT, ctypes.POINTER(PrismOpts), _P, _I64, _P,
+                              ctypes.POINTER(PrismReport), _P, _SZ, _P]),
+    "matfn_polar": (_INT, [_P, _INT, _I64, _I64, _I64, ctypes.POINTER(PrismOpts), _P, _I64, _P,
+                           ctypes.POINTER(PrismReport), _P, _SZ, _P]),
+    "prism_alpha_fit": (_INT, [_P, _I64, _I64, _P, _INT, _INT, _F, _F, _P, _P, _P, _SZ, _P]),
+    "shampoo_apply": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P, _SZ, _P]),
+    "shp_status_string": (ctypes.c_char_p, [_INT]),
+    "shp_version": (ctypes.c_char_p, []),
+}
+
+
+def lib():
+    """Load libshampoo_prism.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m second_order_optimizer_shampoo_b200.build_lib` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib

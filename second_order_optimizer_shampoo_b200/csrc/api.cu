@@ -1,0 +1,525 @@
+// C ABI of the library (declared in include/shampoo_prism.h): argument
+// validation, workspace carving and the launch sequence of each operation.
+// Nothing here touches matrix data on the host; every step runs in the
+// kernels of gemm_tc.cu, sketch_alpha.cu and elementwise.cu.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "internal.h"
+#include "shampoo_prism.h"
+
+using namespace shp;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+// Carves aligned sub-buffers out of the caller's workspace.  With a null base
+// it only measures.
+struct Arena {
+  uint8_t* base;
+  size_t used = 0;
+  explicit Arena(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    used = (used + kAlign - 1) & ~(kAlign - 1);
+    T* p = base != nullptr ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool opts_ok(const shp_prism_opts* o) {
+  if (o == nullptr) return false;
+  if (o->d != 1 && o->d != 2) return false;
+  if (o->p < 1 || o->p > 32) return false;
+  if (!(isfinite(o->lo) && isfinite(o->hi)) || o->lo > o->hi) return false;
+  if (!(o->tol >= 0.f)) return false;
+  if (o->max_iter < 1 || o->max_iter > 256) return false;
+  if (o->prec != SHP_TF32 && o->prec != SHP_3XTF32 && o->prec != SHP_BF16) return false;
+  if (!(o->stall_below >= 0.f) || !(o->stall_ratio >= 0.f)) return false;
+  return true;
+}
+
+Ctl carve_ctl(Arena& a, int64_t batch) {
+  Ctl c;
+  c.bs = a.take<BlockState>(batch);
+  c.active = a.take<int>(batch);
+  c.dnorm = a.take<double>(batch);
+  c.tmo = a.take<int>(batch);
+  c.alpha = a.take<float>(batch);
+  return c;
+}
+
+// Iterate buffers: two ping-pong slots for the iterates (Y and Z, or X), and
+// R and g.  `lo` parts exist only in split (3xTF32) mode.
+struct Bufs {
+  float* Yhi[2];
+  float* Ylo[2];
+  float* Zhi[2];
+  float* Zlo[2];
+  float* Rhi;
+  float* Rlo;
+  float* ghi;
+  float* glo;
+  float* V;
+  Ctl ctl;
+};
+
+Bufs carve_inv_root(Arena& a, int64_t n, int64_t batch, const shp_prism_opts* o) {
+  Bufs b;
+  const bool split = o->prec == SHP_3XTF32;
+  const size_t nn = static_cast<size_t>(n) * n * batch;
+  for (int s = 0; s < 2; ++s) {
+    b.Yhi[s] = a.take<float>(nn);
+    b.Ylo[s] = split ? a.take<float>(nn) : nullptr;
+    b.Zhi[s] = a.take<float>(nn);
+    b.Zlo[s] = split ? a.take<float>(nn) : nullptr;
+  }
+  b.Rhi = a.take<float>(nn);
+  b.Rlo = split ? a.take<float>(nn) : nullptr;
+  b.ghi = a.take<float>(nn);
+  b.glo = split ? a.take<float>(nn) : nullptr;
+  b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * n * o->p * batch);
+  b.ctl = carve_ctl(a, batch);
+  return b;
+}
+
+struct PolarBufs {
+  void* Xhi[2];
+  float* Xlo[2];
+  float* Rhi;
+  float* Rlo;
+  void* ghi;
+  float* glo;
+  float* V;
+  Ctl ctl;
+};
+
+PolarBufs carve_polar(Arena& a, int64_t m, int64_t n, int64_t batch, int storage,
+                      const shp_prism_opts* o) {
+  PolarBufs b;
+  const int64_t k = m < n ? m : n;
+  const bool split = storage == SHP_3XTF32;
+  const bool bf = storage == SHP_BF16;
+  const size_t mn = static_cast<size_t>(m) * n * batch, kk = static_cast<size_t>(k) * k * batch;
+  for (int s = 0; s < 2; ++s) {
+    b.Xhi[s] = bf ? static_cast<void*>(a.take<uint16_t>(mn)) : static_cast<void*>(a.take<float>(mn));
+    b.Xlo[s] = split ? a.take<float>(mn) : nullptr;
+  }
+  b.Rhi = a.take<float>(kk);
+  b.Rlo = split ? a.take<float>(kk) : nullptr;
+  b.ghi = bf ? static_cast<void*>(a.take<uint16_t>(kk)) : static_cast<void*>(a.take<float>(kk));
+  b.glo = split ? a.take<float>(kk) : nullptr;
+  b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * k * o->p * batch);
+  b.ctl = carve_ctl(a, batch);
+  return b;
+}
+
+EpiParams epi(int kind, int fmt, void* hi, float* lo, int64_t ldo, int64_t bso, int M, int N,
+              const Ctl* ctl) {
+  EpiParams e;
+  memset(&e, 0, sizeof(e));
+  e.kind = kind;
+  e.out_fmt = fmt;
+  e.out_hi = hi;
+  e.out_lo = lo;
+  e.ldo = ldo;
+  e.bso = bso;
+  e.s0 = 1.f;
+  e.M = M;
+  e.N = N;
+  if (ctl != nullptr) {
+    e.active = ctl->active;
+    e.status = ctl->tmo;
+    e.alpha = ctl->alpha;
+    e.norm2 = &ctl->bs[0].norm2;
+    e.norm2_stride = static_cast<int>(sizeof(BlockState) / sizeof(float));
+  }
+  return e;
+}
+
+Operand op(const void* hi, const float* lo, bool mn, int64_t ld, int64_t bs) {
+  Operand o;
+  o.hi = hi;
+  o.lo = lo;
+  o.mn = mn;
+  o.ld = ld;
+  o.bstride = bs;
+  return o;
+}
+
+#define CK(x)                                  \
+  do {                                         \
+    if ((x) != cudaSuccess) return SHP_ECUDA; \
+  } while (0)
+
+// The sketch passes and the alpha solve of one iteration: V_1 = R S_k,
+// V_j = R V_{j-1} (j <= 2d+1), then the Gram, quartic and argmin.
+int sketch_and_alpha(const float* Rhi, const float* Rlo, int64_t n, int batch, const float* Sk,
+                     float* V, const shp_prism_opts* o, const Ctl& ctl, float* rep_alpha,
+                     int64_t rep_stride, int rep_slot, cudaStream_t st) {
+  const int64_t np = n * o->p;
+  const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
+  if (!o->fixed_alpha) {
+    CK(sketch_pass(Rhi, Rlo, n, n * n, Sk, 0, V + np, vbs, o->p, batch, ctl.active, st));
+    for (int j = 2; j <= 2 * o->d + 1; ++j)
+      CK(sketch_pass(Rhi, Rlo, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
+                     ctl.active, st));
+  }
+  CK(alpha_solve(V, n, o->p, o->d, batch, o->lo, o->hi, o->fixed_alpha, ctl.active, ctl.alpha,
+                 nullptr, rep_alpha, rep_stride, rep_slot, st));
+  return SHP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* shp_version(void) { return "0.1.0"; }
+
+const char* shp_status_string(int s) {
+  switch (s) {
+    case SHP_OK: return "ok";
+    case SHP_EINVAL: return "invalid argument";
+    case SHP_EUNSUPPORTED: return "unsupported";
+    case SHP_ECUDA: return "CUDA runtime error";
+    case SHP_ENOCONV: return "not converged within max_iter";
+    case SHP_ESTALL: return "residual stalled";
+    case SHP_ENONFINITE: return "non-finite residual";
+    case SHP_ETIMEOUT: return "bounded wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t shp_workspace_bytes(int opk, int64_t m, int64_t n, int64_t batch,
+                           const shp_prism_opts* o) {
+  if (n <= 0 || batch <= 0) return 0;
+  Arena a(nullptr);
+  switch (opk) {
+    case SHP_OP_INV_ROOT:
+      if (!opts_ok(o)) return 0;
+      carve_inv_root(a, n, batch, o);
+      break;
+    case SHP_OP_POLAR:
+      if (!opts_ok(o) || m <= 0) return 0;
+      carve_polar(a, m, n, batch, o->prec, o);
+      break;
+    case SHP_OP_ALPHA_FIT: {
+      const int d = o != nullptr ? o->d : 2, p = o != nullptr ? o->p : 32;
+      a.take<float>(static_cast<size_t>(2 * d + 2) * n * p * batch);
+      break;
+    }
+    case SHP_OP_APPLY: {
+      // T = Lroot G (m x n); split mode also needs hi/lo copies of the inputs
+      const int prec = o != nullptr ? o->prec : SHP_3XTF32;
+      const size_t mn = static_cast<size_t>(m) * n * batch;
+      a.take<float>(mn);
+      if (prec == SHP_3XTF32) {
+        a.take<float>(mn);
+        a.take<float>(static_cast<size_t>(m) * m * batch * 2);
+        a.take<float>(mn * 2);
+        a.take<float>(static_cast<size_t>(n) * n * batch * 2);
+      }
+      break;
+    }
+    case SHP_OP_GRAM_EMA: {
+      const int prec = o != nullptr ? o->prec : SHP_3XTF32;
+      if (prec == SHP_3XTF32) a.take<float>(static_cast<size_t>(m) * n * batch * 2);
+      break;
+    }
+    default:
+      return 0;
+  }
+  return a.used + kAlign;
+}
+
+int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float* L, float* R,
+                     float beta, float eps, int prec, void* ws, size_t ws_bytes,
+                     shp_stream stream) {
+  if (G == nullptr || m <= 0 || n <= 0 || batch <= 0 || m % 4 || n % 4) return SHP_EINVAL;
+  if (!aligned16(G) || (L && !aligned16(L)) || (R && !aligned16(R))) return SHP_EINVAL;
+  if (prec != SHP_TF32 && prec != SHP_3XTF32) return SHP_EINVAL;
+  if (!isfinite(beta) || !isfinite(eps)) return SHP_EINVAL;
+  if (m > INT32_MAX || n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float* Ghi = G;
+  const float* Glo = nullptr;
+  if (prec == SHP_3XTF32) {
+    shp_prism_opts o{};
+    o.prec = prec;
+    if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_GRAM_EMA, m, n, batch, &o))
+      return SHP_EINVAL;
+    Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+    float* hi = a.take<float>(static_cast<size_t>(m) * n * batch);
+    float* lo = a.take<float>(static_cast<size_t>(m) * n * batch);
+    CK(split_copy(G, m * n * batch, hi, lo, st));
+    Ghi = hi;
+    Glo = lo;
+  }
+  const int mode = prec == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32;
+  const int M = static_cast<int>(m), N = static_cast<int>(n), B = static_cast<int>(batch);
+  if (L != nullptr) {  // L <- beta L + (1-beta) G G^T + eps I
+    EpiParams e = epi(EPI_EMA, OUT_F32, L, nullptr, m, m * m, M, M, nullptr);
+    e.s0 = beta;
+    e.s1 = 1.f - beta;
+    e.s2 = eps;
+    CK(gemm_tc(mode, op(Ghi, Glo, false, n, m * n), op(Ghi, Glo, false, n, m * n), M, M, N, B, e,
+               st));
+  }
+  if (R != nullptr) {  // R <- beta R + (1-beta) G^T G + eps I
+    EpiParams e = epi(EPI_EMA, OUT_F32, R, nullptr, n, n * n, N, N, nullptr);
+    e.s0 = beta;
+    e.s1 = 1.f - beta;
+    e.s2 = eps;
+    CK(gemm_tc(mode, op(Ghi, Glo, true, n, m * n), op(Ghi, Glo, true, n, m * n), N, N, M, B, e,
+               st));
+  }
+  return SHP_OK;
+}
+
+int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rroot, int64_t m,
+                  int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
+                  shp_stream stream) {
+  if (!W || !G || !Lroot || !Rroot || m <= 0 || n <= 0 || batch <= 0 || m % 4 || n % 4)
+    return SHP_EINVAL;
+  if (!aligned16(W) || !aligned16(G) || !aligned16(Lroot) || !aligned16(Rroot)) return SHP_EINVAL;
+  if (prec != SHP_TF32 && prec != SHP_3XTF32) return SHP_EINVAL;
+  if (m > INT32_MAX || n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  shp_prism_opts o{};
+  o.prec = prec;
+  if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_APPLY, m, n, batch, &o))
+    return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  const size_t mn = static_cast<size_t>(m) * n * batch;
+  const int mode = prec == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32;
+  const int fmt = prec == SHP_3XTF32 ? OUT_SPLIT : OUT_F32;
+  float* Thi = a.take<float>(mn);
+  float* Tlo = prec == SHP_3XTF32 ? a.take<float>(mn) : nullptr;
+  const float *Lh = Lroot, *Ll = nullptr, *Gh = G, *Gl = nullptr, *Rh = Rroot, *Rl = nullptr;
+  if (prec == SHP_3XTF32) {
+    const size_t mm = static_cast<size_t>(m) * m * batch, nn = static_cast<size_t>(n) * n * batch;
+    float* p = a.take<float>(mm * 2);
+    CK(split_copy(Lroot, mm, p, p + mm, st));
+    Lh = p;
+    Ll = p + mm;
+    p = a.take<float>(mn * 2);
+    CK(split_copy(G, mn, p, p + mn, st));
+    Gh = p;
+    Gl = p + mn;
+    p = a.take<float>(nn * 2);
+    CK(split_copy(Rroot, nn, p, p + nn, st));
+    Rh = p;
+    Rl = p + nn;
+  }
+  const int M = static_cast<int>(m), N = static_cast<int>(n), B = static_cast<int>(batch);
+  // T = Lroot G
+  EpiParams e1 = epi(EPI_STORE, fmt, Thi, Tlo, n, m * n, M, N, nullptr);
+  CK(gemm_tc(mode, op(Lh, Ll, false, m, m * m), op(Gh, Gl, true, n, m * n), M, N, M, B, e1, st));
+  // W <- W - lr T Rroot
+  EpiParams e2 = epi(EPI_APPLY, OUT_F32, W, nullptr, n, m * n, M, N, nullptr);
+  e2.s0 = -lr;
+  CK(gemm_tc(mode, op(Thi, Tlo, false, n, m * n), op(Rh, Rl, true, n, n * n), M, N, N, B, e2, st));
+  return SHP_OK;
+}
+
+int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, int p, int d,
+                    float lo, float hi, float* alpha_out, double* J_coef_out, void* ws,
+                    size_t ws_bytes, shp_stream stream) {
+  if (!R || !S || !alpha_out || n <= 0 || batch <= 0 || p < 1 || p > 32 || (d != 1 && d != 2))
+    return SHP_EINVAL;
+  if (!(isfinite(lo) && isfinite(hi)) || lo > hi) return SHP_EINVAL;
+  if (batch > 65535) return SHP_EUNSUPPORTED;
+  shp_prism_opts o{};
+  o.d = d;
+  o.p = p;
+  if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_ALPHA_FIT, n, n, batch, &o))
+    return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  float* V = a.take<float>(static_cast<size_t>(2 * d + 2) * n * p * batch);
+  const int64_t np = n * p, vbs = static_cast<int64_t>(2 * d + 2) * np;
+  const int B = static_cast<int>(batch);
+  CK(sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, st));
+  for (int j = 2; j <= 2 * d + 1; ++j)
+    CK(sketch_pass(R, nullptr, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, p, B, nullptr,
+                   st));
+  CK(alpha_solve(V, n, p, d, B, lo, hi, 0, nullptr, alpha_out, J_coef_out, nullptr, 0, 0, st));
+  return SHP_OK;
+}
+
+int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
+                   const shp_prism_opts* o, const float* S, int64_t S_count, float* X_out,
+                   const shp_prism_report* rep, void* ws, size_t ws_bytes, shp_stream stream) {
+  if (!A || !X_out || !opts_ok(o) || n <= 0 || batch <= 0 || n % 4) return SHP_EINVAL;
+  if (power != SHP_POW_INV4 && power != SHP_POW_INV2 && power != SHP_POW_SQRT) return SHP_EINVAL;
+  if (o->prec != SHP_TF32 && o->prec != SHP_3XTF32) return SHP_EINVAL;
+  const int npass = power == SHP_POW_INV4 ? 2 : 1;
+  if (!o->fixed_alpha && (S == nullptr || S_count < static_cast<int64_t>(npass) * o->max_iter))
+    return SHP_EINVAL;
+  if (!aligned16(A) || !aligned16(X_out)) return SHP_EINVAL;
+  if (n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_INV_ROOT, n, n, batch, o))
+    return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  Bufs w = carve_inv_root(a, n, batch, o);
+  const Ctl& ctl = w.ctl;
+  const bool split = o->prec == SHP_3XTF32;
+  const int mode = split ? MODE_3XTF32 : MODE_TF32;
+  const int fmt = split ? OUT_SPLIT : OUT_F32;
+  const int N = static_cast<int>(n), B = static_cast<int>(batch);
+  const int64_t nn = n * n;
+  const int mi = o->max_iter;
+  float* rep_res = rep != nullptr ? rep->resid : nullptr;
+  float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
+  int* rep_iters = rep != nullptr ? rep->iters : nullptr;
+
+  for (int pass = 0; pass < npass; ++pass) {
+    CK(reset_pass(ctl, B, pass == 0, st));
+    if (pass == 0) {
+      CK(frob_norm2(A, 0, nn, B, ctl, st));
+      CK(coupled_init(A, n, B, ctl, w.Yhi[0], w.Ylo[0], w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo, st));
+    } else {
+      CK(coupled_restart(n, B, ctl, w.Yhi, w.Ylo, w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo, st));
+    }
+    for (int k = 0; k <= mi; ++k) {
+      const int cur = k & 1, nxt = cur ^ 1;
+      if (k > 0) {  // R_k = I - Z_k Y_k and ||R_k||_F^2
+        EpiParams e = epi(EPI_RESID, fmt, w.Rhi, w.Rlo, n, nn, N, N, &ctl);
+        CK(gemm_tc(mode, op(w.Zhi[cur], w.Zlo[cur], false, n, nn),
+                   op(w.Yhi[cur], w.Ylo[cur], true, n, nn), N, N, N, B, e, st));
+      }
+      CK(control_step(ctl, B, n, k, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
+                      2 * (mi + 1), pass * (mi + 1), rep_iters, pass, st));
+      if (k == mi) break;
+      const float* Sk = S != nullptr ? S + static_cast<int64_t>(pass * mi + k) * n * o->p : nullptr;
+      int r = sketch_and_alpha(w.Rhi, w.Rlo, n, B, Sk, w.V, o, ctl, rep_alpha, 2 * mi,
+                               pass * mi + k, st);
+      if (r != SHP_OK) return r;
+      // g = g_d(R_k; alpha_k); at k = 0 (Z_0 = I) it is also Z_1
+      float* z2hi = k == 0 ? w.Zhi[nxt] : nullptr;
+      float* z2lo = k == 0 ? w.Zlo[nxt] : nullptr;
+      if (o->d == 2) {
+        EpiParams e = epi(EPI_GPOLY, fmt, w.ghi, w.glo, n, nn, N, N, &ctl);
+        e.out2_hi = z2hi;
+        e.out2_lo = z2lo;
+        e.aux_hi = w.Rhi;
+        e.aux_lo = w.Rlo;
+        e.lda_aux = n;
+        e.bs_aux = nn;
+        e.s1 = 0.5f;
+        CK(gemm_tc(mode, op(w.Rhi, w.Rlo, false, n, nn), op(w.Rhi, w.Rlo, true, n, nn), N, N, N,
+                   B, e, st));
+      } else {
+        CK(gform_d1(w.Rhi, w.Rlo, n, B, ctl, fmt, w.ghi, w.glo, z2hi, z2lo, st));
+      }
+      {  // Y_{k+1} = Y_k g
+        EpiParams e = epi(EPI_STORE, fmt, w.Yhi[nxt], w.Ylo[nxt], n, nn, N, N, &ctl);
+        CK(gemm_tc(mode, op(w.Yhi[cur], w.Ylo[cur], false, n, nn), op(w.ghi, w.glo, true, n, nn),
+                   N, N, N, B, e, st));
+      }
+      if (k > 0) {  // Z_{k+1} = g Z_k
+        EpiParams e = epi(EPI_STORE, fmt, w.Zhi[nxt], w.Zlo[nxt], n, nn, N, N, &ctl);
+        CK(gemm_tc(mode, op(w.ghi, w.glo, false, n, nn), op(w.Zhi[cur], w.Zlo[cur], true, n, nn),
+                   N, N, N, B, e, st));
+      }
+    }
+  }
+  if (power == SHP_POW_SQRT) {
+    const float* sh[2] = {w.Yhi[0], w.Yhi[1]};
+    const float* sl[2] = {w.Ylo[0], w.Ylo[1]};
+    CK(coupled_finish(n, B, ctl, 0.5, sh, sl, X_out, st));
+  } else {
+    const float* sh[2] = {w.Zhi[0], w.Zhi[1]};
+    const float* sl[2] = {w.Zlo[0], w.Zlo[1]};
+    CK(coupled_finish(n, B, ctl, power == SHP_POW_INV2 ? -0.5 : -0.25, sh, sl, X_out, st));
+  }
+  if (rep != nullptr) CK(write_status(ctl, B, rep->status, st));
+  return SHP_OK;
+}
+
+int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
+                const shp_prism_opts* o, const float* S, int64_t S_count, void* X_out,
+                const shp_prism_report* rep, void* ws, size_t ws_bytes, shp_stream stream) {
+  if (!G || !X_out || !opts_ok(o) || m <= 0 || n <= 0 || batch <= 0) return SHP_EINVAL;
+  if (storage != SHP_TF32 && storage != SHP_3XTF32 && storage != SHP_BF16) return SHP_EINVAL;
+  const bool bf = storage == SHP_BF16;
+  if (bf ? (n % 8 != 0 || m % 8 != 0) : (n % 4 != 0 || m % 4 != 0)) return SHP_EINVAL;
+  if (!o->fixed_alpha && (S == nullptr || S_count < o->max_iter)) return SHP_EINVAL;
+  if (!aligned16(G) || !aligned16(X_out)) return SHP_EINVAL;
+  if (m > INT32_MAX || n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  shp_prism_opts oo = *o;
+  oo.prec = storage;
+  if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_POLAR, m, n, batch, &oo))
+    return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  PolarBufs w = carve_polar(a, m, n, batch, storage, &oo);
+  const Ctl& ctl = w.ctl;
+  const bool tall = m >= n;
+  const int64_t k = tall ? n : m;  // Gram size
+  const int xmode = bf ? MODE_BF16 : (storage == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32);
+  const int xfmt = bf ? OUT_BF16 : (storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32);
+  const int rmode = bf ? MODE_TF32 : xmode;                  // R and R^2
+  const int rfmt = storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32;
+  const int M = static_cast<int>(m), N = static_cast<int>(n), K = static_cast<int>(k);
+  const int B = static_cast<int>(batch);
+  const int64_t mn = m * n, kk = k * k;
+  const int mi = o->max_iter;
+  float* rep_res = rep != nullptr ? rep->resid : nullptr;
+  float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
+  int* rep_iters = rep != nullptr ? rep->iters : nullptr;
+
+  CK(reset_pass(ctl, B, 1, st));
+  CK(frob_norm2(G, bf, mn, B, ctl, st));
+  CK(polar_init(G, bf, mn, B, ctl, xfmt, w.Xhi[0], w.Xlo[0], st));
+  for (int it = 0; it <= mi; ++it) {
+    const int cur = it & 1, nxt = cur ^ 1;
+    {  // R = I - X^T X (tall) or I - X X^T (wide), and ||R||_F^2
+      EpiParams e = epi(EPI_RESID, rfmt, w.Rhi, w.Rlo, k, kk, K, K, &ctl);
+      if (tall)
+        CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], true, n, mn),
+                   op(w.Xhi[cur], w.Xlo[cur], true, n, mn), K, K, M, B, e, st));
+      else
+        CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn),
+                   op(w.Xhi[cur], w.Xlo[cur], false, n, mn), K, K, N, B, e, st));
+    }
+    CK(control_step(ctl, B, k, it, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
+                    2 * (mi + 1), 0, rep_iters, 0, st));
+    if (it == mi) break;
+    const float* Sk = S != nullptr ? S + static_cast<int64_t>(it) * k * o->p : nullptr;
+    int r = sketch_and_alpha(w.Rhi, w.Rlo, k, B, Sk, w.V, o, ctl, rep_alpha, 2 * mi, it, st);
+    if (r != SHP_OK) return r;
+    if (o->d == 2) {  // g = I + R/2 + alpha R^2, stored like X
+      EpiParams e = epi(EPI_GPOLY, xfmt, w.ghi, w.glo, k, kk, K, K, &ctl);
+      e.aux_hi = w.Rhi;
+      e.aux_lo = w.Rlo;
+      e.lda_aux = k;
+      e.bs_aux = kk;
+      e.s1 = 0.5f;
+      CK(gemm_tc(rmode, op(w.Rhi, w.Rlo, false, k, kk), op(w.Rhi, w.Rlo, true, k, kk), K, K, K, B,
+                 e, st));
+    } else {
+      CK(gform_d1(w.Rhi, w.Rlo, k, B, ctl, xfmt, w.ghi, w.glo, nullptr, nullptr, st));
+    }
+    EpiParams e = epi(EPI_STORE, xfmt, w.Xhi[nxt], w.Xlo[nxt], n, mn, M, N, &ctl);
+    if (tall)  // X <- X g
+      CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn), op(w.ghi, w.glo, true, k, kk),
+                 M, N, N, B, e, st));
+    else  // X <- g^T X (the tall iteration applied to X^T)
+      CK(gemm_tc(xmode, op(w.ghi, w.glo, true, k, kk), op(w.Xhi[cur], w.Xlo[cur], true, n, mn),
+                 M, N, M, B, e, st));
+  }
+  const void* sh[2] = {w.Xhi[0], w.Xhi[1]};
+  const float* sl[2] = {w.Xlo[0], w.Xlo[1]};
+  CK(polar_finish(mn, B, ctl, xfmt, sh, sl, X_out, bf ? 1 : 0, st));
+  if (rep != nullptr) CK(write_status(ctl, B, rep->status, st));
+  return SHP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,322 @@
+// Bandwidth-bound helpers of the Newton-Schulz passes: Frobenius norms and
+// normalisation ("no spectral bounds needed": B = A / ||A||_F puts the
+// spectrum in (0, 1]), identity starts, the d = 1 update polynomial
+// g = I + alpha R, TF32 hi/lo splitting, and the final scaling of the root.
+// All are grid-stride loops over [batch][count] with coalesced accesses.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+#include "shp_common.cuh"
+
+namespace shp {
+
+namespace {
+
+constexpr int EW_THREADS = 256;
+
+dim3 ew_grid(int64_t count, int batch) {
+  int64_t per = (count + EW_THREADS * 8 - 1) / (EW_THREADS * 8);
+  if (per < 1) per = 1;
+  if (per > 1024) per = 1024;
+  return dim3(static_cast<unsigned>(per), static_cast<unsigned>(batch));
+}
+
+SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
+  if (fmt == OUT_F32) {
+    static_cast<float*>(hi)[off] = v;
+  } else if (fmt == OUT_SPLIT) {
+    const float h = tf32_round(v);
+    static_cast<float*>(hi)[off] = h;
+    lo[off] = v - h;
+  } else {
+    static_cast<__nv_bfloat16*>(hi)[off] = __float2bfloat16_rn(v);
+  }
+}
+SHP_DEV float get(int fmt, const void* hi, const float* lo, int64_t off) {
+  if (fmt == OUT_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(hi)[off]);
+  float v = static_cast<const float*>(hi)[off];
+  if (fmt == OUT_SPLIT) v += lo[off];
+  return v;
+}
+
+// Block-wide sum of a float partial into an fp32 atomic.
+SHP_DEV void block_add(float v, float* dst) {
+  __shared__ float red[EW_THREADS / 32];
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int w = 0; w < EW_THREADS / 32; ++w) s += red[w];
+    atomicAdd(dst, s);
+  }
+}
+
+__global__ void k_reset(Ctl ctl, int batch, int first) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= batch) return;
+  BlockState& s = ctl.bs[b];
+  if (first) {
+    s.status = ST_OK;
+    s.iters1 = 0;
+    s.c = 0.f;
+    ctl.dnorm[b] = 0.0;
+    ctl.tmo[b] = 0;
+  } else {
+    s.iters1 = s.iters;
+  }
+  s.norm2 = 0.f;
+  s.prev_res = INFINITY;
+  s.iters = 0;
+  s.pass_status = ST_OK;
+  ctl.active[b] = 1;
+  ctl.alpha[b] = 0.f;
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_frob(const void* X, int bf16, int64_t count, double* dnorm) {
+  const int b = blockIdx.y;
+  double acc = 0.0;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const float v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(X)[b * count + e])
+                         : static_cast<const float*>(X)[b * count + e];
+    acc += static_cast<double>(v) * v;
+  }
+  __shared__ double red[EW_THREADS / 32];
+  acc = warp_sum(acc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int w = 0; w < EW_THREADS / 32; ++w) s += red[w];
+    atomicAdd(&dnorm[b], s);
+  }
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_coupled_init(const float* A, int64_t n, Ctl ctl, int fmt, float* Yhi, float* Ylo,
+                   float* Zhi, float* Zlo, float* Rhi, float* Rlo) {
+  const int b = blockIdx.y;
+  const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
+  const int64_t nn = n * n;
+  float nrm = 0.f;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t off = b * nn + e;
+    const bool diag = (e / n) == (e % n);
+    const float y = A[off] / c;
+    const float r = (diag ? 1.f : 0.f) - y;
+    put(fmt, Yhi, Ylo, off, y);
+    put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
+    put(fmt, Rhi, Rlo, off, r);
+    nrm += r * r;
+  }
+  block_add(nrm, &ctl.bs[b].norm2);
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_coupled_restart(int64_t n, Ctl ctl, int fmt, float* Y0hi, float* Y0lo, const float* Y1hi,
+                      const float* Y1lo, float* Zhi, float* Zlo, float* Rhi, float* Rlo) {
+  const int b = blockIdx.y;
+  const bool from1 = (ctl.bs[b].iters1 & 1) != 0;
+  const int64_t nn = n * n;
+  float nrm = 0.f;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t off = b * nn + e;
+    const bool diag = (e / n) == (e % n);
+    float y;
+    if (from1) {
+      y = get(fmt, Y1hi, Y1lo, off);
+      // copy the exact stored pair, not a re-split of its sum
+      Y0hi[off] = Y1hi[off];
+      if (fmt == OUT_SPLIT) Y0lo[off] = Y1lo[off];
+    } else {
+      y = get(fmt, Y0hi, Y0lo, off);
+    }
+    const float r = (diag ? 1.f : 0.f) - y;
+    put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
+    put(fmt, Rhi, Rlo, off, r);
+    nrm += r * r;
+  }
+  block_add(nrm, &ctl.bs[b].norm2);
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_gform_d1(const float* Rhi, const float* Rlo, int64_t n, Ctl ctl, int fmt, void* ghi,
+               float* glo, void* g2hi, float* g2lo) {
+  const int b = blockIdx.y;
+  if (ctl.active[b] == 0) return;
+  const float a = ctl.alpha[b];
+  const int64_t nn = n * n;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t off = b * nn + e;
+    float r = Rhi[off];
+    if (Rlo != nullptr) r += Rlo[off];
+    const float g = (((e / n) == (e % n)) ? 1.f : 0.f) + a * r;
+    put(fmt, ghi, glo, off, g);
+    if (g2hi != nullptr) put(fmt, g2hi, g2lo, off, g);
+  }
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_coupled_finish(int64_t n, Ctl ctl, double e_c, const float* S0hi, const float* S0lo,
+                     const float* S1hi, const float* S1lo, float* X) {
+  const int b = blockIdx.y;
+  const double c = static_cast<double>(ctl.bs[b].c);
+  double sc;
+  if (e_c == 0.5)
+    sc = sqrt(c);
+  else if (e_c == -0.5)
+    sc = 1.0 / sqrt(c);
+  else
+    sc = 1.0 / sqrt(sqrt(c));  // e_c == -0.25
+  const float scale = static_cast<float>(sc);
+  const bool one = (ctl.bs[b].iters & 1) != 0;
+  const float* hi = one ? S1hi : S0hi;
+  const float* lo = one ? S1lo : S0lo;
+  const int64_t nn = n * n;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t off = b * nn + e;
+    float v = hi[off];
+    if (lo != nullptr) v += lo[off];
+    X[off] = scale * v;
+  }
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_split(const float* X, int64_t count, float* hi, float* lo) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const float v = X[e];
+    const float h = tf32_round(v);
+    hi[e] = h;
+    lo[e] = v - h;
+  }
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_polar_init(const void* G, int gbf16, int64_t count, Ctl ctl, int fmt, void* Xhi,
+                 float* Xlo) {
+  const int b = blockIdx.y;
+  const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
+  const float inv = c > 0.f ? 1.f / c : 0.f;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t off = b * count + e;
+    const float v = gbf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(G)[off])
+                          : static_cast<const float*>(G)[off];
+    put(fmt, Xhi, Xlo, off, v * inv);
+  }
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    k_polar_finish(int64_t count, Ctl ctl, int fmt, const void* S0hi, const float* S0lo,
+                   const void* S1hi, const float* S1lo, void* X, int out_bf16) {
+  const int b = blockIdx.y;
+  const bool one = (ctl.bs[b].iters & 1) != 0;
+  const void* hi = one ? S1hi : S0hi;
+  const float* lo = one ? S1lo : S0lo;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
+       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t off = b * count + e;
+    if (out_bf16 && fmt == OUT_BF16) {
+      static_cast<__nv_bfloat16*>(X)[off] = static_cast<const __nv_bfloat16*>(hi)[off];
+    } else {
+      const float v = get(fmt, hi, lo, off);
+      if (out_bf16)
+        static_cast<__nv_bfloat16*>(X)[off] = __float2bfloat16_rn(v);
+      else
+        static_cast<float*>(X)[off] = v;
+    }
+  }
+}
+
+__global__ void k_write_status(Ctl ctl, int batch, int* out) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= batch) return;
+  out[b] = ctl.tmo[b] != 0 ? ST_ETIMEOUT : ctl.bs[b].status;
+}
+
+}  // namespace
+
+cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st) {
+  k_reset<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, first_pass);
+  return cudaGetLastError();
+}
+
+cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
+                       cudaStream_t st) {
+  k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(X, is_bf16, count, ctl.dnorm);
+  return cudaGetLastError();
+}
+
+cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, float* Yhi,
+                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                         cudaStream_t st) {
+  const int fmt = Ylo != nullptr ? OUT_SPLIT : OUT_F32;
+  k_coupled_init<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(A, n, ctl, fmt, Yhi, Ylo, Zhi,
+                                                               Zlo, Rhi, Rlo);
+  return cudaGetLastError();
+}
+
+cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* Yhi,
+                            float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                            cudaStream_t st) {
+  const int fmt = Ylo[0] != nullptr ? OUT_SPLIT : OUT_F32;
+  k_coupled_restart<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(
+      n, ctl, fmt, Yhi[0], Ylo[0], Yhi[1], Ylo[1], Zhi, Zlo, Rhi, Rlo);
+  return cudaGetLastError();
+}
+
+cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, const Ctl& ctl,
+                     int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st) {
+  k_gform_d1<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(Rhi, Rlo, n, ctl, fmt, ghi, glo,
+                                                           g2hi, g2lo);
+  return cudaGetLastError();
+}
+
+cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_exponent,
+                           const float* const* Shi, const float* const* Slo, float* X_out,
+                           cudaStream_t st) {
+  k_coupled_finish<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(n, ctl, c_exponent, Shi[0],
+                                                                 Slo[0], Shi[1], Slo[1], X_out);
+  return cudaGetLastError();
+}
+
+cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st) {
+  if (count <= 0) return cudaSuccess;
+  k_split<<<ew_grid(count, 1), EW_THREADS, 0, st>>>(X, count, hi, lo);
+  return cudaGetLastError();
+}
+
+cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, const Ctl& ctl,
+                       int fmt, void* Xhi, float* Xlo, cudaStream_t st) {
+  k_polar_init<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, g_bf16, count, ctl, fmt, Xhi,
+                                                             Xlo);
+  return cudaGetLastError();
+}
+
+cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
+                         const void* const* Shi, const float* const* Slo, void* X_out,
+                         int out_bf16, cudaStream_t st) {
+  k_polar_finish<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(count, ctl, fmt, Shi[0], Slo[0],
+                                                               Shi[1], Slo[1], X_out, out_bf16);
+  return cudaGetLastError();
+}
+
+cudaError_t write_status(const Ctl& ctl, int batch, int* report_status, cudaStream_t st) {
+  if (report_status == nullptr) return cudaSuccess;
+  k_write_status<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, report_status);
+  return cudaGetLastError();
+}
+
+}  // namespace shp

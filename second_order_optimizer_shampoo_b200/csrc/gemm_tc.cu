@@ -1,0 +1,347 @@
+// Batched GEMM on the sm_100a tensor cores (tcgen05) with fused epilogues.
+//
+// Every dense product of the Shampoo step and of the PRISM Newton-Schulz
+// iteration (G G^T, G^T G, Z_k Y_k, R_k^2, Y_k g, g Z_k, X_k^T X_k, X_k g and
+// the two products of the preconditioned update) runs through this kernel.
+// The PRISM summary ("Sintesi Tecnica: PRISM", Contributi Chiave 3) stresses
+// that the method stays dominated by GEMMs; this is that GEMM.
+//
+// Design (one CTA per 128 x BN output tile, BN in {64, 128, 256}):
+//   warp 0 lane 0  - TMA producer: 128-byte-swizzled tiles of A and B (and of
+//                    their low parts in split mode) into a STAGES-deep ring;
+//   warp 1 lane 0  - MMA issuer: tcgen05.mma (M = 128, N = BN) into a TMEM
+//                    accumulator, tcgen05.commit frees each smem stage;
+//   all 4 warps    - epilogue: tcgen05.ld 32 lanes x 32 columns, transpose
+//                    through padded smem so each warp store is one coalesced
+//                    128-byte row segment, fused elementwise op, store.
+// Modes: TF32 (fp32 operands read as TF32), 3xTF32 (operands kept as a TF32
+// high part plus an fp32 remainder; acc += Ah*Bh + Ah*Bl + Al*Bh), BF16.
+// No TMA multicast is used anywhere.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "shp_common.cuh"
+
+namespace shp {
+
+namespace {
+
+constexpr int A_BYTES = 128 * 128;        // 128 rows x 128 bytes
+constexpr int B_BYTES_MAX = 256 * 128;    // BN <= 256 rows x 128 bytes
+constexpr int EPI_BYTES = 4 * 32 * 33 * 4;
+
+template <int MODE>
+struct Cfg {
+  static constexpr bool SPLIT = MODE == MODE_3XTF32;
+  static constexpr int ESZ = MODE == MODE_BF16 ? 2 : 4;
+  static constexpr int BK = 128 / ESZ;         // K elements per stage (one 128 B row)
+  static constexpr int UK = MODE == MODE_BF16 ? 16 : 8;  // K per MMA instruction
+  static constexpr int KSTEPS = BK / UK;
+  static constexpr int CHUNK = 128 / ESZ;      // MN elements per 128-byte chunk
+  // MN-major smem layout: 32-bit operands need the 32-byte-atom 128B swizzle
+  // (period 4 rows); 16-bit operands use the plain 128B swizzle (8 rows).
+  static constexpr uint32_t MN_LAYOUT = ESZ == 4 ? 1u : 2u;
+  static constexpr uint32_t MN_SBO = ESZ == 4 ? 512u : 1024u;
+  static constexpr int STAGES = SPLIT ? 2 : 4;
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES_MAX) * (SPLIT ? 2 : 1);
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 256;
+};
+
+SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
+  if (fmt == OUT_F32) {
+    static_cast<float*>(hi)[off] = v;
+  } else if (fmt == OUT_SPLIT) {
+    const float h = tf32_round(v);
+    static_cast<float*>(hi)[off] = h;
+    lo[off] = v - h;
+  } else {
+    static_cast<__nv_bfloat16*>(hi)[off] = __float2bfloat16_rn(v);
+  }
+}
+
+template <int MODE, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(128, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
+              const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tBl,
+              int K, int BN, EpiParams ep) {
+  using C = Cfg<MODE>;
+  const int b = blockIdx.z;
+  if (ep.active != nullptr && ep.active[b] == 0) return;
+  const int m0 = blockIdx.y * 128;
+  const int n0 = blockIdx.x * BN;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* epi = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + EPI_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* done = empty + C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = static_cast<uint32_t>(BN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tA);
+    tma_prefetch_desc(&tB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, ncols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int KB = (K + C::BK - 1) / C::BK;
+  const uint32_t b_bytes = static_cast<uint32_t>(BN) * 128u;
+  const uint32_t tx = (A_BYTES + b_bytes) * (C::SPLIT ? 2u : 1u);
+  bool timed_out = false;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % C::STAGES;
+      if (kb >= C::STAGES && !mbar_wait(&empty[s], ((kb / C::STAGES) - 1) & 1)) {
+        timed_out = true;
+        break;
+      }
+      uint8_t* st = smem + s * C::STAGE_BYTES;
+      const int k0 = kb * C::BK;
+      mbar_arrive_expect_tx(&full[s], tx);
+#pragma unroll 1
+      for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
+        const CUtensorMap* ma = part ? &tAl : &tA;
+        const CUtensorMap* mb = part ? &tBl : &tB;
+        uint8_t* sa = st + part * (A_BYTES + B_BYTES_MAX);
+        uint8_t* sb = sa + A_BYTES;
+        if (A_MN) {
+          for (int i = 0; i < 128 / C::CHUNK; ++i)
+            tma_load_3d(sa + i * C::BK * 128, ma, &full[s], m0 + i * C::CHUNK, k0, b);
+        } else {
+          tma_load_3d(sa, ma, &full[s], k0, m0, b);
+        }
+        if (B_MN) {
+          for (int i = 0; i < BN / C::CHUNK; ++i)
+            tma_load_3d(sb + i * C::BK * 128, mb, &full[s], n0 + i * C::CHUNK, k0, b);
+        } else {
+          tma_load_3d(sb, mb, &full[s], k0, n0, b);
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = instr_desc(MODE == MODE_BF16 ? 1u : 2u, A_MN, B_MN, 128, BN);
+    const uint32_t mn_lbo = C::BK * 128;  // bytes between 128-byte MN chunks
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % C::STAGES;
+      if (!mbar_wait(&full[s], (kb / C::STAGES) & 1)) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = smem_u32(smem + s * C::STAGE_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        uint64_t ad[2], bd[2];
+#pragma unroll
+        for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
+          const uint32_t sa = base + part * (A_BYTES + B_BYTES_MAX);
+          const uint32_t sb = sa + A_BYTES;
+          ad[part] = A_MN ? smem_desc(sa + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
+                          : smem_desc(sa + ks * C::UK * C::ESZ, 16, 1024, 2);
+          bd[part] = B_MN ? smem_desc(sb + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
+                          : smem_desc(sb + ks * C::UK * C::ESZ, 16, 1024, 2);
+        }
+        const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
+        if (MODE == MODE_BF16) {
+          mma_f16(tmem, ad[0], bd[0], idesc, acc0);
+        } else {
+          mma_tf32(tmem, ad[0], bd[0], idesc, acc0);
+          if (C::SPLIT) {
+            mma_tf32(tmem, ad[0], bd[C::SPLIT ? 1 : 0], idesc, 1u);
+            mma_tf32(tmem, ad[C::SPLIT ? 1 : 0], bd[0], idesc, 1u);
+          }
+        }
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  }
+
+  // ---------------- epilogue (all 4 warps; warp w owns TMEM lanes 32w..32w+31)
+  if (!mbar_wait(done, 0)) timed_out = true;
+  __syncwarp();
+  tc_fence_after();
+
+  float* st = epi + warp * (32 * 33);
+  const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;
+  const bool diag_tile = (m0 < n0 + BN) && (n0 < m0 + 128);
+  float nrm = 0.f;
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c * 32), v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) st[lane * 33 + j] = v[j];
+    __syncwarp();
+    const int gj = n0 + c * 32 + lane;
+    if (gj < ep.N) {
+      for (int r = 0; r < 32; ++r) {
+        const int gi = m0 + warp * 32 + r;
+        if (gi >= ep.M) break;
+        const float acc = st[r * 33 + lane];
+        const float eye = (diag_tile && gi == gj) ? 1.f : 0.f;
+        const int64_t off = static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(gi) * ep.ldo + gj;
+        float val;
+        switch (ep.kind) {
+          case EPI_RESID:
+            val = eye - acc;
+            nrm += val * val;
+            break;
+          case EPI_GPOLY: {
+            const int64_t oa = static_cast<int64_t>(b) * ep.bs_aux +
+                               static_cast<int64_t>(gi) * ep.lda_aux + gj;
+            float rv = ep.aux_hi[oa];
+            if (ep.aux_lo != nullptr) rv += ep.aux_lo[oa];
+            val = eye + ep.s1 * rv + alpha * acc;
+            break;
+          }
+          case EPI_EMA:
+            val = ep.s0 * static_cast<const float*>(ep.out_hi)[off] + ep.s1 * acc + ep.s2 * eye;
+            break;
+          case EPI_APPLY:
+            val = static_cast<const float*>(ep.out_hi)[off] + ep.s0 * acc;
+            break;
+          default:
+            val = ep.s0 * acc;
+            break;
+        }
+        put(ep.out_fmt, ep.out_hi, ep.out_lo, off, val);
+        if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, val);
+      }
+    }
+    __syncwarp();
+  }
+  if (ep.kind == EPI_RESID) {
+    nrm = warp_sum(nrm);
+    if (lane == 0) atomicAdd(&ep.norm2[static_cast<int64_t>(b) * ep.norm2_stride], nrm);
+  }
+  if (timed_out && ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over [batch][rows][inner] with the given box, 128-byte swizzle,
+// zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* ptr, int esz, int64_t inner, int64_t rows,
+              int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows,
+              CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * esz),
+                           static_cast<cuuint64_t>((batch > 1 ? bstride : rows * ld) * esz)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE, bool AMN, bool BMN>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMap& b,
+                   const CUtensorMap& bl, int M, int N, int K, int BN, int batch,
+                   const EpiParams& ep, cudaStream_t st) {
+  using C = Cfg<MODE>;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<MODE, AMN, BMN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid((N + BN - 1) / BN, (M + 127) / 128, batch);
+  k_gemm_tc<MODE, AMN, BMN><<<grid, 128, C::SMEM, st>>>(a, al, b, bl, K, BN, ep);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t dispatch(bool amn, bool bmn, const CUtensorMap& a, const CUtensorMap& al,
+                     const CUtensorMap& b, const CUtensorMap& bl, int M, int N, int K, int BN,
+                     int batch, const EpiParams& ep, cudaStream_t st) {
+  if (!amn && !bmn) return launch<MODE, false, false>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  if (!amn && bmn) return launch<MODE, false, true>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  if (amn && !bmn) return launch<MODE, true, false>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  return launch<MODE, true, true>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+}
+
+}  // namespace
+
+cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, int K,
+                    int batch, const EpiParams& ep, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return cudaSuccess;
+  const int esz = mode == MODE_BF16 ? 2 : 4;
+  const int bk = 128 / esz, chunk = 128 / esz;
+  const int BN = N > 128 ? 256 : (N > 64 ? 128 : 64);
+  CUtensorMap ma, mal, mb, mbl;
+  bool ok = true;
+  // A: logical M x K.
+  // MN-major tiles of 32-bit data use the 32-byte-atom swizzle (see Cfg).
+  const CUtensorMapSwizzle mn_swz =
+      esz == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  auto mapA = [&](CUtensorMap* m, const void* p) {
+    return A.mn ? make_map(m, p, esz, M, K, batch, A.ld, A.bstride, chunk, bk, mn_swz)
+                : make_map(m, p, esz, K, M, batch, A.ld, A.bstride, bk, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+  };
+  // B: logical K x N.
+  auto mapB = [&](CUtensorMap* m, const void* p) {
+    return B.mn ? make_map(m, p, esz, N, K, batch, B.ld, B.bstride, chunk, bk, mn_swz)
+                : make_map(m, p, esz, K, N, batch, B.ld, B.bstride, bk, BN,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+  };
+  ok = ok && mapA(&ma, A.hi) && mapB(&mb, B.hi);
+  if (mode == MODE_3XTF32) {
+    if (A.lo == nullptr || B.lo == nullptr) return cudaErrorInvalidValue;
+    ok = ok && mapA(&mal, A.lo) && mapB(&mbl, B.lo);
+  } else {
+    mal = ma;
+    mbl = mb;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  switch (mode) {
+    case MODE_TF32:
+      return dispatch<MODE_TF32>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
+    case MODE_3XTF32:
+      return dispatch<MODE_3XTF32>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
+    case MODE_BF16:
+      return dispatch<MODE_BF16>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace shp

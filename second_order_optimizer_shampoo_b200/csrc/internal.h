@@ -1,0 +1,135 @@
+// Host-side interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace shp {
+
+enum Mode { MODE_TF32 = 0, MODE_3XTF32 = 1, MODE_BF16 = 2 };
+enum EpiKind { EPI_STORE = 0, EPI_RESID = 1, EPI_GPOLY = 2, EPI_EMA = 3, EPI_APPLY = 4 };
+enum OutFmt { OUT_F32 = 0, OUT_SPLIT = 1, OUT_BF16 = 2 };
+
+// Per-block outcome codes (mirrors shp_status in include/shampoo_prism.h).
+enum { ST_OK = 0, ST_ENOCONV = 16, ST_ESTALL = 17, ST_ENONFINITE = 18, ST_ETIMEOUT = 19 };
+
+// A batched row-major operand in HBM.  `hi` holds the fp32 value (TF32 mode),
+// the TF32-rounded high part (split mode, with `lo` = value - hi) or bf16.
+//   mn == false (K-major): element (i, k) of the logical M x K (or N x K
+//     for B^T) operand sits at hi[i * ld + k];
+//   mn == true  (MN-major): element (i, k) sits at hi[k * ld + i].
+struct Operand {
+  const void* hi;
+  const float* lo;
+  bool mn;
+  int64_t ld;       // elements between consecutive memory rows
+  int64_t bstride;  // elements between batch members
+};
+
+// What the epilogue does with accumulator element acc(i, j) of block b.
+//   STORE: v = s0 * acc
+//   RESID: v = [i==j] - acc, and norm2[b] += v^2
+//   GPOLY: v = [i==j] + s1 * aux(i,j) + alpha[b] * acc
+//   EMA:   v = s0 * out(i,j) + s1 * acc + s2 * [i==j]   (read-modify-write)
+//   APPLY: v = out(i,j) + s0 * acc                       (read-modify-write)
+// v is written to `out` (and to `out2` when non-null) in `out_fmt`.
+struct EpiParams {
+  int kind;
+  int out_fmt;
+  void* out_hi;
+  float* out_lo;
+  void* out2_hi;
+  float* out2_lo;
+  int64_t ldo, bso;
+  const float* aux_hi;
+  const float* aux_lo;
+  int64_t lda_aux, bs_aux;
+  const float* alpha;
+  float s0, s1, s2;
+  float* norm2;       // norm2[b * norm2_stride] accumulates ||v||^2 (RESID)
+  int norm2_stride;
+  const int* active;  // blocks with active[b] == 0 are skipped (may be null)
+  int* status;        // receives ST_ETIMEOUT if a pipeline wait runs out (may be null)
+  int M, N;
+};
+
+// C[b] (M x N) = A[b] (M x K) * B[b] (K x N) on tcgen05 tensor cores,
+// followed by the epilogue.  A and B must share `mode`'s storage type.
+cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, int K,
+                    int batch, const EpiParams& ep, cudaStream_t st);
+
+// ---- PRISM sketch and alpha (sketch_alpha.cu)
+// Vout[b] = R[b] * Vin[b]; R is n x n (hi + lo when lo != null); V is n x p.
+// vin_bstride == 0 shares Vin across the batch.
+cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
+                        const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
+                        int p, int batch, const int* active, cudaStream_t st);
+// V is stored per block as [2d+2][n][p] (slot j holds V_j; slot 0 unused).
+// Gram of V_d..V_{2d+1}, the
+// quartic J(alpha) and its minimiser on [lo, hi]; writes alpha[b] and, when
+// non-null, J_coef[b][5] and report_alpha[b * stride + slot].
+cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
+                        int fixed_alpha, const int* active, float* alpha, double* J_coef,
+                        float* report_alpha, int64_t report_stride, int report_slot,
+                        cudaStream_t st);
+
+// ---- per-block control (sketch_alpha.cu)
+struct BlockState {
+  float norm2;     // ||R_k||_F^2 accumulated by the residual epilogue
+  float prev_res;  // residual of the previous iteration
+  float c;         // Frobenius norm of the input (normalisation)
+  int iters;       // update steps taken in the current pass
+  int iters1;      // update steps taken in pass 1 (set when pass 2 starts)
+  int status;      // first non-OK outcome over the passes
+  int pass_status;
+  int pad;
+};
+// Workspace-resident control block of one call.
+struct Ctl {
+  BlockState* bs;
+  int* active;
+  double* dnorm;  // ||input||_F^2 per block
+  int* tmo;       // ST_ETIMEOUT flags from the GEMM pipeline
+  float* alpha;   // alpha_k per block
+};
+cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int k, int max_iter, float tol,
+                         float stall_below, float stall_ratio, float* report_res,
+                         int64_t res_stride, int res_slot, int* report_iters, int iters_slot,
+                         cudaStream_t st);
+
+// ---- elementwise (elementwise.cu)
+// Start of a pass: active = 1, counters cleared; first_pass also clears the
+// status, the timeout flags and the input norms; otherwise iters1 = iters.
+cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st);
+// dnorm[b] += ||X[b]||_F^2 (X fp32 or bf16, rows x cols contiguous per block).
+cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
+                       cudaStream_t st);
+// c = sqrt(dnorm); Y = A / c; Z = I; R = I - Y; norm2 = ||R||_F^2.
+// (lo pointers null in TF32 mode.)
+cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, float* Yhi,
+                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                         cudaStream_t st);
+// Pass 2: Y[0] <- Y[iters1 % 2]; Z = I; R = I - Y; norm2 = ||R||_F^2.
+cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* Yhi,
+                            float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                            cudaStream_t st);
+// g = I + alpha[b] R (d = 1) in `fmt`; also into (g2hi, g2lo) when non-null.
+cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, const Ctl& ctl,
+                     int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st);
+// X_out[b] = c_b^e * S[iters_b % 2][b] (hi + lo), S = the two ping-pong slots.
+cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_exponent,
+                           const float* const* Shi, const float* const* Slo, float* X_out,
+                           cudaStream_t st);
+// hi = tf32(X), lo = X - hi.
+cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st);
+// X0 = G / ||G||_F (uses dnorm) in `fmt`.
+cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, const Ctl& ctl,
+                       int fmt, void* Xhi, float* Xlo, cudaStream_t st);
+// X_out[b] = slot[iters_b % 2][b] in the output storage (bf16 or fp32).
+cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
+                         const void* const* Shi, const float* const* Slo, void* X_out,
+                         int out_bf16, cudaStream_t st);
+// report.status[b] = ETIMEOUT if flagged, else bs[b].status.
+cudaError_t write_status(const Ctl& ctl, int batch, int* report_status, cudaStream_t st);
+
+}  // namespace shp

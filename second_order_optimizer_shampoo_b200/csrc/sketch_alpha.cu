@@ -1,0 +1,338 @@
+// PRISM sketched alpha fit and per-block iteration control.
+//
+// "Sintesi Tecnica: PRISM", Parte II.1-II.2: the top coefficient alpha of the
+// update polynomial g_d(xi; alpha) = f_{d-1}(xi) + alpha xi^d is chosen each
+// iteration by a least-squares fit of the next residual on the spectrum of
+// R_k, constrained to [l, u], and the fit is made on a Gaussian sketch S so
+// that it costs O(n^2 p) instead of traces of high powers of R_k.
+//
+// With g = f + alpha xi^d the next residual of the square-root family is
+//   r(xi; alpha) = 1 - (1 - xi) g^2
+//                = [1 - (1-xi) f^2] - 2 alpha (1-xi) xi^d f - alpha^2 (1-xi) xi^{2d},
+// a polynomial in xi whose coefficients r_j are quadratics in alpha and vanish
+// outside j = d..2d+1.  Hence, with V_j = R_k^j S and M_ij = <V_i, V_j>_F,
+//   J(alpha) = ||r(R_k; alpha) S||_F^2 = sum_{i,j} r_i(alpha) r_j(alpha) M_ij,
+// a quartic in alpha whose minimiser on [lo, hi] is the new alpha_k.
+//
+// Kernels: the skinny products V_j = R V_{j-1} on CUDA cores (fp32 FMA, HBM
+// bound), the Gram/quartic/argmin per block (fp64), and the stop test.
+#include <math.h>
+
+#include "internal.h"
+#include "shp_common.cuh"
+
+namespace shp {
+
+namespace {
+
+constexpr int SK_THREADS = 256;
+constexpr int SK_CHUNK = 256;  // columns of V staged in shared memory per step
+
+// Vout = R * Vin for one block; 8 warps x ROWS rows per CTA.
+template <int P>
+__global__ void __launch_bounds__(SK_THREADS)
+    k_sketch(const float* __restrict__ Rhi, const float* __restrict__ Rlo, int64_t n,
+             int64_t rbs, const float* __restrict__ Vin, int64_t vbs, float* __restrict__ Vout,
+             int64_t obs, int p, const int* __restrict__ active) {
+  constexpr int ROWS = P <= 16 ? 4 : 2;
+  __shared__ float Vs[P][SK_CHUNK];
+  const int b = blockIdx.y;
+  if (active != nullptr && active[b] == 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (8 * ROWS) + warp * ROWS;
+  const float* R = Rhi + b * rbs;
+  const float* RL = Rlo != nullptr ? Rlo + b * rbs : nullptr;
+  const float* V = Vin + b * vbs;
+  float acc[ROWS][P];
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+    for (int j = 0; j < P; ++j) acc[r][j] = 0.f;
+
+  for (int64_t c0 = 0; c0 < n; c0 += SK_CHUNK) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < SK_CHUNK * P; idx += SK_THREADS) {
+      const int cc = idx / P, j = idx % P;
+      const int64_t col = c0 + cc;
+      Vs[j][cc] = (j < p && col < n) ? V[col * p + j] : 0.f;
+    }
+    __syncthreads();
+    for (int cc = lane; cc < SK_CHUNK; cc += 32) {
+      const int64_t col = c0 + cc;
+      if (col >= n) break;
+      float rv[ROWS];
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        const int64_t row = row0 + r;
+        float x = 0.f;
+        if (row < n) {
+          x = R[row * n + col];
+          if (RL != nullptr) x += RL[row * n + col];
+        }
+        rv[r] = x;
+      }
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        const float vj = Vs[j][cc];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r][j] = fmaf(rv[r], vj, acc[r][j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      const float s = warp_sum(acc[r][j]);
+      const int64_t row = row0 + r;
+      if (lane == 0 && row < n && j < p) Vout[b * obs + row * p + j] = s;
+    }
+  }
+}
+
+// Coefficients of r_j(alpha) = T[j][0] + T[j][1] alpha + T[j][2] alpha^2 for
+// j = d..2d+1, written out from the expansion in the file header:
+//   d = 1 (f = 1):        r = (1-2a) xi + (2a - a^2) xi^2 + a^2 xi^3
+//   d = 2 (f = 1 + xi/2): r = (3/4 - 2a) xi^2 + (1/4 + a) xi^3 + (a - a^2) xi^4 + a^2 xi^5
+__device__ const double kRTab1[3][3] = {{1.0, -2.0, 0.0}, {0.0, 2.0, -1.0}, {0.0, 0.0, 1.0}};
+__device__ const double kRTab2[4][3] = {
+    {0.75, -2.0, 0.0}, {0.25, 1.0, 0.0}, {0.0, 1.0, -1.0}, {0.0, 0.0, 1.0}};
+
+__device__ double poly4(const double* c, double a) {
+  return (((c[4] * a + c[3]) * a + c[2]) * a + c[1]) * a + c[0];
+}
+__device__ double dpoly4(const double* c, double a) {
+  return ((4.0 * c[4] * a + 3.0 * c[3]) * a + 2.0 * c[2]) * a + c[1];
+}
+__device__ double d2poly4(const double* c, double a) {
+  return (12.0 * c[4] * a + 6.0 * c[3]) * a + 2.0 * c[2];
+}
+
+// Global minimiser of the quartic J on [lo, hi].  J' is monotone between the
+// real roots of J'' (a quadratic), so each such piece holds at most one root
+// of J', found by bisection and polished by Newton.  The candidate with the
+// least J wins; values within 1e-12 (relative) of the best tie and go to the
+// smaller alpha; a constant or non-finite J gives lo.
+__device__ double argmin_quartic(const double* c, double lo, double hi) {
+  bool finite = true;
+  double scale = 0.0;
+  for (int i = 0; i < 5; ++i) {
+    if (!isfinite(c[i])) finite = false;
+    if (i > 0) scale = fmax(scale, fabs(c[i]));
+  }
+  if (!finite || scale == 0.0) return lo;
+  double brk[4];
+  int nb = 0;
+  brk[nb++] = lo;
+  {
+    const double qa = 12.0 * c[4], qb = 6.0 * c[3], qc = 2.0 * c[2];
+    double r1 = NAN, r2 = NAN;
+    if (qa != 0.0) {
+      const double disc = qb * qb - 4.0 * qa * qc;
+      if (disc >= 0.0) {
+        const double sd = sqrt(disc);
+        const double q = -0.5 * (qb + (qb >= 0.0 ? sd : -sd));
+        if (q != 0.0) {
+          r1 = q / qa;
+          r2 = qc / q;
+        } else {
+          r1 = r2 = 0.0;
+        }
+      }
+    } else if (qb != 0.0) {
+      r1 = -qc / qb;
+    }
+    if (r1 > r2) {
+      const double t = r1;
+      r1 = r2;
+      r2 = t;
+    }
+    if (r1 > lo && r1 < hi) brk[nb++] = r1;
+    if (r2 > lo && r2 < hi && r2 != r1) brk[nb++] = r2;
+  }
+  brk[nb++] = hi;
+  double cand[5];
+  int nc = 0;
+  cand[nc++] = lo;
+  cand[nc++] = hi;
+  for (int s = 0; s + 1 < nb; ++s) {
+    double u = brk[s], v = brk[s + 1];
+    double fu = dpoly4(c, u), fv = dpoly4(c, v);
+    if (fu == 0.0) {
+      cand[nc++] = u;
+      continue;
+    }
+    if (fv == 0.0 || (fu < 0.0) == (fv < 0.0)) continue;
+    for (int it = 0; it < 200 && v - u > 1e-15 * fmax(1.0, fabs(u)); ++it) {
+      const double mid = 0.5 * (u + v);
+      const double fm = dpoly4(c, mid);
+      if (fm == 0.0) {
+        u = v = mid;
+        break;
+      }
+      if ((fm < 0.0) == (fu < 0.0)) {
+        u = mid;
+        fu = fm;
+      } else {
+        v = mid;
+      }
+    }
+    double a = 0.5 * (u + v);
+    for (int it = 0; it < 2; ++it) {
+      const double h = d2poly4(c, a);
+      if (h != 0.0) {
+        const double an = a - dpoly4(c, a) / h;
+        if (an >= brk[s] && an <= brk[s + 1]) a = an;
+      }
+    }
+    if (a > lo && a < hi) cand[nc++] = a;
+  }
+  double best = poly4(c, cand[0]);
+  for (int i = 1; i < nc; ++i) best = fmin(best, poly4(c, cand[i]));
+  const double thr = best + 1e-12 * fmax(fabs(best), 1e-300);
+  double pick = hi;
+  for (int i = 0; i < nc; ++i)
+    if (poly4(c, cand[i]) <= thr && cand[i] < pick) pick = cand[i];
+  return pick;
+}
+
+constexpr int AL_THREADS = 256;
+
+__global__ void __launch_bounds__(AL_THREADS)
+    k_alpha(const float* __restrict__ V, int64_t n, int p, int d, int64_t vbs, float lo,
+            float hi, int fixed, const int* __restrict__ active, float* __restrict__ alpha,
+            double* __restrict__ Jc, float* __restrict__ rep, int64_t rep_stride, int rep_slot) {
+  const int b = blockIdx.x;
+  if (active != nullptr && active[b] == 0) return;
+  if (fixed) {  // plain Taylor step: alpha = lo, no sketch needed
+    if (threadIdx.x == 0) {
+      alpha[b] = lo;
+      if (rep != nullptr) rep[b * rep_stride + rep_slot] = lo;
+    }
+    return;
+  }
+  const int nv = d + 2;               // V_d .. V_{2d+1}
+  const int64_t len = n * p;
+  const float* Vb = V + b * vbs + static_cast<int64_t>(d) * len;
+  double part[10];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) part[i] = 0.0;
+  for (int64_t e = threadIdx.x; e < len; e += AL_THREADS) {
+    double x[4];
+    for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(Vb[i * len + e]);
+    int idx = 0;
+    for (int i = 0; i < nv; ++i)
+      for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
+  }
+  __shared__ double red[AL_THREADS / 32][10];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const double s = warp_sum(part[i]);
+    if (lane == 0) red[warp][i] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  double M[4][4];
+  {
+    int idx = 0;
+    for (int i = 0; i < nv; ++i)
+      for (int j = i; j < nv; ++j) {
+        double s = 0.0;
+        for (int w = 0; w < AL_THREADS / 32; ++w) s += red[w][idx];
+        M[i][j] = M[j][i] = s;
+        ++idx;
+      }
+  }
+  double T[4][3];
+  for (int i = 0; i < nv; ++i)
+    for (int a = 0; a < 3; ++a) T[i][a] = d == 1 ? kRTab1[i][a] : kRTab2[i][a];
+  double coef[5] = {0, 0, 0, 0, 0};
+  for (int a = 0; a < 3; ++a)
+    for (int c = 0; c < 3; ++c) {
+      double s = 0.0;
+      for (int i = 0; i < nv; ++i)
+        for (int j = 0; j < nv; ++j) s += T[i][a] * M[i][j] * T[j][c];
+      coef[a + c] += s;
+    }
+  const double a = argmin_quartic(coef, static_cast<double>(lo), static_cast<double>(hi));
+  alpha[b] = static_cast<float>(a);
+  if (Jc != nullptr)
+    for (int i = 0; i < 5; ++i) Jc[b * 5 + i] = coef[i];
+  if (rep != nullptr) rep[b * rep_stride + rep_slot] = static_cast<float>(a);
+}
+
+__global__ void k_control(BlockState* bs, int* active, int batch, int64_t n, int k, int max_iter,
+                          float tol, float stall_below, float stall_ratio, float* rep_res,
+                          int64_t res_stride, int res_slot, int* rep_iters, int iters_slot) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= batch || active[b] == 0) return;
+  BlockState& s = bs[b];
+  const float r = sqrtf(s.norm2 / static_cast<float>(n));
+  s.norm2 = 0.f;
+  if (rep_res != nullptr) rep_res[b * res_stride + res_slot + k] = r;
+  int st = -1;
+  if (!isfinite(r))
+    st = ST_ENONFINITE;
+  else if (r <= tol)
+    st = ST_OK;
+  else if (k >= max_iter)
+    st = ST_ENOCONV;
+  else if (k >= 1 && s.prev_res < stall_below && r > stall_ratio * s.prev_res)
+    st = ST_ESTALL;
+  s.prev_res = r;
+  if (st >= 0) {
+    active[b] = 0;
+    s.iters = k;
+    s.pass_status = st;
+    if (s.status == ST_OK) s.status = st;
+    if (rep_iters != nullptr) rep_iters[b * 2 + iters_slot] = k;
+  }
+}
+
+}  // namespace
+
+cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
+                        const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
+                        int p, int batch, const int* active, cudaStream_t st) {
+  if (batch <= 0 || n <= 0) return cudaSuccess;
+  const int rows = p <= 16 ? 4 : 2;
+  dim3 grid(static_cast<unsigned>((n + 8 * rows - 1) / (8 * rows)), batch);
+  if (p <= 4)
+    k_sketch<4><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
+                                             vout_bstride, p, active);
+  else if (p <= 8)
+    k_sketch<8><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
+                                             vout_bstride, p, active);
+  else if (p <= 16)
+    k_sketch<16><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
+                                              vout_bstride, p, active);
+  else
+    k_sketch<32><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
+                                              vout_bstride, p, active);
+  return cudaGetLastError();
+}
+
+cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
+                        int fixed_alpha, const int* active, float* alpha, double* J_coef,
+                        float* report_alpha, int64_t report_stride, int report_slot,
+                        cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  const int64_t vbs = static_cast<int64_t>(2 * d + 2) * n * p;
+  k_alpha<<<batch, AL_THREADS, 0, st>>>(V, n, p, d, vbs, lo, hi, fixed_alpha, active, alpha,
+                                        J_coef, report_alpha, report_stride, report_slot);
+  return cudaGetLastError();
+}
+
+cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int k, int max_iter, float tol,
+                         float stall_below, float stall_ratio, float* report_res,
+                         int64_t res_stride, int res_slot, int* report_iters, int iters_slot,
+                         cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  k_control<<<(batch + 127) / 128, 128, 0, st>>>(ctl.bs, ctl.active, batch, n, k, max_iter, tol,
+                                                 stall_below, stall_ratio, report_res, res_stride,
+                                                 res_slot, report_iters, iters_slot);
+  return cudaGetLastError();
+}
+
+}  // namespace shp

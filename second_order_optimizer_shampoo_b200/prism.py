@@ -1,0 +1,167 @@
+"""Python binding of the C ABI (argument marshalling only).
+
+Each function takes CUDA tensors, allocates the scratch buffer the library
+asks for through PyTorch's allocator, and calls the entry point of the same
+name on the current stream.  Every arithmetic step runs in the library's
+kernels; there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi as A
+
+_PREC = {"tf32": A.SHP_TF32, "3xtf32": A.SHP_3XTF32, "bf16": A.SHP_BF16}
+_POW = {"inv4": A.SHP_POW_INV4, "inv2": A.SHP_POW_INV2, "sqrt": A.SHP_POW_SQRT}
+
+
+def status_string(code: int) -> str:
+    return A.lib().shp_status_string(int(code)).decode()
+
+
+def version() -> str:
+    return A.lib().shp_version().decode()
+
+
+def _check(code: int, name: str):
+    if code != A.SHP_OK:
+        raise RuntimeError(f"{name} failed: {status_string(code)} ({code})")
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device (the library has no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def make_opts(d=2, p=8, lo=None, hi=1.0, tol=1e-3, max_iter=40, prec="3xtf32",
+              fixed_alpha=False, stall_below=0.05, stall_ratio=0.75) -> A.PrismOpts:
+    if lo is None:
+        lo = 0.5 if d == 1 else 0.375
+    return A.PrismOpts(d, p, lo, hi, tol, max_iter, _PREC[prec] if isinstance(prec, str) else prec,
+                       int(bool(fixed_alpha)), stall_below, stall_ratio)
+
+
+def shp_workspace_bytes(op: int, m: int, n: int, batch: int, opts: A.PrismOpts | None = None) -> int:
+    return int(A.lib().shp_workspace_bytes(op, m, n, batch,
+                                           ctypes.byref(opts) if opts is not None else None))
+
+
+def _ws(nbytes: int, device):
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def _as3(t, rows, cols):
+    return t.reshape(-1, rows, cols)
+
+
+def shampoo_gram_ema(G, L, R, beta: float, eps: float, prec: str = "tf32", ws=None):
+    """L <- beta L + (1-beta) G G^T + eps I ; R <- beta R + (1-beta) G^T G + eps I (in place)."""
+    _dev(G, L, R)
+    m, n = G.shape[-2], G.shape[-1]
+    batch = G.numel() // (m * n)
+    o = make_opts(prec=prec)
+    need = shp_workspace_bytes(A.SHP_OP_GRAM_EMA, m, n, batch, o)
+    ws = _ws(need, G.device) if ws is None else ws
+    _check(A.lib().shampoo_gram_ema(_p(G), m, n, batch, _p(L), _p(R), beta, eps, _PREC[prec],
+                                    _p(ws), ws.numel(), _stream()), "shampoo_gram_ema")
+
+
+def shampoo_apply(W, G, Lroot, Rroot, lr: float, prec: str = "tf32", ws=None):
+    """W <- W - lr * Lroot G Rroot (in place)."""
+    _dev(W, G, Lroot, Rroot)
+    m, n = W.shape[-2], W.shape[-1]
+    batch = W.numel() // (m * n)
+    o = make_opts(prec=prec)
+    need = shp_workspace_bytes(A.SHP_OP_APPLY, m, n, batch, o)
+    ws = _ws(need, W.device) if ws is None else ws
+    _check(A.lib().shampoo_apply(_p(W), _p(G), _p(Lroot), _p(Rroot), m, n, batch, lr, _PREC[prec],
+                                 _p(ws), ws.numel(), _stream()), "shampoo_apply")
+
+
+def _report(batch, max_iter, device):
+    return {
+        "status": torch.full((batch,), -1, dtype=torch.int32, device=device),
+        "iters": torch.full((batch, 2), -1, dtype=torch.int32, device=device),
+        "resid": torch.full((batch, 2, max_iter + 1), float("nan"), dtype=torch.float32, device=device),
+        "alpha": torch.full((batch, 2, max_iter), float("nan"), dtype=torch.float32, device=device),
+    }
+
+
+def _report_struct(rep):
+    if rep is None:
+        return None
+    return ctypes.byref(A.PrismReport(rep["status"].data_ptr(), rep["iters"].data_ptr(),
+                                      rep["resid"].data_ptr(), rep["alpha"].data_ptr()))
+
+
+def matfn_inv_root(Amat, power="inv4", opts: A.PrismOpts | None = None, S=None, out=None,
+                   report=True, ws=None):
+    """A^(-1/4) (or A^(-1/2), A^(1/2)) of a batch of SPD matrices."""
+    opts = opts or make_opts()
+    _dev(Amat, S, out)
+    n = Amat.shape[-1]
+    batch = Amat.numel() // (n * n)
+    out = torch.empty_like(Amat) if out is None else out
+    rep = _report(batch, opts.max_iter, Amat.device) if report else None
+    need = shp_workspace_bytes(A.SHP_OP_INV_ROOT, n, n, batch, opts)
+    ws = _ws(need, Amat.device) if ws is None else ws
+    s_count = 0 if S is None else S.shape[0]
+    _check(A.lib().matfn_inv_root(_p(Amat), n, batch, _POW[power], ctypes.byref(opts), _p(S),
+                                  s_count, _p(out), _report_struct(rep), _p(ws), ws.numel(),
+                                  _stream()), "matfn_inv_root")
+    return out, rep
+
+
+def matfn_polar(G, opts: A.PrismOpts | None = None, S=None, out=None, report=True, ws=None):
+    """Polar factor of a batch of m x n matrices; bf16 input keeps bf16 storage."""
+    opts = opts or make_opts()
+    _dev(G, S, out)
+    m, n = G.shape[-2], G.shape[-1]
+    batch = G.numel() // (m * n)
+    if G.dtype == torch.bfloat16:
+        storage = A.SHP_BF16
+    elif G.dtype == torch.float32:
+        storage = opts.prec if opts.prec in (A.SHP_TF32, A.SHP_3XTF32) else A.SHP_TF32
+    else:
+        raise ValueError("G must be float32 or bfloat16")
+    out = torch.empty_like(G) if out is None else out
+    rep = _report(batch, opts.max_iter, G.device) if report else None
+    o2 = A.PrismOpts.from_buffer_copy(opts)
+    o2.prec = storage
+    need = shp_workspace_bytes(A.SHP_OP_POLAR, m, n, batch, o2)
+    ws = _ws(need, G.device) if ws is None else ws
+    s_count = 0 if S is None else S.shape[0]
+    _check(A.lib().matfn_polar(_p(G), storage, m, n, batch, ctypes.byref(opts), _p(S), s_count,
+                               _p(out), _report_struct(rep), _p(ws), ws.numel(), _stream()),
+           "matfn_polar")
+    return out, rep
+
+
+def prism_alpha_fit(R, S, d: int, lo: float, hi: float, ws=None):
+    """alpha* on [lo, hi] for each residual in the batch, plus J's coefficients."""
+    _dev(R, S)
+    n = R.shape[-1]
+    batch = R.numel() // (n * n)
+    p = S.shape[-1]
+    alpha = torch.empty(batch, dtype=torch.float32, device=R.device)
+    J = torch.empty(batch, 5, dtype=torch.float64, device=R.device)
+    need = shp_workspace_bytes(A.SHP_OP_ALPHA_FIT, n, n, batch, make_opts(d=d, p=p))
+    ws = _ws(need, R.device) if ws is None else ws
+    _check(A.lib().prism_alpha_fit(_p(R), n, batch, _p(S), p, d, lo, hi, _p(alpha), _p(J), _p(ws),
+                                   ws.numel(), _stream()), "prism_alpha_fit")
+    return alpha, J
