@@ -231,7 +231,13 @@ def prism_alpha_ref(Rk, S, d, lo, hi):
 # Newton-Schulz passes  ([PRISM-it] Parte I: X_{k+1} = X_k f(R_k); [Shampoo] §3.1)
 # ---------------------------------------------------------------------------
 
-def _stop(info, rk, k, opts):
+def _stop(info, rk, k, opts, force=None):
+    if force is not None:
+        # same-recurrence mode: run exactly `force` updates, ignoring tol/stall
+        if k >= force:
+            info.status = OK if rk <= opts.tol else ENOCONV
+            return True
+        return False
     if not np.isfinite(rk):
         info.status = ENONFINITE
         return True
@@ -249,14 +255,16 @@ def _stop(info, rk, k, opts):
     return False
 
 
-def coupled_ref(B, opts: PrismOpts, S, s_offset=0):
+def coupled_ref(B, opts: PrismOpts, S, s_offset=0, force_iters=None):
     """Coupled Newton-Schulz square root with PRISM alpha.
 
     Y_0 = B, Z_0 = I; for k = 0, 1, ...:
         R_k = I - Z_k Y_k;  stop test on ||R_k||_F / sqrt(n);
         alpha_k from the sketch S[s_offset + k];
         g = g_d(R_k; alpha_k);  Y_{k+1} = Y_k g;  Z_{k+1} = g Z_k.
-    Y -> B^(1/2), Z -> B^(-1/2) for SPD B with spectrum in (0, 1]."""
+    Y -> B^(1/2), Z -> B^(-1/2) for SPD B with spectrum in (0, 1].
+    force_iters: run exactly that many updates (the iteration count another
+    implementation took), for same-recurrence comparisons."""
     B = _f64(B)
     n = B.shape[0]
     I = np.eye(n)
@@ -267,7 +275,7 @@ def coupled_ref(B, opts: PrismOpts, S, s_offset=0):
         Rk = I - Z @ Y
         rk = float(np.linalg.norm(Rk) / sqrt(n))
         info.res.append(rk)
-        if _stop(info, rk, k, opts):
+        if _stop(info, rk, k, opts, force_iters):
             break
         if opts.fixed_alpha:
             a, coef = float(opts.lo), np.full(5, np.nan)
@@ -282,26 +290,28 @@ def coupled_ref(B, opts: PrismOpts, S, s_offset=0):
     return Y, Z, info
 
 
-def inv_root_ref(A, power, opts: PrismOpts, S):
+def inv_root_ref(A, power, opts: PrismOpts, S, force_iters=None):
     """A^(-1/4), A^(-1/2) or A^(1/2) of an SPD matrix by PRISM Newton-Schulz.
 
     c = ||A||_F (>= lambda_max, so B = A/c has spectrum in (0, 1]);
     pass 1: (Y1, Z1) = coupled(B) -> A^(1/2) = sqrt(c) Y1, A^(-1/2) = Z1 / sqrt(c);
     pass 2 (A^(-1/4) only): (Y2, Z2) = coupled(Y1) -> A^(-1/4) = c^(-1/4) Z2.
+    force_iters: optional (updates in pass 1, updates in pass 2).
     Returns (X, [PassInfo, ...])."""
     A = _f64(A)
+    f1, f2 = (None, None) if force_iters is None else (list(force_iters) + [None])[:2]
     c = float(np.linalg.norm(A))
     B = A / c
-    Y1, Z1, i1 = coupled_ref(B, opts, S, 0)
+    Y1, Z1, i1 = coupled_ref(B, opts, S, 0, f1)
     if power == POW_SQRT:
         return np.sqrt(c) * Y1, [i1]
     if power == POW_INV2:
         return Z1 / np.sqrt(c), [i1]
-    Y2, Z2, i2 = coupled_ref(Y1, opts, S, opts.max_iter)
+    Y2, Z2, i2 = coupled_ref(Y1, opts, S, opts.max_iter, f2)
     return c ** -0.25 * Z2, [i1, i2]
 
 
-def polar_ref(G, opts: PrismOpts, S):
+def polar_ref(G, opts: PrismOpts, S, force_iters=None):
     """Polar factor U V^T of G = U Sigma V^T by PRISM Newton-Schulz.
 
     A wide G (m < n) is handled as G^T.  X_0 = G / ||G||_F; for k = 0, 1, ...:
@@ -319,7 +329,7 @@ def polar_ref(G, opts: PrismOpts, S):
         Rk = I - X.T @ X
         rk = float(np.linalg.norm(Rk) / sqrt(n))
         info.res.append(rk)
-        if _stop(info, rk, k, opts):
+        if _stop(info, rk, k, opts, force_iters):
             break
         if opts.fixed_alpha:
             a, coef = float(opts.lo), np.full(5, np.nan)
