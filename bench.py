@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of the batched Shampoo preconditioner inverse root on one B200.
+
+Workload (one "step"): A^(-1/4) of 64 SPD blocks of 1024 x 1024, each
+Q diag(lambda) Q^T with lambda log-uniform on [1e-6, 1] (cond 1e6), by two
+coupled Newton-Schulz passes with PRISM alpha (d = 2, Gaussian sketch p = 8,
+alpha in [3/8, 1], residual tol 1e-3 per pass), products on the tensor cores
+in the 3xTF32 split (plain TF32 rounding of A/||A||_F exceeds lambda_min
+and the iteration diverges).
+
+Metric: algorithmic TFLOP/s (2 n^3 per n x n product actually executed,
+summed over blocks) and preconditioners/s, with the fraction of the tensor
+peak.  Under torchrun each rank runs its own independent batch (replicas,
+weak scaling); the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "inv-root/polar TFLOP/s & preconditioners/s at 1024², % of B200 tensor peak"
+N, BATCH, LAM_LO, D, P, TOL, MAX_ITER = 1024, 64, 1e-6, 2, 8, 1e-3, 24
+SEED_A, SEED_S = 103, 1003
+# tensor peak ratios (nominal dense): TF32 / BF16 = 1.1 / 2.25 PFLOP/s
+TF32_OVER_BF16 = 1.1 / 2.25
+
+
+def workload_config(world):
+    return {
+        "workload": "inv4_root_64x1024sq_spd_cond1e6_prism_d2_p8",
+        "n": N, "batch_per_gpu": BATCH, "d": D, "p": P, "tol": TOL, "max_iter": MAX_ITER,
+        "alpha_interval": [0.375, 1.0], "prec": "3xtf32", "lambda": "log-uniform [1e-6, 1]",
+        "l2": "inputs larger than L2 (256 MiB of A plus 3.2 GB of iterates per GPU per step)",
+        "parallelism": f"replicas x{world}",
+    }
+
+
+def gemm_count(iters):
+    """Products of one block: pass with k updates costs 4k - 1 (d = 2)."""
+    return sum(max(4 * int(k) - 1, 0) for k in iters)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_timing(local_ms, local_units, local_flops, local_launches, world):
+    """Max over ranks of the time, sums of the work.  Works with any
+    initialised process group (nccl on the GPUs, gloo in the CPU tests)."""
+    if world == 1:
+        return local_ms, local_units, local_flops, local_launches
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    s = torch.tensor([local_units, local_flops, local_launches], dtype=torch.float64, device=dev)
+    dist.all_reduce(s, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(s[0].item()), float(s[1].item()), int(s[2].item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle leg
+def oracle_sample(A_block, S_np, seconds_hint=None):
+    """Time the float64 oracle on one block; returns (seconds, flops)."""
+    from oracle import prism_ref as o
+    opts = o.PrismOpts(d=D, p=P, lo=0.375, hi=1.0, tol=TOL, max_iter=MAX_ITER)
+    t0 = time.perf_counter()
+    _, infos = o.inv_root_ref(A_block, o.POW_INV4, opts, S_np)
+    dt = time.perf_counter() - t0
+    return dt, gemm_count([i.iters for i in infos]) * 2.0 * N ** 3
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    from second_order_optimizer_shampoo_b200 import synth
+    S_np = synth.sketch_stack(2 * MAX_ITER, N, P, SEED_S)
+    blocks = [synth.spd_block(N, LAM_LO, 1.0, SEED_A, i) for i in range(max(1, args.steps + args.warmup))]
+    for i in range(args.warmup):
+        oracle_sample(blocks[i], S_np)
+    tot_t, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        t, f = oracle_sample(blocks[args.warmup + i], S_np)
+        tot_t += t
+        tot_f += f
+    value = tot_f / tot_t / 1e12
+    cores = os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(1),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "one 1024x1024 block of the 64-block batch per step "
+                                   "(float64 NumPy/LAPACK oracle, same recurrence and sketch)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def gemm_only(args):
+    """The dominant kernel alone: batched 1024^3 3xTF32 products (profiling aid)."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(5)
+    X = torch.randn(args.batch, N, N, device=dev, generator=g)
+    Y = torch.randn(args.batch, N, N, device=dev, generator=g)
+    Xh, Xl = prism.shp_split_tf32(X)
+    Yh, Yl = prism.shp_split_tf32(Y)
+    out = torch.empty_like(X)
+    for _ in range(max(args.warmup, 1) + args.steps):
+        prism.shp_matmul(Xh, Yh, "3xtf32", A_lo=Xl, B_lo=Yl, out=out)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": "gemm", "batch": args.batch, "launches": args.steps + max(args.warmup, 1)}))
+    return 0
+
+
+# ------------------------------------------------------------------ our leg
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", default=None, choices=["gemm"],
+                    help="run only the batched 3xTF32 GEMM (for profiling)")
+    ap.add_argument("--batch", type=int, default=BATCH)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.kernel == "gemm":
+        return gemm_only(args)
+
+    import numpy as np
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism, synth
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    # ---- inputs: each rank its own 64 blocks (seeded by global block index)
+    idx = list(range(rank * BATCH, (rank + 1) * BATCH))
+    A_np = synth.spd_batch(N, BATCH, LAM_LO, 1.0, SEED_A, indices=idx)
+    S_np = synth.sketch_stack(2 * MAX_ITER, N, P, SEED_S)
+    A = torch.from_numpy(A_np).to(dev)
+    S = torch.from_numpy(S_np).to(dev)
+    opts = prism.make_opts(d=D, p=P, tol=TOL, max_iter=MAX_ITER, prec="3xtf32")
+    from second_order_optimizer_shampoo_b200 import _abi
+    ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, N, N, BATCH, opts),
+                     dtype=torch.uint8, device=dev)
+    X = torch.empty_like(A)
+
+    def step():
+        return prism.matfn_inv_root(A, "inv4", opts, S, out=X, ws=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        _, rep = step()
+    torch.cuda.synchronize()
+    iters = rep["iters"].cpu().numpy()
+    status = rep["status"].cpu().numpy()
+    flops_step = float(sum(gemm_count(it) for it in iters)) * 2.0 * N ** 3
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    stream = torch.cuda.current_stream()
+    try:  # nvidia-smi -i takes the UUID, which survives CUDA_VISIBLE_DEVICES remapping
+        clk = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    except Exception:
+        clk = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    time.sleep(0.3)
+    l0 = prism.kernel_launches()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = prism.kernel_launches() - l0
+    clocks = clk.stop()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max, units, flops, launches_all = reduce_timing(ms, BATCH * args.steps, flops_step * args.steps,
+                                                       launches, world)
+    value = flops / (ms_max / 1e3) / 1e12
+    precond_s = units / (ms_max / 1e3)
+
+    peaks, peak_src = load_peaks()
+    tf32_sust = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")) * TF32_OVER_BF16
+    split_peak = tf32_sust / 3.0  # three TF32 products per fp32-accurate product
+
+    # ---- end to end through the public API with host buffers
+    A_host = torch.from_numpy(A_np).pin_memory()
+    S_host = torch.from_numpy(S_np).pin_memory()
+    X_host = torch.empty_like(A_host).pin_memory()
+    st_host = torch.empty(BATCH, dtype=torch.int32).pin_memory()
+    A2 = torch.empty_like(A)
+    S2 = torch.empty_like(S)
+    barrier(world)
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        A2.copy_(A_host, non_blocking=True)
+        S2.copy_(S_host, non_blocking=True)
+        Xd, rep2 = prism.matfn_inv_root(A2, "inv4", opts, S2, out=X, ws=ws)
+        X_host.copy_(Xd, non_blocking=True)
+        st_host.copy_(rep2["status"], non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms, _, _, _ = reduce_timing(f0.elapsed_time(f1), 0, 0, 0, world)
+    e2e_value = flops / (e2e_ms / 1e3) / 1e12
+    h2d = A_host.numel() * 4 + S_host.numel() * 4
+    d2h = X_host.numel() * 4 + st_host.numel() * 4
+
+    # ---- roofline of the dominant kernel: the batched 3xTF32 tcgen05 GEMM,
+    # same launch configuration as inside the step (64 x 1024^3), timed alone
+    Yh, Yl = prism.shp_split_tf32(X)
+    Gh, Gl = prism.shp_split_tf32(A)
+    out = torch.empty_like(A)
+    for _ in range(3):
+        prism.shp_matmul(Yh, Gh, "3xtf32", A_lo=Yl, B_lo=Gl, out=out)
+    torch.cuda.synchronize()
+    reps = 40
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(reps):
+        prism.shp_matmul(Yh, Gh, "3xtf32", A_lo=Yl, B_lo=Gl, out=out)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    gemm_ms = g0.elapsed_time(g1) / reps
+    gemm_achieved = 2.0 * N ** 3 * BATCH / (gemm_ms / 1e3) / 1e12
+    roofline = {
+        "kernel": "k_gemm_tc<3xTF32> (batched 64 x 1024^3)",
+        "bound": "tensor", "achieved": gemm_achieved, "peak": split_peak, "unit": "TFLOP/s",
+        "frac": gemm_achieved / split_peak, "traffic": None,
+        "peak_note": f"{peak_src} sustained BF16 x 1.1/2.25 (TF32) / 3 (3xTF32 products)",
+        "ms_per_launch": gemm_ms,
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_tot, f_tot, nb = 0.0, 0.0, 0
+        for b in range(BATCH):
+            t, f = oracle_sample(A_np[b], S_np)
+            t_tot += t
+            f_tot += f
+            nb += 1
+            if t_tot > 10.0:
+                break
+        cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": f"{nb} of the 64 blocks, float64 NumPy/LAPACK oracle (same recurrence)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(world),
+            "preconditioners_per_s": precond_s,
+            "frac_of_3xtf32_peak": value / (split_peak * world),
+            "iters_per_pass": [int(x) for x in np.median(iters, axis=0)],
+            "status_ok_blocks": int((status == 0).sum()), "blocks": int(len(status)),
+            "gpu_launches": int(launches_all),
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -169,6 +169,28 @@ int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rro
                   int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
                   shp_stream stream);
 
+/* ---- Utilities (no counterpart on the pages; building blocks of the calls
+ * above, exposed for measurement and tests). ---- */
+
+/* C[b] = A[b] * B[b] on the tensor cores, the product every call above is
+ * built from.  Logical shapes: A is M x K, B is K x N, C is M x N fp32
+ * (bf16 for SHP_BF16), all row-major with no padding.  a_trans = 1 reads A
+ * from an K x M row-major buffer (A^T stored), b_trans = 1 reads B from an
+ * N x K row-major buffer.  prec: SHP_TF32 (fp32 inputs), SHP_BF16 (bf16
+ * inputs), or SHP_3XTF32 with A_lo/B_lo the low parts from shp_split_tf32
+ * (A/B then hold the high parts); A_lo/B_lo are ignored otherwise.
+ * One kernel launch; no workspace. */
+int shp_matmul(const void* A, const float* A_lo, int a_trans, const void* B, const float* B_lo,
+               int b_trans, void* C, int64_t M, int64_t N, int64_t K, int64_t batch, int prec,
+               shp_stream stream);
+
+/* hi = TF32(x) (round to nearest), lo = TF32(x - hi), for `count` floats. */
+int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream);
+
+/* Number of kernels this library has launched in the process so far
+ * (host-side counter, all threads and devices). */
+uint64_t shp_kernel_launches(void);
+
 /* Human-readable name of a status code (static storage). */
 const char* shp_status_string(int status);
 

@@ -23,7 +23,8 @@ SHP_POW_INV4, SHP_POW_INV2, SHP_POW_SQRT = 0, 1, 2
 SHP_OP_INV_ROOT, SHP_OP_POLAR, SHP_OP_ALPHA_FIT, SHP_OP_APPLY, SHP_OP_GRAM_EMA = 0, 1, 2, 3, 4
 
 EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar",
-           "prism_alpha_fit", "shampoo_apply", "shp_status_string", "shp_version")
+           "prism_alpha_fit", "shampoo_apply", "shp_matmul", "shp_split_tf32",
+           "shp_kernel_launches", "shp_status_string", "shp_version")
 
 
 class PrismOpts(ctypes.Structure):
@@ -55,6 +56,9 @@ _SIGS = {
                            ctypes.POINTER(PrismReport), _P, _SZ, _P]),
     "prism_alpha_fit": (_INT, [_P, _I64, _I64, _P, _INT, _INT, _F, _F, _P, _P, _P, _SZ, _P]),
     "shampoo_apply": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P, _SZ, _P]),
+    "shp_matmul": (_INT, [_P, _P, _INT, _P, _P, _INT, _P, _I64, _I64, _I64, _I64, _INT, _P]),
+    "shp_split_tf32": (_INT, [_P, _I64, _P, _P, _P]),
+    "shp_kernel_launches": (ctypes.c_uint64, []),
     "shp_status_string": (ctypes.c_char_p, [_INT]),
     "shp_version": (ctypes.c_char_p, []),
 }

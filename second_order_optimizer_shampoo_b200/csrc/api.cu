@@ -9,7 +9,15 @@
 #include "internal.h"
 #include "shampoo_prism.h"
 
+#include <atomic>
+
 using namespace shp;
+
+namespace shp {
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace shp
 
 namespace {
 
@@ -180,6 +188,38 @@ int sketch_and_alpha(const float* Rhi, const float* Rlo, int64_t n, int batch, c
 extern "C" {
 
 const char* shp_version(void) { return "0.1.0"; }
+
+uint64_t shp_kernel_launches(void) { return launch_count(); }
+
+int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream) {
+  if (!X || !hi || !lo || count < 0) return SHP_EINVAL;
+  CK(split_copy(X, count, hi, lo, static_cast<cudaStream_t>(stream)));
+  return SHP_OK;
+}
+
+int shp_matmul(const void* A, const float* A_lo, int a_trans, const void* B, const float* B_lo,
+               int b_trans, void* C, int64_t M, int64_t N, int64_t K, int64_t batch, int prec,
+               shp_stream stream) {
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || batch <= 0) return SHP_EINVAL;
+  if (prec != SHP_TF32 && prec != SHP_3XTF32 && prec != SHP_BF16) return SHP_EINVAL;
+  if (prec == SHP_3XTF32 && (!A_lo || !B_lo)) return SHP_EINVAL;
+  const int64_t q = prec == SHP_BF16 ? 8 : 4;  // elements per 16 bytes
+  // every memory row (M, N or K long, per the transposes) must be 16-byte aligned
+  if ((a_trans ? M : K) % q || (b_trans ? K : N) % q || N % q) return SHP_EINVAL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return SHP_EINVAL;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  const int mode = prec == SHP_BF16 ? MODE_BF16 : (prec == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32);
+  const bool split = prec == SHP_3XTF32;
+  // A^T stored (K x M) is the MN-major view of A; B stored (K x N) is MN-major,
+  // B^T stored (N x K) is K-major.
+  Operand a = op(A, split ? A_lo : nullptr, a_trans != 0, a_trans ? M : K, M * K);
+  Operand b = op(B, split ? B_lo : nullptr, b_trans == 0, b_trans ? K : N, K * N);
+  EpiParams e = epi(EPI_STORE, prec == SHP_BF16 ? OUT_BF16 : OUT_F32, C, nullptr, N, M * N,
+                    static_cast<int>(M), static_cast<int>(N), nullptr);
+  CK(gemm_tc(mode, a, b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+             static_cast<int>(batch), e, static_cast<cudaStream_t>(stream)));
+  return SHP_OK;
+}
 
 const char* shp_status_string(int s) {
   switch (s) {

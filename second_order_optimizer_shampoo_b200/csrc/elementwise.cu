@@ -28,7 +28,7 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
   } else if (fmt == OUT_SPLIT) {
     const float h = tf32_round(v);
     static_cast<float*>(hi)[off] = h;
-    lo[off] = v - h;
+    lo[off] = tf32_round(v - h);  // pre-rounded: the tensor core truncates
   } else {
     static_cast<__nv_bfloat16*>(hi)[off] = __float2bfloat16_rn(v);
   }
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     const float v = X[e];
     const float h = tf32_round(v);
     hi[e] = h;
-    lo[e] = v - h;
+    lo[e] = tf32_round(v - h);
   }
 }
 
@@ -250,12 +250,14 @@ __global__ void k_write_status(Ctl ctl, int batch, int* out) {
 
 cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st) {
   k_reset<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, first_pass);
+  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
                        cudaStream_t st) {
   k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(X, is_bf16, count, ctl.dnorm);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -265,6 +267,7 @@ cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, f
   const int fmt = Ylo != nullptr ? OUT_SPLIT : OUT_F32;
   k_coupled_init<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(A, n, ctl, fmt, Yhi, Ylo, Zhi,
                                                                Zlo, Rhi, Rlo);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -274,6 +277,7 @@ cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* 
   const int fmt = Ylo[0] != nullptr ? OUT_SPLIT : OUT_F32;
   k_coupled_restart<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(
       n, ctl, fmt, Yhi[0], Ylo[0], Yhi[1], Ylo[1], Zhi, Zlo, Rhi, Rlo);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -281,6 +285,7 @@ cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, c
                      int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st) {
   k_gform_d1<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(Rhi, Rlo, n, ctl, fmt, ghi, glo,
                                                            g2hi, g2lo);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -289,12 +294,14 @@ cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_expone
                            cudaStream_t st) {
   k_coupled_finish<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(n, ctl, c_exponent, Shi[0],
                                                                  Slo[0], Shi[1], Slo[1], X_out);
+  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st) {
   if (count <= 0) return cudaSuccess;
   k_split<<<ew_grid(count, 1), EW_THREADS, 0, st>>>(X, count, hi, lo);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -302,6 +309,7 @@ cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, cons
                        int fmt, void* Xhi, float* Xlo, cudaStream_t st) {
   k_polar_init<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, g_bf16, count, ctl, fmt, Xhi,
                                                              Xlo);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -310,12 +318,14 @@ cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
                          int out_bf16, cudaStream_t st) {
   k_polar_finish<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(count, ctl, fmt, Shi[0], Slo[0],
                                                                Shi[1], Slo[1], X_out, out_bf16);
+  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t write_status(const Ctl& ctl, int batch, int* report_status, cudaStream_t st) {
   if (report_status == nullptr) return cudaSuccess;
   k_write_status<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, report_status);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -56,7 +56,7 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
   } else if (fmt == OUT_SPLIT) {
     const float h = tf32_round(v);
     static_cast<float*>(hi)[off] = h;
-    lo[off] = v - h;
+    lo[off] = tf32_round(v - h);  // pre-rounded: the tensor core truncates
   } else {
     static_cast<__nv_bfloat16*>(hi)[off] = __float2bfloat16_rn(v);
   }
@@ -286,6 +286,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMa
   if (e != cudaSuccess) return e;
   dim3 grid((N + BN - 1) / BN, (M + 127) / 128, batch);
   k_gemm_tc<MODE, AMN, BMN><<<grid, 128, C::SMEM, st>>>(a, al, b, bl, K, BN, ep);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -6,6 +6,11 @@
 
 namespace shp {
 
+// Host-side count of kernel launches made by the library (every launcher
+// calls count_launch once per <<<>>>).
+void count_launch();
+uint64_t launch_count();
+
 enum Mode { MODE_TF32 = 0, MODE_3XTF32 = 1, MODE_BF16 = 2 };
 enum EpiKind { EPI_STORE = 0, EPI_RESID = 1, EPI_GPOLY = 2, EPI_EMA = 3, EPI_APPLY = 4 };
 enum OutFmt { OUT_F32 = 0, OUT_SPLIT = 1, OUT_BF16 = 2 };
@@ -14,7 +19,10 @@ enum OutFmt { OUT_F32 = 0, OUT_SPLIT = 1, OUT_BF16 = 2 };
 enum { ST_OK = 0, ST_ENOCONV = 16, ST_ESTALL = 17, ST_ENONFINITE = 18, ST_ETIMEOUT = 19 };
 
 // A batched row-major operand in HBM.  `hi` holds the fp32 value (TF32 mode),
-// the TF32-rounded high part (split mode, with `lo` = value - hi) or bf16.
+// the TF32-rounded high part (split mode, with `lo` = tf32(value - hi), so
+// that hi + lo equals the value to within 2^-22 relative) or bf16.  The
+// tensor cores truncate fp32 operands to TF32, hence both parts are stored
+// already rounded to nearest.
 //   mn == false (K-major): element (i, k) of the logical M x K (or N x K
 //     for B^T) operand sits at hi[i * ld + k];
 //   mn == true  (MN-major): element (i, k) sits at hi[k * ld + i].

@@ -310,6 +310,7 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
   else
     k_sketch<32><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
                                               vout_bstride, p, active);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -321,6 +322,7 @@ cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, floa
   const int64_t vbs = static_cast<int64_t>(2 * d + 2) * n * p;
   k_alpha<<<batch, AL_THREADS, 0, st>>>(V, n, p, d, vbs, lo, hi, fixed_alpha, active, alpha,
                                         J_coef, report_alpha, report_stride, report_slot);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -332,6 +334,7 @@ cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int k, int max_it
   k_control<<<(batch + 127) / 128, 128, 0, st>>>(ctl.bs, ctl.active, batch, n, k, max_iter, tol,
                                                  stall_below, stall_ratio, report_res, res_stride,
                                                  res_slot, report_iters, iters_slot);
+  count_launch();
   return cudaGetLastError();
 }
 

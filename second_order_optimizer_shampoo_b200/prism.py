@@ -165,3 +165,34 @@ def prism_alpha_fit(R, S, d: int, lo: float, hi: float, ws=None):
     _check(A.lib().prism_alpha_fit(_p(R), n, batch, _p(S), p, d, lo, hi, _p(alpha), _p(J), _p(ws),
                                    ws.numel(), _stream()), "prism_alpha_fit")
     return alpha, J
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(A.lib().shp_kernel_launches())
+
+
+def shp_split_tf32(X, hi=None, lo=None):
+    """(hi, lo) with hi = TF32(X), lo = TF32(X - hi)."""
+    _dev(X)
+    hi = torch.empty_like(X) if hi is None else hi
+    lo = torch.empty_like(X) if lo is None else lo
+    _check(A.lib().shp_split_tf32(_p(X), X.numel(), _p(hi), _p(lo), _stream()), "shp_split_tf32")
+    return hi, lo
+
+
+def shp_matmul(Amat, B, prec="tf32", a_trans=False, b_trans=False, A_lo=None, B_lo=None, out=None):
+    """Batched C = op(A) op(B) on the tensor cores (one kernel launch).
+
+    A: [batch][M][K] (or [batch][K][M] with a_trans), B: [batch][K][N] (or
+    [batch][N][K] with b_trans).  For prec='3xtf32' pass the high parts as
+    A/B and the low parts as A_lo/B_lo (see shp_split_tf32)."""
+    _dev(Amat, B, A_lo, B_lo, out)
+    M, K = (Amat.shape[-1], Amat.shape[-2]) if a_trans else (Amat.shape[-2], Amat.shape[-1])
+    N = B.shape[-2] if b_trans else B.shape[-1]
+    batch = Amat.numel() // (M * K)
+    dt = torch.bfloat16 if prec == "bf16" else torch.float32
+    out = torch.empty(batch, M, N, dtype=dt, device=Amat.device) if out is None else out
+    _check(A.lib().shp_matmul(_p(Amat), _p(A_lo), int(a_trans), _p(B), _p(B_lo), int(b_trans),
+                              _p(out), M, N, K, batch, _PREC[prec], _stream()), "shp_matmul")
+    return out

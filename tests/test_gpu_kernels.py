@@ -1,0 +1,101 @@
+"""GPU parity of the single-GEMM entry points and of the alpha fit, element by
+element against the float64 oracle, within the forward-error bound of the
+arithmetic (tests/helpers.py)."""
+import numpy as np
+import pytest
+
+from oracle import prism_ref as o
+from second_order_optimizer_shampoo_b200 import synth
+
+from helpers import gemm_bound, relerr, to_dev, to_host, U_FP32
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(128, 128, 1), (300, 196, 2), (64, 512, 1), (4, 4, 3), (516, 260, 1)]
+
+
+def prism():
+    from second_order_optimizer_shampoo_b200 import prism as p
+    return p
+
+
+@pytest.mark.parametrize("prec", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("m,n,batch", SHAPES)
+def test_gram_ema(prec, m, n, batch):
+    beta, eps = 0.95, 1e-3
+    G = synth.gaussian((batch, m, n), 1.0, 11)
+    L0 = synth.gaussian((batch, m, m), 0.1, 12)
+    L0 = (L0 + L0.transpose(0, 2, 1)).astype(np.float32)
+    R0 = synth.gaussian((batch, n, n), 0.1, 13)
+    R0 = (R0 + R0.transpose(0, 2, 1)).astype(np.float32)
+    Ld, Rd = to_dev(torch, L0), to_dev(torch, R0)
+    prism().shampoo_gram_ema(to_dev(torch, G), Ld, Rd, beta, eps, prec)
+    Lg, Rg = to_host(Ld), to_host(Rd)
+    for b in range(batch):
+        Lr, Rr = o.gram_ema_ref(G[b], L0[b], R0[b], beta, eps)
+        aG = np.abs(G[b].astype(np.float64))
+        bl = (1 - beta) * gemm_bound(aG, aG.T, n, prec) + 4 * U_FP32 * (np.abs(Lr) + beta * np.abs(L0[b]))
+        br = (1 - beta) * gemm_bound(aG.T, aG, m, prec) + 4 * U_FP32 * (np.abs(Rr) + beta * np.abs(R0[b]))
+        assert np.all(np.abs(Lg[b] - Lr) <= bl), np.max(np.abs(Lg[b] - Lr) / bl)
+        assert np.all(np.abs(Rg[b] - Rr) <= br), np.max(np.abs(Rg[b] - Rr) / br)
+
+
+@pytest.mark.parametrize("prec", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("m,n,batch", SHAPES)
+def test_apply(prec, m, n, batch):
+    lr = 0.1
+    W = synth.gaussian((batch, m, n), 0.02, 21)
+    G = synth.gaussian((batch, m, n), 0.02, 22)
+    PL = synth.gaussian((batch, m, m), 1.0, 23)
+    PR = synth.gaussian((batch, n, n), 1.0, 24)
+    Wd = to_dev(torch, W)
+    prism().shampoo_apply(Wd, to_dev(torch, G), to_dev(torch, PL), to_dev(torch, PR), lr, prec)
+    Wg = to_host(Wd)
+    for b in range(batch):
+        Wr = o.apply_ref(W[b], G[b], PL[b], PR[b], lr)
+        aL, aG, aR = (np.abs(x[b].astype(np.float64)) for x in (PL, G, PR))
+        # two chained products: |T| <= |PL||G|, errors add through the second GEMM
+        bound = lr * (gemm_bound(aL, aG, m, prec) @ aR + gemm_bound(aL @ aG, aR, n, prec))
+        bound += 2 * U_FP32 * np.abs(Wr)
+        assert np.all(np.abs(Wg[b] - Wr) <= bound), np.max(np.abs(Wg[b] - Wr) / bound)
+
+
+def residual_like(n, batch, seed, lo=0.0, hi=0.8):
+    """Symmetric matrices with spectrum in [lo, hi] (a residual R_k mid-iteration)."""
+    out = np.empty((batch, n, n), dtype=np.float32)
+    for b in range(batch):
+        g = np.random.default_rng((seed, b))
+        Q, _ = np.linalg.qr(g.standard_normal((n, n)))
+        lam = g.uniform(lo, hi, n)
+        out[b] = ((Q * lam) @ Q.T).astype(np.float32)
+    return out
+
+
+@pytest.mark.parametrize("d", [1, 2])
+@pytest.mark.parametrize("p", [1, 4, 8, 16, 32])
+@pytest.mark.parametrize("n", [64, 260])
+def test_alpha_fit(d, p, n):
+    batch = 3
+    R = residual_like(n, batch, 31 + p + n)
+    R[2] = (R[2] * -0.5).astype(np.float32)  # a residual with negative spectrum (overshoot)
+    S = synth.sketch_stack(1, n, p, 41)[0]
+    lo, hi = (0.5, 1.0) if d == 1 else (0.375, 1.0)
+    a, J = prism().prism_alpha_fit(to_dev(torch, R), to_dev(torch, S), d, lo, hi)
+    a, J = to_host(a), to_host(J)
+    for b in range(batch):
+        ar, Jr = o.prism_alpha_ref(R[b], S, d, lo, hi)
+        assert abs(a[b] - ar) <= 1e-4, (b, a[b], ar)
+        assert np.max(np.abs(J[b] - Jr)) <= 1e-4 * np.max(np.abs(Jr)), (J[b], Jr)
+
+
+def test_alpha_fit_interior_values_and_clamps():
+    # R = xi I gives the closed-form alpha; both an interior value and a clamp
+    n, p = 128, 8
+    S = synth.sketch_stack(1, n, p, 5)[0]
+    R = np.stack([0.5 * np.eye(n), 0.75 * np.eye(n), -0.5 * np.eye(n)]).astype(np.float32)
+    a, _ = prism().prism_alpha_fit(to_dev(torch, R), to_dev(torch, S), 1, 0.5, 1.0)
+    a = to_host(a)
+    assert a[0] == pytest.approx(2 * np.sqrt(2) - 2, abs=1e-5)
+    assert a[1] == pytest.approx(1.0, abs=1e-6)
+    assert a[2] == pytest.approx(0.5, abs=1e-6)

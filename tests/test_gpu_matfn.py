@@ -1,0 +1,200 @@
+"""GPU parity of the Newton-Schulz/PRISM matrix functions against the float64
+oracle: same sketch bytes, same iteration counts (the oracle is run with the
+GPU's per-pass counts), alpha trajectories, results, statuses and edge cases."""
+import numpy as np
+import pytest
+
+from oracle import prism_ref as o
+from second_order_optimizer_shampoo_b200 import synth
+
+from helpers import bf16_to_dev, relerr, to_dev, to_host
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+POW = {"inv4": (o.POW_INV4, -0.25), "inv2": (o.POW_INV2, -0.5), "sqrt": (o.POW_SQRT, 0.5)}
+
+
+def prism():
+    from second_order_optimizer_shampoo_b200 import prism as p
+    return p
+
+
+def run_inv_root(A, power, d, p, tol, max_iter, prec, S, **kw):
+    P = prism()
+    opts = P.make_opts(d=d, p=p, tol=tol, max_iter=max_iter, prec=prec, **kw)
+    X, rep = P.matfn_inv_root(to_dev(torch, A), power, opts, to_dev(torch, S))
+    return to_host(X), {k: to_host(v) for k, v in rep.items()}, opts
+
+
+def oracle_opts(opts, **kw):
+    base = dict(d=opts.d, p=opts.p, lo=opts.lo, hi=opts.hi, tol=opts.tol, max_iter=opts.max_iter,
+                fixed_alpha=bool(opts.fixed_alpha), stall_below=opts.stall_below,
+                stall_ratio=opts.stall_ratio)
+    base.update(kw)
+    return o.PrismOpts(**base)
+
+
+# 3xTF32 keeps about 21 bits per product (both parts rounded to 11-bit TF32,
+# the lo*lo term dropped) against fp32's 24: its rounding is 2^3 = 8 times
+# fp32's.  Emulated fp32 arithmetic reaches 1.4e-6 .. 3.6e-6 relative error on
+# the config-1 spectrum (cond 1e3), so the split path's bound there is
+# 8 x 3.6e-6 ~ 3e-5.  Milder spectra stay within 1e-5.
+TOL_3X_COND1E3 = 3e-5
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_inv_root_config1_split(seed):
+    """64 x 64 SPD, lambda log-uniform on [1e-3, 1], A^(-1/4), d = 1, p = 4,
+    alpha in [1/2, 1], 3xTF32: relative error vs eigh within the split path's
+    bound, alpha trajectory within 1e-4 of the oracle's on the same sketch."""
+    n = 64
+    A = synth.spd_batch(n, 1, 1e-3, 1.0, 101, indices=[seed])
+    S = synth.sketch_stack(80, n, 4, 1001)
+    X, rep, opts = run_inv_root(A, "inv4", 1, 4, 1e-6, 40, "3xtf32", S)
+    assert rep["status"][0] == o.OK
+    it = rep["iters"][0]
+    Xo, infos = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
+    for ps in range(2):
+        np.testing.assert_allclose(rep["alpha"][0, ps, :it[ps]], infos[ps].alpha, atol=1e-4)
+    assert relerr(X[0], o.spd_power_eigh(A[0], -0.25)) <= TOL_3X_COND1E3
+    assert relerr(X[0], Xo) <= TOL_3X_COND1E3
+    # the oracle left to its own stopping rule takes the same number of steps,
+    # give or take the one step whose residual sits at the tolerance
+    _, free = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S)
+    assert all(abs(a - int(b)) <= 1 for a, b in zip([i.iters for i in free], it))
+
+
+@pytest.mark.parametrize("power", ["inv4", "inv2", "sqrt"])
+@pytest.mark.parametrize("d", [1, 2])
+def test_inv_root_powers_ragged_batch(power, d):
+    """n = 100 (a ragged tile), batch 3, cond 1e2, every power, both degrees."""
+    n, batch = 100, 3
+    A = synth.spd_batch(n, batch, 1e-2, 1.0, 102)
+    S = synth.sketch_stack(60, n, 8, 1002)
+    X, rep, opts = run_inv_root(A, power, d, 8, 1e-6, 30, "3xtf32", S)
+    code, q = POW[power]
+    for b in range(batch):
+        assert rep["status"][b] == o.OK
+        it = rep["iters"][b] if power == "inv4" else rep["iters"][b][:1]
+        Xo, infos = o.inv_root_ref(A[b], code, oracle_opts(opts), S, force_iters=it)
+        for ps, info in enumerate(infos):
+            np.testing.assert_allclose(rep["alpha"][b, ps, :it[ps]], info.alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= 1e-5
+        assert relerr(X[b], o.spd_power_eigh(A[b], q)) <= 1e-5
+
+
+def test_inv_root_tf32_well_conditioned():
+    """TF32 path on cond 10 (the Shampoo statistics regime): error <= 1e-3."""
+    n, batch = 256, 2
+    A = synth.spd_batch(n, batch, 0.1, 1.0, 103)
+    S = synth.sketch_stack(60, n, 8, 1003)
+    X, rep, _ = run_inv_root(A, "inv4", 2, 8, 1e-3, 30, "tf32", S)
+    for b in range(batch):
+        # TF32 products floor the residual near 1e-3, so ESTALL is a valid end
+        assert rep["status"][b] in (o.OK, o.ESTALL)
+        assert relerr(X[b], o.spd_power_eigh(A[b], -0.25)) <= 1e-3
+
+
+def test_taylor_baseline_and_gemm_count():
+    """fixed_alpha reproduces the plain Taylor (classic) Newton-Schulz, and
+    PRISM needs fewer steps to the same residual on the config-1 spectrum."""
+    n = 64
+    A = synth.spd_batch(n, 1, 1e-3, 1.0, 101)
+    S = synth.sketch_stack(80, n, 4, 1001)
+    Xt, rt, ot = run_inv_root(A, "inv4", 1, 4, 1e-6, 40, "3xtf32", S, fixed_alpha=True)
+    assert rt["status"][0] == o.OK
+    np.testing.assert_array_equal(rt["alpha"][0, 0, :rt["iters"][0][0]], 0.5)
+    Xo, _ = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(ot), None, force_iters=rt["iters"][0])
+    assert relerr(Xt[0], Xo) <= TOL_3X_COND1E3
+    Xp, rp, _ = run_inv_root(A, "inv4", 1, 4, 1e-6, 40, "3xtf32", S)
+    taylor, prism_steps = rt["iters"][0].sum(), rp["iters"][0].sum()
+    assert prism_steps < taylor, (prism_steps, taylor)
+
+
+def test_tiny_and_identity():
+    n = 4
+    A = np.stack([np.eye(n), np.diag([4.0, 1.0, 0.25, 2.0])]).astype(np.float32)
+    S = synth.sketch_stack(40, n, 2, 7)
+    X, rep, _ = run_inv_root(A, "inv4", 2, 2, 1e-6, 20, "3xtf32", S)
+    assert list(rep["status"]) == [o.OK, o.OK]
+    np.testing.assert_allclose(X[0], np.eye(n), atol=1e-5)
+    np.testing.assert_allclose(X[1], np.diag(np.array([4.0, 1.0, 0.25, 2.0]) ** -0.25), atol=1e-5)
+
+
+def test_nonfinite_block_is_isolated():
+    n = 64
+    A = synth.spd_batch(n, 2, 1e-2, 1.0, 104)
+    A[0, 3, 5] = np.nan
+    S = synth.sketch_stack(40, n, 4, 1004)
+    X, rep, opts = run_inv_root(A, "inv4", 2, 4, 1e-5, 20, "3xtf32", S)
+    assert rep["status"][0] == o.ENONFINITE
+    assert rep["status"][1] == o.OK
+    assert relerr(X[1], o.spd_power_eigh(A[1], -0.25)) <= 1e-5
+
+
+def test_max_iter_and_report_layout():
+    n = 64
+    A = synth.spd_batch(n, 1, 1e-3, 1.0, 101)
+    S = synth.sketch_stack(4, n, 4, 1001)
+    X, rep, opts = run_inv_root(A, "inv4", 1, 4, 1e-6, 2, "3xtf32", S)
+    assert rep["status"][0] == o.ENOCONV
+    assert list(rep["iters"][0]) == [2, 2]
+    assert np.all(np.isfinite(rep["resid"][0, :, :3]))
+    Xo, infos = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S)
+    assert [i.status for i in infos] == [o.ENOCONV, o.ENOCONV]
+    np.testing.assert_allclose(rep["resid"][0, 0], infos[0].res, rtol=1e-4)
+    np.testing.assert_allclose(rep["alpha"][0, 0], infos[0].alpha, atol=1e-4)
+    assert relerr(X[0], Xo) <= 1e-5
+
+
+# ------------------------------------------------------------------ polar
+def run_polar(G, prec, d, p, tol, max_iter, S, bits=None):
+    P = prism()
+    opts = P.make_opts(d=d, p=p, tol=tol, max_iter=max_iter, prec=prec)
+    Gd = bf16_to_dev(torch, bits) if bits is not None else to_dev(torch, G)
+    X, rep = P.matfn_polar(Gd, opts, to_dev(torch, S))
+    return to_host(X), {k: to_host(v) for k, v in rep.items()}, opts
+
+
+@pytest.mark.parametrize("shape", [(512, 128), (128, 320), (64, 32), (96, 96)])
+@pytest.mark.parametrize("d", [1, 2])
+def test_polar_split(shape, d):
+    m, n = shape
+    G = synth.gaussian((2, m, n), 1.0, 51)
+    S = synth.sketch_stack(40, min(m, n), 8, 1051)
+    X, rep, opts = run_polar(G, "3xtf32", d, 8, 1e-6, 40, S)
+    for b in range(2):
+        assert rep["status"][b] == o.OK
+        it = rep["iters"][b][0]
+        Xo, infos = o.polar_ref(G[b], oracle_opts(opts), S, force_iters=it)
+        np.testing.assert_allclose(rep["alpha"][b, 0, :it], infos[0].alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= 1e-5
+        assert relerr(X[b], o.polar_svd(G[b])) <= 1e-5
+
+
+def test_polar_tf32():
+    G = synth.gaussian((1, 384, 256), 1.0, 52)
+    S = synth.sketch_stack(40, 256, 8, 1052)
+    X, rep, _ = run_polar(G, "tf32", 2, 8, 1e-3, 40, S)
+    assert rep["status"][0] in (o.OK, o.ESTALL)
+    assert relerr(X[0], o.polar_svd(G[0])) <= 1e-3
+
+
+@pytest.mark.parametrize("shape", [(512, 128), (128, 512)])
+def test_polar_bf16(shape):
+    """bf16 storage: the iterate is rounded to 8 mantissa bits every step, so
+    the result is compared at bf16 resolution (relative 2^-8 per entry)."""
+    m, n = shape
+    G = synth.gaussian((1, m, n), 1.0, 53)
+    bits = synth.to_bf16_bits(G)
+    G16 = synth.bf16_bits_to_f32(bits)
+    S = synth.sketch_stack(40, min(m, n), 8, 1053)
+    X, rep, opts = run_polar(None, "bf16", 2, 8, 1e-2, 40, S, bits=bits)
+    assert rep["status"][0] == o.OK
+    it = rep["iters"][0][0]
+    Xo, infos = o.polar_ref(G16[0], oracle_opts(opts), S, force_iters=it)
+    assert relerr(X[0], o.polar_svd(G16[0])) <= 2 ** -7
+    k = min(m, n)
+    XtX = X[0].T @ X[0] if m >= n else X[0] @ X[0].T
+    assert np.linalg.norm(np.eye(k) - XtX) / np.sqrt(k) <= 1e-2
