@@ -191,6 +191,33 @@ int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stre
  * (host-side counter, all threads and devices). */
 uint64_t shp_kernel_launches(void);
 
+/* ---- Alpha fit with no caller workspace (no counterpart on the pages). ----
+ *
+ * Same result as prism_alpha_fit, but the sketch vectors live in a fixed
+ * device array inside the library instead of a caller workspace, so the
+ * caller allocates nothing.  It is meant for callers that cannot allocate in
+ * the middle of their work: an optimizer step running under a framework whose
+ * caching allocator owns the free device memory (a raw cudaMalloc can fail
+ * there, and cudaFree synchronises the whole device), or a latency-bound loop
+ * that must not take the implicit synchronisation of cudaMalloc/cudaFree.
+ *
+ *   Limit: (2d+2) * n * p * batch * 4 bytes <= SHP_NOALLOC_SCRATCH_BYTES
+ *          (e.g. n = 1024, p = 8, d = 2: batch <= 21); larger sizes return
+ *          SHP_EUNSUPPORTED before any launch.
+ *   Memory: every GPU that loads the library holds SHP_NOALLOC_SCRATCH_BYTES
+ *          until the process exits.
+ *   Set-up: the first call on a device looks up the array's device address
+ *          (cudaGetSymbolAddress) with that device current; make that first
+ *          call before any stream capture.
+ *   Sharing: all calls use the same array, which keeps the previous call's
+ *          contents (nothing in it needs to start at zero); calls that overlap
+ *          on the GPU race on it, so serialise them (one stream, one thread).
+ * Arguments, layouts and the other return codes are those of prism_alpha_fit. */
+#define SHP_NOALLOC_SCRATCH_BYTES (4u << 20)
+int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const float* S, int p,
+                            int d, float lo, float hi, float* alpha_out, double* J_coef_out,
+                            shp_stream stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* shp_status_string(int status);
 
