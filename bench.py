@@ -246,9 +246,10 @@ def main():
     ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, N, N, BATCH, opts),
                      dtype=torch.uint8, device=dev)
     X = torch.empty_like(A)
+    rep_buf = prism.make_report(BATCH, MAX_ITER, dev)
 
     def step():
-        return prism.matfn_inv_root(A, "inv4", opts, S, out=X, ws=ws)
+        return prism.matfn_inv_root(A, "inv4", opts, S, out=X, ws=ws, report=rep_buf)
 
     for _ in range(max(args.warmup, 3)):
         _, rep = step()
@@ -303,7 +304,7 @@ def main():
     for _ in range(args.steps):
         A2.copy_(A_host, non_blocking=True)
         S2.copy_(S_host, non_blocking=True)
-        Xd, rep2 = prism.matfn_inv_root(A2, "inv4", opts, S2, out=X, ws=ws)
+        Xd, rep2 = prism.matfn_inv_root(A2, "inv4", opts, S2, out=X, ws=ws, report=rep_buf)
         X_host.copy_(Xd, non_blocking=True)
         st_host.copy_(rep2["status"], non_blocking=True)
     f1.record(stream)

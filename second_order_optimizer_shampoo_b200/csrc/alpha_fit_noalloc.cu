@@ -70,14 +70,15 @@ extern "C" int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch,
   if (scratch_address(&V) != cudaSuccess) return SHP_ECUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int B = static_cast<int>(batch);
-  if (shp::sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, st) != cudaSuccess)
+  if (shp::sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, nullptr, 0, st) !=
+      cudaSuccess)
     return SHP_ECUDA;
   for (int j = 2; j <= 2 * d + 1; ++j)
     if (shp::sketch_pass(R, nullptr, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, p, B,
-                         nullptr, st) != cudaSuccess)
+                         nullptr, nullptr, 0, st) != cudaSuccess)
       return SHP_ECUDA;
   if (shp::alpha_solve(V, n, p, d, B, lo, hi, 0, nullptr, alpha_out, J_coef_out, nullptr, 0, 0,
-                       st) != cudaSuccess)
+                       nullptr, st) != cudaSuccess)
     return SHP_ECUDA;
   return SHP_OK;
 }

@@ -3,21 +3,17 @@
 // Nothing here touches matrix data on the host; every step runs in the
 // kernels of gemm_tc.cu, sketch_alpha.cu and elementwise.cu.
 #include <math.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 
 #include "internal.h"
 #include "shampoo_prism.h"
 
-#include <atomic>
+#include <mutex>
+#include <vector>
 
 using namespace shp;
-
-namespace shp {
-static std::atomic<uint64_t> g_launches{0};
-void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
-uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
-}  // namespace shp
 
 namespace {
 
@@ -59,6 +55,8 @@ Ctl carve_ctl(Arena& a, int64_t batch) {
   c.dnorm = a.take<double>(batch);
   c.tmo = a.take<int>(batch);
   c.alpha = a.take<float>(batch);
+  c.it = a.take<int>(1);
+  c.flag = a.take<int>(1);
   return c;
 }
 
@@ -71,6 +69,7 @@ struct Bufs {
   float* Zlo[2];
   float* Rhi;
   float* Rlo;
+  float* Rs;  // plain fp32 R read by the sketch passes (= Rhi in TF32 mode)
   float* ghi;
   float* glo;
   float* V;
@@ -89,6 +88,7 @@ Bufs carve_inv_root(Arena& a, int64_t n, int64_t batch, const shp_prism_opts* o)
   }
   b.Rhi = a.take<float>(nn);
   b.Rlo = split ? a.take<float>(nn) : nullptr;
+  b.Rs = split ? a.take<float>(nn) : b.Rhi;
   b.ghi = a.take<float>(nn);
   b.glo = split ? a.take<float>(nn) : nullptr;
   b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * n * o->p * batch);
@@ -101,6 +101,7 @@ struct PolarBufs {
   float* Xlo[2];
   float* Rhi;
   float* Rlo;
+  float* Rs;  // plain fp32 R read by the sketch passes
   void* ghi;
   float* glo;
   float* V;
@@ -120,6 +121,7 @@ PolarBufs carve_polar(Arena& a, int64_t m, int64_t n, int64_t batch, int storage
   }
   b.Rhi = a.take<float>(kk);
   b.Rlo = split ? a.take<float>(kk) : nullptr;
+  b.Rs = split ? a.take<float>(kk) : b.Rhi;
   b.ghi = bf ? static_cast<void*>(a.take<uint16_t>(kk)) : static_cast<void*>(a.take<float>(kk));
   b.glo = split ? a.take<float>(kk) : nullptr;
   b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * k * o->p * batch);
@@ -165,22 +167,193 @@ Operand op(const void* hi, const float* lo, bool mn, int64_t ld, int64_t bs) {
     if ((x) != cudaSuccess) return SHP_ECUDA; \
   } while (0)
 
-// The sketch passes and the alpha solve of one iteration: V_1 = R S_k,
-// V_j = R V_{j-1} (j <= 2d+1), then the Gram, quartic and argmin.
-int sketch_and_alpha(const float* Rhi, const float* Rlo, int64_t n, int batch, const float* Sk,
-                     float* V, const shp_prism_opts* o, const Ctl& ctl, float* rep_alpha,
-                     int64_t rep_stride, int rep_slot, cudaStream_t st) {
-  const int64_t np = n * o->p;
+// The sketch passes and the alpha solve of iteration k = *ctl.it:
+// V_1 = R S[k] (S_pass is the pass's first slice), V_j = R V_{j-1}
+// (j <= 2d+1), then the Gram, the quartic and its argmin.
+int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass, float* V,
+                     const shp_prism_opts* o, const Ctl& ctl, float* rep_alpha,
+                     int64_t rep_stride, int rep_slot_base, cudaStream_t st) {
+  const int64_t np = n * o->p, nn = n * n;
   const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
   if (!o->fixed_alpha) {
-    CK(sketch_pass(Rhi, Rlo, n, n * n, Sk, 0, V + np, vbs, o->p, batch, ctl.active, st));
+    CK(sketch_pass(Rs, nullptr, n, nn, S_pass, 0, V + np, vbs, o->p, batch, ctl.active, ctl.it,
+                   np, st));
     for (int j = 2; j <= 2 * o->d + 1; ++j)
-      CK(sketch_pass(Rhi, Rlo, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
-                     ctl.active, st));
+      CK(sketch_pass(Rs, nullptr, n, nn, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
+                     ctl.active, nullptr, 0, st));
   }
   CK(alpha_solve(V, n, o->p, o->d, batch, o->lo, o->hi, o->fixed_alpha, ctl.active, ctl.alpha,
-                 nullptr, rep_alpha, rep_stride, rep_slot, st));
+                 nullptr, rep_alpha, rep_stride, rep_slot_base, ctl.it, st));
   return SHP_OK;
+}
+
+// ------------------------------------------------------------------------
+// Device-side iteration loop.  Each Newton-Schulz pass is recorded into a CUDA
+// graph: the k = 0 step, then a conditional WHILE node whose body runs two
+// steps (odd k on ping-pong slot 1, then, behind a conditional IF, even k on
+// slot 0).  After every step a one-CTA kernel advances the device iteration
+// counter and sets the condition to "some block still active"; blocks stop
+// independently in k_control.  No host synchronisation, and no launches for
+// steps after the last block has stopped.  Graphs are cached by the call's
+// pointers and sizes.
+
+struct CallKey {
+  int op, device, power, storage;
+  const void* a;
+  void* x;
+  const void* s;
+  int64_t s_count, m, n, batch;
+  shp_prism_opts o;
+  void* ws;
+  size_t ws_bytes;
+  const void* rep[4];
+};
+
+struct CachedGraph {
+  CallKey key;
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+};
+
+std::mutex g_graph_mu;
+std::vector<CachedGraph> g_graphs;
+constexpr size_t kGraphCacheMax = 16;
+constexpr int kMaxDev = 64;
+cudaStream_t g_cap[kMaxDev][3] = {};
+
+// Adds a conditional node after the current capture frontier of `st`, makes
+// it the new frontier and returns its body graph.
+cudaError_t add_conditional(cudaStream_t st, cudaGraphConditionalHandle h,
+                            cudaGraphConditionalNodeType type, cudaGraph_t* body) {
+  cudaStreamCaptureStatus cs;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t nd = 0;
+  cudaGraph_t g = nullptr;
+  cudaError_t e = cudaStreamGetCaptureInfo(st, &cs, nullptr, &g, &deps, &nd);
+  if (e != cudaSuccess) return e;
+  if (cs != cudaStreamCaptureStatusActive) return cudaErrorStreamCaptureInvalidated;
+  cudaGraphNodeParams p = {cudaGraphNodeTypeConditional};
+  p.conditional.handle = h;
+  p.conditional.type = type;
+  p.conditional.size = 1;
+  cudaGraphNode_t node;
+  e = cudaGraphAddNode(&node, g, deps, nd, &p);
+  if (e != cudaSuccess) return e;
+  *body = p.conditional.phGraph_out[0];
+  return cudaStreamUpdateCaptureDependencies(st, &node, 1, cudaStreamSetCaptureDependencies);
+}
+
+// iter(cur, first, stream) launches one step on ping-pong slot `cur`.
+// With g == nullptr the same steps run from a host loop that reads the
+// condition back after every step (diagnostic mode, SHP_HOST_LOOP=1, for
+// profilers that cannot look inside conditional graphs).
+template <class Iter>
+int record_loop(cudaStream_t const* cs, cudaGraph_t g, const Ctl& ctl, int batch, int max_iter,
+                Iter iter) {
+  if (g == nullptr) {
+    int r = iter(0, true, cs[0]);
+    if (r != SHP_OK) return r;
+    CK(loop_step(ctl, batch, 1, max_iter, 0, cs[0]));
+    for (int k = 1;; ++k) {
+      int flag = 0;
+      CK(cudaMemcpyAsync(&flag, ctl.flag, sizeof(int), cudaMemcpyDeviceToHost, cs[0]));
+      CK(cudaStreamSynchronize(cs[0]));
+      if (flag == 0) break;
+      r = iter(k & 1, false, cs[0]);
+      if (r != SHP_OK) return r;
+      CK(loop_step(ctl, batch, 1, max_iter, 0, cs[0]));
+    }
+    return SHP_OK;
+  }
+  const cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+  int r = iter(0, true, cs[0]);
+  if (r != SHP_OK) return r;
+  cudaGraphConditionalHandle hw, hif;
+  CK(cudaGraphConditionalHandleCreate(&hw, g, 0, cudaGraphCondAssignDefault));
+  CK(loop_step(ctl, batch, 1, max_iter, hw, cs[0]));
+  cudaGraph_t body = nullptr, body2 = nullptr;
+  CK(add_conditional(cs[0], hw, cudaGraphCondTypeWhile, &body));
+  CK(cudaGraphConditionalHandleCreate(&hif, body, 0, cudaGraphCondAssignDefault));
+  CK(cudaStreamBeginCaptureToGraph(cs[1], body, nullptr, nullptr, 0, mode));
+  r = iter(1, false, cs[1]);
+  if (r == SHP_OK && loop_step(ctl, batch, 1, max_iter, hif, cs[1]) != cudaSuccess) r = SHP_ECUDA;
+  if (r == SHP_OK && add_conditional(cs[1], hif, cudaGraphCondTypeIf, &body2) != cudaSuccess)
+    r = SHP_ECUDA;
+  if (r == SHP_OK) {
+    if (cudaStreamBeginCaptureToGraph(cs[2], body2, nullptr, nullptr, 0, mode) != cudaSuccess) {
+      r = SHP_ECUDA;
+    } else {
+      r = iter(0, false, cs[2]);
+      if (r == SHP_OK && loop_step(ctl, batch, 1, max_iter, hif, cs[2]) != cudaSuccess)
+        r = SHP_ECUDA;
+      cudaGraph_t g2 = nullptr;
+      if (cudaStreamEndCapture(cs[2], &g2) != cudaSuccess && r == SHP_OK) r = SHP_ECUDA;
+    }
+  }
+  if (r == SHP_OK && loop_step(ctl, batch, 0, max_iter, hw, cs[1]) != cudaSuccess) r = SHP_ECUDA;
+  cudaGraph_t g1 = nullptr;
+  if (cudaStreamEndCapture(cs[1], &g1) != cudaSuccess && r == SHP_OK) r = SHP_ECUDA;
+  return r;
+}
+
+// Finds or records (rec(capture streams, graph)) the graph of `key` and
+// launches it on `user`.
+template <class Rec>
+int run_graph(CallKey key, Rec rec, cudaStream_t user) {
+  CK(cudaGetDevice(&key.device));
+  if (key.device < 0 || key.device >= kMaxDev) return SHP_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  for (auto& c : g_graphs)
+    if (memcmp(&c.key, &key, sizeof(key)) == 0) {
+      CK(cudaGraphLaunch(c.exec, user));
+      return SHP_OK;
+    }
+  cudaStream_t* cs = g_cap[key.device];
+  for (int i = 0; i < 3; ++i)
+    if (cs[i] == nullptr) CK(cudaStreamCreateWithFlags(&cs[i], cudaStreamNonBlocking));
+  cudaGraph_t g = nullptr;
+  CK(cudaGraphCreate(&g, 0));
+  if (cudaStreamBeginCaptureToGraph(cs[0], g, nullptr, nullptr, 0,
+                                    cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return SHP_ECUDA;
+  }
+  int r = rec(static_cast<cudaStream_t const*>(cs), g);
+  cudaGraph_t g0 = nullptr;
+  if (cudaStreamEndCapture(cs[0], &g0) != cudaSuccess && r == SHP_OK) r = SHP_ECUDA;
+  cudaGraphExec_t exec = nullptr;
+  if (r == SHP_OK && cudaGraphInstantiate(&exec, g, 0) != cudaSuccess) r = SHP_ECUDA;
+  if (r != SHP_OK) {
+    cudaGetLastError();
+    cudaGraphDestroy(g);
+    return r;
+  }
+  if (g_graphs.size() >= kGraphCacheMax) {
+    cudaGraphExecDestroy(g_graphs.front().exec);
+    cudaGraphDestroy(g_graphs.front().graph);
+    g_graphs.erase(g_graphs.begin());
+  }
+  g_graphs.push_back(CachedGraph{key, g, exec});
+  CK(cudaGraphLaunch(exec, user));
+  return SHP_OK;
+}
+
+// Runs `rec` on the user's stream with host-driven loops (SHP_HOST_LOOP set),
+// else through the graph cache.
+template <class Rec>
+int dispatch(const CallKey& key, Rec rec, cudaStream_t user) {
+  if (getenv("SHP_HOST_LOOP") != nullptr) {
+    cudaStream_t cs[3] = {user, user, user};
+    return rec(static_cast<cudaStream_t const*>(cs), static_cast<cudaGraph_t>(nullptr));
+  }
+  return run_graph(key, rec, user);
+}
+
+CallKey make_key(int opk) {
+  CallKey k;
+  memset(&k, 0, sizeof(k));
+  k.op = opk;
+  return k;
 }
 
 }  // namespace
@@ -189,7 +362,10 @@ extern "C" {
 
 const char* shp_version(void) { return "0.1.0"; }
 
-uint64_t shp_kernel_launches(void) { return launch_count(); }
+uint64_t shp_kernel_launches(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return 0;
+  return kernel_runs_gemm() + kernel_runs_sketch() + kernel_runs_elementwise();
+}
 
 int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream) {
   if (!X || !hi || !lo || count < 0) return SHP_EINVAL;
@@ -384,11 +560,12 @@ int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, in
   float* V = a.take<float>(static_cast<size_t>(2 * d + 2) * n * p * batch);
   const int64_t np = n * p, vbs = static_cast<int64_t>(2 * d + 2) * np;
   const int B = static_cast<int>(batch);
-  CK(sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, st));
+  CK(sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, nullptr, 0, st));
   for (int j = 2; j <= 2 * d + 1; ++j)
     CK(sketch_pass(R, nullptr, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, p, B, nullptr,
-                   st));
-  CK(alpha_solve(V, n, p, d, B, lo, hi, 0, nullptr, alpha_out, J_coef_out, nullptr, 0, 0, st));
+                   nullptr, 0, st));
+  CK(alpha_solve(V, n, p, d, B, lo, hi, 0, nullptr, alpha_out, J_coef_out, nullptr, 0, 0,
+                 nullptr, st));
   return SHP_OK;
 }
 
@@ -405,82 +582,119 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
   if (n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
   if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_INV_ROOT, n, n, batch, o))
     return SHP_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
-  Bufs w = carve_inv_root(a, n, batch, o);
-  const Ctl& ctl = w.ctl;
-  const bool split = o->prec == SHP_3XTF32;
-  const int mode = split ? MODE_3XTF32 : MODE_TF32;
-  const int fmt = split ? OUT_SPLIT : OUT_F32;
-  const int N = static_cast<int>(n), B = static_cast<int>(batch);
-  const int64_t nn = n * n;
-  const int mi = o->max_iter;
-  float* rep_res = rep != nullptr ? rep->resid : nullptr;
-  float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
-  int* rep_iters = rep != nullptr ? rep->iters : nullptr;
-
-  for (int pass = 0; pass < npass; ++pass) {
-    CK(reset_pass(ctl, B, pass == 0, st));
-    if (pass == 0) {
-      CK(frob_norm2(A, 0, nn, B, ctl, st));
-      CK(coupled_init(A, n, B, ctl, w.Yhi[0], w.Ylo[0], w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo, st));
-    } else {
-      CK(coupled_restart(n, B, ctl, w.Yhi, w.Ylo, w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo, st));
-    }
-    for (int k = 0; k <= mi; ++k) {
-      const int cur = k & 1, nxt = cur ^ 1;
-      if (k > 0) {  // R_k = I - Z_k Y_k and ||R_k||_F^2
-        EpiParams e = epi(EPI_RESID, fmt, w.Rhi, w.Rlo, n, nn, N, N, &ctl);
-        CK(gemm_tc(mode, op(w.Zhi[cur], w.Zlo[cur], false, n, nn),
-                   op(w.Yhi[cur], w.Ylo[cur], true, n, nn), N, N, N, B, e, st));
-      }
-      CK(control_step(ctl, B, n, k, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
-                      2 * (mi + 1), pass * (mi + 1), rep_iters, pass, st));
-      if (k == mi) break;
-      const float* Sk = S != nullptr ? S + static_cast<int64_t>(pass * mi + k) * n * o->p : nullptr;
-      int r = sketch_and_alpha(w.Rhi, w.Rlo, n, B, Sk, w.V, o, ctl, rep_alpha, 2 * mi,
-                               pass * mi + k, st);
-      if (r != SHP_OK) return r;
-      // g = g_d(R_k; alpha_k); at k = 0 (Z_0 = I) it is also Z_1
-      float* z2hi = k == 0 ? w.Zhi[nxt] : nullptr;
-      float* z2lo = k == 0 ? w.Zlo[nxt] : nullptr;
-      if (o->d == 2) {
-        EpiParams e = epi(EPI_GPOLY, fmt, w.ghi, w.glo, n, nn, N, N, &ctl);
-        e.out2_hi = z2hi;
-        e.out2_lo = z2lo;
-        e.aux_hi = w.Rhi;
-        e.aux_lo = w.Rlo;
-        e.lda_aux = n;
-        e.bs_aux = nn;
-        e.s1 = 0.5f;
-        CK(gemm_tc(mode, op(w.Rhi, w.Rlo, false, n, nn), op(w.Rhi, w.Rlo, true, n, nn), N, N, N,
-                   B, e, st));
+  CallKey key = make_key(0);
+  key.power = power;
+  key.a = A;
+  key.x = X_out;
+  key.s = S;
+  key.s_count = S_count;
+  key.n = n;
+  key.batch = batch;
+  key.o = *o;
+  key.ws = ws;
+  key.ws_bytes = ws_bytes;
+  if (rep != nullptr) {
+    key.rep[0] = rep->status;
+    key.rep[1] = rep->iters;
+    key.rep[2] = rep->resid;
+    key.rep[3] = rep->alpha;
+  }
+  auto record = [&](cudaStream_t const* cs, cudaGraph_t g) -> int {
+    Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) &
+                                    ~(kAlign - 1)));
+    Bufs w = carve_inv_root(a, n, batch, o);
+    const Ctl& ctl = w.ctl;
+    const bool split = o->prec == SHP_3XTF32;
+    const int mode = split ? MODE_3XTF32 : MODE_TF32;
+    const int fmt = split ? OUT_SPLIT : OUT_F32;
+    const int N = static_cast<int>(n), B = static_cast<int>(batch);
+    const int64_t nn = n * n;
+    const int mi = o->max_iter;
+    float* rep_res = rep != nullptr ? rep->resid : nullptr;
+    float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
+    int* rep_iters = rep != nullptr ? rep->iters : nullptr;
+    for (int pass = 0; pass < npass; ++pass) {
+      CK(reset_pass(ctl, B, pass == 0, cs[0]));
+      if (pass == 0) {
+        CK(frob_norm2(A, 0, nn, B, ctl, cs[0]));
+        CK(coupled_init(A, n, B, ctl, w.Yhi[0], w.Ylo[0], w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo,
+                        split ? w.Rs : nullptr, cs[0]));
       } else {
-        CK(gform_d1(w.Rhi, w.Rlo, n, B, ctl, fmt, w.ghi, w.glo, z2hi, z2lo, st));
+        CK(coupled_restart(n, B, ctl, w.Yhi, w.Ylo, w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo,
+                           split ? w.Rs : nullptr, cs[0]));
       }
-      {  // Y_{k+1} = Y_k g
-        EpiParams e = epi(EPI_STORE, fmt, w.Yhi[nxt], w.Ylo[nxt], n, nn, N, N, &ctl);
-        CK(gemm_tc(mode, op(w.Yhi[cur], w.Ylo[cur], false, n, nn), op(w.ghi, w.glo, true, n, nn),
-                   N, N, N, B, e, st));
-      }
-      if (k > 0) {  // Z_{k+1} = g Z_k
-        EpiParams e = epi(EPI_STORE, fmt, w.Zhi[nxt], w.Zlo[nxt], n, nn, N, N, &ctl);
-        CK(gemm_tc(mode, op(w.ghi, w.glo, false, n, nn), op(w.Zhi[cur], w.Zlo[cur], true, n, nn),
-                   N, N, N, B, e, st));
-      }
+      const float* S_pass =
+          S != nullptr ? S + static_cast<int64_t>(pass) * mi * n * o->p : nullptr;
+      // one step of the coupled iteration on ping-pong slot `cur`; the k = 0
+      // step has R_0 = I - B from the start kernel and Z_1 = g (Z_0 = I)
+      auto iter = [&](int cur, bool first, cudaStream_t st) -> int {
+        const int nxt = cur ^ 1;
+        if (!first) {  // R_k = I - Z_k Y_k and ||R_k||_F^2
+          EpiParams e = epi(EPI_RESID, fmt, w.Rhi, w.Rlo, n, nn, N, N, &ctl);
+          if (split) e.out_plain = w.Rs;
+          CK(gemm_tc(mode, op(w.Zhi[cur], w.Zlo[cur], false, n, nn),
+                     op(w.Yhi[cur], w.Ylo[cur], true, n, nn), N, N, N, B, e, st));
+        }
+        CK(control_step(ctl, B, n, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
+                        2 * (mi + 1), pass * (mi + 1), rep_iters, pass, st));
+        int r = sketch_and_alpha(w.Rs, n, B, S_pass, w.V, o, ctl, rep_alpha, 2 * mi, pass * mi,
+                                 st);
+        if (r != SHP_OK) return r;
+        float* z2hi = first ? w.Zhi[nxt] : nullptr;
+        float* z2lo = first ? w.Zlo[nxt] : nullptr;
+        if (o->d == 2) {  // Delta = g - I = R/2 + alpha R^2 in the R R epilogue
+          EpiParams e = epi(EPI_GPOLY, fmt, w.ghi, w.glo, n, nn, N, N, &ctl);
+          e.out2_hi = z2hi;
+          e.out2_lo = z2lo;
+          e.aux_hi = w.Rhi;
+          e.aux_lo = w.Rlo;
+          e.aux_fmt = fmt;
+          e.lda_aux = n;
+          e.bs_aux = nn;
+          e.s1 = 0.5f;
+          CK(gemm_tc(mode, op(w.Rhi, w.Rlo, false, n, nn), op(w.Rhi, w.Rlo, true, n, nn), N, N,
+                     N, B, e, st));
+        } else {
+          CK(gform_d1(w.Rhi, w.Rlo, n, B, ctl, fmt, w.ghi, w.glo, z2hi, z2lo, st));
+        }
+        {  // Y_{k+1} = Y_k g = Y_k + Y_k Delta
+          EpiParams e = epi(EPI_AXPY, fmt, w.Yhi[nxt], w.Ylo[nxt], n, nn, N, N, &ctl);
+          e.aux_hi = w.Yhi[cur];
+          e.aux_lo = w.Ylo[cur];
+          e.aux_fmt = fmt;
+          e.lda_aux = n;
+          e.bs_aux = nn;
+          CK(gemm_tc(mode, op(w.Yhi[cur], w.Ylo[cur], false, n, nn),
+                     op(w.ghi, w.glo, true, n, nn), N, N, N, B, e, st));
+        }
+        if (!first) {  // Z_{k+1} = g Z_k = Z_k + Delta Z_k
+          EpiParams e = epi(EPI_AXPY, fmt, w.Zhi[nxt], w.Zlo[nxt], n, nn, N, N, &ctl);
+          e.aux_hi = w.Zhi[cur];
+          e.aux_lo = w.Zlo[cur];
+          e.aux_fmt = fmt;
+          e.lda_aux = n;
+          e.bs_aux = nn;
+          CK(gemm_tc(mode, op(w.ghi, w.glo, false, n, nn),
+                     op(w.Zhi[cur], w.Zlo[cur], true, n, nn), N, N, N, B, e, st));
+        }
+        return SHP_OK;
+      };
+      int r = record_loop(cs, g, ctl, B, mi, iter);
+      if (r != SHP_OK) return r;
     }
-  }
-  if (power == SHP_POW_SQRT) {
-    const float* sh[2] = {w.Yhi[0], w.Yhi[1]};
-    const float* sl[2] = {w.Ylo[0], w.Ylo[1]};
-    CK(coupled_finish(n, B, ctl, 0.5, sh, sl, X_out, st));
-  } else {
-    const float* sh[2] = {w.Zhi[0], w.Zhi[1]};
-    const float* sl[2] = {w.Zlo[0], w.Zlo[1]};
-    CK(coupled_finish(n, B, ctl, power == SHP_POW_INV2 ? -0.5 : -0.25, sh, sl, X_out, st));
-  }
-  if (rep != nullptr) CK(write_status(ctl, B, rep->status, st));
-  return SHP_OK;
+    if (power == SHP_POW_SQRT) {
+      const float* sh[2] = {w.Yhi[0], w.Yhi[1]};
+      const float* sl[2] = {w.Ylo[0], w.Ylo[1]};
+      CK(coupled_finish(n, B, ctl, 0.5, sh, sl, X_out, cs[0]));
+    } else {
+      const float* sh[2] = {w.Zhi[0], w.Zhi[1]};
+      const float* sl[2] = {w.Zlo[0], w.Zlo[1]};
+      CK(coupled_finish(n, B, ctl, power == SHP_POW_INV2 ? -0.5 : -0.25, sh, sl, X_out, cs[0]));
+    }
+    if (rep != nullptr) CK(write_status(ctl, B, rep->status, cs[0]));
+    return SHP_OK;
+  };
+  return dispatch(key, record, static_cast<cudaStream_t>(stream));
 }
 
 int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
@@ -497,69 +711,98 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
   oo.prec = storage;
   if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_POLAR, m, n, batch, &oo))
     return SHP_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
-  PolarBufs w = carve_polar(a, m, n, batch, storage, &oo);
-  const Ctl& ctl = w.ctl;
-  const bool tall = m >= n;
-  const int64_t k = tall ? n : m;  // Gram size
-  const int xmode = bf ? MODE_BF16 : (storage == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32);
-  const int xfmt = bf ? OUT_BF16 : (storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32);
-  const int rmode = bf ? MODE_TF32 : xmode;                  // R and R^2
-  const int rfmt = storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32;
-  const int M = static_cast<int>(m), N = static_cast<int>(n), K = static_cast<int>(k);
-  const int B = static_cast<int>(batch);
-  const int64_t mn = m * n, kk = k * k;
-  const int mi = o->max_iter;
-  float* rep_res = rep != nullptr ? rep->resid : nullptr;
-  float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
-  int* rep_iters = rep != nullptr ? rep->iters : nullptr;
-
-  CK(reset_pass(ctl, B, 1, st));
-  CK(frob_norm2(G, bf, mn, B, ctl, st));
-  CK(polar_init(G, bf, mn, B, ctl, xfmt, w.Xhi[0], w.Xlo[0], st));
-  for (int it = 0; it <= mi; ++it) {
-    const int cur = it & 1, nxt = cur ^ 1;
-    {  // R = I - X^T X (tall) or I - X X^T (wide), and ||R||_F^2
-      EpiParams e = epi(EPI_RESID, rfmt, w.Rhi, w.Rlo, k, kk, K, K, &ctl);
-      if (tall)
-        CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], true, n, mn),
-                   op(w.Xhi[cur], w.Xlo[cur], true, n, mn), K, K, M, B, e, st));
-      else
-        CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn),
-                   op(w.Xhi[cur], w.Xlo[cur], false, n, mn), K, K, N, B, e, st));
-    }
-    CK(control_step(ctl, B, k, it, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
-                    2 * (mi + 1), 0, rep_iters, 0, st));
-    if (it == mi) break;
-    const float* Sk = S != nullptr ? S + static_cast<int64_t>(it) * k * o->p : nullptr;
-    int r = sketch_and_alpha(w.Rhi, w.Rlo, k, B, Sk, w.V, o, ctl, rep_alpha, 2 * mi, it, st);
-    if (r != SHP_OK) return r;
-    if (o->d == 2) {  // g = I + R/2 + alpha R^2, stored like X
-      EpiParams e = epi(EPI_GPOLY, xfmt, w.ghi, w.glo, k, kk, K, K, &ctl);
-      e.aux_hi = w.Rhi;
-      e.aux_lo = w.Rlo;
-      e.lda_aux = k;
-      e.bs_aux = kk;
-      e.s1 = 0.5f;
-      CK(gemm_tc(rmode, op(w.Rhi, w.Rlo, false, k, kk), op(w.Rhi, w.Rlo, true, k, kk), K, K, K, B,
-                 e, st));
-    } else {
-      CK(gform_d1(w.Rhi, w.Rlo, k, B, ctl, xfmt, w.ghi, w.glo, nullptr, nullptr, st));
-    }
-    EpiParams e = epi(EPI_STORE, xfmt, w.Xhi[nxt], w.Xlo[nxt], n, mn, M, N, &ctl);
-    if (tall)  // X <- X g
-      CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn), op(w.ghi, w.glo, true, k, kk),
-                 M, N, N, B, e, st));
-    else  // X <- g^T X (the tall iteration applied to X^T)
-      CK(gemm_tc(xmode, op(w.ghi, w.glo, true, k, kk), op(w.Xhi[cur], w.Xlo[cur], true, n, mn),
-                 M, N, M, B, e, st));
+  CallKey key = make_key(1);
+  key.storage = storage;
+  key.a = G;
+  key.x = X_out;
+  key.s = S;
+  key.s_count = S_count;
+  key.m = m;
+  key.n = n;
+  key.batch = batch;
+  key.o = oo;
+  key.ws = ws;
+  key.ws_bytes = ws_bytes;
+  if (rep != nullptr) {
+    key.rep[0] = rep->status;
+    key.rep[1] = rep->iters;
+    key.rep[2] = rep->resid;
+    key.rep[3] = rep->alpha;
   }
-  const void* sh[2] = {w.Xhi[0], w.Xhi[1]};
-  const float* sl[2] = {w.Xlo[0], w.Xlo[1]};
-  CK(polar_finish(mn, B, ctl, xfmt, sh, sl, X_out, bf ? 1 : 0, st));
-  if (rep != nullptr) CK(write_status(ctl, B, rep->status, st));
-  return SHP_OK;
+  auto record = [&](cudaStream_t const* cs, cudaGraph_t g) -> int {
+    Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) &
+                                    ~(kAlign - 1)));
+    PolarBufs w = carve_polar(a, m, n, batch, storage, &oo);
+    const Ctl& ctl = w.ctl;
+    const bool tall = m >= n;
+    const int64_t k = tall ? n : m;  // Gram size
+    const int xmode = bf ? MODE_BF16 : (storage == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32);
+    const int xfmt = bf ? OUT_BF16 : (storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32);
+    const int rmode = bf ? MODE_TF32 : xmode;  // R and R^2
+    const int rfmt = storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32;
+    const int M = static_cast<int>(m), N = static_cast<int>(n), K = static_cast<int>(k);
+    const int B = static_cast<int>(batch);
+    const int64_t mn = m * n, kk = k * k;
+    const int mi = o->max_iter;
+    float* rep_res = rep != nullptr ? rep->resid : nullptr;
+    float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
+    int* rep_iters = rep != nullptr ? rep->iters : nullptr;
+    CK(reset_pass(ctl, B, 1, cs[0]));
+    CK(frob_norm2(G, bf, mn, B, ctl, cs[0]));
+    CK(polar_init(G, bf, mn, B, ctl, xfmt, w.Xhi[0], w.Xlo[0], cs[0]));
+    auto iter = [&](int cur, bool, cudaStream_t st) -> int {
+      const int nxt = cur ^ 1;
+      {  // R = I - X^T X (tall) or I - X X^T (wide), and ||R||_F^2
+        EpiParams e = epi(EPI_RESID, rfmt, w.Rhi, w.Rlo, k, kk, K, K, &ctl);
+        if (rfmt == OUT_SPLIT) e.out_plain = w.Rs;
+        if (tall)
+          CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], true, n, mn),
+                     op(w.Xhi[cur], w.Xlo[cur], true, n, mn), K, K, M, B, e, st));
+        else
+          CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn),
+                     op(w.Xhi[cur], w.Xlo[cur], false, n, mn), K, K, N, B, e, st));
+      }
+      CK(control_step(ctl, B, k, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
+                      2 * (mi + 1), 0, rep_iters, 0, st));
+      int r = sketch_and_alpha(w.Rs, k, B, S, w.V, o, ctl, rep_alpha, 2 * mi, 0, st);
+      if (r != SHP_OK) return r;
+      if (o->d == 2) {  // Delta = g - I = R/2 + alpha R^2, stored like X
+        EpiParams e = epi(EPI_GPOLY, xfmt, w.ghi, w.glo, k, kk, K, K, &ctl);
+        e.aux_hi = w.Rhi;
+        e.aux_lo = w.Rlo;
+        e.aux_fmt = rfmt;
+        e.lda_aux = k;
+        e.bs_aux = kk;
+        e.s1 = 0.5f;
+        CK(gemm_tc(rmode, op(w.Rhi, w.Rlo, false, k, kk), op(w.Rhi, w.Rlo, true, k, kk), K, K,
+                   K, B, e, st));
+      } else {
+        CK(gform_d1(w.Rhi, w.Rlo, k, B, ctl, xfmt, w.ghi, w.glo, nullptr, nullptr, st));
+      }
+      // X <- X g = X + X Delta (tall), X <- g^T X = X + Delta^T X (wide)
+      EpiParams e = epi(EPI_AXPY, xfmt, w.Xhi[nxt], w.Xlo[nxt], n, mn, M, N, &ctl);
+      e.aux_hi = w.Xhi[cur];
+      e.aux_lo = w.Xlo[cur];
+      e.aux_fmt = xfmt;
+      e.lda_aux = n;
+      e.bs_aux = mn;
+      if (tall)
+        CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn),
+                   op(w.ghi, w.glo, true, k, kk), M, N, N, B, e, st));
+      else  // the tall iteration applied to X^T
+        CK(gemm_tc(xmode, op(w.ghi, w.glo, true, k, kk),
+                   op(w.Xhi[cur], w.Xlo[cur], true, n, mn), M, N, M, B, e, st));
+      return SHP_OK;
+    };
+    int r = record_loop(cs, g, ctl, B, mi, iter);
+    if (r != SHP_OK) return r;
+    const void* sh[2] = {w.Xhi[0], w.Xhi[1]};
+    const float* sl[2] = {w.Xlo[0], w.Xlo[1]};
+    CK(polar_finish(mn, B, ctl, xfmt, sh, sl, X_out, bf ? 1 : 0, cs[0]));
+    if (rep != nullptr) CK(write_status(ctl, B, rep->status, cs[0]));
+    return SHP_OK;
+  };
+  return dispatch(key, record, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -55,6 +55,7 @@ SHP_DEV void block_add(float v, float* dst) {
 }
 
 __global__ void k_reset(Ctl ctl, int batch, int first) {
+  count_kernel_run();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
   BlockState& s = ctl.bs[b];
@@ -67,6 +68,7 @@ __global__ void k_reset(Ctl ctl, int batch, int first) {
   } else {
     s.iters1 = s.iters;
   }
+  if (b == 0) *ctl.it = 0;
   s.norm2 = 0.f;
   s.prev_res = INFINITY;
   s.iters = 0;
@@ -77,6 +79,7 @@ __global__ void k_reset(Ctl ctl, int batch, int first) {
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_frob(const void* X, int bf16, int64_t count, double* dnorm) {
+  count_kernel_run();
   const int b = blockIdx.y;
   double acc = 0.0;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
@@ -99,7 +102,8 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_init(const float* A, int64_t n, Ctl ctl, int fmt, float* Yhi, float* Ylo,
-                   float* Zhi, float* Zlo, float* Rhi, float* Rlo) {
+                   float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs) {
+  count_kernel_run();
   const int b = blockIdx.y;
   const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
   if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
@@ -114,6 +118,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     put(fmt, Yhi, Ylo, off, y);
     put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
     put(fmt, Rhi, Rlo, off, r);
+    if (Rs != nullptr) Rs[off] = r;
     nrm += r * r;
   }
   block_add(nrm, &ctl.bs[b].norm2);
@@ -121,7 +126,9 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_restart(int64_t n, Ctl ctl, int fmt, float* Y0hi, float* Y0lo, const float* Y1hi,
-                      const float* Y1lo, float* Zhi, float* Zlo, float* Rhi, float* Rlo) {
+                      const float* Y1lo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                      float* Rs) {
+  count_kernel_run();
   const int b = blockIdx.y;
   const bool from1 = (ctl.bs[b].iters1 & 1) != 0;
   const int64_t nn = n * n;
@@ -142,6 +149,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     const float r = (diag ? 1.f : 0.f) - y;
     put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
     put(fmt, Rhi, Rlo, off, r);
+    if (Rs != nullptr) Rs[off] = r;
     nrm += r * r;
   }
   block_add(nrm, &ctl.bs[b].norm2);
@@ -150,6 +158,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 __global__ void __launch_bounds__(EW_THREADS)
     k_gform_d1(const float* Rhi, const float* Rlo, int64_t n, Ctl ctl, int fmt, void* ghi,
                float* glo, void* g2hi, float* g2lo) {
+  count_kernel_run();
   const int b = blockIdx.y;
   if (ctl.active[b] == 0) return;
   const float a = ctl.alpha[b];
@@ -159,15 +168,16 @@ __global__ void __launch_bounds__(EW_THREADS)
     const int64_t off = b * nn + e;
     float r = Rhi[off];
     if (Rlo != nullptr) r += Rlo[off];
-    const float g = (((e / n) == (e % n)) ? 1.f : 0.f) + a * r;
-    put(fmt, ghi, glo, off, g);
-    if (g2hi != nullptr) put(fmt, g2hi, g2lo, off, g);
+    const float dlt = a * r;
+    put(fmt, ghi, glo, off, dlt);
+    if (g2hi != nullptr) put(fmt, g2hi, g2lo, off, (((e / n) == (e % n)) ? 1.f : 0.f) + dlt);
   }
 }
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_finish(int64_t n, Ctl ctl, double e_c, const float* S0hi, const float* S0lo,
                      const float* S1hi, const float* S1lo, float* X) {
+  count_kernel_run();
   const int b = blockIdx.y;
   const double c = static_cast<double>(ctl.bs[b].c);
   double sc;
@@ -193,6 +203,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_split(const float* X, int64_t count, float* hi, float* lo) {
+  count_kernel_run();
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
        e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
     const float v = X[e];
@@ -205,6 +216,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 __global__ void __launch_bounds__(EW_THREADS)
     k_polar_init(const void* G, int gbf16, int64_t count, Ctl ctl, int fmt, void* Xhi,
                  float* Xlo) {
+  count_kernel_run();
   const int b = blockIdx.y;
   const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
   if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
@@ -221,6 +233,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 __global__ void __launch_bounds__(EW_THREADS)
     k_polar_finish(int64_t count, Ctl ctl, int fmt, const void* S0hi, const float* S0lo,
                    const void* S1hi, const float* S1lo, void* X, int out_bf16) {
+  count_kernel_run();
   const int b = blockIdx.y;
   const bool one = (ctl.bs[b].iters & 1) != 0;
   const void* hi = one ? S1hi : S0hi;
@@ -241,6 +254,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 }
 
 __global__ void k_write_status(Ctl ctl, int batch, int* out) {
+  count_kernel_run();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
   out[b] = ctl.tmo[b] != 0 ? ST_ETIMEOUT : ctl.bs[b].status;
@@ -250,34 +264,30 @@ __global__ void k_write_status(Ctl ctl, int batch, int* out) {
 
 cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st) {
   k_reset<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, first_pass);
-  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
                        cudaStream_t st) {
   k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(X, is_bf16, count, ctl.dnorm);
-  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, float* Yhi,
-                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs,
                          cudaStream_t st) {
   const int fmt = Ylo != nullptr ? OUT_SPLIT : OUT_F32;
   k_coupled_init<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(A, n, ctl, fmt, Yhi, Ylo, Zhi,
-                                                               Zlo, Rhi, Rlo);
-  count_launch();
+                                                               Zlo, Rhi, Rlo, Rs);
   return cudaGetLastError();
 }
 
 cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* Yhi,
                             float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
-                            cudaStream_t st) {
+                            float* Rs, cudaStream_t st) {
   const int fmt = Ylo[0] != nullptr ? OUT_SPLIT : OUT_F32;
   k_coupled_restart<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(
-      n, ctl, fmt, Yhi[0], Ylo[0], Yhi[1], Ylo[1], Zhi, Zlo, Rhi, Rlo);
-  count_launch();
+      n, ctl, fmt, Yhi[0], Ylo[0], Yhi[1], Ylo[1], Zhi, Zlo, Rhi, Rlo, Rs);
   return cudaGetLastError();
 }
 
@@ -285,7 +295,6 @@ cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, c
                      int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st) {
   k_gform_d1<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(Rhi, Rlo, n, ctl, fmt, ghi, glo,
                                                            g2hi, g2lo);
-  count_launch();
   return cudaGetLastError();
 }
 
@@ -294,14 +303,12 @@ cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_expone
                            cudaStream_t st) {
   k_coupled_finish<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(n, ctl, c_exponent, Shi[0],
                                                                  Slo[0], Shi[1], Slo[1], X_out);
-  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st) {
   if (count <= 0) return cudaSuccess;
   k_split<<<ew_grid(count, 1), EW_THREADS, 0, st>>>(X, count, hi, lo);
-  count_launch();
   return cudaGetLastError();
 }
 
@@ -309,7 +316,6 @@ cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, cons
                        int fmt, void* Xhi, float* Xlo, cudaStream_t st) {
   k_polar_init<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, g_bf16, count, ctl, fmt, Xhi,
                                                              Xlo);
-  count_launch();
   return cudaGetLastError();
 }
 
@@ -318,15 +324,19 @@ cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
                          int out_bf16, cudaStream_t st) {
   k_polar_finish<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(count, ctl, fmt, Shi[0], Slo[0],
                                                                Shi[1], Slo[1], X_out, out_bf16);
-  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t write_status(const Ctl& ctl, int batch, int* report_status, cudaStream_t st) {
   if (report_status == nullptr) return cudaSuccess;
   k_write_status<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, report_status);
-  count_launch();
   return cudaGetLastError();
+}
+
+uint64_t kernel_runs_elementwise() {
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_kernel_runs, sizeof(v)) != cudaSuccess) return 0;
+  return v;
 }
 
 }  // namespace shp

@@ -11,7 +11,7 @@
 //                    their low parts in split mode) into a STAGES-deep ring;
 //   warp 1 lane 0  - MMA issuer: tcgen05.mma (M = 128, N = BN) into a TMEM
 //                    accumulator, tcgen05.commit frees each smem stage;
-//   all 4 warps    - epilogue: tcgen05.ld 32 lanes x 32 columns, transpose
+//   all 8 warps    - epilogue: tcgen05.ld 32 lanes x 32 columns, transpose
 //                    through padded smem so each warp store is one coalesced
 //                    128-byte row segment, fused elementwise op, store.
 // Modes: TF32 (fp32 operands read as TF32), 3xTF32 (operands kept as a TF32
@@ -31,7 +31,7 @@ namespace {
 
 constexpr int A_BYTES = 128 * 128;        // 128 rows x 128 bytes
 constexpr int B_BYTES_MAX = 256 * 128;    // BN <= 256 rows x 128 bytes
-constexpr int EPI_BYTES = 4 * 32 * 33 * 4;
+constexpr int EPI_BYTES = 8 * 32 * 33 * 4;  // epilogue staging, reuses stage memory
 
 template <int MODE>
 struct Cfg {
@@ -47,7 +47,8 @@ struct Cfg {
   static constexpr uint32_t MN_SBO = ESZ == 4 ? 512u : 1024u;
   static constexpr int STAGES = SPLIT ? 2 : 4;
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES_MAX) * (SPLIT ? 2 : 1);
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static_assert(STAGES * STAGE_BYTES >= EPI_BYTES, "epilogue staging must fit in the stages");
 };
 
 SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
@@ -63,10 +64,11 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
 }
 
 template <int MODE, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
               const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tBl,
               int K, int BN, EpiParams ep) {
+  count_kernel_run();
   using C = Cfg<MODE>;
   const int b = blockIdx.z;
   if (ep.active != nullptr && ep.active[b] == 0) return;
@@ -76,14 +78,16 @@ __global__ void __launch_bounds__(128, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* epi = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + EPI_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* done = empty + C::STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = static_cast<uint32_t>(BN);
+  // Split mode keeps the two small cross products (hi*lo, lo*hi) in a second
+  // accumulator: the tensor cores add into the accumulator with truncation,
+  // so the large hi*hi sum should take as few of those additions as possible.
+  const uint32_t ncols = static_cast<uint32_t>(C::SPLIT ? 2 * BN : BN);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -167,8 +171,9 @@ __global__ void __launch_bounds__(128, 1)
         } else {
           mma_tf32(tmem, ad[0], bd[0], idesc, acc0);
           if (C::SPLIT) {
-            mma_tf32(tmem, ad[0], bd[C::SPLIT ? 1 : 0], idesc, 1u);
-            mma_tf32(tmem, ad[C::SPLIT ? 1 : 0], bd[0], idesc, 1u);
+            const uint32_t tsmall = tmem + static_cast<uint32_t>(BN);
+            mma_tf32(tsmall, ad[0], bd[C::SPLIT ? 1 : 0], idesc, acc0);
+            mma_tf32(tsmall, ad[C::SPLIT ? 1 : 0], bd[0], idesc, 1u);
           }
         }
       }
@@ -177,58 +182,106 @@ __global__ void __launch_bounds__(128, 1)
     mma_commit(done);
   }
 
-  // ---------------- epilogue (all 4 warps; warp w owns TMEM lanes 32w..32w+31)
+  // ---------------- epilogue (8 warps).  Warp w reads TMEM lanes 32(w%4)..+31
+  // (the lane quarter its position in the warpgroup grants) and every other
+  // 32-column chunk starting at w/4.  Each chunk is transposed through padded
+  // shared memory (the pipeline stages are free once `done` fired) so that a
+  // lane owns one column of 32 rows: its 32 loads and 32 stores are
+  // independent and every warp access is one coalesced 128-byte row segment.
   if (!mbar_wait(done, 0)) timed_out = true;
   __syncwarp();
   tc_fence_after();
 
-  float* st = epi + warp * (32 * 33);
+  const int q = warp & 3, h = warp >> 2;
+  float* st = reinterpret_cast<float*>(smem) + warp * (32 * 33);
   const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;
   const bool diag_tile = (m0 < n0 + BN) && (n0 < m0 + 128);
+  const int row0 = m0 + q * 32;
+  const int rcount = ep.M - row0 < 32 ? ep.M - row0 : 32;
+  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY;
+  const bool need_old = ep.kind == EPI_EMA || ep.kind == EPI_APPLY;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
   float nrm = 0.f;
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = h; c < BN / 32; c += 2) {
     float v[32];
-    tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c * 32), v);
+    tmem_ld32(trow + static_cast<uint32_t>(c * 32), v);
+    if (C::SPLIT) {
+      float w[32];
+      tmem_ld32(trow + static_cast<uint32_t>(BN + c * 32), w);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += w[j];
+    }
 #pragma unroll
     for (int j = 0; j < 32; ++j) st[lane * 33 + j] = v[j];
     __syncwarp();
+    float a[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) a[r] = st[r * 33 + lane];
+    __syncwarp();
     const int gj = n0 + c * 32 + lane;
-    if (gj < ep.N) {
+    if (gj < ep.N && rcount > 0) {
+      const int64_t obase = static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row0) * ep.ldo + gj;
+      float x[32];
+      if (need_aux) {
+        const int64_t abase = static_cast<int64_t>(b) * ep.bs_aux +
+                              static_cast<int64_t>(row0) * ep.lda_aux + gj;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          float av = 0.f;
+          if (r < rcount) {
+            const int64_t oa = abase + static_cast<int64_t>(r) * ep.lda_aux;
+            if (ep.aux_fmt == OUT_BF16) {
+              av = __bfloat162float(static_cast<const __nv_bfloat16*>(ep.aux_hi)[oa]);
+            } else {
+              av = static_cast<const float*>(ep.aux_hi)[oa];
+              if (ep.aux_fmt == OUT_SPLIT) av += ep.aux_lo[oa];
+            }
+          }
+          x[r] = av;
+        }
+      } else if (need_old) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+          x[r] = r < rcount ? static_cast<const float*>(ep.out_hi)[obase + static_cast<int64_t>(r) * ep.ldo]
+                            : 0.f;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) x[r] = 0.f;
+      }
+#pragma unroll
       for (int r = 0; r < 32; ++r) {
-        const int gi = m0 + warp * 32 + r;
-        if (gi >= ep.M) break;
-        const float acc = st[r * 33 + lane];
+        if (r >= rcount) break;
+        const int gi = row0 + r;
+        const float acc = a[r];
         const float eye = (diag_tile && gi == gj) ? 1.f : 0.f;
-        const int64_t off = static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(gi) * ep.ldo + gj;
+        const int64_t off = obase + static_cast<int64_t>(r) * ep.ldo;
         float val;
         switch (ep.kind) {
           case EPI_RESID:
             val = eye - acc;
             nrm += val * val;
             break;
-          case EPI_GPOLY: {
-            const int64_t oa = static_cast<int64_t>(b) * ep.bs_aux +
-                               static_cast<int64_t>(gi) * ep.lda_aux + gj;
-            float rv = ep.aux_hi[oa];
-            if (ep.aux_lo != nullptr) rv += ep.aux_lo[oa];
-            val = eye + ep.s1 * rv + alpha * acc;
+          case EPI_GPOLY:
+            val = ep.s1 * x[r] + alpha * acc;
             break;
-          }
+          case EPI_AXPY:
+            val = x[r] + ep.s0 * acc;
+            break;
           case EPI_EMA:
-            val = ep.s0 * static_cast<const float*>(ep.out_hi)[off] + ep.s1 * acc + ep.s2 * eye;
+            val = ep.s0 * x[r] + ep.s1 * acc + ep.s2 * eye;
             break;
           case EPI_APPLY:
-            val = static_cast<const float*>(ep.out_hi)[off] + ep.s0 * acc;
+            val = x[r] + ep.s0 * acc;
             break;
           default:
             val = ep.s0 * acc;
             break;
         }
         put(ep.out_fmt, ep.out_hi, ep.out_lo, off, val);
-        if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, val);
+        if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, val + eye);
+        if (ep.out_plain != nullptr) ep.out_plain[off] = val;
       }
     }
-    __syncwarp();
   }
   if (ep.kind == EPI_RESID) {
     nrm = warp_sum(nrm);
@@ -285,8 +338,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMa
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((N + BN - 1) / BN, (M + 127) / 128, batch);
-  k_gemm_tc<MODE, AMN, BMN><<<grid, 128, C::SMEM, st>>>(a, al, b, bl, K, BN, ep);
-  count_launch();
+  k_gemm_tc<MODE, AMN, BMN><<<grid, 256, C::SMEM, st>>>(a, al, b, bl, K, BN, ep);
   return cudaGetLastError();
 }
 
@@ -343,6 +395,12 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
       return dispatch<MODE_BF16>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
   }
   return cudaErrorInvalidValue;
+}
+
+uint64_t kernel_runs_gemm() {
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_kernel_runs, sizeof(v)) != cudaSuccess) return 0;
+  return v;
 }
 
 }  // namespace shp

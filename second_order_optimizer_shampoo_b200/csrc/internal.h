@@ -6,13 +6,21 @@
 
 namespace shp {
 
-// Host-side count of kernel launches made by the library (every launcher
-// calls count_launch once per <<<>>>).
-void count_launch();
-uint64_t launch_count();
+// Kernels run so far on the current device, per translation unit (device
+// counters read back with a synchronous copy).
+uint64_t kernel_runs_gemm();
+uint64_t kernel_runs_sketch();
+uint64_t kernel_runs_elementwise();
 
 enum Mode { MODE_TF32 = 0, MODE_3XTF32 = 1, MODE_BF16 = 2 };
-enum EpiKind { EPI_STORE = 0, EPI_RESID = 1, EPI_GPOLY = 2, EPI_EMA = 3, EPI_APPLY = 4 };
+enum EpiKind {
+  EPI_STORE = 0,
+  EPI_RESID = 1,
+  EPI_GPOLY = 2,
+  EPI_EMA = 3,
+  EPI_APPLY = 4,
+  EPI_AXPY = 5
+};
 enum OutFmt { OUT_F32 = 0, OUT_SPLIT = 1, OUT_BF16 = 2 };
 
 // Per-block outcome codes (mirrors shp_status in include/shampoo_prism.h).
@@ -37,10 +45,14 @@ struct Operand {
 // What the epilogue does with accumulator element acc(i, j) of block b.
 //   STORE: v = s0 * acc
 //   RESID: v = [i==j] - acc, and norm2[b] += v^2
-//   GPOLY: v = [i==j] + s1 * aux(i,j) + alpha[b] * acc
+//   GPOLY: v = s1 * aux(i,j) + alpha[b] * acc   (Delta = g - I; out2 gets I + Delta)
 //   EMA:   v = s0 * out(i,j) + s1 * acc + s2 * [i==j]   (read-modify-write)
 //   APPLY: v = out(i,j) + s0 * acc                       (read-modify-write)
-// v is written to `out` (and to `out2` when non-null) in `out_fmt`.
+//   AXPY:  v = aux(i,j) + s0 * acc                       (X + X Delta)
+// v is written to `out` (and to `out2` when non-null) in `out_fmt`.  The
+// update polynomial is kept as Delta = g - I and applied as X + X Delta so
+// that its small part keeps full relative precision in every storage format
+// (g itself would round to 2^-8 near 1 in bf16).
 struct EpiParams {
   int kind;
   int out_fmt;
@@ -48,9 +60,11 @@ struct EpiParams {
   float* out_lo;
   void* out2_hi;
   float* out2_lo;
+  float* out_plain;  // optional plain fp32 copy of v (same layout as out)
   int64_t ldo, bso;
-  const float* aux_hi;
+  const void* aux_hi;
   const float* aux_lo;
+  int aux_fmt;  // OUT_F32 / OUT_SPLIT / OUT_BF16
   int64_t lda_aux, bs_aux;
   const float* alpha;
   float s0, s1, s2;
@@ -68,18 +82,20 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
 
 // ---- PRISM sketch and alpha (sketch_alpha.cu)
 // Vout[b] = R[b] * Vin[b]; R is n x n (hi + lo when lo != null); V is n x p.
-// vin_bstride == 0 shares Vin across the batch.
+// vin_bstride == 0 shares Vin across the batch.  When `it` is non-null the
+// input is Vin + (*it) * it_stride (the sketch slice of the current iteration).
 cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
                         const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
-                        int p, int batch, const int* active, cudaStream_t st);
+                        int p, int batch, const int* active, const int* it, int64_t it_stride,
+                        cudaStream_t st);
 // V is stored per block as [2d+2][n][p] (slot j holds V_j; slot 0 unused).
 // Gram of V_d..V_{2d+1}, the
 // quartic J(alpha) and its minimiser on [lo, hi]; writes alpha[b] and, when
-// non-null, J_coef[b][5] and report_alpha[b * stride + slot].
+// non-null, J_coef[b][5] and report_alpha[b * stride + slot (+ *it)].
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
-                        cudaStream_t st);
+                        const int* it, cudaStream_t st);
 
 // ---- per-block control (sketch_alpha.cu)
 struct BlockState {
@@ -99,11 +115,19 @@ struct Ctl {
   double* dnorm;  // ||input||_F^2 per block
   int* tmo;       // ST_ETIMEOUT flags from the GEMM pipeline
   float* alpha;   // alpha_k per block
+  int* it;        // iteration index k of the current pass (device-side loop)
+  int* flag;      // loop condition for the host-driven diagnostic loop
 };
-cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int k, int max_iter, float tol,
+// Stop test of iteration k = *ctl.it for every active block.
+cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int max_iter, float tol,
                          float stall_below, float stall_ratio, float* report_res,
                          int64_t res_stride, int res_slot, int* report_iters, int iters_slot,
                          cudaStream_t st);
+// End of an iteration of the device-side loop: *ctl.it += inc, then the
+// graph conditional `h` = (some block still active and *it <= max_iter + 1);
+// with h == 0 the condition goes to *ctl.flag instead (host-driven loop).
+cudaError_t loop_step(const Ctl& ctl, int batch, int inc, int max_iter,
+                      cudaGraphConditionalHandle h, cudaStream_t st);
 
 // ---- elementwise (elementwise.cu)
 // Start of a pass: active = 1, counters cleared; first_pass also clears the
@@ -113,15 +137,15 @@ cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t s
 cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
                        cudaStream_t st);
 // c = sqrt(dnorm); Y = A / c; Z = I; R = I - Y; norm2 = ||R||_F^2.
-// (lo pointers null in TF32 mode.)
+// (lo pointers null in TF32 mode; Rs, when non-null, gets a plain fp32 R.)
 cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, float* Yhi,
-                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
+                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs,
                          cudaStream_t st);
 // Pass 2: Y[0] <- Y[iters1 % 2]; Z = I; R = I - Y; norm2 = ||R||_F^2.
 cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* Yhi,
                             float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
-                            cudaStream_t st);
-// g = I + alpha[b] R (d = 1) in `fmt`; also into (g2hi, g2lo) when non-null.
+                            float* Rs, cudaStream_t st);
+// Delta = alpha[b] R (d = 1) in `fmt`; I + Delta into (g2hi, g2lo) when non-null.
 cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, const Ctl& ctl,
                      int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st);
 // X_out[b] = c_b^e * S[iters_b % 2][b] (hi + lo), S = the two ping-pong slots.

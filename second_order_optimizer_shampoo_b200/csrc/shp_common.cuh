@@ -17,6 +17,14 @@
 
 namespace shp {
 
+// Kernels this translation unit has run on the current device: the first
+// thread of the first CTA of every kernel adds one (before any early exit).
+static __device__ unsigned long long g_kernel_runs;
+SHP_DEV void count_kernel_run() {
+  if ((threadIdx.x | threadIdx.y | threadIdx.z | blockIdx.x | blockIdx.y | blockIdx.z) == 0)
+    atomicAdd(&g_kernel_runs, 1ull);
+}
+
 SHP_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -33,7 +33,9 @@ template <int P>
 __global__ void __launch_bounds__(SK_THREADS)
     k_sketch(const float* __restrict__ Rhi, const float* __restrict__ Rlo, int64_t n,
              int64_t rbs, const float* __restrict__ Vin, int64_t vbs, float* __restrict__ Vout,
-             int64_t obs, int p, const int* __restrict__ active) {
+             int64_t obs, int p, const int* __restrict__ active, const int* __restrict__ it,
+             int64_t it_stride) {
+  count_kernel_run();
   constexpr int ROWS = P <= 16 ? 4 : 2;
   __shared__ float Vs[P][SK_CHUNK];
   const int b = blockIdx.y;
@@ -42,7 +44,7 @@ __global__ void __launch_bounds__(SK_THREADS)
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (8 * ROWS) + warp * ROWS;
   const float* R = Rhi + b * rbs;
   const float* RL = Rlo != nullptr ? Rlo + b * rbs : nullptr;
-  const float* V = Vin + b * vbs;
+  const float* V = Vin + b * vbs + (it != nullptr ? static_cast<int64_t>(*it) * it_stride : 0);
   float acc[ROWS][P];
 #pragma unroll
   for (int r = 0; r < ROWS; ++r)
@@ -201,9 +203,12 @@ constexpr int AL_THREADS = 256;
 __global__ void __launch_bounds__(AL_THREADS)
     k_alpha(const float* __restrict__ V, int64_t n, int p, int d, int64_t vbs, float lo,
             float hi, int fixed, const int* __restrict__ active, float* __restrict__ alpha,
-            double* __restrict__ Jc, float* __restrict__ rep, int64_t rep_stride, int rep_slot) {
+            double* __restrict__ Jc, float* __restrict__ rep, int64_t rep_stride, int rep_slot,
+            const int* __restrict__ it) {
+  count_kernel_run();
   const int b = blockIdx.x;
   if (active != nullptr && active[b] == 0) return;
+  if (it != nullptr) rep_slot += *it;
   if (fixed) {  // plain Taylor step: alpha = lo, no sketch needed
     if (threadIdx.x == 0) {
       alpha[b] = lo;
@@ -262,11 +267,14 @@ __global__ void __launch_bounds__(AL_THREADS)
   if (rep != nullptr) rep[b * rep_stride + rep_slot] = static_cast<float>(a);
 }
 
-__global__ void k_control(BlockState* bs, int* active, int batch, int64_t n, int k, int max_iter,
-                          float tol, float stall_below, float stall_ratio, float* rep_res,
-                          int64_t res_stride, int res_slot, int* rep_iters, int iters_slot) {
+__global__ void k_control(BlockState* bs, int* active, const int* it, int batch, int64_t n,
+                          int max_iter, float tol, float stall_below, float stall_ratio,
+                          float* rep_res, int64_t res_stride, int res_slot, int* rep_iters,
+                          int iters_slot) {
+  count_kernel_run();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch || active[b] == 0) return;
+  const int k = *it;
   BlockState& s = bs[b];
   const float r = sqrtf(s.norm2 / static_cast<float>(n));
   s.norm2 = 0.f;
@@ -294,48 +302,77 @@ __global__ void k_control(BlockState* bs, int* active, int batch, int64_t n, int
 
 cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
                         const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
-                        int p, int batch, const int* active, cudaStream_t st) {
+                        int p, int batch, const int* active, const int* it, int64_t it_stride,
+                        cudaStream_t st) {
   if (batch <= 0 || n <= 0) return cudaSuccess;
   const int rows = p <= 16 ? 4 : 2;
   dim3 grid(static_cast<unsigned>((n + 8 * rows - 1) / (8 * rows)), batch);
   if (p <= 4)
     k_sketch<4><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
-                                             vout_bstride, p, active);
+                                             vout_bstride, p, active, it, it_stride);
   else if (p <= 8)
     k_sketch<8><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
-                                             vout_bstride, p, active);
+                                             vout_bstride, p, active, it, it_stride);
   else if (p <= 16)
     k_sketch<16><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
-                                              vout_bstride, p, active);
+                                              vout_bstride, p, active, it, it_stride);
   else
     k_sketch<32><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
-                                              vout_bstride, p, active);
-  count_launch();
+                                              vout_bstride, p, active, it, it_stride);
   return cudaGetLastError();
 }
 
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
-                        cudaStream_t st) {
+                        const int* it, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
   const int64_t vbs = static_cast<int64_t>(2 * d + 2) * n * p;
   k_alpha<<<batch, AL_THREADS, 0, st>>>(V, n, p, d, vbs, lo, hi, fixed_alpha, active, alpha,
-                                        J_coef, report_alpha, report_stride, report_slot);
-  count_launch();
+                                        J_coef, report_alpha, report_stride, report_slot, it);
   return cudaGetLastError();
 }
 
-cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int k, int max_iter, float tol,
+cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int max_iter, float tol,
                          float stall_below, float stall_ratio, float* report_res,
                          int64_t res_stride, int res_slot, int* report_iters, int iters_slot,
                          cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
-  k_control<<<(batch + 127) / 128, 128, 0, st>>>(ctl.bs, ctl.active, batch, n, k, max_iter, tol,
-                                                 stall_below, stall_ratio, report_res, res_stride,
-                                                 res_slot, report_iters, iters_slot);
-  count_launch();
+  k_control<<<(batch + 127) / 128, 128, 0, st>>>(ctl.bs, ctl.active, ctl.it, batch, n, max_iter,
+                                                 tol, stall_below, stall_ratio, report_res,
+                                                 res_stride, res_slot, report_iters, iters_slot);
   return cudaGetLastError();
+}
+
+namespace {
+__global__ void k_loop_step(const int* active, int* it, int* flag, int batch, int inc,
+                            int max_iter, cudaGraphConditionalHandle h) {
+  count_kernel_run();
+  int any = 0;
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) any |= active[b];
+  any = __syncthreads_or(any);
+  if (threadIdx.x == 0) {
+    const int k = *it + inc;
+    *it = k;
+    const unsigned cond = (any != 0 && k <= max_iter + 1) ? 1u : 0u;
+    if (h != 0)
+      cudaGraphSetConditional(h, cond);
+    else
+      *flag = static_cast<int>(cond);
+  }
+}
+}  // namespace
+
+cudaError_t loop_step(const Ctl& ctl, int batch, int inc, int max_iter,
+                      cudaGraphConditionalHandle h, cudaStream_t st) {
+  k_loop_step<<<1, 256, 0, st>>>(ctl.active, ctl.it, ctl.flag, batch, inc, max_iter, h);
+  return cudaGetLastError();
+}
+
+uint64_t kernel_runs_sketch() {
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_kernel_runs, sizeof(v)) != cudaSuccess) return 0;
+  return v;
 }
 
 }  // namespace shp

@@ -109,15 +109,25 @@ def _report_struct(rep):
                                       rep["resid"].data_ptr(), rep["alpha"].data_ptr()))
 
 
+def make_report(batch, max_iter, device):
+    """Device tensors for the per-block trajectory (status, iters, resid, alpha)."""
+    return _report(batch, max_iter, device)
+
+
 def matfn_inv_root(Amat, power="inv4", opts: A.PrismOpts | None = None, S=None, out=None,
                    report=True, ws=None):
-    """A^(-1/4) (or A^(-1/2), A^(1/2)) of a batch of SPD matrices."""
+    """A^(-1/4) (or A^(-1/2), A^(1/2)) of a batch of SPD matrices.
+
+    report: True (fresh tensors), False, or a dict from make_report() to reuse;
+    the library caches one CUDA graph per distinct set of pointers and sizes,
+    so reusing out/ws/report buffers keeps repeated calls on the cached graph."""
     opts = opts or make_opts()
     _dev(Amat, S, out)
     n = Amat.shape[-1]
     batch = Amat.numel() // (n * n)
     out = torch.empty_like(Amat) if out is None else out
-    rep = _report(batch, opts.max_iter, Amat.device) if report else None
+    rep = report if isinstance(report, dict) else (
+        _report(batch, opts.max_iter, Amat.device) if report else None)
     need = shp_workspace_bytes(A.SHP_OP_INV_ROOT, n, n, batch, opts)
     ws = _ws(need, Amat.device) if ws is None else ws
     s_count = 0 if S is None else S.shape[0]
@@ -140,7 +150,8 @@ def matfn_polar(G, opts: A.PrismOpts | None = None, S=None, out=None, report=Tru
     else:
         raise ValueError("G must be float32 or bfloat16")
     out = torch.empty_like(G) if out is None else out
-    rep = _report(batch, opts.max_iter, G.device) if report else None
+    rep = report if isinstance(report, dict) else (
+        _report(batch, opts.max_iter, G.device) if report else None)
     o2 = A.PrismOpts.from_buffer_copy(opts)
     o2.prec = storage
     need = shp_workspace_bytes(A.SHP_OP_POLAR, m, n, batch, o2)
