@@ -19,6 +19,8 @@ from __future__ import annotations
 
 import argparse
 import json
+
+import numpy as np
 import os
 import statistics
 import subprocess
@@ -203,6 +205,59 @@ def gemm_only(args):
     return 0
 
 
+PM, PN, PBATCH, PRANK = 4096, 1024, 96, 64
+
+
+def polar_flops(iters):
+    """Algorithmic flops of one polar factor with k updates: per update the
+    symmetric X^T X (n(n+1)m) and R^2 (n(n+1)n) and X Delta (2mn^2), plus the
+    final residual."""
+    k = int(iters)
+    sym = PN * (PN + 1) * PM
+    return k * (sym + PN * (PN + 1) * PN + 2 * PM * PN * PN) + sym
+
+
+def polar_leg(args, dev, stream):
+    """The Muon-style polar batch: 96 matrices 4096 x 1024, rank-64 signal plus
+    0.01 noise, bf16 storage, d = 2, p = 8, until ||I - X^T X||_F / sqrt(n) <= 1e-2."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import _abi, prism, synth
+    bits, _ = synth.lowrank_noise_batch(PM, PN, PRANK, 0.01, PBATCH, 104)
+    G = torch.from_numpy(bits.view("int16")).to(dev).view(torch.bfloat16)
+    S = torch.from_numpy(synth.sketch_stack(40, PN, 8, 1004)).to(dev)
+    opts = prism.make_opts(d=2, p=8, tol=1e-2, max_iter=40, prec="bf16")
+    o2 = _abi.PrismOpts.from_buffer_copy(opts)
+    o2.prec = _abi.SHP_BF16
+    ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_POLAR, PM, PN, PBATCH, o2),
+                     dtype=torch.uint8, device=dev)
+    X = torch.empty_like(G)
+    rep = prism.make_report(PBATCH, 40, dev)
+    for _ in range(2):
+        prism.matfn_polar(G, opts, S, out=X, ws=ws, report=rep)
+    torch.cuda.synchronize()
+    iters = rep["iters"][:, 0].cpu().numpy()
+    ok = int((rep["status"].cpu().numpy() == 0).sum())
+    flops = float(sum(polar_flops(k) for k in iters))
+    reps = 3
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        prism.matfn_polar(G, opts, S, out=X, ws=ws, report=rep)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    peaks, _ = load_peaks()
+    bf16_sust = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": "polar_96x4096x1024_bf16_lowrank64_prism_d2_p8_tol1e-2",
+            "value": tf, "unit": "TFLOP/s", "ms_per_step": ms,
+            "matrices_per_s": PBATCH / (ms / 1e3), "median_iters": float(np.median(iters)),
+            "status_ok": ok, "frac_of_bf16_peak": tf / bf16_sust,
+            "note": "symmetric products counted n(n+1)K; computed as full GEMMs"}
+
+
 # ------------------------------------------------------------------ our leg
 def main():
     ap = argparse.ArgumentParser()
@@ -211,6 +266,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-polar", action="store_true", help="skip the polar-factor leg")
     ap.add_argument("--kernel", default=None, choices=["gemm"],
                     help="run only the batched 3xTF32 GEMM (for profiling)")
     ap.add_argument("--batch", type=int, default=BATCH)
@@ -341,6 +397,8 @@ def main():
         "ms_per_launch": gemm_ms,
     }
 
+    polar = None if args.no_polar else polar_leg(args, dev, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_tot, f_tot, nb = 0.0, 0.0, 0
@@ -369,6 +427,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "roofline": roofline,
+            "polar": polar,
             "cpu_baseline": cpu,
             "clocks": clocks,
         }

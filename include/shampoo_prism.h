@@ -154,7 +154,7 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
 /* One sketched alpha fit ([PRISM] Parte II.1-II.2) on given residuals:
  *   V_0 = S, V_j = R V_{j-1} (j <= 2d+1), M_ij = <V_i, V_j>_F (i, j = d..2d+1),
  *   J(alpha) = sum_ij r_i(alpha) r_j(alpha) M_ij,  alpha* = argmin_{[lo,hi]} J.
- * R: [batch][n][n] fp32; S: [n][p] fp32 shared by the batch;
+ * R: [batch][n][n] fp32 (n a multiple of 4); S: [n][p] fp32 shared by the batch;
  * alpha_out: [batch] fp32; J_coef_out: [batch][5] fp64 coefficients of
  * alpha^0..alpha^4, or NULL. */
 int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, int p, int d,

@@ -61,6 +61,7 @@ extern "C" int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch,
                                        double* J_coef_out, shp_stream stream) {
   if (!R || !S || !alpha_out || n <= 0 || batch <= 0 || p < 1 || p > 32 || (d != 1 && d != 2))
     return SHP_EINVAL;
+  if (n % 4 || (reinterpret_cast<uintptr_t>(R) & 15u) != 0) return SHP_EINVAL;
   if (!(isfinite(lo) && isfinite(hi)) || lo > hi) return SHP_EINVAL;
   if (batch > 65535 || n > INT32_MAX) return SHP_EUNSUPPORTED;
   const int64_t np = n * p;

@@ -548,6 +548,7 @@ int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, in
                     size_t ws_bytes, shp_stream stream) {
   if (!R || !S || !alpha_out || n <= 0 || batch <= 0 || p < 1 || p > 32 || (d != 1 && d != 2))
     return SHP_EINVAL;
+  if (n % 4 || !aligned16(R)) return SHP_EINVAL;
   if (!(isfinite(lo) && isfinite(hi)) || lo > hi) return SHP_EINVAL;
   if (batch > 65535) return SHP_EUNSUPPORTED;
   shp_prism_opts o{};

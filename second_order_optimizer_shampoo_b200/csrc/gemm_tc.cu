@@ -20,6 +20,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "internal.h"
@@ -29,26 +31,38 @@ namespace shp {
 
 namespace {
 
-constexpr int A_BYTES = 128 * 128;        // 128 rows x 128 bytes
-constexpr int B_BYTES_MAX = 256 * 128;    // BN <= 256 rows x 128 bytes
 constexpr int EPI_BYTES = 8 * 32 * 33 * 4;  // epilogue staging, reuses stage memory
 
-template <int MODE>
+// Tiling.  Every operand row of a stage is one 128-byte K row (32 fp32 / 64
+// bf16 elements); the split mode holds four tiles per stage (A and B, high
+// and low parts).  PAIR = false: one CTA computes 128 x BN.  PAIR = true: a
+// cluster of two CTAs computes 256 x BN with one tcgen05 MMA of M = 256; each
+// CTA stages 128 rows of A and BN/2 rows (or columns) of B, which halves the
+// B traffic per SM and leaves room for deeper pipelines.
+template <int MODE, bool PAIR>
 struct Cfg {
   static constexpr bool SPLIT = MODE == MODE_3XTF32;
   static constexpr int ESZ = MODE == MODE_BF16 ? 2 : 4;
-  static constexpr int BK = 128 / ESZ;         // K elements per stage (one 128 B row)
+  static constexpr int ROWB = 128;               // bytes of one K-major row per stage
+  static constexpr int BK = ROWB / ESZ;          // K elements per stage
   static constexpr int UK = MODE == MODE_BF16 ? 16 : 8;  // K per MMA instruction
   static constexpr int KSTEPS = BK / UK;
-  static constexpr int CHUNK = 128 / ESZ;      // MN elements per 128-byte chunk
+  static constexpr int CHUNK = 128 / ESZ;        // MN elements per 128-byte MN chunk
+  // K-major: 128B swizzle, 8-row core groups of 1024 B.
+  static constexpr uint32_t K_LAYOUT = 2u;
+  static constexpr uint32_t K_SBO = 1024u;
   // MN-major smem layout: 32-bit operands need the 32-byte-atom 128B swizzle
   // (period 4 rows); 16-bit operands use the plain 128B swizzle (8 rows).
   static constexpr uint32_t MN_LAYOUT = ESZ == 4 ? 1u : 2u;
   static constexpr uint32_t MN_SBO = ESZ == 4 ? 512u : 1024u;
-  static constexpr int STAGES = SPLIT ? 2 : 4;
-  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES_MAX) * (SPLIT ? 2 : 1);
+  static constexpr int A_BYTES = 128 * ROWB;
+  static constexpr int B_BYTES_MAX = (PAIR ? 128 : 256) * ROWB;
+  static constexpr int PART_BYTES = A_BYTES + B_BYTES_MAX;
+  static constexpr int STAGE_BYTES = PART_BYTES * (SPLIT ? 2 : 1);
+  static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
   static_assert(STAGES * STAGE_BYTES >= EPI_BYTES, "epilogue staging must fit in the stages");
+  static_assert(STAGES >= 2, "need a double-buffered pipeline");
 };
 
 SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
@@ -63,135 +77,16 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
   }
 }
 
-template <int MODE, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(256, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
-              const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tBl,
-              int K, int BN, EpiParams ep) {
-  count_kernel_run();
-  using C = Cfg<MODE>;
-  const int b = blockIdx.z;
-  if (ep.active != nullptr && ep.active[b] == 0) return;
-  const int m0 = blockIdx.y * 128;
-  const int n0 = blockIdx.x * BN;
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* done = empty + C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Split mode keeps the two small cross products (hi*lo, lo*hi) in a second
-  // accumulator: the tensor cores add into the accumulator with truncation,
-  // so the large hi*hi sum should take as few of those additions as possible.
-  const uint32_t ncols = static_cast<uint32_t>(C::SPLIT ? 2 * BN : BN);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(done, 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&tA);
-    tma_prefetch_desc(&tB);
-  }
-  if (warp == 1) tmem_alloc(tmem_slot, ncols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  const int KB = (K + C::BK - 1) / C::BK;
-  const uint32_t b_bytes = static_cast<uint32_t>(BN) * 128u;
-  const uint32_t tx = (A_BYTES + b_bytes) * (C::SPLIT ? 2u : 1u);
-  bool timed_out = false;
-
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % C::STAGES;
-      if (kb >= C::STAGES && !mbar_wait(&empty[s], ((kb / C::STAGES) - 1) & 1)) {
-        timed_out = true;
-        break;
-      }
-      uint8_t* st = smem + s * C::STAGE_BYTES;
-      const int k0 = kb * C::BK;
-      mbar_arrive_expect_tx(&full[s], tx);
-#pragma unroll 1
-      for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
-        const CUtensorMap* ma = part ? &tAl : &tA;
-        const CUtensorMap* mb = part ? &tBl : &tB;
-        uint8_t* sa = st + part * (A_BYTES + B_BYTES_MAX);
-        uint8_t* sb = sa + A_BYTES;
-        if (A_MN) {
-          for (int i = 0; i < 128 / C::CHUNK; ++i)
-            tma_load_3d(sa + i * C::BK * 128, ma, &full[s], m0 + i * C::CHUNK, k0, b);
-        } else {
-          tma_load_3d(sa, ma, &full[s], k0, m0, b);
-        }
-        if (B_MN) {
-          for (int i = 0; i < BN / C::CHUNK; ++i)
-            tma_load_3d(sb + i * C::BK * 128, mb, &full[s], n0 + i * C::CHUNK, k0, b);
-        } else {
-          tma_load_3d(sb, mb, &full[s], k0, n0, b);
-        }
-      }
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    const uint32_t idesc = instr_desc(MODE == MODE_BF16 ? 1u : 2u, A_MN, B_MN, 128, BN);
-    const uint32_t mn_lbo = C::BK * 128;  // bytes between 128-byte MN chunks
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % C::STAGES;
-      if (!mbar_wait(&full[s], (kb / C::STAGES) & 1)) {
-        timed_out = true;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t base = smem_u32(smem + s * C::STAGE_BYTES);
-#pragma unroll
-      for (int ks = 0; ks < C::KSTEPS; ++ks) {
-        uint64_t ad[2], bd[2];
-#pragma unroll
-        for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
-          const uint32_t sa = base + part * (A_BYTES + B_BYTES_MAX);
-          const uint32_t sb = sa + A_BYTES;
-          ad[part] = A_MN ? smem_desc(sa + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
-                          : smem_desc(sa + ks * C::UK * C::ESZ, 16, 1024, 2);
-          bd[part] = B_MN ? smem_desc(sb + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
-                          : smem_desc(sb + ks * C::UK * C::ESZ, 16, 1024, 2);
-        }
-        const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
-        if (MODE == MODE_BF16) {
-          mma_f16(tmem, ad[0], bd[0], idesc, acc0);
-        } else {
-          mma_tf32(tmem, ad[0], bd[0], idesc, acc0);
-          if (C::SPLIT) {
-            const uint32_t tsmall = tmem + static_cast<uint32_t>(BN);
-            mma_tf32(tsmall, ad[0], bd[C::SPLIT ? 1 : 0], idesc, acc0);
-            mma_tf32(tsmall, ad[C::SPLIT ? 1 : 0], bd[0], idesc, 1u);
-          }
-        }
-      }
-      mma_commit(&empty[s]);
-    }
-    mma_commit(done);
-  }
-
-  // ---------------- epilogue (8 warps).  Warp w reads TMEM lanes 32(w%4)..+31
-  // (the lane quarter its position in the warpgroup grants) and every other
-  // 32-column chunk starting at w/4.  Each chunk is transposed through padded
-  // shared memory (the pipeline stages are free once `done` fired) so that a
-  // lane owns one column of 32 rows: its 32 loads and 32 stores are
-  // independent and every warp access is one coalesced 128-byte row segment.
-  if (!mbar_wait(done, 0)) timed_out = true;
-  __syncwarp();
-  tc_fence_after();
-
+// Epilogue of one CTA's 128 x BN accumulator (8 warps).  Warp w reads TMEM
+// lanes 32(w%4)..+31 (the lane quarter its position in the warpgroup grants)
+// and every other 32-column chunk starting at w/4.  Each chunk is transposed
+// through padded shared memory (the pipeline stages are free once the last
+// MMA completed) so that a lane owns one column of 32 rows: its 32 loads and
+// 32 stores are independent and every warp access is one coalesced 128-byte
+// row segment.  Returns this warp's sum of squares (RESID).
+template <bool SPLIT>
+SHP_DEV float epilogue_tile(uint8_t* smem, uint32_t tmem, const EpiParams& ep, int b, int m0,
+                            int n0, int BN, int warp, int lane) {
   const int q = warp & 3, h = warp >> 2;
   float* st = reinterpret_cast<float*>(smem) + warp * (32 * 33);
   const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;
@@ -205,7 +100,7 @@ __global__ void __launch_bounds__(256, 1)
   for (int c = h; c < BN / 32; c += 2) {
     float v[32];
     tmem_ld32(trow + static_cast<uint32_t>(c * 32), v);
-    if (C::SPLIT) {
+    if (SPLIT) {
       float w[32];
       tmem_ld32(trow + static_cast<uint32_t>(BN + c * 32), w);
 #pragma unroll
@@ -220,7 +115,8 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
     const int gj = n0 + c * 32 + lane;
     if (gj < ep.N && rcount > 0) {
-      const int64_t obase = static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row0) * ep.ldo + gj;
+      const int64_t obase =
+          static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row0) * ep.ldo + gj;
       float x[32];
       if (need_aux) {
         const int64_t abase = static_cast<int64_t>(b) * ep.bs_aux +
@@ -242,8 +138,9 @@ __global__ void __launch_bounds__(256, 1)
       } else if (need_old) {
 #pragma unroll
         for (int r = 0; r < 32; ++r)
-          x[r] = r < rcount ? static_cast<const float*>(ep.out_hi)[obase + static_cast<int64_t>(r) * ep.ldo]
-                            : 0.f;
+          x[r] = r < rcount
+                     ? static_cast<const float*>(ep.out_hi)[obase + static_cast<int64_t>(r) * ep.ldo]
+                     : 0.f;
       } else {
 #pragma unroll
         for (int r = 0; r < 32; ++r) x[r] = 0.f;
@@ -283,6 +180,183 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   }
+  return nrm;
+}
+
+template <int MODE, bool A_MN, bool B_MN, bool PAIR>
+__global__ void __launch_bounds__(256, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
+              const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tBl,
+              int K, int BN, EpiParams ep) {
+  count_kernel_run();
+  using C = Cfg<MODE, PAIR>;
+  const int b = blockIdx.z;
+  if (ep.active != nullptr && ep.active[b] == 0) return;  // uniform over a CTA pair
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int m0 = PAIR ? static_cast<int>(blockIdx.y) * 256 + static_cast<int>(rank) * 128
+                      : static_cast<int>(blockIdx.y) * 128;
+  const int n0 = (PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x)) * BN;
+  const int bn_cta = PAIR ? BN / 2 : BN;        // B rows (or columns) this CTA stages
+  const int nb0 = n0 + static_cast<int>(rank) * bn_cta;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* done = empty + C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Split mode keeps the two small cross products (hi*lo, lo*hi) in a second
+  // accumulator: the tensor cores add into the accumulator with truncation,
+  // so the large hi*hi sum should take as few of those additions as possible.
+  const uint32_t ncols = static_cast<uint32_t>(C::SPLIT ? 2 * BN : BN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tA);
+    tma_prefetch_desc(&tB);
+    if (C::SPLIT) {
+      tma_prefetch_desc(&tAl);
+      tma_prefetch_desc(&tBl);
+    }
+  }
+  if (warp == 1) {
+    if (PAIR)
+      tmem_alloc_pair(tmem_slot, ncols);
+    else
+      tmem_alloc(tmem_slot, ncols);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (PAIR) cluster_sync();  // peer barriers initialised, both TMEM allocations done
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int KB = (K + C::BK - 1) / C::BK;
+  const uint32_t b_bytes = static_cast<uint32_t>(bn_cta) * C::ROWB;
+  const uint32_t tx = (C::A_BYTES + b_bytes) * (C::SPLIT ? 2u : 1u) * (PAIR ? 2u : 1u);
+  bool timed_out = false;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer (both CTAs of a pair load their halves;
+    // completion is counted on the leader's full barrier)
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % C::STAGES;
+      if (kb >= C::STAGES && !mbar_wait(&empty[s], ((kb / C::STAGES) - 1) & 1)) {
+        timed_out = true;
+        break;
+      }
+      uint8_t* st = smem + s * C::STAGE_BYTES;
+      const int k0 = kb * C::BK;
+      if (leader) mbar_arrive_expect_tx(&full[s], tx);
+      const uint32_t fbar = PAIR ? mapa_shared(smem_u32(&full[s]), 0) : smem_u32(&full[s]);
+#pragma unroll 1
+      for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
+        const CUtensorMap* ma = part ? &tAl : &tA;
+        const CUtensorMap* mb = part ? &tBl : &tB;
+        uint8_t* sa = st + part * C::PART_BYTES;
+        uint8_t* sb = sa + C::A_BYTES;
+        if (A_MN) {
+          for (int i = 0; i < 128 / C::CHUNK; ++i) {
+            if (PAIR)
+              tma_load_3d_pair(sa + i * C::BK * 128, ma, fbar, m0 + i * C::CHUNK, k0, b);
+            else
+              tma_load_3d(sa + i * C::BK * 128, ma, &full[s], m0 + i * C::CHUNK, k0, b);
+          }
+        } else {
+          if (PAIR)
+            tma_load_3d_pair(sa, ma, fbar, k0, m0, b);
+          else
+            tma_load_3d(sa, ma, &full[s], k0, m0, b);
+        }
+        if (B_MN) {
+          for (int i = 0; i < bn_cta / C::CHUNK; ++i) {
+            if (PAIR)
+              tma_load_3d_pair(sb + i * C::BK * 128, mb, fbar, nb0 + i * C::CHUNK, k0, b);
+            else
+              tma_load_3d(sb + i * C::BK * 128, mb, &full[s], nb0 + i * C::CHUNK, k0, b);
+          }
+        } else {
+          if (PAIR)
+            tma_load_3d_pair(sb, mb, fbar, k0, nb0, b);
+          else
+            tma_load_3d(sb, mb, &full[s], k0, nb0, b);
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------- MMA issuer (the leader of a pair issues for both SMs)
+    const uint32_t idesc =
+        instr_desc(MODE == MODE_BF16 ? 1u : 2u, A_MN, B_MN, PAIR ? 256 : 128, BN);
+    const uint32_t mn_lbo = C::BK * 128;  // bytes between 128-byte MN chunks
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % C::STAGES;
+      if (!mbar_wait(&full[s], (kb / C::STAGES) & 1)) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = smem_u32(smem + s * C::STAGE_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        uint64_t ad[2], bd[2];
+#pragma unroll
+        for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
+          const uint32_t sa = base + part * C::PART_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
+          ad[part] = A_MN ? smem_desc(sa + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
+                          : smem_desc(sa + ks * C::UK * C::ESZ, 16, C::K_SBO, C::K_LAYOUT);
+          bd[part] = B_MN ? smem_desc(sb + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
+                          : smem_desc(sb + ks * C::UK * C::ESZ, 16, C::K_SBO, C::K_LAYOUT);
+        }
+        const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
+        if (MODE == MODE_BF16) {
+          if (PAIR)
+            mma_f16_pair(tmem, ad[0], bd[0], idesc, acc0);
+          else
+            mma_f16(tmem, ad[0], bd[0], idesc, acc0);
+        } else if (C::SPLIT) {
+          const uint32_t tsmall = tmem + static_cast<uint32_t>(BN);
+          if (PAIR) {
+            mma_tf32_pair(tmem, ad[0], bd[0], idesc, acc0);
+            mma_tf32_pair(tsmall, ad[0], bd[1], idesc, acc0);
+            mma_tf32_pair(tsmall, ad[1], bd[0], idesc, 1u);
+          } else {
+            mma_tf32(tmem, ad[0], bd[0], idesc, acc0);
+            mma_tf32(tsmall, ad[0], bd[1], idesc, acc0);
+            mma_tf32(tsmall, ad[1], bd[0], idesc, 1u);
+          }
+        } else {
+          if (PAIR)
+            mma_tf32_pair(tmem, ad[0], bd[0], idesc, acc0);
+          else
+            mma_tf32(tmem, ad[0], bd[0], idesc, acc0);
+        }
+      }
+      if (PAIR)
+        mma_commit_pair(&empty[s], 3);
+      else
+        mma_commit(&empty[s]);
+    }
+    if (PAIR)
+      mma_commit_pair(done, 3);
+    else
+      mma_commit(done);
+  }
+
+  // ---------------- epilogue (all 8 warps of each CTA, on its own TMEM rows)
+  if (!mbar_wait(done, 0)) timed_out = true;
+  __syncwarp();
+  tc_fence_after();
+  float nrm = epilogue_tile<C::SPLIT>(smem, tmem, ep, b, m0, n0, BN, warp, lane);
   if (ep.kind == EPI_RESID) {
     nrm = warp_sum(nrm);
     if (lane == 0) atomicAdd(&ep.norm2[static_cast<int64_t>(b) * ep.norm2_stride], nrm);
@@ -291,7 +365,13 @@ __global__ void __launch_bounds__(256, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, ncols);
+  if (PAIR) cluster_sync();
+  if (warp == 1) {
+    if (PAIR)
+      tmem_dealloc_pair(tmem, ncols);
+    else
+      tmem_dealloc(tmem, ncols);
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -329,27 +409,50 @@ bool make_map(CUtensorMap* m, const void* ptr, int esz, int64_t inner, int64_t r
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE, bool AMN, bool BMN>
+template <int MODE, bool AMN, bool BMN, bool PAIR>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMap& b,
                    const CUtensorMap& bl, int M, int N, int K, int BN, int batch,
                    const EpiParams& ep, cudaStream_t st) {
-  using C = Cfg<MODE>;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<MODE, AMN, BMN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  using C = Cfg<MODE, PAIR>;
+  auto kern = k_gemm_tc<MODE, AMN, BMN, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((N + BN - 1) / BN, (M + 127) / 128, batch);
-  k_gemm_tc<MODE, AMN, BMN><<<grid, 256, C::SMEM, st>>>(a, al, b, bl, K, BN, ep);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = PAIR ? dim3(2 * ((N + BN - 1) / BN), (M + 255) / 256, batch)
+                     : dim3((N + BN - 1) / BN, (M + 127) / 128, batch);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, al, b, bl, K, BN, ep);
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 cudaError_t dispatch(bool amn, bool bmn, const CUtensorMap& a, const CUtensorMap& al,
                      const CUtensorMap& b, const CUtensorMap& bl, int M, int N, int K, int BN,
                      int batch, const EpiParams& ep, cudaStream_t st) {
-  if (!amn && !bmn) return launch<MODE, false, false>(a, al, b, bl, M, N, K, BN, batch, ep, st);
-  if (!amn && bmn) return launch<MODE, false, true>(a, al, b, bl, M, N, K, BN, batch, ep, st);
-  if (amn && !bmn) return launch<MODE, true, false>(a, al, b, bl, M, N, K, BN, batch, ep, st);
-  return launch<MODE, true, true>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  if (!amn && !bmn)
+    return launch<MODE, false, false, PAIR>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  if (!amn && bmn)
+    return launch<MODE, false, true, PAIR>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  if (amn && !bmn)
+    return launch<MODE, true, false, PAIR>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+  return launch<MODE, true, true, PAIR>(a, al, b, bl, M, N, K, BN, batch, ep, st);
+}
+
+template <int MODE>
+cudaError_t dispatch_pair(bool pair, bool amn, bool bmn, const CUtensorMap& a,
+                          const CUtensorMap& al, const CUtensorMap& b, const CUtensorMap& bl,
+                          int M, int N, int K, int BN, int batch, const EpiParams& ep,
+                          cudaStream_t st) {
+  return pair ? dispatch<MODE, true>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st)
+              : dispatch<MODE, false>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st);
 }
 
 }  // namespace
@@ -358,8 +461,14 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
                     int batch, const EpiParams& ep, cudaStream_t st) {
   if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return cudaSuccess;
   const int esz = mode == MODE_BF16 ? 2 : 4;
-  const int bk = 128 / esz, chunk = 128 / esz;
+  const int rowb = 128;  // Cfg<MODE>::ROWB
+  const int bk = rowb / esz, chunk = 128 / esz;
+  const CUtensorMapSwizzle k_swz = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const int BN = N > 128 ? 256 : (N > 64 ? 128 : 64);
+  // CTA pairs (M = 256 per MMA) for full-width tiles; small problems keep one
+  // CTA per 128-row tile.
+  const bool pair = M >= 256 && BN == 256 && getenv("SHP_NO_PAIR") == nullptr;
+  const int bn_cta = pair ? BN / 2 : BN;
   CUtensorMap ma, mal, mb, mbl;
   bool ok = true;
   // A: logical M x K.
@@ -368,14 +477,12 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
       esz == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
   auto mapA = [&](CUtensorMap* m, const void* p) {
     return A.mn ? make_map(m, p, esz, M, K, batch, A.ld, A.bstride, chunk, bk, mn_swz)
-                : make_map(m, p, esz, K, M, batch, A.ld, A.bstride, bk, 128,
-                           CU_TENSOR_MAP_SWIZZLE_128B);
+                : make_map(m, p, esz, K, M, batch, A.ld, A.bstride, bk, 128, k_swz);
   };
   // B: logical K x N.
   auto mapB = [&](CUtensorMap* m, const void* p) {
     return B.mn ? make_map(m, p, esz, N, K, batch, B.ld, B.bstride, chunk, bk, mn_swz)
-                : make_map(m, p, esz, K, N, batch, B.ld, B.bstride, bk, BN,
-                           CU_TENSOR_MAP_SWIZZLE_128B);
+                : make_map(m, p, esz, K, N, batch, B.ld, B.bstride, bk, bn_cta, k_swz);
   };
   ok = ok && mapA(&ma, A.hi) && mapB(&mb, B.hi);
   if (mode == MODE_3XTF32) {
@@ -388,11 +495,14 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
   if (!ok) return cudaErrorInvalidValue;
   switch (mode) {
     case MODE_TF32:
-      return dispatch<MODE_TF32>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
+      return dispatch_pair<MODE_TF32>(pair, A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch,
+                                      ep, st);
     case MODE_3XTF32:
-      return dispatch<MODE_3XTF32>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
+      return dispatch_pair<MODE_3XTF32>(pair, A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch,
+                                        ep, st);
     case MODE_BF16:
-      return dispatch<MODE_BF16>(A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch, ep, st);
+      return dispatch_pair<MODE_BF16>(pair, A.mn, B.mn, ma, mal, mb, mbl, M, N, K, BN, batch,
+                                      ep, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -26,9 +26,12 @@ namespace shp {
 namespace {
 
 constexpr int SK_THREADS = 256;
-constexpr int SK_CHUNK = 256;  // columns of V staged in shared memory per step
 
-// Vout = R * Vin for one block; 8 warps x ROWS rows per CTA.
+// Vout = R * Vin for one block.  Each warp owns ROWS consecutive rows of R
+// and streams them with 128-bit loads (a lane takes 4 consecutive columns);
+// V is staged in shared memory transposed, Vs[j][c], one 32 KB chunk of
+// columns at a time, so that lane reads are conflict-free float4 as well.
+// Requires n % 4 == 0 (16-byte rows).
 template <int P>
 __global__ void __launch_bounds__(SK_THREADS)
     k_sketch(const float* __restrict__ Rhi, const float* __restrict__ Rlo, int64_t n,
@@ -37,7 +40,8 @@ __global__ void __launch_bounds__(SK_THREADS)
              int64_t it_stride) {
   count_kernel_run();
   constexpr int ROWS = P <= 16 ? 4 : 2;
-  __shared__ float Vs[P][SK_CHUNK];
+  constexpr int CK = 8192 / P;  // columns per chunk: Vs is 32 KB
+  __shared__ __align__(16) float Vs[P][CK];
   const int b = blockIdx.y;
   if (active != nullptr && active[b] == 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -51,33 +55,41 @@ __global__ void __launch_bounds__(SK_THREADS)
 #pragma unroll
     for (int j = 0; j < P; ++j) acc[r][j] = 0.f;
 
-  for (int64_t c0 = 0; c0 < n; c0 += SK_CHUNK) {
+  for (int64_t c0 = 0; c0 < n; c0 += CK) {
     __syncthreads();
-    for (int idx = threadIdx.x; idx < SK_CHUNK * P; idx += SK_THREADS) {
+    for (int idx = threadIdx.x; idx < CK * P; idx += SK_THREADS) {
       const int cc = idx / P, j = idx % P;
       const int64_t col = c0 + cc;
       Vs[j][cc] = (j < p && col < n) ? V[col * p + j] : 0.f;
     }
     __syncthreads();
-    for (int cc = lane; cc < SK_CHUNK; cc += 32) {
+    for (int cc = lane * 4; cc < CK; cc += 128) {
       const int64_t col = c0 + cc;
       if (col >= n) break;
-      float rv[ROWS];
+      float4 rv[ROWS];
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {
         const int64_t row = row0 + r;
-        float x = 0.f;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (row < n) {
-          x = R[row * n + col];
-          if (RL != nullptr) x += RL[row * n + col];
+          x = *reinterpret_cast<const float4*>(R + row * n + col);
+          if (RL != nullptr) {
+            const float4 y = *reinterpret_cast<const float4*>(RL + row * n + col);
+            x.x += y.x;
+            x.y += y.y;
+            x.z += y.z;
+            x.w += y.w;
+          }
         }
         rv[r] = x;
       }
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const float vj = Vs[j][cc];
+        const float4 vj = *reinterpret_cast<const float4*>(&Vs[j][cc]);
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) acc[r][j] = fmaf(rv[r], vj, acc[r][j]);
+        for (int r = 0; r < ROWS; ++r)
+          acc[r][j] = fmaf(rv[r].x, vj.x,
+                           fmaf(rv[r].y, vj.y, fmaf(rv[r].z, vj.z, fmaf(rv[r].w, vj.w, acc[r][j]))));
       }
     }
   }
@@ -85,9 +97,9 @@ __global__ void __launch_bounds__(SK_THREADS)
   for (int r = 0; r < ROWS; ++r) {
 #pragma unroll
     for (int j = 0; j < P; ++j) {
-      const float s = warp_sum(acc[r][j]);
+      const float sum = warp_sum(acc[r][j]);
       const int64_t row = row0 + r;
-      if (lane == 0 && row < n && j < p) Vout[b * obs + row * p + j] = s;
+      if (lane == 0 && row < n && j < p) Vout[b * obs + row * p + j] = sum;
     }
   }
 }
