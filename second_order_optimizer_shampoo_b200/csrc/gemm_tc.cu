@@ -60,6 +60,7 @@ struct Cfg {
   static constexpr int PART_BYTES = A_BYTES + B_BYTES_MAX;
   static constexpr int STAGE_BYTES = PART_BYTES * (SPLIT ? 2 : 1);
   static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
+  static constexpr int PP_STAGES = STAGES;
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
   static_assert(STAGES * STAGE_BYTES >= EPI_BYTES, "epilogue staging must fit in the stages");
   static_assert(STAGES >= 2, "need a double-buffered pipeline");
@@ -77,18 +78,17 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
   }
 }
 
-// Epilogue of one CTA's 128 x BN accumulator (8 warps).  Warp w reads TMEM
-// lanes 32(w%4)..+31 (the lane quarter its position in the warpgroup grants)
-// and every other 32-column chunk starting at w/4.  Each chunk is transposed
-// through padded shared memory (the pipeline stages are free once the last
-// MMA completed) so that a lane owns one column of 32 rows: its 32 loads and
-// 32 stores are independent and every warp access is one coalesced 128-byte
-// row segment.  Returns this warp's sum of squares (RESID).
-template <bool SPLIT>
-SHP_DEV float epilogue_tile(uint8_t* smem, uint32_t tmem, const EpiParams& ep, int b, int m0,
-                            int n0, int BN, int warp, int lane) {
-  const int q = warp & 3, h = warp >> 2;
-  float* st = reinterpret_cast<float*>(smem) + warp * (32 * 33);
+// Epilogue of one CTA's 128 x BN accumulator, by 8 warps.  Warp (q, h) reads
+// TMEM lanes 32q..32q+31 (q must be the warp's position in its warpgroup, the
+// lane quarter the hardware grants it) and every other 32-column chunk
+// starting at h.  Each chunk is transposed through padded shared memory `st`
+// (32 x 33 floats per warp) so that a lane owns one column: its RP loads and
+// RP stores per pass are independent and every warp access is one coalesced
+// 128-byte row segment.  DUAL adds the second (cross-term) accumulator that
+// sits BN columns further.  Returns this warp's sum of squares (RESID).
+template <bool DUAL, int RP>
+SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b, int m0, int n0,
+                            int BN, int q, int h, int lane) {
   const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;
   const bool diag_tile = (m0 < n0 + BN) && (n0 < m0 + 128);
   const int row0 = m0 + q * 32;
@@ -98,87 +98,92 @@ SHP_DEV float epilogue_tile(uint8_t* smem, uint32_t tmem, const EpiParams& ep, i
   const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
   float nrm = 0.f;
   for (int c = h; c < BN / 32; c += 2) {
-    float v[32];
-    tmem_ld32(trow + static_cast<uint32_t>(c * 32), v);
-    if (SPLIT) {
-      float w[32];
-      tmem_ld32(trow + static_cast<uint32_t>(BN + c * 32), w);
+    {
+      float v[32];
+      tmem_ld32(trow + static_cast<uint32_t>(c * 32), v);
+      if (DUAL) {
+        float w[32];
+        tmem_ld32(trow + static_cast<uint32_t>(BN + c * 32), w);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] += w[j];
+        for (int j = 0; j < 32; ++j) v[j] += w[j];
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) st[lane * 33 + j] = v[j];
     }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) st[lane * 33 + j] = v[j];
-    __syncwarp();
-    float a[32];
-#pragma unroll
-    for (int r = 0; r < 32; ++r) a[r] = st[r * 33 + lane];
     __syncwarp();
     const int gj = n0 + c * 32 + lane;
-    if (gj < ep.N && rcount > 0) {
-      const int64_t obase =
-          static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row0) * ep.ldo + gj;
-      float x[32];
-      if (need_aux) {
-        const int64_t abase = static_cast<int64_t>(b) * ep.bs_aux +
-                              static_cast<int64_t>(row0) * ep.lda_aux + gj;
+    const bool colok = gj < ep.N && rcount > 0;
+    const int64_t obase =
+        static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row0) * ep.ldo + gj;
+    const int64_t abase =
+        static_cast<int64_t>(b) * ep.bs_aux + static_cast<int64_t>(row0) * ep.lda_aux + gj;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 32; r0 += RP) {
+      float a[RP], x[RP];
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-          float av = 0.f;
-          if (r < rcount) {
-            const int64_t oa = abase + static_cast<int64_t>(r) * ep.lda_aux;
-            if (ep.aux_fmt == OUT_BF16) {
-              av = __bfloat162float(static_cast<const __nv_bfloat16*>(ep.aux_hi)[oa]);
-            } else {
-              av = static_cast<const float*>(ep.aux_hi)[oa];
-              if (ep.aux_fmt == OUT_SPLIT) av += ep.aux_lo[oa];
+      for (int r = 0; r < RP; ++r) a[r] = st[(r0 + r) * 33 + lane];
+      if (colok) {
+        if (need_aux) {
+#pragma unroll
+          for (int r = 0; r < RP; ++r) {
+            float av = 0.f;
+            if (r0 + r < rcount) {
+              const int64_t oa = abase + static_cast<int64_t>(r0 + r) * ep.lda_aux;
+              if (ep.aux_fmt == OUT_BF16) {
+                av = __bfloat162float(static_cast<const __nv_bfloat16*>(ep.aux_hi)[oa]);
+              } else {
+                av = static_cast<const float*>(ep.aux_hi)[oa];
+                if (ep.aux_fmt == OUT_SPLIT) av += ep.aux_lo[oa];
+              }
             }
+            x[r] = av;
           }
-          x[r] = av;
+        } else if (need_old) {
+#pragma unroll
+          for (int r = 0; r < RP; ++r)
+            x[r] = r0 + r < rcount
+                       ? static_cast<const float*>(ep.out_hi)[obase + static_cast<int64_t>(r0 + r) * ep.ldo]
+                       : 0.f;
+        } else {
+#pragma unroll
+          for (int r = 0; r < RP; ++r) x[r] = 0.f;
         }
-      } else if (need_old) {
 #pragma unroll
-        for (int r = 0; r < 32; ++r)
-          x[r] = r < rcount
-                     ? static_cast<const float*>(ep.out_hi)[obase + static_cast<int64_t>(r) * ep.ldo]
-                     : 0.f;
-      } else {
-#pragma unroll
-        for (int r = 0; r < 32; ++r) x[r] = 0.f;
-      }
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        if (r >= rcount) break;
-        const int gi = row0 + r;
-        const float acc = a[r];
-        const float eye = (diag_tile && gi == gj) ? 1.f : 0.f;
-        const int64_t off = obase + static_cast<int64_t>(r) * ep.ldo;
-        float val;
-        switch (ep.kind) {
-          case EPI_RESID:
-            val = eye - acc;
-            nrm += val * val;
-            break;
-          case EPI_GPOLY:
-            val = ep.s1 * x[r] + alpha * acc;
-            break;
-          case EPI_AXPY:
-            val = x[r] + ep.s0 * acc;
-            break;
-          case EPI_EMA:
-            val = ep.s0 * x[r] + ep.s1 * acc + ep.s2 * eye;
-            break;
-          case EPI_APPLY:
-            val = x[r] + ep.s0 * acc;
-            break;
-          default:
-            val = ep.s0 * acc;
-            break;
+        for (int r = 0; r < RP; ++r) {
+          if (r0 + r >= rcount) break;
+          const int gi = row0 + r0 + r;
+          const float acc = a[r];
+          const float eye = (diag_tile && gi == gj) ? 1.f : 0.f;
+          const int64_t off = obase + static_cast<int64_t>(r0 + r) * ep.ldo;
+          float val;
+          switch (ep.kind) {
+            case EPI_RESID:
+              val = eye - acc;
+              nrm += val * val;
+              break;
+            case EPI_GPOLY:
+              val = ep.s1 * x[r] + alpha * acc;
+              break;
+            case EPI_AXPY:
+              val = x[r] + ep.s0 * acc;
+              break;
+            case EPI_EMA:
+              val = ep.s0 * x[r] + ep.s1 * acc + ep.s2 * eye;
+              break;
+            case EPI_APPLY:
+              val = x[r] + ep.s0 * acc;
+              break;
+            default:
+              val = ep.s0 * acc;
+              break;
+          }
+          put(ep.out_fmt, ep.out_hi, ep.out_lo, off, val);
+          if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, val + eye);
+          if (ep.out_plain != nullptr) ep.out_plain[off] = val;
         }
-        put(ep.out_fmt, ep.out_hi, ep.out_lo, off, val);
-        if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, val + eye);
-        if (ep.out_plain != nullptr) ep.out_plain[off] = val;
       }
     }
+    __syncwarp();
   }
   return nrm;
 }
@@ -356,7 +361,8 @@ __global__ void __launch_bounds__(256, 1)
   if (!mbar_wait(done, 0)) timed_out = true;
   __syncwarp();
   tc_fence_after();
-  float nrm = epilogue_tile<C::SPLIT>(smem, tmem, ep, b, m0, n0, BN, warp, lane);
+  float nrm = epilogue_tile<C::SPLIT, 32>(reinterpret_cast<float*>(smem) + warp * (32 * 33), tmem,
+                                          ep, b, m0, n0, BN, warp & 3, warp >> 2, lane);
   if (ep.kind == EPI_RESID) {
     nrm = warp_sum(nrm);
     if (lane == 0) atomicAdd(&ep.norm2[static_cast<int64_t>(b) * ep.norm2_stride], nrm);
@@ -372,6 +378,213 @@ __global__ void __launch_bounds__(256, 1)
     else
       tmem_dealloc(tmem, ncols);
   }
+}
+
+// Persistent CTA-pair GEMM (BN = 256, M >= 256): one cluster of two CTAs per
+// SM pair loops over the output tiles (tile t, t + #clusters, ...).  Warp 0
+// streams operands, warp 1 of the leader issues the MMAs, warps 2..9 run the
+// epilogue.  TMEM holds two 256-column accumulators: while the epilogue
+// drains tile i from one, the MMAs of tile i+1 fill the other, so the
+// epilogue's memory traffic hides behind the next main loop.
+//   full[s]/empty[s]: operand ring (leader's full counts both CTAs' bytes;
+//                     empty is signalled to both CTAs by the leader's commit)
+//   accf[u]:          accumulator u complete (leader's commit, both CTAs)
+//   acce[u]:          accumulator u drained (8 epilogue warps x 2 CTAs arrive
+//                     on the leader's barrier)
+template <int MODE, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(320, 1)
+    k_gemm_pp(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
+              const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tBl,
+              int K, EpiParams ep, int batch) {
+  count_kernel_run();
+  using C = Cfg<MODE, true>;
+  constexpr int BN = 256;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int ncl = static_cast<int>(gridDim.x) / 2, cl = static_cast<int>(blockIdx.x) / 2;
+  const int tiles_n = (ep.N + BN - 1) / BN, tiles_m = (ep.M + 255) / 256;
+  const int per_b = tiles_n * tiles_m, ntiles = per_b * batch;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* stage_epi = reinterpret_cast<float*>(smem + C::PP_STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_epi + 8 * 32 * 33);
+  uint64_t* empty = full + C::PP_STAGES;
+  uint64_t* accf = empty + C::PP_STAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;  // all MMAs of this pair complete (before TMEM is freed)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::PP_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&accf[u], 1);
+      mbar_init(&acce[u], 16);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tA);
+    tma_prefetch_desc(&tB);
+    if (C::SPLIT) {
+      tma_prefetch_desc(&tAl);
+      tma_prefetch_desc(&tBl);
+    }
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, 2 * BN);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // peer barriers initialised, both TMEM allocations done
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int KB = (K + C::BK - 1) / C::BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      const uint32_t tx = (C::A_BYTES + 128u * C::ROWB) * (C::SPLIT ? 2u : 1u) * 2u;
+      int kit = 0;
+      bool stop = false;
+      for (int t = cl; t < ntiles && !stop; t += ncl) {
+        const int b = t / per_b, r = t % per_b;
+        if (ep.active != nullptr && ep.active[b] == 0) continue;
+        const int m0 = (r / tiles_n) * 256 + static_cast<int>(rank) * 128;
+        const int nb0 = (r % tiles_n) * BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < KB; ++kb, ++kit) {
+          const int s = kit % C::PP_STAGES;
+          if (kit >= C::PP_STAGES &&
+              (*abort_flag || !mbar_wait(&empty[s], ((kit / C::PP_STAGES) - 1) & 1))) {
+            *abort_flag = 1;
+            if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
+            stop = true;
+            break;
+          }
+          uint8_t* st = smem + s * C::STAGE_BYTES;
+          const int k0 = kb * C::BK;
+          if (leader) mbar_arrive_expect_tx(&full[s], tx);
+          const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+#pragma unroll 1
+          for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
+            const CUtensorMap* ma = part ? &tAl : &tA;
+            const CUtensorMap* mb = part ? &tBl : &tB;
+            uint8_t* sa = st + part * C::PART_BYTES;
+            uint8_t* sb = sa + C::A_BYTES;
+            if (A_MN) {
+              for (int i = 0; i < 128 / C::CHUNK; ++i)
+                tma_load_3d_pair(sa + i * C::BK * 128, ma, fbar, m0 + i * C::CHUNK, k0, b);
+            } else {
+              tma_load_3d_pair(sa, ma, fbar, k0, m0, b);
+            }
+            if (B_MN) {
+              for (int i = 0; i < 128 / C::CHUNK; ++i)
+                tma_load_3d_pair(sb + i * C::BK * 128, mb, fbar, nb0 + i * C::CHUNK, k0, b);
+            } else {
+              tma_load_3d_pair(sb, mb, fbar, k0, nb0, b);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader of the pair)
+      const uint32_t idesc = instr_desc(MODE == MODE_BF16 ? 1u : 2u, A_MN, B_MN, 256, BN);
+      const uint32_t mn_lbo = C::BK * 128;
+      int kit = 0, tl = 0;
+      bool stop = false;
+      for (int t = cl; t < ntiles && !stop; t += ncl) {
+        const int b = t / per_b;
+        if (ep.active != nullptr && ep.active[b] == 0) continue;
+        const int u = tl & 1, use = tl >> 1;
+        if (use >= 1 && (*abort_flag || !mbar_wait(&acce[u], (use - 1) & 1))) {
+          *abort_flag = 1;
+          if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dacc = tmem + static_cast<uint32_t>(u * BN);
+        for (int kb = 0; kb < KB; ++kb, ++kit) {
+          const int s = kit % C::PP_STAGES;
+          if (*abort_flag || !mbar_wait(&full[s], (kit / C::PP_STAGES) & 1)) {
+            *abort_flag = 1;
+            if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * C::STAGE_BYTES);
+#pragma unroll
+          for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            uint64_t ad[2], bd[2];
+#pragma unroll
+            for (int part = 0; part < (C::SPLIT ? 2 : 1); ++part) {
+              const uint32_t sa = base + part * C::PART_BYTES;
+              const uint32_t sb = sa + C::A_BYTES;
+              ad[part] = A_MN ? smem_desc(sa + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
+                              : smem_desc(sa + ks * C::UK * C::ESZ, 16, C::K_SBO, C::K_LAYOUT);
+              bd[part] = B_MN ? smem_desc(sb + ks * C::UK * 128, mn_lbo, C::MN_SBO, C::MN_LAYOUT)
+                              : smem_desc(sb + ks * C::UK * C::ESZ, 16, C::K_SBO, C::K_LAYOUT);
+            }
+            const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
+            if (MODE == MODE_BF16) {
+              mma_f16_pair(dacc, ad[0], bd[0], idesc, acc0);
+            } else {
+              mma_tf32_pair(dacc, ad[0], bd[0], idesc, acc0);
+              if (C::SPLIT) {
+                mma_tf32_pair(dacc, ad[0], bd[1], idesc, 1u);
+                mma_tf32_pair(dacc, ad[1], bd[0], idesc, 1u);
+              }
+            }
+          }
+          mma_commit_pair(&empty[s], 3);
+        }
+        mma_commit_pair(&accf[u], 3);
+        ++tl;
+      }
+    }
+    if (lane == 0 && leader) mma_commit_pair(drain, 3);  // after every MMA issued above
+  } else {
+    // ---------------- epilogue warps 2..9 (both CTAs, each on its TMEM rows)
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    float* st = stage_epi + (warp - 2) * (32 * 33);
+    int tl = 0;
+    for (int t = cl; t < ntiles; t += ncl) {
+      const int b = t / per_b, r = t % per_b;
+      if (ep.active != nullptr && ep.active[b] == 0) continue;
+      const int u = tl & 1, use = tl >> 1;
+      if (*abort_flag || !mbar_wait(&accf[u], use & 1)) {
+        *abort_flag = 1;
+        if (lane == 0 && ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      const int m0 = (r / tiles_n) * 256 + static_cast<int>(rank) * 128;
+      const int n0 = (r % tiles_n) * BN;
+      float nrm = epilogue_tile<false, 16>(st, tmem + static_cast<uint32_t>(u * BN), ep, b, m0,
+                                          n0, BN, q, h, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acce[u]), 0));
+      if (ep.kind == EPI_RESID) {
+        nrm = warp_sum(nrm);
+        if (lane == 0) atomicAdd(&ep.norm2[static_cast<int64_t>(b) * ep.norm2_stride], nrm);
+      }
+      ++tl;
+    }
+  }
+
+  if (warp == 1) mbar_wait(drain, 0);  // bounded; immediate unless a wait above gave up
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) tmem_dealloc_pair(tmem, 2 * BN);
 }
 
 // ------------------------------------------------------------------ host side
@@ -433,6 +646,49 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMa
   return cudaLaunchKernelEx(&cfg, kern, a, al, b, bl, K, BN, ep);
 }
 
+template <int MODE, bool AMN, bool BMN>
+cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMap& b,
+                      const CUtensorMap& bl, int M, int N, int K, int batch, const EpiParams& ep,
+                      cudaStream_t st) {
+  using C = Cfg<MODE, true>;
+  constexpr int SMEM = 1024 + C::PP_STAGES * C::STAGE_BYTES + 8 * 32 * 33 * 4 + 320;
+  static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
+  static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
+  auto kern = k_gemm_pp<MODE, AMN, BMN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = ((N + 255) / 256) * ((M + 255) / 256) * batch;
+  int ncl = sms / 2;
+  if (ncl > ntiles) ncl = ntiles;
+  if (ncl < 1) ncl = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ncl, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, al, b, bl, K, ep, batch);
+}
+
+template <int MODE>
+cudaError_t dispatch_pp(bool amn, bool bmn, const CUtensorMap& a, const CUtensorMap& al,
+                        const CUtensorMap& b, const CUtensorMap& bl, int M, int N, int K,
+                        int batch, const EpiParams& ep, cudaStream_t st) {
+  if (!amn && !bmn) return launch_pp<MODE, false, false>(a, al, b, bl, M, N, K, batch, ep, st);
+  if (!amn && bmn) return launch_pp<MODE, false, true>(a, al, b, bl, M, N, K, batch, ep, st);
+  if (amn && !bmn) return launch_pp<MODE, true, false>(a, al, b, bl, M, N, K, batch, ep, st);
+  return launch_pp<MODE, true, true>(a, al, b, bl, M, N, K, batch, ep, st);
+}
+
 template <int MODE, bool PAIR>
 cudaError_t dispatch(bool amn, bool bmn, const CUtensorMap& a, const CUtensorMap& al,
                      const CUtensorMap& b, const CUtensorMap& bl, int M, int N, int K, int BN,
@@ -451,6 +707,8 @@ cudaError_t dispatch_pair(bool pair, bool amn, bool bmn, const CUtensorMap& a,
                           const CUtensorMap& al, const CUtensorMap& b, const CUtensorMap& bl,
                           int M, int N, int K, int BN, int batch, const EpiParams& ep,
                           cudaStream_t st) {
+  if (pair && getenv("SHP_NO_PERSIST") == nullptr)
+    return dispatch_pp<MODE>(amn, bmn, a, al, b, bl, M, N, K, batch, ep, st);
   return pair ? dispatch<MODE, true>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st)
               : dispatch<MODE, false>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st);
 }

@@ -187,6 +187,11 @@ SHP_DEV void mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint3
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// Arrive on an mbarrier given by its shared::cluster address (may be the peer's).
+SHP_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
 // Arrive once on the mbarrier at this offset in every CTA of `mask` when the
 // pair's MMAs issued so far complete.
 SHP_DEV void mma_commit_pair(uint64_t* bar, uint16_t mask) {
