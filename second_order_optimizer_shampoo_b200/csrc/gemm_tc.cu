@@ -123,27 +123,44 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
 #pragma unroll
       for (int r = 0; r < RP; ++r) a[r] = st[(r0 + r) * 33 + lane];
       if (colok) {
+        // All RP (or 2 RP) loads of a pass are issued before any is used:
+        // rows past the edge re-read the last valid row (their results are
+        // never stored), so no load sits behind a branch that would make the
+        // warp wait for it before issuing the next.
         if (need_aux) {
+          if (ep.aux_fmt == OUT_BF16) {
+            const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(ep.aux_hi) + abase;
 #pragma unroll
-          for (int r = 0; r < RP; ++r) {
-            float av = 0.f;
-            if (r0 + r < rcount) {
-              const int64_t oa = abase + static_cast<int64_t>(r0 + r) * ep.lda_aux;
-              if (ep.aux_fmt == OUT_BF16) {
-                av = __bfloat162float(static_cast<const __nv_bfloat16*>(ep.aux_hi)[oa]);
-              } else {
-                av = static_cast<const float*>(ep.aux_hi)[oa];
-                if (ep.aux_fmt == OUT_SPLIT) av += ep.aux_lo[oa];
-              }
+            for (int r = 0; r < RP; ++r) {
+              const int rr = r0 + r < rcount ? r0 + r : rcount - 1;
+              x[r] = __bfloat162float(p[static_cast<int64_t>(rr) * ep.lda_aux]);
             }
-            x[r] = av;
+          } else {
+            const float* p = static_cast<const float*>(ep.aux_hi) + abase;
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+              const int rr = r0 + r < rcount ? r0 + r : rcount - 1;
+              x[r] = p[static_cast<int64_t>(rr) * ep.lda_aux];
+            }
+            if (ep.aux_fmt == OUT_SPLIT) {
+              const float* pl = ep.aux_lo + abase;
+              float y[RP];
+#pragma unroll
+              for (int r = 0; r < RP; ++r) {
+                const int rr = r0 + r < rcount ? r0 + r : rcount - 1;
+                y[r] = pl[static_cast<int64_t>(rr) * ep.lda_aux];
+              }
+#pragma unroll
+              for (int r = 0; r < RP; ++r) x[r] += y[r];
+            }
           }
         } else if (need_old) {
+          const float* p = static_cast<const float*>(ep.out_hi) + obase;
 #pragma unroll
-          for (int r = 0; r < RP; ++r)
-            x[r] = r0 + r < rcount
-                       ? static_cast<const float*>(ep.out_hi)[obase + static_cast<int64_t>(r0 + r) * ep.ldo]
-                       : 0.f;
+          for (int r = 0; r < RP; ++r) {
+            const int rr = r0 + r < rcount ? r0 + r : rcount - 1;
+            x[r] = p[static_cast<int64_t>(rr) * ep.ldo];
+          }
         } else {
 #pragma unroll
           for (int r = 0; r < RP; ++r) x[r] = 0.f;
@@ -652,7 +669,6 @@ cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtenso
                       cudaStream_t st) {
   using C = Cfg<MODE, true>;
   constexpr int SMEM = 1024 + C::PP_STAGES * C::STAGE_BYTES + 8 * 32 * 33 * 4 + 320;
-  static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
   static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
   auto kern = k_gemm_pp<MODE, AMN, BMN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
