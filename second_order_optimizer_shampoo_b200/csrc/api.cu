@@ -364,7 +364,8 @@ const char* shp_version(void) { return "0.1.0"; }
 
 uint64_t shp_kernel_launches(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return 0;
-  return kernel_runs_gemm() + kernel_runs_sketch() + kernel_runs_elementwise();
+  return kernel_runs_gemm() + kernel_runs_sketch() + kernel_runs_elementwise() +
+         kernel_runs_small();
 }
 
 int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream) {
@@ -418,10 +419,12 @@ size_t shp_workspace_bytes(int opk, int64_t m, int64_t n, int64_t batch,
   switch (opk) {
     case SHP_OP_INV_ROOT:
       if (!opts_ok(o)) return 0;
+      if (small_block_ok(n, n, o->p)) return kAlign;  // on-chip path: no scratch
       carve_inv_root(a, n, batch, o);
       break;
     case SHP_OP_POLAR:
       if (!opts_ok(o) || m <= 0) return 0;
+      if (o->prec != SHP_BF16 && small_block_ok(m, n, o->p)) return kAlign;
       carve_polar(a, m, n, batch, o->prec, o);
       break;
     case SHP_OP_ALPHA_FIT: {
@@ -580,9 +583,17 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
   if (!o->fixed_alpha && (S == nullptr || S_count < static_cast<int64_t>(npass) * o->max_iter))
     return SHP_EINVAL;
   if (!aligned16(A) || !aligned16(X_out)) return SHP_EINVAL;
-  if (n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  if (n > INT32_MAX || batch > INT32_MAX) return SHP_EUNSUPPORTED;
   if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_INV_ROOT, n, n, batch, o))
     return SHP_EINVAL;
+  if (small_block_ok(n, n, o->p)) {  // one CTA per block, the whole iteration on chip
+    CK(small_inv_root(A, static_cast<int>(n), static_cast<int>(batch), power, *o, S, X_out,
+                      rep ? rep->status : nullptr, rep ? rep->iters : nullptr,
+                      rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr,
+                      static_cast<cudaStream_t>(stream)));
+    return SHP_OK;
+  }
+  if (batch > 65535) return SHP_EUNSUPPORTED;
   CallKey key = make_key(0);
   key.power = power;
   key.a = A;
@@ -707,11 +718,20 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
   if (bf ? (n % 8 != 0 || m % 8 != 0) : (n % 4 != 0 || m % 4 != 0)) return SHP_EINVAL;
   if (!o->fixed_alpha && (S == nullptr || S_count < o->max_iter)) return SHP_EINVAL;
   if (!aligned16(G) || !aligned16(X_out)) return SHP_EINVAL;
-  if (m > INT32_MAX || n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
+  if (m > INT32_MAX || n > INT32_MAX || batch > INT32_MAX) return SHP_EUNSUPPORTED;
   shp_prism_opts oo = *o;
   oo.prec = storage;
   if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_POLAR, m, n, batch, &oo))
     return SHP_EINVAL;
+  if (!bf && small_block_ok(m, n, o->p)) {  // one CTA per block, the whole iteration on chip
+    CK(small_polar(static_cast<const float*>(G), static_cast<int>(m), static_cast<int>(n),
+                   static_cast<int>(batch), oo, S, static_cast<float*>(X_out),
+                   rep ? rep->status : nullptr, rep ? rep->iters : nullptr,
+                   rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr,
+                   static_cast<cudaStream_t>(stream)));
+    return SHP_OK;
+  }
+  if (batch > 65535) return SHP_EUNSUPPORTED;
   CallKey key = make_key(1);
   key.storage = storage;
   key.a = G;

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "shampoo_prism.h"
+
 namespace shp {
 
 // Kernels run so far on the current device, per translation unit (device
@@ -11,6 +13,7 @@ namespace shp {
 uint64_t kernel_runs_gemm();
 uint64_t kernel_runs_sketch();
 uint64_t kernel_runs_elementwise();
+uint64_t kernel_runs_small();
 
 enum Mode { MODE_TF32 = 0, MODE_3XTF32 = 1, MODE_BF16 = 2 };
 enum EpiKind {
@@ -163,5 +166,18 @@ cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
                          int out_bf16, cudaStream_t st);
 // report.status[b] = ETIMEOUT if flagged, else bs[b].status.
 cudaError_t write_status(const Ctl& ctl, int batch, int* report_status, cudaStream_t st);
+
+// ---- on-chip small blocks (small_block.cu): one CTA per block runs the
+// whole iteration in shared memory; products in fp32 FMA.
+// True when an m x n input (n x n for inverse roots) and sketch width p fit.
+bool small_block_ok(int64_t m, int64_t n, int p);
+// power: SHP_POW_*; report pointers may be null (layouts as the ABI's report).
+cudaError_t small_inv_root(const float* A, int n, int batch, int power,
+                           const shp_prism_opts& o, const float* S, float* X,
+                           int* rep_status, int* rep_iters, float* rep_resid, float* rep_alpha,
+                           cudaStream_t st);
+cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
+                        const float* S, float* X, int* rep_status, int* rep_iters,
+                        float* rep_resid, float* rep_alpha, cudaStream_t st);
 
 }  // namespace shp

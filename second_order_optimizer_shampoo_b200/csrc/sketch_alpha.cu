@@ -19,6 +19,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "prism_scalar.cuh"
 #include "shp_common.cuh"
 
 namespace shp {
@@ -104,112 +105,6 @@ __global__ void __launch_bounds__(SK_THREADS)
   }
 }
 
-// Coefficients of r_j(alpha) = T[j][0] + T[j][1] alpha + T[j][2] alpha^2 for
-// j = d..2d+1, written out from the expansion in the file header:
-//   d = 1 (f = 1):        r = (1-2a) xi + (2a - a^2) xi^2 + a^2 xi^3
-//   d = 2 (f = 1 + xi/2): r = (3/4 - 2a) xi^2 + (1/4 + a) xi^3 + (a - a^2) xi^4 + a^2 xi^5
-__device__ const double kRTab1[3][3] = {{1.0, -2.0, 0.0}, {0.0, 2.0, -1.0}, {0.0, 0.0, 1.0}};
-__device__ const double kRTab2[4][3] = {
-    {0.75, -2.0, 0.0}, {0.25, 1.0, 0.0}, {0.0, 1.0, -1.0}, {0.0, 0.0, 1.0}};
-
-__device__ double poly4(const double* c, double a) {
-  return (((c[4] * a + c[3]) * a + c[2]) * a + c[1]) * a + c[0];
-}
-__device__ double dpoly4(const double* c, double a) {
-  return ((4.0 * c[4] * a + 3.0 * c[3]) * a + 2.0 * c[2]) * a + c[1];
-}
-__device__ double d2poly4(const double* c, double a) {
-  return (12.0 * c[4] * a + 6.0 * c[3]) * a + 2.0 * c[2];
-}
-
-// Global minimiser of the quartic J on [lo, hi].  J' is monotone between the
-// real roots of J'' (a quadratic), so each such piece holds at most one root
-// of J', found by bisection and polished by Newton.  The candidate with the
-// least J wins; values within 1e-12 (relative) of the best tie and go to the
-// smaller alpha; a constant or non-finite J gives lo.
-__device__ double argmin_quartic(const double* c, double lo, double hi) {
-  bool finite = true;
-  double scale = 0.0;
-  for (int i = 0; i < 5; ++i) {
-    if (!isfinite(c[i])) finite = false;
-    if (i > 0) scale = fmax(scale, fabs(c[i]));
-  }
-  if (!finite || scale == 0.0) return lo;
-  double brk[4];
-  int nb = 0;
-  brk[nb++] = lo;
-  {
-    const double qa = 12.0 * c[4], qb = 6.0 * c[3], qc = 2.0 * c[2];
-    double r1 = NAN, r2 = NAN;
-    if (qa != 0.0) {
-      const double disc = qb * qb - 4.0 * qa * qc;
-      if (disc >= 0.0) {
-        const double sd = sqrt(disc);
-        const double q = -0.5 * (qb + (qb >= 0.0 ? sd : -sd));
-        if (q != 0.0) {
-          r1 = q / qa;
-          r2 = qc / q;
-        } else {
-          r1 = r2 = 0.0;
-        }
-      }
-    } else if (qb != 0.0) {
-      r1 = -qc / qb;
-    }
-    if (r1 > r2) {
-      const double t = r1;
-      r1 = r2;
-      r2 = t;
-    }
-    if (r1 > lo && r1 < hi) brk[nb++] = r1;
-    if (r2 > lo && r2 < hi && r2 != r1) brk[nb++] = r2;
-  }
-  brk[nb++] = hi;
-  double cand[5];
-  int nc = 0;
-  cand[nc++] = lo;
-  cand[nc++] = hi;
-  for (int s = 0; s + 1 < nb; ++s) {
-    double u = brk[s], v = brk[s + 1];
-    double fu = dpoly4(c, u), fv = dpoly4(c, v);
-    if (fu == 0.0) {
-      cand[nc++] = u;
-      continue;
-    }
-    if (fv == 0.0 || (fu < 0.0) == (fv < 0.0)) continue;
-    for (int it = 0; it < 200 && v - u > 1e-15 * fmax(1.0, fabs(u)); ++it) {
-      const double mid = 0.5 * (u + v);
-      const double fm = dpoly4(c, mid);
-      if (fm == 0.0) {
-        u = v = mid;
-        break;
-      }
-      if ((fm < 0.0) == (fu < 0.0)) {
-        u = mid;
-        fu = fm;
-      } else {
-        v = mid;
-      }
-    }
-    double a = 0.5 * (u + v);
-    for (int it = 0; it < 2; ++it) {
-      const double h = d2poly4(c, a);
-      if (h != 0.0) {
-        const double an = a - dpoly4(c, a) / h;
-        if (an >= brk[s] && an <= brk[s + 1]) a = an;
-      }
-    }
-    if (a > lo && a < hi) cand[nc++] = a;
-  }
-  double best = poly4(c, cand[0]);
-  for (int i = 1; i < nc; ++i) best = fmin(best, poly4(c, cand[i]));
-  const double thr = best + 1e-12 * fmax(fabs(best), 1e-300);
-  double pick = hi;
-  for (int i = 0; i < nc; ++i)
-    if (poly4(c, cand[i]) <= thr && cand[i] < pick) pick = cand[i];
-  return pick;
-}
-
 constexpr int AL_THREADS = 256;
 
 __global__ void __launch_bounds__(AL_THREADS)
@@ -261,17 +156,8 @@ __global__ void __launch_bounds__(AL_THREADS)
         ++idx;
       }
   }
-  double T[4][3];
-  for (int i = 0; i < nv; ++i)
-    for (int a = 0; a < 3; ++a) T[i][a] = d == 1 ? kRTab1[i][a] : kRTab2[i][a];
-  double coef[5] = {0, 0, 0, 0, 0};
-  for (int a = 0; a < 3; ++a)
-    for (int c = 0; c < 3; ++c) {
-      double s = 0.0;
-      for (int i = 0; i < nv; ++i)
-        for (int j = 0; j < nv; ++j) s += T[i][a] * M[i][j] * T[j][c];
-      coef[a + c] += s;
-    }
+  double coef[5];
+  quartic_from_gram(M, d, coef);
   const double a = argmin_quartic(coef, static_cast<double>(lo), static_cast<double>(hi));
   alpha[b] = static_cast<float>(a);
   if (Jc != nullptr)
@@ -291,15 +177,7 @@ __global__ void k_control(BlockState* bs, int* active, const int* it, int batch,
   const float r = sqrtf(s.norm2 / static_cast<float>(n));
   s.norm2 = 0.f;
   if (rep_res != nullptr) rep_res[b * res_stride + res_slot + k] = r;
-  int st = -1;
-  if (!isfinite(r))
-    st = ST_ENONFINITE;
-  else if (r <= tol)
-    st = ST_OK;
-  else if (k >= max_iter)
-    st = ST_ENOCONV;
-  else if (k >= 1 && s.prev_res < stall_below && r > stall_ratio * s.prev_res)
-    st = ST_ESTALL;
+  const int st = stop_rule(r, k, max_iter, tol, s.prev_res, stall_below, stall_ratio);
   s.prev_res = r;
   if (st >= 0) {
     active[b] = 0;

@@ -1,0 +1,464 @@
+// Newton-Schulz/PRISM on chip for small blocks (n <= 64): one CTA per block
+// runs every pass of the coupled iteration (or the whole polar iteration)
+// with all iterates in shared memory.  HBM is touched only to read the input
+// and the sketch slices and to write the result and the report.
+//
+// Block-diagonal Shampoo ("深度学习中的优化器之Shampoo算法原理与二阶优化机制"
+// §3.2) splits large layers into many small preconditioner blocks.  For a
+// 64 x 64 block a product is 0.5 MFLOP, far too little for a launch of its
+// own, so the batched path's per-iteration launches would dominate; here the
+// iteration never leaves the SM.  The steps are exactly those of the batched
+// path ("Sintesi Tecnica: PRISM", Parte I-II): residual, stop test, sketched
+// alpha fit, Delta = g - I, X + X Delta updates.
+//
+// Arithmetic: products on the CUDA cores in fp32 FMA (each thread owns a 4 x 4
+// output tile and streams float4 operands from shared memory), at least as
+// accurate as either fp32 storage mode of the batched path; the alpha fit and
+// the norms in fp64.  Four 64 x 68 fp32 buffers (68 KB) per CTA, three CTAs
+// per SM.
+#include <math.h>
+
+#include "internal.h"
+#include "prism_scalar.cuh"
+#include "shampoo_prism.h"
+#include "shp_common.cuh"
+
+namespace shp {
+
+namespace {
+
+constexpr int SB_NMAX = 64;
+// Row stride in floats: rows 4 apart (the two row groups one warp reads) land
+// 16 banks apart, so the float4 operand reads are conflict-free.
+constexpr int SB_LD = 68;
+constexpr int SB_MAT = SB_NMAX * SB_LD;
+constexpr int SB_THREADS = 256;
+constexpr int SB_PMAX = 16;
+constexpr int SB_SMEM = 4 * SB_MAT * static_cast<int>(sizeof(float));
+static_assert(4 * SB_NMAX * SB_PMAX <= SB_MAT, "sketch slots must fit one matrix buffer");
+
+struct SmallCfg {
+  int d, p, max_iter, fixed_alpha;
+  float lo, hi, tol, stall_below, stall_ratio;
+};
+
+// Sum over the CTA; every thread receives the result.
+SHP_DEV double block_sum(double v, double* red) {
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red may still be read by the previous call
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double s = 0.0;
+#pragma unroll
+  for (int w = 0; w < SB_THREADS / 32; ++w) s += red[w];
+  return s;
+}
+
+// acc = op(A) B on this thread's 4 x 4 tile (rows r0.., columns c0..), K a
+// multiple of 4.  op(A) = A (row-major M x K) or, with AT, the transpose of
+// the row-major K x M matrix A.
+template <bool AT>
+SHP_DEV void tile_mm(const float* A, const float* B, int K, int r0, int c0, float acc[4][4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < K; k += 4) {
+    float a[4][4], b[4][4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const float4 v = *reinterpret_cast<const float4*>(B + (k + kk) * SB_LD + c0);
+      b[kk][0] = v.x;
+      b[kk][1] = v.y;
+      b[kk][2] = v.z;
+      b[kk][3] = v.w;
+    }
+    if (AT) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const float4 v = *reinterpret_cast<const float4*>(A + (k + kk) * SB_LD + r0);
+        a[0][kk] = v.x;
+        a[1][kk] = v.y;
+        a[2][kk] = v.z;
+        a[3][kk] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(A + (r0 + i) * SB_LD + k);
+        a[i][0] = v.x;
+        a[i][1] = v.y;
+        a[i][2] = v.z;
+        a[i][3] = v.w;
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i][kk], b[kk][j], acc[i][j]);
+  }
+}
+
+SHP_DEV void store_row4(float* C, int row, int c0, const float* v) {
+  *reinterpret_cast<float4*>(C + row * SB_LD + c0) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// R = I - op(A) B on the n x n tile grid; returns this thread's sum of squares.
+template <bool AT>
+SHP_DEV float residual(const float* A, const float* B, int K, int n, float* R, int r0, int c0) {
+  float nrm = 0.f;
+  if (r0 < n && c0 < n) {
+    float acc[4][4];
+    tile_mm<AT>(A, B, K, r0, c0, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[j] = (r0 + i == c0 + j ? 1.f : 0.f) - acc[i][j];
+        nrm += v[j] * v[j];
+      }
+      store_row4(R, r0 + i, c0, v);
+    }
+  }
+  return nrm;
+}
+
+// C = X + A B (X may be A or B, C must be neither), rows x cols, inner K.
+SHP_DEV void axpy_mm(const float* A, const float* B, const float* X, int K, int rows, int cols,
+                     float* C, int r0, int c0) {
+  if (r0 >= rows || c0 >= cols) return;
+  float acc[4][4];
+  tile_mm<false>(A, B, K, r0, c0, acc);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 x = *reinterpret_cast<const float4*>(X + (r0 + i) * SB_LD + c0);
+    const float v[4] = {x.x + acc[i][0], x.y + acc[i][1], x.z + acc[i][2], x.w + acc[i][3]};
+    store_row4(C, r0 + i, c0, v);
+  }
+}
+
+// Delta = g - I: alpha R in place (d = 1), or W = R/2 + alpha R^2 (d = 2).
+// Returns the buffer that holds Delta.
+SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, int r0, int c0) {
+  if (d == 1) {
+    for (int e = threadIdx.x; e < n * n; e += SB_THREADS) {
+      const int i = e / n, j = e - i * n;
+      R[i * SB_LD + j] *= alpha;
+    }
+    __syncthreads();
+    return R;
+  }
+  if (r0 < n && c0 < n) {
+    float acc[4][4];
+    tile_mm<false>(R, R, n, r0, c0, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 r = *reinterpret_cast<const float4*>(R + (r0 + i) * SB_LD + c0);
+      const float v[4] = {0.5f * r.x + alpha * acc[i][0], 0.5f * r.y + alpha * acc[i][1],
+                          0.5f * r.z + alpha * acc[i][2], 0.5f * r.w + alpha * acc[i][3]};
+      store_row4(W, r0 + i, c0, v);
+    }
+  }
+  __syncthreads();
+  return W;
+}
+
+// Sketched alpha of one iteration: V_j = R^j S_k for j <= 2d+1 (S_k = n x p
+// slice in HBM), Gram of V_d..V_{2d+1} in fp64, argmin of the quartic on
+// [lo, hi].  V is a free matrix buffer: slot j - d holds V_j (d = 2 parks
+// V_1 in slot 2 and S in slot 3 until they are overwritten).
+SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float* Sk, float* V,
+                           double (*red)[10], float* s_alpha) {
+  const int p = o.p, d = o.d, np = n * p, tid = threadIdx.x;
+  float* slot[4] = {V, V + np, V + 2 * np, V + 3 * np};
+  for (int e = tid; e < np; e += SB_THREADS) slot[3][e] = Sk[e];
+  __syncthreads();
+  const float* src = slot[3];
+  for (int j = 1; j <= 2 * d + 1; ++j) {
+    float* dst = j >= d ? slot[j - d] : slot[2];
+    for (int e = tid; e < np; e += SB_THREADS) {
+      const int row = e / p, col = e - row * p;
+      const float* Rr = R + row * SB_LD;
+      float s = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < n; ++k) s = fmaf(Rr[k], src[k * p + col], s);
+      dst[e] = s;
+    }
+    __syncthreads();
+    src = dst;
+  }
+  const int nv = d + 2;
+  double part[10];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) part[i] = 0.0;
+  for (int e = tid; e < np; e += SB_THREADS) {
+    double x[4];
+    for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(slot[i][e]);
+    int idx = 0;
+    for (int i = 0; i < nv; ++i)
+      for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const double s = warp_sum(part[i]);
+    if (lane == 0) red[warp][i] = s;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double M[4][4];
+    int idx = 0;
+    for (int i = 0; i < nv; ++i)
+      for (int j = i; j < nv; ++j) {
+        double s = 0.0;
+        for (int w = 0; w < SB_THREADS / 32; ++w) s += red[w][idx];
+        M[i][j] = M[j][i] = s;
+        ++idx;
+      }
+    double coef[5];
+    quartic_from_gram(M, d, coef);
+    *s_alpha = static_cast<float>(
+        argmin_quartic(coef, static_cast<double>(o.lo), static_cast<double>(o.hi)));
+  }
+  __syncthreads();
+  return *s_alpha;
+}
+
+// Report slots: resid[b][pass][k] (max_iter + 1 per pass), alpha[b][pass][k]
+// (max_iter per pass), iters[b][pass], status[b].
+struct SmallReport {
+  int* status;
+  int* iters;
+  float* resid;
+  float* alpha;
+};
+
+// Coupled Newton-Schulz for A^(1/2), A^(-1/2) (one pass) or A^(-1/4) (a
+// second pass on Y_1), one CTA per n x n block.
+__global__ void __launch_bounds__(SB_THREADS, 3)
+    k_small_inv_root(const float* __restrict__ A, int n, int npass, int power, SmallCfg o,
+                     const float* __restrict__ S, float* __restrict__ X, SmallReport rep) {
+  count_kernel_run();
+  extern __shared__ __align__(16) float sm[];
+  __shared__ double red[SB_THREADS / 32][10];
+  __shared__ float s_alpha;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
+  const int64_t nn = static_cast<int64_t>(n) * n;
+  const float* Ab = A + b * nn;
+  float *Y = sm, *Z = sm + SB_MAT, *R = sm + 2 * SB_MAT, *W = sm + 3 * SB_MAT;
+
+  // c = ||A||_F (fp64) and Y_0 = A / c
+  double part = 0.0;
+  for (int e = tid; e < nn; e += SB_THREADS) {
+    const float v = Ab[e];
+    part += static_cast<double>(v) * v;
+  }
+  const float c = static_cast<float>(sqrt(block_sum(part, red[0])));
+  for (int e = tid; e < nn; e += SB_THREADS) {
+    const int i = e / n, j = e - i * n;
+    Y[i * SB_LD + j] = Ab[e] / c;
+  }
+  __syncthreads();
+
+  int status = ST_OK;
+  const int mi = o.max_iter;
+  for (int pass = 0; pass < npass; ++pass) {
+    // Z_0 = I, R_0 = I - Y_0 (pass 2 starts from Y_1)
+    float nrm = 0.f;
+    for (int e = tid; e < nn; e += SB_THREADS) {
+      const int i = e / n, j = e - i * n;
+      const float id = i == j ? 1.f : 0.f;
+      const float r = id - Y[i * SB_LD + j];
+      Z[i * SB_LD + j] = id;
+      R[i * SB_LD + j] = r;
+      nrm += r * r;
+    }
+    double n2 = block_sum(nrm, red[0]);
+    float prev = INFINITY;
+    for (int k = 0;; ++k) {
+      if (k > 0) n2 = block_sum(residual<false>(Z, Y, n, n, R, r0, c0), red[0]);
+      // every thread evaluates the stop rule on the same reduced norm
+      const float r = sqrtf(static_cast<float>(n2) / static_cast<float>(n));
+      const int st = stop_rule(r, k, mi, o.tol, prev, o.stall_below, o.stall_ratio);
+      if (tid == 0 && rep.resid != nullptr) rep.resid[(2 * b + pass) * (mi + 1) + k] = r;
+      prev = r;
+      if (st >= 0) {
+        if (tid == 0 && rep.iters != nullptr) rep.iters[2 * b + pass] = k;
+        if (status == ST_OK) status = st;
+        break;
+      }
+      const float alpha =
+          o.fixed_alpha ? o.lo
+                        : sketch_alpha(R, n, o, S + (static_cast<int64_t>(pass) * mi + k) * n * o.p,
+                                       W, red, &s_alpha);
+      if (tid == 0 && rep.alpha != nullptr) rep.alpha[(2 * b + pass) * mi + k] = alpha;
+      float* D = form_delta(o.d, alpha, R, W, n, r0, c0);
+      float* T = o.d == 1 ? W : R;  // the buffer Delta does not occupy
+      axpy_mm(Y, D, Y, n, n, n, T, r0, c0);  // Y_{k+1} = Y_k + Y_k Delta
+      __syncthreads();
+      if (k == 0) {  // Z_1 = I + Delta
+        for (int e = tid; e < nn; e += SB_THREADS) {
+          const int i = e / n, j = e - i * n;
+          Y[i * SB_LD + j] = (i == j ? 1.f : 0.f) + D[i * SB_LD + j];
+        }
+      } else {  // Z_{k+1} = Z_k + Delta Z_k
+        axpy_mm(D, Z, Z, n, n, n, Y, r0, c0);
+      }
+      __syncthreads();
+      float* oldZ = Z;
+      Z = Y;
+      Y = T;
+      if (o.d == 1)
+        W = oldZ;
+      else
+        R = oldZ;
+    }
+  }
+
+  double sc;
+  const double cd = static_cast<double>(c);
+  if (power == SHP_POW_SQRT)
+    sc = sqrt(cd);
+  else if (power == SHP_POW_INV2)
+    sc = 1.0 / sqrt(cd);
+  else
+    sc = 1.0 / sqrt(sqrt(cd));
+  const float scale = static_cast<float>(sc);
+  const float* Src = power == SHP_POW_SQRT ? Y : Z;
+  float* Xb = X + b * nn;
+  for (int e = tid; e < nn; e += SB_THREADS) {
+    const int i = e / n, j = e - i * n;
+    Xb[e] = scale * Src[i * SB_LD + j];
+  }
+  if (tid == 0 && rep.status != nullptr) rep.status[b] = status;
+}
+
+// Polar factor of an m x n block (m, n <= 64): the tall iteration on G (or on
+// G^T when m < n), X_0 = G / ||G||_F, R = I - X^T X, X <- X + X Delta.
+__global__ void __launch_bounds__(SB_THREADS, 3)
+    k_small_polar(const float* __restrict__ G, int m, int n, SmallCfg o,
+                  const float* __restrict__ S, float* __restrict__ Xout, SmallReport rep) {
+  count_kernel_run();
+  extern __shared__ __align__(16) float sm[];
+  __shared__ double red[SB_THREADS / 32][10];
+  __shared__ float s_alpha;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
+  const bool tall = m >= n;
+  const int rows = tall ? m : n, k_n = tall ? n : m;  // X is rows x k_n
+  const int64_t mn = static_cast<int64_t>(m) * n;
+  const float* Gb = G + b * mn;
+  float *X = sm, *R = sm + SB_MAT, *W = sm + 2 * SB_MAT, *T = sm + 3 * SB_MAT;
+
+  double part = 0.0;
+  for (int e = tid; e < mn; e += SB_THREADS) {
+    const float v = Gb[e];
+    part += static_cast<double>(v) * v;
+  }
+  const float c = static_cast<float>(sqrt(block_sum(part, red[0])));
+  const float inv = c > 0.f ? 1.f / c : 0.f;
+  for (int e = tid; e < mn; e += SB_THREADS) {
+    const int i = e / n, j = e - i * n;  // G(i, j)
+    if (tall)
+      X[i * SB_LD + j] = Gb[e] * inv;
+    else
+      X[j * SB_LD + i] = Gb[e] * inv;
+  }
+  __syncthreads();
+
+  const int mi = o.max_iter;
+  int status = ST_OK;
+  float prev = INFINITY;
+  for (int k = 0;; ++k) {
+    const double n2 = block_sum(residual<true>(X, X, rows, k_n, R, r0, c0), red[0]);
+    const float r = sqrtf(static_cast<float>(n2) / static_cast<float>(k_n));
+    const int st = stop_rule(r, k, mi, o.tol, prev, o.stall_below, o.stall_ratio);
+    if (tid == 0 && rep.resid != nullptr) rep.resid[2 * b * (mi + 1) + k] = r;
+    prev = r;
+    if (st >= 0) {
+      if (tid == 0 && rep.iters != nullptr) rep.iters[2 * b] = k;
+      status = st;
+      break;
+    }
+    const float alpha =
+        o.fixed_alpha ? o.lo
+                      : sketch_alpha(R, k_n, o, S + static_cast<int64_t>(k) * k_n * o.p, T, red,
+                                     &s_alpha);
+    if (tid == 0 && rep.alpha != nullptr) rep.alpha[2 * b * mi + k] = alpha;
+    float* D = form_delta(o.d, alpha, R, W, k_n, r0, c0);
+    axpy_mm(X, D, X, k_n, rows, k_n, T, r0, c0);  // X_{k+1} = X_k + X_k Delta
+    __syncthreads();
+    float* t = X;
+    X = T;
+    T = t;
+  }
+
+  float* Xb = Xout + b * mn;
+  for (int e = tid; e < mn; e += SB_THREADS) {
+    const int i = e / n, j = e - i * n;
+    Xb[e] = tall ? X[i * SB_LD + j] : X[j * SB_LD + i];
+  }
+  if (tid == 0 && rep.status != nullptr) rep.status[b] = status;
+}
+
+SmallCfg make_cfg(const shp_prism_opts& s) {
+  SmallCfg c;
+  c.d = s.d;
+  c.p = s.p;
+  c.max_iter = s.max_iter;
+  c.fixed_alpha = s.fixed_alpha;
+  c.lo = s.lo;
+  c.hi = s.hi;
+  c.tol = s.tol;
+  c.stall_below = s.stall_below;
+  c.stall_ratio = s.stall_ratio;
+  return c;
+}
+
+template <typename K>
+cudaError_t prepare(K kern) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SB_SMEM);
+}
+
+}  // namespace
+
+bool small_block_ok(int64_t m, int64_t n, int p) {
+  return m > 0 && n > 0 && m <= SB_NMAX && n <= SB_NMAX && p <= SB_PMAX;
+}
+
+cudaError_t small_inv_root(const float* A, int n, int batch, int power, const shp_prism_opts& o,
+                           const float* S, float* X, int* rep_status, int* rep_iters,
+                           float* rep_resid, float* rep_alpha, cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  cudaError_t e = prepare(k_small_inv_root);
+  if (e != cudaSuccess) return e;
+  const int npass = power == SHP_POW_INV4 ? 2 : 1;
+  k_small_inv_root<<<batch, SB_THREADS, SB_SMEM, st>>>(
+      A, n, npass, power, make_cfg(o), S, X, SmallReport{rep_status, rep_iters, rep_resid, rep_alpha});
+  return cudaGetLastError();
+}
+
+cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
+                        const float* S, float* X, int* rep_status, int* rep_iters,
+                        float* rep_resid, float* rep_alpha, cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  cudaError_t e = prepare(k_small_polar);
+  if (e != cudaSuccess) return e;
+  k_small_polar<<<batch, SB_THREADS, SB_SMEM, st>>>(
+      G, m, n, make_cfg(o), S, X, SmallReport{rep_status, rep_iters, rep_resid, rep_alpha});
+  return cudaGetLastError();
+}
+
+uint64_t kernel_runs_small() {
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_kernel_runs, sizeof(v)) != cudaSuccess) return 0;
+  return v;
+}
+
+}  // namespace shp
