@@ -36,10 +36,11 @@ N, BATCH, LAM_LO, D, P, TOL, MAX_ITER = 1024, 64, 1e-6, 2, 8, 1e-3, 24
 SEED_A, SEED_S = 103, 1003
 # tensor peak ratios (nominal dense): TF32 / BF16 = 1.1 / 2.25 PFLOP/s
 TF32_OVER_BF16 = 1.1 / 2.25
-# dram__bytes_read.sum + dram__bytes_write.sum of one 64 x 1024^3 3xTF32 launch
-# of the persistent GEMM (ncu capture of 16 blocks scaled x4 by the blocks
-# processed; None until captured for the current kernel)
-GEMM_TRAFFIC_PER_LAUNCH = None
+# dram__bytes_read.sum + dram__bytes_write.sum (bytes) of one 64 x 1024^3 3xTF32
+# launch of the persistent GEMM: an ncu capture of 16 blocks (289.5 MB read,
+# 41.8 MB written) scaled x4 by the blocks processed, as every operand and
+# output grows with the batch
+GEMM_TRAFFIC_PER_LAUNCH = 4 * (289.454e6 + 41.826e6)
 
 
 def workload_config(world):
@@ -211,6 +212,9 @@ def gemm_only(args):
 
 SB_N, SB_BATCH, SB_P, SB_MAX_ITER = 64, 16384, 4, 50
 FP32_LANES_PER_SM, SMS = 128, 148
+# dram__bytes_read.sum + dram__bytes_write.sum of one full-size small-block
+# launch (ncu capture of this workload)
+SMALL_TRAFFIC_PER_LAUNCH = 291.870e6 + 264.608e6
 
 
 def small_block_leg(args, dev, stream, sm_max_mhz):
@@ -255,9 +259,31 @@ def small_block_leg(args, dev, stream, sm_max_mhz):
             "median_iters_per_pass": [int(x) for x in np.median(iters, axis=0)],
             "hbm_gbs": hbm_bytes / (ms / 1e3) / 1e9, "hbm_peak_gbs": peaks["hbm_gbs"],
             "roofline": {"bound": "alu", "achieved": tf, "peak": fma_peak, "unit": "TFLOP/s",
-                         "frac": tf / fma_peak,
+                         "frac": tf / fma_peak, "traffic": SMALL_TRAFFIC_PER_LAUNCH,
+                         "traffic_unit": "bytes per launch", "algorithmic_bytes": hbm_bytes,
                          "peak_note": f"fp32 FMA: {SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 "
                                       f"flop x {sm_max_mhz:.0f} MHz (max SM clock)"}}
+
+
+def small_only(args):
+    """The small-block kernel alone (profiling aid): --batch blocks of 64 x 64."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism, synth
+    dev = torch.device("cuda", 0)
+    batch = args.batch if args.batch != BATCH else SB_BATCH
+    A = torch.from_numpy(synth.spd_batch(SB_N, batch, 1e-3, 1.0, 101)).to(dev)
+    S = torch.from_numpy(synth.sketch_stack(2 * SB_MAX_ITER, SB_N, SB_P, 1001)).to(dev)
+    opts = prism.make_opts(d=1, p=SB_P, lo=0.5, tol=1e-6, max_iter=SB_MAX_ITER, prec="3xtf32")
+    X = torch.empty_like(A)
+    rep = prism.make_report(batch, SB_MAX_ITER, dev)
+    for _ in range(max(args.warmup, 1) + args.steps):
+        prism.matfn_inv_root(A, "inv4", opts, S, out=X, report=rep)
+    torch.cuda.synchronize()
+    ok = int((rep["status"].cpu().numpy() == 0).sum())
+    print(json.dumps({"kernel": "small", "batch": batch, "status_ok": ok,
+                      "launches": args.steps + max(args.warmup, 1)}))
+    return 0
 
 
 PM, PN, PBATCH, PRANK = 4096, 1024, 96, 64
@@ -323,14 +349,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-polar", action="store_true", help="skip the polar-factor leg")
     ap.add_argument("--no-small", action="store_true", help="skip the small-block leg")
-    ap.add_argument("--kernel", default=None, choices=["gemm"],
-                    help="run only the batched 3xTF32 GEMM (for profiling)")
+    ap.add_argument("--kernel", default=None, choices=["gemm", "small"],
+                    help="run only the batched 3xTF32 GEMM or the small-block kernel "
+                         "(for profiling; --batch sets the batch)")
     ap.add_argument("--batch", type=int, default=BATCH)
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.kernel == "gemm":
         return gemm_only(args)
+    if args.kernel == "small":
+        return small_only(args)
 
     import numpy as np
     import torch
@@ -451,7 +480,8 @@ def main():
         "kernel": "k_gemm_tc<3xTF32> (batched 64 x 1024^3)",
         "bound": "tensor", "achieved": gemm_achieved, "peak": split_peak_burst,
         "unit": "TFLOP/s", "frac": gemm_achieved / split_peak_burst,
-        "traffic": GEMM_TRAFFIC_PER_LAUNCH,
+        "traffic": GEMM_TRAFFIC_PER_LAUNCH, "traffic_unit": "bytes per launch",
+        "algorithmic_bytes": 5 * BATCH * N * N * 4,
         "peak_note": f"{peak_src} burst BF16 x 1.1/2.25 (TF32) / 3 (3xTF32 products)",
         "ms_per_launch": gemm_ms,
     }
