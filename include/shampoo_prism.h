@@ -29,8 +29,11 @@
  *     CUDA runtime error at launch; the stream may hold partial work).
  *     Numerical outcomes are per-block codes written to `report.status` on the
  *     device; the caller reads them after synchronising the stream.
- *   - No exceptions cross this boundary; the library keeps no state between
- *     calls other than cached kernel attributes.
+ *   - No exceptions cross this boundary.  State kept between calls: cached
+ *     kernel attributes, and up to 16 instantiated CUDA graphs of the matrix
+ *     functions keyed by every pointer, size and option of a call (a repeated
+ *     call with the same buffers replays its graph; the oldest
+ *     entry is replaced).
  */
 #ifndef SHAMPOO_PRISM_H
 #define SHAMPOO_PRISM_H
@@ -135,7 +138,10 @@ int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float*
  * S: [S_count][n][p] fp32 Gaussian sketches shared by the batch; pass 1
  *   iteration k uses S[k], pass 2 uses S[max_iter + k]; S_count must be
  *   >= max_iter (one pass) or >= 2 * max_iter (SHP_POW_INV4).
- * Output of a block that stopped without converging is its last iterate. */
+ * Output of a block that stopped without converging is its last iterate.
+ * Blocks with n <= 64 and p <= 16 run on chip, one CTA per block with fp32
+ * products for either precision; they need a 256-byte workspace and allow
+ * batch > 65535. */
 int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
                    const shp_prism_opts* opts, const float* S, int64_t S_count, float* X_out,
                    const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
@@ -146,7 +152,8 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
  *   X_{k+1} = X_k g_d(R_k; alpha_k).  A wide G (m < n) is handled as G^T.
  * G, X_out: [batch][m][n], bf16 (storage = SHP_BF16; the iterate is kept in
  *   bf16 with fp32 accumulation) or fp32 (storage = SHP_TF32 / SHP_3XTF32).
- * S: [S_count][min(m,n)][p] fp32, S_count >= max_iter. */
+ * S: [S_count][min(m,n)][p] fp32, S_count >= max_iter.
+ * fp32 inputs with m, n <= 64 and p <= 16 run on chip (as matfn_inv_root). */
 int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
                 const shp_prism_opts* opts, const float* S, int64_t S_count, void* X_out,
                 const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
