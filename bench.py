@@ -286,6 +286,119 @@ def small_only(args):
     return 0
 
 
+def _time(fn, stream, reps):
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def shampoo_step_leg(args, dev, stream):
+    """One Shampoo step on a 1024 x 1024 weight: 10 EMA steps of L and R with
+    fresh G (TF32), L^(-1/4) and R^(-1/4) by PRISM (d = 2, p = 8, tol 1e-3,
+    TF32) as one batch of two, and W -= 1e-3 L^(-1/4) G R^(-1/4)."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import _abi, prism, synth
+    n, beta, eps, lr, mi = 1024, 0.95, 1e-6, 1e-3, 30
+    W0 = torch.from_numpy(synth.gaussian((1, n, n), 0.02, 102, index=0)).to(dev)
+    Gs = [torch.from_numpy(synth.gaussian((1, n, n), 0.02, 102, index=t + 1)).to(dev)
+          for t in range(10)]
+    S = torch.from_numpy(synth.sketch_stack(2 * mi, n, 8, 1002)).to(dev)
+    opts = prism.make_opts(d=2, p=8, tol=1e-3, max_iter=mi, prec="tf32")
+    LR = torch.zeros(2, n, n, device=dev)
+    W = W0.clone()
+    roots = torch.empty_like(LR)
+    rep = prism.make_report(2, mi, dev)
+    ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, n, n, 2, opts),
+                     dtype=torch.uint8, device=dev)
+    eye = torch.eye(n, device=dev) * eps
+
+    def step():
+        LR.copy_(eye.expand(2, n, n))
+        W.copy_(W0)
+        for G in Gs:
+            prism.shampoo_gram_ema(G, LR[0:1], LR[1:2], beta, eps, "tf32")
+        prism.matfn_inv_root(LR, "inv4", opts, S, out=roots, ws=ws, report=rep)
+        prism.shampoo_apply(W, Gs[-1], roots[0:1], roots[1:2], lr, "tf32")
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    iters = rep["iters"].cpu().numpy()
+    ms = _time(step, stream, 10)
+    products = sum(max(4 * int(k) - 1, 0) for blk in iters for k in blk)
+    flops = 10 * 2 * n * (n + 1) * n + products * 2.0 * n ** 3 + 2 * 2.0 * n ** 3
+    return {"workload": "shampoo_step_1024sq_ema10_inv4_d2_p8_tf32_apply", "ms_per_step": ms,
+            "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "preconditioners_per_s": 2 / (ms / 1e3),
+            "iters_per_pass": [[int(k) for k in blk] for blk in iters],
+            "status": [int(x) for x in rep["status"].cpu().numpy()],
+            "note": "EMA products counted n(n+1)n (symmetric), computed as full GEMMs"}
+
+
+def gemm_count_leg(args, dev, stream, A):
+    """GEMMs to residual 1e-3 per pass on the config-3 batch: PRISM d = 2
+    against the fixed-coefficient (Taylor) iterations d = 2 and d = 1."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism, synth
+    mi = 40
+    S = torch.from_numpy(synth.sketch_stack(2 * mi, N, P, SEED_S)).to(dev)
+    out = {}
+    for name, d, fixed in (("prism_d2", 2, False), ("taylor_d2", 2, True),
+                           ("taylor_d1", 1, True)):
+        opts = prism.make_opts(d=d, p=P, tol=TOL, max_iter=mi, prec="3xtf32", fixed_alpha=fixed)
+        X, rep = prism.matfn_inv_root(A, "inv4", opts, S)
+        torch.cuda.synchronize()
+        it = rep["iters"].cpu().numpy()
+        per = (3 if d == 1 else 4)
+        counts = [sum(max(per * int(k) - 1, 0) for k in blk) for blk in it]
+        out[name] = {"median_iters_per_pass": [int(x) for x in np.median(it, axis=0)],
+                     "median_gemms_per_block": float(np.median(counts)),
+                     "status_ok": int((rep["status"].cpu().numpy() == 0).sum())}
+    return out
+
+
+def single_block_leg(args, dev, stream):
+    """Config 1 as single calls: one 64 x 64 A^(-1/4) (d = 1, p = 4, tol 1e-6)
+    and one 64 x 32 polar factor, microseconds per call."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import _abi, prism, synth
+    A = torch.from_numpy(synth.spd_batch(64, 1, 1e-3, 1.0, 101)).to(dev)
+    S = torch.from_numpy(synth.sketch_stack(100, 64, 4, 1001)).to(dev)
+    opts = prism.make_opts(d=1, p=4, lo=0.5, tol=1e-6, max_iter=50, prec="3xtf32")
+    X = torch.empty_like(A)
+    rep = prism.make_report(1, 50, dev)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    G = torch.from_numpy(synth.gaussian((1, 64, 32), 1.0, 101)).to(dev)
+    Sp = torch.from_numpy(synth.sketch_stack(50, 32, 4, 1001)).to(dev)
+    Xp = torch.empty_like(G)
+    repp = prism.make_report(1, 50, dev)
+
+    def root():
+        prism.matfn_inv_root(A, "inv4", opts, S, out=X, ws=ws, report=rep)
+
+    def polar():
+        prism.matfn_polar(G, opts, Sp, out=Xp, ws=ws, report=repp)
+
+    for _ in range(5):
+        root()
+        polar()
+    torch.cuda.synchronize()
+    return {"workload": "inv4_root_64sq_cond1e3_d1_p4_tol1e-6 + polar_64x32_d1_p4",
+            "us_per_inv_root": 1e3 * _time(root, stream, 50),
+            "us_per_polar": 1e3 * _time(polar, stream, 50),
+            "iters_inv_root": [int(k) for k in rep["iters"].cpu().numpy()[0]],
+            "iters_polar": int(repp["iters"].cpu().numpy()[0][0])}
+
+
 PM, PN, PBATCH, PRANK = 4096, 1024, 96, 64
 
 
@@ -349,6 +462,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-polar", action="store_true", help="skip the polar-factor leg")
     ap.add_argument("--no-small", action="store_true", help="skip the small-block leg")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the Shampoo-step, GEMM-count and single-block legs")
     ap.add_argument("--kernel", default=None, choices=["gemm", "small"],
                     help="run only the batched 3xTF32 GEMM or the small-block kernel "
                          "(for profiling; --batch sets the batch)")
@@ -487,6 +602,10 @@ def main():
     }
 
     polar = None if args.no_polar else polar_leg(args, dev, stream)
+    extra = not args.no_extra and world == 1
+    step2 = shampoo_step_leg(args, dev, stream) if extra else None
+    counts = gemm_count_leg(args, dev, stream, A) if extra else None
+    single = single_block_leg(args, dev, stream) if extra else None
     small = None if args.no_small else small_block_leg(args, dev, stream,
                                                         peaks.get("sm_max_mhz", 1965.0))
 
@@ -520,6 +639,9 @@ def main():
             "roofline": roofline,
             "polar": polar,
             "small_blocks": small,
+            "shampoo_step_1024": step2,
+            "gemms_to_residual": counts,
+            "single_64": single,
             "cpu_baseline": cpu,
             "clocks": clocks,
         }

@@ -9,7 +9,7 @@ Every function follows one passage of the source pages, cited in its
 docstring by page title and section:
 
 * [Shampoo]  "深度学习中的优化器之Shampoo算法原理与二阶优化机制"
-  (algorithm.idocdown.com), sections 2.2, 2.3, 3.1, 6.3.
+  (algorithm.idocdown.com), sections 2.2, 2.3, 3.1, 5.1, 5.2, 6.3.
 * [PRISM-it] "Sintesi Tecnica: PRISM" (gist.science), "Parte I" and
   "Parte II" (residual-form iteration, adaptive polynomial, alpha fit,
   clamp, randomized sketch).
@@ -25,6 +25,9 @@ Readings taken where the pages are silent (each is listed in the design doc):
   constant objective gives alpha = lo).
 * Sketch slices: pass 1 iteration k uses S[k]; pass 2 iteration k uses
   S[max_iter + k]; the polar iteration k uses S[k].
+* The momentum variant follows the recursion the page prints
+  (M_t = gamma M_{t-1} + P_t, W -= eta M_t), which is heavy-ball although
+  the page calls it Nesterov.
 * Stopping: residual ||R_k||_F / sqrt(n) <= tol, checked before the update;
   at most max_iter updates; a non-finite residual stops with ENONFINITE; a
   residual that stops shrinking once small stops with ESTALL.
@@ -106,6 +109,29 @@ def apply_ref(W, G, PL, PR, lr):
     W_{t+1} = W_t - lr * L^(-1/4) G R^(-1/4), with PL = L^(-1/4), PR = R^(-1/4)."""
     W, G, PL, PR = _f64(W), _f64(G), _f64(PL), _f64(PR)
     return W - lr * (PL @ G @ PR)
+
+
+def apply_variant_ref(W, G, PL, PR, lr, M=None, gamma=0.0, acc=None):
+    """The update variants of [Shampoo] §5 on P = L^(-1/4) G R^(-1/4):
+
+    §5.1 adaptive step: the running sum of squared gradient norms grows by
+    ||G_t||_F^2 and the step is lr / sqrt(1 + that sum), so with `acc` (the
+    sum before this step) eta = lr / sqrt(1 + acc + ||G||_F^2);
+    §5.2 momentum, in the recursion the page prints: M_t = gamma M_{t-1} + P_t
+    and W_{t+1} = W_t - eta M_t.
+
+    Without M the step is W - eta P; without acc, eta = lr.  Returns
+    (W, M, acc) after the step (M and acc None when not used)."""
+    W, G, PL, PR = _f64(W), _f64(G), _f64(PL), _f64(PR)
+    P = PL @ G @ PR
+    eta = lr
+    if acc is not None:
+        acc = float(acc) + float(np.sum(G * G))
+        eta = lr / sqrt(1.0 + acc)
+    if M is not None:
+        M = gamma * _f64(M) + P
+        return W - eta * M, M, acc
+    return W - eta * P, None, acc
 
 
 # ---------------------------------------------------------------------------

@@ -339,6 +339,62 @@ def test_apply_closed_forms():
             assert got[i, j] == pytest.approx(W[i, j] - 0.01 * a[i] * G[i, j] * b[j], rel=1e-15)
 
 
+def test_apply_momentum_closed_form():
+    """[Shampoo] §5.2 with a constant gradient and identity preconditioners:
+    M_t = sum_{i<t} gamma^i G = (1 - gamma^t)/(1 - gamma) G, so after T steps
+    W_T = W_0 - lr G sum_{t=1..T} (1 - gamma^t)/(1 - gamma)."""
+    rng = np.random.default_rng(5)
+    W0, G = rng.standard_normal((4, 6)), rng.standard_normal((4, 6))
+    lr, gamma, T = 0.05, 0.9, 5
+    W, M = W0, np.zeros_like(W0)
+    for _ in range(T):
+        W, M, acc = o.apply_variant_ref(W, G, np.eye(4), np.eye(6), lr, M=M, gamma=gamma)
+        assert acc is None
+    geo = sum((1 - gamma ** t) / (1 - gamma) for t in range(1, T + 1))
+    np.testing.assert_allclose(W, W0 - lr * geo * G, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(M, (1 - gamma ** T) / (1 - gamma) * G, rtol=1e-13)
+    # gamma = 0 is the plain update
+    W1, M1, _ = o.apply_variant_ref(W0, G, np.eye(4), np.eye(6), lr, M=np.ones_like(W0),
+                                    gamma=0.0)
+    np.testing.assert_allclose(W1, W0 - lr * G, rtol=1e-15)
+
+
+def test_apply_adaptive_step_closed_form():
+    """[Shampoo] §5.1: eta_t = lr / sqrt(1 + sum_{i<=t} ||G_i||^2).  With
+    G_t = c_t E (E a unit matrix entry) and identity preconditioners,
+    W_T = W_0 - sum_t lr c_t / sqrt(1 + sum_{i<=t} c_i^2) E."""
+    W0 = np.zeros((3, 3))
+    E = np.zeros((3, 3))
+    E[1, 2] = 1.0
+    lr, cs = 0.1, [2.0, 0.5, 3.0, 1.0]
+    W, acc, want, run = W0, 0.0, 0.0, 0.0
+    for c in cs:
+        W, M, acc = o.apply_variant_ref(W, c * E, np.eye(3), np.eye(3), lr, acc=acc)
+        assert M is None
+        run += c * c
+        want += lr * c / np.sqrt(1.0 + run)
+    assert acc == pytest.approx(sum(c * c for c in cs), rel=1e-15)
+    np.testing.assert_allclose(W, -want * E, rtol=1e-14, atol=1e-16)
+
+
+def test_apply_variants_diagonal_preconditioners():
+    """P = PL G PR in that order (diagonal PL, PR: P_ij = a_i G_ij b_j), both
+    variants together: a transposed or swapped factor fails this."""
+    rng = np.random.default_rng(6)
+    m, n, lr, gamma = 5, 3, 0.01, 0.8
+    W0, G, M0 = (rng.standard_normal((m, n)) for _ in range(3))
+    a, b = rng.uniform(1, 2, m), rng.uniform(1, 2, n)
+    acc0 = 2.5
+    W, M, acc = o.apply_variant_ref(W0, G, np.diag(a), np.diag(b), lr, M=M0, gamma=gamma,
+                                    acc=acc0)
+    eta = lr / np.sqrt(1.0 + acc0 + np.sum(G * G))
+    for i in range(m):
+        for j in range(n):
+            mij = gamma * M0[i, j] + a[i] * G[i, j] * b[j]
+            assert M[i, j] == pytest.approx(mij, rel=1e-14)
+            assert W[i, j] == pytest.approx(W0[i, j] - eta * mij, rel=1e-14)
+
+
 def test_shampoo_step_vs_eigh():
     rng = np.random.default_rng(8)
     m, n, eps, beta, lr = 16, 8, 1e-6, 0.95, 1e-3
