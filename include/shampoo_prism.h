@@ -176,6 +176,19 @@ int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rro
                   int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
                   shp_stream stream);
 
+/* Preconditioned update with the variants of [Shampoo] 5.1-5.2, P = Lroot G Rroot:
+ *   adaptive step (gnorm2_acc non-NULL): acc[b] += ||G[b]||_F^2 and
+ *     eta_b = lr / sqrt(1 + acc[b]); otherwise eta_b = lr;
+ *   momentum (M non-NULL), the recursion as the page prints it:
+ *     M <- gamma M + P,  W <- W - eta_b M;  otherwise W <- W - eta_b P.
+ * W, G, M: [batch][m][n] fp32 (W and M updated in place; M 16-byte aligned);
+ * gnorm2_acc: [batch] fp64 running sums, updated in place; Lroot, Rroot as in
+ * shampoo_apply.  With M = gnorm2_acc = NULL this is shampoo_apply.
+ * Workspace: shp_workspace_bytes(SHP_OP_APPLY, m, n, batch, opts). */
+int shampoo_apply_ex(float* W, float* M, double* gnorm2_acc, const float* G, const float* Lroot,
+                     const float* Rroot, int64_t m, int64_t n, int64_t batch, float lr,
+                     float gamma, int prec, void* ws, size_t ws_bytes, shp_stream stream);
+
 /* ---- Utilities (no counterpart on the pages; building blocks of the calls
  * above, exposed for measurement and tests). ---- */
 

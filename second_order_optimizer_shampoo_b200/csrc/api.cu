@@ -433,9 +433,12 @@ size_t shp_workspace_bytes(int opk, int64_t m, int64_t n, int64_t batch,
       break;
     }
     case SHP_OP_APPLY: {
-      // T = Lroot G (m x n); split mode also needs hi/lo copies of the inputs
+      // per-block norms and steps; T = Lroot G (m x n); split mode also
+      // needs hi/lo copies of the inputs
       const int prec = o != nullptr ? o->prec : SHP_3XTF32;
       const size_t mn = static_cast<size_t>(m) * n * batch;
+      a.take<double>(static_cast<size_t>(batch));
+      a.take<float>(static_cast<size_t>(batch));
       a.take<float>(mn);
       if (prec == SHP_3XTF32) {
         a.take<float>(mn);
@@ -500,25 +503,36 @@ int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float*
   return SHP_OK;
 }
 
-int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rroot, int64_t m,
-                  int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
-                  shp_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// W <- W - eta P (or the momentum form) with P = Lroot G Rroot; shared by
+// shampoo_apply and shampoo_apply_ex.
+int apply_impl(float* W, float* Mom, double* acc, const float* G, const float* Lroot,
+               const float* Rroot, int64_t m, int64_t n, int64_t batch, float lr, float gamma,
+               int prec, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (!W || !G || !Lroot || !Rroot || m <= 0 || n <= 0 || batch <= 0 || m % 4 || n % 4)
     return SHP_EINVAL;
   if (!aligned16(W) || !aligned16(G) || !aligned16(Lroot) || !aligned16(Rroot)) return SHP_EINVAL;
+  if ((Mom && !aligned16(Mom)) || !isfinite(lr) || !isfinite(gamma)) return SHP_EINVAL;
   if (prec != SHP_TF32 && prec != SHP_3XTF32) return SHP_EINVAL;
   if (m > INT32_MAX || n > INT32_MAX || batch > 65535) return SHP_EUNSUPPORTED;
   shp_prism_opts o{};
   o.prec = prec;
   if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_APPLY, m, n, batch, &o))
     return SHP_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
   const size_t mn = static_cast<size_t>(m) * n * batch;
   const int mode = prec == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32;
   const int fmt = prec == SHP_3XTF32 ? OUT_SPLIT : OUT_F32;
+  double* dn = a.take<double>(static_cast<size_t>(batch));
+  float* eta = a.take<float>(static_cast<size_t>(batch));
   float* Thi = a.take<float>(mn);
   float* Tlo = prec == SHP_3XTF32 ? a.take<float>(mn) : nullptr;
+  const int M = static_cast<int>(m), N = static_cast<int>(n), B = static_cast<int>(batch);
+  if (acc != nullptr)  // [Shampoo] 5.1: acc += ||G||_F^2, eta = lr / sqrt(1 + acc)
+    CK(adaptive_step(G, m * n, B, dn, acc, lr, eta, st));
   const float *Lh = Lroot, *Ll = nullptr, *Gh = G, *Gl = nullptr, *Rh = Rroot, *Rl = nullptr;
   if (prec == SHP_3XTF32) {
     const size_t mm = static_cast<size_t>(m) * m * batch, nn = static_cast<size_t>(n) * n * batch;
@@ -535,15 +549,41 @@ int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rro
     Rh = p;
     Rl = p + nn;
   }
-  const int M = static_cast<int>(m), N = static_cast<int>(n), B = static_cast<int>(batch);
   // T = Lroot G
   EpiParams e1 = epi(EPI_STORE, fmt, Thi, Tlo, n, m * n, M, N, nullptr);
   CK(gemm_tc(mode, op(Lh, Ll, false, m, m * m), op(Gh, Gl, true, n, m * n), M, N, M, B, e1, st));
-  // W <- W - lr T Rroot
-  EpiParams e2 = epi(EPI_APPLY, OUT_F32, W, nullptr, n, m * n, M, N, nullptr);
-  e2.s0 = -lr;
+  // W <- W - eta T Rroot, or M <- gamma M + T Rroot and W <- W - eta M ([Shampoo] 5.2)
+  EpiParams e2 = epi(Mom ? EPI_MOMENTUM : EPI_APPLY, OUT_F32, W, nullptr, n, m * n, M, N, nullptr);
+  e2.s0 = acc != nullptr ? -1.f : -lr;
+  e2.alpha = acc != nullptr ? eta : nullptr;
+  if (Mom != nullptr) {
+    e2.aux_hi = Mom;
+    e2.aux_fmt = OUT_F32;
+    e2.lda_aux = n;
+    e2.bs_aux = m * n;
+    e2.out2_hi = Mom;
+    e2.s1 = gamma;
+  }
   CK(gemm_tc(mode, op(Thi, Tlo, false, n, m * n), op(Rh, Rl, true, n, n * n), M, N, N, B, e2, st));
   return SHP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rroot, int64_t m,
+                  int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
+                  shp_stream stream) {
+  return apply_impl(W, nullptr, nullptr, G, Lroot, Rroot, m, n, batch, lr, 0.f, prec, ws,
+                    ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int shampoo_apply_ex(float* W, float* M, double* gnorm2_acc, const float* G, const float* Lroot,
+                     const float* Rroot, int64_t m, int64_t n, int64_t batch, float lr,
+                     float gamma, int prec, void* ws, size_t ws_bytes, shp_stream stream) {
+  return apply_impl(W, M, gnorm2_acc, G, Lroot, Rroot, m, n, batch, lr, gamma, prec, ws,
+                    ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, int p, int d,

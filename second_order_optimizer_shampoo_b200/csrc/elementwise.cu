@@ -253,6 +253,16 @@ __global__ void __launch_bounds__(EW_THREADS)
   }
 }
 
+// acc[b] += ||G_b||_F^2 (from dn, fp64), eta[b] = lr / sqrt(1 + acc[b]).
+__global__ void k_adaptive_eta(const double* dn, double* acc, float lr, float* eta, int batch) {
+  count_kernel_run();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= batch) return;
+  const double a = acc[b] + dn[b];
+  acc[b] = a;
+  eta[b] = static_cast<float>(static_cast<double>(lr) / sqrt(1.0 + a));
+}
+
 __global__ void k_write_status(Ctl ctl, int batch, int* out) {
   count_kernel_run();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -324,6 +334,15 @@ cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
                          int out_bf16, cudaStream_t st) {
   k_polar_finish<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(count, ctl, fmt, Shi[0], Slo[0],
                                                                Shi[1], Slo[1], X_out, out_bf16);
+  return cudaGetLastError();
+}
+
+cudaError_t adaptive_step(const float* G, int64_t count, int batch, double* dn, double* acc,
+                          float lr, float* eta, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(dn, 0, sizeof(double) * batch, st);
+  if (e != cudaSuccess) return e;
+  k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, 0, count, dn);
+  k_adaptive_eta<<<(batch + 127) / 128, 128, 0, st>>>(dn, acc, lr, eta, batch);
   return cudaGetLastError();
 }
 

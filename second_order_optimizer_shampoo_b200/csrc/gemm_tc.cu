@@ -89,12 +89,13 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
 template <bool DUAL, int RP>
 SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b, int m0, int n0,
                             int BN, int q, int h, int lane) {
-  const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;
+  const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;  // GPOLY
+  const float eta = ep.alpha != nullptr ? ep.alpha[b] : 1.f;    // APPLY, MOMENTUM
   const bool diag_tile = (m0 < n0 + BN) && (n0 < m0 + 128);
   const int row0 = m0 + q * 32;
   const int rcount = ep.M - row0 < 32 ? ep.M - row0 : 32;
-  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY;
-  const bool need_old = ep.kind == EPI_EMA || ep.kind == EPI_APPLY;
+  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;
+  const bool need_old = ep.kind == EPI_EMA || ep.kind == EPI_APPLY || ep.kind == EPI_MOMENTUM;
   const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
   float nrm = 0.f;
   for (int c = h; c < BN / 32; c += 2) {
@@ -119,7 +120,7 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
         static_cast<int64_t>(b) * ep.bs_aux + static_cast<int64_t>(row0) * ep.lda_aux + gj;
 #pragma unroll 1
     for (int r0 = 0; r0 < 32; r0 += RP) {
-      float a[RP], x[RP];
+      float a[RP], x[RP], w[RP];
 #pragma unroll
       for (int r = 0; r < RP; ++r) a[r] = st[(r0 + r) * 33 + lane];
       if (colok) {
@@ -154,16 +155,20 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
               for (int r = 0; r < RP; ++r) x[r] += y[r];
             }
           }
-        } else if (need_old) {
+        } else {
+#pragma unroll
+          for (int r = 0; r < RP; ++r) x[r] = 0.f;
+        }
+        if (need_old) {
           const float* p = static_cast<const float*>(ep.out_hi) + obase;
 #pragma unroll
           for (int r = 0; r < RP; ++r) {
             const int rr = r0 + r < rcount ? r0 + r : rcount - 1;
-            x[r] = p[static_cast<int64_t>(rr) * ep.ldo];
+            w[r] = p[static_cast<int64_t>(rr) * ep.ldo];
           }
         } else {
 #pragma unroll
-          for (int r = 0; r < RP; ++r) x[r] = 0.f;
+          for (int r = 0; r < RP; ++r) w[r] = 0.f;
         }
 #pragma unroll
         for (int r = 0; r < RP; ++r) {
@@ -172,7 +177,7 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
           const float acc = a[r];
           const float eye = (diag_tile && gi == gj) ? 1.f : 0.f;
           const int64_t off = obase + static_cast<int64_t>(r0 + r) * ep.ldo;
-          float val;
+          float val, val2 = -1.f;
           switch (ep.kind) {
             case EPI_RESID:
               val = eye - acc;
@@ -185,17 +190,23 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
               val = x[r] + ep.s0 * acc;
               break;
             case EPI_EMA:
-              val = ep.s0 * x[r] + ep.s1 * acc + ep.s2 * eye;
+              val = ep.s0 * w[r] + ep.s1 * acc + ep.s2 * eye;
               break;
             case EPI_APPLY:
-              val = x[r] + ep.s0 * acc;
+              val = w[r] + ep.s0 * eta * acc;
+              break;
+            case EPI_MOMENTUM:
+              val2 = ep.s1 * x[r] + acc;
+              val = w[r] + ep.s0 * eta * val2;
               break;
             default:
               val = ep.s0 * acc;
               break;
           }
           put(ep.out_fmt, ep.out_hi, ep.out_lo, off, val);
-          if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, val + eye);
+          if (ep.out2_hi != nullptr)
+            put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off,
+                ep.kind == EPI_MOMENTUM ? val2 : val + eye);
           if (ep.out_plain != nullptr) ep.out_plain[off] = val;
         }
       }

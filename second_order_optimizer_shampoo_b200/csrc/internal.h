@@ -22,7 +22,8 @@ enum EpiKind {
   EPI_GPOLY = 2,
   EPI_EMA = 3,
   EPI_APPLY = 4,
-  EPI_AXPY = 5
+  EPI_AXPY = 5,
+  EPI_MOMENTUM = 6
 };
 enum OutFmt { OUT_F32 = 0, OUT_SPLIT = 1, OUT_BF16 = 2 };
 
@@ -50,8 +51,10 @@ struct Operand {
 //   RESID: v = [i==j] - acc, and norm2[b] += v^2
 //   GPOLY: v = s1 * aux(i,j) + alpha[b] * acc   (Delta = g - I; out2 gets I + Delta)
 //   EMA:   v = s0 * out(i,j) + s1 * acc + s2 * [i==j]   (read-modify-write)
-//   APPLY: v = out(i,j) + s0 * acc                       (read-modify-write)
+//   APPLY: v = out(i,j) + s0 * eta[b] * acc              (read-modify-write)
 //   AXPY:  v = aux(i,j) + s0 * acc                       (X + X Delta)
+//   MOMENTUM: m = s1 * aux(i,j) + acc, v = out(i,j) + s0 * eta[b] * m; out2 gets m
+// (eta[b] = alpha[b] when alpha is non-null, else 1).
 // v is written to `out` (and to `out2` when non-null) in `out_fmt`.  The
 // update polynomial is kept as Delta = g - I and applied as X + X Delta so
 // that its small part keeps full relative precision in every storage format
@@ -164,6 +167,10 @@ cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, cons
 cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
                          const void* const* Shi, const float* const* Slo, void* X_out,
                          int out_bf16, cudaStream_t st);
+// Adaptive step of the update ([Shampoo] 5.1): acc[b] += ||G_b||_F^2 (G fp32,
+// count elements per block; dn is [batch] fp64 scratch), eta[b] = lr / sqrt(1 + acc[b]).
+cudaError_t adaptive_step(const float* G, int64_t count, int batch, double* dn, double* acc,
+                          float lr, float* eta, cudaStream_t st);
 // report.status[b] = ETIMEOUT if flagged, else bs[b].status.
 cudaError_t write_status(const Ctl& ctl, int batch, int* report_status, cudaStream_t st);
 

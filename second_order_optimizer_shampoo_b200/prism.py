@@ -93,6 +93,24 @@ def shampoo_apply(W, G, Lroot, Rroot, lr: float, prec: str = "tf32", ws=None):
                                  _p(ws), ws.numel(), _stream()), "shampoo_apply")
 
 
+def shampoo_apply_ex(W, G, Lroot, Rroot, lr: float, prec: str = "tf32", M=None, gamma=0.0,
+                     gnorm2_acc=None, ws=None):
+    """Update variants (in place): with gnorm2_acc (float64 [batch]) the step is
+    lr / sqrt(1 + acc) after acc += ||G||_F^2; with M (momentum buffer)
+    M <- gamma M + P and W <- W - eta M; P = Lroot G Rroot."""
+    _dev(W, G, Lroot, Rroot, M, gnorm2_acc)
+    if gnorm2_acc is not None and gnorm2_acc.dtype != torch.float64:
+        raise ValueError("gnorm2_acc must be float64")
+    m, n = W.shape[-2], W.shape[-1]
+    batch = W.numel() // (m * n)
+    o = make_opts(prec=prec)
+    need = shp_workspace_bytes(A.SHP_OP_APPLY, m, n, batch, o)
+    ws = _ws(need, W.device) if ws is None else ws
+    _check(A.lib().shampoo_apply_ex(_p(W), _p(M), _p(gnorm2_acc), _p(G), _p(Lroot), _p(Rroot),
+                                    m, n, batch, lr, gamma, _PREC[prec], _p(ws), ws.numel(),
+                                    _stream()), "shampoo_apply_ex")
+
+
 def _report(batch, max_iter, device):
     return {
         "status": torch.full((batch,), -1, dtype=torch.int32, device=device),

@@ -99,6 +99,23 @@ def test_invalid_arguments_rejected_before_launch():
                            None) == A.SHP_EINVAL
 
 
+def test_apply_ex_validation():
+    L = A.lib()
+    fake = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10004)
+    # misaligned momentum buffer
+    assert L.shampoo_apply_ex(fake, mis, None, fake, fake, fake, 64, 64, 1, 1e-3, 0.9,
+                              A.SHP_TF32, fake, 1 << 30, None) == A.SHP_EINVAL
+    # non-finite step or momentum factor
+    assert L.shampoo_apply_ex(fake, None, None, fake, fake, fake, 64, 64, 1, float("nan"), 0.9,
+                              A.SHP_TF32, fake, 1 << 30, None) == A.SHP_EINVAL
+    assert L.shampoo_apply_ex(fake, fake, fake, fake, fake, fake, 64, 64, 1, 1e-3,
+                              float("inf"), A.SHP_TF32, fake, 1 << 30, None) == A.SHP_EINVAL
+    # workspace too small
+    assert L.shampoo_apply_ex(fake, None, fake, fake, fake, fake, 64, 64, 1, 1e-3, 0.0,
+                              A.SHP_TF32, fake, 8, None) == A.SHP_EINVAL
+
+
 def test_binding_refuses_cpu_tensors():
     torch = pytest.importorskip("torch")
     from second_order_optimizer_shampoo_b200 import prism

@@ -61,6 +61,54 @@ def test_apply(prec, m, n, batch):
         assert np.all(np.abs(Wg[b] - Wr) <= bound), np.max(np.abs(Wg[b] - Wr) / bound)
 
 
+@pytest.mark.parametrize("variant", ["momentum", "adaptive", "both"])
+@pytest.mark.parametrize("prec", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("m,n,batch", [(256, 512, 2), (300, 196, 1)])
+def test_apply_variants(variant, prec, m, n, batch):
+    """Three steps of shampoo_apply_ex against the oracle's update variants
+    ([Shampoo] 5.1-5.2): W, the momentum buffer and the running sum of squared
+    gradient norms, each within the forward-error bound accumulated over the
+    steps (the per-step bound of test_apply on P, carried through
+    M = gamma M + P and W -= eta M)."""
+    P = prism()
+    lr, gamma = 0.05, 0.9
+    use_m, use_acc = variant in ("momentum", "both"), variant in ("adaptive", "both")
+    W = synth.gaussian((batch, m, n), 0.02, 61)
+    PL = synth.gaussian((batch, m, m), 0.1, 62)
+    PR = synth.gaussian((batch, n, n), 0.1, 63)
+    Gs = [synth.gaussian((batch, m, n), 0.02, 64, index=t) for t in range(3)]
+    Wd, PLd, PRd = to_dev(torch, W), to_dev(torch, PL), to_dev(torch, PR)
+    Md = torch.zeros_like(Wd) if use_m else None
+    accd = torch.full((batch,), 0.25, dtype=torch.float64, device="cuda") if use_acc else None
+    for G in Gs:
+        P.shampoo_apply_ex(Wd, to_dev(torch, G), PLd, PRd, lr, prec, M=Md, gamma=gamma,
+                           gnorm2_acc=accd)
+    Wg = to_host(Wd)
+    for b in range(batch):
+        Wr, Mr, accr = W[b].astype(np.float64), (np.zeros((m, n)) if use_m else None), \
+            (0.25 if use_acc else None)
+        aL, aR = np.abs(PL[b].astype(np.float64)), np.abs(PR[b].astype(np.float64))
+        eW, eM = 2 * U_FP32 * np.abs(Wr), np.zeros((m, n))
+        for G in Gs:
+            Wr, Mr, accr = o.apply_variant_ref(Wr, G[b], PL[b], PR[b], lr, M=Mr, gamma=gamma,
+                                               acc=accr)
+            aG = np.abs(G[b].astype(np.float64))
+            eP = gemm_bound(aL, aG, m, prec) @ aR + gemm_bound(aL @ aG, aR, n, prec)
+            eta = lr / np.sqrt(1 + accr) if use_acc else lr
+            step = np.abs(Mr) if use_m else np.abs(o.apply_ref(0 * Wr, G[b], PL[b], PR[b], -1.0))
+            if use_m:
+                eM = gamma * eM + eP + 2 * U_FP32 * np.abs(Mr)
+                eW = eW + eta * (eM + 2 * U_FP32 * step) + 2 * U_FP32 * np.abs(Wr)
+            else:
+                eW = eW + eta * (eP + 2 * U_FP32 * step) + 2 * U_FP32 * np.abs(Wr)
+        assert np.all(np.abs(Wg[b] - Wr) <= eW), np.max(np.abs(Wg[b] - Wr) / eW)
+        if use_m:
+            Mg = to_host(Md)[b]
+            assert np.all(np.abs(Mg - Mr) <= eM), np.max(np.abs(Mg - Mr) / eM)
+        if use_acc:
+            assert to_host(accd)[b] == pytest.approx(accr, rel=1e-12)
+
+
 def residual_like(n, batch, seed, lo=0.0, hi=0.8):
     """Symmetric matrices with spectrum in [lo, hi] (a residual R_k mid-iteration)."""
     out = np.empty((batch, n, n), dtype=np.float32)
