@@ -45,7 +45,7 @@ GEMM_TRAFFIC_PER_LAUNCH = 4 * (289.454e6 + 41.826e6)
 
 def workload_config(world):
     return {
-        "workload": "inv4_root_64x1024sq_spd_cond1e6_prism_d2_p8",
+        "workload": f"inv4_root_{BATCH}x1024sq_spd_cond1e6_prism_d2_p8",
         "n": N, "batch_per_gpu": BATCH, "d": D, "p": P, "tol": TOL, "max_iter": MAX_ITER,
         "alpha_interval": [0.375, 1.0], "prec": "3xtf32", "lambda": "log-uniform [1e-6, 1]",
         "l2": "inputs larger than L2 (256 MiB of A plus 3.2 GB of iterates per GPU per step)",
@@ -399,6 +399,43 @@ def single_block_leg(args, dev, stream):
             "iters_polar": int(repp["iters"].cpu().numpy()[0][0])}
 
 
+def large_sqrt_leg(args, dev, stream):
+    """A^(1/2) of one 10240 x 10240 Marchenko-Pastur matrix (A = X X^T / 20480 +
+    1e-4 I), PRISM d = 2, p = 16, tol 1e-6, split path; GEMMs to the residual
+    against the fixed-coefficient iterations d = 2 and d = 1."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import _abi, prism, synth
+    n, mi = 10240, 40
+    A = torch.from_numpy(synth.mp_spd(n, 2 * n, 1e-4, 105)[None]).to(dev)
+    S = torch.from_numpy(synth.sketch_stack(mi, n, 16, 1005)).to(dev)
+    out = {"workload": "sqrt_10240sq_marchenko_pastur_prism_d2_p16_tol1e-6_3xtf32"}
+    for name, d, fixed in (("prism_d2", 2, False), ("taylor_d2", 2, True),
+                           ("taylor_d1", 1, True)):
+        opts = prism.make_opts(d=d, p=16, tol=1e-6, max_iter=mi, prec="3xtf32",
+                               fixed_alpha=fixed)
+        ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, n, n, 1, opts),
+                         dtype=torch.uint8, device=dev)
+        X = torch.empty_like(A)
+        rep = prism.make_report(1, mi, dev)
+
+        def call():
+            prism.matfn_inv_root(A, "sqrt", opts, S, out=X, ws=ws, report=rep)
+
+        call()
+        torch.cuda.synchronize()
+        k = int(rep["iters"].cpu().numpy()[0][0])
+        gemms = max((3 if d == 1 else 4) * k - 1, 0)
+        entry = {"iters": k, "gemms": gemms, "status": int(rep["status"].cpu().numpy()[0])}
+        if name == "prism_d2":
+            ms = _time(call, stream, 3)
+            tf = gemms * 2.0 * n ** 3 / (ms / 1e3) / 1e12
+            entry.update({"ms": ms, "value": tf, "unit": "TFLOP/s"})
+        out[name] = entry
+        del ws
+    return out
+
+
 PM, PN, PBATCH, PRANK = 4096, 1024, 96, 64
 
 
@@ -454,6 +491,7 @@ def polar_leg(args, dev, stream):
 
 # ------------------------------------------------------------------ our leg
 def main():
+    global BATCH
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -462,11 +500,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-polar", action="store_true", help="skip the polar-factor leg")
     ap.add_argument("--no-small", action="store_true", help="skip the small-block leg")
+    ap.add_argument("--large", action="store_true",
+                    help="add the 10240^2 square-root leg (builds a 10240 x 20480 product "
+                         "on the host first)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the Shampoo-step, GEMM-count and single-block legs")
-    ap.add_argument("--kernel", default=None, choices=["gemm", "small"],
-                    help="run only the batched 3xTF32 GEMM or the small-block kernel "
-                         "(for profiling; --batch sets the batch)")
+    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar"],
+                    help="run only the batched 3xTF32 GEMM, the small-block kernel or the "
+                         "polar leg (for profiling; --batch sets the GEMM/small batch)")
     ap.add_argument("--batch", type=int, default=BATCH)
     args = ap.parse_args()
     if args.impl == "reference":
@@ -475,6 +516,11 @@ def main():
         return gemm_only(args)
     if args.kernel == "small":
         return small_only(args)
+    if args.kernel == "polar":
+        import torch
+        print(json.dumps(polar_leg(args, torch.device("cuda", 0), torch.cuda.current_stream())))
+        return 0
+    BATCH = args.batch  # blocks per GPU of the main workload (64 unless profiling)
 
     import numpy as np
     import torch
@@ -491,7 +537,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    # ---- inputs: each rank its own 64 blocks (seeded by global block index)
+    # ---- inputs: each rank its own BATCH blocks (seeded by global block index)
     idx = list(range(rank * BATCH, (rank + 1) * BATCH))
     A_np = synth.spd_batch(N, BATCH, LAM_LO, 1.0, SEED_A, indices=idx)
     S_np = synth.sketch_stack(2 * MAX_ITER, N, P, SEED_S)
@@ -606,6 +652,7 @@ def main():
     step2 = shampoo_step_leg(args, dev, stream) if extra else None
     counts = gemm_count_leg(args, dev, stream, A) if extra else None
     single = single_block_leg(args, dev, stream) if extra else None
+    large = large_sqrt_leg(args, dev, stream) if args.large and world == 1 else None
     small = None if args.no_small else small_block_leg(args, dev, stream,
                                                         peaks.get("sm_max_mhz", 1965.0))
 
@@ -621,7 +668,7 @@ def main():
                 break
         cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
                "kind": "oracle",
-               "sample": f"{nb} of the 64 blocks, float64 NumPy/LAPACK oracle (same recurrence)"}
+               "sample": f"{nb} of the {BATCH} blocks, float64 NumPy/LAPACK oracle (same recurrence)"}
 
     if rank == 0:
         line = {
@@ -642,6 +689,7 @@ def main():
             "shampoo_step_1024": step2,
             "gemms_to_residual": counts,
             "single_64": single,
+            "sqrt_10240": large,
             "cpu_baseline": cpu,
             "clocks": clocks,
         }

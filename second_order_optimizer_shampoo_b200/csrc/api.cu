@@ -175,11 +175,6 @@ int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass,
                      int64_t rep_stride, int rep_slot_base, cudaStream_t st) {
   const int64_t np = n * o->p, nn = n * n;
   const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
-  if (!o->fixed_alpha && sketch_chain_ok(n, o->p)) {  // one launch, R re-read from L2
-    CK(sketch_chain(Rs, n, batch, S_pass, ctl.it, o->p, o->d, o->lo, o->hi, ctl.active,
-                    ctl.alpha, rep_alpha, rep_stride, rep_slot_base, st));
-    return SHP_OK;
-  }
   if (!o->fixed_alpha) {
     CK(sketch_pass(Rs, nullptr, n, nn, S_pass, 0, V + np, vbs, o->p, batch, ctl.active, ctl.it,
                    np, st));
@@ -347,8 +342,6 @@ int run_graph(CallKey key, Rec rec, cudaStream_t user) {
 // else through the graph cache.
 template <class Rec>
 int dispatch(const CallKey& key, Rec rec, cudaStream_t user) {
-  // host-side setup of kernels the recorder may launch, outside any capture
-  if (sketch_chain_prepare() != cudaSuccess) return SHP_ECUDA;
   if (getenv("SHP_HOST_LOOP") != nullptr) {
     cudaStream_t cs[3] = {user, user, user};
     return rec(static_cast<cudaStream_t const*>(cs), static_cast<cudaGraph_t>(nullptr));

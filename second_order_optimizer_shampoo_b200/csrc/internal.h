@@ -103,18 +103,6 @@ cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, floa
                         float* report_alpha, int64_t report_stride, int report_slot,
                         const int* it, cudaStream_t st);
 
-// Sketch chain and alpha fit of every active block in one launch (one
-// thread-block cluster per block, V_j exchanged through distributed shared
-// memory): alpha[b] and report[b * stride + slot + *it] as alpha_solve.
-// R: plain fp32 [batch][n][n]; S: the pass's slices [.][n][p], slice *it used.
-bool sketch_chain_ok(int64_t n, int p);
-// Host-side setup (kernel attributes, resident-cluster count); call before
-// capturing a graph that launches sketch_chain.
-cudaError_t sketch_chain_prepare();
-cudaError_t sketch_chain(const float* R, int64_t n, int batch, const float* S, const int* it,
-                         int p, int d, float lo, float hi, const int* active, float* alpha,
-                         float* rep, int64_t rep_stride, int rep_slot, cudaStream_t st);
-
 // ---- per-block control (sketch_alpha.cu)
 struct BlockState {
   float norm2;     // ||R_k||_F^2 accumulated by the residual epilogue

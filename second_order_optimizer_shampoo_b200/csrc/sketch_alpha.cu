@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(AL_THREADS)
     if (lane == 0) red[warp][i] = s;
   }
   __syncthreads();
-  if (threadIdx.x != 0) return;
+  if (threadIdx.x >= 32) return;  // warp 0 forms J and finds its minimiser
   double M[4][4];
   {
     int idx = 0;
@@ -158,178 +158,12 @@ __global__ void __launch_bounds__(AL_THREADS)
   }
   double coef[5];
   quartic_from_gram(M, d, coef);
-  const double a = argmin_quartic(coef, static_cast<double>(lo), static_cast<double>(hi));
+  const double a = argmin_quartic_warp(coef, static_cast<double>(lo), static_cast<double>(hi));
+  if (threadIdx.x != 0) return;
   alpha[b] = static_cast<float>(a);
   if (Jc != nullptr)
     for (int i = 0; i < 5; ++i) Jc[b * 5 + i] = coef[i];
   if (rep != nullptr) rep[b * rep_stride + rep_slot] = static_cast<float>(a);
-}
-
-// ------------------------------------------------------------------------
-// The whole sketch chain and alpha fit of one block in one cluster.
-//
-// Eight CTAs (one thread-block cluster) own one block at a time and loop over
-// the batch.  CTA r computes rows [r n/8, (r+1) n/8) of every V_j = R V_{j-1},
-// j = 1..2d+1, and writes them into the V_j buffer of all eight CTAs through
-// distributed shared memory; one cluster barrier per power makes V_j whole
-// everywhere.  Only 8 x (the resident clusters) blocks' R (4 MB each at
-// n = 1024) are live at a time, so the 2d+1 reads of R after the first come
-// from L2.  The fp64 Gram of V_d..V_{2d+1} is reduced over the cluster into
-// the leader CTA, whose thread 0 forms the quartic and takes its argmin: the
-// same arithmetic as k_sketch + k_alpha, with one launch instead of 2d+2.
-constexpr int SC_CS = 8;
-constexpr int SC_THREADS = 512;
-constexpr int SC_WARPS = SC_THREADS / 32;
-constexpr int SC_VFLOATS = 8192;  // n * P per V buffer (32 KB)
-// 2 V buffers + own rows of d+2 powers; padded so that one CTA fits per SM
-constexpr int SC_SMEM = 120 * 1024;
-static_assert((2 * SC_VFLOATS + 4 * (SC_VFLOATS / SC_CS)) * 4 <= SC_SMEM, "sketch chain smem");
-
-SHP_DEV void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-SHP_DEV void st_cluster_f64(uint32_t addr, double v) {
-  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
-}
-
-template <int P>
-__global__ void __launch_bounds__(SC_THREADS, 1)
-    k_sketch_chain(const float* __restrict__ R, int n, int batch, const float* __restrict__ S,
-                   const int* __restrict__ it, int p, int d, float lo, float hi,
-                   const int* __restrict__ active, float* __restrict__ alpha,
-                   float* __restrict__ rep, int64_t rep_stride, int rep_slot) {
-  count_kernel_run();
-  extern __shared__ __align__(16) float sc_sm[];
-  __shared__ double gpart[SC_WARPS][10];
-  __shared__ double gclu[SC_CS][10];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t crank = cluster_rank();
-  const int cl = static_cast<int>(blockIdx.x) / SC_CS, ncl = static_cast<int>(gridDim.x) / SC_CS;
-  const int rows = (n + SC_CS - 1) / SC_CS;
-  const int r_begin = static_cast<int>(crank) * rows;
-  const int r_end = r_begin + rows < n ? r_begin + rows : n;
-  const int nv = d + 2;
-  const int k = it != nullptr ? *it : 0;
-  const float* Sk = S + static_cast<int64_t>(k) * n * p;
-  float* Vown = sc_sm + 2 * P * n;  // [nv][rows][P]
-
-  for (int b = cl; b < batch; b += ncl) {
-    if (active != nullptr && active[b] == 0) continue;  // uniform over the cluster
-    float* Vc = sc_sm;          // V_{j-1}, transposed [P][n]
-    float* Vn = sc_sm + P * n;  // V_j
-    for (int idx = tid; idx < P * n; idx += SC_THREADS) {
-      const int j = idx / n, col = idx - j * n;
-      Vc[idx] = j < p ? Sk[static_cast<int64_t>(col) * p + j] : 0.f;
-    }
-    __syncthreads();
-    const float* Rb = R + static_cast<int64_t>(b) * n * n;
-    for (int jp = 1; jp <= 2 * d + 1; ++jp) {
-      // two rows per warp step; each lane takes 4 consecutive columns of
-      // every 128-column stripe, four stripes in flight
-      for (int row = r_begin + 2 * warp; row < r_end; row += 2 * SC_WARPS) {
-        const bool two = row + 1 < r_end;
-        const float* r0p = Rb + static_cast<int64_t>(row) * n;
-        const float* r1p = two ? r0p + n : r0p;
-        float acc0[P], acc1[P];
-#pragma unroll
-        for (int j = 0; j < P; ++j) acc0[j] = acc1[j] = 0.f;
-        for (int c0 = lane * 4; c0 < n; c0 += 512) {
-          float4 x0[4], x1[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int c = c0 + 128 * t;
-            x0[t] = c < n ? *reinterpret_cast<const float4*>(r0p + c) : make_float4(0, 0, 0, 0);
-            x1[t] = c < n ? *reinterpret_cast<const float4*>(r1p + c) : make_float4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int c = c0 + 128 * t;
-            if (c >= n) break;
-#pragma unroll
-            for (int j = 0; j < P; ++j) {
-              const float4 v = *reinterpret_cast<const float4*>(Vc + j * n + c);
-              acc0[j] = fmaf(x0[t].x, v.x, fmaf(x0[t].y, v.y, fmaf(x0[t].z, v.z,
-                        fmaf(x0[t].w, v.w, acc0[j]))));
-              acc1[j] = fmaf(x1[t].x, v.x, fmaf(x1[t].y, v.y, fmaf(x1[t].z, v.z,
-                        fmaf(x1[t].w, v.w, acc1[j]))));
-            }
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < P; ++j) {
-          acc0[j] = warp_sum(acc0[j]);
-          acc1[j] = warp_sum(acc1[j]);
-        }
-        // lane q < 8 stores both rows' P values into CTA q's V_j; lane 8 + j
-        // keeps column j of the rows this CTA owns (powers d..2d+1)
-        if (lane < SC_CS) {
-          const uint32_t base = mapa_shared(smem_u32(Vn), static_cast<uint32_t>(lane));
-#pragma unroll
-          for (int j = 0; j < P; ++j) {
-            st_cluster_f32(base + static_cast<uint32_t>((j * n + row) * 4), acc0[j]);
-            if (two) st_cluster_f32(base + static_cast<uint32_t>((j * n + row + 1) * 4), acc1[j]);
-          }
-        } else if (jp >= d && lane < SC_CS + P) {
-          const int j = lane - SC_CS;
-          float* o = Vown + (static_cast<int64_t>(jp - d) * rows + (row - r_begin)) * P;
-          float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < P; ++jj) {
-            if (jj == j) {
-              v0 = acc0[jj];
-              v1 = acc1[jj];
-            }
-          }
-          o[j] = v0;
-          if (two) o[P + j] = v1;
-        }
-      }
-      cluster_sync();  // V_j complete in every CTA of the cluster
-      float* t = Vc;
-      Vc = Vn;
-      Vn = t;
-    }
-    // fp64 Gram of the owned rows of V_d .. V_{2d+1}, reduced into the leader
-    double part[10];
-#pragma unroll
-    for (int i = 0; i < 10; ++i) part[i] = 0.0;
-    const int cnt = (r_end - r_begin) * P;
-    for (int e = tid; e < cnt; e += SC_THREADS) {
-      double x[4];
-      for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(Vown[static_cast<int64_t>(i) * rows * P + e]);
-      int idx = 0;
-      for (int i = 0; i < nv; ++i)
-        for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
-    }
-#pragma unroll
-    for (int i = 0; i < 10; ++i) {
-      const double v = warp_sum(part[i]);
-      if (lane == 0) gpart[warp][i] = v;
-    }
-    __syncthreads();
-    if (tid < 10) {
-      double v = 0.0;
-      for (int w = 0; w < SC_WARPS; ++w) v += gpart[w][tid];
-      st_cluster_f64(mapa_shared(smem_u32(&gclu[crank][tid]), 0), v);
-    }
-    cluster_sync();  // partials in the leader; V buffers free for the next block
-    if (crank == 0 && tid == 0) {
-      double M[4][4];
-      int idx = 0;
-      for (int i = 0; i < nv; ++i)
-        for (int j = i; j < nv; ++j) {
-          double v = 0.0;
-          for (int q = 0; q < SC_CS; ++q) v += gclu[q][idx];
-          M[i][j] = M[j][i] = v;
-          ++idx;
-        }
-      double coef[5];
-      quartic_from_gram(M, d, coef);
-      const double a = argmin_quartic(coef, static_cast<double>(lo), static_cast<double>(hi));
-      alpha[b] = static_cast<float>(a);
-      if (rep != nullptr) rep[b * rep_stride + rep_slot + k] = static_cast<float>(a);
-    }
-  }
 }
 
 __global__ void k_control(BlockState* bs, int* active, const int* it, int batch, int64_t n,
@@ -424,89 +258,6 @@ cudaError_t loop_step(const Ctl& ctl, int batch, int inc, int max_iter,
                       cudaGraphConditionalHandle h, cudaStream_t st) {
   k_loop_step<<<1, 256, 0, st>>>(ctl.active, ctl.it, ctl.flag, batch, inc, max_iter, h);
   return cudaGetLastError();
-}
-
-bool sketch_chain_ok(int64_t n, int p) {
-  const int P = p <= 4 ? 4 : (p <= 8 ? 8 : 16);
-  return p <= 16 && n >= 64 && n * P <= SC_VFLOATS;
-}
-
-namespace {
-constexpr int kMaxDev = 64;
-int g_chain_clusters[kMaxDev] = {0};  // resident clusters per device (0 = not queried)
-
-template <int P>
-void chain_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, cudaStream_t st) {
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = SC_CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg->blockDim = dim3(SC_THREADS, 1, 1);
-  cfg->dynamicSmemBytes = SC_SMEM;
-  cfg->stream = st;
-  cfg->attrs = attr;
-  cfg->numAttrs = 1;
-}
-
-template <int P>
-cudaError_t prepare_chain(int dev) {
-  auto kern = k_sketch_chain<P>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC_SMEM);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  chain_config<P>(&cfg, attr, nullptr);
-  cfg.gridDim = dim3(SC_CS * 148, 1, 1);
-  int mc = 0;
-  e = cudaOccupancyMaxActiveClusters(&mc, kern, &cfg);
-  if (e != cudaSuccess) return e;
-  // every p bucket has the same footprint: keep the smallest answer
-  if (g_chain_clusters[dev] == 0 || mc < g_chain_clusters[dev]) g_chain_clusters[dev] = mc < 1 ? 1 : mc;
-  return cudaSuccess;
-}
-
-template <int P>
-cudaError_t launch_chain(const float* R, int n, int batch, const float* S, const int* it, int p,
-                         int d, float lo, float hi, const int* active, float* alpha,
-                         float* rep, int64_t rep_stride, int rep_slot, cudaStream_t st) {
-  auto kern = k_sketch_chain<P>;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  chain_config<P>(&cfg, attr, st);
-  const int mc = dev < kMaxDev && g_chain_clusters[dev] > 0 ? g_chain_clusters[dev] : 1;
-  cfg.gridDim = dim3(SC_CS * (batch < mc ? batch : mc), 1, 1);
-  return cudaLaunchKernelEx(&cfg, kern, R, n, batch, S, it, p, d, lo, hi, active, alpha, rep,
-                            rep_stride, rep_slot);
-}
-}  // namespace
-
-cudaError_t sketch_chain_prepare() {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev >= kMaxDev) return e;
-  if (g_chain_clusters[dev] > 0) return cudaSuccess;
-  e = prepare_chain<4>(dev);
-  if (e == cudaSuccess) e = prepare_chain<8>(dev);
-  if (e == cudaSuccess) e = prepare_chain<16>(dev);
-  return e;
-}
-
-cudaError_t sketch_chain(const float* R, int64_t n, int batch, const float* S, const int* it,
-                         int p, int d, float lo, float hi, const int* active, float* alpha,
-                         float* rep, int64_t rep_stride, int rep_slot, cudaStream_t st) {
-  if (batch <= 0) return cudaSuccess;
-  const int N = static_cast<int>(n);
-  if (p <= 4)
-    return launch_chain<4>(R, N, batch, S, it, p, d, lo, hi, active, alpha, rep, rep_stride,
-                           rep_slot, st);
-  if (p <= 8)
-    return launch_chain<8>(R, N, batch, S, it, p, d, lo, hi, active, alpha, rep, rep_stride,
-                           rep_slot, st);
-  return launch_chain<16>(R, N, batch, S, it, p, d, lo, hi, active, alpha, rep, rep_stride,
-                          rep_slot, st);
 }
 
 uint64_t kernel_runs_sketch() {

@@ -210,7 +210,7 @@ SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float
     if (lane == 0) red[warp][i] = s;
   }
   __syncthreads();
-  if (tid == 0) {
+  if (tid < 32) {  // warp 0: every lane forms J, the warp finds its minimiser
     double M[4][4];
     int idx = 0;
     for (int i = 0; i < nv; ++i)
@@ -222,8 +222,9 @@ SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float
       }
     double coef[5];
     quartic_from_gram(M, d, coef);
-    *s_alpha = static_cast<float>(
-        argmin_quartic(coef, static_cast<double>(o.lo), static_cast<double>(o.hi)));
+    const double a =
+        argmin_quartic_warp(coef, static_cast<double>(o.lo), static_cast<double>(o.hi));
+    if (tid == 0) *s_alpha = static_cast<float>(a);
   }
   __syncthreads();
   return *s_alpha;
