@@ -12,7 +12,7 @@ docstring by page title and section:
   (algorithm.idocdown.com), sections 2.2, 2.3, 3.1, 5.1, 5.2, 6.3.
 * [PRISM-it] "Sintesi Tecnica: PRISM" (gist.science), "Parte I" and
   "Parte II" (residual-form iteration, adaptive polynomial, alpha fit,
-  clamp, randomized sketch).
+  clamp, randomized sketch; R_k = I - X_k^2 for sign functions).
 * [PRISM-zh] "PRISM：分布无关的自适应矩阵函数计算" (euno.news), "方法论".
 
 Readings taken where the pages are silent (each is listed in the design doc):
@@ -369,6 +369,37 @@ def polar_ref(G, opts: PrismOpts, S, force_iters=None):
     return (X.T if wide else X), [info]
 
 
+def sign_ref(A, opts: PrismOpts, S, force_iters=None):
+    """Matrix sign function of a symmetric A by PRISM Newton-Schulz, the
+    residual R_k = I - X_k^2 that [PRISM-it] Parte I names for sign functions:
+    X_0 = A / ||A||_F; for k = 0, 1, ...: R_k = I - X_k X_k; stop test;
+    alpha_k from S[k]; X_{k+1} = X_k g_d(R_k; alpha_k).  The scalar map is
+    x -> x (1 - (1 - x^2))^(-1/2) = sign(x), so the same Taylor family and
+    alpha objective apply as for the polar factor."""
+    A = _f64(A)
+    n = A.shape[0]
+    I = np.eye(n)
+    X = A / np.linalg.norm(A)
+    info = PassInfo()
+    k = 0
+    while True:
+        Rk = I - X @ X
+        rk = float(np.linalg.norm(Rk) / sqrt(n))
+        info.res.append(rk)
+        if _stop(info, rk, k, opts, force_iters):
+            break
+        if opts.fixed_alpha:
+            a, coef = float(opts.lo), np.full(5, np.nan)
+        else:
+            a, coef = prism_alpha_ref(Rk, S[k], opts.d, opts.lo, opts.hi)
+        info.alpha.append(a)
+        info.J_coef.append(coef)
+        X = X @ matrix_poly(g_coeffs(opts.d, a), Rk)
+        k += 1
+    info.iters = k
+    return X, [info]
+
+
 # ---------------------------------------------------------------------------
 # Exact references  ([Shampoo] §3.1: eigendecomposition; SVD for the polar factor)
 # ---------------------------------------------------------------------------
@@ -377,6 +408,12 @@ def spd_power_eigh(A, q):
     """A^q = Q diag(lambda^q) Q^T from a symmetric eigendecomposition."""
     w, Q = np.linalg.eigh(_f64(A))
     return (Q * w[None, :] ** q) @ Q.T
+
+
+def sign_eigh(A):
+    """sign(A) = Q diag(sign(lambda)) Q^T from a symmetric eigendecomposition."""
+    w, Q = np.linalg.eigh(_f64(A))
+    return (Q * np.sign(w)[None, :]) @ Q.T
 
 
 def polar_svd(G):

@@ -327,6 +327,53 @@ def test_polar_textbook_and_singular_value_recurrence():
     np.testing.assert_allclose(X, want, atol=1e-15)
 
 
+# ---------------------------------------------------------------- sign
+def test_sign_of_indefinite_matches_eigh():
+    """sign(A) of a symmetric indefinite matrix: involutory (X^2 = I), commutes
+    with A, and equals Q sign(Lambda) Q^T."""
+    rng = np.random.default_rng(31)
+    Q = rot(12, 7)
+    lam = np.array([3.0, -2.0, 0.5, -0.1, 1.0, -1.0, 0.05, -4.0, 2.5, -0.3, 0.7, -0.02])
+    A = (Q * lam) @ Q.T
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=80, stall_below=0.0)
+    X, infos = o.sign_ref(A, opts, rng.standard_normal((100, 12, 4)))
+    assert infos[0].status == o.OK
+    np.testing.assert_allclose(X @ X, np.eye(12), atol=1e-11)
+    np.testing.assert_allclose(X @ A, A @ X, atol=1e-11)
+    np.testing.assert_allclose(X, (Q * np.sign(lam)) @ Q.T, atol=1e-10)
+    np.testing.assert_allclose(o.sign_eigh(A), (Q * np.sign(lam)) @ Q.T, atol=1e-12)
+
+
+def test_sign_textbook_and_eigenvalue_recurrence():
+    """d = 1, alpha = 1/2: X <- X (3I - X^2)/2; on a diagonal input each
+    eigenvalue follows x <- x (3 - x^2)/2 with its sign kept."""
+    lam = np.array([2.0, -1.0, 0.3, -0.05])
+    opts = o.PrismOpts(d=1, p=2, lo=0.5, tol=0.0, max_iter=6, fixed_alpha=True, stall_below=0.0)
+    X, _ = o.sign_ref(np.diag(lam), opts, None)
+    x = lam / np.linalg.norm(lam)
+    for _ in range(6):
+        x = x * (3 - x * x) / 2
+    np.testing.assert_allclose(X, np.diag(x), atol=1e-15)
+
+
+def test_sign_of_spd_is_identity_and_equals_polar():
+    """An SPD input has sign I; for a symmetric input the sign iteration and
+    the polar iteration (R = I - X^T X) coincide step by step."""
+    rng = np.random.default_rng(32)
+    Q = rot(10, 3)
+    A = (Q * np.linspace(0.1, 2.0, 10)) @ Q.T
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=60, stall_below=0.0)
+    S = rng.standard_normal((60, 10, 4))
+    X, _ = o.sign_ref(A, opts, S)
+    np.testing.assert_allclose(X, np.eye(10), atol=1e-11)
+    B = (Q * np.array([1.0, -2.0, 0.5, -0.5, 3.0, -0.2, 0.9, -1.1, 0.3, -0.7])) @ Q.T
+    opts5 = o.PrismOpts(d=2, p=4, lo=0.375, tol=0.0, max_iter=5, stall_below=0.0)
+    Xs, si = o.sign_ref(B, opts5, S)
+    Xp, pi = o.polar_ref(B, opts5, S)
+    np.testing.assert_allclose(si[0].alpha, pi[0].alpha, atol=1e-12)
+    np.testing.assert_allclose(Xs, Xp, atol=1e-12)
+
+
 # ---------------------------------------------------------------- apply / step
 def test_apply_closed_forms():
     rng = np.random.default_rng(4)
