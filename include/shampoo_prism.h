@@ -158,6 +158,17 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
                 const shp_prism_opts* opts, const float* S, int64_t S_count, void* X_out,
                 const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
 
+/* Matrix sign function of a batch of symmetric n x n matrices ([PRISM] Parte I:
+ * the residual of sign functions is R_k = I - X_k^2):
+ *   X_0 = A / ||A||_F; R_k = I - X_k X_k; stop test; alpha_k from S[k];
+ *   X_{k+1} = X_k g_d(R_k; alpha_k)  ->  sign(A) = Q sign(Lambda) Q^T.
+ * A, X_out: [batch][n][n], bf16 or fp32 storage as in matfn_polar (A must be
+ * symmetric and nonsingular; for an SPD A the result is I).  Workspace:
+ * shp_workspace_bytes(SHP_OP_POLAR, n, n, batch, opts with prec = storage). */
+int matfn_sign(const void* A, int storage, int64_t n, int64_t batch, const shp_prism_opts* opts,
+               const float* S, int64_t S_count, void* X_out, const shp_prism_report* report,
+               void* ws, size_t ws_bytes, shp_stream stream);
+
 /* One sketched alpha fit ([PRISM] Parte II.1-II.2) on given residuals:
  *   V_0 = S, V_j = R V_{j-1} (j <= 2d+1), M_ij = <V_i, V_j>_F (i, j = d..2d+1),
  *   J(alpha) = sum_ij r_i(alpha) r_j(alpha) M_ij,  alpha* = argmin_{[lo,hi]} J.

@@ -749,9 +749,17 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
   return dispatch(key, record, static_cast<cudaStream_t>(stream));
 }
 
-int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
-                const shp_prism_opts* o, const float* S, int64_t S_count, void* X_out,
-                const shp_prism_report* rep, void* ws, size_t ws_bytes, shp_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// The polar iteration (R = I - X^T X, or I - X X^T for a wide G) and, with
+// `sign`, the sign iteration of a symmetric square matrix (R = I - X X): the
+// two differ only in the orientation of the first factor of the residual.
+int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
+               const shp_prism_opts* o, const float* S, int64_t S_count, void* X_out,
+               const shp_prism_report* rep, void* ws, size_t ws_bytes, shp_stream stream,
+               bool sign) {
   if (!G || !X_out || !opts_ok(o) || m <= 0 || n <= 0 || batch <= 0) return SHP_EINVAL;
   if (storage != SHP_TF32 && storage != SHP_3XTF32 && storage != SHP_BF16) return SHP_EINVAL;
   const bool bf = storage == SHP_BF16;
@@ -767,12 +775,12 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
     CK(small_polar(static_cast<const float*>(G), static_cast<int>(m), static_cast<int>(n),
                    static_cast<int>(batch), oo, S, static_cast<float*>(X_out),
                    rep ? rep->status : nullptr, rep ? rep->iters : nullptr,
-                   rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr,
+                   rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr, sign,
                    static_cast<cudaStream_t>(stream)));
     return SHP_OK;
   }
   if (batch > 65535) return SHP_EUNSUPPORTED;
-  CallKey key = make_key(1);
+  CallKey key = make_key(sign ? 2 : 1);
   key.storage = storage;
   key.a = G;
   key.x = X_out;
@@ -816,7 +824,11 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
       {  // R = I - X^T X (tall) or I - X X^T (wide), and ||R||_F^2
         EpiParams e = epi(EPI_RESID, rfmt, w.Rhi, w.Rlo, k, kk, K, K, &ctl);
         if (rfmt == OUT_SPLIT) e.out_plain = w.Rs;
-        if (tall)
+        e.sym = 1;  // X^T X: upper-triangle tiles, mirrored
+        if (sign)  // X X (X symmetric)
+          CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn),
+                     op(w.Xhi[cur], w.Xlo[cur], true, n, mn), K, K, M, B, e, st));
+        else if (tall)
           CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], true, n, mn),
                      op(w.Xhi[cur], w.Xlo[cur], true, n, mn), K, K, M, B, e, st));
         else
@@ -829,6 +841,7 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
       if (r != SHP_OK) return r;
       if (o->d == 2) {  // Delta = g - I = R/2 + alpha R^2, stored like X
         EpiParams e = epi(EPI_GPOLY, xfmt, w.ghi, w.glo, k, kk, K, K, &ctl);
+        e.sym = 1;  // R symmetric (mirrored above), so R R and Delta are too
         e.aux_hi = w.Rhi;
         e.aux_lo = w.Rlo;
         e.aux_fmt = rfmt;
@@ -864,6 +877,24 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
     return SHP_OK;
   };
   return dispatch(key, record, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
+                const shp_prism_opts* o, const float* S, int64_t S_count, void* X_out,
+                const shp_prism_report* rep, void* ws, size_t ws_bytes, shp_stream stream) {
+  return polar_impl(G, storage, m, n, batch, o, S, S_count, X_out, rep, ws, ws_bytes, stream,
+                    false);
+}
+
+int matfn_sign(const void* A, int storage, int64_t n, int64_t batch, const shp_prism_opts* o,
+               const float* S, int64_t S_count, void* X_out, const shp_prism_report* rep,
+               void* ws, size_t ws_bytes, shp_stream stream) {
+  return polar_impl(A, storage, n, n, batch, o, S, S_count, X_out, rep, ws, ws_bytes, stream,
+                    true);
 }
 
 }  // extern "C"

@@ -21,6 +21,7 @@
 #include <cudaTypedefs.h>
 
 #include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -78,6 +79,90 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
   }
 }
 
+// The epilogue update of RP consecutive rows of one column (EpiKind): acc
+// a[r], aux x[r], old output w[r]; row dr is on the diagonal (or none).
+// v[r] is what `out` receives, v2[r] what `out2` receives; returns the sum
+// of squares of the first nrows values for RESID.  The kind is tested once.
+template <int RP>
+SHP_DEV float epi_rows(const EpiParams& ep, const float* a, const float* x, const float* w,
+                       int dr, int nrows, float alpha, float eta, float* v, float* v2) {
+  float sq = 0.f;
+  switch (ep.kind) {
+    case EPI_RESID:
+#pragma unroll
+      for (int r = 0; r < RP; ++r) {
+        v[r] = (r == dr ? 1.f : 0.f) - a[r];
+        if (r < nrows) sq += v[r] * v[r];
+      }
+      break;
+    case EPI_GPOLY:
+#pragma unroll
+      for (int r = 0; r < RP; ++r) v[r] = ep.s1 * x[r] + alpha * a[r];
+      break;
+    case EPI_AXPY:
+#pragma unroll
+      for (int r = 0; r < RP; ++r) v[r] = x[r] + ep.s0 * a[r];
+      break;
+    case EPI_EMA:
+#pragma unroll
+      for (int r = 0; r < RP; ++r)
+        v[r] = ep.s0 * w[r] + ep.s1 * a[r] + (r == dr ? ep.s2 : 0.f);
+      break;
+    case EPI_APPLY: {
+      const float c = ep.s0 * eta;
+#pragma unroll
+      for (int r = 0; r < RP; ++r) v[r] = w[r] + c * a[r];
+      break;
+    }
+    case EPI_MOMENTUM: {
+      const float c = ep.s0 * eta;
+#pragma unroll
+      for (int r = 0; r < RP; ++r) {
+        v2[r] = ep.s1 * x[r] + a[r];
+        v[r] = w[r] + c * v2[r];
+      }
+      return 0.f;
+    }
+    default:
+#pragma unroll
+      for (int r = 0; r < RP; ++r) v[r] = ep.s0 * a[r];
+      break;
+  }
+  if (ep.out2_hi != nullptr) {  // I + Delta
+#pragma unroll
+    for (int r = 0; r < RP; ++r) v2[r] = v[r] + (r == dr ? 1.f : 0.f);
+  }
+  return sq;
+}
+
+// Stores v[r] at off + r * ld for r < nrows in format fmt (one branch).
+template <int RP>
+SHP_DEV void store_rows(int fmt, void* hi, float* lo, int64_t off, int64_t ld, const float* v,
+                        int nrows) {
+  if (fmt == OUT_F32) {
+    float* p = static_cast<float*>(hi) + off;
+#pragma unroll
+    for (int r = 0; r < RP; ++r)
+      if (r < nrows) p[r * ld] = v[r];
+  } else if (fmt == OUT_SPLIT) {
+    float* p = static_cast<float*>(hi) + off;
+    float* q = lo + off;
+#pragma unroll
+    for (int r = 0; r < RP; ++r) {
+      if (r < nrows) {
+        const float h = tf32_round(v[r]);
+        p[r * ld] = h;
+        q[r * ld] = tf32_round(v[r] - h);  // pre-rounded: the tensor core truncates
+      }
+    }
+  } else {
+    __nv_bfloat16* p = static_cast<__nv_bfloat16*>(hi) + off;
+#pragma unroll
+    for (int r = 0; r < RP; ++r)
+      if (r < nrows) p[r * ld] = __float2bfloat16_rn(v[r]);
+  }
+}
+
 // Epilogue of one CTA's 128 x BN accumulator, by 8 warps.  Warp (q, h) reads
 // TMEM lanes 32q..32q+31 (q must be the warp's position in its warpgroup, the
 // lane quarter the hardware grants it) and every other 32-column chunk
@@ -88,7 +173,7 @@ SHP_DEV void put(int fmt, void* hi, float* lo, int64_t off, float v) {
 // sits BN columns further.  Returns this warp's sum of squares (RESID).
 template <bool DUAL, int RP>
 SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b, int m0, int n0,
-                            int BN, int q, int h, int lane) {
+                            int BN, int q, int h, int lane, bool mirror = false) {
   const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;  // GPOLY
   const float eta = ep.alpha != nullptr ? ep.alpha[b] : 1.f;    // APPLY, MOMENTUM
   const bool diag_tile = (m0 < n0 + BN) && (n0 < m0 + 128);
@@ -170,50 +255,60 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
 #pragma unroll
           for (int r = 0; r < RP; ++r) w[r] = 0.f;
         }
+        // One branch on the kind and one on each format per pass, then
+        // straight-line loops over the RP rows.
+        const int nrows = rcount - r0 < RP ? rcount - r0 : RP;
+        const int dr = diag_tile ? gj - row0 - r0 : -1;  // row of the diagonal, if here
+        float v[RP], v2[RP];
+        nrm += epi_rows<RP>(ep, a, x, w, dr, nrows, alpha, eta, v, v2);
+        const int64_t off = obase + static_cast<int64_t>(r0) * ep.ldo;
+        store_rows<RP>(ep.out_fmt, ep.out_hi, ep.out_lo, off, ep.ldo, v, nrows);
+        if (ep.out2_hi != nullptr)
+          store_rows<RP>(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, ep.ldo, v2, nrows);
+        if (ep.out_plain != nullptr)
+          store_rows<RP>(OUT_F32, ep.out_plain, nullptr, off, ep.ldo, v, nrows);
+        if (mirror) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) {
-          if (r0 + r >= rcount) break;
-          const int gi = row0 + r0 + r;
-          const float acc = a[r];
-          const float eye = (diag_tile && gi == gj) ? 1.f : 0.f;
-          const int64_t off = obase + static_cast<int64_t>(r0 + r) * ep.ldo;
-          float val, val2 = -1.f;
-          switch (ep.kind) {
-            case EPI_RESID:
-              val = eye - acc;
-              nrm += val * val;
-              break;
-            case EPI_GPOLY:
-              val = ep.s1 * x[r] + alpha * acc;
-              break;
-            case EPI_AXPY:
-              val = x[r] + ep.s0 * acc;
-              break;
-            case EPI_EMA:
-              val = ep.s0 * w[r] + ep.s1 * acc + ep.s2 * eye;
-              break;
-            case EPI_APPLY:
-              val = w[r] + ep.s0 * eta * acc;
-              break;
-            case EPI_MOMENTUM:
-              val2 = ep.s1 * x[r] + acc;
-              val = w[r] + ep.s0 * eta * val2;
-              break;
-            default:
-              val = ep.s0 * acc;
-              break;
-          }
-          put(ep.out_fmt, ep.out_hi, ep.out_lo, off, val);
-          if (ep.out2_hi != nullptr)
-            put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off,
-                ep.kind == EPI_MOMENTUM ? val2 : val + eye);
-          if (ep.out_plain != nullptr) ep.out_plain[off] = val;
+          for (int r = 0; r < RP; ++r) st[(r0 + r) * 33 + lane] = v[r];
         }
       }
     }
     __syncwarp();
+    if (mirror) {
+      // the chunk's values, now in st, also go to the transposed position:
+      // lane = row of the tile, so each store is one coalesced row segment
+      if (lane < rcount) {
+        const int64_t mcol = static_cast<int64_t>(row0 + lane);
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+          const int mrow = n0 + c * 32 + j;
+          if (mrow >= ep.N) break;
+          const int64_t off = static_cast<int64_t>(b) * ep.bso + mrow * ep.ldo + mcol;
+          const float v = st[lane * 33 + j];
+          put(ep.out_fmt, ep.out_hi, ep.out_lo, off, v);
+          if (ep.out_plain != nullptr) ep.out_plain[off] = v;
+        }
+      }
+      __syncwarp();
+    }
   }
   return nrm;
+}
+
+// Tile r of one batch member: row-major over tiles_m x tiles_n, or, for a
+// symmetric result, row by row over the tiles with tn >= tm.
+SHP_DEV void tile_coords(int r, int tiles_n, bool sym, int& tm, int& tn) {
+  if (!sym) {
+    tm = r / tiles_n;
+    tn = r % tiles_n;
+    return;
+  }
+  tm = 0;
+  while (r >= tiles_n - tm) {
+    r -= tiles_n - tm;
+    ++tm;
+  }
+  tn = tm + r;
 }
 
 template <int MODE, bool A_MN, bool B_MN, bool PAIR>
@@ -389,7 +484,7 @@ __global__ void __launch_bounds__(256, 1)
   if (!mbar_wait(done, 0)) timed_out = true;
   __syncwarp();
   tc_fence_after();
-  float nrm = epilogue_tile<C::SPLIT, 32>(reinterpret_cast<float*>(smem) + warp * (32 * 33), tmem,
+  float nrm = epilogue_tile<C::SPLIT, 16>(reinterpret_cast<float*>(smem) + warp * (32 * 33), tmem,
                                           ep, b, m0, n0, BN, warp & 3, warp >> 2, lane);
   if (ep.kind == EPI_RESID) {
     nrm = warp_sum(nrm);
@@ -431,7 +526,10 @@ __global__ void __launch_bounds__(320, 1)
   const bool leader = rank == 0;
   const int ncl = static_cast<int>(gridDim.x) / 2, cl = static_cast<int>(blockIdx.x) / 2;
   const int tiles_n = (ep.N + BN - 1) / BN, tiles_m = (ep.M + 255) / 256;
-  const int per_b = tiles_n * tiles_m, ntiles = per_b * batch;
+  // symmetric result (M == N): only the tiles on and above the diagonal
+  const bool sym = ep.sym != 0 && ep.M == ep.N;
+  const int per_b = sym ? tiles_n * (tiles_n + 1) / 2 : tiles_n * tiles_m;
+  const int ntiles = per_b * batch;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -482,8 +580,10 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = cl; t < ntiles && !stop; t += ncl) {
         const int b = t / per_b, r = t % per_b;
         if (ep.active != nullptr && ep.active[b] == 0) continue;
-        const int m0 = (r / tiles_n) * 256 + static_cast<int>(rank) * 128;
-        const int nb0 = (r % tiles_n) * BN + static_cast<int>(rank) * 128;
+        int tm, tn;
+        tile_coords(r, tiles_n, sym, tm, tn);
+        const int m0 = tm * 256 + static_cast<int>(rank) * 128;
+        const int nb0 = tn * BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < KB; ++kb, ++kit) {
           const int s = kit % C::PP_STAGES;
           if (kit >= C::PP_STAGES &&
@@ -593,10 +693,16 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
       tc_fence_after();
-      const int m0 = (r / tiles_n) * 256 + static_cast<int>(rank) * 128;
-      const int n0 = (r % tiles_n) * BN;
+      int tm, tn;
+      tile_coords(r, tiles_n, sym, tm, tn);
+      const int m0 = tm * 256 + static_cast<int>(rank) * 128;
+      const int n0 = tn * BN;
+      // an off-diagonal tile of a symmetric result also writes its mirror image
+      // and counts twice in ||R||^2
+      const bool mirror = sym && tn != tm;
       float nrm = epilogue_tile<false, 16>(st, tmem + static_cast<uint32_t>(u * BN), ep, b, m0,
-                                          n0, BN, q, h, lane);
+                                          n0, BN, q, h, lane, mirror);
+      if (mirror) nrm *= 2.f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acce[u]), 0));
@@ -687,7 +793,8 @@ cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtenso
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int ntiles = ((N + 255) / 256) * ((M + 255) / 256) * batch;
+  const int tn = (N + 255) / 256;
+  const int ntiles = (ep.sym && M == N ? tn * (tn + 1) / 2 : tn * ((M + 255) / 256)) * batch;
   int ncl = sms / 2;
   if (ncl > ntiles) ncl = ntiles;
   if (ncl < 1) ncl = 1;

@@ -79,6 +79,10 @@ struct EpiParams {
   const int* active;  // blocks with active[b] == 0 are skipped (may be null)
   int* status;        // receives ST_ETIMEOUT if a pipeline wait runs out (may be null)
   int M, N;
+  // The result is symmetric (M == N, kinds RESID/GPOLY/STORE, no out2): the
+  // persistent kernel computes the tiles on and above the diagonal and writes
+  // each off-diagonal tile's mirror image too; other kernels compute it all.
+  int sym;
 };
 
 // C[b] (M x N) = A[b] (M x K) * B[b] (K x N) on tcgen05 tensor cores,
@@ -183,8 +187,9 @@ cudaError_t small_inv_root(const float* A, int n, int batch, int power,
                            const shp_prism_opts& o, const float* S, float* X,
                            int* rep_status, int* rep_iters, float* rep_resid, float* rep_alpha,
                            cudaStream_t st);
+// sign: the sign function of a symmetric square G (R = I - X X).
 cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
                         const float* S, float* X, int* rep_status, int* rep_iters,
-                        float* rep_resid, float* rep_alpha, cudaStream_t st);
+                        float* rep_resid, float* rep_alpha, bool sign, cudaStream_t st);
 
 }  // namespace shp

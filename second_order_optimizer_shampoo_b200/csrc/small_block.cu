@@ -341,10 +341,12 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
 }
 
 // Polar factor of an m x n block (m, n <= 64): the tall iteration on G (or on
-// G^T when m < n), X_0 = G / ||G||_F, R = I - X^T X, X <- X + X Delta.
+// G^T when m < n), X_0 = G / ||G||_F, R = I - X^T X, X <- X + X Delta.  With
+// `sign` (m == n, G symmetric) the residual is I - X X: the sign function.
 __global__ void __launch_bounds__(SB_THREADS, 3)
     k_small_polar(const float* __restrict__ G, int m, int n, SmallCfg o,
-                  const float* __restrict__ S, float* __restrict__ Xout, SmallReport rep) {
+                  const float* __restrict__ S, float* __restrict__ Xout, SmallReport rep,
+                  int sign) {
   count_kernel_run();
   extern __shared__ __align__(16) float sm[];
   __shared__ double red[SB_THREADS / 32][10];
@@ -377,7 +379,10 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   int status = ST_OK;
   float prev = INFINITY;
   for (int k = 0;; ++k) {
-    const double n2 = block_sum(residual<true>(X, X, rows, k_n, R, r0, c0), red[0]);
+    // R = I - X^T X (polar) or I - X X (sign of a symmetric X, m == n)
+    const double n2 = block_sum(sign ? residual<false>(X, X, rows, k_n, R, r0, c0)
+                                     : residual<true>(X, X, rows, k_n, R, r0, c0),
+                                red[0]);
     const float r = sqrtf(static_cast<float>(n2) / static_cast<float>(k_n));
     const int st = stop_rule(r, k, mi, o.tol, prev, o.stall_below, o.stall_ratio);
     if (tid == 0 && rep.resid != nullptr) rep.resid[2 * b * (mi + 1) + k] = r;
@@ -447,12 +452,13 @@ cudaError_t small_inv_root(const float* A, int n, int batch, int power, const sh
 
 cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
                         const float* S, float* X, int* rep_status, int* rep_iters,
-                        float* rep_resid, float* rep_alpha, cudaStream_t st) {
+                        float* rep_resid, float* rep_alpha, bool sign, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
   cudaError_t e = prepare(k_small_polar);
   if (e != cudaSuccess) return e;
   k_small_polar<<<batch, SB_THREADS, SB_SMEM, st>>>(
-      G, m, n, make_cfg(o), S, X, SmallReport{rep_status, rep_iters, rep_resid, rep_alpha});
+      G, m, n, make_cfg(o), S, X, SmallReport{rep_status, rep_iters, rep_resid, rep_alpha},
+      sign ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -181,6 +181,35 @@ def matfn_polar(G, opts: A.PrismOpts | None = None, S=None, out=None, report=Tru
     return out, rep
 
 
+def matfn_sign(Amat, opts: A.PrismOpts | None = None, S=None, out=None, report=True, ws=None):
+    """Matrix sign function of a batch of symmetric n x n matrices (bf16 input
+    keeps bf16 storage)."""
+    opts = opts or make_opts()
+    _dev(Amat, S, out)
+    n = Amat.shape[-1]
+    if Amat.shape[-2] != n:
+        raise ValueError("matfn_sign needs square matrices")
+    batch = Amat.numel() // (n * n)
+    if Amat.dtype == torch.bfloat16:
+        storage = A.SHP_BF16
+    elif Amat.dtype == torch.float32:
+        storage = opts.prec if opts.prec in (A.SHP_TF32, A.SHP_3XTF32) else A.SHP_TF32
+    else:
+        raise ValueError("A must be float32 or bfloat16")
+    out = torch.empty_like(Amat) if out is None else out
+    rep = report if isinstance(report, dict) else (
+        _report(batch, opts.max_iter, Amat.device) if report else None)
+    o2 = A.PrismOpts.from_buffer_copy(opts)
+    o2.prec = storage
+    need = shp_workspace_bytes(A.SHP_OP_POLAR, n, n, batch, o2)
+    ws = _ws(need, Amat.device) if ws is None else ws
+    s_count = 0 if S is None else S.shape[0]
+    _check(A.lib().matfn_sign(_p(Amat), storage, n, batch, ctypes.byref(opts), _p(S), s_count,
+                              _p(out), _report_struct(rep), _p(ws), ws.numel(), _stream()),
+           "matfn_sign")
+    return out, rep
+
+
 def prism_alpha_fit(R, S, d: int, lo: float, hi: float, ws=None):
     """alpha* on [lo, hi] for each residual in the batch, plus J's coefficients."""
     _dev(R, S)

@@ -157,7 +157,10 @@ def run_polar(G, prec, d, p, tol, max_iter, S, bits=None):
     return to_host(X), {k: to_host(v) for k, v in rep.items()}, opts
 
 
-@pytest.mark.parametrize("shape", [(512, 128), (128, 320), (64, 32), (96, 96)])
+# (1024, 768) and (520, 600) run X^T X and R R on the persistent kernel's
+# upper-triangle tiles with mirrored stores (the latter with ragged tiles).
+@pytest.mark.parametrize("shape", [(512, 128), (128, 320), (64, 32), (96, 96), (1024, 768),
+                                   (520, 600)])
 @pytest.mark.parametrize("d", [1, 2])
 def test_polar_split(shape, d):
     m, n = shape
@@ -198,3 +201,63 @@ def test_polar_bf16(shape):
     k = min(m, n)
     XtX = X[0].T @ X[0] if m >= n else X[0] @ X[0].T
     assert np.linalg.norm(np.eye(k) - XtX) / np.sqrt(k) <= 1e-2
+
+
+# ------------------------------------------------------------------ sign
+def sym_indefinite(n, batch, seed):
+    """Symmetric matrices Q diag(lambda) Q^T with |lambda| log-uniform on
+    [1e-2, 1] and random signs."""
+    out = np.empty((batch, n, n), dtype=np.float32)
+    for b in range(batch):
+        g = np.random.default_rng((seed, b))
+        Q, Rq = np.linalg.qr(g.standard_normal((n, n)))
+        Q = Q * np.sign(np.diag(Rq))
+        lam = np.exp(g.uniform(np.log(1e-2), 0.0, n)) * g.choice([-1.0, 1.0], n)
+        out[b] = ((Q * lam) @ Q.T).astype(np.float32)
+    return out
+
+
+@pytest.mark.parametrize("n", [48, 256, 520])
+@pytest.mark.parametrize("d", [1, 2])
+def test_sign_split(n, d):
+    """sign(A) of symmetric indefinite A (on chip at n = 48, persistent
+    upper-triangle tiles at 256 and the ragged 520) against the oracle with
+    the same iteration count and against eigh."""
+    P = prism()
+    A = sym_indefinite(n, 2, 71 + n)
+    S = synth.sketch_stack(40, n, 8, 1071)
+    opts = P.make_opts(d=d, p=8, tol=1e-6, max_iter=40, prec="3xtf32")
+    X, rep = P.matfn_sign(to_dev(torch, A), opts, to_dev(torch, S))
+    X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
+    for b in range(2):
+        # the split path's residual floor (~1e-6 at n = 520) may end a pass by
+        # the stall rule just above tol; the result is then as accurate
+        assert rep["status"][b] in (o.OK, o.ESTALL), rep["status"]
+        it = rep["iters"][b][0]
+        assert rep["resid"][b, 0, it] <= 4e-6
+        Xo, infos = o.sign_ref(A[b], oracle_opts(opts), S, force_iters=it)
+        np.testing.assert_allclose(rep["alpha"][b, 0, :it], infos[0].alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= 1e-5
+        assert relerr(X[b], o.sign_eigh(A[b])) <= 1e-5
+
+
+def test_sign_bf16_and_spd():
+    """bf16 storage (residual and the error at bf16 resolution) and an SPD
+    input, whose sign is the identity."""
+    P = prism()
+    n = 256
+    A = sym_indefinite(n, 1, 81)
+    bits = synth.to_bf16_bits(A)
+    A16 = synth.bf16_bits_to_f32(bits)
+    S = synth.sketch_stack(40, n, 8, 1081)
+    opts = P.make_opts(d=2, p=8, tol=1e-2, max_iter=40, prec="bf16")
+    X, rep = P.matfn_sign(bf16_to_dev(torch, bits), opts, to_dev(torch, S))
+    assert to_host(rep["status"])[0] == o.OK
+    Xh = to_host(X)[0].astype(np.float64)
+    assert np.linalg.norm(np.eye(n) - Xh @ Xh) / np.sqrt(n) <= 1e-2 + 2 ** -7
+    assert relerr(Xh, o.sign_eigh(A16[0])) <= 2 ** -6
+    spd = synth.spd_batch(n, 1, 1e-2, 1.0, 82)
+    opts2 = P.make_opts(d=2, p=8, tol=1e-6, max_iter=40, prec="3xtf32")
+    X2, rep2 = P.matfn_sign(to_dev(torch, spd), opts2, to_dev(torch, S))
+    assert to_host(rep2["status"])[0] == o.OK
+    np.testing.assert_allclose(to_host(X2)[0], np.eye(n), atol=1e-5)
