@@ -13,7 +13,8 @@ docstring by page title and section:
 * [PRISM-it] "Sintesi Tecnica: PRISM" (gist.science), "Parte I" and
   "Parte II" (residual-form iteration, adaptive polynomial, alpha fit,
   clamp, randomized sketch; R_k = I - X_k^2 for sign functions).
-* [PRISM-zh] "PRISM：分布无关的自适应矩阵函数计算" (euno.news), "方法论".
+* [PRISM-zh] "PRISM：分布无关的自适应矩阵函数计算" (euno.news), "方法论"
+  (item 3: adaptive degree selection).
 
 Readings taken where the pages are silent (each is listed in the design doc):
 * The residual series is the Taylor series of (1 - xi)^(-1/2); the printed
@@ -63,7 +64,9 @@ class PrismOpts:
     fixed_alpha: use alpha = lo every step (the plain Taylor Newton-Schulz
     baseline); stall_below/stall_ratio: stop with ESTALL when the previous
     residual is below stall_below and the new one is not smaller than
-    stall_ratio times it.
+    stall_ratio times it; adaptive_degree: each pass starts at degree 1 and
+    raises to d once the sketched degree-1 fit predicts a contraction above
+    raise_above (see fit_step).
     """
     d: int = 2
     p: int = 8
@@ -74,6 +77,8 @@ class PrismOpts:
     fixed_alpha: bool = False
     stall_below: float = 0.05
     stall_ratio: float = 0.75
+    adaptive_degree: bool = False
+    raise_above: float = 0.9
 
 
 @dataclass
@@ -81,6 +86,7 @@ class PassInfo:
     alpha: list = field(default_factory=list)
     res: list = field(default_factory=list)
     J_coef: list = field(default_factory=list)
+    degree: list = field(default_factory=list)
     iters: int = 0
     status: int = OK
 
@@ -253,6 +259,31 @@ def prism_alpha_ref(Rk, S, d, lo, hi):
     return _argmin_quartic(coef, lo, hi), coef
 
 
+def fit_step(Rk, Sk, deg, opts: PrismOpts):
+    """alpha of one iteration at the current degree, and the degree itself.
+
+    Adaptive degree ([PRISM-zh] 方法论 3: the sketch's residual is monitored
+    and the degree raised only when needed): the pass starts at degree 1; the
+    degree-1 fit predicts the next sketched residual sqrt(J_1(alpha*)), and
+    when its ratio to the current one, ||R_k S_k||_F, exceeds raise_above the
+    degree becomes opts.d for this and every later iteration of the pass.
+    The interval of degree e is [c_e, hi] with c_e its Taylor coefficient
+    (1/2, 3/8), as for the fixed degrees.  Returns (alpha, coef, degree)."""
+    if opts.fixed_alpha:
+        return float(opts.lo), np.full(5, np.nan), deg
+    if not opts.adaptive_degree:
+        a, coef = prism_alpha_ref(Rk, Sk, deg, opts.lo, opts.hi)
+        return a, coef, deg
+    a, coef = prism_alpha_ref(Rk, Sk, deg, taylor_coeffs(deg)[deg], opts.hi)
+    if deg < opts.d:
+        J = float(np.polynomial.polynomial.polyval(a, coef))
+        base = float(np.sum((_f64(Rk) @ _f64(Sk)) ** 2))
+        if base > 0.0 and sqrt(max(J, 0.0) / base) > opts.raise_above:
+            deg = opts.d
+            a, coef = prism_alpha_ref(Rk, Sk, deg, taylor_coeffs(deg)[deg], opts.hi)
+    return a, coef, deg
+
+
 # ---------------------------------------------------------------------------
 # Newton-Schulz passes  ([PRISM-it] Parte I: X_{k+1} = X_k f(R_k); [Shampoo] §3.1)
 # ---------------------------------------------------------------------------
@@ -296,6 +327,7 @@ def coupled_ref(B, opts: PrismOpts, S, s_offset=0, force_iters=None):
     I = np.eye(n)
     Y, Z = B.copy(), I.copy()
     info = PassInfo()
+    deg = 1 if opts.adaptive_degree else opts.d
     k = 0
     while True:
         Rk = I - Z @ Y
@@ -303,13 +335,11 @@ def coupled_ref(B, opts: PrismOpts, S, s_offset=0, force_iters=None):
         info.res.append(rk)
         if _stop(info, rk, k, opts, force_iters):
             break
-        if opts.fixed_alpha:
-            a, coef = float(opts.lo), np.full(5, np.nan)
-        else:
-            a, coef = prism_alpha_ref(Rk, S[s_offset + k], opts.d, opts.lo, opts.hi)
+        a, coef, deg = fit_step(Rk, None if S is None else S[s_offset + k], deg, opts)
         info.alpha.append(a)
         info.J_coef.append(coef)
-        g = matrix_poly(g_coeffs(opts.d, a), Rk)
+        info.degree.append(deg)
+        g = matrix_poly(g_coeffs(deg, a), Rk)
         Y, Z = Y @ g, g @ Z
         k += 1
     info.iters = k
@@ -350,6 +380,7 @@ def polar_ref(G, opts: PrismOpts, S, force_iters=None):
     I = np.eye(n)
     X = G / np.linalg.norm(G)
     info = PassInfo()
+    deg = 1 if opts.adaptive_degree else opts.d
     k = 0
     while True:
         Rk = I - X.T @ X
@@ -357,13 +388,11 @@ def polar_ref(G, opts: PrismOpts, S, force_iters=None):
         info.res.append(rk)
         if _stop(info, rk, k, opts, force_iters):
             break
-        if opts.fixed_alpha:
-            a, coef = float(opts.lo), np.full(5, np.nan)
-        else:
-            a, coef = prism_alpha_ref(Rk, S[k], opts.d, opts.lo, opts.hi)
+        a, coef, deg = fit_step(Rk, None if S is None else S[k], deg, opts)
         info.alpha.append(a)
         info.J_coef.append(coef)
-        X = X @ matrix_poly(g_coeffs(opts.d, a), Rk)
+        info.degree.append(deg)
+        X = X @ matrix_poly(g_coeffs(deg, a), Rk)
         k += 1
     info.iters = k
     return (X.T if wide else X), [info]
@@ -381,6 +410,7 @@ def sign_ref(A, opts: PrismOpts, S, force_iters=None):
     I = np.eye(n)
     X = A / np.linalg.norm(A)
     info = PassInfo()
+    deg = 1 if opts.adaptive_degree else opts.d
     k = 0
     while True:
         Rk = I - X @ X
@@ -388,13 +418,11 @@ def sign_ref(A, opts: PrismOpts, S, force_iters=None):
         info.res.append(rk)
         if _stop(info, rk, k, opts, force_iters):
             break
-        if opts.fixed_alpha:
-            a, coef = float(opts.lo), np.full(5, np.nan)
-        else:
-            a, coef = prism_alpha_ref(Rk, S[k], opts.d, opts.lo, opts.hi)
+        a, coef, deg = fit_step(Rk, None if S is None else S[k], deg, opts)
         info.alpha.append(a)
         info.J_coef.append(coef)
-        X = X @ matrix_poly(g_coeffs(opts.d, a), Rk)
+        info.degree.append(deg)
+        X = X @ matrix_poly(g_coeffs(deg, a), Rk)
         k += 1
     info.iters = k
     return X, [info]

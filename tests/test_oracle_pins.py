@@ -327,6 +327,46 @@ def test_polar_textbook_and_singular_value_recurrence():
     np.testing.assert_allclose(X, want, atol=1e-15)
 
 
+# ---------------------------------------------------------------- adaptive degree
+def test_adaptive_degree_limits_reduce_to_fixed_degrees():
+    """raise_above = inf never raises (the degree-1 run with [1/2, 1]);
+    raise_above = 0 raises at the first step (the degree-2 run with [3/8, 1])."""
+    rng = np.random.default_rng(41)
+    A, _ = spd(24, np.logspace(-3, 0, 24), 41)
+    S = rng.standard_normal((120, 24, 4))
+    base = dict(p=4, tol=1e-10, max_iter=50, stall_below=0.0)
+    never = o.PrismOpts(d=2, adaptive_degree=True, raise_above=np.inf, **base)
+    always = o.PrismOpts(d=2, adaptive_degree=True, raise_above=0.0, **base)
+    d1 = o.PrismOpts(d=1, lo=0.5, **base)
+    d2 = o.PrismOpts(d=2, lo=0.375, **base)
+    for ad, fixed in ((never, d1), (always, d2)):
+        Xa, ia = o.inv_root_ref(A, o.POW_INV4, ad, S)
+        Xf, if_ = o.inv_root_ref(A, o.POW_INV4, fixed, S)
+        for pa, pf in zip(ia, if_):
+            assert pa.degree == [fixed.d] * pa.iters
+            np.testing.assert_allclose(pa.alpha, pf.alpha, atol=1e-14)
+        np.testing.assert_allclose(Xa, Xf, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("xi,raised", [(0.9, False), (0.99, True)])
+def test_adaptive_degree_rule_on_scalar_residual(xi, raised):
+    """B = (1 - xi) I gives R_0 = xi I: the degree-1 fit's predicted ratio is
+    min over alpha in [1/2, 1] of |r(xi; alpha)| / xi, attained at alpha = 1
+    for these xi: 0.71 at xi = 0.9 (kept below raise_above = 0.9) and 0.9701
+    at xi = 0.99 (raised)."""
+    n = 6
+    opts = o.PrismOpts(d=2, p=3, adaptive_degree=True, raise_above=0.9, tol=1e-12,
+                       max_iter=30, stall_below=0.0)
+    S = np.random.default_rng(42).standard_normal((30, n, 3))
+    info = o.coupled_ref((1 - xi) * np.eye(n), opts, S)[2]
+    q = abs((1 - 2) + (2 - 1) * xi + xi * xi)  # r(xi; 1) / xi
+    assert (q > 0.9) == raised
+    assert info.degree[0] == (2 if raised else 1)
+    assert info.alpha[0] == pytest.approx(1.0 if not raised else info.alpha[0])
+    # the degree never goes back down within a pass
+    assert all(b >= a for a, b in zip(info.degree, info.degree[1:]))
+
+
 # ---------------------------------------------------------------- sign
 def test_sign_of_indefinite_matches_eigh():
     """sign(A) of a symmetric indefinite matrix: involutory (X^2 = I), commutes
