@@ -85,6 +85,12 @@ typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_
  *   fixed_alpha 1: alpha = lo every step (plain Taylor Newton-Schulz)
  *   stall_below, stall_ratio: stop with SHP_ESTALL when the previous residual
  *               is below stall_below and the new one exceeds stall_ratio times it
+ *   adaptive_degree 1: every pass starts at degree 1 and raises to d (= 2) for
+ *               the rest of the pass once the sketched degree-1 fit predicts a
+ *               contraction ||r(R_k) S_k||_F / ||R_k S_k||_F above raise_above
+ *               ([PRISM] 方法论 3, adaptive degree selection); the interval of
+ *               degree e is then [c_e, hi] with c_e its Taylor coefficient
+ *               (1/2, 3/8) and lo is not used; needs fixed_alpha = 0
  */
 typedef struct {
   int d;
@@ -96,6 +102,8 @@ typedef struct {
   int fixed_alpha;
   float stall_below;
   float stall_ratio;
+  int adaptive_degree;
+  float raise_above;
 } shp_prism_opts;
 
 /* Optional per-block trajectory, all device pointers, each may be NULL.
@@ -103,12 +111,14 @@ typedef struct {
  *   iters  [B][2]                   update steps in pass 1 and pass 2
  *   resid  [B][2][max_iter + 1]     ||R_k||_F / sqrt(n) at every k
  *   alpha  [B][2][max_iter]         alpha_k used at every update
+ *   degree [B][2][max_iter]         degree of g used at every update
  * Entries after a block stops are left untouched. */
 typedef struct {
   int32_t* status;
   int32_t* iters;
   float* resid;
   float* alpha;
+  int32_t* degree;
 } shp_prism_report;
 
 /* Bytes of scratch the call `op` needs for these sizes (0 if none).  For

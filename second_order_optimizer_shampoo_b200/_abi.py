@@ -34,12 +34,14 @@ class PrismOpts(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("p", ctypes.c_int), ("lo", ctypes.c_float),
                 ("hi", ctypes.c_float), ("tol", ctypes.c_float), ("max_iter", ctypes.c_int),
                 ("prec", ctypes.c_int), ("fixed_alpha", ctypes.c_int),
-                ("stall_below", ctypes.c_float), ("stall_ratio", ctypes.c_float)]
+                ("stall_below", ctypes.c_float), ("stall_ratio", ctypes.c_float),
+                ("adaptive_degree", ctypes.c_int), ("raise_above", ctypes.c_float)]
 
 
 class PrismReport(ctypes.Structure):
     _fields_ = [("status", ctypes.c_void_p), ("iters", ctypes.c_void_p),
-                ("resid", ctypes.c_void_p), ("alpha", ctypes.c_void_p)]
+                ("resid", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("degree", ctypes.c_void_p)]
 
 
 _lib = None

@@ -45,6 +45,9 @@ bool opts_ok(const shp_prism_opts* o) {
   if (o->max_iter < 1 || o->max_iter > 256) return false;
   if (o->prec != SHP_TF32 && o->prec != SHP_3XTF32 && o->prec != SHP_BF16) return false;
   if (!(o->stall_below >= 0.f) || !(o->stall_ratio >= 0.f)) return false;
+  if (o->adaptive_degree != 0 &&
+      (o->d != 2 || o->fixed_alpha != 0 || !(o->raise_above >= 0.f)))
+    return false;
   return true;
 }
 
@@ -52,6 +55,9 @@ Ctl carve_ctl(Arena& a, int64_t batch) {
   Ctl c;
   c.bs = a.take<BlockState>(batch);
   c.active = a.take<int>(batch);
+  c.deg = a.take<int>(batch);
+  c.act1 = a.take<int>(batch);
+  c.act2 = a.take<int>(batch);
   c.dnorm = a.take<double>(batch);
   c.tmo = a.take<int>(batch);
   c.alpha = a.take<float>(batch);
@@ -172,7 +178,8 @@ Operand op(const void* hi, const float* lo, bool mn, int64_t ld, int64_t bs) {
 // (j <= 2d+1), then the Gram, the quartic and its argmin.
 int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass, float* V,
                      const shp_prism_opts* o, const Ctl& ctl, float* rep_alpha,
-                     int64_t rep_stride, int rep_slot_base, cudaStream_t st) {
+                     int64_t rep_stride, int rep_slot_base, cudaStream_t st,
+                     int* rep_degree = nullptr) {
   const int64_t np = n * o->p, nn = n * n;
   const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
   if (!o->fixed_alpha) {
@@ -182,8 +189,9 @@ int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass,
       CK(sketch_pass(Rs, nullptr, n, nn, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
                      ctl.active, nullptr, 0, st));
   }
+  AdaptiveDeg ad{o->adaptive_degree, o->raise_above, ctl.deg, ctl.act1, ctl.act2, rep_degree};
   CK(alpha_solve(V, n, o->p, o->d, batch, o->lo, o->hi, o->fixed_alpha, ctl.active, ctl.alpha,
-                 nullptr, rep_alpha, rep_stride, rep_slot_base, ctl.it, st));
+                 nullptr, rep_alpha, rep_stride, rep_slot_base, ctl.it, st, &ad));
   return SHP_OK;
 }
 
@@ -206,7 +214,7 @@ struct CallKey {
   shp_prism_opts o;
   void* ws;
   size_t ws_bytes;
-  const void* rep[4];
+  const void* rep[5];
 };
 
 struct CachedGraph {
@@ -630,7 +638,7 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
     CK(small_inv_root(A, static_cast<int>(n), static_cast<int>(batch), power, *o, S, X_out,
                       rep ? rep->status : nullptr, rep ? rep->iters : nullptr,
                       rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr,
-                      static_cast<cudaStream_t>(stream)));
+                      rep ? rep->degree : nullptr, static_cast<cudaStream_t>(stream)));
     return SHP_OK;
   }
   if (batch > 65535) return SHP_EUNSUPPORTED;
@@ -650,6 +658,7 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
     key.rep[1] = rep->iters;
     key.rep[2] = rep->resid;
     key.rep[3] = rep->alpha;
+    key.rep[4] = rep->degree;
   }
   auto record = [&](cudaStream_t const* cs, cudaGraph_t g) -> int {
     Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) &
@@ -665,8 +674,9 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
     float* rep_res = rep != nullptr ? rep->resid : nullptr;
     float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
     int* rep_iters = rep != nullptr ? rep->iters : nullptr;
+    int* rep_degree = rep != nullptr ? rep->degree : nullptr;
     for (int pass = 0; pass < npass; ++pass) {
-      CK(reset_pass(ctl, B, pass == 0, cs[0]));
+      CK(reset_pass(ctl, B, pass == 0, cs[0], o->adaptive_degree ? 1 : o->d));
       if (pass == 0) {
         CK(frob_norm2(A, 0, nn, B, ctl, cs[0]));
         CK(coupled_init(A, n, B, ctl, w.Yhi[0], w.Ylo[0], w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo,
@@ -690,12 +700,17 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
         CK(control_step(ctl, B, n, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
                         2 * (mi + 1), pass * (mi + 1), rep_iters, pass, st));
         int r = sketch_and_alpha(w.Rs, n, B, S_pass, w.V, o, ctl, rep_alpha, 2 * mi, pass * mi,
-                                 st);
+                                 st, rep_degree);
         if (r != SHP_OK) return r;
         float* z2hi = first ? w.Zhi[nxt] : nullptr;
         float* z2lo = first ? w.Zlo[nxt] : nullptr;
+        // adaptive degree: blocks at degree 1 and 2 take the two launches below,
+        // each masked to its own blocks
+        if (o->adaptive_degree)
+          CK(gform_d1(w.Rhi, w.Rlo, n, B, ctl, fmt, w.ghi, w.glo, z2hi, z2lo, st, ctl.act1));
         if (o->d == 2) {  // Delta = g - I = R/2 + alpha R^2 in the R R epilogue
           EpiParams e = epi(EPI_GPOLY, fmt, w.ghi, w.glo, n, nn, N, N, &ctl);
+          if (o->adaptive_degree) e.active = ctl.act2;
           e.out2_hi = z2hi;
           e.out2_lo = z2lo;
           e.aux_hi = w.Rhi;
@@ -775,8 +790,8 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
     CK(small_polar(static_cast<const float*>(G), static_cast<int>(m), static_cast<int>(n),
                    static_cast<int>(batch), oo, S, static_cast<float*>(X_out),
                    rep ? rep->status : nullptr, rep ? rep->iters : nullptr,
-                   rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr, sign,
-                   static_cast<cudaStream_t>(stream)));
+                   rep ? rep->resid : nullptr, rep ? rep->alpha : nullptr,
+                   rep ? rep->degree : nullptr, sign, static_cast<cudaStream_t>(stream)));
     return SHP_OK;
   }
   if (batch > 65535) return SHP_EUNSUPPORTED;
@@ -797,6 +812,7 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
     key.rep[1] = rep->iters;
     key.rep[2] = rep->resid;
     key.rep[3] = rep->alpha;
+    key.rep[4] = rep->degree;
   }
   auto record = [&](cudaStream_t const* cs, cudaGraph_t g) -> int {
     Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) &
@@ -816,7 +832,8 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
     float* rep_res = rep != nullptr ? rep->resid : nullptr;
     float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
     int* rep_iters = rep != nullptr ? rep->iters : nullptr;
-    CK(reset_pass(ctl, B, 1, cs[0]));
+    int* rep_degree = rep != nullptr ? rep->degree : nullptr;
+    CK(reset_pass(ctl, B, 1, cs[0], o->adaptive_degree ? 1 : o->d));
     CK(frob_norm2(G, bf, mn, B, ctl, cs[0]));
     CK(polar_init(G, bf, mn, B, ctl, xfmt, w.Xhi[0], w.Xlo[0], cs[0]));
     auto iter = [&](int cur, bool, cudaStream_t st) -> int {
@@ -837,10 +854,14 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
       }
       CK(control_step(ctl, B, k, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
                       2 * (mi + 1), 0, rep_iters, 0, st));
-      int r = sketch_and_alpha(w.Rs, k, B, S, w.V, o, ctl, rep_alpha, 2 * mi, 0, st);
+      int r = sketch_and_alpha(w.Rs, k, B, S, w.V, o, ctl, rep_alpha, 2 * mi, 0, st, rep_degree);
       if (r != SHP_OK) return r;
+      if (o->adaptive_degree)  // degree-1 blocks; the R R launch below takes the others
+        CK(gform_d1(w.Rhi, w.Rlo, k, B, ctl, xfmt, w.ghi, w.glo, nullptr, nullptr, st,
+                    ctl.act1));
       if (o->d == 2) {  // Delta = g - I = R/2 + alpha R^2, stored like X
         EpiParams e = epi(EPI_GPOLY, xfmt, w.ghi, w.glo, k, kk, K, K, &ctl);
+        if (o->adaptive_degree) e.active = ctl.act2;
         e.sym = 1;  // R symmetric (mirrored above), so R R and Delta are too
         e.aux_hi = w.Rhi;
         e.aux_lo = w.Rlo;

@@ -54,10 +54,11 @@ SHP_DEV void block_add(float v, float* dst) {
   }
 }
 
-__global__ void k_reset(Ctl ctl, int batch, int first) {
+__global__ void k_reset(Ctl ctl, int batch, int first, int start_degree) {
   count_kernel_run();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
+  if (start_degree > 0 && ctl.deg != nullptr) ctl.deg[b] = start_degree;
   BlockState& s = ctl.bs[b];
   if (first) {
     s.status = ST_OK;
@@ -156,11 +157,11 @@ __global__ void __launch_bounds__(EW_THREADS)
 }
 
 __global__ void __launch_bounds__(EW_THREADS)
-    k_gform_d1(const float* Rhi, const float* Rlo, int64_t n, Ctl ctl, int fmt, void* ghi,
-               float* glo, void* g2hi, float* g2lo) {
+    k_gform_d1(const float* Rhi, const float* Rlo, int64_t n, Ctl ctl, const int* active,
+               int fmt, void* ghi, float* glo, void* g2hi, float* g2lo) {
   count_kernel_run();
   const int b = blockIdx.y;
-  if (ctl.active[b] == 0) return;
+  if (active[b] == 0) return;
   const float a = ctl.alpha[b];
   const int64_t nn = n * n;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
@@ -272,8 +273,9 @@ __global__ void k_write_status(Ctl ctl, int batch, int* out) {
 
 }  // namespace
 
-cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st) {
-  k_reset<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, first_pass);
+cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st,
+                       int start_degree) {
+  k_reset<<<(batch + 127) / 128, 128, 0, st>>>(ctl, batch, first_pass, start_degree);
   return cudaGetLastError();
 }
 
@@ -302,9 +304,10 @@ cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* 
 }
 
 cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, const Ctl& ctl,
-                     int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st) {
-  k_gform_d1<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(Rhi, Rlo, n, ctl, fmt, ghi, glo,
-                                                           g2hi, g2lo);
+                     int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st,
+                     const int* active) {
+  k_gform_d1<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(
+      Rhi, Rlo, n, ctl, active != nullptr ? active : ctl.active, fmt, ghi, glo, g2hi, g2lo);
   return cudaGetLastError();
 }
 

@@ -102,10 +102,23 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
 // Gram of V_d..V_{2d+1}, the
 // quartic J(alpha) and its minimiser on [lo, hi]; writes alpha[b] and, when
 // non-null, J_coef[b][5] and report_alpha[b * stride + slot (+ *it)].
+// Adaptive degree state of a call (all [batch] device arrays): the current
+// degree of each block, the active blocks at degree 1 and 2 (masks of the
+// launches that form Delta), and the report's degree trajectory (may be null).
+struct AdaptiveDeg {
+  int enabled;
+  float raise_above;
+  int* deg;
+  int* act1;
+  int* act2;
+  int* rep_degree;
+};
+// With ad enabled (d = 2): V holds V_1..V_5 and each block fits at its
+// current degree, raising it by the rule of shp_prism_opts.adaptive_degree.
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
-                        const int* it, cudaStream_t st);
+                        const int* it, cudaStream_t st, const AdaptiveDeg* ad = nullptr);
 
 // ---- per-block control (sketch_alpha.cu)
 struct BlockState {
@@ -122,6 +135,9 @@ struct BlockState {
 struct Ctl {
   BlockState* bs;
   int* active;
+  int* deg;       // current degree of each block (adaptive degree)
+  int* act1;      // active blocks at degree 1 / 2 (adaptive degree)
+  int* act2;
   double* dnorm;  // ||input||_F^2 per block
   int* tmo;       // ST_ETIMEOUT flags from the GEMM pipeline
   float* alpha;   // alpha_k per block
@@ -142,7 +158,9 @@ cudaError_t loop_step(const Ctl& ctl, int batch, int inc, int max_iter,
 // ---- elementwise (elementwise.cu)
 // Start of a pass: active = 1, counters cleared; first_pass also clears the
 // status, the timeout flags and the input norms; otherwise iters1 = iters.
-cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st);
+// start_degree > 0 also sets every block's degree (adaptive degree).
+cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t st,
+                       int start_degree = 0);
 // dnorm[b] += ||X[b]||_F^2 (X fp32 or bf16, rows x cols contiguous per block).
 cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
                        cudaStream_t st);
@@ -156,8 +174,10 @@ cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* 
                             float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
                             float* Rs, cudaStream_t st);
 // Delta = alpha[b] R (d = 1) in `fmt`; I + Delta into (g2hi, g2lo) when non-null.
+// `active` overrides ctl.active (the degree-1 mask under adaptive degree).
 cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, const Ctl& ctl,
-                     int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st);
+                     int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st,
+                     const int* active = nullptr);
 // X_out[b] = c_b^e * S[iters_b % 2][b] (hi + lo), S = the two ping-pong slots.
 cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_exponent,
                            const float* const* Shi, const float* const* Slo, float* X_out,
@@ -186,10 +206,11 @@ bool small_block_ok(int64_t m, int64_t n, int p);
 cudaError_t small_inv_root(const float* A, int n, int batch, int power,
                            const shp_prism_opts& o, const float* S, float* X,
                            int* rep_status, int* rep_iters, float* rep_resid, float* rep_alpha,
-                           cudaStream_t st);
+                           int* rep_degree, cudaStream_t st);
 // sign: the sign function of a symmetric square G (R = I - X X).
 cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
                         const float* S, float* X, int* rep_status, int* rep_iters,
-                        float* rep_resid, float* rep_alpha, bool sign, cudaStream_t st);
+                        float* rep_resid, float* rep_alpha, int* rep_degree, bool sign,
+                        cudaStream_t st);
 
 }  // namespace shp

@@ -107,63 +107,121 @@ __global__ void __launch_bounds__(SK_THREADS)
 
 constexpr int AL_THREADS = 256;
 
-__global__ void __launch_bounds__(AL_THREADS)
-    k_alpha(const float* __restrict__ V, int64_t n, int p, int d, int64_t vbs, float lo,
-            float hi, int fixed, const int* __restrict__ active, float* __restrict__ alpha,
-            double* __restrict__ Jc, float* __restrict__ rep, int64_t rep_stride, int rep_slot,
-            const int* __restrict__ it) {
+// Per-block alpha of one iteration.  Without adaptive degree: the Gram of
+// V_d..V_{2d+1}, the quartic and its minimiser on [lo, hi].  With adaptive
+// degree (d = 2): the Gram of V_1..V_5 at once; a block at degree 1 fits on
+// V_1..V_3 over [1/2, hi] and, when sqrt(J_1(alpha*)) / ||V_1||_F exceeds
+// raise_above, moves to degree 2 (V_2..V_5 over [3/8, hi]) for the rest of
+// the pass.  act1/act2 then mark the active blocks at each degree for the
+// masked launches that form Delta.
+struct AlphaArgs {
+  const float* V;
+  int64_t n, vbs;
+  int p, d, fixed;
+  float lo, hi;
+  const int* active;
+  float* alpha;
+  double* Jc;
+  float* rep;
+  int64_t rep_stride;
+  int rep_slot;
+  const int* it;
+  int adaptive;
+  float raise_above;
+  int* deg;
+  int* act1;
+  int* act2;
+  int* rep_deg;
+};
+
+__global__ void __launch_bounds__(AL_THREADS) k_alpha(AlphaArgs g) {
   count_kernel_run();
   const int b = blockIdx.x;
-  if (active != nullptr && active[b] == 0) return;
-  if (it != nullptr) rep_slot += *it;
-  if (fixed) {  // plain Taylor step: alpha = lo, no sketch needed
-    if (threadIdx.x == 0) {
-      alpha[b] = lo;
-      if (rep != nullptr) rep[b * rep_stride + rep_slot] = lo;
+  if (g.active != nullptr && g.active[b] == 0) {
+    if (g.adaptive && threadIdx.x == 0) {
+      g.act1[b] = 0;
+      g.act2[b] = 0;
     }
     return;
   }
-  const int nv = d + 2;               // V_d .. V_{2d+1}
-  const int64_t len = n * p;
-  const float* Vb = V + b * vbs + static_cast<int64_t>(d) * len;
-  double part[10];
+  const int rep_slot = g.rep_slot + (g.it != nullptr ? *g.it : 0);
+  if (g.fixed) {  // plain Taylor step: alpha = lo, no sketch needed
+    if (threadIdx.x == 0) {
+      g.alpha[b] = g.lo;
+      if (g.rep != nullptr) g.rep[b * g.rep_stride + rep_slot] = g.lo;
+      if (g.rep_deg != nullptr) g.rep_deg[b * g.rep_stride + rep_slot] = g.d;
+    }
+    return;
+  }
+  const int first = g.adaptive ? 1 : g.d;     // V_first .. V_{first + nv - 1}
+  const int nv = g.adaptive ? 5 : g.d + 2;
+  const int64_t len = g.n * g.p;
+  const float* Vb = g.V + b * g.vbs + static_cast<int64_t>(first) * len;
+  double part[15];
 #pragma unroll
-  for (int i = 0; i < 10; ++i) part[i] = 0.0;
+  for (int i = 0; i < 15; ++i) part[i] = 0.0;
   for (int64_t e = threadIdx.x; e < len; e += AL_THREADS) {
-    double x[4];
+    double x[5];
     for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(Vb[i * len + e]);
     int idx = 0;
     for (int i = 0; i < nv; ++i)
       for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
   }
-  __shared__ double red[AL_THREADS / 32][10];
+  __shared__ double red[AL_THREADS / 32][15];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < 10; ++i) {
+  for (int i = 0; i < 15; ++i) {
     const double s = warp_sum(part[i]);
     if (lane == 0) red[warp][i] = s;
   }
   __syncthreads();
   if (threadIdx.x >= 32) return;  // warp 0 forms J and finds its minimiser
-  double M[4][4];
+  double G[5][5];
   {
     int idx = 0;
     for (int i = 0; i < nv; ++i)
       for (int j = i; j < nv; ++j) {
         double s = 0.0;
         for (int w = 0; w < AL_THREADS / 32; ++w) s += red[w][idx];
-        M[i][j] = M[j][i] = s;
+        G[i][j] = G[j][i] = s;
         ++idx;
       }
   }
+  // fit at degree e on the Gram block starting at V_e (offset e - first)
+  auto fit = [&](int e, double lo, double* coef) {
+    double M[4][4];
+    const int o = e - first;
+    for (int i = 0; i < e + 2; ++i)
+      for (int j = 0; j < e + 2; ++j) M[i][j] = G[o + i][o + j];
+    quartic_from_gram(M, e, coef);
+    return argmin_quartic_warp(coef, lo, static_cast<double>(g.hi));
+  };
   double coef[5];
-  quartic_from_gram(M, d, coef);
-  const double a = argmin_quartic_warp(coef, static_cast<double>(lo), static_cast<double>(hi));
+  int dcur = g.d;
+  double a;
+  if (!g.adaptive) {
+    a = fit(g.d, static_cast<double>(g.lo), coef);
+  } else {
+    dcur = g.deg[b];
+    if (dcur == 1) {
+      a = fit(1, 0.5, coef);
+      const double J = poly4(coef, a), base = G[0][0];  // ||V_1||^2 = ||R_k S_k||^2
+      if (base > 0.0 && sqrt(fmax(J, 0.0) / base) > static_cast<double>(g.raise_above))
+        dcur = 2;
+    }
+    if (dcur == 2) a = fit(2, 0.375, coef);
+  }
   if (threadIdx.x != 0) return;
-  alpha[b] = static_cast<float>(a);
-  if (Jc != nullptr)
-    for (int i = 0; i < 5; ++i) Jc[b * 5 + i] = coef[i];
-  if (rep != nullptr) rep[b * rep_stride + rep_slot] = static_cast<float>(a);
+  g.alpha[b] = static_cast<float>(a);
+  if (g.Jc != nullptr)
+    for (int i = 0; i < 5; ++i) g.Jc[b * 5 + i] = coef[i];
+  if (g.rep != nullptr) g.rep[b * g.rep_stride + rep_slot] = static_cast<float>(a);
+  if (g.rep_deg != nullptr) g.rep_deg[b * g.rep_stride + rep_slot] = dcur;
+  if (g.adaptive) {
+    g.deg[b] = dcur;
+    g.act1[b] = dcur == 1;
+    g.act2[b] = dcur == 2;
+  }
 }
 
 __global__ void k_control(BlockState* bs, int* active, const int* it, int batch, int64_t n,
@@ -216,11 +274,31 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
-                        const int* it, cudaStream_t st) {
+                        const int* it, cudaStream_t st, const AdaptiveDeg* ad) {
   if (batch <= 0) return cudaSuccess;
-  const int64_t vbs = static_cast<int64_t>(2 * d + 2) * n * p;
-  k_alpha<<<batch, AL_THREADS, 0, st>>>(V, n, p, d, vbs, lo, hi, fixed_alpha, active, alpha,
-                                        J_coef, report_alpha, report_stride, report_slot, it);
+  AlphaArgs g;
+  g.V = V;
+  g.n = n;
+  g.vbs = static_cast<int64_t>(2 * d + 2) * n * p;
+  g.p = p;
+  g.d = d;
+  g.fixed = fixed_alpha;
+  g.lo = lo;
+  g.hi = hi;
+  g.active = active;
+  g.alpha = alpha;
+  g.Jc = J_coef;
+  g.rep = report_alpha;
+  g.rep_stride = report_stride;
+  g.rep_slot = report_slot;
+  g.it = it;
+  g.adaptive = ad != nullptr && ad->enabled;
+  g.raise_above = ad != nullptr ? ad->raise_above : 0.f;
+  g.deg = ad != nullptr ? ad->deg : nullptr;
+  g.act1 = ad != nullptr ? ad->act1 : nullptr;
+  g.act2 = ad != nullptr ? ad->act2 : nullptr;
+  g.rep_deg = ad != nullptr ? ad->rep_degree : nullptr;
+  k_alpha<<<batch, AL_THREADS, 0, st>>>(g);
   return cudaGetLastError();
 }
 

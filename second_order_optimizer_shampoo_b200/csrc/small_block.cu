@@ -38,8 +38,8 @@ constexpr int SB_SMEM = 4 * SB_MAT * static_cast<int>(sizeof(float));
 static_assert(4 * SB_NMAX * SB_PMAX <= SB_MAT, "sketch slots must fit one matrix buffer");
 
 struct SmallCfg {
-  int d, p, max_iter, fixed_alpha;
-  float lo, hi, tol, stall_below, stall_ratio;
+  int d, p, max_iter, fixed_alpha, adaptive;
+  float lo, hi, tol, stall_below, stall_ratio, raise_above;
 };
 
 // Sum over the CTA; every thread receives the result.
@@ -168,37 +168,31 @@ SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, int r0,
   return W;
 }
 
-// Sketched alpha of one iteration: V_j = R^j S_k for j <= 2d+1 (S_k = n x p
-// slice in HBM), Gram of V_d..V_{2d+1} in fp64, argmin of the quartic on
-// [lo, hi].  V is a free matrix buffer: slot j - d holds V_j (d = 2 parks
-// V_1 in slot 2 and S in slot 3 until they are overwritten).
-SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float* Sk, float* V,
-                           double (*red)[10], float* s_alpha) {
-  const int p = o.p, d = o.d, np = n * p, tid = threadIdx.x;
-  float* slot[4] = {V, V + np, V + 2 * np, V + 3 * np};
-  for (int e = tid; e < np; e += SB_THREADS) slot[3][e] = Sk[e];
-  __syncthreads();
-  const float* src = slot[3];
-  for (int j = 1; j <= 2 * d + 1; ++j) {
-    float* dst = j >= d ? slot[j - d] : slot[2];
-    for (int e = tid; e < np; e += SB_THREADS) {
-      const int row = e / p, col = e - row * p;
-      const float* Rr = R + row * SB_LD;
-      float s = 0.f;
+// Vout = R Vin (n x p, row-major) by the whole CTA.
+SHP_DEV void sketch_power(const float* R, const float* Vin, float* Vout, int n, int p) {
+  for (int e = threadIdx.x; e < n * p; e += SB_THREADS) {
+    const int row = e / p, col = e - row * p;
+    const float* Rr = R + row * SB_LD;
+    float s = 0.f;
 #pragma unroll 8
-      for (int k = 0; k < n; ++k) s = fmaf(Rr[k], src[k * p + col], s);
-      dst[e] = s;
-    }
-    __syncthreads();
-    src = dst;
+    for (int k = 0; k < n; ++k) s = fmaf(Rr[k], Vin[k * p + col], s);
+    Vout[e] = s;
   }
-  const int nv = d + 2;
+  __syncthreads();
+}
+
+// alpha of degree e from V_e..V_{2e+1} (slot (j - 1) & 3 holds V_j): fp64
+// Gram, quartic, minimiser on [lo, hi] by warp 0; every thread gets alpha and,
+// through *s_ratio, sqrt(J(alpha)) / ||V_1||_F (the predicted contraction).
+SHP_DEV float fit_degree(float* const* slot, int np, int e, double lo, double hi,
+                         double (*red)[10], float* s_alpha, float* s_ratio) {
+  const int tid = threadIdx.x, nv = e + 2;
   double part[10];
 #pragma unroll
   for (int i = 0; i < 10; ++i) part[i] = 0.0;
-  for (int e = tid; e < np; e += SB_THREADS) {
+  for (int q = tid; q < np; q += SB_THREADS) {
     double x[4];
-    for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(slot[i][e]);
+    for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(slot[(e + i - 1) & 3][q]);
     int idx = 0;
     for (int i = 0; i < nv; ++i)
       for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
@@ -221,22 +215,53 @@ SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float
         ++idx;
       }
     double coef[5];
-    quartic_from_gram(M, d, coef);
-    const double a =
-        argmin_quartic_warp(coef, static_cast<double>(o.lo), static_cast<double>(o.hi));
-    if (tid == 0) *s_alpha = static_cast<float>(a);
+    quartic_from_gram(M, e, coef);
+    const double a = argmin_quartic_warp(coef, lo, hi);
+    if (tid == 0) {
+      *s_alpha = static_cast<float>(a);
+      const double base = M[0][0];  // ||V_1||^2 when e = 1
+      *s_ratio = base > 0.0 ? static_cast<float>(sqrt(fmax(poly4(coef, a), 0.0) / base)) : 0.f;
+    }
   }
   __syncthreads();
   return *s_alpha;
 }
 
+// Sketched alpha of one iteration at degree *deg: V_j = R^j S_k (S_k = n x p
+// slice in HBM), slot (j - 1) & 3 of the free buffer V holds V_j (S sits in
+// slot 3 until V_4 replaces it).  With adaptive degree a block at degree 1
+// fits on V_1..V_3 and, when the predicted contraction exceeds raise_above,
+// continues to V_5 and fits at degree 2, which *deg keeps from then on.
+SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float* Sk, float* V,
+                           int* deg, double (*red)[10], float* s_alpha, float* s_ratio) {
+  const int p = o.p, np = n * p;
+  float* slot[4] = {V, V + np, V + 2 * np, V + 3 * np};
+  for (int e = threadIdx.x; e < np; e += SB_THREADS) slot[3][e] = Sk[e];
+  __syncthreads();
+  sketch_power(R, slot[3], slot[0], n, p);  // V_1
+  sketch_power(R, slot[0], slot[1], n, p);  // V_2
+  sketch_power(R, slot[1], slot[2], n, p);  // V_3
+  float a = 0.f;
+  if (*deg == 1) {
+    a = fit_degree(slot, np, 1, o.adaptive ? 0.5 : static_cast<double>(o.lo),
+                   static_cast<double>(o.hi), red, s_alpha, s_ratio);
+    if (!(o.adaptive && *s_ratio > o.raise_above)) return a;
+    *deg = 2;
+  }
+  sketch_power(R, slot[2], slot[3], n, p);  // V_4
+  sketch_power(R, slot[3], slot[0], n, p);  // V_5
+  return fit_degree(slot, np, 2, o.adaptive ? 0.375 : static_cast<double>(o.lo),
+                    static_cast<double>(o.hi), red, s_alpha, s_ratio);
+}
+
 // Report slots: resid[b][pass][k] (max_iter + 1 per pass), alpha[b][pass][k]
-// (max_iter per pass), iters[b][pass], status[b].
+// and degree[b][pass][k] (max_iter per pass), iters[b][pass], status[b].
 struct SmallReport {
   int* status;
   int* iters;
   float* resid;
   float* alpha;
+  int* degree;
 };
 
 // Coupled Newton-Schulz for A^(1/2), A^(-1/2) (one pass) or A^(-1/4) (a
@@ -247,7 +272,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   count_kernel_run();
   extern __shared__ __align__(16) float sm[];
   __shared__ double red[SB_THREADS / 32][10];
-  __shared__ float s_alpha;
+  __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
   const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
   const int64_t nn = static_cast<int64_t>(n) * n;
@@ -282,6 +307,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
     }
     double n2 = block_sum(nrm, red[0]);
     float prev = INFINITY;
+    int deg = o.adaptive ? 1 : o.d;  // the degree of g for this pass (adaptive degree)
     for (int k = 0;; ++k) {
       if (k > 0) n2 = block_sum(residual<false>(Z, Y, n, n, R, r0, c0), red[0]);
       // every thread evaluates the stop rule on the same reduced norm
@@ -297,10 +323,11 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
       const float alpha =
           o.fixed_alpha ? o.lo
                         : sketch_alpha(R, n, o, S + (static_cast<int64_t>(pass) * mi + k) * n * o.p,
-                                       W, red, &s_alpha);
+                                       W, &deg, red, &s_alpha, &s_ratio);
       if (tid == 0 && rep.alpha != nullptr) rep.alpha[(2 * b + pass) * mi + k] = alpha;
-      float* D = form_delta(o.d, alpha, R, W, n, r0, c0);
-      float* T = o.d == 1 ? W : R;  // the buffer Delta does not occupy
+      if (tid == 0 && rep.degree != nullptr) rep.degree[(2 * b + pass) * mi + k] = deg;
+      float* D = form_delta(deg, alpha, R, W, n, r0, c0);
+      float* T = deg == 1 ? W : R;  // the buffer Delta does not occupy
       axpy_mm(Y, D, Y, n, n, n, T, r0, c0);  // Y_{k+1} = Y_k + Y_k Delta
       __syncthreads();
       if (k == 0) {  // Z_1 = I + Delta
@@ -315,7 +342,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
       float* oldZ = Z;
       Z = Y;
       Y = T;
-      if (o.d == 1)
+      if (deg == 1)
         W = oldZ;
       else
         R = oldZ;
@@ -350,7 +377,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   count_kernel_run();
   extern __shared__ __align__(16) float sm[];
   __shared__ double red[SB_THREADS / 32][10];
-  __shared__ float s_alpha;
+  __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
   const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
   const bool tall = m >= n;
@@ -378,6 +405,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   const int mi = o.max_iter;
   int status = ST_OK;
   float prev = INFINITY;
+  int deg = o.adaptive ? 1 : o.d;
   for (int k = 0;; ++k) {
     // R = I - X^T X (polar) or I - X X (sign of a symmetric X, m == n)
     const double n2 = block_sum(sign ? residual<false>(X, X, rows, k_n, R, r0, c0)
@@ -394,10 +422,11 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
     }
     const float alpha =
         o.fixed_alpha ? o.lo
-                      : sketch_alpha(R, k_n, o, S + static_cast<int64_t>(k) * k_n * o.p, T, red,
-                                     &s_alpha);
+                      : sketch_alpha(R, k_n, o, S + static_cast<int64_t>(k) * k_n * o.p, T, &deg,
+                                     red, &s_alpha, &s_ratio);
     if (tid == 0 && rep.alpha != nullptr) rep.alpha[2 * b * mi + k] = alpha;
-    float* D = form_delta(o.d, alpha, R, W, k_n, r0, c0);
+    if (tid == 0 && rep.degree != nullptr) rep.degree[2 * b * mi + k] = deg;
+    float* D = form_delta(deg, alpha, R, W, k_n, r0, c0);
     axpy_mm(X, D, X, k_n, rows, k_n, T, r0, c0);  // X_{k+1} = X_k + X_k Delta
     __syncthreads();
     float* t = X;
@@ -424,6 +453,8 @@ SmallCfg make_cfg(const shp_prism_opts& s) {
   c.tol = s.tol;
   c.stall_below = s.stall_below;
   c.stall_ratio = s.stall_ratio;
+  c.adaptive = s.adaptive_degree;
+  c.raise_above = s.raise_above;
   return c;
 }
 
@@ -440,25 +471,27 @@ bool small_block_ok(int64_t m, int64_t n, int p) {
 
 cudaError_t small_inv_root(const float* A, int n, int batch, int power, const shp_prism_opts& o,
                            const float* S, float* X, int* rep_status, int* rep_iters,
-                           float* rep_resid, float* rep_alpha, cudaStream_t st) {
+                           float* rep_resid, float* rep_alpha, int* rep_degree, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
   cudaError_t e = prepare(k_small_inv_root);
   if (e != cudaSuccess) return e;
   const int npass = power == SHP_POW_INV4 ? 2 : 1;
   k_small_inv_root<<<batch, SB_THREADS, SB_SMEM, st>>>(
-      A, n, npass, power, make_cfg(o), S, X, SmallReport{rep_status, rep_iters, rep_resid, rep_alpha});
+      A, n, npass, power, make_cfg(o), S, X,
+      SmallReport{rep_status, rep_iters, rep_resid, rep_alpha, rep_degree});
   return cudaGetLastError();
 }
 
 cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
                         const float* S, float* X, int* rep_status, int* rep_iters,
-                        float* rep_resid, float* rep_alpha, bool sign, cudaStream_t st) {
+                        float* rep_resid, float* rep_alpha, int* rep_degree, bool sign,
+                        cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
   cudaError_t e = prepare(k_small_polar);
   if (e != cudaSuccess) return e;
   k_small_polar<<<batch, SB_THREADS, SB_SMEM, st>>>(
-      G, m, n, make_cfg(o), S, X, SmallReport{rep_status, rep_iters, rep_resid, rep_alpha},
-      sign ? 1 : 0);
+      G, m, n, make_cfg(o), S, X,
+      SmallReport{rep_status, rep_iters, rep_resid, rep_alpha, rep_degree}, sign ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -49,11 +49,13 @@ def _stream():
 
 
 def make_opts(d=2, p=8, lo=None, hi=1.0, tol=1e-3, max_iter=40, prec="3xtf32",
-              fixed_alpha=False, stall_below=0.05, stall_ratio=0.75) -> A.PrismOpts:
+              fixed_alpha=False, stall_below=0.05, stall_ratio=0.75, adaptive_degree=False,
+              raise_above=0.9) -> A.PrismOpts:
     if lo is None:
         lo = 0.5 if d == 1 else 0.375
     return A.PrismOpts(d, p, lo, hi, tol, max_iter, _PREC[prec] if isinstance(prec, str) else prec,
-                       int(bool(fixed_alpha)), stall_below, stall_ratio)
+                       int(bool(fixed_alpha)), stall_below, stall_ratio,
+                       int(bool(adaptive_degree)), raise_above)
 
 
 def shp_workspace_bytes(op: int, m: int, n: int, batch: int, opts: A.PrismOpts | None = None) -> int:
@@ -117,18 +119,22 @@ def _report(batch, max_iter, device):
         "iters": torch.full((batch, 2), -1, dtype=torch.int32, device=device),
         "resid": torch.full((batch, 2, max_iter + 1), float("nan"), dtype=torch.float32, device=device),
         "alpha": torch.full((batch, 2, max_iter), float("nan"), dtype=torch.float32, device=device),
+        "degree": torch.full((batch, 2, max_iter), -1, dtype=torch.int32, device=device),
     }
 
 
 def _report_struct(rep):
     if rep is None:
         return None
+    deg = rep.get("degree")
     return ctypes.byref(A.PrismReport(rep["status"].data_ptr(), rep["iters"].data_ptr(),
-                                      rep["resid"].data_ptr(), rep["alpha"].data_ptr()))
+                                      rep["resid"].data_ptr(), rep["alpha"].data_ptr(),
+                                      deg.data_ptr() if deg is not None else None))
 
 
 def make_report(batch, max_iter, device):
-    """Device tensors for the per-block trajectory (status, iters, resid, alpha)."""
+    """Device tensors for the per-block trajectory (status, iters, resid, alpha,
+    degree)."""
     return _report(batch, max_iter, device)
 
 

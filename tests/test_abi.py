@@ -99,6 +99,20 @@ def test_invalid_arguments_rejected_before_launch():
                            None) == A.SHP_EINVAL
 
 
+def test_adaptive_degree_validation():
+    """Adaptive degree needs d = 2 (the degree it raises to), a fitted alpha
+    and a threshold >= 0."""
+    L = A.lib()
+    fake = ctypes.c_void_p(0x10000)
+    for bad in (opts(adaptive_degree=1, d=1), opts(adaptive_degree=1, fixed_alpha=1),
+                opts(adaptive_degree=1, raise_above=-0.5)):
+        assert L.shp_workspace_bytes(A.SHP_OP_INV_ROOT, 1024, 1024, 4, ctypes.byref(bad)) == 0
+        assert L.matfn_inv_root(fake, 64, 1, 0, ctypes.byref(bad), fake, 80, fake, None, fake,
+                                1 << 40, None) == A.SHP_EINVAL
+    good = opts(adaptive_degree=1, raise_above=0.9)
+    assert L.shp_workspace_bytes(A.SHP_OP_INV_ROOT, 1024, 1024, 4, ctypes.byref(good)) > 0
+
+
 def test_apply_ex_validation():
     L = A.lib()
     fake = ctypes.c_void_p(0x10000)

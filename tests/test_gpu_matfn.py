@@ -30,7 +30,8 @@ def run_inv_root(A, power, d, p, tol, max_iter, prec, S, **kw):
 def oracle_opts(opts, **kw):
     base = dict(d=opts.d, p=opts.p, lo=opts.lo, hi=opts.hi, tol=opts.tol, max_iter=opts.max_iter,
                 fixed_alpha=bool(opts.fixed_alpha), stall_below=opts.stall_below,
-                stall_ratio=opts.stall_ratio)
+                stall_ratio=opts.stall_ratio, adaptive_degree=bool(opts.adaptive_degree),
+                raise_above=opts.raise_above)
     base.update(kw)
     return o.PrismOpts(**base)
 
@@ -261,3 +262,62 @@ def test_sign_bf16_and_spd():
     X2, rep2 = P.matfn_sign(to_dev(torch, spd), opts2, to_dev(torch, S))
     assert to_host(rep2["status"])[0] == o.OK
     np.testing.assert_allclose(to_host(X2)[0], np.eye(n), atol=1e-5)
+
+
+# ------------------------------------------------------------------ adaptive degree
+def mixed_batch(n, seed):
+    """Blocks that keep degree 1 (cond 10) and blocks that raise to 2 at the
+    first step (cond 1e3); see the thresholds in the test."""
+    easy = synth.spd_batch(n, 2, 1e-1, 1.0, seed)
+    hard = synth.spd_batch(n, 2, 1e-3, 1.0, seed + 1)
+    return np.stack([easy[0], hard[0], easy[1], hard[1]])
+
+
+# raise_above between the first-step predicted contractions of the two kinds
+# of blocks (float64: n = 48 easy 0.70-0.72, hard 0.89-0.90; n = 256 easy
+# 0.86, hard 0.93); the oracle's degree trajectories do not change within
+# +-0.015 of it.  The split path's bound at cond 1e3 is 3e-5 (as above); the
+# on-chip path computes in fp32 (1e-5).
+@pytest.mark.parametrize("n,threshold,tol_x", [(48, 0.8, 1e-5), (256, 0.895, TOL_3X_COND1E3)])
+def test_adaptive_degree_inv_root(n, threshold, tol_x):
+    """Per-block degrees in one batch (on chip at n = 48, masked launches at
+    n = 256): degree trajectories, alphas and roots against the oracle."""
+    P = prism()
+    A = mixed_batch(n, 91)
+    S = synth.sketch_stack(80, n, 8, 1091)
+    opts = P.make_opts(d=2, p=8, tol=1e-6, max_iter=40, prec="3xtf32", adaptive_degree=True,
+                       raise_above=threshold)
+    X, rep = P.matfn_inv_root(to_dev(torch, A), "inv4", opts, to_dev(torch, S))
+    X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
+    for b in range(4):
+        assert rep["status"][b] == o.OK, rep["status"]
+        it = rep["iters"][b]
+        Xo, infos = o.inv_root_ref(A[b], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
+        for ps, info in enumerate(infos):
+            assert list(rep["degree"][b, ps, :it[ps]]) == info.degree, (b, ps)
+            np.testing.assert_allclose(rep["alpha"][b, ps, :it[ps]], info.alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= tol_x
+    # the easy blocks stay at degree 1 for the first pass, the hard ones raise at once
+    assert rep["degree"][0, 0, 0] == 1 and rep["degree"][1, 0, 0] == 2
+
+
+@pytest.mark.parametrize("shape", [(48, 40), (320, 256)])
+def test_adaptive_degree_polar(shape):
+    """Frobenius normalisation starts every singular value near 1/sqrt(n), so
+    the polar iteration raises to degree 2 at once: the masked R R launch and
+    the on-chip degree switch, against the oracle."""
+    P = prism()
+    m, n = shape
+    G = synth.gaussian((2, m, n), 1.0, 93)
+    S = synth.sketch_stack(40, n, 8, 1093)
+    opts = P.make_opts(d=2, p=8, tol=1e-6, max_iter=40, prec="3xtf32", adaptive_degree=True,
+                       raise_above=0.9)
+    X, rep = P.matfn_polar(to_dev(torch, G), opts, to_dev(torch, S))
+    X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
+    for b in range(2):
+        assert rep["status"][b] == o.OK
+        it = rep["iters"][b][0]
+        Xo, infos = o.polar_ref(G[b], oracle_opts(opts), S, force_iters=it)
+        assert list(rep["degree"][b, 0, :it]) == infos[0].degree
+        np.testing.assert_allclose(rep["alpha"][b, 0, :it], infos[0].alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= 1e-5
