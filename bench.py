@@ -365,6 +365,39 @@ def gemm_count_leg(args, dev, stream, A):
     return out
 
 
+SWEEP_SIGMA_MIN = (1e-1, 1e-2, 1e-3, 1e-4)
+
+
+def sigma_sweep_leg(args, dev, stream):
+    """Polar factor of 8 matrices 1024 x 1024 with singular values log-uniform
+    on [sigma_min, 1], to ||I - X^T X||_F / sqrt(n) <= 1e-6 (split path):
+    iterations and GEMMs of PRISM d = 2 against the fixed-coefficient d = 2
+    and d = 1 iterations, per sigma_min."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism, synth
+    n, batch, mi = 1024, 8, 60
+    S = torch.from_numpy(synth.sketch_stack(mi, n, 8, 1006)).to(dev)
+    out = {"workload": "polar_8x1024sq_sigma_min_sweep_tol1e-6_3xtf32", "rows": []}
+    for smin in SWEEP_SIGMA_MIN:
+        G = torch.from_numpy(synth.singular_spectrum(n, n, smin, batch, 106)).to(dev)
+        row = {"sigma_min": smin}
+        for name, d, fixed in (("prism_d2", 2, False), ("taylor_d2", 2, True),
+                               ("taylor_d1", 1, True)):
+            opts = prism.make_opts(d=d, p=8, tol=1e-6, max_iter=mi, prec="3xtf32",
+                                   fixed_alpha=fixed)
+            _, rep = prism.matfn_polar(G, opts, S)
+            torch.cuda.synchronize()
+            it = rep["iters"][:, 0].cpu().numpy()
+            # per update: X^T X, R R (d = 2 only), X Delta; plus the final residual
+            gem = [int(k) * (2 if d == 1 else 3) + 1 for k in it]
+            row[name] = {"median_iters": float(np.median(it)),
+                         "median_gemms": float(np.median(gem)),
+                         "status_ok": int((rep["status"].cpu().numpy() == 0).sum())}
+        out["rows"].append(row)
+    return out
+
+
 def single_block_leg(args, dev, stream):
     """Config 1 as single calls: one 64 x 64 A^(-1/4) (d = 1, p = 4, tol 1e-6)
     and one 64 x 32 polar factor, microseconds per call."""
@@ -652,6 +685,7 @@ def main():
     step2 = shampoo_step_leg(args, dev, stream) if extra else None
     counts = gemm_count_leg(args, dev, stream, A) if extra else None
     single = single_block_leg(args, dev, stream) if extra else None
+    sweep = sigma_sweep_leg(args, dev, stream) if extra else None
     large = large_sqrt_leg(args, dev, stream) if args.large and world == 1 else None
     small = None if args.no_small else small_block_leg(args, dev, stream,
                                                         peaks.get("sm_max_mhz", 1965.0))
@@ -689,6 +723,7 @@ def main():
             "shampoo_step_1024": step2,
             "gemms_to_residual": counts,
             "single_64": single,
+            "polar_sigma_sweep": sweep,
             "sqrt_10240": large,
             "cpu_baseline": cpu,
             "clocks": clocks,

@@ -21,6 +21,7 @@ import numpy as np
 __all__ = [
     "spd_block",
     "spd_batch",
+    "singular_spectrum",
     "gaussian",
     "lowrank_noise",
     "lowrank_noise_batch",
@@ -66,6 +67,24 @@ def spd_batch(n: int, batch: int, lam_lo: float, lam_hi: float, seed: int,
     out = np.empty((len(idx), n, n), dtype=np.float32)
     for j, i in enumerate(idx):
         out[j] = spd_block(n, lam_lo, lam_hi, seed, i)
+    return out
+
+
+def singular_spectrum(m: int, n: int, sigma_min: float, batch: int, seed: int) -> np.ndarray:
+    """[batch, m, n] fp32 matrices U diag(sigma) V^T (m >= n) with U, V the
+    orthogonal factors of QR factorisations of N(0,1) matrices (signs fixed)
+    and sigma log-uniform on [sigma_min, 1], largest set to 1: the sigma_min
+    sweep of the polar iteration."""
+    out = np.empty((batch, m, n), dtype=np.float32)
+    for b in range(batch):
+        g = _rng(seed, b)
+        U, Ru = np.linalg.qr(g.standard_normal((m, n)))
+        U = U * np.sign(np.diag(Ru))[None, :]
+        V, Rv = np.linalg.qr(g.standard_normal((n, n)))
+        V = V * np.sign(np.diag(Rv))[None, :]
+        sig = np.exp(g.uniform(np.log(sigma_min), 0.0, size=n))
+        sig[0] = 1.0
+        out[b] = ((U * sig[None, :]) @ V.T).astype(np.float32)
     return out
 
 
