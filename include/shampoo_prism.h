@@ -168,6 +168,22 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
                 const shp_prism_opts* opts, const float* S, int64_t S_count, void* X_out,
                 const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
 
+/* Polar factors of a batch of small blocks of different shapes, each on chip
+ * (one CTA per block, fp32 products): block b is the row-major m_b x n_b
+ * matrix at G + offsets[b] and its factor goes to X_out + offsets[b].
+ *   dims    [batch][2] int32 (m_b, n_b), each in 4..64 and a multiple of 4
+ *   offsets [batch] int64 element offsets of the blocks in G and X_out
+ *   S       [S_count][64][p] fp32 (p <= 16); block b uses the first
+ *           min(m_b, n_b) rows of slice k at iteration k
+ * dims and offsets are DEVICE arrays, read by the kernel: a block whose
+ * dims are out of range gets report.status SHP_EINVAL and is left untouched.
+ * The batched polar decomposition of variable-size diagonal blocks (e.g. the
+ * groups of close eigenvalues of a block-rotation optimizer). */
+int matfn_polar_varsize(const float* G, const int32_t* dims, const int64_t* offsets,
+                        int64_t batch, const shp_prism_opts* opts, const float* S,
+                        int64_t S_count, float* X_out, const shp_prism_report* report,
+                        shp_stream stream);
+
 /* Matrix sign function of a batch of symmetric n x n matrices ([PRISM] Parte I:
  * the residual of sign functions is R_k = I - X_k^2):
  *   X_0 = A / ||A||_F; R_k = I - X_k X_k; stop test; alpha_k from S[k];

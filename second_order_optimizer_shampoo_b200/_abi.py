@@ -24,7 +24,8 @@ SHP_OP_INV_ROOT, SHP_OP_POLAR, SHP_OP_ALPHA_FIT, SHP_OP_APPLY, SHP_OP_GRAM_EMA =
 # fixed device scratch of prism_alpha_fit_noalloc
 SHP_NOALLOC_SCRATCH_BYTES = 4 << 20
 
-EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar", "matfn_sign",
+EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar", "matfn_polar_varsize",
+           "matfn_sign",
            "prism_alpha_fit", "shampoo_apply", "shampoo_apply_ex", "shp_matmul", "shp_split_tf32",
            "shp_kernel_launches", "prism_alpha_fit_noalloc", "shp_status_string",
            "shp_version")
@@ -59,6 +60,8 @@ _SIGS = {
                               ctypes.POINTER(PrismReport), _P, _SZ, _P]),
     "matfn_polar": (_INT, [_P, _INT, _I64, _I64, _I64, ctypes.POINTER(PrismOpts), _P, _I64, _P,
                            ctypes.POINTER(PrismReport), _P, _SZ, _P]),
+    "matfn_polar_varsize": (_INT, [_P, _P, _P, _I64, ctypes.POINTER(PrismOpts), _P, _I64, _P,
+                                   ctypes.POINTER(PrismReport), _P]),
     "matfn_sign": (_INT, [_P, _INT, _I64, _I64, ctypes.POINTER(PrismOpts), _P, _I64, _P,
                           ctypes.POINTER(PrismReport), _P, _SZ, _P]),
     "prism_alpha_fit": (_INT, [_P, _I64, _I64, _P, _INT, _INT, _F, _F, _P, _P, _P, _SZ, _P]),

@@ -911,6 +911,22 @@ int matfn_polar(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
                     false);
 }
 
+int matfn_polar_varsize(const float* G, const int32_t* dims, const int64_t* offsets,
+                        int64_t batch, const shp_prism_opts* o, const float* S, int64_t S_count,
+                        float* X_out, const shp_prism_report* rep, shp_stream stream) {
+  if (!G || !dims || !offsets || !X_out || !opts_ok(o) || batch <= 0) return SHP_EINVAL;
+  if (o->p > 16) return SHP_EINVAL;
+  if (!o->fixed_alpha && (S == nullptr || S_count < o->max_iter)) return SHP_EINVAL;
+  if (!aligned16(G) || !aligned16(X_out)) return SHP_EINVAL;
+  if (batch > INT32_MAX) return SHP_EUNSUPPORTED;
+  CK(small_polar_varsize(G, dims, reinterpret_cast<const int64_t*>(offsets),
+                         static_cast<int>(batch), *o, S, X_out, rep ? rep->status : nullptr,
+                         rep ? rep->iters : nullptr, rep ? rep->resid : nullptr,
+                         rep ? rep->alpha : nullptr, rep ? rep->degree : nullptr,
+                         static_cast<cudaStream_t>(stream)));
+  return SHP_OK;
+}
+
 int matfn_sign(const void* A, int storage, int64_t n, int64_t batch, const shp_prism_opts* o,
                const float* S, int64_t S_count, void* X_out, const shp_prism_report* rep,
                void* ws, size_t ws_bytes, shp_stream stream) {

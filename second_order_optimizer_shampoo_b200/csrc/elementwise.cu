@@ -221,13 +221,14 @@ __global__ void __launch_bounds__(EW_THREADS)
   const int b = blockIdx.y;
   const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
   if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
-  const float inv = c > 0.f ? 1.f / c : 0.f;
+  // X_0 = G / ||G||_F as written: a zero block gives 0/0 and stops with
+  // SHP_ENONFINITE at its first residual
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
        e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
     const int64_t off = b * count + e;
     const float v = gbf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(G)[off])
                           : static_cast<const float*>(G)[off];
-    put(fmt, Xhi, Xlo, off, v * inv);
+    put(fmt, Xhi, Xlo, off, v / c);
   }
 }
 

@@ -28,7 +28,14 @@ enum EpiKind {
 enum OutFmt { OUT_F32 = 0, OUT_SPLIT = 1, OUT_BF16 = 2 };
 
 // Per-block outcome codes (mirrors shp_status in include/shampoo_prism.h).
-enum { ST_OK = 0, ST_ENOCONV = 16, ST_ESTALL = 17, ST_ENONFINITE = 18, ST_ETIMEOUT = 19 };
+enum {
+  ST_OK = 0,
+  ST_EINVAL = 1,  // a block's own arguments are out of range (per-block shapes)
+  ST_ENOCONV = 16,
+  ST_ESTALL = 17,
+  ST_ENONFINITE = 18,
+  ST_ETIMEOUT = 19
+};
 
 // A batched row-major operand in HBM.  `hi` holds the fp32 value (TF32 mode),
 // the TF32-rounded high part (split mode, with `lo` = tf32(value - hi), so
@@ -207,6 +214,13 @@ cudaError_t small_inv_root(const float* A, int n, int batch, int power,
                            const shp_prism_opts& o, const float* S, float* X,
                            int* rep_status, int* rep_iters, float* rep_resid, float* rep_alpha,
                            int* rep_degree, cudaStream_t st);
+// Blocks of different shapes: block b is dims[2b] x dims[2b+1] (<= 64,
+// multiples of 4) at G + offsets[b] / X + offsets[b]; sketch slices are
+// 64 x p and a block uses their first min(m_b, n_b) rows.
+cudaError_t small_polar_varsize(const float* G, const int* dims, const int64_t* offsets,
+                                int batch, const shp_prism_opts& o, const float* S, float* X,
+                                int* rep_status, int* rep_iters, float* rep_resid,
+                                float* rep_alpha, int* rep_degree, cudaStream_t st);
 // sign: the sign function of a symmetric square G (R = I - X X).
 cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism_opts& o,
                         const float* S, float* X, int* rep_status, int* rep_iters,

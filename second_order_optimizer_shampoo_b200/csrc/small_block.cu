@@ -373,17 +373,28 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
 __global__ void __launch_bounds__(SB_THREADS, 3)
     k_small_polar(const float* __restrict__ G, int m, int n, SmallCfg o,
                   const float* __restrict__ S, float* __restrict__ Xout, SmallReport rep,
-                  int sign) {
+                  int sign, const int* __restrict__ dims, const int64_t* __restrict__ offs,
+                  int64_t s_stride) {
   count_kernel_run();
   extern __shared__ __align__(16) float sm[];
   __shared__ double red[SB_THREADS / 32][10];
   __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
   const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
+  int64_t boff = static_cast<int64_t>(b) * m * n;
+  if (dims != nullptr) {  // blocks of different shapes, packed at offs[b]
+    m = dims[2 * b];
+    n = dims[2 * b + 1];
+    boff = offs[b];
+    if (m < 4 || n < 4 || m > SB_NMAX || n > SB_NMAX || (m & 3) || (n & 3) || boff < 0) {
+      if (tid == 0 && rep.status != nullptr) rep.status[b] = ST_EINVAL;
+      return;
+    }
+  }
   const bool tall = m >= n;
   const int rows = tall ? m : n, k_n = tall ? n : m;  // X is rows x k_n
   const int64_t mn = static_cast<int64_t>(m) * n;
-  const float* Gb = G + b * mn;
+  const float* Gb = G + boff;
   float *X = sm, *R = sm + SB_MAT, *W = sm + 2 * SB_MAT, *T = sm + 3 * SB_MAT;
 
   double part = 0.0;
@@ -392,13 +403,13 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
     part += static_cast<double>(v) * v;
   }
   const float c = static_cast<float>(sqrt(block_sum(part, red[0])));
-  const float inv = c > 0.f ? 1.f / c : 0.f;
+  // X_0 = G / ||G||_F as written (a zero block: 0/0, SHP_ENONFINITE)
   for (int e = tid; e < mn; e += SB_THREADS) {
     const int i = e / n, j = e - i * n;  // G(i, j)
     if (tall)
-      X[i * SB_LD + j] = Gb[e] * inv;
+      X[i * SB_LD + j] = Gb[e] / c;
     else
-      X[j * SB_LD + i] = Gb[e] * inv;
+      X[j * SB_LD + i] = Gb[e] / c;
   }
   __syncthreads();
 
@@ -422,7 +433,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
     }
     const float alpha =
         o.fixed_alpha ? o.lo
-                      : sketch_alpha(R, k_n, o, S + static_cast<int64_t>(k) * k_n * o.p, T, &deg,
+                      : sketch_alpha(R, k_n, o, S + static_cast<int64_t>(k) * s_stride, T, &deg,
                                      red, &s_alpha, &s_ratio);
     if (tid == 0 && rep.alpha != nullptr) rep.alpha[2 * b * mi + k] = alpha;
     if (tid == 0 && rep.degree != nullptr) rep.degree[2 * b * mi + k] = deg;
@@ -434,7 +445,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
     T = t;
   }
 
-  float* Xb = Xout + b * mn;
+  float* Xb = Xout + boff;
   for (int e = tid; e < mn; e += SB_THREADS) {
     const int i = e / n, j = e - i * n;
     Xb[e] = tall ? X[i * SB_LD + j] : X[j * SB_LD + i];
@@ -489,9 +500,25 @@ cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism
   if (batch <= 0) return cudaSuccess;
   cudaError_t e = prepare(k_small_polar);
   if (e != cudaSuccess) return e;
+  const int k_n = m >= n ? n : m;
   k_small_polar<<<batch, SB_THREADS, SB_SMEM, st>>>(
       G, m, n, make_cfg(o), S, X,
-      SmallReport{rep_status, rep_iters, rep_resid, rep_alpha, rep_degree}, sign ? 1 : 0);
+      SmallReport{rep_status, rep_iters, rep_resid, rep_alpha, rep_degree}, sign ? 1 : 0,
+      nullptr, nullptr, static_cast<int64_t>(k_n) * o.p);
+  return cudaGetLastError();
+}
+
+cudaError_t small_polar_varsize(const float* G, const int* dims, const int64_t* offsets,
+                                int batch, const shp_prism_opts& o, const float* S, float* X,
+                                int* rep_status, int* rep_iters, float* rep_resid,
+                                float* rep_alpha, int* rep_degree, cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  cudaError_t e = prepare(k_small_polar);
+  if (e != cudaSuccess) return e;
+  k_small_polar<<<batch, SB_THREADS, SB_SMEM, st>>>(
+      G, 0, 0, make_cfg(o), S, X,
+      SmallReport{rep_status, rep_iters, rep_resid, rep_alpha, rep_degree}, 0, dims, offsets,
+      static_cast<int64_t>(SB_NMAX) * o.p);
   return cudaGetLastError();
 }
 

@@ -187,6 +187,26 @@ def matfn_polar(G, opts: A.PrismOpts | None = None, S=None, out=None, report=Tru
     return out, rep
 
 
+def matfn_polar_varsize(G, dims, offsets, opts: A.PrismOpts | None = None, S=None, out=None,
+                        report=True):
+    """Polar factors of small blocks of different shapes packed in the fp32
+    tensor G: block b is dims[b] = (m_b, n_b) at element offsets[b] (dims int32
+    [batch, 2], offsets int64 [batch], both on the device)."""
+    opts = opts or make_opts()
+    _dev(G, dims, offsets, S, out)
+    if G.dtype != torch.float32 or dims.dtype != torch.int32 or offsets.dtype != torch.int64:
+        raise ValueError("G float32, dims int32, offsets int64")
+    batch = dims.shape[0]
+    out = torch.empty_like(G) if out is None else out
+    rep = report if isinstance(report, dict) else (
+        _report(batch, opts.max_iter, G.device) if report else None)
+    s_count = 0 if S is None else S.shape[0]
+    _check(A.lib().matfn_polar_varsize(_p(G), _p(dims), _p(offsets), batch, ctypes.byref(opts),
+                                       _p(S), s_count, _p(out), _report_struct(rep), _stream()),
+           "matfn_polar_varsize")
+    return out, rep
+
+
 def matfn_sign(Amat, opts: A.PrismOpts | None = None, S=None, out=None, report=True, ws=None):
     """Matrix sign function of a batch of symmetric n x n matrices (bf16 input
     keeps bf16 storage)."""

@@ -157,3 +157,68 @@ def test_small_batched_16384_blocks():
                                force_iters=rep["iters"][b])
         assert relerr(X[b], Xo) <= TOL_FP32
         assert relerr(X[b], o.spd_power_eigh(A[b], -0.25)) <= TOL_FP32
+
+
+@pytest.mark.parametrize("n", [32, 128])
+def test_zero_and_indefinite_blocks_are_isolated(n):
+    """Faults injected on the host (on chip at n = 32, batched at n = 128): a
+    zero block stops with ENONFINITE (0/0 in the normalisation, as the oracle),
+    an indefinite block (R_0 has eigenvalues above 1) diverges and stops with
+    ENONFINITE or ENOCONV, and the good block between them is unaffected."""
+    P = prism()
+    good = synth.spd_batch(n, 1, 1e-2, 1.0, 205)[0]
+    Q, _ = np.linalg.qr(np.random.default_rng(206).standard_normal((n, n)))
+    lam = np.linspace(-1.0, 1.0, n)
+    lam[np.abs(lam) < 0.1] = 0.5
+    indef = ((Q * lam) @ Q.T).astype(np.float32)
+    A = np.stack([np.zeros((n, n), np.float32), good, indef])
+    S = synth.sketch_stack(60, n, 4, 1206)
+    opts = P.make_opts(d=2, p=4, tol=1e-6, max_iter=30, prec="3xtf32")
+    X, rep = P.matfn_inv_root(to_dev(torch, A), "inv4", opts, to_dev(torch, S))
+    X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
+    assert rep["status"][0] == o.ENONFINITE
+    assert rep["status"][1] == o.OK
+    assert rep["status"][2] in (o.ENONFINITE, o.ENOCONV)
+    assert relerr(X[1], o.spd_power_eigh(good, -0.25)) <= 3e-5
+    _, infos = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S)
+    assert infos[0].status == o.ENONFINITE
+    # polar of a zero block: the same status as the oracle's
+    Gz = np.zeros((2, n, n // 2), np.float32)
+    Gz[1] = synth.gaussian((n, n // 2), 1.0, 207)
+    _, rp = P.matfn_polar(to_dev(torch, Gz), P.make_opts(d=2, p=4, tol=1e-6, max_iter=30,
+                                                         prec="3xtf32"),
+                          to_dev(torch, synth.sketch_stack(40, n // 2, 4, 1207)))
+    assert list(to_host(rp["status"])) == [o.ENONFINITE, o.OK]
+
+
+def test_polar_varsize_blocks():
+    """Blocks of different shapes packed in one buffer, one CTA each: every
+    block against the oracle (its sketch = the first min(m, n) rows of each
+    64 x p slice) and the SVD; a block with out-of-range dims reports EINVAL
+    and leaves its output untouched."""
+    P = prism()
+    shapes = [(64, 32), (48, 48), (40, 12), (16, 64), (8, 8), (60, 36), (68, 8)]
+    blocks = [synth.gaussian(s, 1.0, 208, index=i) for i, s in enumerate(shapes)]
+    offs = np.cumsum([0] + [m * n for m, n in shapes])[:-1].astype(np.int64)
+    G = np.concatenate([b.ravel() for b in blocks]).astype(np.float32)
+    S = synth.sketch_stack(40, 64, 8, 1208)
+    opts = P.make_opts(d=2, p=8, tol=1e-6, max_iter=40, prec="3xtf32")
+    dims = torch.tensor(shapes, dtype=torch.int32, device="cuda")
+    out0 = torch.full((G.size,), 7.0, dtype=torch.float32, device="cuda")
+    X, rep = P.matfn_polar_varsize(to_dev(torch, G), dims,
+                                   torch.tensor(offs, device="cuda"), opts, to_dev(torch, S),
+                                   out=out0)
+    X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
+    for i, (m, n) in enumerate(shapes):
+        Xb = X[offs[i]: offs[i] + m * n].reshape(m, n)
+        if m > 64:
+            assert rep["status"][i] == 1  # SHP_EINVAL
+            assert np.all(Xb == 7.0)
+            continue
+        assert rep["status"][i] == o.OK, (i, rep["status"])
+        it = rep["iters"][i][0]
+        k = min(m, n)
+        Xo, infos = o.polar_ref(blocks[i], oracle_opts(opts), S[:, :k, :], force_iters=it)
+        np.testing.assert_allclose(rep["alpha"][i, 0, :it], infos[0].alpha, atol=1e-4)
+        assert relerr(Xb, Xo) <= TOL_FP32
+        assert relerr(Xb, o.polar_svd(blocks[i])) <= TOL_FP32
