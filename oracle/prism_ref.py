@@ -356,15 +356,17 @@ def inv_root_ref(A, power, opts: PrismOpts, S, force_iters=None):
     Returns (X, [PassInfo, ...])."""
     A = _f64(A)
     f1, f2 = (None, None) if force_iters is None else (list(force_iters) + [None])[:2]
-    c = float(np.linalg.norm(A))
-    B = A / c
+    c = np.float64(np.linalg.norm(A))  # numpy arithmetic: c = 0 gives non-finite, not an error
+    with np.errstate(divide="ignore", invalid="ignore"):
+        B = A / c
     Y1, Z1, i1 = coupled_ref(B, opts, S, 0, f1)
     if power == POW_SQRT:
         return np.sqrt(c) * Y1, [i1]
     if power == POW_INV2:
         return Z1 / np.sqrt(c), [i1]
     Y2, Z2, i2 = coupled_ref(Y1, opts, S, opts.max_iter, f2)
-    return c ** -0.25 * Z2, [i1, i2]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return c ** -0.25 * Z2, [i1, i2]
 
 
 def polar_ref(G, opts: PrismOpts, S, force_iters=None):

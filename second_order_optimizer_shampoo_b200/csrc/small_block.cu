@@ -168,15 +168,22 @@ SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, int r0,
   return W;
 }
 
-// Vout = R Vin (n x p, row-major) by the whole CTA.
+// Vout = R Vin (n x p, row-major) by the whole CTA; each dot product runs as
+// four interleaved partial sums (k mod 4) so that its FMA chain is n/4 long.
 SHP_DEV void sketch_power(const float* R, const float* Vin, float* Vout, int n, int p) {
   for (int e = threadIdx.x; e < n * p; e += SB_THREADS) {
     const int row = e / p, col = e - row * p;
     const float* Rr = R + row * SB_LD;
-    float s = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < n; ++k) s = fmaf(Rr[k], Vin[k * p + col], s);
-    Vout[e] = s;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < n; k += 4) {
+      const float4 r = *reinterpret_cast<const float4*>(Rr + k);
+      s0 = fmaf(r.x, Vin[k * p + col], s0);
+      s1 = fmaf(r.y, Vin[(k + 1) * p + col], s1);
+      s2 = fmaf(r.z, Vin[(k + 2) * p + col], s2);
+      s3 = fmaf(r.w, Vin[(k + 3) * p + col], s3);
+    }
+    Vout[e] = (s0 + s1) + (s2 + s3);
   }
   __syncthreads();
 }
