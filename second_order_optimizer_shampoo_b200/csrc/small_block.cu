@@ -55,11 +55,31 @@ SHP_DEV double block_sum(double v, double* red) {
   return s;
 }
 
-// acc = op(A) B on this thread's 4 x 4 tile (rows r0.., columns c0..), K a
-// multiple of 4.  op(A) = A (row-major M x K) or, with AT, the transpose of
-// the row-major K x M matrix A.
+// A thread's 4 x 4 output tile: rows rb, rb + rs, rb + 2 rs, rb + 3 rs and
+// columns c0..c0+3.  Products with a row-major left factor use strided rows
+// (rs = 16): a warp covers 4 consecutive row indices x 8 column groups, so
+// each float4 operand read touches 4 rows (16 banks apart in total) of A and
+// 128 contiguous bytes of B, one wavefront each.  Products with a
+// transposed left factor read 4 consecutive rows of A^T as one float4 and
+// use consecutive rows (rs = 1).
+struct Tile {
+  int rb, rs, c0;
+  SHP_DEV int row(int i) const { return rb + rs * i; }
+};
+
+SHP_DEV Tile tile_rows_strided() {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  return Tile{4 * (w >> 1) + (l >> 3), 16, 4 * (8 * (w & 1) + (l & 7))};
+}
+SHP_DEV Tile tile_rows_consecutive() {
+  const int t = static_cast<int>(threadIdx.x);
+  return Tile{4 * (t >> 4), 1, 4 * (t & 15)};
+}
+
+// acc = op(A) B on tile t, K a multiple of 4.  op(A) = A (row-major M x K) or,
+// with AT, the transpose of the row-major K x M matrix A (t.rs must be 1).
 template <bool AT>
-SHP_DEV void tile_mm(const float* A, const float* B, int K, int r0, int c0, float acc[4][4]) {
+SHP_DEV void tile_mm(const float* A, const float* B, int K, const Tile& t, float acc[4][4]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -69,7 +89,7 @@ SHP_DEV void tile_mm(const float* A, const float* B, int K, int r0, int c0, floa
     float a[4][4], b[4][4];
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      const float4 v = *reinterpret_cast<const float4*>(B + (k + kk) * SB_LD + c0);
+      const float4 v = *reinterpret_cast<const float4*>(B + (k + kk) * SB_LD + t.c0);
       b[kk][0] = v.x;
       b[kk][1] = v.y;
       b[kk][2] = v.z;
@@ -78,7 +98,7 @@ SHP_DEV void tile_mm(const float* A, const float* B, int K, int r0, int c0, floa
     if (AT) {
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const float4 v = *reinterpret_cast<const float4*>(A + (k + kk) * SB_LD + r0);
+        const float4 v = *reinterpret_cast<const float4*>(A + (k + kk) * SB_LD + t.rb);
         a[0][kk] = v.x;
         a[1][kk] = v.y;
         a[2][kk] = v.z;
@@ -87,7 +107,7 @@ SHP_DEV void tile_mm(const float* A, const float* B, int K, int r0, int c0, floa
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(A + (r0 + i) * SB_LD + k);
+        const float4 v = *reinterpret_cast<const float4*>(A + t.row(i) * SB_LD + k);
         a[i][0] = v.x;
         a[i][1] = v.y;
         a[i][2] = v.z;
@@ -107,22 +127,25 @@ SHP_DEV void store_row4(float* C, int row, int c0, const float* v) {
   *reinterpret_cast<float4*>(C + row * SB_LD + c0) = make_float4(v[0], v[1], v[2], v[3]);
 }
 
-// R = I - op(A) B on the n x n tile grid; returns this thread's sum of squares.
+// R = I - op(A) B on the n x n grid; returns this thread's sum of squares.
+// Rows of the tile past n are computed from in-buffer data and not stored.
 template <bool AT>
-SHP_DEV float residual(const float* A, const float* B, int K, int n, float* R, int r0, int c0) {
+SHP_DEV float residual(const float* A, const float* B, int K, int n, float* R, const Tile& t) {
   float nrm = 0.f;
-  if (r0 < n && c0 < n) {
+  if (t.rb < n && t.c0 < n) {
     float acc[4][4];
-    tile_mm<AT>(A, B, K, r0, c0, acc);
+    tile_mm<AT>(A, B, K, t, acc);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
+      const int r = t.row(i);
+      if (r >= n) break;
       float v[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        v[j] = (r0 + i == c0 + j ? 1.f : 0.f) - acc[i][j];
+        v[j] = (r == t.c0 + j ? 1.f : 0.f) - acc[i][j];
         nrm += v[j] * v[j];
       }
-      store_row4(R, r0 + i, c0, v);
+      store_row4(R, r, t.c0, v);
     }
   }
   return nrm;
@@ -130,21 +153,23 @@ SHP_DEV float residual(const float* A, const float* B, int K, int n, float* R, i
 
 // C = X + A B (X may be A or B, C must be neither), rows x cols, inner K.
 SHP_DEV void axpy_mm(const float* A, const float* B, const float* X, int K, int rows, int cols,
-                     float* C, int r0, int c0) {
-  if (r0 >= rows || c0 >= cols) return;
+                     float* C, const Tile& t) {
+  if (t.rb >= rows || t.c0 >= cols) return;
   float acc[4][4];
-  tile_mm<false>(A, B, K, r0, c0, acc);
+  tile_mm<false>(A, B, K, t, acc);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float4 x = *reinterpret_cast<const float4*>(X + (r0 + i) * SB_LD + c0);
+    const int r = t.row(i);
+    if (r >= rows) break;
+    const float4 x = *reinterpret_cast<const float4*>(X + r * SB_LD + t.c0);
     const float v[4] = {x.x + acc[i][0], x.y + acc[i][1], x.z + acc[i][2], x.w + acc[i][3]};
-    store_row4(C, r0 + i, c0, v);
+    store_row4(C, r, t.c0, v);
   }
 }
 
 // Delta = g - I: alpha R in place (d = 1), or W = R/2 + alpha R^2 (d = 2).
 // Returns the buffer that holds Delta.
-SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, int r0, int c0) {
+SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, const Tile& t) {
   if (d == 1) {
     for (int e = threadIdx.x; e < n * n; e += SB_THREADS) {
       const int i = e / n, j = e - i * n;
@@ -153,15 +178,17 @@ SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, int r0,
     __syncthreads();
     return R;
   }
-  if (r0 < n && c0 < n) {
+  if (t.rb < n && t.c0 < n) {
     float acc[4][4];
-    tile_mm<false>(R, R, n, r0, c0, acc);
+    tile_mm<false>(R, R, n, t, acc);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 r = *reinterpret_cast<const float4*>(R + (r0 + i) * SB_LD + c0);
-      const float v[4] = {0.5f * r.x + alpha * acc[i][0], 0.5f * r.y + alpha * acc[i][1],
-                          0.5f * r.z + alpha * acc[i][2], 0.5f * r.w + alpha * acc[i][3]};
-      store_row4(W, r0 + i, c0, v);
+      const int r = t.row(i);
+      if (r >= n) break;
+      const float4 q = *reinterpret_cast<const float4*>(R + r * SB_LD + t.c0);
+      const float v[4] = {0.5f * q.x + alpha * acc[i][0], 0.5f * q.y + alpha * acc[i][1],
+                          0.5f * q.z + alpha * acc[i][2], 0.5f * q.w + alpha * acc[i][3]};
+      store_row4(W, r, t.c0, v);
     }
   }
   __syncthreads();
@@ -281,7 +308,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   __shared__ double red[SB_THREADS / 32][10];
   __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
-  const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
+  const Tile ts = tile_rows_strided();
   const int64_t nn = static_cast<int64_t>(n) * n;
   const float* Ab = A + b * nn;
   float *Y = sm, *Z = sm + SB_MAT, *R = sm + 2 * SB_MAT, *W = sm + 3 * SB_MAT;
@@ -316,7 +343,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
     float prev = INFINITY;
     int deg = o.adaptive ? 1 : o.d;  // the degree of g for this pass (adaptive degree)
     for (int k = 0;; ++k) {
-      if (k > 0) n2 = block_sum(residual<false>(Z, Y, n, n, R, r0, c0), red[0]);
+      if (k > 0) n2 = block_sum(residual<false>(Z, Y, n, n, R, ts), red[0]);
       // every thread evaluates the stop rule on the same reduced norm
       const float r = sqrtf(static_cast<float>(n2) / static_cast<float>(n));
       const int st = stop_rule(r, k, mi, o.tol, prev, o.stall_below, o.stall_ratio);
@@ -333,9 +360,9 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
                                        W, &deg, red, &s_alpha, &s_ratio);
       if (tid == 0 && rep.alpha != nullptr) rep.alpha[(2 * b + pass) * mi + k] = alpha;
       if (tid == 0 && rep.degree != nullptr) rep.degree[(2 * b + pass) * mi + k] = deg;
-      float* D = form_delta(deg, alpha, R, W, n, r0, c0);
+      float* D = form_delta(deg, alpha, R, W, n, ts);
       float* T = deg == 1 ? W : R;  // the buffer Delta does not occupy
-      axpy_mm(Y, D, Y, n, n, n, T, r0, c0);  // Y_{k+1} = Y_k + Y_k Delta
+      axpy_mm(Y, D, Y, n, n, n, T, ts);  // Y_{k+1} = Y_k + Y_k Delta
       __syncthreads();
       if (k == 0) {  // Z_1 = I + Delta
         for (int e = tid; e < nn; e += SB_THREADS) {
@@ -343,7 +370,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
           Y[i * SB_LD + j] = (i == j ? 1.f : 0.f) + D[i * SB_LD + j];
         }
       } else {  // Z_{k+1} = Z_k + Delta Z_k
-        axpy_mm(D, Z, Z, n, n, n, Y, r0, c0);
+        axpy_mm(D, Z, Z, n, n, n, Y, ts);
       }
       __syncthreads();
       float* oldZ = Z;
@@ -387,7 +414,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   __shared__ double red[SB_THREADS / 32][10];
   __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
-  const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
+  const Tile ts = tile_rows_strided(), tc = tile_rows_consecutive();
   int64_t boff = static_cast<int64_t>(b) * m * n;
   if (dims != nullptr) {  // blocks of different shapes, packed at offs[b]
     m = dims[2 * b];
@@ -426,8 +453,8 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   int deg = o.adaptive ? 1 : o.d;
   for (int k = 0;; ++k) {
     // R = I - X^T X (polar) or I - X X (sign of a symmetric X, m == n)
-    const double n2 = block_sum(sign ? residual<false>(X, X, rows, k_n, R, r0, c0)
-                                     : residual<true>(X, X, rows, k_n, R, r0, c0),
+    const double n2 = block_sum(sign ? residual<false>(X, X, rows, k_n, R, ts)
+                                     : residual<true>(X, X, rows, k_n, R, tc),
                                 red[0]);
     const float r = sqrtf(static_cast<float>(n2) / static_cast<float>(k_n));
     const int st = stop_rule(r, k, mi, o.tol, prev, o.stall_below, o.stall_ratio);
@@ -444,8 +471,8 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
                                      red, &s_alpha, &s_ratio);
     if (tid == 0 && rep.alpha != nullptr) rep.alpha[2 * b * mi + k] = alpha;
     if (tid == 0 && rep.degree != nullptr) rep.degree[2 * b * mi + k] = deg;
-    float* D = form_delta(deg, alpha, R, W, k_n, r0, c0);
-    axpy_mm(X, D, X, k_n, rows, k_n, T, r0, c0);  // X_{k+1} = X_k + X_k Delta
+    float* D = form_delta(deg, alpha, R, W, k_n, ts);
+    axpy_mm(X, D, X, k_n, rows, k_n, T, ts);  // X_{k+1} = X_k + X_k Delta
     __syncthreads();
     float* t = X;
     X = T;
