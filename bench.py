@@ -58,6 +58,17 @@ def gemm_count(iters):
     return sum(max(4 * int(k) - 1, 0) for k in iters)
 
 
+def pass_flops(k, n):
+    """Algorithmic flops of one coupled pass with k updates (d = 2): 4k - 1
+    full n x n x n products (2n^3 each).  Z_k Y_k, R_k^2 and the updates are
+    symmetric only in exact arithmetic and are formed in full."""
+    return gemm_count([k]) * 2.0 * n ** 3
+
+
+def block_flops(iters, n):
+    return sum(pass_flops(k, n) for k in iters)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -157,7 +168,7 @@ def oracle_sample(A_block, S_np, seconds_hint=None):
     t0 = time.perf_counter()
     _, infos = o.inv_root_ref(A_block, o.POW_INV4, opts, S_np)
     dt = time.perf_counter() - t0
-    return dt, gemm_count([i.iters for i in infos]) * 2.0 * N ** 3
+    return dt, block_flops([i.iters for i in infos], N)
 
 
 def run_reference(args):
@@ -332,14 +343,14 @@ def shampoo_step_leg(args, dev, stream):
     torch.cuda.synchronize()
     iters = rep["iters"].cpu().numpy()
     ms = _time(step, stream, 10)
-    products = sum(max(4 * int(k) - 1, 0) for blk in iters for k in blk)
-    flops = 10 * 2 * n * (n + 1) * n + products * 2.0 * n ** 3 + 2 * 2.0 * n ** 3
+    flops = 10 * 2 * n * (n + 1) * n + sum(block_flops(blk, n) for blk in iters) + 2 * 2.0 * n ** 3
     return {"workload": "shampoo_step_1024sq_ema10_inv4_d2_p8_tf32_apply", "ms_per_step": ms,
             "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
             "preconditioners_per_s": 2 / (ms / 1e3),
             "iters_per_pass": [[int(k) for k in blk] for blk in iters],
             "status": [int(x) for x in rep["status"].cpu().numpy()],
-            "note": "EMA products counted n(n+1)n (symmetric), computed as full GEMMs"}
+            "note": "EMA products counted n(n+1)n (symmetric results, formed on their "
+                    "upper-triangle tiles); inverse-root products and the apply at 2n^3"}
 
 
 def gemm_count_leg(args, dev, stream, A):
@@ -591,7 +602,7 @@ def main():
     torch.cuda.synchronize()
     iters = rep["iters"].cpu().numpy()
     status = rep["status"].cpu().numpy()
-    flops_step = float(sum(gemm_count(it) for it in iters)) * 2.0 * N ** 3
+    flops_step = float(sum(block_flops(it, N) for it in iters))
 
     # ---- timed region (device time, CUDA events on the launching stream)
     stream = torch.cuda.current_stream()

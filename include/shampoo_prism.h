@@ -132,14 +132,17 @@ size_t shp_workspace_bytes(int op, int64_t m, int64_t n, int64_t batch,
  *   R <- beta R + (1 - beta) G^T G + eps I      (R: n x n, in place)
  * G: [batch][m][n] fp32; L: [batch][m][m]; R: [batch][n][n].
  * prec: SHP_TF32 or SHP_3XTF32 (the latter needs workspace for the split G).
- * Either L or R may be NULL to skip that factor. */
+ * Either L or R may be NULL to skip that factor.  L and R are symmetric by
+ * construction and must be on entry: each product is formed on its tiles on
+ * and above the diagonal, and the result is written to both triangles. */
 int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float* L, float* R,
                      float beta, float eps, int prec, void* ws, size_t ws_bytes,
                      shp_stream stream);
 
 /* Matrix power of a batch of SPD matrices by coupled Newton-Schulz with PRISM
  * alpha ([PRISM] Parte I-II; [Shampoo] 2.3 step 3 and 3.1):
- *   c = ||A||_F, B = A / c;  pass 1: Y_0 = B, Z_0 = I, for k = 0, 1, ...:
+ *   c = ||A||_F, B = (A + A^T) / (2c) (A / c for a symmetric A);
+ *   pass 1: Y_0 = B, Z_0 = I, for k = 0, 1, ...:
  *   R_k = I - Z_k Y_k, stop test, alpha_k = argmin_{[lo,hi]} ||r(R_k;alpha) S_k||_F,
  *   g = g_d(R_k; alpha_k), Y_{k+1} = Y_k g, Z_{k+1} = g Z_k.
  *   SHP_POW_SQRT -> sqrt(c) Y;  SHP_POW_INV2 -> Z / sqrt(c);

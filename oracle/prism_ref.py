@@ -350,6 +350,8 @@ def inv_root_ref(A, power, opts: PrismOpts, S, force_iters=None):
     """A^(-1/4), A^(-1/2) or A^(1/2) of an SPD matrix by PRISM Newton-Schulz.
 
     c = ||A||_F (>= lambda_max, so B = A/c has spectrum in (0, 1]);
+    the method is stated for a symmetric A, so B is taken as the symmetric
+    part (A + A^T) / (2c), which is A / c itself for a symmetric input;
     pass 1: (Y1, Z1) = coupled(B) -> A^(1/2) = sqrt(c) Y1, A^(-1/2) = Z1 / sqrt(c);
     pass 2 (A^(-1/4) only): (Y2, Z2) = coupled(Y1) -> A^(-1/4) = c^(-1/4) Z2.
     force_iters: optional (updates in pass 1, updates in pass 2).
@@ -358,7 +360,7 @@ def inv_root_ref(A, power, opts: PrismOpts, S, force_iters=None):
     f1, f2 = (None, None) if force_iters is None else (list(force_iters) + [None])[:2]
     c = np.float64(np.linalg.norm(A))  # numpy arithmetic: c = 0 gives non-finite, not an error
     with np.errstate(divide="ignore", invalid="ignore"):
-        B = A / c
+        B = 0.5 * (A + A.T) / c
     Y1, Z1, i1 = coupled_ref(B, opts, S, 0, f1)
     if power == POW_SQRT:
         return np.sqrt(c) * Y1, [i1]

@@ -497,6 +497,7 @@ int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float*
     e.s0 = beta;
     e.s1 = 1.f - beta;
     e.s2 = eps;
+    e.sym = 1;  // G G^T and L symmetric: upper-triangle tiles, mirrored
     CK(gemm_tc(mode, op(Ghi, Glo, false, n, m * n), op(Ghi, Glo, false, n, m * n), M, M, N, B, e,
                st));
   }
@@ -505,6 +506,7 @@ int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float*
     e.s0 = beta;
     e.s1 = 1.f - beta;
     e.s2 = eps;
+    e.sym = 1;
     CK(gemm_tc(mode, op(Ghi, Glo, true, n, m * n), op(Ghi, Glo, true, n, m * n), N, N, M, B, e,
                st));
   }
@@ -691,6 +693,13 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
       // step has R_0 = I - B from the start kernel and Z_1 = g (Z_0 = I)
       auto iter = [&](int cur, bool first, cudaStream_t st) -> int {
         const int nxt = cur ^ 1;
+        // Every product here is formed in full, although Z_k Y_k, R_k^2,
+        // Y_k g and g Z_k are symmetric in exact arithmetic: Z_k and Y_k only
+        // commute up to rounding, and keeping one triangle (mirroring) turns
+        // that non-commuting error into a symmetric one the coupled pair no
+        // longer corrects.  In fp32 at cond 1e6 it costs the inverse root two
+        // orders of magnitude of accuracy (residual and R^2 mirrored) or
+        // diverges (updates mirrored).
         if (!first) {  // R_k = I - Z_k Y_k and ||R_k||_F^2
           EpiParams e = epi(EPI_RESID, fmt, w.Rhi, w.Rlo, n, nn, N, N, &ctl);
           if (split) e.out_plain = w.Rs;

@@ -101,26 +101,44 @@ __global__ void __launch_bounds__(EW_THREADS)
   }
 }
 
+// Start of pass 1 (c = ||A||_F from k_frob): Y_0 = B = (A + A^T) / (2c),
+// Z_0 = I, R_0 = I - B.  The method is stated for a symmetric A and every
+// later product is formed on its upper-triangle tiles, so the start takes the
+// symmetric part, which is A / c bit for bit when A is symmetric.  A^T comes
+// through a padded 32 x 32 shared-memory transpose: both reads are coalesced.
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_init(const float* A, int64_t n, Ctl ctl, int fmt, float* Yhi, float* Ylo,
                    float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs) {
   count_kernel_run();
+  __shared__ float tt[32][33];
   const int b = blockIdx.y;
   const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
   if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
-  const int64_t nn = n * n;
+  const int64_t nn = n * n, T = (n + 31) / 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const float* Ab = A + b * nn;
   float nrm = 0.f;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
-       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
-    const int64_t off = b * nn + e;
-    const bool diag = (e / n) == (e % n);
-    const float y = A[off] / c;
-    const float r = (diag ? 1.f : 0.f) - y;
-    put(fmt, Yhi, Ylo, off, y);
-    put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
-    put(fmt, Rhi, Rlo, off, r);
-    if (Rs != nullptr) Rs[off] = r;
-    nrm += r * r;
+  for (int64_t t = blockIdx.x; t < T * T; t += gridDim.x) {
+    const int64_t i0 = (t / T) * 32, j0 = (t % T) * 32;
+    __syncthreads();  // the previous tile's reads of tt are done
+    for (int r = ty; r < 32; r += EW_THREADS / 32) {  // tt[x][r] = A(j0 + r, i0 + x)
+      const int64_t row = j0 + r, col = i0 + tx;
+      tt[tx][r] = (row < n && col < n) ? Ab[row * n + col] : 0.f;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += EW_THREADS / 32) {
+      const int64_t row = i0 + r, col = j0 + tx;  // A^T(row, col) = tt[r][tx]
+      if (row >= n || col >= n) continue;
+      const int64_t off = b * nn + row * n + col;
+      const bool diag = row == col;
+      const float y = 0.5f * (Ab[row * n + col] + tt[r][tx]) / c;
+      const float rr = (diag ? 1.f : 0.f) - y;
+      put(fmt, Yhi, Ylo, off, y);
+      put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
+      put(fmt, Rhi, Rlo, off, rr);
+      if (Rs != nullptr) Rs[off] = rr;
+      nrm += rr * rr;
+    }
   }
   block_add(nrm, &ctl.bs[b].norm2);
 }

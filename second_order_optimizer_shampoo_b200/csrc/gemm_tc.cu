@@ -286,6 +286,8 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
           const int64_t off = static_cast<int64_t>(b) * ep.bso + mrow * ep.ldo + mcol;
           const float v = st[lane * 33 + j];
           put(ep.out_fmt, ep.out_hi, ep.out_lo, off, v);
+          // a mirrored tile holds no diagonal element, so out2 = I + v is v here
+          if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, v);
           if (ep.out_plain != nullptr) ep.out_plain[off] = v;
         }
       }

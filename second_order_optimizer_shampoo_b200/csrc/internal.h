@@ -86,9 +86,11 @@ struct EpiParams {
   const int* active;  // blocks with active[b] == 0 are skipped (may be null)
   int* status;        // receives ST_ETIMEOUT if a pipeline wait runs out (may be null)
   int M, N;
-  // The result is symmetric (M == N, kinds RESID/GPOLY/STORE, no out2): the
-  // persistent kernel computes the tiles on and above the diagonal and writes
-  // each off-diagonal tile's mirror image too; other kernels compute it all.
+  // The result is symmetric (M == N; any kind but MOMENTUM, whose out2 is not
+  // of the form I + v): the persistent kernel computes the tiles on and above
+  // the diagonal and writes each off-diagonal tile's mirror image too (to out,
+  // out2 and out_plain); other kernels compute it all.  Read-modify-write and
+  // aux operands are read on the upper tiles only, so they must be symmetric.
   int sym;
 };
 

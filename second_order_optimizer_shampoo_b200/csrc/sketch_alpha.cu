@@ -27,80 +27,118 @@ namespace shp {
 namespace {
 
 constexpr int SK_THREADS = 256;
+constexpr int SK_GROUPS = 2;  // row groups per warp in one CTA
 
-// Vout = R * Vin for one block.  Each warp owns ROWS consecutive rows of R
-// and streams them with 128-bit loads (a lane takes 4 consecutive columns);
-// V is staged in shared memory transposed, Vs[j][c], one 32 KB chunk of
-// columns at a time, so that lane reads are conflict-free float4 as well.
-// Requires n % 4 == 0 (16-byte rows).
+// Vout = R * Vin for one block: HBM-bound, every byte of R read once.
+// Each warp owns ROWS consecutive rows of R per group and streams them with
+// 128-bit loads (a lane takes 4 consecutive columns), two 128-column steps
+// per iteration so that 2 * ROWS loads per lane are in flight before the
+// first is used; a CTA covers GROUPS groups per warp so that one staging of V
+// serves 8 * ROWS * GROUPS rows.  V is staged in shared memory transposed,
+// Vs[j][c], one 32 KB chunk of columns at a time, with rows padded by 4
+// floats so that both the staging stores and the float4 reads of a warp are
+// conflict-free.  Rows past n re-read row n-1 (never stored), which keeps
+// the loads free of branches.  Requires n % 4 == 0 (16-byte rows).
 template <int P>
-__global__ void __launch_bounds__(SK_THREADS)
+__global__ void __launch_bounds__(SK_THREADS, 2)
     k_sketch(const float* __restrict__ Rhi, const float* __restrict__ Rlo, int64_t n,
              int64_t rbs, const float* __restrict__ Vin, int64_t vbs, float* __restrict__ Vout,
              int64_t obs, int p, const int* __restrict__ active, const int* __restrict__ it,
              int64_t it_stride) {
   count_kernel_run();
-  constexpr int ROWS = P <= 16 ? 4 : 2;
-  constexpr int CK = 8192 / P;  // columns per chunk: Vs is 32 KB
-  __shared__ __align__(16) float Vs[P][CK];
+  constexpr int ROWS = P <= 8 ? 4 : 2;
+  constexpr int CK = 8192 / P;  // columns per chunk (a multiple of 256)
+  constexpr int LDV = CK + 4;
+  __shared__ __align__(16) float Vs[P][LDV];
   const int b = blockIdx.y;
   if (active != nullptr && active[b] == 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (8 * ROWS) + warp * ROWS;
+  const int64_t cta_row0 = static_cast<int64_t>(blockIdx.x) * (8 * ROWS * SK_GROUPS);
   const float* R = Rhi + b * rbs;
   const float* RL = Rlo != nullptr ? Rlo + b * rbs : nullptr;
   const float* V = Vin + b * vbs + (it != nullptr ? static_cast<int64_t>(*it) * it_stride : 0);
-  float acc[ROWS][P];
-#pragma unroll
-  for (int r = 0; r < ROWS; ++r)
-#pragma unroll
-    for (int j = 0; j < P; ++j) acc[r][j] = 0.f;
+  const bool one_chunk = n <= CK;  // V staged once for every group
 
-  for (int64_t c0 = 0; c0 < n; c0 += CK) {
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < CK * P; idx += SK_THREADS) {
-      const int cc = idx / P, j = idx % P;
-      const int64_t col = c0 + cc;
-      Vs[j][cc] = (j < p && col < n) ? V[col * p + j] : 0.f;
-    }
-    __syncthreads();
-    for (int cc = lane * 4; cc < CK; cc += 128) {
-      const int64_t col = c0 + cc;
-      if (col >= n) break;
-      float4 rv[ROWS];
+  for (int g = 0; g < SK_GROUPS; ++g) {
+    const int64_t row0 = cta_row0 + static_cast<int64_t>(g * 8 + warp) * ROWS;
+    if (cta_row0 + static_cast<int64_t>(g * 8) * ROWS >= n) break;  // uniform over the CTA
+    int64_t roff[ROWS];
 #pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        const int64_t row = row0 + r;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (row < n) {
-          x = *reinterpret_cast<const float4*>(R + row * n + col);
-          if (RL != nullptr) {
-            const float4 y = *reinterpret_cast<const float4*>(RL + row * n + col);
-            x.x += y.x;
-            x.y += y.y;
-            x.z += y.z;
-            x.w += y.w;
+    for (int r = 0; r < ROWS; ++r) roff[r] = (row0 + r < n ? row0 + r : n - 1) * n;
+    float acc[ROWS][P];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+      for (int j = 0; j < P; ++j) acc[r][j] = 0.f;
+
+    for (int64_t c0 = 0; c0 < n; c0 += CK) {
+      if (!(one_chunk && g > 0)) {
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < CK * (P / 4); idx += SK_THREADS) {
+          const int cc = idx / (P / 4), q = 4 * (idx % (P / 4));
+          const int64_t col = c0 + cc;
+          const float* src = V + col * p + q;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            Vs[q + e][cc] = (col < n && q + e < p) ? __ldg(src + e) : 0.f;
+        }
+        __syncthreads();
+      }
+      for (int cc = lane * 4; cc < CK; cc += 256) {
+        const int64_t col = c0 + cc;
+        if (col >= n) break;
+        const bool second = col + 128 < n;
+        float4 x0[ROWS], x1[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          x0[r] = *reinterpret_cast<const float4*>(R + roff[r] + col);
+          x1[r] = second ? *reinterpret_cast<const float4*>(R + roff[r] + col + 128)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (RL != nullptr) {
+#pragma unroll
+          for (int r = 0; r < ROWS; ++r) {
+            const float4 y0 = *reinterpret_cast<const float4*>(RL + roff[r] + col);
+            x0[r].x += y0.x;
+            x0[r].y += y0.y;
+            x0[r].z += y0.z;
+            x0[r].w += y0.w;
+            if (second) {
+              const float4 y1 = *reinterpret_cast<const float4*>(RL + roff[r] + col + 128);
+              x1[r].x += y1.x;
+              x1[r].y += y1.y;
+              x1[r].z += y1.z;
+              x1[r].w += y1.w;
+            }
           }
         }
-        rv[r] = x;
-      }
 #pragma unroll
-      for (int j = 0; j < P; ++j) {
-        const float4 vj = *reinterpret_cast<const float4*>(&Vs[j][cc]);
+        for (int j = 0; j < P; ++j) {
+          const float4 v0 = *reinterpret_cast<const float4*>(&Vs[j][cc]);
+          const float4 v1 = *reinterpret_cast<const float4*>(&Vs[j][cc + 128]);
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r)
-          acc[r][j] = fmaf(rv[r].x, vj.x,
-                           fmaf(rv[r].y, vj.y, fmaf(rv[r].z, vj.z, fmaf(rv[r].w, vj.w, acc[r][j]))));
+          for (int r = 0; r < ROWS; ++r) {
+            float a = acc[r][j];
+            a = fmaf(x0[r].x, v0.x, a);
+            a = fmaf(x0[r].y, v0.y, a);
+            a = fmaf(x0[r].z, v0.z, a);
+            a = fmaf(x0[r].w, v0.w, a);
+            a = fmaf(x1[r].x, v1.x, a);
+            a = fmaf(x1[r].y, v1.y, a);
+            a = fmaf(x1[r].z, v1.z, a);
+            acc[r][j] = fmaf(x1[r].w, v1.w, a);
+          }
+        }
       }
     }
-  }
 #pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
+    for (int r = 0; r < ROWS; ++r) {
 #pragma unroll
-    for (int j = 0; j < P; ++j) {
-      const float sum = warp_sum(acc[r][j]);
-      const int64_t row = row0 + r;
-      if (lane == 0 && row < n && j < p) Vout[b * obs + row * p + j] = sum;
+      for (int j = 0; j < P; ++j) {
+        const float sum = warp_sum(acc[r][j]);
+        const int64_t row = row0 + r;
+        if (lane == 0 && row < n && j < p) Vout[b * obs + row * p + j] = sum;
+      }
     }
   }
 }
@@ -254,8 +292,8 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
                         int p, int batch, const int* active, const int* it, int64_t it_stride,
                         cudaStream_t st) {
   if (batch <= 0 || n <= 0) return cudaSuccess;
-  const int rows = p <= 16 ? 4 : 2;
-  dim3 grid(static_cast<unsigned>((n + 8 * rows - 1) / (8 * rows)), batch);
+  const int rows = (p <= 8 ? 4 : 2) * 8 * SK_GROUPS;  // rows per CTA (ROWS x 8 warps x groups)
+  dim3 grid(static_cast<unsigned>((n + rows - 1) / rows), batch);
   if (p <= 4)
     k_sketch<4><<<grid, SK_THREADS, 0, st>>>(Rhi, Rlo, n, r_bstride, Vin, vin_bstride, Vout,
                                              vout_bstride, p, active, it, it_stride);

@@ -313,7 +313,8 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   const float* Ab = A + b * nn;
   float *Y = sm, *Z = sm + SB_MAT, *R = sm + 2 * SB_MAT, *W = sm + 3 * SB_MAT;
 
-  // c = ||A||_F (fp64) and Y_0 = A / c
+  // c = ||A||_F (fp64) and Y_0 = (A + A^T) / (2c), the symmetric part (A / c
+  // bit for bit when A is symmetric); A^T is read back from L1/L2
   double part = 0.0;
   for (int e = tid; e < nn; e += SB_THREADS) {
     const float v = Ab[e];
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   const float c = static_cast<float>(sqrt(block_sum(part, red[0])));
   for (int e = tid; e < nn; e += SB_THREADS) {
     const int i = e / n, j = e - i * n;
-    Y[i * SB_LD + j] = Ab[e] / c;
+    Y[i * SB_LD + j] = 0.5f * (Ab[e] + Ab[j * n + i]) / c;
   }
   __syncthreads();
 

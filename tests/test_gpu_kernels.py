@@ -32,6 +32,14 @@ def test_gram_ema(prec, m, n, batch):
     Ld, Rd = to_dev(torch, L0), to_dev(torch, R0)
     prism().shampoo_gram_ema(to_dev(torch, G), Ld, Rd, beta, eps, prec)
     Lg, Rg = to_host(Ld), to_host(Rd)
+    # from 256 on, the products are formed on the upper-triangle tiles and
+    # mirrored: off the diagonal tiles the statistics are exactly symmetric,
+    # on them to the rounding of the 3xTF32 cross terms
+    for X, k in ((Lg, m), (Rg, n)):
+        if k >= 256:
+            asym = np.abs(X - X.transpose(0, 2, 1))
+            assert asym.max() <= 4 * U_FP32 * np.abs(X).max()
+            np.testing.assert_array_equal(asym[:, 256:, :256], 0)
     for b in range(batch):
         Lr, Rr = o.gram_ema_ref(G[b], L0[b], R0[b], beta, eps)
         aG = np.abs(G[b].astype(np.float64))

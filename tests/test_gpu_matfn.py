@@ -85,6 +85,27 @@ def test_inv_root_powers_ragged_batch(power, d):
         assert relerr(X[b], o.spd_power_eigh(A[b], q)) <= 1e-5
 
 
+def test_inv_root_ragged_tiles_and_nonsymmetric_input():
+    """n = 520 (three 256-wide tiles, the last ragged) on the persistent
+    path; a non-symmetric input is taken as its symmetric part (A + A^T) / 2,
+    as the oracle does."""
+    n, batch = 520, 2
+    A = synth.spd_batch(n, batch, 1e-2, 1.0, 105)
+    E = synth.gaussian((n, n), 1e-4, 106)
+    A[1] = A[1] + E  # block 1: symmetric part SPD, not symmetric itself
+    S = synth.sketch_stack(60, n, 8, 1005)
+    X, rep, opts = run_inv_root(A, "inv4", 2, 8, 1e-6, 30, "3xtf32", S)
+    for b in range(batch):
+        assert rep["status"][b] == o.OK
+        it = rep["iters"][b]
+        Xo, infos = o.inv_root_ref(A[b], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
+        for ps, info in enumerate(infos):
+            np.testing.assert_allclose(rep["alpha"][b, ps, :it[ps]], info.alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= 1e-5
+        As = 0.5 * (A[b].astype(np.float64) + A[b].astype(np.float64).T)
+        assert relerr(X[b], o.spd_power_eigh(As, -0.25)) <= 1e-5
+
+
 def test_inv_root_tf32_well_conditioned():
     """TF32 path on cond 10 (the Shampoo statistics regime): error <= 1e-3."""
     n, batch = 256, 2

@@ -60,6 +60,25 @@ def test_small_inv_root_parity(n, d, power):
         assert relerr(X[b], o.spd_power_eigh(A[b], q)) <= TOL_FP32
 
 
+def test_small_nonsymmetric_input_takes_symmetric_part():
+    """A block that is SPD plus a small antisymmetric part: the on-chip path
+    starts from (A + A^T) / (2c) as the oracle does."""
+    P = prism()
+    n = 40
+    A = synth.spd_batch(n, 1, 1e-2, 1.0, 205)
+    K = synth.gaussian((n, n), 1e-2, 206)
+    A[0] = A[0] + (K - K.T)
+    S = synth.sketch_stack(80, n, 8, 1205)
+    opts = P.make_opts(d=2, p=8, tol=1e-6, max_iter=40, prec="3xtf32")
+    X, rep = P.matfn_inv_root(to_dev(torch, A), "inv4", opts, to_dev(torch, S))
+    X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
+    assert rep["status"][0] == o.OK
+    Xo, _ = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S, force_iters=rep["iters"][0])
+    assert relerr(X[0], Xo) <= TOL_FP32
+    As = 0.5 * (A[0].astype(np.float64) + A[0].astype(np.float64).T)
+    assert relerr(X[0], o.spd_power_eigh(As, -0.25)) <= TOL_FP32
+
+
 def test_small_sketch_width_16_degree_2():
     """p = 16, d = 2 fills the four sketch slots of one matrix buffer."""
     P = prism()

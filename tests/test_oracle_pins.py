@@ -274,6 +274,22 @@ def test_inverse_roots_vs_eigh_and_identities(d):
     np.testing.assert_allclose(Xs @ Xs, A, atol=1e-10)
 
 
+def test_inverse_root_takes_symmetric_part():
+    """A non-symmetric input whose symmetric part is the SPD matrix with a
+    known spectrum: the root is that of the symmetric part, from the
+    closed form Q diag(lambda^(-1/4)) Q^T (an antisymmetric addition leaves
+    the symmetric part unchanged)."""
+    n = 24
+    lam = np.exp(np.random.default_rng(11).uniform(np.log(1e-2), np.log(1.0), n))
+    A, Q = spd(n, lam, 12)
+    K = np.random.default_rng(13).standard_normal((n, n)) * 0.05
+    opts = o.PrismOpts(d=2, p=4, lo=0.375, tol=1e-13, max_iter=60, stall_below=0.0)
+    S = np.random.default_rng(14).standard_normal((200, n, 4))
+    X, infos = o.inv_root_ref(A + (K - K.T), o.POW_INV4, opts, S)
+    assert [i.status for i in infos] == [o.OK, o.OK]
+    np.testing.assert_allclose(X, (Q * lam ** -0.25) @ Q.T, atol=1e-10)
+
+
 def test_eigh_reference_on_diagonal():
     lam = np.array([4.0, 1.0, 0.0625, 16.0])
     np.testing.assert_allclose(o.spd_power_eigh(np.diag(lam), -0.25),
