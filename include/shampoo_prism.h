@@ -281,6 +281,10 @@ int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const floa
 /* Human-readable name of a status code (static storage). */
 const char* shp_status_string(int status);
 
+/* Name of the CUDA error (e.g. "cudaErrorInvalidValue") behind the latest
+ * SHP_ECUDA returned on this host thread, or "none" (static storage). */
+const char* shp_last_cuda_error(void);
+
 /* Library version, e.g. "0.1.0" (static storage). */
 const char* shp_version(void);
 

@@ -27,7 +27,7 @@ SHP_NOALLOC_SCRATCH_BYTES = 4 << 20
 EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar", "matfn_polar_varsize",
            "matfn_sign",
            "prism_alpha_fit", "shampoo_apply", "shampoo_apply_ex", "shp_matmul", "shp_split_tf32",
-           "shp_kernel_launches", "prism_alpha_fit_noalloc", "shp_status_string",
+           "shp_kernel_launches", "prism_alpha_fit_noalloc", "shp_status_string", "shp_last_cuda_error",
            "shp_version")
 
 
@@ -73,6 +73,7 @@ _SIGS = {
     "shp_kernel_launches": (ctypes.c_uint64, []),
     "prism_alpha_fit_noalloc": (_INT, [_P, _I64, _I64, _P, _INT, _INT, _F, _F, _P, _P, _P]),
     "shp_status_string": (ctypes.c_char_p, [_INT]),
+    "shp_last_cuda_error": (ctypes.c_char_p, []),
     "shp_version": (ctypes.c_char_p, []),
 }
 

@@ -168,9 +168,16 @@ Operand op(const void* hi, const float* lo, bool mn, int64_t ld, int64_t bs) {
   return o;
 }
 
-#define CK(x)                                  \
-  do {                                         \
-    if ((x) != cudaSuccess) return SHP_ECUDA; \
+// The CUDA error behind this host thread's latest SHP_ECUDA.
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+#define CK(x)                           \
+  do {                                  \
+    const cudaError_t ck_e_ = (x);      \
+    if (ck_e_ != cudaSuccess) {         \
+      g_last_cuda = ck_e_;              \
+      return SHP_ECUDA;                 \
+    }                                   \
   } while (0)
 
 // The sketch passes and the alpha solve of iteration k = *ctl.it:
@@ -184,10 +191,10 @@ int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass,
   const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
   if (!o->fixed_alpha) {
     CK(sketch_pass(Rs, nullptr, n, nn, S_pass, 0, V + np, vbs, o->p, batch, ctl.active, ctl.it,
-                   np, st));
+                   np, st, ctl.tmo));
     for (int j = 2; j <= 2 * o->d + 1; ++j)
       CK(sketch_pass(Rs, nullptr, n, nn, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
-                     ctl.active, nullptr, 0, st));
+                     ctl.active, nullptr, 0, st, ctl.tmo));
   }
   AdaptiveDeg ad{o->adaptive_degree, o->raise_above, ctl.deg, ctl.act1, ctl.act2, rep_degree};
   CK(alpha_solve(V, n, o->p, o->d, batch, o->lo, o->hi, o->fixed_alpha, ctl.active, ctl.alpha,
@@ -404,6 +411,11 @@ int shp_matmul(const void* A, const float* A_lo, int a_trans, const void* B, con
   CK(gemm_tc(mode, a, b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
              static_cast<int>(batch), e, static_cast<cudaStream_t>(stream)));
   return SHP_OK;
+}
+
+const char* shp_last_cuda_error(void) {
+  if (g_last_cuda == cudaSuccess) return "none";
+  return cudaGetErrorName(g_last_cuda);
 }
 
 const char* shp_status_string(int s) {

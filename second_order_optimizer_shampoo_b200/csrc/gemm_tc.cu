@@ -738,8 +738,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map over [batch][rows][inner] with the given box, 128-byte swizzle,
-// zero fill outside the tensor.
+// 3-D map over [batch][rows][inner] with the given box and swizzle, zero
+// fill outside the tensor.
 bool make_map(CUtensorMap* m, const void* ptr, int esz, int64_t inner, int64_t rows,
               int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows,
               CUtensorMapSwizzle swz) {
@@ -850,6 +850,12 @@ cudaError_t dispatch_pair(bool pair, bool amn, bool bmn, const CUtensorMap& a,
 }
 
 }  // namespace
+
+bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
+                     int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows) {
+  return make_map(m, ptr, 4, inner, rows, batch, ld, bstride, box_inner, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
 
 cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, int K,
                     int batch, const EpiParams& ep, cudaStream_t st) {

@@ -99,14 +99,22 @@ struct EpiParams {
 cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, int K,
                     int batch, const EpiParams& ep, cudaStream_t st);
 
+// 3-D fp32 tensor map over [batch][rows][inner] (row stride ld, batch stride
+// bstride, in elements) with a box of box_rows x box_inner, no swizzle and
+// zero fill outside the tensor.  False if the driver rejects it.
+bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
+                     int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows);
+
 // ---- PRISM sketch and alpha (sketch_alpha.cu)
 // Vout[b] = R[b] * Vin[b]; R is n x n (hi + lo when lo != null); V is n x p.
 // vin_bstride == 0 shares Vin across the batch.  When `it` is non-null the
 // input is Vin + (*it) * it_stride (the sketch slice of the current iteration).
+// A pipeline wait of the bulk-copy variant that runs out sets tmo[b] (if
+// non-null) to ST_ETIMEOUT.
 cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
                         const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
                         int p, int batch, const int* active, const int* it, int64_t it_stride,
-                        cudaStream_t st);
+                        cudaStream_t st, int* tmo = nullptr);
 // V is stored per block as [2d+2][n][p] (slot j holds V_j; slot 0 unused).
 // Gram of V_d..V_{2d+1}, the
 // quartic J(alpha) and its minimiser on [lo, hi]; writes alpha[b] and, when

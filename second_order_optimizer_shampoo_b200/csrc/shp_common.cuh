@@ -63,6 +63,10 @@ SHP_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+SHP_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ----------------------------------------------------------------- TMA
 SHP_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -17,6 +17,7 @@
 // Kernels: the skinny products V_j = R V_{j-1} on CUDA cores (fp32 FMA, HBM
 // bound), the Gram/quartic/argmin per block (fp64), and the stop test.
 #include <math.h>
+#include <stdlib.h>
 
 #include "internal.h"
 #include "prism_scalar.cuh"
@@ -28,6 +29,45 @@ namespace {
 
 constexpr int SK_THREADS = 256;
 constexpr int SK_GROUPS = 2;  // row groups per warp in one CTA
+
+// Warp reduction of ROWS x P row sums (acc[r * P + j], one partial per lane)
+// by recursive halving: at the step with offset o each lane keeps the half of
+// its values selected by its lane bit o and adds the partner's copy of that
+// half, so 31 shuffles (for 32 values) leave lane l holding the total of
+// value l, where a shuffle tree per value would take 5 per value.  Stores
+// row0 + r, column j of Vb (rows >= n and columns >= p are not stored).
+template <int ROWS, int P>
+SHP_DEV void store_row_sums(float (&acc)[ROWS * P], int lane, int64_t row0, int64_t n, int p,
+                            float* Vb) {
+  constexpr int NV = ROWS * P;
+  static_assert(NV == 16 || NV == 32 || NV == 64, "16, 32 or 64 sums per warp");
+  constexpr int STEPS = NV >= 32 ? 5 : 4;
+#pragma unroll
+  for (int st = 0; st < STEPS; ++st) {
+    const int o = 16 >> st;
+    const int h = (NV >> st) / 2;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = up ? acc[i] : acc[i + h];
+      const float keep = up ? acc[i + h] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  if constexpr (NV == 16) {  // lanes l and l ^ 1 hold halves of value l >> 1
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+    if ((lane & 1) == 0) {
+      const int idx = lane >> 1, r = idx / P, j = idx % P;
+      if (row0 + r < n && j < p) Vb[(row0 + r) * p + j] = acc[0];
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < NV / 32; ++k) {  // this lane holds values lane * NV/32 + k
+      const int idx = lane * (NV / 32) + k, r = idx / P, j = idx % P;
+      if (row0 + r < n && j < p) Vb[(row0 + r) * p + j] = acc[k];
+    }
+  }
+}
 
 // Vout = R * Vin for one block: HBM-bound, every byte of R read once.
 // Each warp owns ROWS consecutive rows of R per group and streams them with
@@ -65,11 +105,9 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
     int64_t roff[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) roff[r] = (row0 + r < n ? row0 + r : n - 1) * n;
-    float acc[ROWS][P];
+    float acc[ROWS * P];
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r)
-#pragma unroll
-      for (int j = 0; j < P; ++j) acc[r][j] = 0.f;
+    for (int i = 0; i < ROWS * P; ++i) acc[i] = 0.f;
 
     for (int64_t c0 = 0; c0 < n; c0 += CK) {
       if (!(one_chunk && g > 0)) {
@@ -118,7 +156,7 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
           const float4 v1 = *reinterpret_cast<const float4*>(&Vs[j][cc + 128]);
 #pragma unroll
           for (int r = 0; r < ROWS; ++r) {
-            float a = acc[r][j];
+            float a = acc[r * P + j];
             a = fmaf(x0[r].x, v0.x, a);
             a = fmaf(x0[r].y, v0.y, a);
             a = fmaf(x0[r].z, v0.z, a);
@@ -126,20 +164,193 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
             a = fmaf(x1[r].x, v1.x, a);
             a = fmaf(x1[r].y, v1.y, a);
             a = fmaf(x1[r].z, v1.z, a);
-            acc[r][j] = fmaf(x1[r].w, v1.w, a);
+            acc[r * P + j] = fmaf(x1[r].w, v1.w, a);
           }
         }
       }
     }
+    store_row_sums<ROWS, P>(acc, lane, row0, n, p, Vout + b * obs);
+  }
+}
+
+// The same product with R streamed through shared memory by TMA, for blocks
+// whose V fits in shared memory whole: a persistent grid, one CTA per SM,
+// each CTA a contiguous range of work items (RPI = 8 * ROWS rows of one
+// block).  Warp 8 (one lane) issues one tiled load per stage (SC = 256
+// columns x RPI rows, zero filled past the edges) into an NST-deep ring, so
+// up to NST * 32 KB of R is in flight per SM whatever the register file
+// holds; warps 0..7 each reduce ROWS rows of a stage against Vs exactly as
+// k_sketch does from registers.  Every wait, the V hand-over between items
+// of different blocks included, is an mbarrier wait with a bound; one that
+// runs out marks the block's timeout flag and the CTA unwinds after its
+// copies have landed.
+constexpr int ST_SC = 256;  // columns per stage
+constexpr int ST_NST = 4;   // ring depth
+constexpr int ST_CONS = 8;  // consumer warps
+
+template <int P>
+struct SkTma {
+  static constexpr int ROWS = P <= 8 ? 4 : 2;
+  static constexpr int RPI = ST_CONS * ROWS;        // rows per work item
+  static constexpr int STAGE_FLOATS = RPI * ST_SC;  // 32 KB (P <= 8) or 16 KB
+  static size_t smem_bytes(int64_t n) {
+    const int64_t ldv = (n + ST_SC - 1) / ST_SC * ST_SC + 4;
+    return 128 + static_cast<size_t>(ST_NST) * STAGE_FLOATS * 4 + static_cast<size_t>(P) * ldv * 4 +
+           (2 * ST_NST + 2) * 8 + 16;
+  }
+};
+
+// A wait that ran out: flag the block and leave (every other waiter then
+// runs out too, or sees the flag first).
+SHP_DEV void sketch_give_up(volatile int* abort_flag, int* tmo, int b, int lane) {
+  *abort_flag = 1;
+  __threadfence_block();
+  if (lane == 0 && tmo != nullptr) atomicExch(&tmo[b], ST_ETIMEOUT);
+}
+
+template <int P>
+__global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
+    k_sketch_tma(const __grid_constant__ CUtensorMap tR, int64_t n,
+                 const float* __restrict__ Vin, int64_t vbs, float* __restrict__ Vout,
+                 int64_t obs, int p, int batch, const int* __restrict__ active,
+                 const int* __restrict__ it, int64_t it_stride, int* tmo) {
+  count_kernel_run();
+  using K = SkTma<P>;
+  constexpr int ROWS = K::ROWS, RPI = K::RPI;
+  constexpr int NCT = 32 * ST_CONS;  // consumer threads
+  extern __shared__ __align__(16) uint8_t sk_smem[];
+  float* ring = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(sk_smem) + 127) & ~static_cast<uintptr_t>(127));
+  const int64_t ldv = (n + ST_SC - 1) / ST_SC * ST_SC + 4;
+  float* Vs = ring + ST_NST * K::STAGE_FLOATS;
+  uint64_t* full = reinterpret_cast<uint64_t*>(Vs + P * ldv);
+  uint64_t* empty = full + ST_NST;
+  uint64_t* vbar = empty + ST_NST;  // [2] old V released, new V staged
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(vbar + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gpb = (n + RPI - 1) / RPI;  // items per block
+  const int64_t items = gpb * batch;
+  const int64_t i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
+  const int nch = static_cast<int>((n + ST_SC - 1) / ST_SC);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tR);
+    for (int s = 0; s < ST_NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ST_CONS);
+    }
+    mbar_init(&vbar[0], ST_CONS);
+    mbar_init(&vbar[1], ST_CONS);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == ST_CONS) {
+    // ---------------- producer: one lane issues every copy
+    if (lane == 0) {
+      int kit = 0;
+      int last_b = -1;
+      for (int64_t t = i0; t < i1 && !*abort_flag; ++t) {
+        const int b = static_cast<int>(t / gpb);
+        if (active != nullptr && active[b] == 0) continue;
+        const int r0 = static_cast<int>((t % gpb) * RPI);
+        last_b = b;
+        for (int c = 0; c < nch; ++c, ++kit) {
+          const int s = kit % ST_NST;
+          if (kit >= ST_NST && !mbar_wait(&empty[s], ((kit / ST_NST) - 1) & 1)) {
+            sketch_give_up(abort_flag, tmo, b, 0);
+            break;
+          }
+          // the full box lands (zeros past the edges); x = c * 256 is aligned
+          mbar_arrive_expect_tx(&full[s], K::STAGE_FLOATS * 4u);
+          tma_load_3d(ring + s * K::STAGE_FLOATS, &tR, &full[s], c * ST_SC, r0, b);
+        }
+      }
+      // every copy issued has landed before the CTA may exit
+      const int first = kit > ST_NST ? kit - ST_NST : 0;
+      for (int k = first; k < kit; ++k)
+        if (!mbar_wait(&full[k % ST_NST], (k / ST_NST) & 1) && last_b >= 0)
+          sketch_give_up(abort_flag, tmo, last_b, 0);
+    }
+    return;
+  }
+
+  // ---------------- consumers: warps 0..7
+  int kit = 0, ns = 0;  // stages consumed, V stagings
+  int cur_b = -1;
+  for (int64_t t = i0; t < i1; ++t) {
+    if (*abort_flag) break;
+    const int b = static_cast<int>(t / gpb);
+    if (active != nullptr && active[b] == 0) continue;
+    if (b != cur_b) {  // stage V of block b (all consumer warps; the producer runs on)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&vbar[0]);  // this warp is done with the old V
+      if (!mbar_wait(&vbar[0], ns & 1)) {
+        sketch_give_up(abort_flag, tmo, b, lane);
+        break;
+      }
+      const float* V = Vin + b * vbs + (it != nullptr ? static_cast<int64_t>(*it) * it_stride : 0);
+      for (int64_t idx = threadIdx.x; idx < ldv * (P / 4); idx += NCT) {
+        const int64_t col = idx / (P / 4);
+        const int q = 4 * static_cast<int>(idx % (P / 4));
+        const float* src = V + col * p + q;
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
+        for (int e = 0; e < 4; ++e)
+          Vs[(q + e) * ldv + col] = (col < n && q + e < p) ? __ldg(src + e) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&vbar[1]);  // this warp's part of V is written
+      if (!mbar_wait(&vbar[1], ns & 1)) {
+        sketch_give_up(abort_flag, tmo, b, lane);
+        break;
+      }
+      ++ns;
+      cur_b = b;
+    }
+    const int64_t r0 = (t % gpb) * RPI;
+    float acc[ROWS * P];
+#pragma unroll
+    for (int i = 0; i < ROWS * P; ++i) acc[i] = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nch; ++c, ++kit) {
+      const int s = kit % ST_NST;
+      if (*abort_flag || !mbar_wait(&full[s], (kit / ST_NST) & 1)) {
+        sketch_give_up(abort_flag, tmo, b, lane);
+        ok = false;
+        break;
+      }
+      const float* st = ring + s * K::STAGE_FLOATS + (warp * ROWS) * ST_SC + lane * 4;
+      float4 x0[ROWS], x1[ROWS];
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        x0[r] = *reinterpret_cast<const float4*>(st + r * ST_SC);
+        x1[r] = *reinterpret_cast<const float4*>(st + r * ST_SC + 128);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // this warp's reads of the stage are done
+      // past the last column: R is zero filled and Vs zero padded
+      const float* vp = Vs + static_cast<int64_t>(c) * ST_SC + lane * 4;
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const float sum = warp_sum(acc[r][j]);
-        const int64_t row = row0 + r;
-        if (lane == 0 && row < n && j < p) Vout[b * obs + row * p + j] = sum;
+        const float4 v0 = *reinterpret_cast<const float4*>(vp + j * ldv);
+        const float4 v1 = *reinterpret_cast<const float4*>(vp + j * ldv + 128);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          float a = acc[r * P + j];
+          a = fmaf(x0[r].x, v0.x, a);
+          a = fmaf(x0[r].y, v0.y, a);
+          a = fmaf(x0[r].z, v0.z, a);
+          a = fmaf(x0[r].w, v0.w, a);
+          a = fmaf(x1[r].x, v1.x, a);
+          a = fmaf(x1[r].y, v1.y, a);
+          a = fmaf(x1[r].z, v1.z, a);
+          acc[r * P + j] = fmaf(x1[r].w, v1.w, a);
+        }
       }
     }
+    if (!ok) break;
+    store_row_sums<ROWS, P>(acc, lane, r0 + warp * ROWS, n, p, Vout + b * obs);
   }
 }
 
@@ -172,6 +383,43 @@ struct AlphaArgs {
   int* rep_deg;
 };
 
+// This thread's partial sums of <V_i, V_j> (i <= j < NV, packed row by row)
+// over elements threadIdx.x + k * AL_THREADS; NV is a compile-time constant so
+// that the 15 partials and the loaded values stay in registers, and two
+// elements are loaded per step to keep 2 NV loads in flight.
+template <int NV>
+SHP_DEV void gram_partials(const float* __restrict__ Vb, int64_t len, double (&part)[15]) {
+#pragma unroll
+  for (int i = 0; i < 15; ++i) part[i] = 0.0;
+  int64_t e = threadIdx.x;
+  for (; e + AL_THREADS < len; e += 2 * AL_THREADS) {
+    float x[NV], y[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      x[i] = __ldg(Vb + i * len + e);
+      y[i] = __ldg(Vb + i * len + e + AL_THREADS);
+    }
+    int idx = 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = i; j < NV; ++j, ++idx)
+        part[idx] = fma(static_cast<double>(x[i]), static_cast<double>(x[j]),
+                        fma(static_cast<double>(y[i]), static_cast<double>(y[j]), part[idx]));
+  }
+  if (e < len) {
+    float x[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) x[i] = __ldg(Vb + i * len + e);
+    int idx = 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = i; j < NV; ++j, ++idx)
+        part[idx] = fma(static_cast<double>(x[i]), static_cast<double>(x[j]), part[idx]);
+  }
+}
+
 __global__ void __launch_bounds__(AL_THREADS) k_alpha(AlphaArgs g) {
   count_kernel_run();
   const int b = blockIdx.x;
@@ -196,15 +444,12 @@ __global__ void __launch_bounds__(AL_THREADS) k_alpha(AlphaArgs g) {
   const int64_t len = g.n * g.p;
   const float* Vb = g.V + b * g.vbs + static_cast<int64_t>(first) * len;
   double part[15];
-#pragma unroll
-  for (int i = 0; i < 15; ++i) part[i] = 0.0;
-  for (int64_t e = threadIdx.x; e < len; e += AL_THREADS) {
-    double x[5];
-    for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(Vb[i * len + e]);
-    int idx = 0;
-    for (int i = 0; i < nv; ++i)
-      for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
-  }
+  if (nv == 3)
+    gram_partials<3>(Vb, len, part);
+  else if (nv == 4)
+    gram_partials<4>(Vb, len, part);
+  else
+    gram_partials<5>(Vb, len, part);
   __shared__ double red[AL_THREADS / 32][15];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
@@ -287,11 +532,55 @@ __global__ void k_control(BlockState* bs, int* active, const int* it, int batch,
 
 }  // namespace
 
+namespace {
+
+template <int P>
+bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin, int64_t vbs,
+                       float* Vout, int64_t obs, int p, int batch, const int* active,
+                       const int* it, int64_t it_stride, int* tmo, cudaStream_t st,
+                       cudaError_t* err) {
+  const size_t smem = SkTma<P>::smem_bytes(n);
+  if (smem > 200 * 1024) return false;  // V does not fit whole: the register kernel
+  CUtensorMap tR;
+  if (!tensor_map_rows(&tR, R, n, n, batch, n, rbs, ST_SC, SkTma<P>::RPI)) return false;
+  auto kern = k_sketch_tma<P>;
+  *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(smem));
+  if (*err != cudaSuccess) return true;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t items = (n + SkTma<P>::RPI - 1) / SkTma<P>::RPI * batch;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  kern<<<grid, 32 * (ST_CONS + 1), smem, st>>>(tR, n, Vin, vbs, Vout, obs, p, batch, active, it,
+                                                it_stride, tmo);
+  *err = cudaGetLastError();
+  return true;
+}
+
+}  // namespace
+
 cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
                         const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
                         int p, int batch, const int* active, const int* it, int64_t it_stride,
-                        cudaStream_t st) {
+                        cudaStream_t st, int* tmo) {
   if (batch <= 0 || n <= 0) return cudaSuccess;
+  // plain fp32 R with 16-byte aligned rows: the bulk-copy kernel when V fits
+  if (Rlo == nullptr && (reinterpret_cast<uintptr_t>(Rhi) & 15) == 0 && n % 4 == 0 &&
+      r_bstride % 4 == 0 && getenv("SHP_SKETCH_REGS") == nullptr) {
+    cudaError_t e = cudaSuccess;
+    bool done = false;
+    if (p <= 4)
+      done = launch_sketch_tma<4>(Rhi, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
+                                  batch, active, it, it_stride, tmo, st, &e);
+    else if (p <= 8)
+      done = launch_sketch_tma<8>(Rhi, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
+                                  batch, active, it, it_stride, tmo, st, &e);
+    else if (p <= 16)
+      done = launch_sketch_tma<16>(Rhi, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
+                                   batch, active, it, it_stride, tmo, st, &e);
+    if (done) return e;
+  }
   const int rows = (p <= 8 ? 4 : 2) * 8 * SK_GROUPS;  // rows per CTA (ROWS x 8 warps x groups)
   dim3 grid(static_cast<unsigned>((n + rows - 1) / rows), batch);
   if (p <= 4)

@@ -27,7 +27,10 @@ def version() -> str:
 
 def _check(code: int, name: str):
     if code != A.SHP_OK:
-        raise RuntimeError(f"{name} failed: {status_string(code)} ({code})")
+        extra = ""
+        if code == A.SHP_ECUDA:
+            extra = f", {A.lib().shp_last_cuda_error().decode()}"
+        raise RuntimeError(f"{name} failed: {status_string(code)} ({code}{extra})")
 
 
 def _dev(*ts):

@@ -31,6 +31,8 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
     assert L.shp_version().decode().count(".") == 2
     assert L.shp_status_string(A.SHP_ESTALL).decode() == "residual stalled"
+    # argument checks fail before any CUDA call, so no CUDA error is recorded
+    assert L.shp_last_cuda_error().decode() == "none"
 
 
 def opts(**kw):
