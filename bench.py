@@ -41,6 +41,10 @@ TF32_OVER_BF16 = 1.1 / 2.25
 # 41.8 MB written) scaled x4 by the blocks processed, as every operand and
 # output grows with the batch
 GEMM_TRAFFIC_PER_LAUNCH = 4 * (289.454e6 + 41.826e6)
+# dram__bytes_read.sum + dram__bytes_write.sum of one k_sketch_tma<8> launch
+# over 48 x 1024^2 (201.393 MB read, 4.802 MB written), scaled x 64/48 by the
+# rows processed and x 5 for the passes of one alpha fit (d = 2)
+SKETCH_TRAFFIC_PER_FIT = 5 * 64 / 48 * (201.393e6 + 4.802e6)
 
 
 def workload_config(world):
@@ -533,6 +537,65 @@ def polar_leg(args, dev, stream):
             "note": "symmetric products counted n(n+1)K; computed as full GEMMs"}
 
 
+def sketch_leg(R, S0, stream, peaks, peak_src):
+    """Roofline of the sketch kernel (HBM bound): the alpha fit of d = 2 on a
+    stack of n x n fp32 residuals, 5 passes V_j = R V_{j-1} (R read once per
+    pass; 256 MiB at the config-3 size, larger than L2) plus the per-block
+    Gram/argmin, replayed from a CUDA graph as inside the step (no host gaps)."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism
+    batch, n = R.shape[0], R.shape[-1]
+    p = S0.shape[-1]
+    v_dim = 2 * D + 1
+    for _ in range(3):
+        prism.prism_alpha_fit(R, S0, D, 0.375, 1.0)
+    torch.cuda.synchronize()
+    fit_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(fit_graph):
+        prism.prism_alpha_fit(R, S0, D, 0.375, 1.0)
+    for _ in range(3):
+        fit_graph.replay()
+    torch.cuda.synchronize()
+    reps = 20
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for _ in range(reps):
+        fit_graph.replay()
+    k1.record(stream)
+    torch.cuda.synchronize()
+    fit_ms = k0.elapsed_time(k1) / reps
+    del fit_graph
+    sk_bytes = v_dim * (batch * n * n * 4 + 2 * batch * n * p * 4)  # R once, V in and out
+    sk_gbs = sk_bytes / (fit_ms / 1e3) / 1e9
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    full = batch == BATCH and n == N and p == P
+    return {
+        "kernel": f"k_sketch_tma<8> x 5 + k_alpha (alpha fit, d = 2, {batch} x {n}^2, p = {p})",
+        "bound": "hbm", "achieved": sk_gbs, "peak": hbm, "unit": "GB/s", "frac": sk_gbs / hbm,
+        "traffic": SKETCH_TRAFFIC_PER_FIT if full else None, "algorithmic_bytes": sk_bytes,
+        "ms_per_fit": fit_ms,
+        "peak_note": f"{peak_src} STREAM-style copy bandwidth; the alpha kernel's time is included",
+    }
+
+
+def sketch_only(args):
+    """The sketch leg alone on --batch seeded N(0, 0.01^2) symmetric residuals
+    1024 x 1024 (for profiling k_sketch_tma)."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import synth
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    R = torch.randn(args.batch, N, N, device=dev, generator=g) * 0.01
+    R = (R + R.transpose(1, 2)).contiguous()
+    S0 = torch.from_numpy(synth.sketch_stack(1, N, P, SEED_S)[0]).to(dev)
+    peaks, src = load_peaks()
+    print(json.dumps(sketch_leg(R, S0, torch.cuda.current_stream(), peaks, src)))
+    return 0
+
+
 # ------------------------------------------------------------------ our leg
 def main():
     global BATCH
@@ -549,9 +612,10 @@ def main():
                          "on the host first)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the Shampoo-step, GEMM-count and single-block legs")
-    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar"],
-                    help="run only the batched 3xTF32 GEMM, the small-block kernel or the "
-                         "polar leg (for profiling; --batch sets the GEMM/small batch)")
+    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar", "sketch"],
+                    help="run only the batched 3xTF32 GEMM, the small-block kernel, the "
+                         "polar leg or the sketch leg (for profiling; --batch sets the "
+                         "GEMM/small/sketch batch)")
     ap.add_argument("--batch", type=int, default=BATCH)
     args = ap.parse_args()
     if args.impl == "reference":
@@ -560,6 +624,8 @@ def main():
         return gemm_only(args)
     if args.kernel == "small":
         return small_only(args)
+    if args.kernel == "sketch":
+        return sketch_only(args)
     if args.kernel == "polar":
         import torch
         print(json.dumps(polar_leg(args, torch.device("cuda", 0), torch.cuda.current_stream())))
@@ -720,6 +786,8 @@ def main():
         "ms_per_launch": gemm_ms,
     }
 
+    sketch_roof = sketch_leg(A, S[0], stream, peaks, peak_src)
+
     polar = None if args.no_polar else polar_leg(args, dev, stream)
     extra = not args.no_extra and world == 1
     step2 = shampoo_step_leg(args, dev, stream) if extra else None
@@ -760,6 +828,7 @@ def main():
                     "note": "two buffer sets; H2D of step i+1 and D2H of step i-1 overlap "
                             "step i on their own streams"},
             "roofline": roofline,
+            "roofline_sketch": sketch_roof,
             "polar": polar,
             "small_blocks": small,
             "shampoo_step_1024": step2,

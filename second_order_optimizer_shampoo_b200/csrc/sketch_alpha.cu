@@ -250,10 +250,15 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
     // ---------------- producer: one lane issues every copy
     if (lane == 0) {
       int kit = 0;
-      int last_b = -1;
+      int last_b = -1, seen_b = -1;
+      bool seen_on = true;
       for (int64_t t = i0; t < i1 && !*abort_flag; ++t) {
         const int b = static_cast<int>(t / gpb);
-        if (active != nullptr && active[b] == 0) continue;
+        if (b != seen_b) {  // one global read per block, not per item
+          seen_b = b;
+          seen_on = active == nullptr || active[b] != 0;
+        }
+        if (!seen_on) continue;
         const int r0 = static_cast<int>((t % gpb) * RPI);
         last_b = b;
         for (int c = 0; c < nch; ++c, ++kit) {
@@ -278,11 +283,16 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
 
   // ---------------- consumers: warps 0..7
   int kit = 0, ns = 0;  // stages consumed, V stagings
-  int cur_b = -1;
+  int cur_b = -1, seen_b = -1;
+  bool seen_on = true;
   for (int64_t t = i0; t < i1; ++t) {
     if (*abort_flag) break;
     const int b = static_cast<int>(t / gpb);
-    if (active != nullptr && active[b] == 0) continue;
+    if (b != seen_b) {  // one global read per block, not per item
+      seen_b = b;
+      seen_on = active == nullptr || active[b] != 0;
+    }
+    if (!seen_on) continue;
     if (b != cur_b) {  // stage V of block b (all consumer warps; the producer runs on)
       __syncwarp();
       if (lane == 0) mbar_arrive(&vbar[0]);  // this warp is done with the old V
@@ -335,18 +345,23 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
       for (int j = 0; j < P; ++j) {
         const float4 v0 = *reinterpret_cast<const float4*>(vp + j * ldv);
         const float4 v1 = *reinterpret_cast<const float4*>(vp + j * ldv + 128);
+        // the ROWS chains advance together: consecutive FMAs are independent
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-          float a = acc[r * P + j];
-          a = fmaf(x0[r].x, v0.x, a);
-          a = fmaf(x0[r].y, v0.y, a);
-          a = fmaf(x0[r].z, v0.z, a);
-          a = fmaf(x0[r].w, v0.w, a);
-          a = fmaf(x1[r].x, v1.x, a);
-          a = fmaf(x1[r].y, v1.y, a);
-          a = fmaf(x1[r].z, v1.z, a);
-          acc[r * P + j] = fmaf(x1[r].w, v1.w, a);
-        }
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x0[r].x, v0.x, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x0[r].y, v0.y, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x0[r].z, v0.z, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x0[r].w, v0.w, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x1[r].x, v1.x, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x1[r].y, v1.y, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x1[r].z, v1.z, acc[r * P + j]);
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x1[r].w, v1.w, acc[r * P + j]);
       }
     }
     if (!ok) break;
@@ -544,12 +559,18 @@ bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin,
   CUtensorMap tR;
   if (!tensor_map_rows(&tR, R, n, n, batch, n, rbs, ST_SC, SkTma<P>::RPI)) return false;
   auto kern = k_sketch_tma<P>;
-  *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(smem));
-  if (*err != cudaSuccess) return true;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // the attribute allows the largest size used (set once per device and P;
+  // calls from several host threads at once may each set it, which is safe)
+  static int set_for_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = -1;
+  if (dev < 0 || set_for_dev[dev] == 0) {
+    *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (*err != cudaSuccess) return true;
+    if (dev >= 0) set_for_dev[dev] = 1;
+  }
+  int sms = 148;
+  if (dev >= 0) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t items = (n + SkTma<P>::RPI - 1) / SkTma<P>::RPI * batch;
   const int grid = static_cast<int>(items < sms ? items : sms);
   kern<<<grid, 32 * (ST_CONS + 1), smem, st>>>(tR, n, Vin, vbs, Vout, obs, p, batch, active, it,
