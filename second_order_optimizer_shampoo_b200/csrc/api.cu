@@ -862,8 +862,13 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
       {  // R = I - X^T X (tall) or I - X X^T (wide), and ||R||_F^2
         EpiParams e = epi(EPI_RESID, rfmt, w.Rhi, w.Rlo, k, kk, K, K, &ctl);
         if (rfmt == OUT_SPLIT) e.out_plain = w.Rs;
-        e.sym = 1;  // X^T X: upper-triangle tiles, mirrored
-        if (sign)  // X X (X symmetric)
+        // X^T X is a Gram matrix, symmetric in any arithmetic: upper-triangle
+        // tiles, mirrored.  X X (sign) is symmetric only while X is, and X
+        // picks up a rounding-level asymmetry from X + X Delta: keeping one
+        // triangle of X X there raised the residual floor tenfold (fp32,
+        // 512^2: 8e-6 instead of 3.5e-7), so it is formed in full.
+        e.sym = sign ? 0 : 1;
+        if (sign)  // X X
           CK(gemm_tc(xmode, op(w.Xhi[cur], w.Xlo[cur], false, n, mn),
                      op(w.Xhi[cur], w.Xlo[cur], true, n, mn), K, K, M, B, e, st));
         else if (tall)
@@ -883,7 +888,7 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
       if (o->d == 2) {  // Delta = g - I = R/2 + alpha R^2, stored like X
         EpiParams e = epi(EPI_GPOLY, xfmt, w.ghi, w.glo, k, kk, K, K, &ctl);
         if (o->adaptive_degree) e.active = ctl.act2;
-        e.sym = 1;  // R symmetric (mirrored above), so R R and Delta are too
+        e.sym = sign ? 0 : 1;  // R exactly symmetric (mirrored above): R R and Delta too
         e.aux_hi = w.Rhi;
         e.aux_lo = w.Rlo;
         e.aux_fmt = rfmt;
