@@ -21,6 +21,8 @@ Readings taken where the pages are silent (each is listed in the design doc):
   interval [1/2, 1] for d = 1 fixes its first coefficient at 1/2.
 * A^(-1/4) is two nested coupled square-root passes: pass 1 on B = A/||A||_F
   gives Y1 ~ B^(1/2); pass 2 on Y1 gives Z2 ~ Y1^(-1/2) = B^(-1/4).
+* The inverse root is stated for symmetric A: a non-symmetric input is
+  replaced by its symmetric part, B = (A + A^T) / (2 ||A||_F).
 * alpha minimises the sketched objective ||r(R_k; alpha) S_k||_F^2 over
   [lo, hi] (global minimum of a quartic; ties go to the smaller alpha; a
   constant objective gives alpha = lo).
