@@ -175,6 +175,15 @@ def oracle_sample(A_block, S_np, seconds_hint=None):
     return dt, block_flops([i.iters for i in infos], N)
 
 
+def eigh_sample(A_block):
+    """Time the eigendecomposition route to A^(-1/4) (float64 LAPACK eigh) on
+    one block: the direct method the iteration replaces; returns seconds."""
+    from oracle import prism_ref as o
+    t0 = time.perf_counter()
+    o.spd_power_eigh(A_block, -0.25)
+    return time.perf_counter() - t0
+
+
 def run_reference(args):
     world, rank, _ = dist_setup()
     if rank != 0:
@@ -191,6 +200,7 @@ def run_reference(args):
         tot_f += f
     value = tot_f / tot_t / 1e12
     cores = os.cpu_count()
+    t_eigh = eigh_sample(blocks[0])
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -201,6 +211,8 @@ def run_reference(args):
                          "sample": "one 1024x1024 block of the 64-block batch per step "
                                    "(float64 NumPy/LAPACK oracle, same recurrence and sketch)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "eigh_reference": {"ms_per_block": 1e3 * t_eigh, "cores": cores,
+                           "kind": "float64 LAPACK eigh route to A^(-1/4), one 1024x1024 block"},
     }
     print(json.dumps(line))
     return 0
@@ -810,7 +822,9 @@ def main():
                 break
         cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
                "kind": "oracle",
-               "sample": f"{nb} of the {BATCH} blocks, float64 NumPy/LAPACK oracle (same recurrence)"}
+               "sample": f"{nb} of the {BATCH} blocks, float64 NumPy/LAPACK oracle (same recurrence)",
+               "ms_per_block": 1e3 * t_tot / nb,
+               "eigh_ms_per_block": 1e3 * eigh_sample(A_np[0])}
 
     if rank == 0:
         line = {
