@@ -16,7 +16,7 @@ docstring by page title and section:
 * [PRISM-zh] "PRISM：分布无关的自适应矩阵函数计算" (euno.news), "方法论"
   (item 3: adaptive degree selection).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 * The residual series is the Taylor series of (1 - xi)^(-1/2); the printed
   interval [1/2, 1] for d = 1 fixes its first coefficient at 1/2.
 * A^(-1/4) is two nested coupled square-root passes: pass 1 on B = A/||A||_F
