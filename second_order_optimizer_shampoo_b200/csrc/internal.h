@@ -101,7 +101,7 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
 
 // 3-D fp32 tensor map over [batch][rows][inner] (row stride ld, batch stride
 // bstride, in elements) with a box of box_rows x box_inner, no swizzle and
-// zero fill outside the tensor.  False if the driver rejects it.
+// zero fill outside the tensor.  False if cuTensorMapEncodeTiled rejects it.
 bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
                      int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows);
 
