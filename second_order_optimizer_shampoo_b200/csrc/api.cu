@@ -693,10 +693,10 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
       CK(reset_pass(ctl, B, pass == 0, cs[0], o->adaptive_degree ? 1 : o->d));
       if (pass == 0) {
         CK(frob_norm2(A, 0, nn, B, ctl, cs[0]));
-        CK(coupled_init(A, n, B, ctl, w.Yhi[0], w.Ylo[0], w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo,
+        CK(coupled_init(A, n, B, ctl, w.Yhi[0], w.Ylo[0], w.Rhi, w.Rlo,
                         split ? w.Rs : nullptr, cs[0]));
       } else {
-        CK(coupled_restart(n, B, ctl, w.Yhi, w.Ylo, w.Zhi[0], w.Zlo[0], w.Rhi, w.Rlo,
+        CK(coupled_restart(n, B, ctl, w.Yhi, w.Ylo, w.Rhi, w.Rlo,
                            split ? w.Rs : nullptr, cs[0]));
       }
       const float* S_pass =
@@ -773,11 +773,12 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
     if (power == SHP_POW_SQRT) {
       const float* sh[2] = {w.Yhi[0], w.Yhi[1]};
       const float* sl[2] = {w.Ylo[0], w.Ylo[1]};
-      CK(coupled_finish(n, B, ctl, 0.5, sh, sl, X_out, cs[0]));
+      CK(coupled_finish(n, B, ctl, 0.5, sh, sl, X_out, false, cs[0]));
     } else {
       const float* sh[2] = {w.Zhi[0], w.Zhi[1]};
       const float* sl[2] = {w.Zlo[0], w.Zlo[1]};
-      CK(coupled_finish(n, B, ctl, power == SHP_POW_INV2 ? -0.5 : -0.25, sh, sl, X_out, cs[0]));
+      CK(coupled_finish(n, B, ctl, power == SHP_POW_INV2 ? -0.5 : -0.25, sh, sl, X_out, true,
+                        cs[0]));
     }
     if (rep != nullptr) CK(write_status(ctl, B, rep->status, cs[0]));
     return SHP_OK;

@@ -102,13 +102,14 @@ __global__ void __launch_bounds__(EW_THREADS)
 }
 
 // Start of pass 1 (c = ||A||_F from k_frob): Y_0 = B = (A + A^T) / (2c),
-// Z_0 = I, R_0 = I - B.  The method is stated for a symmetric A and every
+// R_0 = I - B.  Z_0 = I is not stored: the first step writes Z_1 = I + Delta
+// directly and k_coupled_finish stands in I for a block that made no step.  The method is stated for a symmetric A and every
 // later product is formed on its upper-triangle tiles, so the start takes the
 // symmetric part, which is A / c bit for bit when A is symmetric.  A^T comes
 // through a padded 32 x 32 shared-memory transpose: both reads are coalesced.
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_init(const float* A, int64_t n, Ctl ctl, int fmt, float* Yhi, float* Ylo,
-                   float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs) {
+                   float* Rhi, float* Rlo, float* Rs) {
   count_kernel_run();
   __shared__ float tt[32][33];
   const int b = blockIdx.y;
@@ -134,7 +135,6 @@ __global__ void __launch_bounds__(EW_THREADS)
       const float y = 0.5f * (Ab[row * n + col] + tt[r][tx]) / c;
       const float rr = (diag ? 1.f : 0.f) - y;
       put(fmt, Yhi, Ylo, off, y);
-      put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
       put(fmt, Rhi, Rlo, off, rr);
       if (Rs != nullptr) Rs[off] = rr;
       nrm += rr * rr;
@@ -145,8 +145,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_restart(int64_t n, Ctl ctl, int fmt, float* Y0hi, float* Y0lo, const float* Y1hi,
-                      const float* Y1lo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
-                      float* Rs) {
+                      const float* Y1lo, float* Rhi, float* Rlo, float* Rs) {
   count_kernel_run();
   const int b = blockIdx.y;
   const bool from1 = (ctl.bs[b].iters1 & 1) != 0;
@@ -166,7 +165,6 @@ __global__ void __launch_bounds__(EW_THREADS)
       y = get(fmt, Y0hi, Y0lo, off);
     }
     const float r = (diag ? 1.f : 0.f) - y;
-    put(fmt, Zhi, Zlo, off, diag ? 1.f : 0.f);
     put(fmt, Rhi, Rlo, off, r);
     if (Rs != nullptr) Rs[off] = r;
     nrm += r * r;
@@ -195,7 +193,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_coupled_finish(int64_t n, Ctl ctl, double e_c, const float* S0hi, const float* S0lo,
-                     const float* S1hi, const float* S1lo, float* X) {
+                     const float* S1hi, const float* S1lo, float* X, int z_slots) {
   count_kernel_run();
   const int b = blockIdx.y;
   const double c = static_cast<double>(ctl.bs[b].c);
@@ -210,12 +208,19 @@ __global__ void __launch_bounds__(EW_THREADS)
   const bool one = (ctl.bs[b].iters & 1) != 0;
   const float* hi = one ? S1hi : S0hi;
   const float* lo = one ? S1lo : S0lo;
+  // Z_0 = I is never stored: a block whose last pass made no step gets I
+  const bool identity = z_slots != 0 && ctl.bs[b].iters == 0;
   const int64_t nn = n * n;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < nn;
        e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
     const int64_t off = b * nn + e;
-    float v = hi[off];
-    if (lo != nullptr) v += lo[off];
+    float v;
+    if (identity) {
+      v = (e / n) == (e % n) ? 1.f : 0.f;
+    } else {
+      v = hi[off];
+      if (lo != nullptr) v += lo[off];
+    }
     X[off] = scale * v;
   }
 }
@@ -305,20 +310,19 @@ cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, con
 }
 
 cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, float* Yhi,
-                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs,
-                         cudaStream_t st) {
+                         float* Ylo, float* Rhi, float* Rlo, float* Rs, cudaStream_t st) {
   const int fmt = Ylo != nullptr ? OUT_SPLIT : OUT_F32;
-  k_coupled_init<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(A, n, ctl, fmt, Yhi, Ylo, Zhi,
-                                                               Zlo, Rhi, Rlo, Rs);
+  k_coupled_init<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(A, n, ctl, fmt, Yhi, Ylo, Rhi,
+                                                               Rlo, Rs);
   return cudaGetLastError();
 }
 
 cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* Yhi,
-                            float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
-                            float* Rs, cudaStream_t st) {
+                            float* const* Ylo, float* Rhi, float* Rlo, float* Rs,
+                            cudaStream_t st) {
   const int fmt = Ylo[0] != nullptr ? OUT_SPLIT : OUT_F32;
   k_coupled_restart<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(
-      n, ctl, fmt, Yhi[0], Ylo[0], Yhi[1], Ylo[1], Zhi, Zlo, Rhi, Rlo, Rs);
+      n, ctl, fmt, Yhi[0], Ylo[0], Yhi[1], Ylo[1], Rhi, Rlo, Rs);
   return cudaGetLastError();
 }
 
@@ -332,9 +336,9 @@ cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, c
 
 cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_exponent,
                            const float* const* Shi, const float* const* Slo, float* X_out,
-                           cudaStream_t st) {
-  k_coupled_finish<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(n, ctl, c_exponent, Shi[0],
-                                                                 Slo[0], Shi[1], Slo[1], X_out);
+                           bool z_slots, cudaStream_t st) {
+  k_coupled_finish<<<ew_grid(n * n, batch), EW_THREADS, 0, st>>>(
+      n, ctl, c_exponent, Shi[0], Slo[0], Shi[1], Slo[1], X_out, z_slots ? 1 : 0);
   return cudaGetLastError();
 }
 

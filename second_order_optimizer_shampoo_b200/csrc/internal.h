@@ -181,24 +181,26 @@ cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t s
 // dnorm[b] += ||X[b]||_F^2 (X fp32 or bf16, rows x cols contiguous per block).
 cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
                        cudaStream_t st);
-// c = sqrt(dnorm); Y = A / c; Z = I; R = I - Y; norm2 = ||R||_F^2.
+// c = sqrt(dnorm); Y = (A + A^T) / (2c); R = I - Y; norm2 = ||R||_F^2.
+// Z_0 = I is implied (the first step writes Z_1; see coupled_finish).
 // (lo pointers null in TF32 mode; Rs, when non-null, gets a plain fp32 R.)
 cudaError_t coupled_init(const float* A, int64_t n, int batch, const Ctl& ctl, float* Yhi,
-                         float* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo, float* Rs,
-                         cudaStream_t st);
-// Pass 2: Y[0] <- Y[iters1 % 2]; Z = I; R = I - Y; norm2 = ||R||_F^2.
+                         float* Ylo, float* Rhi, float* Rlo, float* Rs, cudaStream_t st);
+// Pass 2: Y[0] <- Y[iters1 % 2]; R = I - Y; norm2 = ||R||_F^2 (Z_0 = I implied).
 cudaError_t coupled_restart(int64_t n, int batch, const Ctl& ctl, float* const* Yhi,
-                            float* const* Ylo, float* Zhi, float* Zlo, float* Rhi, float* Rlo,
-                            float* Rs, cudaStream_t st);
+                            float* const* Ylo, float* Rhi, float* Rlo, float* Rs,
+                            cudaStream_t st);
 // Delta = alpha[b] R (d = 1) in `fmt`; I + Delta into (g2hi, g2lo) when non-null.
 // `active` overrides ctl.active (the degree-1 mask under adaptive degree).
 cudaError_t gform_d1(const float* Rhi, const float* Rlo, int64_t n, int batch, const Ctl& ctl,
                      int fmt, void* ghi, float* glo, void* g2hi, float* g2lo, cudaStream_t st,
                      const int* active = nullptr);
-// X_out[b] = c_b^e * S[iters_b % 2][b] (hi + lo), S = the two ping-pong slots.
+// X_out[b] = c_b^e * S[iters_b % 2][b] (hi + lo), S = the two ping-pong slots;
+// with z_slots (S holds Z, whose Z_0 = I is not stored) a block that made no
+// step in its last pass gets c_b^e * I.
 cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_exponent,
                            const float* const* Shi, const float* const* Slo, float* X_out,
-                           cudaStream_t st);
+                           bool z_slots, cudaStream_t st);
 // hi = tf32(X), lo = X - hi.
 cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st);
 // X0 = G / ||G||_F (uses dnorm) in `fmt`.

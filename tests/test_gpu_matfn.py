@@ -106,6 +106,24 @@ def test_inv_root_ragged_tiles_and_nonsymmetric_input():
         assert relerr(X[b], o.spd_power_eigh(As, -0.25)) <= 1e-5
 
 
+@pytest.mark.parametrize("power", ["inv4", "inv2", "sqrt"])
+def test_inv_root_zero_steps_batched(power):
+    """A tolerance every residual meets at k = 0 (n = 256, the persistent
+    path): no step is taken, so Z stays Z_0 = I, which is never stored and
+    comes from the finish kernel: c^(-1/4) I, c^(-1/2) I, or sqrt(c) B."""
+    n = 256
+    A = synth.spd_batch(n, 2, 1e-2, 1.0, 107)
+    S = synth.sketch_stack(40, n, 8, 1007)
+    X, rep, opts = run_inv_root(A, power, 2, 8, 10.0, 20, "3xtf32", S)
+    code, _ = POW[power]
+    for b in range(2):
+        assert rep["status"][b] == o.OK
+        it = rep["iters"][b] if power == "inv4" else rep["iters"][b][:1]
+        assert list(it) == [0] * len(it)
+        Xo, _ = o.inv_root_ref(A[b], code, oracle_opts(opts), S, force_iters=it)
+        assert relerr(X[b], Xo) <= 1e-6
+
+
 def test_inv_root_tf32_well_conditioned():
     """TF32 path on cond 10 (the Shampoo statistics regime): error <= 1e-3."""
     n, batch = 256, 2
