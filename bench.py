@@ -790,14 +790,18 @@ def main():
     torch.cuda.synchronize()
     gemm_ms = g0.elapsed_time(g1) / reps
     gemm_achieved = 2.0 * N ** 3 * BATCH / (gemm_ms / 1e3) / 1e12
+    step_ms = ms_max / args.steps
     roofline = {
-        "kernel": "k_gemm_tc<3xTF32> (batched 64 x 1024^3)",
+        "kernel": "k_gemm_pp<3xTF32> (persistent CTA pairs, batched 64 x 1024^3)",
         "bound": "tensor", "achieved": gemm_achieved, "peak": split_peak_burst,
         "unit": "TFLOP/s", "frac": gemm_achieved / split_peak_burst,
         "traffic": GEMM_TRAFFIC_PER_LAUNCH, "traffic_unit": "bytes per launch",
         "algorithmic_bytes": 5 * BATCH * N * N * 4,
         "peak_note": f"{peak_src} burst BF16 x 1.1/2.25 (TF32) / 3 (3xTF32 products)",
         "ms_per_launch": gemm_ms,
+        # the step's products at this kernel's rate, as a share of the step time
+        # (to set beside the kernel's share of the ncu launch list of the step)
+        "step_share_est": flops_step / (gemm_achieved * 1e12) / (step_ms / 1e3),
     }
 
     sketch_roof = sketch_leg(A, S[0], stream, peaks, peak_src)
