@@ -203,7 +203,10 @@ int matfn_sign(const void* A, int storage, int64_t n, int64_t batch, const shp_p
  *   J(alpha) = sum_ij r_i(alpha) r_j(alpha) M_ij,  alpha* = argmin_{[lo,hi]} J.
  * R: [batch][n][n] fp32 (n a multiple of 4); S: [n][p] fp32 shared by the batch;
  * alpha_out: [batch] fp32; J_coef_out: [batch][5] fp64 coefficients of
- * alpha^0..alpha^4, or NULL. */
+ * alpha^0..alpha^4, or NULL.  The passes stream R through shared memory by TMA
+ * when V fits there (n * p up to about 16K), else through registers; their
+ * pipeline waits are bounded, and this call (no report) leaves alpha_out
+ * undefined if one runs out, which only a device fault can cause. */
 int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, int p, int d,
                     float lo, float hi, float* alpha_out, double* J_coef_out, void* ws,
                     size_t ws_bytes, shp_stream stream);
