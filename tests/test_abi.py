@@ -25,6 +25,19 @@ def test_header_parses():
     assert set(names) == set(A.EXPORTS), names
 
 
+def test_header_constants_match_the_binding():
+    """Every SHP_* enumerator and #define of the header has the same value in
+    the Python binding (the binding restates them, so drift would go silent)."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    found = dict(re.findall(r"\b(SHP_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    m = re.search(r"#define\s+SHP_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m, "SHP_NOALLOC_SCRATCH_BYTES"
+    found["SHP_NOALLOC_SCRATCH_BYTES"] = str(int(m.group(1)) << int(m.group(2)))
+    assert len(found) >= 20, found
+    for name, value in found.items():
+        assert getattr(A, name) == int(value), name
+
+
 def test_library_exports_every_declared_symbol():
     L = A.lib()
     for name in declared_functions():
