@@ -566,3 +566,37 @@ def test_stop_rules():
     Y, Z, info = o.coupled_ref(np.eye(4), opts, S)
     assert info.status == o.OK and info.iters == 0 and info.res == [0.0]
     np.testing.assert_array_equal(Y, np.eye(4))
+
+
+# The stall rule (stop with ESTALL when the previous residual is below
+# stall_below and the new one is above stall_ratio times it), pinned on a
+# residual sequence worked out by hand.  B = (1 - 0.9) I with Z_0 = I gives
+# R_k = xi_k I, so ||R_k||_F / sqrt(n) = xi_k, and a fixed alpha = 1/4 at d = 1
+# maps xi to 0.5 xi + 0.4375 xi^2 + 0.0625 xi^3:
+#   xi = 0.9, 0.84994, 0.77939, 0.68504, 0.56793, 0.43652
+# (successive ratios 0.944, 0.917, 0.879, 0.829, 0.769).
+STALL_XI0 = 0.9
+
+
+@pytest.mark.parametrize("stall_below,stall_ratio,max_iter,status,iters", [
+    # the first residual below 0.8 is xi_2; xi_3 / xi_2 = 0.879 > 0.75: stop at k = 3
+    # (a rule reading the residual before the previous one would stop at k = 4)
+    (0.8, 0.75, 10, o.ESTALL, 3),
+    # below 0.9 already at xi_1; xi_2 / xi_1 = 0.917 > 0.75: stop at k = 2
+    (0.86, 0.75, 10, o.ESTALL, 2),
+    # no ratio exceeds 0.9 once below 0.8: no stall, max_iter ends the pass
+    # (a reversed comparison would stop at k = 3)
+    (0.8, 0.9, 5, o.ENOCONV, 5),
+    # never below 0.5 within 4 steps: no stall
+    (0.5, 0.75, 4, o.ENOCONV, 4),
+])
+def test_stall_rule_on_scalar_residual(stall_below, stall_ratio, max_iter, status, iters):
+    n = 4
+    opts = o.PrismOpts(d=1, p=2, lo=0.25, hi=1.0, tol=1e-12, max_iter=max_iter,
+                       fixed_alpha=True, stall_below=stall_below, stall_ratio=stall_ratio)
+    B = (1.0 - STALL_XI0) * np.eye(n)
+    _, _, info = o.coupled_ref(B, opts, None)
+    assert info.status == status and info.iters == iters, (info.status, info.iters)
+    want = [0.9, 0.8499375, 0.7793903636596528, 0.6850442777023162, 0.5679272072594314,
+            0.4365241771417045]
+    np.testing.assert_allclose(info.res, want[: iters + 1], rtol=1e-12)
