@@ -62,7 +62,11 @@ typedef enum {
 typedef enum {
   SHP_TF32 = 0,   /* fp32 storage, products on TF32 tensor cores                  */
   SHP_3XTF32 = 1, /* fp32 storage split as hi (TF32) + lo; acc += hh + hl + lh     */
-  SHP_BF16 = 2    /* bf16 storage, fp32 accumulation (polar factor only)           */
+  SHP_BF16 = 2,   /* bf16 storage, fp32 accumulation (polar factor only)           */
+  SHP_OZAKI = 3   /* fp64 storage; every product split into five int8 digit slices
+                     per operand and accumulated exactly on the int8 tensor cores
+                     (about 2^-40 of the row/column maxima per product; inverse
+                     roots only; see shp_matmul_f64)                               */
 } shp_precision;
 
 typedef enum {
@@ -81,7 +85,8 @@ typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_
  *               Taylor coefficient 3/8 and 1 for d = 2
  *   tol         stop when ||R_k||_F / sqrt(n) <= tol (checked before an update)
  *   max_iter    at most this many update steps per pass (<= 256)
- *   prec        SHP_TF32 / SHP_3XTF32 (SHP_BF16 only for polar storage)
+ *   prec        SHP_TF32 / SHP_3XTF32 / SHP_OZAKI (inverse roots); SHP_BF16
+ *               only for polar storage
  *   fixed_alpha 1: alpha = lo every step (plain Taylor Newton-Schulz)
  *   stall_below, stall_ratio: stop with SHP_ESTALL when the previous residual
  *               is below stall_below and the new one exceeds stall_ratio times it
@@ -91,6 +96,12 @@ typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_
  *               ([PRISM] 方法论 3, adaptive degree selection); the interval of
  *               degree e is then [c_e, hi] with c_e its Taylor coefficient
  *               (1/2, 3/8) and lo is not used; needs fixed_alpha = 0
+ *   host_loop   0 (default): the iteration loop runs on the device inside a
+ *               cached CUDA graph (conditional WHILE/IF nodes), with no host
+ *               synchronisation; 1: the same kernels are launched from a host
+ *               loop that synchronises the stream once per iteration to read
+ *               the loop condition (for profilers and launch tracers that do
+ *               not look inside CUDA graphs; slower, never captured)
  */
 typedef struct {
   int d;
@@ -104,6 +115,7 @@ typedef struct {
   float stall_ratio;
   int adaptive_degree;
   float raise_above;
+  int host_loop;
 } shp_prism_opts;
 
 /* Optional per-block trajectory, all device pointers, each may be NULL.
@@ -152,9 +164,12 @@ int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float*
  *   iteration k uses S[k], pass 2 uses S[max_iter + k]; S_count must be
  *   >= max_iter (one pass) or >= 2 * max_iter (SHP_POW_INV4).
  * Output of a block that stopped without converging is its last iterate.
- * Blocks with n <= 64 and p <= 16 run on chip, one CTA per block with fp32
- * products for either precision; they need a 256-byte workspace and allow
- * batch > 65535. */
+ * prec SHP_OZAKI keeps the iterates in fp64 and forms every product from
+ * int8 digit slices (n <= 26000); it is the path for ill-conditioned inputs
+ * (condition 1e6 and above), where fp32 storage cannot reach 1e-5.
+ * Otherwise, blocks with n <= 64 and p <= 16 run on chip, one CTA per block
+ * with fp32 products for either precision; they need a 256-byte workspace
+ * and allow batch > 65535. */
 int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
                    const shp_prism_opts* opts, const float* S, int64_t S_count, float* X_out,
                    const shp_prism_report* report, void* ws, size_t ws_bytes, shp_stream stream);
@@ -205,8 +220,8 @@ int matfn_sign(const void* A, int storage, int64_t n, int64_t batch, const shp_p
  * alpha_out: [batch] fp32; J_coef_out: [batch][5] fp64 coefficients of
  * alpha^0..alpha^4, or NULL.  The passes stream R through shared memory by TMA
  * when V fits there (n * p up to about 16K), else through registers; their
- * pipeline waits are bounded, and this call (no report) leaves alpha_out
- * undefined if one runs out, which only a device fault can cause. */
+ * pipeline waits are bounded, and a block whose wait runs out (which only a
+ * device fault can cause) gets alpha_out = NaN and NaN coefficients. */
 int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, int p, int d,
                     float lo, float hi, float* alpha_out, double* J_coef_out, void* ws,
                     size_t ws_bytes, shp_stream stream);
@@ -247,6 +262,20 @@ int shp_matmul(const void* A, const float* A_lo, int a_trans, const void* B, con
                int b_trans, void* C, int64_t M, int64_t N, int64_t K, int64_t batch, int prec,
                shp_stream stream);
 
+/* C[b] = A[b] * B[b] in fp64-grade arithmetic on the int8 tensor cores (the
+ * Ozaki scheme: Ozaki, Ogita, Oishi, Rump, Numer. Algorithms 2012; the
+ * integer-unit form of Ootomo, Ozaki, Yokota, IJHPCA 2024).  Each row of A
+ * and each column of B is scaled by a power of two and written as five
+ * signed 8-bit digits; the 15 digit products of weight >= 2^-32 are
+ * accumulated exactly in int32 and combined in fp64, so |C - AB|_ij is about
+ * K 2^-40 max_k|A_ik| max_k|B_kj| (or below).  A: [batch][M][K], B:
+ * [batch][K][N], C: [batch][M][N], fp64 row-major, N even, K <= 26000; a NaN
+ * or Inf in a row of A or a column of B makes that row/column of C NaN.
+ * Workspace: shp_matmul_f64_workspace_bytes(M, N, K, batch). */
+size_t shp_matmul_f64_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch);
+int shp_matmul_f64(const double* A, const double* B, double* C, int64_t M, int64_t N, int64_t K,
+                   int64_t batch, void* ws, size_t ws_bytes, shp_stream stream);
+
 /* hi = TF32(x) (round to nearest), lo = TF32(x - hi), for `count` floats. */
 int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream);
 
@@ -264,7 +293,7 @@ uint64_t shp_kernel_launches(void);
  * there, and cudaFree synchronises the whole device), or a latency-bound loop
  * that must not take the implicit synchronisation of cudaMalloc/cudaFree.
  *
- *   Limit: (2d+2) * n * p * batch * 4 bytes <= SHP_NOALLOC_SCRATCH_BYTES
+ *   Limit: ((2d+2) * n * p + 1) * batch * 4 bytes <= SHP_NOALLOC_SCRATCH_BYTES
  *          (e.g. n = 1024, p = 8, d = 2: batch <= 21); larger sizes return
  *          SHP_EUNSUPPORTED before any launch.
  *   Memory: every GPU that loads the library holds SHP_NOALLOC_SCRATCH_BYTES
@@ -273,9 +302,12 @@ uint64_t shp_kernel_launches(void);
  *          (cudaGetSymbolAddress) with that device current; make that first
  *          call before any stream capture.
  *   Sharing: all calls use the same array, which keeps the previous call's
- *          contents (nothing in it needs to start at zero); calls that overlap
- *          on the GPU race on it, so serialise them (one stream, one thread).
- * Arguments, layouts and the other return codes are those of prism_alpha_fit. */
+ *          contents (the sketch vectors need no clearing; the per-block
+ *          timeout flags stored after them are cleared by every call); calls
+ *          that overlap on the GPU race on it, so serialise them (one stream,
+ *          one thread).
+ * Arguments, layouts, the NaN alpha of a timed-out block and the other return
+ * codes are those of prism_alpha_fit. */
 #define SHP_NOALLOC_SCRATCH_BYTES (4u << 20)
 int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const float* S, int p,
                             int d, float lo, float hi, float* alpha_out, double* J_coef_out,

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(HERE, "libshampoo_prism.so")
 SHP_OK, SHP_EINVAL, SHP_EUNSUPPORTED, SHP_ECUDA = 0, 1, 2, 3
 SHP_ENOCONV, SHP_ESTALL, SHP_ENONFINITE, SHP_ETIMEOUT = 16, 17, 18, 19
 # precisions / storage
-SHP_TF32, SHP_3XTF32, SHP_BF16 = 0, 1, 2
+SHP_TF32, SHP_3XTF32, SHP_BF16, SHP_OZAKI = 0, 1, 2, 3
 # powers
 SHP_POW_INV4, SHP_POW_INV2, SHP_POW_SQRT = 0, 1, 2
 # workspace queries
@@ -27,6 +27,7 @@ SHP_NOALLOC_SCRATCH_BYTES = 4 << 20
 EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar", "matfn_polar_varsize",
            "matfn_sign",
            "prism_alpha_fit", "shampoo_apply", "shampoo_apply_ex", "shp_matmul", "shp_split_tf32",
+           "shp_matmul_f64_workspace_bytes", "shp_matmul_f64",
            "shp_kernel_launches", "prism_alpha_fit_noalloc", "shp_status_string", "shp_last_cuda_error",
            "shp_version")
 
@@ -36,7 +37,8 @@ class PrismOpts(ctypes.Structure):
                 ("hi", ctypes.c_float), ("tol", ctypes.c_float), ("max_iter", ctypes.c_int),
                 ("prec", ctypes.c_int), ("fixed_alpha", ctypes.c_int),
                 ("stall_below", ctypes.c_float), ("stall_ratio", ctypes.c_float),
-                ("adaptive_degree", ctypes.c_int), ("raise_above", ctypes.c_float)]
+                ("adaptive_degree", ctypes.c_int), ("raise_above", ctypes.c_float),
+                ("host_loop", ctypes.c_int)]
 
 
 class PrismReport(ctypes.Structure):
@@ -70,6 +72,8 @@ _SIGS = {
                                 _P]),
     "shp_matmul": (_INT, [_P, _P, _INT, _P, _P, _INT, _P, _I64, _I64, _I64, _I64, _INT, _P]),
     "shp_split_tf32": (_INT, [_P, _I64, _P, _P, _P]),
+    "shp_matmul_f64_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64]),
+    "shp_matmul_f64": (_INT, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "shp_kernel_launches": (ctypes.c_uint64, []),
     "prism_alpha_fit_noalloc": (_INT, [_P, _I64, _I64, _P, _INT, _INT, _F, _F, _P, _P, _P]),
     "shp_status_string": (ctypes.c_char_p, [_INT]),

@@ -16,10 +16,16 @@
 // once per device, with that device current, on the first call made on it.
 // That first call should therefore come before any stream capture.
 //
-// All calls share the one array and it keeps the previous call's contents;
-// nothing in it needs to start at zero (each sketch pass writes every element
-// it later reads), but calls that overlap on the GPU (on different streams,
-// or from different host threads) race on it.
+// All calls share the one array and it keeps the previous call's contents.
+// The sketch vectors need no clearing (each pass writes every element it
+// later reads); the per-block timeout flags after them are cleared at the
+// start of every call (cudaMemsetAsync, which allocates nothing).  Calls that
+// overlap on the GPU (on different streams, or from different host threads)
+// race on the array.
+//
+// A bounded pipeline wait of the sketch passes that runs out (which only a
+// device fault can cause) sets its block's flag, and that block's alpha comes
+// out as NaN rather than as a fit on incomplete vectors.
 #include <math.h>
 
 #include <mutex>
@@ -66,20 +72,24 @@ extern "C" int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch,
   if (batch > 65535 || n > INT32_MAX) return SHP_EUNSUPPORTED;
   const int64_t np = n * p;
   const int64_t vbs = static_cast<int64_t>(2 * d + 2) * np;
-  if (vbs * batch > static_cast<int64_t>(kScratchFloats)) return SHP_EUNSUPPORTED;
+  // V for every block, then one timeout flag per block
+  if ((vbs + 1) * batch > static_cast<int64_t>(kScratchFloats)) return SHP_EUNSUPPORTED;
   float* V = nullptr;
   if (scratch_address(&V) != cudaSuccess) return SHP_ECUDA;
+  int* tmo = reinterpret_cast<int*>(V + vbs * batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int B = static_cast<int>(batch);
-  if (shp::sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, nullptr, 0, st) !=
-      cudaSuccess)
+  if (cudaMemsetAsync(tmo, 0, sizeof(int) * static_cast<size_t>(batch), st) != cudaSuccess)
+    return SHP_ECUDA;
+  if (shp::sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, nullptr, 0, st,
+                       tmo) != cudaSuccess)
     return SHP_ECUDA;
   for (int j = 2; j <= 2 * d + 1; ++j)
     if (shp::sketch_pass(R, nullptr, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, p, B,
-                         nullptr, nullptr, 0, st) != cudaSuccess)
+                         nullptr, nullptr, 0, st, tmo) != cudaSuccess)
       return SHP_ECUDA;
   if (shp::alpha_solve(V, n, p, d, B, lo, hi, 0, nullptr, alpha_out, J_coef_out, nullptr, 0, 0,
-                       nullptr, st) != cudaSuccess)
+                       nullptr, st, nullptr, tmo) != cudaSuccess)
     return SHP_ECUDA;
   return SHP_OK;
 }

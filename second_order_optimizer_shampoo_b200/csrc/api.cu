@@ -43,11 +43,14 @@ bool opts_ok(const shp_prism_opts* o) {
   if (!(isfinite(o->lo) && isfinite(o->hi)) || o->lo > o->hi) return false;
   if (!(o->tol >= 0.f)) return false;
   if (o->max_iter < 1 || o->max_iter > 256) return false;
-  if (o->prec != SHP_TF32 && o->prec != SHP_3XTF32 && o->prec != SHP_BF16) return false;
+  if (o->prec != SHP_TF32 && o->prec != SHP_3XTF32 && o->prec != SHP_BF16 &&
+      o->prec != SHP_OZAKI)
+    return false;
   if (!(o->stall_below >= 0.f) || !(o->stall_ratio >= 0.f)) return false;
   if (o->adaptive_degree != 0 &&
       (o->d != 2 || o->fixed_alpha != 0 || !(o->raise_above >= 0.f)))
     return false;
+  if (o->host_loop != 0 && o->host_loop != 1) return false;
   return true;
 }
 
@@ -97,6 +100,49 @@ Bufs carve_inv_root(Arena& a, int64_t n, int64_t batch, const shp_prism_opts* o)
   b.Rs = split ? a.take<float>(nn) : b.Rhi;
   b.ghi = a.take<float>(nn);
   b.glo = split ? a.take<float>(nn) : nullptr;
+  b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * n * o->p * batch);
+  b.ctl = carve_ctl(a, batch);
+  return b;
+}
+
+// fp64 iterates (updated in place: every product reads the digit slices,
+// and the epilogue reads and writes an element of Y or Z only at its own
+// position), their slices, a plain fp32 R for the sketch.
+struct OzBufs {
+  double* Y;
+  double* Z;
+  double* R;
+  double* D;  // Delta = g - I
+  float* Rs;
+  OzSlices sY, sZ, sR, sD;
+  unsigned* maxbuf;
+  float* V;
+  Ctl ctl;
+};
+
+OzSlices carve_slices(Arena& a, int64_t rows, int64_t cols, int64_t batch, bool want_rows,
+                      bool want_cols) {
+  OzSlices s{};
+  s.rows = want_rows ? a.take<int8_t>(oz_slices_bytes(rows, cols, batch)) : nullptr;
+  s.cols = want_cols ? a.take<int8_t>(oz_slices_bytes(cols, rows, batch)) : nullptr;
+  s.rscale = want_rows ? a.take<double>(static_cast<size_t>(rows) * batch) : nullptr;
+  s.cscale = want_cols ? a.take<double>(static_cast<size_t>(cols) * batch) : nullptr;
+  return s;
+}
+
+OzBufs carve_inv_root_oz(Arena& a, int64_t n, int64_t batch, const shp_prism_opts* o) {
+  OzBufs b;
+  const size_t nn = static_cast<size_t>(n) * n * batch;
+  b.Y = a.take<double>(nn);
+  b.Z = a.take<double>(nn);
+  b.R = a.take<double>(nn);
+  b.D = a.take<double>(nn);
+  b.Rs = a.take<float>(nn);
+  b.sY = carve_slices(a, n, n, batch, true, true);
+  b.sZ = carve_slices(a, n, n, batch, true, true);
+  b.sR = carve_slices(a, n, n, batch, true, true);
+  b.sD = carve_slices(a, n, n, batch, true, true);
+  b.maxbuf = a.take<unsigned>(static_cast<size_t>(2 * n) * batch);
   b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * n * o->p * batch);
   b.ctl = carve_ctl(a, batch);
   return b;
@@ -260,8 +306,8 @@ cudaError_t add_conditional(cudaStream_t st, cudaGraphConditionalHandle h,
 
 // iter(cur, first, stream) launches one step on ping-pong slot `cur`.
 // With g == nullptr the same steps run from a host loop that reads the
-// condition back after every step (diagnostic mode, SHP_HOST_LOOP=1, for
-// profilers that cannot look inside conditional graphs).
+// condition back after every step (opts.host_loop = 1, for profilers and
+// launch tracers that do not look inside conditional graphs).
 template <class Iter>
 int record_loop(cudaStream_t const* cs, cudaGraph_t g, const Ctl& ctl, int batch, int max_iter,
                 Iter iter) {
@@ -353,11 +399,11 @@ int run_graph(CallKey key, Rec rec, cudaStream_t user) {
   return SHP_OK;
 }
 
-// Runs `rec` on the user's stream with host-driven loops (SHP_HOST_LOOP set),
+// Runs `rec` on the user's stream with host-driven loops (opts.host_loop),
 // else through the graph cache.
 template <class Rec>
 int dispatch(const CallKey& key, Rec rec, cudaStream_t user) {
-  if (getenv("SHP_HOST_LOOP") != nullptr) {
+  if (key.o.host_loop != 0) {
     cudaStream_t cs[3] = {user, user, user};
     return rec(static_cast<cudaStream_t const*>(cs), static_cast<cudaGraph_t>(nullptr));
   }
@@ -380,7 +426,7 @@ const char* shp_version(void) { return "0.1.0"; }
 uint64_t shp_kernel_launches(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return 0;
   return kernel_runs_gemm() + kernel_runs_sketch() + kernel_runs_elementwise() +
-         kernel_runs_small();
+         kernel_runs_small() + kernel_runs_ozaki();
 }
 
 int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream) {
@@ -439,9 +485,14 @@ size_t shp_workspace_bytes(int opk, int64_t m, int64_t n, int64_t batch,
   switch (opk) {
     case SHP_OP_INV_ROOT:
       if (!opts_ok(o)) return 0;
+      if (o->prec == SHP_OZAKI) {
+        carve_inv_root_oz(a, n, batch, o);
+        break;
+      }
       if (small_block_ok(n, n, o->p)) return kAlign;  // on-chip path: no scratch
       carve_inv_root(a, n, batch, o);
       break;
+
     case SHP_OP_POLAR:
       if (!opts_ok(o) || m <= 0) return 0;
       if (o->prec != SHP_BF16 && small_block_ok(m, n, o->p)) return kAlign;
@@ -450,6 +501,7 @@ size_t shp_workspace_bytes(int opk, int64_t m, int64_t n, int64_t batch,
     case SHP_OP_ALPHA_FIT: {
       const int d = o != nullptr ? o->d : 2, p = o != nullptr ? o->p : 32;
       a.take<float>(static_cast<size_t>(2 * d + 2) * n * p * batch);
+      a.take<int>(static_cast<size_t>(batch));  // timeout flags of the sketch passes
       break;
     }
     case SHP_OP_APPLY: {
@@ -590,9 +642,183 @@ int apply_impl(float* W, float* Mom, double* acc, const float* G, const float* L
   return SHP_OK;
 }
 
+// The inverse-root passes with fp64 iterates and Ozaki-scheme products: the
+// same recurrence and launch order as the split path, each product from the
+// digit slices of its operands, each new iterate sliced after it is formed.
+int inv_root_oz(const float* A, int64_t n, int64_t batch, int power, const shp_prism_opts* o,
+                const float* S, int64_t S_count, float* X_out, const shp_prism_report* rep,
+                void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const int npass = power == SHP_POW_INV4 ? 2 : 1;
+  if (!o->fixed_alpha && (S == nullptr || S_count < static_cast<int64_t>(npass) * o->max_iter))
+    return SHP_EINVAL;
+  if (!aligned16(A) || !aligned16(X_out)) return SHP_EINVAL;
+  if (n > 26000 || batch > 65535) return SHP_EUNSUPPORTED;  // int32 level sums stay exact
+  if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_INV_ROOT, n, n, batch, o))
+    return SHP_EINVAL;
+  CallKey key = make_key(3);
+  key.power = power;
+  key.a = A;
+  key.x = X_out;
+  key.s = S;
+  key.s_count = S_count;
+  key.n = n;
+  key.batch = batch;
+  key.o = *o;
+  key.ws = ws;
+  key.ws_bytes = ws_bytes;
+  if (rep != nullptr) {
+    key.rep[0] = rep->status;
+    key.rep[1] = rep->iters;
+    key.rep[2] = rep->resid;
+    key.rep[3] = rep->alpha;
+    key.rep[4] = rep->degree;
+  }
+  auto record = [&](cudaStream_t const* cs, cudaGraph_t g) -> int {
+    Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) &
+                                    ~(kAlign - 1)));
+    OzBufs w = carve_inv_root_oz(a, n, batch, o);
+    const Ctl& ctl = w.ctl;
+    const int N = static_cast<int>(n), B = static_cast<int>(batch);
+    const int64_t nn = n * n;
+    const int mi = o->max_iter;
+    float* rep_res = rep != nullptr ? rep->resid : nullptr;
+    float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
+    int* rep_iters = rep != nullptr ? rep->iters : nullptr;
+    int* rep_degree = rep != nullptr ? rep->degree : nullptr;
+    auto slice = [&](const double* X, const OzSlices& sl, float* x32, cudaStream_t st) {
+      return oz_slice(X, N, N, n, nn, B, ctl.active, w.maxbuf, sl, x32, st);
+    };
+    // product of the left operand's row slices and the right one's column slices
+    auto epi = [&](int kind, double* out, const OzSlices& l, const OzSlices& r) {
+      OzEpi e;
+      memset(&e, 0, sizeof(e));
+      e.kind = kind;
+      e.out = out;
+      e.ldo = n;
+      e.bso = nn;
+      e.sa = l.rscale;
+      e.sb = r.cscale;
+      e.alpha = ctl.alpha;
+      e.s0 = 1.f;
+      e.norm2 = &ctl.bs[0].norm2;
+      e.norm2_stride = static_cast<int>(sizeof(BlockState) / sizeof(float));
+      e.active = ctl.active;
+      e.status = ctl.tmo;
+      e.M = N;
+      e.N = N;
+      return e;
+    };
+    for (int pass = 0; pass < npass; ++pass) {
+      CK(reset_pass(ctl, B, pass == 0, cs[0], o->adaptive_degree ? 1 : o->d));
+      if (pass == 0) {
+        CK(frob_norm2(A, 0, nn, B, ctl, cs[0]));
+        CK(oz_init(A, n, B, ctl, w.Y, w.R, cs[0]));
+        CK(slice(w.Y, w.sY, nullptr, cs[0]));
+      } else {  // Y is pass 1's result, its slices are current
+        CK(oz_restart(n, B, ctl, w.Y, w.R, cs[0]));
+      }
+      CK(slice(w.R, w.sR, w.Rs, cs[0]));
+      const float* S_pass =
+          S != nullptr ? S + static_cast<int64_t>(pass) * mi * n * o->p : nullptr;
+      auto iter = [&](int, bool first, cudaStream_t st) -> int {
+        if (!first) {  // R_k = I - Z_k Y_k and ||R_k||_F^2
+          OzEpi e = epi(EPI_RESID, w.R, w.sZ, w.sY);
+          CK(gemm_oz(w.sZ.rows, w.sY.cols, N, N, N, B, e, st));
+          CK(slice(w.R, w.sR, w.Rs, st));
+        }
+        CK(control_step(ctl, B, n, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
+                        2 * (mi + 1), pass * (mi + 1), rep_iters, pass, st));
+        int r = sketch_and_alpha(w.Rs, n, B, S_pass, w.V, o, ctl, rep_alpha, 2 * mi, pass * mi,
+                                 st, rep_degree);
+        if (r != SHP_OK) return r;
+        double* z1 = first ? w.Z : nullptr;  // Z_1 = I + Delta (Z_0 = I is not stored)
+        if (o->adaptive_degree) CK(oz_gform_d1(w.R, n, B, ctl, w.D, z1, st, ctl.act1));
+        if (o->d == 2) {  // Delta = R/2 + alpha R^2 in the R R epilogue
+          OzEpi e = epi(EPI_GPOLY, w.D, w.sR, w.sR);
+          if (o->adaptive_degree) e.active = ctl.act2;
+          e.out2 = z1;
+          e.aux = w.R;
+          e.lda = n;
+          e.bsa = nn;
+          e.s1 = 0.5f;
+          CK(gemm_oz(w.sR.rows, w.sR.cols, N, N, N, B, e, st));
+        } else {
+          CK(oz_gform_d1(w.R, n, B, ctl, w.D, z1, st));
+        }
+        CK(slice(w.D, w.sD, nullptr, st));
+        {  // Y_{k+1} = Y_k + Y_k Delta (in place)
+          OzEpi e = epi(EPI_AXPY, w.Y, w.sY, w.sD);
+          e.aux = w.Y;
+          e.lda = n;
+          e.bsa = nn;
+          CK(gemm_oz(w.sY.rows, w.sD.cols, N, N, N, B, e, st));
+        }
+        if (!first) {  // Z_{k+1} = Z_k + Delta Z_k (in place)
+          OzEpi e = epi(EPI_AXPY, w.Z, w.sD, w.sZ);
+          e.aux = w.Z;
+          e.lda = n;
+          e.bsa = nn;
+          CK(gemm_oz(w.sD.rows, w.sZ.cols, N, N, N, B, e, st));
+        }
+        CK(slice(w.Y, w.sY, nullptr, st));
+        CK(slice(w.Z, w.sZ, nullptr, st));
+        return SHP_OK;
+      };
+      int r = record_loop(cs, g, ctl, B, mi, iter);
+      if (r != SHP_OK) return r;
+    }
+    if (power == SHP_POW_SQRT)
+      CK(oz_finish(n, B, ctl, 0.5, w.Y, X_out, false, cs[0]));
+    else
+      CK(oz_finish(n, B, ctl, power == SHP_POW_INV2 ? -0.5 : -0.25, w.Z, X_out, true, cs[0]));
+    if (rep != nullptr) CK(write_status(ctl, B, rep->status, cs[0]));
+    return SHP_OK;
+  };
+  return dispatch(key, record, stream);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t shp_matmul_f64_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch) {
+  if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
+  Arena a(nullptr);
+  carve_slices(a, M, K, batch, true, false);
+  carve_slices(a, K, N, batch, false, true);
+  a.take<unsigned>(static_cast<size_t>(M + 2 * K + N) * batch);
+  return a.used + kAlign;
+}
+
+int shp_matmul_f64(const double* A, const double* B, double* C, int64_t M, int64_t N, int64_t K,
+                   int64_t batch, void* ws, size_t ws_bytes, shp_stream stream) {
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || batch <= 0 || N % 2) return SHP_EINVAL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return SHP_EINVAL;
+  if (M > INT32_MAX || N > INT32_MAX || K > 26000 || batch > 65535) return SHP_EUNSUPPORTED;
+  if (ws == nullptr || ws_bytes < shp_matmul_f64_workspace_bytes(M, N, K, batch)) return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  const OzSlices sa = carve_slices(a, M, K, batch, true, false);
+  const OzSlices sb = carve_slices(a, K, N, batch, false, true);
+  unsigned* maxbuf = a.take<unsigned>(static_cast<size_t>(M + 2 * K + N) * batch);
+  const int m = static_cast<int>(M), nc = static_cast<int>(N), k = static_cast<int>(K);
+  const int bt = static_cast<int>(batch);
+  CK(oz_slice(A, m, k, K, M * K, bt, nullptr, maxbuf, sa, nullptr, st));
+  CK(oz_slice(B, k, nc, N, K * N, bt, nullptr, maxbuf + (M + K) * batch, sb, nullptr, st));
+  OzEpi e;
+  memset(&e, 0, sizeof(e));
+  e.kind = EPI_STORE;
+  e.out = C;
+  e.ldo = N;
+  e.bso = M * N;
+  e.sa = sa.rscale;
+  e.sb = sb.cscale;
+  e.s0 = 1.f;
+  e.M = m;
+  e.N = nc;
+  CK(gemm_oz(sa.rows, sb.cols, m, nc, k, bt, e, st));
+  return SHP_OK;
+}
 
 int shampoo_apply(float* W, const float* G, const float* Lroot, const float* Rroot, int64_t m,
                   int64_t n, int64_t batch, float lr, int prec, void* ws, size_t ws_bytes,
@@ -624,14 +850,16 @@ int prism_alpha_fit(const float* R, int64_t n, int64_t batch, const float* S, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
   float* V = a.take<float>(static_cast<size_t>(2 * d + 2) * n * p * batch);
+  int* tmo = a.take<int>(static_cast<size_t>(batch));
   const int64_t np = n * p, vbs = static_cast<int64_t>(2 * d + 2) * np;
   const int B = static_cast<int>(batch);
-  CK(sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, nullptr, 0, st));
+  CK(cudaMemsetAsync(tmo, 0, sizeof(int) * static_cast<size_t>(batch), st));
+  CK(sketch_pass(R, nullptr, n, n * n, S, 0, V + np, vbs, p, B, nullptr, nullptr, 0, st, tmo));
   for (int j = 2; j <= 2 * d + 1; ++j)
     CK(sketch_pass(R, nullptr, n, n * n, V + (j - 1) * np, vbs, V + j * np, vbs, p, B, nullptr,
-                   nullptr, 0, st));
+                   nullptr, 0, st, tmo));
   CK(alpha_solve(V, n, p, d, B, lo, hi, 0, nullptr, alpha_out, J_coef_out, nullptr, 0, 0,
-                 nullptr, st));
+                 nullptr, st, nullptr, tmo));
   return SHP_OK;
 }
 
@@ -640,6 +868,9 @@ int matfn_inv_root(const float* A, int64_t n, int64_t batch, int power,
                    const shp_prism_report* rep, void* ws, size_t ws_bytes, shp_stream stream) {
   if (!A || !X_out || !opts_ok(o) || n <= 0 || batch <= 0 || n % 4) return SHP_EINVAL;
   if (power != SHP_POW_INV4 && power != SHP_POW_INV2 && power != SHP_POW_SQRT) return SHP_EINVAL;
+  if (o->prec == SHP_OZAKI)
+    return inv_root_oz(A, n, batch, power, o, S, S_count, X_out, rep, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
   if (o->prec != SHP_TF32 && o->prec != SHP_3XTF32) return SHP_EINVAL;
   const int npass = power == SHP_POW_INV4 ? 2 : 1;
   if (!o->fixed_alpha && (S == nullptr || S_count < static_cast<int64_t>(npass) * o->max_iter))

@@ -843,13 +843,28 @@ cudaError_t dispatch_pair(bool pair, bool amn, bool bmn, const CUtensorMap& a,
                           const CUtensorMap& al, const CUtensorMap& b, const CUtensorMap& bl,
                           int M, int N, int K, int BN, int batch, const EpiParams& ep,
                           cudaStream_t st) {
-  if (pair && getenv("SHP_NO_PERSIST") == nullptr)
-    return dispatch_pp<MODE>(amn, bmn, a, al, b, bl, M, N, K, batch, ep, st);
-  return pair ? dispatch<MODE, true>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st)
-              : dispatch<MODE, false>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st);
+  if (pair) return dispatch_pp<MODE>(amn, bmn, a, al, b, bl, M, N, K, batch, ep, st);
+  return dispatch<MODE, false>(amn, bmn, a, al, b, bl, M, N, K, BN, batch, ep, st);
 }
 
 }  // namespace
+
+bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t K, int64_t rows, int slices,
+                       int64_t batch, int64_t ldk, int box_k, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(slices), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(ldk), static_cast<cuuint64_t>(rows * ldk),
+                           static_cast<cuuint64_t>(slices * rows * ldk)};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_k), static_cast<cuuint32_t>(box_rows),
+                       static_cast<cuuint32_t>(slices), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<int8_t*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
                      int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows) {
@@ -867,7 +882,7 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
   const int BN = N > 128 ? 256 : (N > 64 ? 128 : 64);
   // CTA pairs (M = 256 per MMA) for full-width tiles; small problems keep one
   // CTA per 128-row tile.
-  const bool pair = M >= 256 && BN == 256 && getenv("SHP_NO_PAIR") == nullptr;
+  const bool pair = M >= 256 && BN == 256;
   const int bn_cta = pair ? BN / 2 : BN;
   CUtensorMap ma, mal, mb, mbl;
   bool ok = true;

@@ -105,6 +105,13 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
 bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
                      int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows);
 
+// 4-D int8 map over [batch][slices][rows][K] (row stride ldk bytes, a
+// multiple of 16) with a box of all slices x box_rows x box_k bytes and the
+// 64-byte swizzle, zero fill outside the tensor: the digit slices of the
+// Ozaki-scheme products (ozaki.cu).
+bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t K, int64_t rows, int slices,
+                       int64_t batch, int64_t ldk, int box_k, int box_rows);
+
 // ---- PRISM sketch and alpha (sketch_alpha.cu)
 // Vout[b] = R[b] * Vin[b]; R is n x n (hi + lo when lo != null); V is n x p.
 // vin_bstride == 0 shares Vin across the batch.  When `it` is non-null the
@@ -132,10 +139,13 @@ struct AdaptiveDeg {
 };
 // With ad enabled (d = 2): V holds V_1..V_5 and each block fits at its
 // current degree, raising it by the rule of shp_prism_opts.adaptive_degree.
+// tmo (may be null): a block whose flag is set (a sketch wait ran out, so V
+// is incomplete) gets alpha = NaN and NaN coefficients instead of a fit.
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
-                        const int* it, cudaStream_t st, const AdaptiveDeg* ad = nullptr);
+                        const int* it, cudaStream_t st, const AdaptiveDeg* ad = nullptr,
+                        const int* tmo = nullptr);
 
 // ---- per-block control (sketch_alpha.cu)
 struct BlockState {
@@ -238,5 +248,64 @@ cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism
                         const float* S, float* X, int* rep_status, int* rep_iters,
                         float* rep_resid, float* rep_alpha, int* rep_degree, bool sign,
                         cudaStream_t st);
+
+// ---- fp64-grade products on the int8 tensor cores (ozaki.cu)
+// Digit slices of an fp64 matrix X (rows x cols): the row slicing serves X
+// as the left operand A, the column slicing (stored transposed, i.e. as the
+// row slicing of X^T) as the right operand B.  Row r of a slice buffer is
+// oz_ldk(K) bytes long (K = cols for `rows`, rows for `cols`).
+struct OzSlices {
+  int8_t* rows;    // [batch][S][rows][oz_ldk(cols)], weights rscale
+  int8_t* cols;    // [batch][S][cols][oz_ldk(rows)], weights cscale
+  double* rscale;  // [batch][rows]
+  double* cscale;  // [batch][cols]
+};
+// Epilogue of one Ozaki product C = A B (acc = the fp64 value of C):
+//   STORE v = s0 acc; RESID v = [i==j] - acc, norm2 += v^2;
+//   GPOLY v = s1 aux + alpha[b] acc (out2 = I + v); AXPY v = aux + s0 acc.
+// out, out2 and aux are fp64 [batch][M][N] (ld / batch strides in elements);
+// sa [batch][M] and sb [batch][N] are the slice weights of A and B.
+struct OzEpi {
+  int kind;
+  double* out;
+  double* out2;
+  int64_t ldo, bso;
+  const double* aux;
+  int64_t lda, bsa;
+  const double* sa;
+  const double* sb;
+  const float* alpha;
+  float s0, s1;
+  float* norm2;
+  int norm2_stride;
+  const int* active;
+  int* status;
+  int M, N;
+};
+int64_t oz_ldk(int64_t k);                                     // slice row length (bytes)
+size_t oz_slices_bytes(int64_t rows, int64_t k, int64_t batch);  // one slicing's digits
+int oz_slice_count();
+// Slices of X ([batch][rows][cols] at ld / bs); out.rows / out.cols may be
+// null to skip that slicing; maxbuf is (rows + cols) * batch unsigned of
+// scratch; x32 (may be null) gets a plain fp32 copy of X.  Blocks with
+// active[b] == 0 are skipped.
+cudaError_t oz_slice(const double* X, int rows, int cols, int64_t ld, int64_t bs, int batch,
+                     const int* active, unsigned* maxbuf, const OzSlices& out, float* x32,
+                     cudaStream_t st);
+// C = A B from A's row slices ([batch][S][M][oz_ldk(K)]) and B's column
+// slices ([batch][S][N][oz_ldk(K)]), then the epilogue.
+cudaError_t gemm_oz(const int8_t* Arows, const int8_t* Bcols, int M, int N, int K, int batch,
+                    const OzEpi& ep, cudaStream_t st);
+// fp64 storage kernels of the inverse-root passes (see the fp32 versions).
+cudaError_t oz_init(const float* A, int64_t n, int batch, const Ctl& ctl, double* Y, double* R,
+                    cudaStream_t st);
+cudaError_t oz_restart(int64_t n, int batch, const Ctl& ctl, const double* Y, double* R,
+                       cudaStream_t st);
+cudaError_t oz_gform_d1(const double* R, int64_t n, int batch, const Ctl& ctl, double* D,
+                        double* D2, cudaStream_t st, const int* active = nullptr);
+cudaError_t oz_finish(int64_t n, int batch, const Ctl& ctl, double c_exponent, const double* S,
+                      float* X_out, bool z_slots, cudaStream_t st);
+uint64_t kernel_runs_ozaki();
+
 
 }  // namespace shp

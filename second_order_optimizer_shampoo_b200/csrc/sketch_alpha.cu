@@ -396,6 +396,7 @@ struct AlphaArgs {
   int* act1;
   int* act2;
   int* rep_deg;
+  const int* tmo;  // blocks whose sketch timed out: alpha = NaN
 };
 
 // This thread's partial sums of <V_i, V_j> (i <= j < NV, packed row by row)
@@ -446,6 +447,14 @@ __global__ void __launch_bounds__(AL_THREADS) k_alpha(AlphaArgs g) {
     return;
   }
   const int rep_slot = g.rep_slot + (g.it != nullptr ? *g.it : 0);
+  if (g.tmo != nullptr && g.tmo[b] != 0) {  // V is incomplete: no fit
+    if (threadIdx.x == 0) {
+      g.alpha[b] = __int_as_float(0x7fc00000);
+      if (g.Jc != nullptr)
+        for (int i = 0; i < 5; ++i) g.Jc[b * 5 + i] = __longlong_as_double(0x7ff8000000000000ll);
+    }
+    return;
+  }
   if (g.fixed) {  // plain Taylor step: alpha = lo, no sketch needed
     if (threadIdx.x == 0) {
       g.alpha[b] = g.lo;
@@ -588,7 +597,7 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
   if (batch <= 0 || n <= 0) return cudaSuccess;
   // plain fp32 R with 16-byte aligned rows: the bulk-copy kernel when V fits
   if (Rlo == nullptr && (reinterpret_cast<uintptr_t>(Rhi) & 15) == 0 && n % 4 == 0 &&
-      r_bstride % 4 == 0 && getenv("SHP_SKETCH_REGS") == nullptr) {
+      r_bstride % 4 == 0) {
     cudaError_t e = cudaSuccess;
     bool done = false;
     if (p <= 4)
@@ -622,9 +631,11 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
-                        const int* it, cudaStream_t st, const AdaptiveDeg* ad) {
+                        const int* it, cudaStream_t st, const AdaptiveDeg* ad,
+                        const int* tmo) {
   if (batch <= 0) return cudaSuccess;
   AlphaArgs g;
+  g.tmo = tmo;
   g.V = V;
   g.n = n;
   g.vbs = static_cast<int64_t>(2 * d + 2) * n * p;

@@ -13,7 +13,7 @@ import torch
 
 from . import _abi as A
 
-_PREC = {"tf32": A.SHP_TF32, "3xtf32": A.SHP_3XTF32, "bf16": A.SHP_BF16}
+_PREC = {"tf32": A.SHP_TF32, "3xtf32": A.SHP_3XTF32, "bf16": A.SHP_BF16, "ozaki": A.SHP_OZAKI}
 _POW = {"inv4": A.SHP_POW_INV4, "inv2": A.SHP_POW_INV2, "sqrt": A.SHP_POW_SQRT}
 
 
@@ -53,12 +53,12 @@ def _stream():
 
 def make_opts(d=2, p=8, lo=None, hi=1.0, tol=1e-3, max_iter=40, prec="3xtf32",
               fixed_alpha=False, stall_below=0.05, stall_ratio=0.75, adaptive_degree=False,
-              raise_above=0.9) -> A.PrismOpts:
+              raise_above=0.9, host_loop=False) -> A.PrismOpts:
     if lo is None:
         lo = 0.5 if d == 1 else 0.375
     return A.PrismOpts(d, p, lo, hi, tol, max_iter, _PREC[prec] if isinstance(prec, str) else prec,
                        int(bool(fixed_alpha)), stall_below, stall_ratio,
-                       int(bool(adaptive_degree)), raise_above)
+                       int(bool(adaptive_degree)), raise_above, int(bool(host_loop)))
 
 
 def shp_workspace_bytes(op: int, m: int, n: int, batch: int, opts: A.PrismOpts | None = None) -> int:
@@ -282,4 +282,21 @@ def shp_matmul(Amat, B, prec="tf32", a_trans=False, b_trans=False, A_lo=None, B_
     out = torch.empty(batch, M, N, dtype=dt, device=Amat.device) if out is None else out
     _check(A.lib().shp_matmul(_p(Amat), _p(A_lo), int(a_trans), _p(B), _p(B_lo), int(b_trans),
                               _p(out), M, N, K, batch, _PREC[prec], _stream()), "shp_matmul")
+    return out
+
+
+def shp_matmul_f64(Amat, B, out=None, ws=None):
+    """Batched C = A B in fp64-grade arithmetic on the int8 tensor cores (the
+    Ozaki scheme); A [batch][M][K], B [batch][K][N] float64."""
+    _dev(Amat, B, out)
+    if Amat.dtype != torch.float64 or B.dtype != torch.float64:
+        raise ValueError("shp_matmul_f64 takes float64 tensors")
+    M, K = Amat.shape[-2], Amat.shape[-1]
+    N = B.shape[-1]
+    batch = Amat.numel() // (M * K)
+    out = torch.empty(batch, M, N, dtype=torch.float64, device=Amat.device) if out is None else out
+    need = int(A.lib().shp_matmul_f64_workspace_bytes(M, N, K, batch))
+    ws = _ws(need, Amat.device) if ws is None else ws
+    _check(A.lib().shp_matmul_f64(_p(Amat), _p(B), _p(out), M, N, K, batch, _p(ws), ws.numel(),
+                                  _stream()), "shp_matmul_f64")
     return out

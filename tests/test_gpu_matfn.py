@@ -391,3 +391,54 @@ def test_sigma_min_sweep_prism_fewer_gemms():
         bound = 2e-5 if smin >= 1e-2 else 2e-4
         for b in range(2):
             assert relerr(Xp[b], o.polar_svd(G[b])) <= bound
+
+
+@pytest.mark.parametrize("n", [64, 100])
+@pytest.mark.parametrize("stall_below,stall_ratio,max_iter", [
+    (0.8, 0.75, 10), (0.86, 0.75, 10), (0.8, 0.9, 5)])
+def test_stall_decision_matches_oracle(n, stall_below, stall_ratio, max_iter):
+    """The stop rule on residual sequences with wide margins: A = I gives
+    B = A / ||A||_F = I / sqrt(n) and, with a fixed alpha = 1/4 (d = 1),
+    ||R_k||_F / sqrt(n) = xi_k with xi_0 = 1 - 1/sqrt(n) and
+    xi_{k+1} = 0.5 xi + 0.4375 xi^2 + 0.0625 xi^3: for n = 100 the sequence
+    0.9, 0.850, 0.779, 0.685, ... of the oracle's stall pin, for n = 64
+    0.875, 0.814, 0.731, 0.624, ... (every ratio and residual at least 0.014
+    from the thresholds).  The GPU stops at the same step with the same status
+    as the oracle (ESTALL, or ENOCONV at max_iter), on the on-chip path
+    (n = 64) and the batched tensor-core path (n = 100)."""
+    P = prism()
+    A = np.eye(n, dtype=np.float32)[None]
+    opts = P.make_opts(d=1, p=4, lo=0.25, hi=1.0, tol=1e-9, max_iter=max_iter, prec="3xtf32",
+                       fixed_alpha=True, stall_below=stall_below, stall_ratio=stall_ratio)
+    _, rep = P.matfn_inv_root(to_dev(torch, A), "inv2", opts, None)
+    rep = {k: to_host(v) for k, v in rep.items()}
+    _, infos = o.inv_root_ref(A[0], o.POW_INV2, oracle_opts(opts), None)
+    assert infos[0].status in (o.ESTALL, o.ENOCONV)
+    assert int(rep["status"][0]) == infos[0].status
+    assert int(rep["iters"][0, 0]) == infos[0].iters
+    np.testing.assert_allclose(rep["resid"][0, 0, :infos[0].iters + 1], infos[0].res, rtol=1e-5)
+
+
+@pytest.mark.parametrize("prec", ["3xtf32", "ozaki"])
+def test_inv_root_pass2_zero_steps_beside_ordinary_block(prec):
+    """Block 0 is A = I (n = 128): B = I / sqrt(n), so pass 1 starts at
+    residual 1 - n^(-1/2) = 0.91 and iterates, while pass 2 starts from
+    Y_1 = n^(-1/4) I at residual 1 - n^(-1/4) = 0.70 and, with tol 0.8, stops
+    at its first check.  Z_0 = I of pass 2 is never stored, so the finish
+    kernel must stand in I for that block alone: X = c^(-1/4) I with
+    c = ||A||_F = sqrt(n) (the method's output at this tolerance, as the
+    oracle gives it), while block 1 beside it iterates in both passes."""
+    P = prism()
+    n = 128
+    A = synth.spd_batch(n, 2, 1e-2, 1.0, 114)
+    A[0] = np.eye(n, dtype=np.float32)
+    S = synth.sketch_stack(60, n, 8, 1014)
+    X, rep, opts = run_inv_root(A, "inv4", 2, 8, 0.8, 30, prec, S)
+    assert rep["iters"][0][0] >= 1 and rep["iters"][0][1] == 0, rep["iters"]
+    assert rep["status"][0] == o.OK
+    np.testing.assert_allclose(X[0], n ** -0.125 * np.eye(n), rtol=1e-6, atol=1e-7)
+    Xo, _ = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S, force_iters=rep["iters"][0])
+    assert relerr(X[0], Xo) <= 1e-6
+    assert rep["status"][1] == o.OK and rep["iters"][1][1] >= 1
+    Xo, _ = o.inv_root_ref(A[1], o.POW_INV4, oracle_opts(opts), S, force_iters=rep["iters"][1])
+    assert relerr(X[1], Xo) <= 1e-5

@@ -58,13 +58,20 @@ def test_noalloc_matches_workspace_entry_point(d, p, n, batch):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
+    """The scratch holds (2d+2) n p floats of sketch vectors and one timeout
+    flag per block: the largest batch that fits runs, one more is refused
+    before any launch."""
     n, p, d = 1024, 8, 2
-    per_block = (2 * d + 2) * n * p * 4
-    batch = A.SHP_NOALLOC_SCRATCH_BYTES // per_block + 1
-    Rd = torch.zeros(1, n, n, device="cuda")
+    per_block = ((2 * d + 2) * n * p + 1) * 4
+    fits = A.SHP_NOALLOC_SCRATCH_BYTES // per_block
+    Rd = torch.zeros(fits + 1, n, n, device="cuda")
     Sd = torch.zeros(n, p, device="cuda")
-    out = torch.zeros(batch, device="cuda")
-    rc = A.lib().prism_alpha_fit_noalloc(ctypes.c_void_p(Rd.data_ptr()), n, batch,
-                                         ctypes.c_void_p(Sd.data_ptr()), p, d, 0.375, 1.0,
-                                         ctypes.c_void_p(out.data_ptr()), None, None)
-    assert rc == A.SHP_EUNSUPPORTED
+    out = torch.zeros(fits + 1, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for batch, want in ((fits + 1, A.SHP_EUNSUPPORTED), (fits, A.SHP_OK)):
+        rc = A.lib().prism_alpha_fit_noalloc(ctypes.c_void_p(Rd.data_ptr()), n, batch,
+                                             ctypes.c_void_p(Sd.data_ptr()), p, d, 0.375, 1.0,
+                                             ctypes.c_void_p(out.data_ptr()), None, stream)
+        assert rc == want, (batch, rc)
+    # R = 0 makes J constant: every block takes the lower end of the interval
+    np.testing.assert_array_equal(out[:fits].cpu().numpy(), np.float32(0.375))
