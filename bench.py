@@ -218,6 +218,47 @@ def run_reference(args):
     return 0
 
 
+def step_only(args):
+    """One config-3 step alone (profiling aid): --batch blocks of 1024^2 at
+    cond 1e6, every kernel launched from the host loop so that profilers see
+    each launch; --prec selects the product path."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism, synth
+    dev = torch.device("cuda", 0)
+    A = torch.from_numpy(synth.spd_batch(N, args.batch, LAM_LO, 1.0, SEED_A)).to(dev)
+    S = torch.from_numpy(synth.sketch_stack(2 * MAX_ITER, N, P, SEED_S)).to(dev)
+    opts = prism.make_opts(d=D, p=P, tol=TOL, max_iter=MAX_ITER, prec=args.prec, host_loop=True)
+    X = torch.empty_like(A)
+    rep = prism.make_report(args.batch, MAX_ITER, dev)
+    for _ in range(max(args.warmup, 1) + args.steps):
+        prism.matfn_inv_root(A, "inv4", opts, S, out=X, report=rep)
+    torch.cuda.synchronize()
+    ok = int((rep["status"].cpu().numpy() == 0).sum())
+    print(json.dumps({"kernel": "step", "prec": args.prec, "batch": args.batch, "status_ok": ok,
+                      "iters": rep["iters"].cpu().numpy()[0].tolist()}))
+    return 0
+
+
+def ozgemm_only(args):
+    """The Ozaki-scheme GEMM alone (profiling aid): --batch products of
+    1024^2 fp64 matrices through shp_matmul_f64 (slicing, then one k_gemm_oz)."""
+    import torch
+
+    from second_order_optimizer_shampoo_b200 import prism
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(5)
+    X = torch.randn(args.batch, N, N, device=dev, generator=g, dtype=torch.float64)
+    Y = torch.randn(args.batch, N, N, device=dev, generator=g, dtype=torch.float64)
+    out = torch.empty_like(X)
+    for _ in range(max(args.warmup, 1) + args.steps):
+        prism.shp_matmul_f64(X, Y, out=out)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": "ozgemm", "batch": args.batch,
+                      "launches": args.steps + max(args.warmup, 1)}))
+    return 0
+
+
 def gemm_only(args):
     """The dominant kernel alone: batched 1024^3 3xTF32 products (profiling aid)."""
     import torch
@@ -626,7 +667,9 @@ def main():
                          "on the host first)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the Shampoo-step, GEMM-count and single-block legs")
-    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar", "sketch"],
+    ap.add_argument("--prec", default="ozaki", choices=["ozaki", "3xtf32", "tf32"],
+                    help="product path of --kernel step")
+    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar", "sketch", "step", "ozgemm"],
                     help="run only the batched 3xTF32 GEMM, the small-block kernel, the "
                          "polar leg or the sketch leg (for profiling; --batch sets the "
                          "GEMM/small/sketch batch)")
@@ -636,6 +679,10 @@ def main():
         return run_reference(args)
     if args.kernel == "gemm":
         return gemm_only(args)
+    if args.kernel == "step":
+        return step_only(args)
+    if args.kernel == "ozgemm":
+        return ozgemm_only(args)
     if args.kernel == "small":
         return small_only(args)
     if args.kernel == "sketch":

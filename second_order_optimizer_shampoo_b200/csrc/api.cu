@@ -115,7 +115,8 @@ struct OzBufs {
   double* D;  // Delta = g - I
   float* Rs;
   OzSlices sY, sZ, sR, sD;
-  unsigned* maxbuf;
+  unsigned* maxbuf;   // row and column maxima keys of the matrix being sliced
+  unsigned* maxbuf2;  // ... of Z_1 = I + Delta, written beside Delta
   float* V;
   Ctl ctl;
 };
@@ -143,6 +144,7 @@ OzBufs carve_inv_root_oz(Arena& a, int64_t n, int64_t batch, const shp_prism_opt
   b.sR = carve_slices(a, n, n, batch, true, true);
   b.sD = carve_slices(a, n, n, batch, true, true);
   b.maxbuf = a.take<unsigned>(static_cast<size_t>(2 * n) * batch);
+  b.maxbuf2 = a.take<unsigned>(static_cast<size_t>(2 * n) * batch);
   b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * n * o->p * batch);
   b.ctl = carve_ctl(a, batch);
   return b;
@@ -685,10 +687,13 @@ int inv_root_oz(const float* A, int64_t n, int64_t batch, int power, const shp_p
     float* rep_alpha = rep != nullptr ? rep->alpha : nullptr;
     int* rep_iters = rep != nullptr ? rep->iters : nullptr;
     int* rep_degree = rep != nullptr ? rep->degree : nullptr;
-    auto slice = [&](const double* X, const OzSlices& sl, float* x32, cudaStream_t st) {
-      return oz_slice(X, N, N, n, nn, B, ctl.active, w.maxbuf, sl, x32, st);
+    // have_max: the maxima in `mb` were folded in by the epilogue that wrote X
+    auto slice = [&](const double* X, const OzSlices& sl, float* x32, unsigned* mb,
+                     bool have_max, cudaStream_t st) {
+      return oz_slice(X, N, N, n, nn, B, ctl.active, mb, have_max, sl, x32, st);
     };
-    // product of the left operand's row slices and the right one's column slices
+    // product of the left operand's row slices and the right one's column
+    // slices; the epilogue folds the maxima of `out` into w.maxbuf
     auto epi = [&](int kind, double* out, const OzSlices& l, const OzSlices& r) {
       OzEpi e;
       memset(&e, 0, sizeof(e));
@@ -706,6 +711,8 @@ int inv_root_oz(const float* A, int64_t n, int64_t batch, int power, const shp_p
       e.status = ctl.tmo;
       e.M = N;
       e.N = N;
+      e.rmax = w.maxbuf;
+      e.cmax = w.maxbuf + static_cast<int64_t>(B) * N;
       return e;
     };
     for (int pass = 0; pass < npass; ++pass) {
@@ -713,18 +720,19 @@ int inv_root_oz(const float* A, int64_t n, int64_t batch, int power, const shp_p
       if (pass == 0) {
         CK(frob_norm2(A, 0, nn, B, ctl, cs[0]));
         CK(oz_init(A, n, B, ctl, w.Y, w.R, cs[0]));
-        CK(slice(w.Y, w.sY, nullptr, cs[0]));
+        CK(slice(w.Y, w.sY, nullptr, w.maxbuf, false, cs[0]));
       } else {  // Y is pass 1's result, its slices are current
         CK(oz_restart(n, B, ctl, w.Y, w.R, cs[0]));
       }
-      CK(slice(w.R, w.sR, w.Rs, cs[0]));
+      CK(slice(w.R, w.sR, w.Rs, w.maxbuf, false, cs[0]));
       const float* S_pass =
           S != nullptr ? S + static_cast<int64_t>(pass) * mi * n * o->p : nullptr;
       auto iter = [&](int, bool first, cudaStream_t st) -> int {
         if (!first) {  // R_k = I - Z_k Y_k and ||R_k||_F^2
           OzEpi e = epi(EPI_RESID, w.R, w.sZ, w.sY);
+          CK(oz_clear_max(w.maxbuf, N, N, B, st));
           CK(gemm_oz(w.sZ.rows, w.sY.cols, N, N, N, B, e, st));
-          CK(slice(w.R, w.sR, w.Rs, st));
+          CK(slice(w.R, w.sR, w.Rs, w.maxbuf, true, st));
         }
         CK(control_step(ctl, B, n, mi, o->tol, o->stall_below, o->stall_ratio, rep_res,
                         2 * (mi + 1), pass * (mi + 1), rep_iters, pass, st));
@@ -732,36 +740,48 @@ int inv_root_oz(const float* A, int64_t n, int64_t batch, int power, const shp_p
                                  st, rep_degree);
         if (r != SHP_OK) return r;
         double* z1 = first ? w.Z : nullptr;  // Z_1 = I + Delta (Z_0 = I is not stored)
+        // Delta comes from the GEMM epilogue (which folds in its maxima) unless
+        // some or all blocks form it elementwise (d = 1, adaptive degree)
+        const bool d_max = o->d == 2 && !o->adaptive_degree;
         if (o->adaptive_degree) CK(oz_gform_d1(w.R, n, B, ctl, w.D, z1, st, ctl.act1));
         if (o->d == 2) {  // Delta = R/2 + alpha R^2 in the R R epilogue
           OzEpi e = epi(EPI_GPOLY, w.D, w.sR, w.sR);
           if (o->adaptive_degree) e.active = ctl.act2;
           e.out2 = z1;
+          if (z1 != nullptr) {
+            e.rmax2 = w.maxbuf2;
+            e.cmax2 = w.maxbuf2 + static_cast<int64_t>(B) * N;
+            CK(oz_clear_max(w.maxbuf2, N, N, B, st));
+          }
           e.aux = w.R;
           e.lda = n;
           e.bsa = nn;
           e.s1 = 0.5f;
+          CK(oz_clear_max(w.maxbuf, N, N, B, st));
           CK(gemm_oz(w.sR.rows, w.sR.cols, N, N, N, B, e, st));
         } else {
           CK(oz_gform_d1(w.R, n, B, ctl, w.D, z1, st));
         }
-        CK(slice(w.D, w.sD, nullptr, st));
+        CK(slice(w.D, w.sD, nullptr, w.maxbuf, d_max, st));
+        if (first) CK(slice(w.Z, w.sZ, nullptr, w.maxbuf2, d_max, st));
         {  // Y_{k+1} = Y_k + Y_k Delta (in place)
           OzEpi e = epi(EPI_AXPY, w.Y, w.sY, w.sD);
           e.aux = w.Y;
           e.lda = n;
           e.bsa = nn;
+          CK(oz_clear_max(w.maxbuf, N, N, B, st));
           CK(gemm_oz(w.sY.rows, w.sD.cols, N, N, N, B, e, st));
+          CK(slice(w.Y, w.sY, nullptr, w.maxbuf, true, st));
         }
         if (!first) {  // Z_{k+1} = Z_k + Delta Z_k (in place)
           OzEpi e = epi(EPI_AXPY, w.Z, w.sD, w.sZ);
           e.aux = w.Z;
           e.lda = n;
           e.bsa = nn;
+          CK(oz_clear_max(w.maxbuf, N, N, B, st));
           CK(gemm_oz(w.sD.rows, w.sZ.cols, N, N, N, B, e, st));
+          CK(slice(w.Z, w.sZ, nullptr, w.maxbuf, true, st));
         }
-        CK(slice(w.Y, w.sY, nullptr, st));
-        CK(slice(w.Z, w.sZ, nullptr, st));
         return SHP_OK;
       };
       int r = record_loop(cs, g, ctl, B, mi, iter);
@@ -803,8 +823,8 @@ int shp_matmul_f64(const double* A, const double* B, double* C, int64_t M, int64
   unsigned* maxbuf = a.take<unsigned>(static_cast<size_t>(M + 2 * K + N) * batch);
   const int m = static_cast<int>(M), nc = static_cast<int>(N), k = static_cast<int>(K);
   const int bt = static_cast<int>(batch);
-  CK(oz_slice(A, m, k, K, M * K, bt, nullptr, maxbuf, sa, nullptr, st));
-  CK(oz_slice(B, k, nc, N, K * N, bt, nullptr, maxbuf + (M + K) * batch, sb, nullptr, st));
+  CK(oz_slice(A, m, k, K, M * K, bt, nullptr, maxbuf, false, sa, nullptr, st));
+  CK(oz_slice(B, k, nc, N, K * N, bt, nullptr, maxbuf + (M + K) * batch, false, sb, nullptr, st));
   OzEpi e;
   memset(&e, 0, sizeof(e));
   e.kind = EPI_STORE;

@@ -849,16 +849,15 @@ cudaError_t dispatch_pair(bool pair, bool amn, bool bmn, const CUtensorMap& a,
 
 }  // namespace
 
-bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t K, int64_t rows, int slices,
-                       int64_t batch, int64_t ldk, int box_k, int box_rows) {
+bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t rows, int slices,
+                       int64_t blocks, int box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(slices), static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(ldk), static_cast<cuuint64_t>(rows * ldk),
-                           static_cast<cuuint64_t>(slices * rows * ldk)};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_k), static_cast<cuuint32_t>(box_rows),
-                       static_cast<cuuint32_t>(slices), 1};
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices),
+                        static_cast<cuuint64_t>(blocks)};
+  cuuint64_t strides[3] = {64, static_cast<cuuint64_t>(rows * 64),
+                           static_cast<cuuint64_t>(slices * rows * 64)};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(slices), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<int8_t*>(ptr), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,

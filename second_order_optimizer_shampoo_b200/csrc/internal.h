@@ -105,12 +105,11 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
 bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
                      int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows);
 
-// 4-D int8 map over [batch][slices][rows][K] (row stride ldk bytes, a
-// multiple of 16) with a box of all slices x box_rows x box_k bytes and the
-// 64-byte swizzle, zero fill outside the tensor: the digit slices of the
-// Ozaki-scheme products (ozaki.cu).
-bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t K, int64_t rows, int slices,
-                       int64_t batch, int64_t ldk, int box_k, int box_rows);
+// 4-D int8 map over [blocks][slices][rows][64] (the K-blocked digit slices of
+// the Ozaki-scheme products, ozaki.cu) with a box of all slices x box_rows x
+// 64 bytes and the 64-byte swizzle, zero fill past `rows`.
+bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t rows, int slices,
+                       int64_t blocks, int box_rows);
 
 // ---- PRISM sketch and alpha (sketch_alpha.cu)
 // Vout[b] = R[b] * Vin[b]; R is n x n (hi + lo when lo != null); V is n x p.
@@ -251,12 +250,12 @@ cudaError_t small_polar(const float* G, int m, int n, int batch, const shp_prism
 
 // ---- fp64-grade products on the int8 tensor cores (ozaki.cu)
 // Digit slices of an fp64 matrix X (rows x cols): the row slicing serves X
-// as the left operand A, the column slicing (stored transposed, i.e. as the
-// row slicing of X^T) as the right operand B.  Row r of a slice buffer is
-// oz_ldk(K) bytes long (K = cols for `rows`, rows for `cols`).
+// as the left operand A, the column slicing (that of X^T) as the right
+// operand B.  Both are K-blocked: [batch][K / 64][S][rows of the operand][64]
+// with K padded to oz_ldk(K) (K = cols for `rows`, rows for `cols`).
 struct OzSlices {
-  int8_t* rows;    // [batch][S][rows][oz_ldk(cols)], weights rscale
-  int8_t* cols;    // [batch][S][cols][oz_ldk(rows)], weights cscale
+  int8_t* rows;    // [batch][cols / 64][S][rows][64], weights rscale
+  int8_t* cols;    // [batch][rows / 64][S][cols][64], weights cscale
   double* rscale;  // [batch][rows]
   double* cscale;  // [batch][cols]
 };
@@ -281,17 +280,26 @@ struct OzEpi {
   const int* active;
   int* status;
   int M, N;
+  // maxima keys (high word of |v|) of out and out2 by row [batch][M] and by
+  // column [batch][N], folded in with atomicMax (may be null)
+  unsigned* rmax;
+  unsigned* cmax;
+  unsigned* rmax2;
+  unsigned* cmax2;
 };
-int64_t oz_ldk(int64_t k);                                     // slice row length (bytes)
+int64_t oz_ldk(int64_t k);                                     // K padded to whole blocks
 size_t oz_slices_bytes(int64_t rows, int64_t k, int64_t batch);  // one slicing's digits
 int oz_slice_count();
 // Slices of X ([batch][rows][cols] at ld / bs); out.rows / out.cols may be
-// null to skip that slicing; maxbuf is (rows + cols) * batch unsigned of
-// scratch; x32 (may be null) gets a plain fp32 copy of X.  Blocks with
-// active[b] == 0 are skipped.
+// null to skip that slicing; maxbuf holds the row maxima keys [batch][rows]
+// and then the column ones [batch][cols]: with have_max they were folded in
+// by the epilogue that wrote X (after oz_clear_max), otherwise they are
+// computed here first.  x32 (may be null) gets a plain fp32 copy of X.
+// Blocks with active[b] == 0 are skipped.
 cudaError_t oz_slice(const double* X, int rows, int cols, int64_t ld, int64_t bs, int batch,
-                     const int* active, unsigned* maxbuf, const OzSlices& out, float* x32,
-                     cudaStream_t st);
+                     const int* active, unsigned* maxbuf, bool have_max, const OzSlices& out,
+                     float* x32, cudaStream_t st);
+cudaError_t oz_clear_max(unsigned* maxbuf, int rows, int cols, int batch, cudaStream_t st);
 // C = A B from A's row slices ([batch][S][M][oz_ldk(K)]) and B's column
 // slices ([batch][S][N][oz_ldk(K)]), then the epilogue.
 cudaError_t gemm_oz(const int8_t* Arows, const int8_t* Bcols, int M, int N, int K, int batch,

@@ -28,12 +28,15 @@
 // Kernel k_gemm_oz: one cluster of two CTAs per SM pair, persistent over
 // 256 x 96 output tiles.  Warp 0 loads all five slices of a 64-byte K step of
 // A (128 rows per CTA) and of B^T (48 rows per CTA) with one 4-D TMA copy
-// each into a 3-deep ring; the leader's warp 1 issues 30 tcgen05.mma
+// each into a 4-deep ring; the leader's warp 1 issues 30 tcgen05.mma
 // kind::i8 (M = 256, N = 96, K = 32) per stage into five int32 accumulators
-// (TMEM columns 0..479); warps 2..9 combine the levels in fp64 and run the
-// epilogue straight from registers (each thread owns one row: 16-column
-// chunks, 16-byte stores).  Five accumulators fill TMEM, so a tile's epilogue
-// is not overlapped with the next tile's products.  No TMA multicast.
+// (TMEM columns 0..479); warps 2..13 first drain their 32 columns of the five
+// accumulators into fp64 registers and release TMEM (the next tile's products
+// start then), and only after that apply the scales and the elementwise
+// update, store (each thread owns one row, 16-byte stores) and fold the row
+// and column maxima of the output into the arrays the next slicing reads.
+// Five accumulators fill TMEM, so this split is what overlaps a tile's
+// epilogue traffic with the next tile's products.  No TMA multicast.
 #include <math.h>
 #include <stdint.h>
 
@@ -47,7 +50,10 @@ namespace {
 constexpr int OZ_S = 5;                              // digit slices per operand
 constexpr int OZ_BN = 96;                            // tile columns (pair tile 256 x 96)
 constexpr int OZ_BK = 64;                            // K bytes per stage
-constexpr int OZ_STAGES = 3;
+#ifndef OZ_STAGES_N
+#define OZ_STAGES_N 4
+#endif
+constexpr int OZ_STAGES = OZ_STAGES_N;
 constexpr int OZ_A_SLICE = 128 * OZ_BK;              // one slice of A per CTA: 8 KB
 constexpr int OZ_B_SLICE = (OZ_BN / 2) * OZ_BK;      // one slice of B^T per CTA: 3 KB
 constexpr int OZ_A_BYTES = OZ_S * OZ_A_SLICE;
@@ -119,17 +125,39 @@ SHP_DEV void oz_scale_of(unsigned key, double& factor, double& sigma) {
   sigma = __longlong_as_double(static_cast<long long>(1023 + e) << 52) * (1.0 / 127.0);
 }
 
-// The five balanced base-256 digits of x (top digit first), given the row's
-// factor 2^-e: T = rint(x 2^-e 127 2^32).
-SHP_DEV void oz_digits(double x, double factor, int (&d)[OZ_S]) {
-  long long T = __double2ll_rn((x * factor) * 545460846592.0);  // 127 * 2^32
+// Exact conversions through the fp64 adder instead of the (much narrower)
+// conversion unit: an int32 v is the double with high word 0x43300000 and low
+// word v ^ 2^31, less 2^52 + 2^31; rint(t) for |t| < 2^51 is the low part of
+// t + 1.5 * 2^52 (the addition rounds to nearest even, as rint does).
+SHP_DEV double i32_to_f64(uint32_t v) {
+  return __hiloint2double(0x43300000, static_cast<int>(v ^ 0x80000000u)) - 4503601774854144.0;
+}
+SHP_DEV long long rint_to_i64(double t) {
+  return __double_as_longlong(t + 6755399441055744.0) - 0x4338000000000000ll;
+}
+
+// Digit slices of four consecutive elements x[0..3] that share the factor
+// 2^-e of their row (or column): T = rint(x 2^-e 127 2^32) in balanced base
+// 256.  With U = T + 0x80808080 the low word holds D_4 .. D_1 offset by 128
+// byte by byte (so XOR 0x80 gives each digit's two's-complement byte) and the
+// high word is D_0; w[s] receives the four elements' digit s, one per byte.
+SHP_DEV void oz_digits4(const double (&x)[4], double factor, uint32_t (&w)[OZ_S]) {
+  uint32_t lo[4], hi[4];
 #pragma unroll
-  for (int s = OZ_S - 1; s >= 1; --s) {
-    const int lo = static_cast<int>(static_cast<signed char>(T & 0xff));
-    d[s] = lo;
-    T = (T - lo) >> 8;
+  for (int e = 0; e < 4; ++e) {
+    const long long T = rint_to_i64((x[e] * factor) * 545460846592.0);  // 127 * 2^32
+    const long long U = T + 0x80808080ll;
+    lo[e] = static_cast<uint32_t>(U) ^ 0x80808080u;
+    hi[e] = static_cast<uint32_t>(U >> 32);
   }
-  d[0] = static_cast<int>(T);
+  // 4 x 4 byte transpose: byte k of lo[e] is digit 4 - k of element e
+  const uint32_t t0 = __byte_perm(lo[0], lo[1], 0x5140), t1 = __byte_perm(lo[0], lo[1], 0x7362);
+  const uint32_t t2 = __byte_perm(lo[2], lo[3], 0x5140), t3 = __byte_perm(lo[2], lo[3], 0x7362);
+  w[4] = __byte_perm(t0, t2, 0x5410);
+  w[3] = __byte_perm(t0, t2, 0x7632);
+  w[2] = __byte_perm(t1, t3, 0x5410);
+  w[1] = __byte_perm(t1, t3, 0x7632);
+  w[0] = __byte_perm(__byte_perm(hi[0], hi[1], 0x0040), __byte_perm(hi[2], hi[3], 0x0040), 0x5410);
 }
 
 // ------------------------------------------------------------- slicing
@@ -180,17 +208,19 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Digit slices of a 64 x 64 tile of X: row slicing (A role) into
-// rsl[b][s][i][j] with weights rscale[b][i], column slicing (B role, stored
-// transposed, i.e. the row slicing of X^T) into csl[b][s][j][i] with weights
-// cscale[b][j].  Either output may be null.  Columns up to the padded row
-// length of a slice buffer get digits of 0 past the matrix edge.  x32, when
-// non-null, gets a plain fp32 copy of X.
+// Digit slices of a 64 x 64 tile of X.  Slices are stored K-blocked, so that
+// the copy of one 64-byte K step of every slice of a 128-row tile is one
+// contiguous stretch of memory: digit s of element (row, k) of an operand
+// with R rows sits at [b][k / 64][s][row][k % 64].  Row slicing (A role, K =
+// the column index) goes to rsl with weights rscale[b][i], column slicing (B
+// role, K = the row index: the row slicing of X^T) to csl with weights
+// cscale[b][j].  Either output may be null.  Past the matrix edge the last K
+// block holds digits of 0.  x32, when non-null, gets a plain fp32 copy of X.
 __global__ void __launch_bounds__(256)
     k_oz_slice(const double* __restrict__ X, int rows, int cols, int64_t ld, int64_t bs,
                const int* __restrict__ active, const unsigned* __restrict__ rmax,
-               const unsigned* __restrict__ cmax, int8_t* rsl, int64_t ldr, int8_t* csl,
-               int64_t ldc, double* rscale, double* cscale, float* x32) {
+               const unsigned* __restrict__ cmax, int8_t* rsl, int8_t* csl, double* rscale,
+               double* cscale, float* x32) {
   count_kernel_run();
   const int b = blockIdx.z;
   if (active != nullptr && active[b] == 0) return;
@@ -216,133 +246,191 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   const int idx = threadIdx.x >> 2, seg = (threadIdx.x & 3) * 16;
   // row slicing: this thread's row r0 + idx, columns c0 + seg .. + 15
-  if (rsl != nullptr && r0 + idx < rows && c0 + seg < ldr) {
+  const int64_t nkb_r = (cols + SL_T - 1) / SL_T, nkb_c = (rows + SL_T - 1) / SL_T;
+  if (rsl != nullptr && r0 + idx < rows) {
     const int r = r0 + idx;
     double f, sg;
     oz_scale_of(rmax[static_cast<int64_t>(b) * rows + r], f, sg);
     if (blockIdx.x == 0 && seg == 0 && rscale != nullptr) rscale[static_cast<int64_t>(b) * rows + r] = sg;
     uint32_t w[OZ_S][4];
 #pragma unroll
-    for (int s = 0; s < OZ_S; ++s)
+    for (int g = 0; g < 4; ++g) {
+      double x[4];
+      uint32_t d[OZ_S];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) w[s][q] = 0u;
+      for (int e = 0; e < 4; ++e) x[e] = tile[idx][seg + 4 * g + e];
+      oz_digits4(x, f, d);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      int d[OZ_S];
-      oz_digits(tile[idx][seg + j], f, d);
-#pragma unroll
-      for (int s = 0; s < OZ_S; ++s) w[s][j >> 2] |= (static_cast<uint32_t>(d[s]) & 0xffu) << (8 * (j & 3));
+      for (int q = 0; q < OZ_S; ++q) w[q][g] = d[q];
     }
 #pragma unroll
-    for (int s = 0; s < OZ_S; ++s) {
-      int8_t* dst = rsl + ((static_cast<int64_t>(b) * OZ_S + s) * rows + r) * ldr + c0 + seg;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
+    for (int q = 0; q < OZ_S; ++q) {
+      int8_t* dst =
+          rsl + ((((b * nkb_r + blockIdx.x) * OZ_S + q) * rows + r) * SL_T) + seg;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
     }
   }
   // column slicing: this thread's column c0 + idx, rows r0 + seg .. + 15
-  if (csl != nullptr && c0 + idx < cols && r0 + seg < ldc) {
+  if (csl != nullptr && c0 + idx < cols) {
     const int c = c0 + idx;
     double f, sg;
     oz_scale_of(cmax[static_cast<int64_t>(b) * cols + c], f, sg);
     if (blockIdx.y == 0 && seg == 0 && cscale != nullptr) cscale[static_cast<int64_t>(b) * cols + c] = sg;
     uint32_t w[OZ_S][4];
 #pragma unroll
-    for (int s = 0; s < OZ_S; ++s)
+    for (int g = 0; g < 4; ++g) {
+      double x[4];
+      uint32_t d[OZ_S];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) w[s][q] = 0u;
+      for (int e = 0; e < 4; ++e) x[e] = tile[seg + 4 * g + e][idx];
+      oz_digits4(x, f, d);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      int d[OZ_S];
-      oz_digits(tile[seg + j][idx], f, d);
-#pragma unroll
-      for (int s = 0; s < OZ_S; ++s) w[s][j >> 2] |= (static_cast<uint32_t>(d[s]) & 0xffu) << (8 * (j & 3));
+      for (int q = 0; q < OZ_S; ++q) w[q][g] = d[q];
     }
 #pragma unroll
-    for (int s = 0; s < OZ_S; ++s) {
-      int8_t* dst = csl + ((static_cast<int64_t>(b) * OZ_S + s) * cols + c) * ldc + r0 + seg;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
+    for (int q = 0; q < OZ_S; ++q) {
+      int8_t* dst =
+          csl + ((((b * nkb_c + blockIdx.y) * OZ_S + q) * cols + c) * SL_T) + seg;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
     }
   }
 }
 
 // ------------------------------------------------------------- the GEMM
-// Epilogue of one thread's row (rows past M skip memory but still take part
-// in the warp-collective TMEM loads): 16-column chunks, levels combined in
-// fp64, then the kind's elementwise update.
-SHP_DEV double oz_tile_epilogue(uint32_t trow, const OzEpi& ep, int b, int row, int n0, int h) {
+constexpr int OZ_EPI_WARPS = 12;  // 4 TMEM lane quarters x 3 groups of 32 columns
+constexpr int OZ_THREADS = 32 * (2 + OZ_EPI_WARPS);
+
+SHP_DEV void tmem_ld8_nowait(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+}
+
+// Phase 1 of a tile's epilogue: this thread's row, 32 columns of the five
+// level accumulators, combined in fp64 (exact up to the last bits): the TMEM
+// accumulators are free again once every warp has done this.
+SHP_DEV void oz_drain(uint32_t taddr, double (&acc)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t l[OZ_S][8];
+#pragma unroll
+    for (int L = 0; L < OZ_S; ++L)
+      tmem_ld8_nowait(taddr + static_cast<uint32_t>(L * OZ_BN + 8 * c), l[L]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      double t = i32_to_f64(l[OZ_S - 1][j]);
+#pragma unroll
+      for (int L = OZ_S - 2; L >= 0; --L) t = fma(t, 0.00390625, i32_to_f64(l[L][j]));
+      acc[8 * c + j] = t;
+    }
+  }
+}
+
+// Maximum over the warp's 32 rows of each of 8 column keys, by recursive
+// halving (9 shuffles): lanes 4c .. 4c + 3 end with the maximum of column c.
+SHP_DEV uint32_t col_max8(uint32_t (&k)[8], int lane) {
+#pragma unroll
+  for (int st = 0; st < 3; ++st) {
+    const int o = 16 >> st, h = 4 >> st;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const uint32_t send = up ? k[i] : k[i + h];
+      const uint32_t keep = up ? k[i + h] : k[i];
+      k[i] = max(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+  uint32_t v = k[0];
+  v = max(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  v = max(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return v;
+}
+
+// Phase 2: scales, the kind's elementwise update, fp64 stores (16 bytes at a
+// time; a thread owns one row) and the row/column maxima of what is stored,
+// which the next slicing needs.  Rows past M take part in the shuffles only.
+SHP_DEV double oz_finish_tile(const double (&acc)[32], const OzEpi& ep, int b, int row, int col00,
+                              int lane) {
   const bool rowok = row < ep.M;
   const double sa = rowok ? ep.sa[static_cast<int64_t>(b) * ep.M + row] : 0.0;
   const double alpha = ep.alpha != nullptr ? static_cast<double>(ep.alpha[b]) : 0.0;
   const double* sb = ep.sb + static_cast<int64_t>(b) * ep.N;
   double nrm = 0.0;
-#pragma unroll 1
-  for (int c = 0; c < OZ_BN / 32; ++c) {
-    const int col0 = n0 + h * (OZ_BN / 2) + c * 16;
-    __syncwarp();  // the TMEM loads below are warp-collective
-    uint32_t l[OZ_S][16];
+  uint32_t rk = 0u, rk2 = 0u;
 #pragma unroll
-    for (int L = 0; L < OZ_S; ++L)
-      tmem_ld16_nowait(trow + static_cast<uint32_t>(L * OZ_BN + h * (OZ_BN / 2) + c * 16), l[L]);
-    tmem_wait_ld();
-    if (!rowok || col0 >= ep.N) continue;
-    const int nv = ep.N - col0 < 16 ? ep.N - col0 : 16;  // a multiple of 4
-    double v[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      double t = static_cast<double>(static_cast<int>(l[OZ_S - 1][j]));
-#pragma unroll
-      for (int L = OZ_S - 2; L >= 0; --L)
-        t = fma(t, 0.00390625, static_cast<double>(static_cast<int>(l[L][j])));
-      const double sbj = j < nv ? __ldg(sb + col0 + j) : 0.0;
-      v[j] = t * sa * sbj;
-    }
+  for (int c = 0; c < 4; ++c) {
+    const int col0 = col00 + 8 * c;
+    const int nv = col0 >= ep.N ? 0 : (ep.N - col0 < 8 ? ep.N - col0 : 8);  // 0, 4 or 8
+    const bool ok = rowok && nv > 0;
     const int64_t off = static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row) * ep.ldo + col0;
-    double x[16];
-    if (ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY) {
+    double x[8];
+    if (ok && (ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY)) {
       const double* ap = ep.aux + static_cast<int64_t>(b) * ep.bsa + static_cast<int64_t>(row) * ep.lda + col0;
 #pragma unroll
-      for (int j = 0; j < 16; j += 2) {
+      for (int j = 0; j < 8; j += 2) {
         double2 a2 = make_double2(0.0, 0.0);
         if (j < nv) a2 = *reinterpret_cast<const double2*>(ap + j);
         x[j] = a2.x;
         x[j + 1] = a2.y;
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = 0.0;
     }
-    double out[16];
+    double out[8];
     const int dcol = row - col0;  // column j of this chunk is on the diagonal when j == dcol
-    switch (ep.kind) {
-      case EPI_RESID:
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          out[j] = (j == dcol ? 1.0 : 0.0) - v[j];
-          if (j < nv) nrm += out[j] * out[j];
-        }
-        break;
-      case EPI_GPOLY:
-#pragma unroll
-        for (int j = 0; j < 16; ++j) out[j] = static_cast<double>(ep.s1) * x[j] + alpha * v[j];
-        break;
-      case EPI_AXPY:
-#pragma unroll
-        for (int j = 0; j < 16; ++j) out[j] = x[j] + static_cast<double>(ep.s0) * v[j];
-        break;
-      default:
-#pragma unroll
-        for (int j = 0; j < 16; ++j) out[j] = static_cast<double>(ep.s0) * v[j];
-        break;
+    for (int j = 0; j < 8; ++j) {
+      const double v = ok && j < nv ? acc[8 * c + j] * sa * __ldg(sb + col0 + j) : 0.0;
+      switch (ep.kind) {
+        case EPI_RESID: out[j] = (j == dcol ? 1.0 : 0.0) - v; break;
+        case EPI_GPOLY: out[j] = static_cast<double>(ep.s1) * x[j] + alpha * v; break;
+        case EPI_AXPY: out[j] = x[j] + static_cast<double>(ep.s0) * v; break;
+        default: out[j] = static_cast<double>(ep.s0) * v; break;
+      }
     }
-    double* op = ep.out + off;
+    uint32_t ck[8], ck2[8];
 #pragma unroll
-    for (int j = 0; j < 16; j += 2)
-      if (j < nv) *reinterpret_cast<double2*>(op + j) = make_double2(out[j], out[j + 1]);
-    if (ep.out2 != nullptr) {  // I + Delta
-      double* o2 = ep.out2 + off;
-#pragma unroll
-      for (int j = 0; j < 16; j += 2)
-        if (j < nv)
-          *reinterpret_cast<double2*>(o2 + j) =
-              make_double2(out[j] + (j == dcol ? 1.0 : 0.0), out[j + 1] + (j + 1 == dcol ? 1.0 : 0.0));
+    for (int j = 0; j < 8; ++j) {
+      const bool in = ok && j < nv;
+      if (in && ep.kind == EPI_RESID) nrm += out[j] * out[j];
+      ck[j] = in ? abs_key(out[j]) : 0u;
+      ck2[j] = in ? abs_key(out[j] + (j == dcol ? 1.0 : 0.0)) : 0u;
+      rk = max(rk, ck[j]);
+      rk2 = max(rk2, ck2[j]);
     }
+    if (ok) {
+      double* op = ep.out + off;
+#pragma unroll
+      for (int j = 0; j < 8; j += 2)
+        if (j < nv) *reinterpret_cast<double2*>(op + j) = make_double2(out[j], out[j + 1]);
+      if (ep.out2 != nullptr) {  // I + Delta
+        double* o2 = ep.out2 + off;
+#pragma unroll
+        for (int j = 0; j < 8; j += 2)
+          if (j < nv)
+            *reinterpret_cast<double2*>(o2 + j) = make_double2(
+                out[j] + (j == dcol ? 1.0 : 0.0), out[j + 1] + (j + 1 == dcol ? 1.0 : 0.0));
+      }
+    }
+    if (ep.cmax != nullptr) {
+      const uint32_t m = col_max8(ck, lane);
+      if ((lane & 3) == 0 && (lane >> 2) < nv && m != 0u)
+        atomicMax(&ep.cmax[static_cast<int64_t>(b) * ep.N + col0 + (lane >> 2)], m);
+      if (ep.out2 != nullptr) {
+        const uint32_t m2 = col_max8(ck2, lane);
+        if ((lane & 3) == 0 && (lane >> 2) < nv && m2 != 0u)
+          atomicMax(&ep.cmax2[static_cast<int64_t>(b) * ep.N + col0 + (lane >> 2)], m2);
+      }
+    }
+  }
+  if (ep.rmax != nullptr && rowok) {
+    if (rk != 0u) atomicMax(&ep.rmax[static_cast<int64_t>(b) * ep.M + row], rk);
+    if (ep.out2 != nullptr && rk2 != 0u)
+      atomicMax(&ep.rmax2[static_cast<int64_t>(b) * ep.M + row], rk2);
   }
   return nrm;
 }
@@ -350,8 +438,9 @@ SHP_DEV double oz_tile_epilogue(uint32_t trow, const OzEpi& ep, int b, int row, 
 //   full[s]/empty[s]: operand ring (the leader's full barrier counts both
 //                     CTAs' bytes; empty is signalled to both by the commit)
 //   accf:             the five level accumulators of the current tile complete
-//   acce:             ... drained (8 epilogue warps x 2 CTAs arrive on the leader's)
-__global__ void __launch_bounds__(320, 1)
+//   acce:             ... drained into registers (12 epilogue warps x 2 CTAs
+//                     arrive on the leader's)
+__global__ void __launch_bounds__(OZ_THREADS, 1)
     k_gemm_oz(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
               int K, OzEpi ep, int batch) {
   count_kernel_run();
@@ -380,7 +469,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
-    mbar_init(acce, 16);
+    mbar_init(acce, 2 * OZ_EPI_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -419,8 +508,8 @@ __global__ void __launch_bounds__(320, 1)
           uint8_t* st = smem + s * OZ_STAGE;
           if (leader) mbar_arrive_expect_tx(&full[s], tx);
           const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
-          tma_load_4d_pair(st, &tA, fbar, kb * OZ_BK, m0, 0, b);
-          tma_load_4d_pair(st + OZ_A_BYTES, &tB, fbar, kb * OZ_BK, nb0, 0, b);
+          tma_load_4d_pair(st, &tA, fbar, 0, m0, 0, b * KB + kb);
+          tma_load_4d_pair(st + OZ_A_BYTES, &tB, fbar, 0, nb0, 0, b * KB + kb);
         }
       }
     }
@@ -449,7 +538,12 @@ __global__ void __launch_bounds__(320, 1)
             break;
           }
           tc_fence_after();
+          // the descriptors' start-address field holds address >> 4 (shared
+          // memory addresses stay below 2^18, so adding offsets >> 4 to the
+          // base descriptor never carries out of the field)
           const uint32_t base = smem_u32(smem + s * OZ_STAGE);
+          const uint64_t ad0 = smem_desc(base, 16, 512, 4);
+          const uint64_t bd0 = smem_desc(base + OZ_A_BYTES, 16, 512, 4);
 #pragma unroll
           for (int ks = 0; ks < OZ_BK / 32; ++ks) {
 #pragma unroll
@@ -457,9 +551,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
               for (int sa = 0; sa <= L; ++sa) {
                 const int sb = L - sa;
-                const uint64_t ad = smem_desc(base + sa * OZ_A_SLICE + ks * 32, 16, 512, 4);
-                const uint64_t bd =
-                    smem_desc(base + OZ_A_BYTES + sb * OZ_B_SLICE + ks * 32, 16, 512, 4);
+                const uint64_t ad = ad0 + static_cast<uint64_t>((sa * OZ_A_SLICE + ks * 32) >> 4);
+                const uint64_t bd = bd0 + static_cast<uint64_t>((sb * OZ_B_SLICE + ks * 32) >> 4);
                 mma_i8_pair(tmem + static_cast<uint32_t>(L * OZ_BN), ad, bd, idesc,
                             (kb > 0 || ks > 0 || sa > 0) ? 1u : 0u);
               }
@@ -474,8 +567,10 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (lane == 0 && leader) mma_commit_pair(drain, 3);  // after every MMA issued above
   } else {
-    // ---------------- epilogue warps 2..9 (both CTAs, each on its TMEM rows)
-    const int q = warp & 3, h = (warp - 2) >> 2;
+    // ---------------- epilogue warps 2..13 (both CTAs, each on its TMEM rows):
+    // drain the accumulators, release them to the next tile's products, then
+    // finish this tile while those run
+    const int q = warp & 3, g = (warp - 2) >> 2;
     int tl = 0;
     for (int t = cl; t < ntiles; t += ncl) {
       const int b = t / per_b, r = t % per_b;
@@ -487,13 +582,14 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
       tc_fence_after();
-      const int tm = r / tiles_n, tn = r % tiles_n;
-      const int row = tm * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-      double nrm = oz_tile_epilogue(tmem + (static_cast<uint32_t>(q * 32) << 16), ep, b, row,
-                                    tn * OZ_BN, h);
+      double acc[32];
+      oz_drain(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(32 * g), acc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(acce), 0));
+      const int tm = r / tiles_n, tn = r % tiles_n;
+      const int row = tm * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      double nrm = oz_finish_tile(acc, ep, b, row, tn * OZ_BN + 32 * g, lane);
       if (ep.kind == EPI_RESID) {
         nrm = warp_sum(nrm);
         if (lane == 0)
@@ -628,7 +724,7 @@ __global__ void __launch_bounds__(EW)
 }  // namespace
 
 // ------------------------------------------------------------- host side
-int64_t oz_ldk(int64_t k) { return (k + 15) / 16 * 16; }
+int64_t oz_ldk(int64_t k) { return (k + SL_T - 1) / SL_T * SL_T; }
 
 size_t oz_slices_bytes(int64_t rows, int64_t k, int64_t batch) {
   return static_cast<size_t>(OZ_S) * rows * oz_ldk(k) * batch;
@@ -636,32 +732,37 @@ size_t oz_slices_bytes(int64_t rows, int64_t k, int64_t batch) {
 
 int oz_slice_count() { return OZ_S; }
 
+cudaError_t oz_clear_max(unsigned* maxbuf, int rows, int cols, int batch, cudaStream_t st) {
+  return cudaMemsetAsync(maxbuf, 0, sizeof(unsigned) * static_cast<size_t>(batch) * (rows + cols),
+                         st);
+}
+
 cudaError_t oz_slice(const double* X, int rows, int cols, int64_t ld, int64_t bs, int batch,
-                     const int* active, unsigned* maxbuf, const OzSlices& out, float* x32,
-                     cudaStream_t st) {
+                     const int* active, unsigned* maxbuf, bool have_max, const OzSlices& out,
+                     float* x32, cudaStream_t st) {
   if (rows <= 0 || cols <= 0 || batch <= 0) return cudaSuccess;
   unsigned* rmax = maxbuf;
   unsigned* cmax = maxbuf + static_cast<int64_t>(batch) * rows;
-  cudaError_t e = cudaMemsetAsync(
-      maxbuf, 0, sizeof(unsigned) * static_cast<size_t>(batch) * (rows + cols), st);
-  if (e != cudaSuccess) return e;
-  const dim3 grid((cols + SL_T - 1) / SL_T, (rows + SL_T - 1) / SL_T, batch);
-  k_oz_absmax<<<grid, 256, 0, st>>>(X, rows, cols, ld, bs, active, rmax, cmax);
-  // the slicing tiles cover the padded slice rows too (digits 0 past the edge)
-  const int64_t ldr = oz_ldk(cols), ldc = oz_ldk(rows);
-  const dim3 grid2((ldr + SL_T - 1) / SL_T, (ldc + SL_T - 1) / SL_T, batch);
-  k_oz_slice<<<grid2, 256, 0, st>>>(X, rows, cols, ld, bs, active, rmax, cmax, out.rows, ldr,
-                                    out.cols, ldc, out.rscale, out.cscale, x32);
+  if (!have_max) {
+    cudaError_t e = oz_clear_max(maxbuf, rows, cols, batch, st);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((cols + SL_T - 1) / SL_T, (rows + SL_T - 1) / SL_T, batch);
+    k_oz_absmax<<<grid, 256, 0, st>>>(X, rows, cols, ld, bs, active, rmax, cmax);
+  }
+  const dim3 grid2((cols + SL_T - 1) / SL_T, (rows + SL_T - 1) / SL_T, batch);
+  k_oz_slice<<<grid2, 256, 0, st>>>(X, rows, cols, ld, bs, active, rmax, cmax, out.rows,
+                                    out.cols, out.rscale, out.cscale, x32);
   return cudaGetLastError();
 }
 
 cudaError_t gemm_oz(const int8_t* Arows, const int8_t* Bcols, int M, int N, int K, int batch,
                     const OzEpi& ep, cudaStream_t st) {
   if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return cudaSuccess;
+  static_assert(OZ_BK == SL_T, "a GEMM stage is one K block of the slice layout");
   CUtensorMap ma, mb;
-  const int64_t ldk = oz_ldk(K);
-  if (!tensor_map_slices(&ma, Arows, K, M, OZ_S, batch, ldk, OZ_BK, 128) ||
-      !tensor_map_slices(&mb, Bcols, K, N, OZ_S, batch, ldk, OZ_BK, OZ_BN / 2))
+  const int64_t nkb = (K + OZ_BK - 1) / OZ_BK;
+  if (!tensor_map_slices(&ma, Arows, M, OZ_S, nkb * batch, 128) ||
+      !tensor_map_slices(&mb, Bcols, N, OZ_S, nkb * batch, OZ_BN / 2))
     return cudaErrorInvalidValue;
   static int attr_set[64];
   int dev = 0, sms = 148;
@@ -679,7 +780,7 @@ cudaError_t gemm_oz(const int8_t* Arows, const int8_t* Bcols, int M, int N, int 
   if (ncl < 1) ncl = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ncl, 1, 1);
-  cfg.blockDim = dim3(320, 1, 1);
+  cfg.blockDim = dim3(OZ_THREADS, 1, 1);
   cfg.dynamicSmemBytes = OZ_SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
