@@ -4,14 +4,18 @@
 Workload (one "step"): A^(-1/4) of 64 SPD blocks of 1024 x 1024, each
 Q diag(lambda) Q^T with lambda log-uniform on [1e-6, 1] (cond 1e6), by two
 coupled Newton-Schulz passes with PRISM alpha (d = 2, Gaussian sketch p = 8,
-alpha in [3/8, 1], residual tol 1e-3 per pass), products on the tensor cores
-in the 3xTF32 split (plain TF32 rounding of A/||A||_F exceeds lambda_min
-and the iteration diverges).
+alpha in [3/8, 1], residual tol 1e-3 per pass), on the fp64-grade path:
+fp64 iterates, every product by the Ozaki scheme on the int8 tensor cores
+(five digit slices per operand, exact int32 accumulation).  fp32 storage
+cannot hold this spectrum: TF32 rounding of A/||A||_F makes the blocks
+indefinite and the 3xTF32 split ends about 4e-2 from eigh; both are reported
+beside the headline as context.
 
 Metric: algorithmic TFLOP/s (2 n^3 per n x n product actually executed,
-summed over blocks) and preconditioners/s, with the fraction of the tensor
-peak.  Under torchrun each rank runs its own independent batch (replicas,
-weak scaling); the time is the max over ranks.
+summed over blocks) and preconditioners/s, with the fraction of the int8
+tensor peak that the dominant kernel reaches (15 int8 digit products per
+fp64-grade product).  Under torchrun each rank runs its own independent batch
+(replicas, weak scaling); the time is the max over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -34,13 +38,20 @@ sys.path.insert(0, ROOT)
 METRIC = "inv-root/polar TFLOP/s & preconditioners/s at 1024², % of B200 tensor peak"
 N, BATCH, LAM_LO, D, P, TOL, MAX_ITER = 1024, 64, 1e-6, 2, 8, 1e-3, 24
 SEED_A, SEED_S = 103, 1003
-# tensor peak ratios (nominal dense): TF32 / BF16 = 1.1 / 2.25 PFLOP/s
+PREC = "ozaki"
+OZ_SLICES = 5
+OZ_PRODUCTS = OZ_SLICES * (OZ_SLICES + 1) // 2  # int8 digit products per fp64-grade product
+# blocks whose accuracy the bench reports (the two where the float64 oracle,
+# stopped at residual 1e-3 per pass, is farthest from eigh, and two others)
+ACC_BLOCKS = (0, 5, 37, 63)
+# tensor peak ratios (nominal dense), used only where a peak is not measured
 TF32_OVER_BF16 = 1.1 / 2.25
-# dram__bytes_read.sum + dram__bytes_write.sum (bytes) of one 64 x 1024^3 3xTF32
-# launch of the persistent GEMM: an ncu capture of 16 blocks (290.1 MB read,
-# 43.4 MB written) scaled x4 by the blocks processed, as every operand and
-# output grows with the batch
+# dram__bytes_read.sum + dram__bytes_write.sum of one 3xTF32 persistent GEMM
+# launch (64 x 1024^3): an ncu capture of 16 blocks scaled x4 by the blocks
 GEMM_TRAFFIC_PER_LAUNCH = 4 * (290.093e6 + 43.367e6)
+# ... of one k_gemm_oz launch with the accumulate (X + X Delta) epilogue,
+# 64 x 1024^3: not captured for the current kernel
+OZ_GEMM_TRAFFIC_PER_LAUNCH = None
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_sketch_tma<8> launch
 # over 48 x 1024^2 (201.393 MB read, 4.646 MB written), scaled x 64/48 by the
 # rows processed and x 5 for the passes of one alpha fit (d = 2)
@@ -51,8 +62,9 @@ def workload_config(world):
     return {
         "workload": f"inv4_root_{BATCH}x1024sq_spd_cond1e6_prism_d2_p8",
         "n": N, "batch_per_gpu": BATCH, "d": D, "p": P, "tol": TOL, "max_iter": MAX_ITER,
-        "alpha_interval": [0.375, 1.0], "prec": "3xtf32", "lambda": "log-uniform [1e-6, 1]",
-        "l2": "inputs larger than L2 (256 MiB of A plus 3.2 GB of iterates per GPU per step)",
+        "alpha_interval": [0.375, 1.0], "prec": "ozaki (fp64 iterates, int8 x5 digit products)",
+        "lambda": "log-uniform [1e-6, 1]",
+        "l2": "inputs larger than L2 (256 MiB of A plus 4.6 GB of iterates and slices per GPU)",
         "parallelism": f"replicas x{world}",
     }
 
@@ -81,6 +93,47 @@ def load_peaks():
         return pk, "measured"
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def measure_tensor_peaks(dev):
+    """Burst tensor-core peaks of this GPU, measured the way the BF16 figure
+    of MEASURED_PEAKS.json is: the best of 10 library GEMMs of 8192^3 (cuBLAS
+    through torch) in TF32 (fp32 inputs, TF32 allowed), BF16, and int8
+    (int32 accumulation)."""
+    import torch
+    n = 8192
+
+    def best(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        t = 1e9
+        for _ in range(10):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t = min(t, e0.elapsed_time(e1))
+        return 2.0 * n ** 3 / (t / 1e3) / 1e12
+
+    g = torch.Generator(device=dev).manual_seed(1)
+    a = torch.randn(n, n, device=dev, generator=g)
+    b = torch.randn(n, n, device=dev, generator=g)
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    tf32 = best(lambda: a @ b)
+    torch.backends.cuda.matmul.allow_tf32 = prev
+    ab, bb = a.bfloat16(), b.bfloat16()
+    bf16 = best(lambda: ab @ bb)
+    ai = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8, generator=g)
+    bi = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8, generator=g).t().contiguous().t()
+    i8 = best(lambda: torch._int_mm(ai, bi))
+    del a, b, ab, bb, ai, bi
+    torch.cuda.empty_cache()
+    return {"tf32_tflops": tf32, "bf16_tflops": bf16, "int8_tops": i8,
+            "how": "best of 10 cuBLAS 8192^3 GEMMs via torch (burst)"}
 
 
 # ------------------------------------------------------------------ clocks
@@ -413,8 +466,9 @@ def shampoo_step_leg(args, dev, stream):
 
 
 def gemm_count_leg(args, dev, stream, A):
-    """GEMMs to residual 1e-3 per pass on the config-3 batch: PRISM d = 2
-    against the fixed-coefficient (Taylor) iterations d = 2 and d = 1."""
+    """GEMMs to residual 1e-3 per pass on the config-3 batch (the headline
+    path): PRISM d = 2 against the fixed-coefficient (Taylor) iterations
+    d = 2 and d = 1."""
     import torch
 
     from second_order_optimizer_shampoo_b200 import prism, synth
@@ -423,7 +477,7 @@ def gemm_count_leg(args, dev, stream, A):
     out = {}
     for name, d, fixed in (("prism_d2", 2, False), ("taylor_d2", 2, True),
                            ("taylor_d1", 1, True)):
-        opts = prism.make_opts(d=d, p=P, tol=TOL, max_iter=mi, prec="3xtf32", fixed_alpha=fixed)
+        opts = prism.make_opts(d=d, p=P, tol=TOL, max_iter=mi, prec=PREC, fixed_alpha=fixed)
         X, rep = prism.matfn_inv_root(A, "inv4", opts, S)
         torch.cuda.synchronize()
         it = rep["iters"].cpu().numpy()
@@ -504,19 +558,20 @@ def single_block_leg(args, dev, stream):
 
 def large_sqrt_leg(args, dev, stream):
     """A^(1/2) of one 10240 x 10240 Marchenko-Pastur matrix (A = X X^T / 20480 +
-    1e-4 I), PRISM d = 2, p = 16, tol 1e-6, split path; GEMMs to the residual
-    against the fixed-coefficient iterations d = 2 and d = 1."""
+    1e-4 I), PRISM d = 2, p = 16, tol 1e-6, on the fp64-grade path (the one
+    that reaches 1e-5 against eigh at this size); GEMMs to the residual
+    against the fixed-coefficient iterations d = 2 and d = 1; the 3xTF32
+    split timed beside it."""
     import torch
 
     from second_order_optimizer_shampoo_b200 import _abi, prism, synth
     n, mi = 10240, 40
     A = torch.from_numpy(synth.mp_spd(n, 2 * n, 1e-4, 105)[None]).to(dev)
     S = torch.from_numpy(synth.sketch_stack(mi, n, 16, 1005)).to(dev)
-    out = {"workload": "sqrt_10240sq_marchenko_pastur_prism_d2_p16_tol1e-6_3xtf32"}
-    for name, d, fixed in (("prism_d2", 2, False), ("taylor_d2", 2, True),
-                           ("taylor_d1", 1, True)):
-        opts = prism.make_opts(d=d, p=16, tol=1e-6, max_iter=mi, prec="3xtf32",
-                               fixed_alpha=fixed)
+    out = {"workload": "sqrt_10240sq_marchenko_pastur_prism_d2_p16_tol1e-6_ozaki"}
+    for name, d, fixed, pr in (("prism_d2", 2, False, "ozaki"), ("taylor_d2", 2, True, "ozaki"),
+                               ("taylor_d1", 1, True, "ozaki"), ("prism_d2_3xtf32", 2, False, "3xtf32")):
+        opts = prism.make_opts(d=d, p=16, tol=1e-6, max_iter=mi, prec=pr, fixed_alpha=fixed)
         ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, n, n, 1, opts),
                          dtype=torch.uint8, device=dev)
         X = torch.empty_like(A)
@@ -530,13 +585,52 @@ def large_sqrt_leg(args, dev, stream):
         k = int(rep["iters"].cpu().numpy()[0][0])
         gemms = max((3 if d == 1 else 4) * k - 1, 0)
         entry = {"iters": k, "gemms": gemms, "status": int(rep["status"].cpu().numpy()[0])}
-        if name == "prism_d2":
+        if not fixed:
             ms = _time(call, stream, 3)
             tf = gemms * 2.0 * n ** 3 / (ms / 1e3) / 1e12
             entry.update({"ms": ms, "value": tf, "unit": "TFLOP/s"})
         out[name] = entry
-        del ws
+        del ws, X
+        torch.cuda.empty_cache()
     return out
+
+
+def tf32_batched_leg(args, dev, stream, tp):
+    """The TF32 path where it applies: 64 SPD blocks 1024^2 in the Shampoo
+    statistics regime (lambda log-uniform on [1e-2, 1], cond 1e2), A^(-1/4),
+    d = 2, p = 8, tol 1e-3, against the measured TF32 tensor peak; accuracy
+    of two blocks against eigh."""
+    import torch
+
+    from oracle import prism_ref as o
+    from second_order_optimizer_shampoo_b200 import _abi, prism, synth
+    mi = 30
+    A_np = synth.spd_batch(N, BATCH, 1e-2, 1.0, 107)
+    A = torch.from_numpy(A_np).to(dev)
+    S = torch.from_numpy(synth.sketch_stack(2 * mi, N, P, 1007)).to(dev)
+    opts = prism.make_opts(d=D, p=P, tol=1e-3, max_iter=mi, prec="tf32")
+    ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, N, N, BATCH, opts),
+                     dtype=torch.uint8, device=dev)
+    X = torch.empty_like(A)
+    rep = prism.make_report(BATCH, mi, dev)
+    call = lambda: prism.matfn_inv_root(A, "inv4", opts, S, out=X, ws=ws, report=rep)  # noqa: E731
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = _time(call, stream, 10)
+    it = rep["iters"].cpu().numpy()
+    tf = float(sum(block_flops(k, N) for k in it)) / (ms / 1e3) / 1e12
+    Xh = X.cpu().numpy()
+    errs = []
+    for b in (0, BATCH - 1):
+        r = o.spd_power_eigh(A_np[b], -0.25)
+        errs.append(float(np.linalg.norm(Xh[b] - r) / np.linalg.norm(r)))
+    st = rep["status"].cpu().numpy()
+    return {"workload": "inv4_root_64x1024sq_spd_cond1e2_prism_d2_p8_tol1e-3_tf32",
+            "ms": ms, "value": tf, "unit": "TFLOP/s", "frac_of_tf32_peak": tf / tp["tf32_tflops"],
+            "median_iters_per_pass": [int(x) for x in np.median(it, axis=0)],
+            "ok_or_stall_blocks": int(((st == 0) | (st == 17)).sum()), "max_vs_eigh": max(errs),
+            "peak_note": "measured TF32 burst (cuBLAS 8192^3)"}
 
 
 PM, PN, PBATCH, PRANK = 4096, 1024, 96, 64
@@ -551,7 +645,7 @@ def polar_flops(iters):
     return k * (sym + PN * (PN + 1) * PN + 2 * PM * PN * PN) + sym
 
 
-def polar_leg(args, dev, stream):
+def polar_leg(args, dev, stream, peaks=None):
     """The Muon-style polar batch: 96 matrices 4096 x 1024, rank-64 signal plus
     0.01 noise, bf16 storage, d = 2, p = 8, until ||I - X^T X||_F / sqrt(n) <= 1e-2."""
     import torch
@@ -582,14 +676,15 @@ def polar_leg(args, dev, stream):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
-    peaks, _ = load_peaks()
+    peaks, src = load_peaks() if peaks is None else (peaks, "given")
     bf16_sust = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     tf = flops / (ms / 1e3) / 1e12
     return {"workload": "polar_96x4096x1024_bf16_lowrank64_prism_d2_p8_tol1e-2",
             "value": tf, "unit": "TFLOP/s", "ms_per_step": ms,
             "matrices_per_s": PBATCH / (ms / 1e3), "median_iters": float(np.median(iters)),
             "status_ok": ok, "frac_of_bf16_peak": tf / bf16_sust,
-            "note": "symmetric products counted n(n+1)K; computed as full GEMMs"}
+            "note": "symmetric products (X^T X, R R) formed on their upper-triangle tiles "
+                    "and counted n(n+1)K; peak: sustained BF16"}
 
 
 def sketch_leg(R, S0, stream, peaks, peak_src):
@@ -662,8 +757,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-polar", action="store_true", help="skip the polar-factor leg")
     ap.add_argument("--no-small", action="store_true", help="skip the small-block leg")
-    ap.add_argument("--large", action="store_true",
-                    help="add the 10240^2 square-root leg (builds a 10240 x 20480 product "
+    ap.add_argument("--no-large", action="store_true",
+                    help="skip the 10240^2 square-root leg (it builds a 10240 x 20480 product "
                          "on the host first)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the Shampoo-step, GEMM-count and single-block legs")
@@ -696,7 +791,7 @@ def main():
     import numpy as np
     import torch
 
-    from second_order_optimizer_shampoo_b200 import prism, synth
+    from second_order_optimizer_shampoo_b200 import _abi, prism, synth
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -714,8 +809,7 @@ def main():
     S_np = synth.sketch_stack(2 * MAX_ITER, N, P, SEED_S)
     A = torch.from_numpy(A_np).to(dev)
     S = torch.from_numpy(S_np).to(dev)
-    opts = prism.make_opts(d=D, p=P, tol=TOL, max_iter=MAX_ITER, prec="3xtf32")
-    from second_order_optimizer_shampoo_b200 import _abi
+    opts = prism.make_opts(d=D, p=P, tol=TOL, max_iter=MAX_ITER, prec=PREC)
     ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, N, N, BATCH, opts),
                      dtype=torch.uint8, device=dev)
     X = torch.empty_like(A)
@@ -757,12 +851,7 @@ def main():
                                                        launches, world)
     value = flops / (ms_max / 1e3) / 1e12
     precond_s = units / (ms_max / 1e3)
-
-    peaks, peak_src = load_peaks()
-    tf32_sust = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")) * TF32_OVER_BF16
-    split_peak = tf32_sust / 3.0  # three TF32 products per fp32-accurate product
-    # the GEMM timed alone below is a burst: its peak is the burst figure
-    split_peak_burst = peaks.get("bf16_tflops") * TF32_OVER_BF16 / 3.0
+    X_host_res = X.cpu().numpy()
 
     # ---- end to end through the public API with host buffers.  Every step
     # copies its input from pinned host memory and its result and statuses
@@ -818,50 +907,95 @@ def main():
     h2d = A_host.numel() * 4 + S_host.numel() * 4
     d2h = X_host[0].numel() * 4 + st_host[0].numel() * 4
     e2e_ok = bool(all(int((h.numpy() == 0).sum()) == BATCH for h in st_host))
+    del A2, S2, X2, rep2
 
-    # ---- roofline of the dominant kernel: the batched 3xTF32 tcgen05 GEMM,
-    # same launch configuration as inside the step (64 x 1024^3), timed alone
-    Yh, Yl = prism.shp_split_tf32(X)
-    Gh, Gl = prism.shp_split_tf32(A)
-    out = torch.empty_like(A)
+    peaks, peak_src = load_peaks()
+    tp = measure_tensor_peaks(dev)
+
+    # ---- roofline of the dominant kernel: k_gemm_oz in the step's launch
+    # shape (64 x 1024^3) and its in-step epilogue (C <- C + A B, fp64 read,
+    # combine, write, maxima), timed alone with the operands' slices reused
+    g = torch.Generator(device=dev).manual_seed(9)
+    Xa = torch.randn(BATCH, N, N, device=dev, dtype=torch.float64, generator=g)
+    Xb = torch.randn(BATCH, N, N, device=dev, dtype=torch.float64, generator=g)
+    Cc = torch.zeros_like(Xa)
+    mws = torch.empty(int(_abi.lib().shp_matmul_f64_workspace_bytes(N, N, N, BATCH)),
+                      dtype=torch.uint8, device=dev)
+    prism.shp_matmul_f64(Xa, Xb, out=Cc, ws=mws)
     for _ in range(3):
-        prism.shp_matmul(Yh, Gh, "3xtf32", A_lo=Yl, B_lo=Gl, out=out)
+        prism.shp_matmul_f64(Xa, Xb, out=Cc, ws=mws, reuse_a=True, reuse_b=True, accumulate=True)
     torch.cuda.synchronize()
-    reps = 40
+    reps = 20
     g0 = torch.cuda.Event(enable_timing=True)
     g1 = torch.cuda.Event(enable_timing=True)
     g0.record(stream)
     for _ in range(reps):
-        prism.shp_matmul(Yh, Gh, "3xtf32", A_lo=Yl, B_lo=Gl, out=out)
+        prism.shp_matmul_f64(Xa, Xb, out=Cc, ws=mws, reuse_a=True, reuse_b=True, accumulate=True)
     g1.record(stream)
     torch.cuda.synchronize()
     gemm_ms = g0.elapsed_time(g1) / reps
-    gemm_achieved = 2.0 * N ** 3 * BATCH / (gemm_ms / 1e3) / 1e12
+    del Xa, Xb, Cc, mws
+    torch.cuda.empty_cache()
+    int8_ops = OZ_PRODUCTS * 2.0 * N ** 3 * BATCH
+    int8_rate = int8_ops / (gemm_ms / 1e3) / 1e12
     step_ms = ms_max / args.steps
     roofline = {
-        "kernel": "k_gemm_pp<3xTF32> (persistent CTA pairs, batched 64 x 1024^3)",
-        "bound": "tensor", "achieved": gemm_achieved, "peak": split_peak_burst,
-        "unit": "TFLOP/s", "frac": gemm_achieved / split_peak_burst,
-        "traffic": GEMM_TRAFFIC_PER_LAUNCH, "traffic_unit": "bytes per launch",
-        "algorithmic_bytes": 5 * BATCH * N * N * 4,
-        "peak_note": f"{peak_src} burst BF16 x 1.1/2.25 (TF32) / 3 (3xTF32 products)",
-        "ms_per_launch": gemm_ms,
+        "kernel": "k_gemm_oz (Ozaki int8 x5, persistent CTA pairs, 64 x 1024^3, C += A B)",
+        "bound": "tensor", "achieved": int8_rate, "peak": tp["int8_tops"], "unit": "TOP/s int8",
+        "frac": int8_rate / tp["int8_tops"], "traffic": OZ_GEMM_TRAFFIC_PER_LAUNCH,
+        "traffic_unit": "bytes per launch",
+        "algorithmic_bytes": BATCH * N * N * (2 * OZ_SLICES + 16),
+        "peak_note": "measured here: best cuBLAS int8 8192^3 (burst)",
+        "ms_per_launch": gemm_ms, "fp64_equiv_tflops": 2.0 * N ** 3 * BATCH / (gemm_ms / 1e3) / 1e12,
         # the step's products at this kernel's rate, as a share of the step time
-        # (to set beside the kernel's share of the ncu launch list of the step)
-        "step_share_est": flops_step / (gemm_achieved * 1e12) / (step_ms / 1e3),
+        "step_share_est": flops_step / (2.0 * N ** 3 * BATCH / (gemm_ms / 1e3)) / (step_ms / 1e3),
     }
+
+    # ---- accuracy of the headline result and the fp32-storage paths
+    from oracle import prism_ref as o
+    acc_blocks = [b for b in ACC_BLOCKS if b < BATCH]
+    refs = {b: o.spd_power_eigh(A_np[b], -0.25) for b in acc_blocks}
+
+    def rel(x, r):
+        return float(np.linalg.norm(x - r) / np.linalg.norm(r))
+
+    acc = {"blocks": acc_blocks,
+           "ozaki_vs_eigh": [rel(X_host_res[b], refs[b]) for b in acc_blocks]}
+    fp32_paths = {}
+    if world == 1 and not args.no_extra:
+        for name, pr in (("split_3xtf32", "3xtf32"), ("tf32", "tf32")):
+            o3 = prism.make_opts(d=D, p=P, tol=TOL, max_iter=MAX_ITER, prec=pr)
+            ws3 = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, N, N, BATCH, o3),
+                              dtype=torch.uint8, device=dev)
+            X3 = torch.empty_like(A)
+            r3 = prism.make_report(BATCH, MAX_ITER, dev)
+            call = lambda: prism.matfn_inv_root(A, "inv4", o3, S, out=X3, ws=ws3, report=r3)  # noqa: E731
+            call()
+            torch.cuda.synchronize()
+            t3 = _time(call, stream, 5)
+            it3 = r3["iters"].cpu().numpy()
+            st3 = r3["status"].cpu().numpy()
+            X3h = X3.cpu().numpy()
+            errs = [rel(X3h[b], refs[b]) for b in acc_blocks]
+            fp32_paths[name] = {
+                "ms": t3, "tflops": float(sum(block_flops(k, N) for k in it3)) / (t3 / 1e3) / 1e12,
+                "ok_blocks": int((st3 == 0).sum()), "max_vs_eigh": max(errs) if np.all(np.isfinite(errs)) else None}
+            acc[name + "_vs_eigh"] = errs
+            del ws3, X3
+            torch.cuda.empty_cache()
 
     sketch_roof = sketch_leg(A, S[0], stream, peaks, peak_src)
 
-    polar = None if args.no_polar else polar_leg(args, dev, stream)
+    polar = None if args.no_polar else polar_leg(args, dev, stream, peaks)
     extra = not args.no_extra and world == 1
     step2 = shampoo_step_leg(args, dev, stream) if extra else None
     counts = gemm_count_leg(args, dev, stream, A) if extra else None
     single = single_block_leg(args, dev, stream) if extra else None
     sweep = sigma_sweep_leg(args, dev, stream) if extra else None
-    large = large_sqrt_leg(args, dev, stream) if args.large and world == 1 else None
+    tf32b = tf32_batched_leg(args, dev, stream, tp) if extra else None
     small = None if args.no_small else small_block_leg(args, dev, stream,
                                                         peaks.get("sm_max_mhz", 1965.0))
+    large = large_sqrt_leg(args, dev, stream) if extra and not args.no_large else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -878,35 +1012,60 @@ def main():
                "sample": f"{nb} of the {BATCH} blocks, float64 NumPy/LAPACK oracle (same recurrence)",
                "ms_per_block": 1e3 * t_tot / nb,
                "eigh_ms_per_block": 1e3 * eigh_sample(A_np[0])}
+        # the oracle's own distance from eigh on the reported blocks
+        oo = o.PrismOpts(d=D, p=P, lo=0.375, hi=1.0, tol=TOL, max_iter=MAX_ITER)
+        oxs = {b: o.inv_root_ref(A_np[b], o.POW_INV4, oo, S_np,
+                                 force_iters=iters[b])[0] for b in acc_blocks}
+        acc["oracle_vs_eigh"] = [rel(oxs[b], refs[b]) for b in acc_blocks]
+        acc["ozaki_vs_oracle"] = [rel(X_host_res[b], oxs[b]) for b in acc_blocks]
+
+    def r4(x):
+        if isinstance(x, float):
+            return float(f"{x:.4g}")
+        if isinstance(x, dict):
+            return {k: r4(v) for k, v in x.items()}
+        if isinstance(x, list):
+            return [r4(v) for v in x]
+        return x
 
     if rank == 0:
+        # the detailed legs first and the headline keys last: the end of the
+        # line is what a truncated log keeps
         line = {
+            "polar_sigma_sweep": sweep,
+            "gemms_to_residual": counts,
+            "single_64": single,
+            "small_blocks": small,
+            "shampoo_step_1024": step2,
+            "tf32_batched": tf32b,
+            "sqrt_10240": large,
+            "polar": polar,
+            "roofline_sketch": sketch_roof,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_max / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(world),
             "preconditioners_per_s": precond_s,
-            "frac_of_3xtf32_peak": value / (split_peak * world),
             "iters_per_pass": [int(x) for x in np.median(iters, axis=0)],
             "status_ok_blocks": int((status == 0).sum()), "blocks": int(len(status)),
             "gpu_launches": int(launches_all),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "status_ok": e2e_ok,
-                    "note": "two buffer sets; H2D of step i+1 and D2H of step i-1 overlap "
-                            "step i on their own streams"},
+                    "d2h_bytes_per_step": d2h, "status_ok": e2e_ok},
+            "peaks": tp,
+            "fp32_paths": fp32_paths,
+            "polar_tflops": polar["value"] if polar else None,
+            "polar_frac_bf16": polar["frac_of_bf16_peak"] if polar else None,
+            "sqrt10240_ms": large["prism_d2"]["ms"] if large else None,
+            "sqrt10240_gemms": {k: large[k]["gemms"] for k in ("prism_d2", "taylor_d2", "taylor_d1")} if large else None,
+            "tf32_1024_tflops": tf32b["value"] if tf32b else None,
+            "tf32_1024_frac": tf32b["frac_of_tf32_peak"] if tf32b else None,
+            "sketch_frac_hbm": sketch_roof["frac"],
+            "accuracy": acc,
             "roofline": roofline,
-            "roofline_sketch": sketch_roof,
-            "polar": polar,
-            "small_blocks": small,
-            "shampoo_step_1024": step2,
-            "gemms_to_residual": counts,
-            "single_64": single,
-            "polar_sigma_sweep": sweep,
-            "sqrt_10240": large,
-            "cpu_baseline": cpu,
-            "clocks": clocks,
         }
-        print(json.dumps(line))
+        print(json.dumps(r4(line), separators=(",", ":")))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -276,6 +276,21 @@ size_t shp_matmul_f64_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t b
 int shp_matmul_f64(const double* A, const double* B, double* C, int64_t M, int64_t N, int64_t K,
                    int64_t batch, void* ws, size_t ws_bytes, shp_stream stream);
 
+/* shp_matmul_f64 for an operand that does not change between calls: with
+ * SHP_MATMUL_REUSE_A (SHP_MATMUL_REUSE_B) the digit slices of A (B) are not
+ * formed again but taken from `ws` as the previous call with the same A (B),
+ * sizes and workspace left them (e.g. applying one fixed matrix to many
+ * right-hand sides); the product is then a single GEMM launch.  Reusing
+ * slices of an operand whose values changed gives the product with the old
+ * values.  With SHP_MATMUL_ACCUMULATE the product is added to C
+ * (C <- C + A B, in place).  flags = 0 is shp_matmul_f64. */
+#define SHP_MATMUL_REUSE_A 1
+#define SHP_MATMUL_REUSE_B 2
+#define SHP_MATMUL_ACCUMULATE 4
+int shp_matmul_f64_ex(const double* A, const double* B, double* C, int64_t M, int64_t N,
+                      int64_t K, int64_t batch, int flags, void* ws, size_t ws_bytes,
+                      shp_stream stream);
+
 /* hi = TF32(x) (round to nearest), lo = TF32(x - hi), for `count` floats. */
 int shp_split_tf32(const float* X, int64_t count, float* hi, float* lo, shp_stream stream);
 

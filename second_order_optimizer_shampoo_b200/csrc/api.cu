@@ -812,7 +812,15 @@ size_t shp_matmul_f64_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t b
 
 int shp_matmul_f64(const double* A, const double* B, double* C, int64_t M, int64_t N, int64_t K,
                    int64_t batch, void* ws, size_t ws_bytes, shp_stream stream) {
+  return shp_matmul_f64_ex(A, B, C, M, N, K, batch, 0, ws, ws_bytes, stream);
+}
+
+int shp_matmul_f64_ex(const double* A, const double* B, double* C, int64_t M, int64_t N,
+                      int64_t K, int64_t batch, int flags, void* ws, size_t ws_bytes,
+                      shp_stream stream) {
   if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || batch <= 0 || N % 2) return SHP_EINVAL;
+  if (flags & ~(SHP_MATMUL_REUSE_A | SHP_MATMUL_REUSE_B | SHP_MATMUL_ACCUMULATE))
+    return SHP_EINVAL;
   if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return SHP_EINVAL;
   if (M > INT32_MAX || N > INT32_MAX || K > 26000 || batch > 65535) return SHP_EUNSUPPORTED;
   if (ws == nullptr || ws_bytes < shp_matmul_f64_workspace_bytes(M, N, K, batch)) return SHP_EINVAL;
@@ -823,14 +831,22 @@ int shp_matmul_f64(const double* A, const double* B, double* C, int64_t M, int64
   unsigned* maxbuf = a.take<unsigned>(static_cast<size_t>(M + 2 * K + N) * batch);
   const int m = static_cast<int>(M), nc = static_cast<int>(N), k = static_cast<int>(K);
   const int bt = static_cast<int>(batch);
-  CK(oz_slice(A, m, k, K, M * K, bt, nullptr, maxbuf, false, sa, nullptr, st));
-  CK(oz_slice(B, k, nc, N, K * N, bt, nullptr, maxbuf + (M + K) * batch, false, sb, nullptr, st));
+  if (!(flags & SHP_MATMUL_REUSE_A))
+    CK(oz_slice(A, m, k, K, M * K, bt, nullptr, maxbuf, false, sa, nullptr, st));
+  if (!(flags & SHP_MATMUL_REUSE_B))
+    CK(oz_slice(B, k, nc, N, K * N, bt, nullptr, maxbuf + (M + K) * batch, false, sb, nullptr,
+                st));
   OzEpi e;
   memset(&e, 0, sizeof(e));
-  e.kind = EPI_STORE;
+  e.kind = (flags & SHP_MATMUL_ACCUMULATE) ? EPI_AXPY : EPI_STORE;
   e.out = C;
   e.ldo = N;
   e.bso = M * N;
+  if (flags & SHP_MATMUL_ACCUMULATE) {  // C <- C + A B, element by element in place
+    e.aux = C;
+    e.lda = N;
+    e.bsa = M * N;
+  }
   e.sa = sa.rscale;
   e.sb = sb.cscale;
   e.s0 = 1.f;

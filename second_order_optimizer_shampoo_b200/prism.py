@@ -285,18 +285,28 @@ def shp_matmul(Amat, B, prec="tf32", a_trans=False, b_trans=False, A_lo=None, B_
     return out
 
 
-def shp_matmul_f64(Amat, B, out=None, ws=None):
+def shp_matmul_f64(Amat, B, out=None, ws=None, reuse_a=False, reuse_b=False, accumulate=False):
     """Batched C = A B in fp64-grade arithmetic on the int8 tensor cores (the
-    Ozaki scheme); A [batch][M][K], B [batch][K][N] float64."""
+    Ozaki scheme); A [batch][M][K], B [batch][K][N] float64.  reuse_a /
+    reuse_b take that operand's digit slices from `ws` as the previous call
+    with the same operand and workspace left them; accumulate adds the
+    product to `out` (which must then be given)."""
     _dev(Amat, B, out)
     if Amat.dtype != torch.float64 or B.dtype != torch.float64:
         raise ValueError("shp_matmul_f64 takes float64 tensors")
     M, K = Amat.shape[-2], Amat.shape[-1]
     N = B.shape[-1]
     batch = Amat.numel() // (M * K)
+    if accumulate and out is None:
+        raise ValueError("accumulate needs out")
     out = torch.empty(batch, M, N, dtype=torch.float64, device=Amat.device) if out is None else out
     need = int(A.lib().shp_matmul_f64_workspace_bytes(M, N, K, batch))
-    ws = _ws(need, Amat.device) if ws is None else ws
-    _check(A.lib().shp_matmul_f64(_p(Amat), _p(B), _p(out), M, N, K, batch, _p(ws), ws.numel(),
-                                  _stream()), "shp_matmul_f64")
+    if ws is None:
+        if reuse_a or reuse_b:
+            raise ValueError("reusing slices needs the workspace of the previous call")
+        ws = _ws(need, Amat.device)
+    flags = ((A.SHP_MATMUL_REUSE_A if reuse_a else 0) | (A.SHP_MATMUL_REUSE_B if reuse_b else 0)
+             | (A.SHP_MATMUL_ACCUMULATE if accumulate else 0))
+    _check(A.lib().shp_matmul_f64_ex(_p(Amat), _p(B), _p(out), M, N, K, batch, flags, _p(ws),
+                                     ws.numel(), _stream()), "shp_matmul_f64")
     return out

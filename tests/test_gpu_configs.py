@@ -1,6 +1,8 @@
 """The five workloads at their full sizes, in the launch configuration the
 benchmark uses, checked on outputs the oracle can compute (sampled blocks) or
 on properties that hold at any size."""
+import functools
+
 import numpy as np
 import pytest
 
@@ -59,49 +61,44 @@ def test_config2_shampoo_step():
     assert relerr(dW, dW_ref) <= 1e-3
 
 
-def subspace_err(X, A, frac=1e-2):
-    """Relative error of X against A^(-1/4) restricted to the eigenvectors
-    with lambda >= frac * lambda_max (components TF32/fp32 products keep)."""
-    w, Q = np.linalg.eigh(A.astype(np.float64))
-    Xe = (Q * w ** -0.25) @ Q.T
-    Pk = Q[:, w >= frac * w.max()]
-    return relerr(X @ Pk, Xe @ Pk), relerr(X, Xe)
+# Config 3 runs on the fp64-grade path (SHP_OZAKI).  TF32 and the 3xTF32
+# split keep fp32 iterates, and at cond 1e6 that is far from enough: rounding
+# B = A / ||A||_F to TF32 makes the blocks indefinite (the iteration
+# diverges), and the 3xTF32 split ends 3.5e-2 .. 4.1e-2 from eigh.  The
+# tolerance that applies is the split-precision one, 1e-5, against the
+# same-recurrence oracle.  Against eigh the method itself, stopped at the
+# config's residual 1e-3 per pass, ends 3e-6 .. 1.7e-5 away (float64 oracle,
+# all 64 blocks), so there the bound is the oracle's own distance plus 1e-5.
+TOL_SPLIT = 1e-5
+SAMPLED = (0, 1, 5, 32, 37, 63)  # includes the blocks where the oracle is farthest from eigh
 
 
 def test_config3_batched_inverse_root():
-    """64 SPD blocks 1024^2, cond 1e6, d = 2, p = 8, tol 1e-3 per pass, split
-    path (TF32 rounding of A/||A|| makes these blocks indefinite).  Sampled
-    blocks against the oracle; alpha parity on identical residuals."""
+    """64 SPD blocks 1024^2, lambda log-uniform on [1e-6, 1] (cond 1e6),
+    A^(-1/4), d = 2, p = 8, tol 1e-3 per pass, in the bench's launch
+    configuration.  Sampled blocks: the result and the alpha trajectories
+    against the float64 oracle run with the GPU's iteration counts, the
+    result against eigh, and the free-running oracle's iteration counts."""
     P = prism()
     n, batch = 1024, 64
     A = synth.spd_batch(n, batch, 1e-6, 1.0, 103)
     S = synth.sketch_stack(48, n, 8, 1003)
-    opts = P.make_opts(d=2, p=8, tol=1e-3, max_iter=24, prec="3xtf32")
+    opts = P.make_opts(d=2, p=8, tol=1e-3, max_iter=24, prec="ozaki")
     X, rep = P.matfn_inv_root(to_dev(torch, A), "inv4", opts, to_dev(torch, S))
     X, rep = to_host(X), {k: to_host(v) for k, v in rep.items()}
     assert np.all(rep["status"] == o.OK), rep["status"]
-    assert np.all(rep["resid"][np.arange(batch), 0, rep["iters"][:, 0]] <= 1e-3)
-    for b in (0, 1, batch // 2, batch - 1):
+    for ps in range(2):
+        assert np.all(rep["resid"][np.arange(batch), ps, rep["iters"][:, ps]] <= 1e-3)
+    for b in SAMPLED:
+        it = rep["iters"][b]
+        Xo, infos = o.inv_root_ref(A[b], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
+        for ps, info in enumerate(infos):
+            np.testing.assert_allclose(rep["alpha"][b, ps, :it[ps]], info.alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= TOL_SPLIT, b
+        ref = o.spd_power_eigh(A[b], -0.25)
+        assert relerr(X[b], ref) <= relerr(Xo, ref) + TOL_SPLIT, b
         _, free = o.inv_root_ref(A[b], o.POW_INV4, oracle_opts(opts), S)
-        assert all(abs(f.iters - int(g)) <= 1 for f, g in zip(free, rep["iters"][b]))
-        sub, full = subspace_err(X[b], A[b])
-        assert sub <= 1e-3, (b, sub, full)
-        assert full <= 1e-1, (b, sub, full)
-    # alpha on identical residuals: the oracle's R_k of block 0, rounded to fp32
-    B0 = A[0].astype(np.float64) / np.linalg.norm(A[0].astype(np.float64))
-    Y, Z = B0.copy(), np.eye(n)
-    Rs, Ss = [], []
-    for k in range(4):
-        Rk = np.eye(n) - Z @ Y
-        Rs.append(Rk.astype(np.float32))
-        Ss.append(S[k])
-        a, _ = o.prism_alpha_ref(Rk, S[k], 2, 0.375, 1.0)
-        g = o.matrix_poly(o.g_coeffs(2, a), Rk)
-        Y, Z = Y @ g, g @ Z
-    for Rk, Sk in zip(Rs, Ss):
-        ag, _ = P.prism_alpha_fit(to_dev(torch, Rk[None]), to_dev(torch, Sk), 2, 0.375, 1.0)
-        ar, _ = o.prism_alpha_ref(Rk, Sk, 2, 0.375, 1.0)
-        assert abs(float(to_host(ag)[0]) - ar) <= 1e-4
+        assert all(abs(f.iters - int(g)) <= 1 for f, g in zip(free, it))
 
 
 def test_config4_polar_bf16():
@@ -134,41 +131,41 @@ def test_config4_polar_bf16():
         assert abs(float(to_host(ag)[0]) - ar) <= 1e-4
 
 
-# The tensor cores add into their fp32 accumulator with truncation: measured on
-# all-positive products, one fp32-grade (3xTF32) product of length K is biased
-# by about -(K/8) 2^-25 (the hi*hi accumulator takes K/8 truncating additions).
-# At K = 10240 that is 3.8e-5, so the split path's bound on the full-size
-# square root is 1e-4 (the 1e-5 target holds at n = 1024, where K/8 2^-25 =
-# 3.8e-6).
+# Config 5 names the 3xTF32 split; at n = 10240 that path's accumulation
+# (the tensor cores add into fp32 with truncation: about -(K/8) 2^-25 of bias
+# per product, 3.8e-5 at K = 10240) keeps it from 1e-5, so the 1e-5 target is
+# checked on the fp64-grade path (SHP_OZAKI), and the 3xTF32 path is held to
+# the bound its accumulation allows (an unmet target of that path).
 TOL_3X_K10240 = 1e-4
 
 
-@pytest.mark.parametrize("n,samples", [(1024, 2048), (10240, 20480)])
-def test_config5_square_root(n, samples):
-    """A = X X^T / samples + 1e-4 I (Marchenko-Pastur, ratio 1/2), A^(1/2) by
-    d = 2, p = 16, split path, tol 1e-6.  At n = 1024 the whole result is
-    compared with eigh (1e-5); at n = 10240 sampled entries of X X against A
-    and the symmetry of X, within the bound the accumulation allows there."""
-    P = prism()
+@functools.lru_cache(maxsize=1)
+def config5_input(n, samples):
+    """The Marchenko-Pastur input and its float64 square root by eigh (both
+    built once per size: at n = 10240 that is a few minutes of host work)."""
     A = synth.mp_spd(n, samples, 1e-4, 105)
+    return A, o.spd_power_eigh(A, 0.5)
+
+
+@pytest.mark.parametrize("prec", ["ozaki", "3xtf32"])
+@pytest.mark.parametrize("n,samples", [(1024, 2048), (10240, 20480)])
+def test_config5_square_root(n, samples, prec):
+    """A = X X^T / samples + 1e-4 I (Marchenko-Pastur, ratio 1/2), A^(1/2) by
+    d = 2, p = 16, tol 1e-6: the whole result against the float64
+    eigendecomposition (at n = 10240 too) and, at n = 1024, against the
+    same-recurrence oracle."""
+    P = prism()
+    A, root = config5_input(n, samples)
     S = synth.sketch_stack(40, n, 16, 1005)
-    opts = P.make_opts(d=2, p=16, tol=1e-6, max_iter=40, prec="3xtf32")
+    opts = P.make_opts(d=2, p=16, tol=1e-6, max_iter=40, prec=prec)
     Xd, rep = P.matfn_inv_root(to_dev(torch, A[None]), "sqrt", opts, to_dev(torch, S))
     rep = {k: to_host(v) for k, v in rep.items()}
     assert rep["status"][0] in (o.OK, o.ESTALL), rep
     X = to_host(Xd)[0].astype(np.float64)
+    del Xd
+    tol = TOL_SPLIT if (prec == "ozaki" or n <= 2048) else TOL_3X_K10240
+    assert relerr(X, root) <= tol
     if n <= 2048:
-        assert relerr(X, o.spd_power_eigh(A, 0.5)) <= 1e-5
-        Xo, infos = o.inv_root_ref(A, o.POW_SQRT, oracle_opts(opts), S,
-                                   force_iters=rep["iters"][0][:1])
-        assert relerr(X, Xo) <= 1e-5
-        return
-    rng = np.random.default_rng(0)
-    I = rng.integers(0, n, 64)
-    J = rng.integers(0, n, 64)
-    A64 = A.astype(np.float64)
-    XX = np.einsum("ik,ki->i", X[I, :], X[:, J])
-    scale = np.einsum("ik,ki->i", np.abs(X[I, :]), np.abs(X[:, J]))
-    # |X^2 - A| <= 2 delta |X||X| for a relative error delta of X
-    assert np.all(np.abs(XX - A64[I, J]) <= 2 * TOL_3X_K10240 * scale + 1e-7)
-    assert relerr(X[I], X[:, I].T) <= TOL_3X_K10240   # the true root is symmetric
+        Xo, _ = o.inv_root_ref(A, o.POW_SQRT, oracle_opts(opts), S,
+                               force_iters=rep["iters"][0][:1])
+        assert relerr(X, Xo) <= tol

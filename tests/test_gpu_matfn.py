@@ -36,19 +36,27 @@ def oracle_opts(opts, **kw):
     return o.PrismOpts(**base)
 
 
-# 3xTF32 keeps about 21 bits per product (both parts rounded to 11-bit TF32,
-# the lo*lo term dropped) against fp32's 24: its rounding is 2^3 = 8 times
-# fp32's.  Emulated fp32 arithmetic reaches 1.4e-6 .. 3.6e-6 relative error on
-# the config-1 spectrum (cond 1e3), so the split path's bound there is
-# 8 x 3.6e-6 ~ 3e-5.  Milder spectra stay within 1e-5.
+# Tolerances.  The split-precision target is 1e-5 (relative Frobenius error
+# against eigh and against the same-recurrence oracle).
+#   - SHP_OZAKI (fp64 iterates, Ozaki products of about 2^-40) meets it on
+#     every spectrum tested, cond 1e6 included: TOL_SPLIT.
+#   - The on-chip small-block path computes every product in fp32 FMA (a few
+#     u_fp32 = 6e-8 per step, amplified by cond(A)^(1/4) ~ 6 at cond 1e3):
+#     TOL_SPLIT as well.
+#   - The 3xTF32 split keeps the iterates in fp32 and adds into the tensor
+#     core's truncating fp32 accumulator: at cond 1e3 it ends 8e-6 .. 1.7e-5
+#     from eigh, so it is held to TOL_3X_COND1E3 = 3e-5 and misses the 1e-5
+#     target there (an unmet target of that path, met by SHP_OZAKI).
+TOL_SPLIT = 1e-5
 TOL_3X_COND1E3 = 3e-5
 
 
 @pytest.mark.parametrize("seed", range(4))
-def test_inv_root_config1_split(seed):
-    """64 x 64 SPD, lambda log-uniform on [1e-3, 1], A^(-1/4), d = 1, p = 4,
-    alpha in [1/2, 1], 3xTF32: relative error vs eigh within the split path's
-    bound, alpha trajectory within 1e-4 of the oracle's on the same sketch."""
+def test_inv_root_config1_onchip(seed):
+    """Config 1 as stated: 64 x 64 SPD, lambda log-uniform on [1e-3, 1],
+    A^(-1/4), d = 1, p = 4, alpha in [1/2, 1].  n <= 64 runs the on-chip
+    kernel (fp32 products): relative error vs eigh and vs the same-recurrence
+    oracle within 1e-5, alpha trajectory within 1e-4 of the oracle's."""
     n = 64
     A = synth.spd_batch(n, 1, 1e-3, 1.0, 101, indices=[seed])
     S = synth.sketch_stack(80, n, 4, 1001)
@@ -58,12 +66,32 @@ def test_inv_root_config1_split(seed):
     Xo, infos = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
     for ps in range(2):
         np.testing.assert_allclose(rep["alpha"][0, ps, :it[ps]], infos[ps].alpha, atol=1e-4)
-    assert relerr(X[0], o.spd_power_eigh(A[0], -0.25)) <= TOL_3X_COND1E3
-    assert relerr(X[0], Xo) <= TOL_3X_COND1E3
+    assert relerr(X[0], o.spd_power_eigh(A[0], -0.25)) <= TOL_SPLIT
+    assert relerr(X[0], Xo) <= TOL_SPLIT
     # the oracle left to its own stopping rule takes the same number of steps,
     # give or take the one step whose residual sits at the tolerance
     _, free = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S)
     assert all(abs(a - int(b)) <= 1 for a, b in zip([i.iters for i in free], it))
+
+
+@pytest.mark.parametrize("prec,tol", [("3xtf32", TOL_3X_COND1E3), ("ozaki", TOL_SPLIT)])
+@pytest.mark.parametrize("seed", range(2))
+def test_inv_root_config1_spectrum_tensor_cores(seed, prec, tol):
+    """The config-1 spectrum (cond 1e3, d = 1, p = 4) at n = 128, which takes
+    the batched tensor-core path: the 3xTF32 split within its own bound, the
+    Ozaki path within the 1e-5 split target; both against eigh and the
+    same-recurrence oracle, alpha within 1e-4."""
+    n = 128
+    A = synth.spd_batch(n, 1, 1e-3, 1.0, 131, indices=[seed])
+    S = synth.sketch_stack(80, n, 4, 1031)
+    X, rep, opts = run_inv_root(A, "inv4", 1, 4, 1e-6, 40, prec, S)
+    assert rep["status"][0] in (o.OK, o.ESTALL)
+    it = rep["iters"][0]
+    Xo, infos = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
+    for ps in range(2):
+        np.testing.assert_allclose(rep["alpha"][0, ps, :it[ps]], infos[ps].alpha, atol=1e-4)
+    assert relerr(X[0], o.spd_power_eigh(A[0], -0.25)) <= tol
+    assert relerr(X[0], Xo) <= tol
 
 
 @pytest.mark.parametrize("power", ["inv4", "inv2", "sqrt"])
@@ -146,7 +174,7 @@ def test_taylor_baseline_and_gemm_count():
     assert rt["status"][0] == o.OK
     np.testing.assert_array_equal(rt["alpha"][0, 0, :rt["iters"][0][0]], 0.5)
     Xo, _ = o.inv_root_ref(A[0], o.POW_INV4, oracle_opts(ot), None, force_iters=rt["iters"][0])
-    assert relerr(Xt[0], Xo) <= TOL_3X_COND1E3
+    assert relerr(Xt[0], Xo) <= TOL_SPLIT  # n = 64: the on-chip fp32 path
     Xp, rp, _ = run_inv_root(A, "inv4", 1, 4, 1e-6, 40, "3xtf32", S)
     taylor, prism_steps = rt["iters"][0].sum(), rp["iters"][0].sum()
     assert prism_steps < taylor, (prism_steps, taylor)

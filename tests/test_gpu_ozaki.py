@@ -156,3 +156,24 @@ def test_inv_root_ozaki_nan_block_isolated(power):
     for b in (0, 2):
         assert rep["status"][b] in (o.OK, o.ESTALL)
         assert relerr(X[b], o.spd_power_eigh(A[b], q)) <= 1e-5
+
+
+def test_matmul_f64_reuse_and_accumulate():
+    """Slices of a fixed left operand reused against a new right operand, and
+    C <- C + A B in place: both as the plain call gives them."""
+    P = prism()
+    rng = np.random.default_rng(11)
+    batch, M, N, K = 2, 160, 96, 200
+    A = to_dev(torch, rng.standard_normal((batch, M, K)))
+    B1 = to_dev(torch, rng.standard_normal((batch, K, N)))
+    B2 = to_dev(torch, rng.standard_normal((batch, K, N)))
+    C0 = to_dev(torch, rng.standard_normal((batch, M, N)))
+    ws = torch.empty(int(P.A.lib().shp_matmul_f64_workspace_bytes(M, N, K, batch)),
+                     dtype=torch.uint8, device="cuda")
+    ref1 = to_host(P.shp_matmul_f64(A, B1, ws=ws))
+    ref2 = to_host(P.shp_matmul_f64(A, B2))
+    got2 = to_host(P.shp_matmul_f64(A, B2, ws=ws, reuse_a=True))  # A's slices from the first call
+    np.testing.assert_array_equal(got2, ref2)
+    C = C0.clone()
+    P.shp_matmul_f64(A, B1, out=C, ws=ws, accumulate=True)
+    np.testing.assert_allclose(to_host(C), to_host(C0) + ref1, rtol=0, atol=1e-13 * np.abs(ref1).max())
