@@ -87,7 +87,10 @@ typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_
  *   max_iter    at most this many update steps per pass (<= 256)
  *   prec        SHP_TF32 / SHP_3XTF32 / SHP_OZAKI (inverse roots); SHP_BF16
  *               only for polar storage
- *   fixed_alpha 1: alpha = lo every step (plain Taylor Newton-Schulz)
+ *   fixed_alpha 1: alpha = lo every step (plain Taylor Newton-Schulz; with
+ *               d = 2 and lo = 3/8 this is Chebyshev's third-order method for
+ *               the inverse square root, which PRISM accelerates by fitting
+ *               alpha instead)
  *   stall_below, stall_ratio: stop with SHP_ESTALL when the previous residual
  *               is below stall_below and the new one exceeds stall_ratio times it
  *   adaptive_degree 1: every pass starts at degree 1 and raises to d (= 2) for
@@ -327,6 +330,31 @@ uint64_t shp_kernel_launches(void);
 int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const float* S, int p,
                             int d, float lo, float hi, float* alpha_out, double* J_coef_out,
                             shp_stream stream);
+
+/* ---- Self-test of the bounded waits (no counterpart on the pages). ----
+ * Every pipeline wait inside the kernels is bounded: a wait that runs out
+ * records SHP_ETIMEOUT, the other roles of the CTA give up at their next
+ * wait, the copies and tensor-core operations already issued are waited for,
+ * tensor memory is freed, and the stream stays usable.  This call makes one
+ * such wait run out on purpose, by pointing it at a barrier nothing completes
+ * (limit about 10 ms), in one small launch of the kernel `which` selects:
+ *   SHP_SELFTEST_GEMM    persistent CTA-pair GEMM: the producer's first wait
+ *                        (nothing issued yet)
+ *   SHP_SELFTEST_OZAKI   Ozaki-scheme GEMM: the same wait
+ *   SHP_SELFTEST_SKETCH  TMA sketch: the consumers' first V hand-over, with
+ *                        the producer's copies in flight (they are drained),
+ *                        in the first pass of a whole alpha fit (d = 1)
+ * status: one device int32, set to SHP_ETIMEOUT by the kernel (cleared
+ * first).  alpha_out: one device float (may be NULL), for SHP_SELFTEST_SKETCH
+ * the fit's alpha, which must come out NaN (no fit on incomplete vectors).
+ * ws: at least SHP_SELFTEST_WS_BYTES of device scratch, 256-byte aligned
+ * (zeroed by the call).  Returns SHP_OK once launched. */
+#define SHP_SELFTEST_GEMM 0
+#define SHP_SELFTEST_OZAKI 1
+#define SHP_SELFTEST_SKETCH 2
+#define SHP_SELFTEST_WS_BYTES (4u << 20)
+int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void* ws,
+                              size_t ws_bytes, shp_stream stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* shp_status_string(int status);

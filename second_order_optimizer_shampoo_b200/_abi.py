@@ -23,6 +23,9 @@ SHP_POW_INV4, SHP_POW_INV2, SHP_POW_SQRT = 0, 1, 2
 SHP_OP_INV_ROOT, SHP_OP_POLAR, SHP_OP_ALPHA_FIT, SHP_OP_APPLY, SHP_OP_GRAM_EMA = 0, 1, 2, 3, 4
 # shp_matmul_f64_ex flags
 SHP_MATMUL_REUSE_A, SHP_MATMUL_REUSE_B, SHP_MATMUL_ACCUMULATE = 1, 2, 4
+# bounded-wait self-test
+SHP_SELFTEST_GEMM, SHP_SELFTEST_OZAKI, SHP_SELFTEST_SKETCH = 0, 1, 2
+SHP_SELFTEST_WS_BYTES = 4 << 20
 # fixed device scratch of prism_alpha_fit_noalloc
 SHP_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -30,7 +33,7 @@ EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_p
            "matfn_sign",
            "prism_alpha_fit", "shampoo_apply", "shampoo_apply_ex", "shp_matmul", "shp_split_tf32",
            "shp_matmul_f64_workspace_bytes", "shp_matmul_f64", "shp_matmul_f64_ex",
-           "shp_kernel_launches", "prism_alpha_fit_noalloc", "shp_status_string", "shp_last_cuda_error",
+           "shp_kernel_launches", "prism_alpha_fit_noalloc", "shp_selftest_bounded_wait", "shp_status_string", "shp_last_cuda_error",
            "shp_version")
 
 
@@ -79,6 +82,7 @@ _SIGS = {
     "shp_matmul_f64_ex": (_INT, [_P, _P, _P, _I64, _I64, _I64, _I64, _INT, _P, _SZ, _P]),
     "shp_kernel_launches": (ctypes.c_uint64, []),
     "prism_alpha_fit_noalloc": (_INT, [_P, _I64, _I64, _P, _INT, _INT, _F, _F, _P, _P, _P]),
+    "shp_selftest_bounded_wait": (_INT, [_INT, _P, _P, _P, _SZ, _P]),
     "shp_status_string": (ctypes.c_char_p, [_INT]),
     "shp_last_cuda_error": (ctypes.c_char_p, []),
     "shp_version": (ctypes.c_char_p, []),

@@ -801,6 +801,61 @@ int inv_root_oz(const float* A, int64_t n, int64_t batch, int power, const shp_p
 
 extern "C" {
 
+int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void* ws,
+                              size_t ws_bytes, shp_stream stream) {
+  if (status == nullptr || ws == nullptr || ws_bytes < SHP_SELFTEST_WS_BYTES) return SHP_EINVAL;
+  if (which != SHP_SELFTEST_GEMM && which != SHP_SELFTEST_OZAKI && which != SHP_SELFTEST_SKETCH)
+    return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  CK(cudaMemsetAsync(ws, 0, SHP_SELFTEST_WS_BYTES, st));
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  constexpr int n = 256, p = 8;  // one 256 x 256 product (a single CTA-pair tile)
+  if (which == SHP_SELFTEST_GEMM) {
+    float* A = a.take<float>(n * n);
+    float* B = a.take<float>(n * n);
+    float* C = a.take<float>(n * n);
+    EpiParams e = epi(EPI_STORE, OUT_F32, C, nullptr, n, n * n, n, n, nullptr);
+    e.status = status;
+    e.selftest = 1;
+    CK(gemm_tc(MODE_TF32, op(A, nullptr, false, n, n * n), op(B, nullptr, true, n, n * n), n, n,
+               n, 1, e, st));
+  } else if (which == SHP_SELFTEST_OZAKI) {
+    const OzSlices sa = carve_slices(a, n, n, 1, true, false);
+    const OzSlices sb = carve_slices(a, n, n, 1, false, true);
+    double* C = a.take<double>(n * n);
+    OzEpi e;
+    memset(&e, 0, sizeof(e));
+    e.kind = EPI_STORE;
+    e.out = C;
+    e.ldo = n;
+    e.bso = n * n;
+    e.sa = sa.rscale;
+    e.sb = sb.cscale;
+    e.s0 = 1.f;
+    e.M = n;
+    e.N = n;
+    e.status = status;
+    e.selftest = 1;
+    CK(gemm_oz(sa.rows, sb.cols, n, n, n, 1, e, st));
+  } else {  // the alpha fit of one block (d = 1) whose first sketch pass times out
+    float* R = a.take<float>(n * n);
+    float* S = a.take<float>(n * p);
+    float* V = a.take<float>(4 * n * p);
+    float* alpha = alpha_out != nullptr ? alpha_out : a.take<float>(1);
+    const int64_t np = static_cast<int64_t>(n) * p;
+    CK(sketch_pass(R, nullptr, n, n * n, S, 0, V + np, 4 * np, p, 1, nullptr, nullptr, 0, st,
+                   status, 1));
+    for (int j = 2; j <= 3; ++j)
+      CK(sketch_pass(R, nullptr, n, n * n, V + (j - 1) * np, 4 * np, V + j * np, 4 * np, p, 1,
+                     nullptr, nullptr, 0, st, status));
+    CK(alpha_solve(V, n, p, 1, 1, 0.5f, 1.f, 0, nullptr, alpha, nullptr, nullptr, 0, 0, nullptr,
+                   st, nullptr, status));
+  }
+  if (a.used > SHP_SELFTEST_WS_BYTES - kAlign) return SHP_EUNSUPPORTED;  // cannot happen
+  return SHP_OK;
+}
+
 size_t shp_matmul_f64_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch) {
   if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return 0;
   Arena a(nullptr);

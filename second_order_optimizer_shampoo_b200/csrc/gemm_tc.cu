@@ -542,8 +542,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* accf = empty + C::PP_STAGES;
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;  // all MMAs of this pair complete (before TMEM is freed)
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+  uint64_t* never = drain + 1;  // completed by nothing: the self-test's wait
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(never + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -556,6 +557,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&acce[u], 16);
     }
     mbar_init(drain, 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tA);
@@ -579,6 +581,13 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t tx = (C::A_BYTES + 128u * C::ROWB) * (C::SPLIT ? 2u : 1u) * 2u;
       int kit = 0;
       bool stop = false;
+      // bounded-wait self-test: before any copy is issued, wait on a barrier
+      // nothing completes; it runs out, and the CTA unwinds with nothing in flight
+      if (ep.selftest && !mbar_wait(never, 0, nullptr, SHP_SELFTEST_LIMIT)) {
+        *abort_flag = 1;
+        if (ep.status != nullptr) atomicExch(&ep.status[0], ST_ETIMEOUT);
+        stop = true;
+      }
       for (int t = cl; t < ntiles && !stop; t += ncl) {
         const int b = t / per_b, r = t % per_b;
         if (ep.active != nullptr && ep.active[b] == 0) continue;
@@ -589,7 +598,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int kb = 0; kb < KB; ++kb, ++kit) {
           const int s = kit % C::PP_STAGES;
           if (kit >= C::PP_STAGES &&
-              (*abort_flag || !mbar_wait(&empty[s], ((kit / C::PP_STAGES) - 1) & 1))) {
+              (*abort_flag || !mbar_wait(&empty[s], ((kit / C::PP_STAGES) - 1) & 1, abort_flag))) {
             *abort_flag = 1;
             if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
             stop = true;
@@ -632,7 +641,7 @@ __global__ void __launch_bounds__(320, 1)
         const int b = t / per_b;
         if (ep.active != nullptr && ep.active[b] == 0) continue;
         const int u = tl & 1, use = tl >> 1;
-        if (use >= 1 && (*abort_flag || !mbar_wait(&acce[u], (use - 1) & 1))) {
+        if (use >= 1 && (*abort_flag || !mbar_wait(&acce[u], (use - 1) & 1, abort_flag))) {
           *abort_flag = 1;
           if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
           break;
@@ -641,7 +650,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t dacc = tmem + static_cast<uint32_t>(u * BN);
         for (int kb = 0; kb < KB; ++kb, ++kit) {
           const int s = kit % C::PP_STAGES;
-          if (*abort_flag || !mbar_wait(&full[s], (kit / C::PP_STAGES) & 1)) {
+          if (*abort_flag || !mbar_wait(&full[s], (kit / C::PP_STAGES) & 1, abort_flag)) {
             *abort_flag = 1;
             if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
             stop = true;
@@ -688,7 +697,7 @@ __global__ void __launch_bounds__(320, 1)
       const int b = t / per_b, r = t % per_b;
       if (ep.active != nullptr && ep.active[b] == 0) continue;
       const int u = tl & 1, use = tl >> 1;
-      if (*abort_flag || !mbar_wait(&accf[u], use & 1)) {
+      if (*abort_flag || !mbar_wait(&accf[u], use & 1, abort_flag)) {
         *abort_flag = 1;
         if (lane == 0 && ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
         break;
@@ -850,17 +859,20 @@ cudaError_t dispatch_pair(bool pair, bool amn, bool bmn, const CUtensorMap& a,
 }  // namespace
 
 bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t rows, int slices,
-                       int64_t blocks, int box_rows) {
+                       int64_t blocks, int kb_bytes, int box_rows) {
   auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices),
+  if (fn == nullptr || (kb_bytes != 64 && kb_bytes != 128)) return false;
+  const cuuint64_t kb = static_cast<cuuint64_t>(kb_bytes);
+  cuuint64_t dims[4] = {kb, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices),
                         static_cast<cuuint64_t>(blocks)};
-  cuuint64_t strides[3] = {64, static_cast<cuuint64_t>(rows * 64),
-                           static_cast<cuuint64_t>(slices * rows * 64)};
-  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(slices), 1};
+  cuuint64_t strides[3] = {kb, static_cast<cuuint64_t>(rows) * kb,
+                           static_cast<cuuint64_t>(slices) * rows * kb};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(kb_bytes), static_cast<cuuint32_t>(box_rows),
+                       static_cast<cuuint32_t>(slices), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<int8_t*>(ptr), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  kb_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

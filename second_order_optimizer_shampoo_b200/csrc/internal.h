@@ -92,6 +92,9 @@ struct EpiParams {
   // out2 and out_plain); other kernels compute it all.  Read-modify-write and
   // aux operands are read on the upper tiles only, so they must be symmetric.
   int sym;
+  // bounded-wait self-test (persistent kernel): the producer first waits on a
+  // barrier nothing completes; status[0] receives ST_ETIMEOUT
+  int selftest;
 };
 
 // C[b] (M x N) = A[b] (M x K) * B[b] (K x N) on tcgen05 tensor cores,
@@ -105,22 +108,24 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
 bool tensor_map_rows(CUtensorMap* m, const float* ptr, int64_t inner, int64_t rows,
                      int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_rows);
 
-// 4-D int8 map over [blocks][slices][rows][64] (the K-blocked digit slices of
-// the Ozaki-scheme products, ozaki.cu) with a box of all slices x box_rows x
-// 64 bytes and the 64-byte swizzle, zero fill past `rows`.
+// 4-D int8 map over [blocks][slices][rows][kb_bytes] (the K-blocked digit
+// slices of the Ozaki-scheme products, ozaki.cu; kb_bytes 64 or 128) with a
+// box of all slices x box_rows x kb_bytes and the swizzle of that row
+// length, zero fill past `rows`.
 bool tensor_map_slices(CUtensorMap* m, const int8_t* ptr, int64_t rows, int slices,
-                       int64_t blocks, int box_rows);
+                       int64_t blocks, int kb_bytes, int box_rows);
 
 // ---- PRISM sketch and alpha (sketch_alpha.cu)
 // Vout[b] = R[b] * Vin[b]; R is n x n (hi + lo when lo != null); V is n x p.
 // vin_bstride == 0 shares Vin across the batch.  When `it` is non-null the
 // input is Vin + (*it) * it_stride (the sketch slice of the current iteration).
 // A pipeline wait of the bulk-copy variant that runs out sets tmo[b] (if
-// non-null) to ST_ETIMEOUT.
+// non-null) to ST_ETIMEOUT.  selftest (bulk-copy variant only): the first V
+// hand-over waits on a barrier nothing completes, so that wait runs out.
 cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
                         const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
                         int p, int batch, const int* active, const int* it, int64_t it_stride,
-                        cudaStream_t st, int* tmo = nullptr);
+                        cudaStream_t st, int* tmo = nullptr, int selftest = 0);
 // V is stored per block as [2d+2][n][p] (slot j holds V_j; slot 0 unused).
 // Gram of V_d..V_{2d+1}, the
 // quartic J(alpha) and its minimiser on [lo, hi]; writes alpha[b] and, when
@@ -286,6 +291,7 @@ struct OzEpi {
   unsigned* cmax;
   unsigned* rmax2;
   unsigned* cmax2;
+  int selftest;  // as EpiParams::selftest
 };
 int64_t oz_ldk(int64_t k);                                     // K padded to whole blocks
 size_t oz_slices_bytes(int64_t rows, int64_t k, int64_t batch);  // one slicing's digits

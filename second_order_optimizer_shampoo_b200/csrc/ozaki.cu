@@ -49,9 +49,16 @@ namespace {
 
 constexpr int OZ_S = 5;                              // digit slices per operand
 constexpr int OZ_BN = 96;                            // tile columns (pair tile 256 x 96)
-constexpr int OZ_BK = 64;                            // K bytes per stage
+#ifndef OZ_KB_BYTES
+#define OZ_KB_BYTES 64
+#endif
+constexpr int OZ_BK = OZ_KB_BYTES;                   // K bytes per stage = per slice K block
+// the shared-memory swizzle that matches a K row of OZ_BK bytes
+constexpr uint32_t OZ_SW_LAYOUT = OZ_BK == 128 ? 2u : 4u;    // 128-byte / 64-byte swizzle
+constexpr uint32_t OZ_SW_SBO = 8u * OZ_BK;                   // bytes between 8-row groups
+static_assert(OZ_BK == 64 || OZ_BK == 128, "K rows of 64 or 128 bytes");
 #ifndef OZ_STAGES_N
-#define OZ_STAGES_N 4
+#define OZ_STAGES_N (OZ_BK == 128 ? 2 : 4)
 #endif
 constexpr int OZ_STAGES = OZ_STAGES_N;
 constexpr int OZ_A_SLICE = 128 * OZ_BK;              // one slice of A per CTA: 8 KB
@@ -63,7 +70,8 @@ constexpr int OZ_SMEM = 1024 + OZ_STAGES * OZ_STAGE + 256;
 constexpr uint32_t OZ_TMEM_COLS = 512;               // 5 x 96 used
 static_assert(OZ_S * OZ_BN <= 512, "level accumulators must fit in TMEM");
 static_assert(OZ_SMEM <= 232448, "ozaki GEMM exceeds shared memory");
-static_assert(OZ_A_SLICE % 512 == 0 && OZ_B_SLICE % 512 == 0, "64-byte swizzle atoms are 512 B");
+static_assert(OZ_A_SLICE % (8 * OZ_BK) == 0 && OZ_B_SLICE % (8 * OZ_BK) == 0,
+              "slices start on swizzle atoms");
 
 // ------------------------------------------------------------- device helpers
 SHP_DEV void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t mbar, int x, int y,
@@ -246,7 +254,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   const int idx = threadIdx.x >> 2, seg = (threadIdx.x & 3) * 16;
   // row slicing: this thread's row r0 + idx, columns c0 + seg .. + 15
-  const int64_t nkb_r = (cols + SL_T - 1) / SL_T, nkb_c = (rows + SL_T - 1) / SL_T;
+  const int64_t nkb_r = (cols + OZ_BK - 1) / OZ_BK, nkb_c = (rows + OZ_BK - 1) / OZ_BK;
   if (rsl != nullptr && r0 + idx < rows) {
     const int r = r0 + idx;
     double f, sg;
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int q = 0; q < OZ_S; ++q) {
       int8_t* dst =
-          rsl + ((((b * nkb_r + blockIdx.x) * OZ_S + q) * rows + r) * SL_T) + seg;
+          rsl + ((((b * nkb_r + c0 / OZ_BK) * OZ_S + q) * rows + r) * OZ_BK) + c0 % OZ_BK + seg;
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
     }
   }
@@ -290,7 +298,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int q = 0; q < OZ_S; ++q) {
       int8_t* dst =
-          csl + ((((b * nkb_c + blockIdx.y) * OZ_S + q) * cols + c) * SL_T) + seg;
+          csl + ((((b * nkb_c + r0 / OZ_BK) * OZ_S + q) * cols + c) * OZ_BK) + r0 % OZ_BK + seg;
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
     }
   }
@@ -459,8 +467,9 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
   uint64_t* accf = empty + OZ_STAGES;
   uint64_t* acce = accf + 1;
   uint64_t* drain = acce + 1;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+  uint64_t* never = drain + 1;  // completed by nothing: the self-test's wait
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(never + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -471,6 +480,7 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
     mbar_init(accf, 1);
     mbar_init(acce, 2 * OZ_EPI_WARPS);
     mbar_init(drain, 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tA);
@@ -490,6 +500,13 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
       const uint32_t tx = 2u * OZ_STAGE;
       int kit = 0;
       bool stop = false;
+      // bounded-wait self-test: before any copy is issued, wait on a barrier
+      // nothing completes; it runs out, and the CTA unwinds with nothing in flight
+      if (ep.selftest && !mbar_wait(never, 0, nullptr, SHP_SELFTEST_LIMIT)) {
+        *abort_flag = 1;
+        if (ep.status != nullptr) atomicExch(&ep.status[0], ST_ETIMEOUT);
+        stop = true;
+      }
       for (int t = cl; t < ntiles && !stop; t += ncl) {
         const int b = t / per_b, r = t % per_b;
         if (ep.active != nullptr && ep.active[b] == 0) continue;
@@ -499,7 +516,7 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
         for (int kb = 0; kb < KB; ++kb, ++kit) {
           const int s = kit % OZ_STAGES;
           if (kit >= OZ_STAGES &&
-              (*abort_flag || !mbar_wait(&empty[s], ((kit / OZ_STAGES) - 1) & 1))) {
+              (*abort_flag || !mbar_wait(&empty[s], ((kit / OZ_STAGES) - 1) & 1, abort_flag))) {
             *abort_flag = 1;
             if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
             stop = true;
@@ -523,7 +540,7 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
       for (int t = cl; t < ntiles && !stop; t += ncl) {
         const int b = t / per_b;
         if (ep.active != nullptr && ep.active[b] == 0) continue;
-        if (tl >= 1 && (*abort_flag || !mbar_wait(acce, (tl - 1) & 1))) {
+        if (tl >= 1 && (*abort_flag || !mbar_wait(acce, (tl - 1) & 1, abort_flag))) {
           *abort_flag = 1;
           if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
           break;
@@ -531,7 +548,7 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
         tc_fence_after();
         for (int kb = 0; kb < KB; ++kb, ++kit) {
           const int s = kit % OZ_STAGES;
-          if (*abort_flag || !mbar_wait(&full[s], (kit / OZ_STAGES) & 1)) {
+          if (*abort_flag || !mbar_wait(&full[s], (kit / OZ_STAGES) & 1, abort_flag)) {
             *abort_flag = 1;
             if (ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
             stop = true;
@@ -542,8 +559,8 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
           // memory addresses stay below 2^18, so adding offsets >> 4 to the
           // base descriptor never carries out of the field)
           const uint32_t base = smem_u32(smem + s * OZ_STAGE);
-          const uint64_t ad0 = smem_desc(base, 16, 512, 4);
-          const uint64_t bd0 = smem_desc(base + OZ_A_BYTES, 16, 512, 4);
+          const uint64_t ad0 = smem_desc(base, 16, OZ_SW_SBO, OZ_SW_LAYOUT);
+          const uint64_t bd0 = smem_desc(base + OZ_A_BYTES, 16, OZ_SW_SBO, OZ_SW_LAYOUT);
 #pragma unroll
           for (int ks = 0; ks < OZ_BK / 32; ++ks) {
 #pragma unroll
@@ -575,7 +592,7 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
     for (int t = cl; t < ntiles; t += ncl) {
       const int b = t / per_b, r = t % per_b;
       if (ep.active != nullptr && ep.active[b] == 0) continue;
-      if (*abort_flag || !mbar_wait(accf, tl & 1)) {
+      if (*abort_flag || !mbar_wait(accf, tl & 1, abort_flag)) {
         *abort_flag = 1;
         if (lane == 0 && ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
         break;
@@ -724,7 +741,7 @@ __global__ void __launch_bounds__(EW)
 }  // namespace
 
 // ------------------------------------------------------------- host side
-int64_t oz_ldk(int64_t k) { return (k + SL_T - 1) / SL_T * SL_T; }
+int64_t oz_ldk(int64_t k) { return (k + OZ_BK - 1) / OZ_BK * OZ_BK; }
 
 size_t oz_slices_bytes(int64_t rows, int64_t k, int64_t batch) {
   return static_cast<size_t>(OZ_S) * rows * oz_ldk(k) * batch;
@@ -749,7 +766,8 @@ cudaError_t oz_slice(const double* X, int rows, int cols, int64_t ld, int64_t bs
     const dim3 grid((cols + SL_T - 1) / SL_T, (rows + SL_T - 1) / SL_T, batch);
     k_oz_absmax<<<grid, 256, 0, st>>>(X, rows, cols, ld, bs, active, rmax, cmax);
   }
-  const dim3 grid2((cols + SL_T - 1) / SL_T, (rows + SL_T - 1) / SL_T, batch);
+  // the slicing tiles cover whole K blocks (digits 0 past the matrix edge)
+  const dim3 grid2((oz_ldk(cols) + SL_T - 1) / SL_T, (oz_ldk(rows) + SL_T - 1) / SL_T, batch);
   k_oz_slice<<<grid2, 256, 0, st>>>(X, rows, cols, ld, bs, active, rmax, cmax, out.rows,
                                     out.cols, out.rscale, out.cscale, x32);
   return cudaGetLastError();
@@ -758,11 +776,11 @@ cudaError_t oz_slice(const double* X, int rows, int cols, int64_t ld, int64_t bs
 cudaError_t gemm_oz(const int8_t* Arows, const int8_t* Bcols, int M, int N, int K, int batch,
                     const OzEpi& ep, cudaStream_t st) {
   if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return cudaSuccess;
-  static_assert(OZ_BK == SL_T, "a GEMM stage is one K block of the slice layout");
+  static_assert(OZ_BK % SL_T == 0, "a K block of the slice layout is whole slicing tiles");
   CUtensorMap ma, mb;
   const int64_t nkb = (K + OZ_BK - 1) / OZ_BK;
-  if (!tensor_map_slices(&ma, Arows, M, OZ_S, nkb * batch, 128) ||
-      !tensor_map_slices(&mb, Bcols, N, OZ_S, nkb * batch, OZ_BN / 2))
+  if (!tensor_map_slices(&ma, Arows, M, OZ_S, nkb * batch, OZ_BK, 128) ||
+      !tensor_map_slices(&mb, Bcols, N, OZ_S, nkb * batch, OZ_BK, OZ_BN / 2))
     return cudaErrorInvalidValue;
   static int attr_set[64];
   int dev = 0, sms = 148;

@@ -52,16 +52,25 @@ SHP_DEV uint32_t mbar_try_wait(uint32_t addr, uint32_t parity) {
       : "memory");
   return ok;
 }
-// Bounded wait on phase `parity`; returns false if the limit ran out.
-SHP_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait on phase `parity`; returns false if `limit` cycles ran out or,
+// when `abort` is given, once another role of the CTA has set it (so that a
+// CTA whose wait gave up unwinds without every other waiter spinning to its
+// own limit).
+SHP_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort = nullptr,
+                       long long limit = SHP_SPIN_LIMIT) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(addr, parity)) {
-    if (clock64() - t0 > SHP_SPIN_LIMIT) return false;
+    if (clock64() - t0 > limit) return false;
+    if (abort != nullptr && *abort) return false;
   }
   return true;
 }
+
+// Limit of the wait a bounded-wait self-test points at a barrier nothing
+// completes (about 10 ms): long enough to be a real wait, short for a test.
+#define SHP_SELFTEST_LIMIT (20000000LL)
 
 SHP_DEV void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");

@@ -196,7 +196,7 @@ struct SkTma {
   static size_t smem_bytes(int64_t n) {
     const int64_t ldv = (n + ST_SC - 1) / ST_SC * ST_SC + 4;
     return 128 + static_cast<size_t>(ST_NST) * STAGE_FLOATS * 4 + static_cast<size_t>(P) * ldv * 4 +
-           (2 * ST_NST + 2) * 8 + 16;
+           (2 * ST_NST + 3) * 8 + 16;
   }
 };
 
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
     k_sketch_tma(const __grid_constant__ CUtensorMap tR, int64_t n,
                  const float* __restrict__ Vin, int64_t vbs, float* __restrict__ Vout,
                  int64_t obs, int p, int batch, const int* __restrict__ active,
-                 const int* __restrict__ it, int64_t it_stride, int* tmo) {
+                 const int* __restrict__ it, int64_t it_stride, int* tmo, int selftest) {
   count_kernel_run();
   using K = SkTma<P>;
   constexpr int ROWS = K::ROWS, RPI = K::RPI;
@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(Vs + P * ldv);
   uint64_t* empty = full + ST_NST;
   uint64_t* vbar = empty + ST_NST;  // [2] old V released, new V staged
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(vbar + 2);
+  uint64_t* never = vbar + 2;       // completed by nothing: the self-test's wait
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(never + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gpb = (n + RPI - 1) / RPI;  // items per block
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
     }
     mbar_init(&vbar[0], ST_CONS);
     mbar_init(&vbar[1], ST_CONS);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
         last_b = b;
         for (int c = 0; c < nch; ++c, ++kit) {
           const int s = kit % ST_NST;
-          if (kit >= ST_NST && !mbar_wait(&empty[s], ((kit / ST_NST) - 1) & 1)) {
+          if (kit >= ST_NST && !mbar_wait(&empty[s], ((kit / ST_NST) - 1) & 1, abort_flag)) {
             sketch_give_up(abort_flag, tmo, b, 0);
             break;
           }
@@ -294,6 +296,12 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
     }
     if (!seen_on) continue;
     if (b != cur_b) {  // stage V of block b (all consumer warps; the producer runs on)
+      // bounded-wait self-test: the first V hand-over waits on a barrier
+      // nothing completes, with the producer's copies already in flight
+      if (selftest && !mbar_wait(never, 0, nullptr, SHP_SELFTEST_LIMIT)) {
+        sketch_give_up(abort_flag, tmo, b, lane);
+        break;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&vbar[0]);  // this warp is done with the old V
       if (!mbar_wait(&vbar[0], ns & 1)) {
@@ -561,7 +569,7 @@ namespace {
 template <int P>
 bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin, int64_t vbs,
                        float* Vout, int64_t obs, int p, int batch, const int* active,
-                       const int* it, int64_t it_stride, int* tmo, cudaStream_t st,
+                       const int* it, int64_t it_stride, int* tmo, int selftest, cudaStream_t st,
                        cudaError_t* err) {
   const size_t smem = SkTma<P>::smem_bytes(n);
   if (smem > 200 * 1024) return false;  // V does not fit whole: the register kernel
@@ -583,7 +591,7 @@ bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin,
   const int64_t items = (n + SkTma<P>::RPI - 1) / SkTma<P>::RPI * batch;
   const int grid = static_cast<int>(items < sms ? items : sms);
   kern<<<grid, 32 * (ST_CONS + 1), smem, st>>>(tR, n, Vin, vbs, Vout, obs, p, batch, active, it,
-                                                it_stride, tmo);
+                                                it_stride, tmo, selftest);
   *err = cudaGetLastError();
   return true;
 }
@@ -593,7 +601,7 @@ bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin,
 cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r_bstride,
                         const float* Vin, int64_t vin_bstride, float* Vout, int64_t vout_bstride,
                         int p, int batch, const int* active, const int* it, int64_t it_stride,
-                        cudaStream_t st, int* tmo) {
+                        cudaStream_t st, int* tmo, int selftest) {
   if (batch <= 0 || n <= 0) return cudaSuccess;
   // plain fp32 R with 16-byte aligned rows: the bulk-copy kernel when V fits
   if (Rlo == nullptr && (reinterpret_cast<uintptr_t>(Rhi) & 15) == 0 && n % 4 == 0 &&
@@ -602,13 +610,13 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
     bool done = false;
     if (p <= 4)
       done = launch_sketch_tma<4>(Rhi, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
-                                  batch, active, it, it_stride, tmo, st, &e);
+                                  batch, active, it, it_stride, tmo, selftest, st, &e);
     else if (p <= 8)
       done = launch_sketch_tma<8>(Rhi, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
-                                  batch, active, it, it_stride, tmo, st, &e);
+                                  batch, active, it, it_stride, tmo, selftest, st, &e);
     else if (p <= 16)
       done = launch_sketch_tma<16>(Rhi, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
-                                   batch, active, it, it_stride, tmo, st, &e);
+                                   batch, active, it, it_stride, tmo, selftest, st, &e);
     if (done) return e;
   }
   const int rows = (p <= 8 ? 4 : 2) * 8 * SK_GROUPS;  // rows per CTA (ROWS x 8 warps x groups)

@@ -310,3 +310,18 @@ def shp_matmul_f64(Amat, B, out=None, ws=None, reuse_a=False, reuse_b=False, acc
     _check(A.lib().shp_matmul_f64_ex(_p(Amat), _p(B), _p(out), M, N, K, batch, flags, _p(ws),
                                      ws.numel(), _stream()), "shp_matmul_f64")
     return out
+
+
+def selftest_bounded_wait(which: str, device=None):
+    """Make one bounded pipeline wait run out on purpose ("gemm", "ozaki" or
+    "sketch"); returns (status the kernel recorded, alpha of the sketch's fit)
+    -- SHP_ETIMEOUT and, for "sketch", NaN are expected."""
+    code = {"gemm": A.SHP_SELFTEST_GEMM, "ozaki": A.SHP_SELFTEST_OZAKI,
+            "sketch": A.SHP_SELFTEST_SKETCH}[which]
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    status = torch.full((1,), -1, dtype=torch.int32, device=device)
+    alpha = torch.zeros(1, dtype=torch.float32, device=device)
+    ws = torch.empty(A.SHP_SELFTEST_WS_BYTES, dtype=torch.uint8, device=device)
+    _check(A.lib().shp_selftest_bounded_wait(code, _p(status), _p(alpha), _p(ws), ws.numel(),
+                                             _stream()), "shp_selftest_bounded_wait")
+    return int(status.item()), float(alpha.item())

@@ -470,3 +470,30 @@ def test_inv_root_pass2_zero_steps_beside_ordinary_block(prec):
     assert rep["status"][1] == o.OK and rep["iters"][1][1] >= 1
     Xo, _ = o.inv_root_ref(A[1], o.POW_INV4, oracle_opts(opts), S, force_iters=rep["iters"][1])
     assert relerr(X[1], Xo) <= 1e-5
+
+
+# residual floors of the paths at cond 1e3: fp32 products on chip and the
+# 3xTF32 split end near 1e-6 (the last residuals differ from the float64
+# oracle's by that much), the Ozaki path near 1e-12
+@pytest.mark.parametrize("n,prec,tol,res_floor", [(48, "3xtf32", TOL_SPLIT, 3e-6),
+                                                  (256, "3xtf32", TOL_3X_COND1E3, 3e-6),
+                                                  (256, "ozaki", TOL_SPLIT, 1e-9)])
+def test_chebyshev_variant(n, prec, tol, res_floor):
+    """Chebyshev's third-order method (the d = 2 step with the coefficient
+    fixed at 3/8, PRISM Contributi Chiave 1 names it among the iterations
+    PRISM accelerates): on chip and on the tensor cores, against the oracle's
+    same iteration (residuals, result), and PRISM's fitted alpha needs no
+    more steps to the same tolerance."""
+    A = synth.spd_batch(n, 2, 1e-3, 1.0, 121)
+    S = synth.sketch_stack(80, n, 8, 1021)
+    Xc, rc, oc = run_inv_root(A, "inv4", 2, 8, 1e-6, 40, prec, S, lo=0.375, fixed_alpha=True)
+    Xp, rp, _ = run_inv_root(A, "inv4", 2, 8, 1e-6, 40, prec, S)
+    for b in range(2):
+        assert rc["status"][b] in (o.OK, o.ESTALL)
+        it = rc["iters"][b]
+        np.testing.assert_array_equal(rc["alpha"][b, 0, :it[0]], 0.375)
+        Xo, infos = o.inv_root_ref(A[b], o.POW_INV4, oracle_opts(oc), None, force_iters=it)
+        np.testing.assert_allclose(rc["resid"][b, 0, :it[0] + 1], infos[0].res, rtol=1e-3,
+                                   atol=res_floor)
+        assert relerr(Xc[b], Xo) <= tol
+        assert rp["iters"][b].sum() <= rc["iters"][b].sum()

@@ -600,3 +600,43 @@ def test_stall_rule_on_scalar_residual(stall_below, stall_ratio, max_iter, statu
     want = [0.9, 0.8499375, 0.7793903636596528, 0.6850442777023162, 0.5679272072594314,
             0.4365241771417045]
     np.testing.assert_allclose(info.res, want[: iters + 1], rtol=1e-12)
+
+
+# Chebyshev's third-order root-finding step, x <- x - f/f' - f'' f^2 / (2 f'^3)
+# (Traub, Iterative Methods for the Solution of Equations, 1964), applied to
+# f(x) = x^-2 - a, whose root is a^(-1/2): written here from f and its
+# derivatives, not from any polynomial of the oracle.
+def chebyshev_inv_sqrt_step(x, a):
+    f = x ** -2 - a
+    f1 = -2.0 * x ** -3
+    f2 = 6.0 * x ** -4
+    return x - f / f1 - f2 * f * f / (2.0 * f1 ** 3)
+
+
+@pytest.mark.parametrize("rotated", [False, True])
+def test_chebyshev_is_the_fixed_degree2_taylor_step(rotated):
+    """The Chebyshev variant PRISM accelerates is the d = 2 step with the top
+    coefficient fixed at its Taylor value 3/8: on B = Q diag(lam) Q^T the
+    oracle's Z_k (fixed_alpha, d = 2, lo = 3/8) has eigenvalues that follow
+    Chebyshev's step for a^(-1/2), a = lam, from z_0 = 1."""
+    n, steps = 6, 5
+    lam = np.array([0.9, 0.6, 0.35, 0.2, 0.08, 0.03])
+    Q = rot(n, 21) if rotated else np.eye(n)
+    B = (Q * lam) @ Q.T
+    opts = o.PrismOpts(d=2, p=2, lo=0.375, hi=1.0, tol=0.0, max_iter=steps, fixed_alpha=True,
+                       stall_below=0.0)
+    _, Z, info = o.coupled_ref(B, opts, None)
+    z = np.ones(n)
+    for _ in range(steps):
+        z = chebyshev_inv_sqrt_step(z, lam)
+    np.testing.assert_allclose(Q.T @ Z @ Q, np.diag(z), rtol=1e-12, atol=1e-13)
+    assert info.iters == steps and all(a == 0.375 for a in info.alpha)
+    # third order: one step maps the residual eigenvalue xi = 1 - lam z^2 to
+    # 5/8 xi^3 + 15/64 xi^4 + 9/64 xi^5 (worked out by hand from r = 1 - (1-xi) g^2
+    # with g = 1 + xi/2 + 3 xi^2/8: no xi^2 term), and so does the oracle's table
+    xi = 1.0 - lam
+    xi1 = 1.0 - lam * chebyshev_inv_sqrt_step(np.ones(n), lam) ** 2
+    np.testing.assert_allclose(xi1, 5 / 8 * xi ** 3 + 15 / 64 * xi ** 4 + 9 / 64 * xi ** 5,
+                               rtol=1e-12)
+    np.testing.assert_allclose(o.residual_coeffs(2, 0.375), [0, 0, 0, 5 / 8, 15 / 64, 9 / 64],
+                               atol=1e-15)
