@@ -294,18 +294,24 @@ def step_only(args):
 
 
 def ozgemm_only(args):
-    """The Ozaki-scheme GEMM alone (profiling aid): --batch products of
-    1024^2 fp64 matrices through shp_matmul_f64 (slicing, then one k_gemm_oz)."""
+    """The Ozaki-scheme GEMM alone (profiling aid), as the bench's roofline
+    times it: --batch products of 1024^2 fp64 matrices through
+    shp_matmul_f64; the first call slices both operands, every later one
+    reuses the slices and accumulates (C <- C + A B, the step's epilogue), so
+    it is one k_gemm_oz launch."""
     import torch
 
-    from second_order_optimizer_shampoo_b200 import prism
+    from second_order_optimizer_shampoo_b200 import _abi, prism
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(5)
     X = torch.randn(args.batch, N, N, device=dev, generator=g, dtype=torch.float64)
     Y = torch.randn(args.batch, N, N, device=dev, generator=g, dtype=torch.float64)
-    out = torch.empty_like(X)
+    out = torch.zeros_like(X)
+    ws = torch.empty(int(_abi.lib().shp_matmul_f64_workspace_bytes(N, N, N, args.batch)),
+                     dtype=torch.uint8, device=dev)
+    prism.shp_matmul_f64(X, Y, out=out, ws=ws)
     for _ in range(max(args.warmup, 1) + args.steps):
-        prism.shp_matmul_f64(X, Y, out=out)
+        prism.shp_matmul_f64(X, Y, out=out, ws=ws, reuse_a=True, reuse_b=True, accumulate=True)
     torch.cuda.synchronize()
     print(json.dumps({"kernel": "ozgemm", "batch": args.batch,
                       "launches": args.steps + max(args.warmup, 1)}))

@@ -324,9 +324,14 @@ __global__ void __launch_bounds__(256, 1)
   if (ep.active != nullptr && ep.active[b] == 0) return;  // uniform over a CTA pair
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const bool leader = rank == 0;
-  const int m0 = PAIR ? static_cast<int>(blockIdx.y) * 256 + static_cast<int>(rank) * 128
-                      : static_cast<int>(blockIdx.y) * 128;
-  const int n0 = (PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x)) * BN;
+  // a symmetric result on square tiles (one CTA each): blockIdx.x enumerates
+  // the tiles on and above the diagonal; off-diagonal ones also write their
+  // mirror image
+  const bool sym = !PAIR && ep.sym != 0 && ep.M == ep.N && BN == 128;
+  int tmi = static_cast<int>(blockIdx.y), tni = static_cast<int>(PAIR ? blockIdx.x >> 1 : blockIdx.x);
+  if (sym) tile_coords(static_cast<int>(blockIdx.x), (ep.N + 127) / 128, true, tmi, tni);
+  const int m0 = PAIR ? tmi * 256 + static_cast<int>(rank) * 128 : tmi * 128;
+  const int n0 = tni * BN;
   const int bn_cta = PAIR ? BN / 2 : BN;        // B rows (or columns) this CTA stages
   const int nb0 = n0 + static_cast<int>(rank) * bn_cta;
 
@@ -486,8 +491,10 @@ __global__ void __launch_bounds__(256, 1)
   if (!mbar_wait(done, 0)) timed_out = true;
   __syncwarp();
   tc_fence_after();
+  const bool mirror = sym && tmi != tni;
   float nrm = epilogue_tile<C::SPLIT, 16>(reinterpret_cast<float*>(smem) + warp * (32 * 33), tmem,
-                                          ep, b, m0, n0, BN, warp & 3, warp >> 2, lane);
+                                          ep, b, m0, n0, BN, warp & 3, warp >> 2, lane, mirror);
+  if (mirror) nrm *= 2.f;
   if (ep.kind == EPI_RESID) {
     nrm = warp_sum(nrm);
     if (lane == 0) atomicAdd(&ep.norm2[static_cast<int64_t>(b) * ep.norm2_stride], nrm);
@@ -776,8 +783,11 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = PAIR ? dim3(2 * ((N + BN - 1) / BN), (M + 255) / 256, batch)
-                     : dim3((N + BN - 1) / BN, (M + 127) / 128, batch);
+  const int tq = (N + 127) / 128;
+  const bool sym = !PAIR && ep.sym != 0 && M == N && BN == 128;
+  cfg.gridDim = PAIR  ? dim3(2 * ((N + BN - 1) / BN), (M + 255) / 256, batch)
+                : sym ? dim3(tq * (tq + 1) / 2, 1, batch)
+                      : dim3((N + BN - 1) / BN, (M + 127) / 128, batch);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
@@ -890,10 +900,23 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
   const int rowb = 128;  // Cfg<MODE>::ROWB
   const int bk = rowb / esz, chunk = 128 / esz;
   const CUtensorMapSwizzle k_swz = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  const int BN = N > 128 ? 256 : (N > 64 ? 128 : 64);
+  int BN = N > 128 ? 256 : (N > 64 ? 128 : 64);
   // CTA pairs (M = 256 per MMA) for full-width tiles; small problems keep one
-  // CTA per 128-row tile.
-  const bool pair = M >= 256 && BN == 256;
+  // CTA per 128-row tile.  When the 256 x 256 tiles would leave most SM pairs
+  // idle (a few blocks, e.g. the two Kronecker factors of one weight), one CTA
+  // per 128 x 128 tile puts four times as many SMs to work.
+  bool pair = M >= 256 && BN == 256;
+  if (pair && !ep.selftest) {  // the self-test exercises the persistent pair kernel
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tn = (N + 255) / 256, tm = (M + 255) / 256;
+    const int64_t tiles = static_cast<int64_t>(ep.sym && M == N ? tn * (tn + 1) / 2 : tn * tm) * batch;
+    if (2 * tiles < sms) {
+      pair = false;
+      BN = 128;
+    }
+  }
   const int bn_cta = pair ? BN / 2 : BN;
   CUtensorMap ma, mal, mb, mbl;
   bool ok = true;
