@@ -427,7 +427,18 @@ def _time(fn, stream, reps):
     return e0.elapsed_time(e1) / reps
 
 
-def shampoo_step_leg(args, dev, stream):
+def shampoo_only(args):
+    """One config-2 Shampoo step alone (profiling aid), the inverse roots
+    with the host loop so that profilers see each launch."""
+    import torch
+    dev = torch.device("cuda", 0)
+    out = shampoo_step_leg(args, dev, torch.cuda.current_stream(), host_loop=True,
+                           reps=args.steps)
+    print(json.dumps({"kernel": "shampoo", "ms_per_step": out["ms_per_step"]}))
+    return 0
+
+
+def shampoo_step_leg(args, dev, stream, host_loop=False, reps=10):
     """One Shampoo step on a 1024 x 1024 weight: 10 EMA steps of L and R with
     fresh G (TF32), L^(-1/4) and R^(-1/4) by PRISM (d = 2, p = 8, tol 1e-3,
     TF32) as one batch of two, and W -= 1e-3 L^(-1/4) G R^(-1/4)."""
@@ -439,7 +450,7 @@ def shampoo_step_leg(args, dev, stream):
     Gs = [torch.from_numpy(synth.gaussian((1, n, n), 0.02, 102, index=t + 1)).to(dev)
           for t in range(10)]
     S = torch.from_numpy(synth.sketch_stack(2 * mi, n, 8, 1002)).to(dev)
-    opts = prism.make_opts(d=2, p=8, tol=1e-3, max_iter=mi, prec="tf32")
+    opts = prism.make_opts(d=2, p=8, tol=1e-3, max_iter=mi, prec="tf32", host_loop=host_loop)
     LR = torch.zeros(2, n, n, device=dev)
     W = W0.clone()
     roots = torch.empty_like(LR)
@@ -460,7 +471,7 @@ def shampoo_step_leg(args, dev, stream):
         step()
     torch.cuda.synchronize()
     iters = rep["iters"].cpu().numpy()
-    ms = _time(step, stream, 10)
+    ms = _time(step, stream, reps)
     flops = 10 * 2 * n * (n + 1) * n + sum(block_flops(blk, n) for blk in iters) + 2 * 2.0 * n ** 3
     return {"workload": "shampoo_step_1024sq_ema10_inv4_d2_p8_tf32_apply", "ms_per_step": ms,
             "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
@@ -770,7 +781,8 @@ def main():
                     help="skip the Shampoo-step, GEMM-count and single-block legs")
     ap.add_argument("--prec", default="ozaki", choices=["ozaki", "3xtf32", "tf32"],
                     help="product path of --kernel step")
-    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar", "sketch", "step", "ozgemm"],
+    ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar", "sketch", "step", "ozgemm",
+                             "shampoo"],
                     help="run only the batched 3xTF32 GEMM, the small-block kernel, the "
                          "polar leg or the sketch leg (for profiling; --batch sets the "
                          "GEMM/small/sketch batch)")
@@ -784,6 +796,8 @@ def main():
         return step_only(args)
     if args.kernel == "ozgemm":
         return ozgemm_only(args)
+    if args.kernel == "shampoo":
+        return shampoo_only(args)
     if args.kernel == "small":
         return small_only(args)
     if args.kernel == "sketch":
