@@ -92,6 +92,35 @@ SHP_DEV void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// The same product with the A operand held in the tensor core's collector
+// buffer across consecutive instructions: FILL reads A from shared memory and
+// keeps it, USE takes the kept copy, LAST takes it and frees the buffer.  The
+// products of one A digit slice against several B slices then read that slice
+// from shared memory once instead of once per product.
+enum { COLL_FILL = 0, COLL_USE = 1, COLL_LAST = 2 };
+template <int C>
+SHP_DEV void mma_i8_pair_coll(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                              uint32_t accumulate) {
+  if constexpr (C == COLL_FILL)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8.collector::a::fill [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  else if constexpr (C == COLL_USE)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8.collector::a::use [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 // kind::i8 instruction descriptor: D s32, A and B signed 8-bit, both K-major.
 constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
@@ -561,17 +590,26 @@ __global__ void __launch_bounds__(OZ_THREADS, 1)
           const uint32_t base = smem_u32(smem + s * OZ_STAGE);
           const uint64_t ad0 = smem_desc(base, 16, OZ_SW_SBO, OZ_SW_LAYOUT);
           const uint64_t bd0 = smem_desc(base + OZ_A_BYTES, 16, OZ_SW_SBO, OZ_SW_LAYOUT);
+          // A slice sa meets B slices 0 .. S-1-sa (level sa + sb); the first
+          // product of a k-step into each level comes from sa = 0
 #pragma unroll
           for (int ks = 0; ks < OZ_BK / 32; ++ks) {
 #pragma unroll
-            for (int L = 0; L < OZ_S; ++L) {
+            for (int sa = 0; sa < OZ_S; ++sa) {
+              const uint64_t ad = ad0 + static_cast<uint64_t>((sa * OZ_A_SLICE + ks * 32) >> 4);
+              const uint32_t acc = (kb > 0 || ks > 0 || sa > 0) ? 1u : 0u;
 #pragma unroll
-              for (int sa = 0; sa <= L; ++sa) {
-                const int sb = L - sa;
-                const uint64_t ad = ad0 + static_cast<uint64_t>((sa * OZ_A_SLICE + ks * 32) >> 4);
+              for (int sb = 0; sb < OZ_S - sa; ++sb) {
                 const uint64_t bd = bd0 + static_cast<uint64_t>((sb * OZ_B_SLICE + ks * 32) >> 4);
-                mma_i8_pair(tmem + static_cast<uint32_t>(L * OZ_BN), ad, bd, idesc,
-                            (kb > 0 || ks > 0 || sa > 0) ? 1u : 0u);
+                const uint32_t d = tmem + static_cast<uint32_t>((sa + sb) * OZ_BN);
+                if (sa == OZ_S - 1)
+                  mma_i8_pair(d, ad, bd, idesc, acc);
+                else if (sb == 0)
+                  mma_i8_pair_coll<COLL_FILL>(d, ad, bd, idesc, acc);
+                else if (sb < OZ_S - 1 - sa)
+                  mma_i8_pair_coll<COLL_USE>(d, ad, bd, idesc, acc);
+                else
+                  mma_i8_pair_coll<COLL_LAST>(d, ad, bd, idesc, acc);
               }
             }
           }
