@@ -310,10 +310,15 @@ def ozgemm_only(args):
     ws = torch.empty(int(_abi.lib().shp_matmul_f64_workspace_bytes(N, N, N, args.batch)),
                      dtype=torch.uint8, device=dev)
     prism.shp_matmul_f64(X, Y, out=out, ws=ws)
-    for _ in range(max(args.warmup, 1) + args.steps):
+    for _ in range(max(args.warmup, 1)):
         prism.shp_matmul_f64(X, Y, out=out, ws=ws, reuse_a=True, reuse_b=True, accumulate=True)
-    torch.cuda.synchronize()
-    print(json.dumps({"kernel": "ozgemm", "batch": args.batch,
+    stream = torch.cuda.current_stream()
+    ms = _time(lambda: prism.shp_matmul_f64(X, Y, out=out, ws=ws, reuse_a=True, reuse_b=True,
+                                            accumulate=True), stream, args.steps)
+    flops = 2.0 * args.batch * N ** 3
+    print(json.dumps({"kernel": "ozgemm", "batch": args.batch, "ms_per_launch": ms,
+                      "fp64_tflops": flops / (ms / 1e3) / 1e12,
+                      "int8_tops": 15 * flops / (ms / 1e3) / 1e12,
                       "launches": args.steps + max(args.warmup, 1)}))
     return 0
 
@@ -662,22 +667,24 @@ def polar_flops(iters):
     return k * (sym + PN * (PN + 1) * PN + 2 * PM * PN * PN) + sym
 
 
-def polar_leg(args, dev, stream, peaks=None):
+def polar_leg(args, dev, stream, peaks=None, batch=PBATCH, host_loop=False):
     """The Muon-style polar batch: 96 matrices 4096 x 1024, rank-64 signal plus
-    0.01 noise, bf16 storage, d = 2, p = 8, until ||I - X^T X||_F / sqrt(n) <= 1e-2."""
+    0.01 noise, bf16 storage, d = 2, p = 8, until ||I - X^T X||_F / sqrt(n) <= 1e-2.
+    `batch` and `host_loop` serve profiling (fewer matrices; every launch
+    issued from the host, where profilers see it)."""
     import torch
 
     from second_order_optimizer_shampoo_b200 import _abi, prism, synth
-    bits, _ = synth.lowrank_noise_batch(PM, PN, PRANK, 0.01, PBATCH, 104)
+    bits, _ = synth.lowrank_noise_batch(PM, PN, PRANK, 0.01, batch, 104)
     G = torch.from_numpy(bits.view("int16")).to(dev).view(torch.bfloat16)
     S = torch.from_numpy(synth.sketch_stack(40, PN, 8, 1004)).to(dev)
-    opts = prism.make_opts(d=2, p=8, tol=1e-2, max_iter=40, prec="bf16")
+    opts = prism.make_opts(d=2, p=8, tol=1e-2, max_iter=40, prec="bf16", host_loop=host_loop)
     o2 = _abi.PrismOpts.from_buffer_copy(opts)
     o2.prec = _abi.SHP_BF16
-    ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_POLAR, PM, PN, PBATCH, o2),
+    ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_POLAR, PM, PN, batch, o2),
                      dtype=torch.uint8, device=dev)
     X = torch.empty_like(G)
-    rep = prism.make_report(PBATCH, 40, dev)
+    rep = prism.make_report(batch, 40, dev)
     for _ in range(2):
         prism.matfn_polar(G, opts, S, out=X, ws=ws, report=rep)
     torch.cuda.synchronize()
@@ -696,9 +703,9 @@ def polar_leg(args, dev, stream, peaks=None):
     peaks, src = load_peaks() if peaks is None else (peaks, "given")
     bf16_sust = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     tf = flops / (ms / 1e3) / 1e12
-    return {"workload": "polar_96x4096x1024_bf16_lowrank64_prism_d2_p8_tol1e-2",
+    return {"workload": f"polar_{batch}x4096x1024_bf16_lowrank64_prism_d2_p8_tol1e-2",
             "value": tf, "unit": "TFLOP/s", "ms_per_step": ms,
-            "matrices_per_s": PBATCH / (ms / 1e3), "median_iters": float(np.median(iters)),
+            "matrices_per_s": batch / (ms / 1e3), "median_iters": float(np.median(iters)),
             "status_ok": ok, "frac_of_bf16_peak": tf / bf16_sust,
             "note": "symmetric products (X^T X, R R) formed on their upper-triangle tiles "
                     "and counted n(n+1)K; peak: sustained BF16"}
@@ -783,9 +790,10 @@ def main():
                     help="product path of --kernel step")
     ap.add_argument("--kernel", default=None, choices=["gemm", "small", "polar", "sketch", "step", "ozgemm",
                              "shampoo"],
-                    help="run only the batched 3xTF32 GEMM, the small-block kernel, the "
-                         "polar leg or the sketch leg (for profiling; --batch sets the "
-                         "GEMM/small/sketch batch)")
+                    help="run one piece alone for profiling: the batched 3xTF32 GEMM, the "
+                         "small-block kernel, the polar leg (host-launched loop), the sketch "
+                         "leg, the inverse-root step, the Ozaki GEMM or the Shampoo step "
+                         "(--batch sets the GEMM/small/sketch/polar/step batch)")
     ap.add_argument("--batch", type=int, default=BATCH)
     args = ap.parse_args()
     if args.impl == "reference":
@@ -804,7 +812,8 @@ def main():
         return sketch_only(args)
     if args.kernel == "polar":
         import torch
-        print(json.dumps(polar_leg(args, torch.device("cuda", 0), torch.cuda.current_stream())))
+        print(json.dumps(polar_leg(args, torch.device("cuda", 0), torch.cuda.current_stream(),
+                                   batch=args.batch, host_loop=True)))
         return 0
     BATCH = args.batch  # blocks per GPU of the main workload (64 unless profiling)
 

@@ -523,6 +523,143 @@ __global__ void __launch_bounds__(256, 1)
 //   accf[u]:          accumulator u complete (leader's commit, both CTAs)
 //   acce[u]:          accumulator u drained (8 epilogue warps x 2 CTAs arrive
 //                     on the leader's barrier)
+// ------------------------------------------ lane-per-row epilogue (bf16 out)
+// Eight consecutive values of format fmt at element offset off, as fp32
+// (bf16: one 16-byte load; fp32: two; split: two of hi and two of lo).
+SHP_DEV void ld8(int fmt, const void* hi, const float* lo, int64_t off, float* x) {
+  if (fmt == OUT_BF16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(hi) + off);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(hi) + off);
+    const float4 a = p[0], b = p[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    if (fmt == OUT_SPLIT) {
+      const float4* q = reinterpret_cast<const float4*>(lo + off);
+      const float4 c = q[0], d = q[1];
+      x[0] += c.x; x[1] += c.y; x[2] += c.z; x[3] += c.w;
+      x[4] += d.x; x[5] += d.y; x[6] += d.z; x[7] += d.w;
+    }
+  }
+}
+
+SHP_DEV float ld1(int fmt, const void* hi, const float* lo, int64_t off) {
+  if (fmt == OUT_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(hi)[off]);
+  const float h = static_cast<const float*>(hi)[off];
+  return fmt == OUT_SPLIT ? h + lo[off] : h;
+}
+
+// Eight values rounded to bf16, one 16-byte store at element offset off.
+SHP_DEV void st8_bf16(void* hi, int64_t off, const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&t);
+  }
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(hi) + off) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Epilogue of one CTA's 128 x 256 accumulator into a bf16 result, by 8 warps
+// with a lane per row: warp (q, h) reads TMEM lanes 32q..32q+31 (the lane
+// quarter of its warpgroup position q) and the 32-column chunks c = h, h + 2,
+// ...; lane i holds row m0 + 32q + i of the chunk in registers, reads that
+// row's aux values and writes its 32 results as four 16-byte stores, with no
+// shared-memory pass and every load of a chunk issued before any use.  For
+// bf16 rows (64 bytes per chunk) this measured faster than a lane-per-column
+// epilogue transposed through shared memory: four times fewer instructions
+// outweigh the less coalesced stores; for fp32 rows the transposed epilogue
+// wins and is used instead.  Chunks that cross the matrix edge go element by
+// element.  A mirrored off-diagonal tile of a symmetric result is also
+// written transposed: there lanes hold consecutive columns of the image, so
+// those stores are coalesced.  Needs ep.vec (16-byte aligned rows) and an
+// out2_hi/out_plain-free store, or out2 in bf16 too.  Returns this lane's sum
+// of squares (RESID).
+SHP_DEV float epilogue_lane_rows(uint32_t tmem, const EpiParams& ep, int b, int m0, int n0, int q,
+                                 int h, int lane, bool mirror) {
+  const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;  // GPOLY
+  const float eta = ep.alpha != nullptr ? ep.alpha[b] : 1.f;    // APPLY, MOMENTUM
+  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;
+  const bool need_old = ep.kind == EPI_EMA || ep.kind == EPI_APPLY || ep.kind == EPI_MOMENTUM;
+  const int row = m0 + q * 32 + lane;
+  const bool rowok = row < ep.M;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  const int64_t obase = static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(row) * ep.ldo;
+  const int64_t abase =
+      static_cast<int64_t>(b) * ep.bs_aux + static_cast<int64_t>(row) * ep.lda_aux;
+  float nrm = 0.f;
+  for (int c = h; c < 8; c += 2) {
+    const int cb = n0 + c * 32;
+    float a[32];
+    tmem_ld32(trow + static_cast<uint32_t>(c * 32), a);  // the whole warp
+    if (rowok && cb < ep.N) {
+      if (cb + 32 <= ep.N) {
+        float x[32], w[32];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (need_aux) {
+            ld8(ep.aux_fmt, ep.aux_hi, ep.aux_lo, abase + cb + 8 * g, x + 8 * g);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[8 * g + j] = 0.f;
+          }
+          if (need_old) {  // read-modify-write kinds store fp32 (never this path)
+            ld8(OUT_F32, ep.out_hi, nullptr, obase + cb + 8 * g, w + 8 * g);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[8 * g + j] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float v[8], v2[8];
+          nrm += epi_rows<8>(ep, a + 8 * g, x + 8 * g, w + 8 * g, row - cb - 8 * g, 8, alpha, eta,
+                             v, v2);
+          st8_bf16(ep.out_hi, obase + cb + 8 * g, v);
+          if (ep.out2_hi != nullptr) st8_bf16(ep.out2_hi, obase + cb + 8 * g, v2);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) a[8 * g + j] = v[j];  // kept for the mirror image
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int col = cb + j;
+          if (col < ep.N) {
+            float x = need_aux ? ld1(ep.aux_fmt, ep.aux_hi, ep.aux_lo, abase + col) : 0.f;
+            float w = need_old ? static_cast<const float*>(ep.out_hi)[obase + col] : 0.f;
+            float v, v2;
+            nrm += epi_rows<1>(ep, &a[j], &x, &w, col == row ? 0 : -1, 1, alpha, eta, &v, &v2);
+            put(OUT_BF16, ep.out_hi, nullptr, obase + col, v);
+            if (ep.out2_hi != nullptr) put(OUT_BF16, ep.out2_hi, nullptr, obase + col, v2);
+            a[j] = v;
+          }
+        }
+      }
+      if (mirror) {
+        // the image of column cb + j is row cb + j; lanes write its
+        // consecutive columns m0 + 32q + lane.  A mirrored tile holds no
+        // diagonal element, so out2 = I + v is v there.
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (cb + j < ep.N) {
+            const int64_t off = static_cast<int64_t>(b) * ep.bso +
+                                static_cast<int64_t>(cb + j) * ep.ldo + row;
+            put(OUT_BF16, ep.out_hi, nullptr, off, a[j]);
+            if (ep.out2_hi != nullptr) put(OUT_BF16, ep.out2_hi, nullptr, off, a[j]);
+          }
+        }
+      }
+    }
+  }
+  return nrm;
+}
+
 template <int MODE, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(320, 1)
     k_gemm_pp(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
@@ -718,8 +855,10 @@ __global__ void __launch_bounds__(320, 1)
       // an off-diagonal tile of a symmetric result also writes its mirror image
       // and counts twice in ||R||^2
       const bool mirror = sym && tn != tm;
-      float nrm = epilogue_tile<false, 16>(st, tmem + static_cast<uint32_t>(u * BN), ep, b, m0,
-                                          n0, BN, q, h, lane, mirror);
+      float nrm = ep.vec ? epilogue_lane_rows(tmem + static_cast<uint32_t>(u * BN), ep, b, m0, n0,
+                                              q, h, lane, mirror)
+                         : epilogue_tile<false, 16>(st, tmem + static_cast<uint32_t>(u * BN), ep, b,
+                                                    m0, n0, BN, q, h, lane, mirror);
       if (mirror) nrm *= 2.f;
       tc_fence_before();
       __syncwarp();
@@ -801,11 +940,36 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMa
   return cudaLaunchKernelEx(&cfg, kern, a, al, b, bl, K, BN, ep);
 }
 
+// The lane-per-row epilogue applies: a bf16 result (and out2, if any) with no
+// plain fp32 copy, and every row the epilogue reads or writes starting on a
+// 16-byte boundary (base pointers aligned, row and batch strides whole
+// multiples of 16 bytes in each buffer's element size).
+bool lane_rows_ok(const EpiParams& ep) {
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  auto st = [](int64_t ld, int64_t bs, int esz) {
+    return (ld * esz) % 16 == 0 && (bs * esz) % 16 == 0;
+  };
+  if (ep.out_fmt != OUT_BF16 || ep.out_plain != nullptr) return false;
+  if (!al(ep.out_hi) || !st(ep.ldo, ep.bso, 2)) return false;
+  if (ep.out2_hi != nullptr && !al(ep.out2_hi)) return false;
+  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;
+  const bool need_old = ep.kind == EPI_EMA || ep.kind == EPI_APPLY || ep.kind == EPI_MOMENTUM;
+  if (need_old) return false;  // read-modify-write kinds keep fp32 storage
+  if (need_aux) {
+    const int ea = ep.aux_fmt == OUT_BF16 ? 2 : 4;
+    if (!al(ep.aux_hi) || !st(ep.lda_aux, ep.bs_aux, ea)) return false;
+    if (ep.aux_fmt == OUT_SPLIT && !al(ep.aux_lo)) return false;
+  }
+  return true;
+}
+
 template <int MODE, bool AMN, bool BMN>
 cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtensorMap& b,
-                      const CUtensorMap& bl, int M, int N, int K, int batch, const EpiParams& ep,
+                      const CUtensorMap& bl, int M, int N, int K, int batch, const EpiParams& ep_in,
                       cudaStream_t st) {
   using C = Cfg<MODE, true>;
+  EpiParams ep = ep_in;
+  ep.vec = lane_rows_ok(ep) ? 1 : 0;
   constexpr int SMEM = 1024 + C::PP_STAGES * C::STAGE_BYTES + 8 * 32 * 33 * 4 + 320;
   static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
   auto kern = k_gemm_pp<MODE, AMN, BMN>;

@@ -95,6 +95,9 @@ struct EpiParams {
   // bounded-wait self-test (persistent kernel): the producer first waits on a
   // barrier nothing completes; status[0] receives ST_ETIMEOUT
   int selftest;
+  // set by the persistent kernel's launcher: a bf16 result whose rows (and
+  // aux rows) start on 16-byte boundaries takes the lane-per-row epilogue
+  int vec;
 };
 
 // C[b] (M x N) = A[b] (M x K) * B[b] (K x N) on tcgen05 tensor cores,
