@@ -660,10 +660,121 @@ SHP_DEV float epilogue_lane_rows(uint32_t tmem, const EpiParams& ep, int b, int 
   return nrm;
 }
 
+// Byte offset of 16-byte group g of row r in a box of 64-byte rows stored
+// with the tensor maps' 64-byte swizzle (address bits 4-5 XOR bits 7-8).
+SHP_DEV uint32_t sw64_off(int r, int g) {
+  return static_cast<uint32_t>(r * 64 + ((g ^ ((r >> 1) & 3)) << 4));
+}
+
+// The lane-per-row epilogue with bulk-tensor (TMA) traffic, for bf16 results
+// with no out2 and bf16 or no aux (ep.vec == 2): per 32-column chunk, each
+// lane packs its row's 32 results into the warp's 32 x 32 bf16 box `wbuf`
+// (64-byte swizzle: conflict-free, four 16-byte stores per lane) and lane 0
+// stores the box with one tensor store (tO), which also clips rows and
+// columns outside the matrix.  The aux box arrives in `wbuf + 2048` by tensor
+// load (tX) on the warp's barrier `abar`, one chunk ahead: the caller issues
+// the tile's first chunk, each chunk issues the next.  `apar` is the
+// barrier's phase; `pending` tracks a load in flight (drained before exit).
+// The caller runs it only for warps with rows inside the matrix (no tensor
+// access starts past the last row).  Returns this lane's sum of squares
+// (RESID), or sets `stop` if a wait gave up.
+SHP_DEV float epilogue_rows_tma(uint32_t tmem, const CUtensorMap* tO, const CUtensorMap* tX,
+                                uint8_t* wbuf, uint64_t* abar, uint32_t& apar, bool& pending,
+                                const EpiParams& ep, int b, int m0, int n0, int q, int h,
+                                int lane, bool mirror, volatile int* abort_flag, bool& stop) {
+  const float alpha = ep.alpha != nullptr ? ep.alpha[b] : 0.f;  // GPOLY
+  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;
+  const int row0 = m0 + q * 32;
+  const int row = row0 + lane;
+  const int vrows = row < ep.M ? 8 : 0;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  uint8_t* obuf = wbuf;
+  uint8_t* xbuf = wbuf + 2048;
+  float nrm = 0.f;
+  for (int c = h; c < 8; c += 2) {
+    const int cb = n0 + c * 32;
+    if (cb >= ep.N) break;
+    float a[32];
+    tmem_ld32(trow + static_cast<uint32_t>(c * 32), a);  // the whole warp
+    float x[32];
+    if (need_aux) {
+      if (!mbar_wait(abar, apar, abort_flag)) {
+        stop = true;
+        return nrm;
+      }
+      apar ^= 1u;
+      pending = false;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const uint4 u = *reinterpret_cast<const uint4*>(xbuf + sw64_off(lane, g));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          x[8 * g + 2 * i] = __uint_as_float(w[i] << 16);
+          x[8 * g + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+      }
+      __syncwarp();  // every lane has read the box
+      const int cn = c + 2;
+      if (cn < 8 && n0 + cn * 32 < ep.N) {
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(abar, 2048);
+          tma_load_3d(xbuf, tX, abar, n0 + cn * 32, row0, b);
+        }
+        pending = true;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = 0.f;
+    }
+    float v[32];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int nv = ep.N - cb - 8 * g;  // columns of this group inside the matrix
+      float w0[8], v2[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w0[j] = 0.f;
+      nrm += epi_rows<8>(ep, a + 8 * g, x + 8 * g, w0, row - cb - 8 * g,
+                         nv < vrows ? (nv > 0 ? nv : 0) : vrows, alpha, 1.f, v + 8 * g, v2);
+    }
+    if (lane == 0) bulk_wait_read_all();  // the previous store has read obuf
+    __syncwarp();
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 t = __floats2bfloat162_rn(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&t);
+      }
+      *reinterpret_cast<uint4*>(obuf + sw64_off(lane, g)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(tO, obuf, cb, row0, b);
+      bulk_commit();
+    }
+    if (mirror && row < ep.M) {
+      // the image of column cb + j is row cb + j; lanes write its
+      // consecutive columns row0 + lane (a mirrored tile holds no diagonal)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (cb + j < ep.N)
+          put(OUT_BF16, ep.out_hi, nullptr,
+              static_cast<int64_t>(b) * ep.bso + static_cast<int64_t>(cb + j) * ep.ldo + row, v[j]);
+      }
+    }
+  }
+  return nrm;
+}
+
 template <int MODE, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(320, 1)
     k_gemm_pp(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tAl,
               const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tBl,
+              const __grid_constant__ CUtensorMap tO, const __grid_constant__ CUtensorMap tX,
               int K, EpiParams ep, int batch) {
   count_kernel_run();
   using C = Cfg<MODE, true>;
@@ -687,8 +798,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;  // all MMAs of this pair complete (before TMEM is freed)
   uint64_t* never = drain + 1;  // completed by nothing: the self-test's wait
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(never + 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1) + 1;
+  uint64_t* auxb = never + 1;   // per epilogue warp: its aux box has landed (ep.vec == 2)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(auxb + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxb + 8) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -702,6 +814,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(drain, 1);
     mbar_init(never, 1);
+    for (int w = 0; w < 8; ++w) mbar_init(&auxb[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tA);
@@ -836,11 +949,31 @@ __global__ void __launch_bounds__(320, 1)
     // ---------------- epilogue warps 2..9 (both CTAs, each on its TMEM rows)
     const int q = warp & 3, h = (warp - 2) >> 2;
     float* st = stage_epi + (warp - 2) * (32 * 33);
+    // the bulk-tensor epilogue's 4 KB per warp (out box, aux box) in the same region
+    uint8_t* wbuf = reinterpret_cast<uint8_t*>(stage_epi) + (warp - 2) * 4096;
+    uint64_t* abar = &auxb[warp - 2];
+    const bool tma_epi = ep.vec == 2;
+    const bool aux_tma = tma_epi && (ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY);
+    uint32_t apar = 0;
+    bool pending = false;
     int tl = 0;
     for (int t = cl; t < ntiles; t += ncl) {
       const int b = t / per_b, r = t % per_b;
       if (ep.active != nullptr && ep.active[b] == 0) continue;
       const int u = tl & 1, use = tl >> 1;
+      int tm, tn;
+      tile_coords(r, tiles_n, sym, tm, tn);
+      const int m0 = tm * 256 + static_cast<int>(rank) * 128;
+      const int n0 = tn * BN;
+      // rows of this warp inside the matrix (tensor traffic only for those)
+      const bool rows_in = m0 + q * 32 < ep.M;
+      if (aux_tma && rows_in && n0 + h * 32 < ep.N) {  // the first aux box, during the wait
+        if (lane == 0) {
+          mbar_arrive_expect_tx(abar, 2048);
+          tma_load_3d(wbuf + 2048, &tX, abar, n0 + h * 32, m0 + q * 32, b);
+        }
+        pending = true;
+      }
       if (*abort_flag || !mbar_wait(&accf[u], use & 1, abort_flag)) {
         *abort_flag = 1;
         if (lane == 0 && ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
@@ -848,17 +981,28 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
       tc_fence_after();
-      int tm, tn;
-      tile_coords(r, tiles_n, sym, tm, tn);
-      const int m0 = tm * 256 + static_cast<int>(rank) * 128;
-      const int n0 = tn * BN;
       // an off-diagonal tile of a symmetric result also writes its mirror image
       // and counts twice in ||R||^2
       const bool mirror = sym && tn != tm;
-      float nrm = ep.vec ? epilogue_lane_rows(tmem + static_cast<uint32_t>(u * BN), ep, b, m0, n0,
-                                              q, h, lane, mirror)
-                         : epilogue_tile<false, 16>(st, tmem + static_cast<uint32_t>(u * BN), ep, b,
-                                                    m0, n0, BN, q, h, lane, mirror);
+      float nrm;
+      if (tma_epi && !rows_in) {
+        nrm = 0.f;
+      } else if (tma_epi) {
+        bool stop = false;
+        nrm = epilogue_rows_tma(tmem + static_cast<uint32_t>(u * BN), &tO, &tX, wbuf, abar, apar,
+                                pending, ep, b, m0, n0, q, h, lane, mirror, abort_flag, stop);
+        if (stop) {
+          *abort_flag = 1;
+          if (lane == 0 && ep.status != nullptr) atomicExch(&ep.status[b], ST_ETIMEOUT);
+          break;
+        }
+      } else if (ep.vec) {
+        nrm = epilogue_lane_rows(tmem + static_cast<uint32_t>(u * BN), ep, b, m0, n0, q, h, lane,
+                                 mirror);
+      } else {
+        nrm = epilogue_tile<false, 16>(st, tmem + static_cast<uint32_t>(u * BN), ep, b, m0, n0, BN,
+                                       q, h, lane, mirror);
+      }
       if (mirror) nrm *= 2.f;
       tc_fence_before();
       __syncwarp();
@@ -868,6 +1012,14 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) atomicAdd(&ep.norm2[static_cast<int64_t>(b) * ep.norm2_stride], nrm);
       }
       ++tl;
+    }
+    if (tma_epi) {
+      // nothing of this warp's bulk traffic may outlive the CTA: a tensor load
+      // left in flight by a wait that gave up lands first (bounded wait), and
+      // the tensor stores complete
+      if (pending) mbar_wait(abar, apar);
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
   }
 
@@ -970,6 +1122,18 @@ cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtenso
   using C = Cfg<MODE, true>;
   EpiParams ep = ep_in;
   ep.vec = lane_rows_ok(ep) ? 1 : 0;
+  // bf16 result boxes of 32 x 32 by tensor store (and bf16 aux boxes by
+  // tensor load) when there is no second output and no non-bf16 aux
+  CUtensorMap tO, tX;
+  memset(&tO, 0, sizeof(tO));
+  memset(&tX, 0, sizeof(tX));
+  const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;
+  if (ep.vec && ep.out2_hi == nullptr && ep.kind != EPI_MOMENTUM &&
+      (!need_aux || ep.aux_fmt == OUT_BF16) &&
+      make_map(&tO, ep.out_hi, 2, N, M, batch, ep.ldo, ep.bso, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
+      (!need_aux || make_map(&tX, ep.aux_hi, 2, N, M, batch, ep.lda_aux, ep.bs_aux, 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_64B)))
+    ep.vec = 2;
   constexpr int SMEM = 1024 + C::PP_STAGES * C::STAGE_BYTES + 8 * 32 * 33 * 4 + 320;
   static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
   auto kern = k_gemm_pp<MODE, AMN, BMN>;
@@ -995,7 +1159,7 @@ cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtenso
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, al, b, bl, K, ep, batch);
+  return cudaLaunchKernelEx(&cfg, kern, a, al, b, bl, tO, tX, K, ep, batch);
 }
 
 template <int MODE>
