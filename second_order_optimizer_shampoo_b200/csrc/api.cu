@@ -156,6 +156,7 @@ struct PolarBufs {
   float* Rhi;
   float* Rlo;
   float* Rs;  // plain fp32 R read by the sketch passes
+  uint16_t* Rb;  // bf16 copy of R, the operands of R R (bf16 storage)
   void* ghi;
   float* glo;
   float* V;
@@ -176,6 +177,7 @@ PolarBufs carve_polar(Arena& a, int64_t m, int64_t n, int64_t batch, int storage
   b.Rhi = a.take<float>(kk);
   b.Rlo = split ? a.take<float>(kk) : nullptr;
   b.Rs = split ? a.take<float>(kk) : b.Rhi;
+  b.Rb = bf ? a.take<uint16_t>(kk) : nullptr;
   b.ghi = bf ? static_cast<void*>(a.take<uint16_t>(kk)) : static_cast<void*>(a.take<float>(kk));
   b.glo = split ? a.take<float>(kk) : nullptr;
   b.V = a.take<float>(static_cast<size_t>(2 * o->d + 2) * k * o->p * batch);
@@ -1167,7 +1169,10 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
     const int64_t k = tall ? n : m;  // Gram size
     const int xmode = bf ? MODE_BF16 : (storage == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32);
     const int xfmt = bf ? OUT_BF16 : (storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32);
-    const int rmode = bf ? MODE_TF32 : xmode;  // R and R^2
+    // R R: bf16 storage multiplies the bf16 copy of R (fp32 accumulation,
+    // as the iterate's own products); R itself stays fp32 for R/2 and the
+    // sketch
+    const int rmode = xmode;
     const int rfmt = storage == SHP_3XTF32 ? OUT_SPLIT : OUT_F32;
     const int M = static_cast<int>(m), N = static_cast<int>(n), K = static_cast<int>(k);
     const int B = static_cast<int>(batch);
@@ -1185,6 +1190,7 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
       {  // R = I - X^T X (tall) or I - X X^T (wide), and ||R||_F^2
         EpiParams e = epi(EPI_RESID, rfmt, w.Rhi, w.Rlo, k, kk, K, K, &ctl);
         if (rfmt == OUT_SPLIT) e.out_plain = w.Rs;
+        e.out_b16 = w.Rb;
         // X^T X is a Gram matrix, symmetric in any arithmetic: upper-triangle
         // tiles, mirrored.  X X (sign) is symmetric only while X is, and X
         // picks up a rounding-level asymmetry from X + X Delta: keeping one
@@ -1218,8 +1224,12 @@ int polar_impl(const void* G, int storage, int64_t m, int64_t n, int64_t batch,
         e.lda_aux = k;
         e.bs_aux = kk;
         e.s1 = 0.5f;
-        CK(gemm_tc(rmode, op(w.Rhi, w.Rlo, false, k, kk), op(w.Rhi, w.Rlo, true, k, kk), K, K,
-                   K, B, e, st));
+        if (bf)
+          CK(gemm_tc(rmode, op(w.Rb, nullptr, false, k, kk), op(w.Rb, nullptr, true, k, kk), K, K,
+                     K, B, e, st));
+        else
+          CK(gemm_tc(rmode, op(w.Rhi, w.Rlo, false, k, kk), op(w.Rhi, w.Rlo, true, k, kk), K, K,
+                     K, B, e, st));
       } else {
         CK(gform_d1(w.Rhi, w.Rlo, k, B, ctl, xfmt, w.ghi, w.glo, nullptr, nullptr, st));
       }

@@ -267,6 +267,8 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
           store_rows<RP>(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, ep.ldo, v2, nrows);
         if (ep.out_plain != nullptr)
           store_rows<RP>(OUT_F32, ep.out_plain, nullptr, off, ep.ldo, v, nrows);
+        if (ep.out_b16 != nullptr)
+          store_rows<RP>(OUT_BF16, ep.out_b16, nullptr, off, ep.ldo, v, nrows);
         if (mirror) {
 #pragma unroll
           for (int r = 0; r < RP; ++r) st[(r0 + r) * 33 + lane] = v[r];
@@ -289,6 +291,7 @@ SHP_DEV float epilogue_tile(float* st, uint32_t tmem, const EpiParams& ep, int b
           // a mirrored tile holds no diagonal element, so out2 = I + v is v here
           if (ep.out2_hi != nullptr) put(ep.out_fmt, ep.out2_hi, ep.out2_lo, off, v);
           if (ep.out_plain != nullptr) ep.out_plain[off] = v;
+          if (ep.out_b16 != nullptr) put(OUT_BF16, ep.out_b16, nullptr, off, v);
         }
       }
       __syncwarp();
@@ -1101,7 +1104,7 @@ bool lane_rows_ok(const EpiParams& ep) {
   auto st = [](int64_t ld, int64_t bs, int esz) {
     return (ld * esz) % 16 == 0 && (bs * esz) % 16 == 0;
   };
-  if (ep.out_fmt != OUT_BF16 || ep.out_plain != nullptr) return false;
+  if (ep.out_fmt != OUT_BF16 || ep.out_plain != nullptr || ep.out_b16 != nullptr) return false;
   if (!al(ep.out_hi) || !st(ep.ldo, ep.bso, 2)) return false;
   if (ep.out2_hi != nullptr && !al(ep.out2_hi)) return false;
   const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;

@@ -74,6 +74,7 @@ struct EpiParams {
   void* out2_hi;
   float* out2_lo;
   float* out_plain;  // optional plain fp32 copy of v (same layout as out)
+  void* out_b16;     // optional bf16 copy of v (same layout as out)
   int64_t ldo, bso;
   const void* aux_hi;
   const float* aux_lo;
@@ -89,7 +90,7 @@ struct EpiParams {
   // The result is symmetric (M == N; any kind but MOMENTUM, whose out2 is not
   // of the form I + v): the persistent kernel computes the tiles on and above
   // the diagonal and writes each off-diagonal tile's mirror image too (to out,
-  // out2 and out_plain); other kernels compute it all.  Read-modify-write and
+  // out2, out_plain and out_b16); other kernels compute it all.  Read-modify-write and
   // aux operands are read on the upper tiles only, so they must be symmetric.
   int sym;
   // bounded-wait self-test (persistent kernel): the producer first waits on a
