@@ -446,7 +446,9 @@ def shampoo_only(args):
 def shampoo_step_leg(args, dev, stream, host_loop=False, reps=10):
     """One Shampoo step on a 1024 x 1024 weight: 10 EMA steps of L and R with
     fresh G (TF32), L^(-1/4) and R^(-1/4) by PRISM (d = 2, p = 8, tol 1e-3,
-    TF32) as one batch of two, and W -= 1e-3 L^(-1/4) G R^(-1/4)."""
+    TF32) as one batch of two, and W -= 1e-3 L^(-1/4) G R^(-1/4).  The ten
+    gradients are all given, so the EMA steps go through one
+    shampoo_gram_ema_steps call; the ten one-step calls are timed beside it."""
     import torch
 
     from second_order_optimizer_shampoo_b200 import _abi, prism, synth
@@ -463,12 +465,22 @@ def shampoo_step_leg(args, dev, stream, host_loop=False, reps=10):
     ws = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_INV_ROOT, n, n, 2, opts),
                      dtype=torch.uint8, device=dev)
     eye = torch.eye(n, device=dev) * eps
+    Gst = torch.stack(Gs)  # [10][1][n][n]
+    ws_ema = torch.empty(prism.shp_workspace_bytes(_abi.SHP_OP_GRAM_EMA_STEPS, n, n, 10,
+                                                   prism.make_opts(prec="tf32")),
+                         dtype=torch.uint8, device=dev)
+
+    def ema_steps():
+        prism.shampoo_gram_ema_steps(Gst, LR[0:1], LR[1:2], beta, eps, "tf32", ws=ws_ema)
+
+    def ema_one_step_calls():
+        for G in Gs:
+            prism.shampoo_gram_ema(G, LR[0:1], LR[1:2], beta, eps, "tf32")
 
     def step():
         LR.copy_(eye.expand(2, n, n))
         W.copy_(W0)
-        for G in Gs:
-            prism.shampoo_gram_ema(G, LR[0:1], LR[1:2], beta, eps, "tf32")
+        ema_steps()
         prism.matfn_inv_root(LR, "inv4", opts, S, out=roots, ws=ws, report=rep)
         prism.shampoo_apply(W, Gs[-1], roots[0:1], roots[1:2], lr, "tf32")
 
@@ -477,10 +489,13 @@ def shampoo_step_leg(args, dev, stream, host_loop=False, reps=10):
     torch.cuda.synchronize()
     iters = rep["iters"].cpu().numpy()
     ms = _time(step, stream, reps)
+    ms_ema_steps = _time(ema_steps, stream, reps)
+    ms_ema_calls = _time(ema_one_step_calls, stream, reps)
     flops = 10 * 2 * n * (n + 1) * n + sum(block_flops(blk, n) for blk in iters) + 2 * 2.0 * n ** 3
     return {"workload": "shampoo_step_1024sq_ema10_inv4_d2_p8_tf32_apply", "ms_per_step": ms,
             "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
             "preconditioners_per_s": 2 / (ms / 1e3),
+            "ema10_steps_call_ms": ms_ema_steps, "ema10_one_step_calls_ms": ms_ema_calls,
             "iters_per_pass": [[int(k) for k in blk] for blk in iters],
             "status": [int(x) for x in rep["status"].cpu().numpy()],
             "note": "EMA products counted n(n+1)n (symmetric results, formed on their "

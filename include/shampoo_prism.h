@@ -76,7 +76,7 @@ typedef enum {
 } shp_power;
 
 typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_OP_APPLY = 3,
-               SHP_OP_GRAM_EMA = 4 } shp_op;
+               SHP_OP_GRAM_EMA = 4, SHP_OP_GRAM_EMA_STEPS = 5 } shp_op;
 
 /* Knobs of a PRISM Newton-Schulz pass ([PRISM] Parte I-II).
  *   d           degree of g_d; 1 or 2
@@ -153,6 +153,23 @@ size_t shp_workspace_bytes(int op, int64_t m, int64_t n, int64_t batch,
 int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float* L, float* R,
                      float beta, float eps, int prec, void* ws, size_t ws_bytes,
                      shp_stream stream);
+
+/* `count` successive EMA steps of the Kronecker factors, one per gradient of
+ * the stack G: [count][batch][m][n] fp32 ([Shampoo] 2.3 step 2 applied for
+ * t = 1 .. count):
+ *   L <- beta L + (1 - beta) G_t G_t^T + eps I,  R <- beta R + (1 - beta) G_t^T G_t + eps I.
+ * The result equals `count` calls of shampoo_gram_ema with G_1 .. G_count up
+ * to rounding order: every product G_t G_t^T is formed as that call forms it
+ * (one batched launch over t and the blocks), then the recurrence is replayed
+ * element by element in fp32.  For training loops that hold several
+ * gradients at once (accumulated micro-batches, a replayed window).
+ * count * batch <= 65535.  Workspace: shp_workspace_bytes(SHP_OP_GRAM_EMA_STEPS,
+ * m, n, count * batch, opts with prec) -- the products of both factors (and
+ * the split G for SHP_3XTF32).  L, R, prec, NULL factors and errors as in
+ * shampoo_gram_ema. */
+int shampoo_gram_ema_steps(const float* G, int64_t count, int64_t m, int64_t n, int64_t batch,
+                           float* L, float* R, float beta, float eps, int prec, void* ws,
+                           size_t ws_bytes, shp_stream stream);
 
 /* Matrix power of a batch of SPD matrices by coupled Newton-Schulz with PRISM
  * alpha ([PRISM] Parte I-II; [Shampoo] 2.3 step 3 and 3.1):

@@ -21,6 +21,7 @@ SHP_TF32, SHP_3XTF32, SHP_BF16, SHP_OZAKI = 0, 1, 2, 3
 SHP_POW_INV4, SHP_POW_INV2, SHP_POW_SQRT = 0, 1, 2
 # workspace queries
 SHP_OP_INV_ROOT, SHP_OP_POLAR, SHP_OP_ALPHA_FIT, SHP_OP_APPLY, SHP_OP_GRAM_EMA = 0, 1, 2, 3, 4
+SHP_OP_GRAM_EMA_STEPS = 5
 # shp_matmul_f64_ex flags
 SHP_MATMUL_REUSE_A, SHP_MATMUL_REUSE_B, SHP_MATMUL_ACCUMULATE = 1, 2, 4
 # bounded-wait self-test
@@ -29,7 +30,7 @@ SHP_SELFTEST_WS_BYTES = 4 << 20
 # fixed device scratch of prism_alpha_fit_noalloc
 SHP_NOALLOC_SCRATCH_BYTES = 4 << 20
 
-EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "matfn_inv_root", "matfn_polar", "matfn_polar_varsize",
+EXPORTS = ("shp_workspace_bytes", "shampoo_gram_ema", "shampoo_gram_ema_steps", "matfn_inv_root", "matfn_polar", "matfn_polar_varsize",
            "matfn_sign",
            "prism_alpha_fit", "shampoo_apply", "shampoo_apply_ex", "shp_matmul", "shp_split_tf32",
            "shp_matmul_f64_workspace_bytes", "shp_matmul_f64", "shp_matmul_f64_ex",
@@ -63,6 +64,8 @@ _INT = ctypes.c_int
 _SIGS = {
     "shp_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64, ctypes.POINTER(PrismOpts)]),
     "shampoo_gram_ema": (_INT, [_P, _I64, _I64, _I64, _P, _P, _F, _F, _INT, _P, _SZ, _P]),
+    "shampoo_gram_ema_steps": (_INT, [_P, _I64, _I64, _I64, _I64, _P, _P, _F, _F, _INT, _P, _SZ,
+                                      _P]),
     "matfn_inv_root": (_INT, [_P, _I64, _I64, _INT, ctypes.POINTER(PrismOpts), _P, _I64, _P,
                               ctypes.POINTER(PrismReport), _P, _SZ, _P]),
     "matfn_polar": (_INT, [_P, _INT, _I64, _I64, _I64, ctypes.POINTER(PrismOpts), _P, _I64, _P,

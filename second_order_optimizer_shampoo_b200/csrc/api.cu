@@ -529,6 +529,13 @@ size_t shp_workspace_bytes(int opk, int64_t m, int64_t n, int64_t batch,
       if (prec == SHP_3XTF32) a.take<float>(static_cast<size_t>(m) * n * batch * 2);
       break;
     }
+    case SHP_OP_GRAM_EMA_STEPS: {  // batch = count x blocks
+      const int prec = o != nullptr ? o->prec : SHP_3XTF32;
+      if (prec == SHP_3XTF32) a.take<float>(static_cast<size_t>(m) * n * batch * 2);
+      a.take<float>(static_cast<size_t>(m) * m * batch);  // the products G G^T
+      a.take<float>(static_cast<size_t>(n) * n * batch);  // and G^T G
+      break;
+    }
     default:
       return 0;
   }
@@ -577,6 +584,55 @@ int shampoo_gram_ema(const float* G, int64_t m, int64_t n, int64_t batch, float*
     e.sym = 1;
     CK(gemm_tc(mode, op(Ghi, Glo, true, n, m * n), op(Ghi, Glo, true, n, m * n), N, N, M, B, e,
                st));
+  }
+  return SHP_OK;
+}
+
+int shampoo_gram_ema_steps(const float* G, int64_t count, int64_t m, int64_t n, int64_t batch,
+                           float* L, float* R, float beta, float eps, int prec, void* ws,
+                           size_t ws_bytes, shp_stream stream) {
+  if (G == nullptr || count <= 0 || m <= 0 || n <= 0 || batch <= 0 || m % 4 || n % 4)
+    return SHP_EINVAL;
+  if (!aligned16(G) || (L && !aligned16(L)) || (R && !aligned16(R))) return SHP_EINVAL;
+  if (prec != SHP_TF32 && prec != SHP_3XTF32) return SHP_EINVAL;
+  if (!isfinite(beta) || !isfinite(eps)) return SHP_EINVAL;
+  if (m > INT32_MAX || n > INT32_MAX || count > 65535 || count * batch > 65535)
+    return SHP_EUNSUPPORTED;
+  const int64_t cb = count * batch;
+  shp_prism_opts o{};
+  o.prec = prec;
+  if (ws == nullptr || ws_bytes < shp_workspace_bytes(SHP_OP_GRAM_EMA_STEPS, m, n, cb, &o))
+    return SHP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena a(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~(kAlign - 1)));
+  const float* Ghi = G;
+  const float* Glo = nullptr;
+  if (prec == SHP_3XTF32) {
+    float* hi = a.take<float>(static_cast<size_t>(m) * n * cb);
+    float* lo = a.take<float>(static_cast<size_t>(m) * n * cb);
+    CK(split_copy(G, m * n * cb, hi, lo, st));
+    Ghi = hi;
+    Glo = lo;
+  }
+  float* PL = a.take<float>(static_cast<size_t>(m) * m * cb);
+  float* PR = a.take<float>(static_cast<size_t>(n) * n * cb);
+  const int mode = prec == SHP_3XTF32 ? MODE_3XTF32 : MODE_TF32;
+  const int M = static_cast<int>(m), N = static_cast<int>(n), CB = static_cast<int>(cb);
+  // every step's product in one batched launch (each formed exactly as the
+  // one-step call forms it), then the recurrence replayed element by element
+  if (L != nullptr) {
+    EpiParams e = epi(EPI_STORE, OUT_F32, PL, nullptr, m, m * m, M, M, nullptr);
+    e.sym = 1;
+    CK(gemm_tc(mode, op(Ghi, Glo, false, n, m * n), op(Ghi, Glo, false, n, m * n), M, M, N, CB, e,
+               st));
+    CK(ema_replay(L, PL, m, static_cast<int>(count), static_cast<int>(batch), beta, eps, st));
+  }
+  if (R != nullptr) {
+    EpiParams e = epi(EPI_STORE, OUT_F32, PR, nullptr, n, n * n, N, N, nullptr);
+    e.sym = 1;
+    CK(gemm_tc(mode, op(Ghi, Glo, true, n, m * n), op(Ghi, Glo, true, n, m * n), N, N, M, CB, e,
+               st));
+    CK(ema_replay(R, PR, n, static_cast<int>(count), static_cast<int>(batch), beta, eps, st));
   }
   return SHP_OK;
 }

@@ -237,6 +237,47 @@ __global__ void __launch_bounds__(EW_THREADS)
   }
 }
 
+// The EMA recurrence of the Kronecker factors replayed element by element
+// over precomputed products: L <- beta L + (1 - beta) P_t + eps [i == j] for
+// t = 0 .. count-1, P: [count][batch][n][n] (both triangles), 4 columns per
+// thread (n % 4 == 0).  The products of up to four steps are loaded before
+// they are folded in, so the loads overlap.
+__global__ void __launch_bounds__(EW_THREADS)
+    k_ema_replay(float* L, const float* P, int64_t n, int count, int64_t pstride, float beta,
+                 float eps) {
+  count_kernel_run();
+  const int b = blockIdx.y;
+  const int64_t nn = n * n, n4 = nn / 4;
+  float4* Lb = reinterpret_cast<float4*>(L + b * nn);
+  const float4* Pb = reinterpret_cast<const float4*>(P + b * nn);
+  const int64_t ps4 = pstride / 4;
+  const float w = 1.f - beta;
+  for (int64_t e4 = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e4 < n4;
+       e4 += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+    const int64_t e = 4 * e4, row = e / n, col = e % n;
+    const int dj = static_cast<int>(row - col);  // the diagonal sits at component dj, if in 0..3
+    const float ex = dj == 0 ? eps : 0.f, ey = dj == 1 ? eps : 0.f;
+    const float ez = dj == 2 ? eps : 0.f, ew = dj == 3 ? eps : 0.f;
+    float4 l = Lb[e4];
+    for (int t0 = 0; t0 < count; t0 += 4) {
+      float4 q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (t0 + u < count) q[u] = Pb[(t0 + u) * ps4 + e4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u < count) {
+          l.x = beta * l.x + w * q[u].x + ex;
+          l.y = beta * l.y + w * q[u].y + ey;
+          l.z = beta * l.z + w * q[u].z + ez;
+          l.w = beta * l.w + w * q[u].w + ew;
+        }
+      }
+    }
+    Lb[e4] = l;
+  }
+}
+
 __global__ void __launch_bounds__(EW_THREADS)
     k_polar_init(const void* G, int gbf16, int64_t count, Ctl ctl, int fmt, void* Xhi,
                  float* Xlo) {
@@ -345,6 +386,16 @@ cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_expone
 cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st) {
   if (count <= 0) return cudaSuccess;
   k_split<<<ew_grid(count, 1), EW_THREADS, 0, st>>>(X, count, hi, lo);
+  return cudaGetLastError();
+}
+
+cudaError_t ema_replay(float* L, const float* P, int64_t n, int count, int batch, float beta,
+                       float eps, cudaStream_t st) {
+  if (count <= 0 || batch <= 0) return cudaSuccess;
+  const int64_t n4 = n * n / 4;  // one float4 per thread
+  const dim3 grid(static_cast<unsigned>((n4 + EW_THREADS - 1) / EW_THREADS), batch);
+  k_ema_replay<<<grid, EW_THREADS, 0, st>>>(
+      L, P, n, count, static_cast<int64_t>(batch) * n * n, beta, eps);
   return cudaGetLastError();
 }
 

@@ -220,6 +220,10 @@ cudaError_t coupled_finish(int64_t n, int batch, const Ctl& ctl, double c_expone
                            const float* const* Shi, const float* const* Slo, float* X_out,
                            bool z_slots, cudaStream_t st);
 // hi = tf32(X), lo = X - hi.
+// L[b] <- beta L[b] + (1 - beta) P[t][b] + eps I for t = 0 .. count-1 in
+// turn (the EMA recurrence over precomputed products P: [count][batch][n][n]).
+cudaError_t ema_replay(float* L, const float* P, int64_t n, int count, int batch, float beta,
+                       float eps, cudaStream_t st);
 cudaError_t split_copy(const float* X, int64_t count, float* hi, float* lo, cudaStream_t st);
 // X0 = G / ||G||_F (uses dnorm) in `fmt`.
 cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, const Ctl& ctl,

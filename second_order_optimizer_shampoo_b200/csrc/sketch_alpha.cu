@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
   }
 }
 
-constexpr int AL_THREADS = 256;
+constexpr int AL_THREADS = 512;
 
 // Per-block alpha of one iteration.  Without adaptive degree: the Gram of
 // V_d..V_{2d+1}, the quartic and its minimiser on [lo, hi].  With adaptive
@@ -409,29 +409,33 @@ struct AlphaArgs {
 
 // This thread's partial sums of <V_i, V_j> (i <= j < NV, packed row by row)
 // over elements threadIdx.x + k * AL_THREADS; NV is a compile-time constant so
-// that the 15 partials and the loaded values stay in registers, and two
-// elements are loaded per step to keep 2 NV loads in flight.
+// that the 15 partials and the loaded values stay in registers.  Four
+// elements are loaded per step (4 NV loads in flight): the sums are short
+// (n p elements per block) and their cost is the load latency, not the fp64
+// arithmetic.
 template <int NV>
 SHP_DEV void gram_partials(const float* __restrict__ Vb, int64_t len, double (&part)[15]) {
 #pragma unroll
   for (int i = 0; i < 15; ++i) part[i] = 0.0;
+  constexpr int U = 4;
   int64_t e = threadIdx.x;
-  for (; e + AL_THREADS < len; e += 2 * AL_THREADS) {
-    float x[NV], y[NV];
+  for (; e + (U - 1) * AL_THREADS < len; e += U * AL_THREADS) {
+    float x[U][NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      x[i] = __ldg(Vb + i * len + e);
-      y[i] = __ldg(Vb + i * len + e + AL_THREADS);
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) x[u][i] = __ldg(Vb + i * len + e + u * AL_THREADS);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      int idx = 0;
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int j = i; j < NV; ++j, ++idx)
+          part[idx] = fma(static_cast<double>(x[u][i]), static_cast<double>(x[u][j]), part[idx]);
     }
-    int idx = 0;
-#pragma unroll
-    for (int i = 0; i < NV; ++i)
-#pragma unroll
-      for (int j = i; j < NV; ++j, ++idx)
-        part[idx] = fma(static_cast<double>(x[i]), static_cast<double>(x[j]),
-                        fma(static_cast<double>(y[i]), static_cast<double>(y[j]), part[idx]));
   }
-  if (e < len) {
+  for (; e < len; e += AL_THREADS) {
     float x[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) x[i] = __ldg(Vb + i * len + e);

@@ -86,6 +86,22 @@ def shampoo_gram_ema(G, L, R, beta: float, eps: float, prec: str = "tf32", ws=No
                                     _p(ws), ws.numel(), _stream()), "shampoo_gram_ema")
 
 
+def shampoo_gram_ema_steps(G, L, R, beta: float, eps: float, prec: str = "tf32", ws=None):
+    """count successive EMA steps, one per gradient of G: [count][batch][m][n]
+    (or [count][m][n]): L <- beta L + (1-beta) G_t G_t^T + eps I and
+    R <- beta R + (1-beta) G_t^T G_t + eps I for t = 1..count (in place)."""
+    _dev(G, L, R)
+    m, n = G.shape[-2], G.shape[-1]
+    count = G.shape[0]
+    batch = G.numel() // (count * m * n)
+    o = make_opts(prec=prec)
+    need = shp_workspace_bytes(A.SHP_OP_GRAM_EMA_STEPS, m, n, count * batch, o)
+    ws = _ws(need, G.device) if ws is None else ws
+    _check(A.lib().shampoo_gram_ema_steps(_p(G), count, m, n, batch, _p(L), _p(R), beta, eps,
+                                          _PREC[prec], _p(ws), ws.numel(), _stream()),
+           "shampoo_gram_ema_steps")
+
+
 def shampoo_apply(W, G, Lroot, Rroot, lr: float, prec: str = "tf32", ws=None):
     """W <- W - lr * Lroot G Rroot (in place)."""
     _dev(W, G, Lroot, Rroot)

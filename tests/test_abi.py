@@ -73,6 +73,11 @@ def test_workspace_sizes():
     assert L.shp_workspace_bytes(A.SHP_OP_INV_ROOT, n, n, batch, ctypes.byref(opts(d=3))) == 0
     assert L.shp_workspace_bytes(A.SHP_OP_INV_ROOT, n, n, batch, ctypes.byref(opts(p=33))) == 0
     assert L.shp_workspace_bytes(99, n, n, batch, ctypes.byref(o)) == 0
+    # several EMA steps at once: the products of both factors (plus split G)
+    we = L.shp_workspace_bytes(A.SHP_OP_GRAM_EMA_STEPS, 512, 256, 10, ctypes.byref(o1))
+    assert (512 * 512 + 256 * 256) * 4 * 10 <= we < (512 * 512 + 256 * 256) * 4 * 10 + (1 << 20)
+    we3 = L.shp_workspace_bytes(A.SHP_OP_GRAM_EMA_STEPS, 512, 256, 10, ctypes.byref(o))
+    assert we3 - we == 2 * 512 * 256 * 4 * 10
 
 
 def test_invalid_arguments_rejected_before_launch():
@@ -108,6 +113,14 @@ def test_invalid_arguments_rejected_before_launch():
     mis = ctypes.c_void_p(0x10004)
     assert L.shampoo_gram_ema(mis, 64, 64, 1, fake, fake, 0.9, 1e-6, A.SHP_TF32, fake, 1 << 30,
                               None) == A.SHP_EINVAL
+    assert L.shampoo_gram_ema_steps(fake, 0, 64, 64, 1, fake, fake, 0.9, 1e-6, A.SHP_TF32, fake,
+                                    1 << 30, None) == A.SHP_EINVAL
+    assert L.shampoo_gram_ema_steps(mis, 2, 64, 64, 1, fake, fake, 0.9, 1e-6, A.SHP_TF32, fake,
+                                    1 << 30, None) == A.SHP_EINVAL
+    assert L.shampoo_gram_ema_steps(fake, 2, 64, 64, 1, fake, fake, 0.9, 1e-6, A.SHP_TF32, fake,
+                                    16, None) == A.SHP_EINVAL  # workspace too small
+    assert L.shampoo_gram_ema_steps(fake, 300, 64, 64, 300, fake, fake, 0.9, 1e-6, A.SHP_TF32,
+                                    fake, 1 << 40, None) == A.SHP_EUNSUPPORTED
     assert L.shampoo_apply(fake, fake, fake, fake, 64, 62, 1, 1e-3, A.SHP_TF32, fake, 1 << 30,
                            None) == A.SHP_EINVAL
     assert L.shampoo_apply(fake, fake, fake, fake, 64, 64, 1, 1e-3, 5, fake, 1 << 30,

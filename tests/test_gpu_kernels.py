@@ -50,6 +50,48 @@ def test_gram_ema(prec, m, n, batch):
 
 
 @pytest.mark.parametrize("prec", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("m,n,batch,count", [(128, 128, 1, 10), (300, 196, 2, 3), (516, 260, 1, 1),
+                                             (1024, 1024, 1, 10)])
+def test_gram_ema_steps(prec, m, n, batch, count):
+    """count EMA steps in one call against the oracle's one-step recurrence
+    applied count times, element by element within the bound of the count
+    products (each weighted (1-beta) beta^(count-t)) and of the fp32
+    recurrence; and against count one-step GPU calls (same products, only the
+    order of the fp32 sums differs)."""
+    beta, eps = 0.95, 1e-3
+    G = synth.gaussian((count, batch, m, n), 1.0, 31)
+    L0 = synth.gaussian((batch, m, m), 0.1, 32)
+    L0 = (L0 + L0.transpose(0, 2, 1)).astype(np.float32)
+    R0 = synth.gaussian((batch, n, n), 0.1, 33)
+    R0 = (R0 + R0.transpose(0, 2, 1)).astype(np.float32)
+    P = prism()
+    Ld, Rd = to_dev(torch, L0), to_dev(torch, R0)
+    P.shampoo_gram_ema_steps(to_dev(torch, G), Ld, Rd, beta, eps, prec)
+    Lg, Rg = to_host(Ld), to_host(Rd)
+    L1, R1 = to_dev(torch, L0), to_dev(torch, R0)
+    for t in range(count):
+        P.shampoo_gram_ema(to_dev(torch, G[t]), L1, R1, beta, eps, prec)
+    L1, R1 = to_host(L1), to_host(R1)
+    for b in range(batch):
+        Lr, Rr = L0[b].astype(np.float64), R0[b].astype(np.float64)
+        bl = 4 * U_FP32 * count * np.abs(Lr)
+        br = 4 * U_FP32 * count * np.abs(Rr)
+        for t in range(count):
+            Lr, Rr = o.gram_ema_ref(G[t, b], Lr, Rr, beta, eps)
+            aG = np.abs(G[t, b].astype(np.float64))
+            w = (1 - beta) * beta ** (count - 1 - t)
+            bl = bl + w * gemm_bound(aG, aG.T, n, prec)
+            br = br + w * gemm_bound(aG.T, aG, m, prec)
+        bl = bl + 4 * U_FP32 * count * np.abs(Lr)
+        br = br + 4 * U_FP32 * count * np.abs(Rr)
+        assert np.all(np.abs(Lg[b] - Lr) <= bl), np.max(np.abs(Lg[b] - Lr) / bl)
+        assert np.all(np.abs(Rg[b] - Rr) <= br), np.max(np.abs(Rg[b] - Rr) / br)
+        # the one-step calls: identical products, recurrence in another order
+        assert np.max(np.abs(Lg[b] - L1[b])) <= 8 * U_FP32 * count * np.abs(Lr).max()
+        assert np.max(np.abs(Rg[b] - R1[b])) <= 8 * U_FP32 * count * np.abs(Rr).max()
+
+
+@pytest.mark.parametrize("prec", ["tf32", "3xtf32"])
 @pytest.mark.parametrize("m,n,batch", SHAPES)
 def test_apply(prec, m, n, batch):
     lr = 0.1
