@@ -49,9 +49,10 @@ TF32_OVER_BF16 = 1.1 / 2.25
 # dram__bytes_read.sum + dram__bytes_write.sum of one 3xTF32 persistent GEMM
 # launch (64 x 1024^3): an ncu capture of 16 blocks scaled x4 by the blocks
 GEMM_TRAFFIC_PER_LAUNCH = 4 * (290.093e6 + 43.367e6)
-# ... of one k_gemm_oz launch with the accumulate (X + X Delta) epilogue,
-# 64 x 1024^3: not captured for the current kernel
-OZ_GEMM_TRAFFIC_PER_LAUNCH = None
+# ... of one k_gemm_oz launch with the accumulate (C <- C + A B) epilogue,
+# 64 x 1024^3: an ncu capture of 16 products (302.37 MB read, 93.54 MB
+# written) scaled x4 by the products
+OZ_GEMM_TRAFFIC_PER_LAUNCH = 4 * (302.37e6 + 93.54e6)
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_sketch_tma<8> launch
 # over 48 x 1024^2 (201.393 MB read, 4.646 MB written), scaled x 64/48 by the
 # rows processed and x 5 for the passes of one alpha fit (d = 2)
