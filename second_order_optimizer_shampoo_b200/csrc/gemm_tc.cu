@@ -670,13 +670,14 @@ SHP_DEV uint32_t sw64_off(int r, int g) {
 }
 
 // The lane-per-row epilogue with bulk-tensor (TMA) traffic, for bf16 results
-// with no out2 and bf16 or no aux (ep.vec == 2): per 32-column chunk, each
+// with no out2 (ep.vec == 2): per 32-column chunk, each
 // lane packs its row's 32 results into the warp's 32 x 32 bf16 box `wbuf`
 // (64-byte swizzle: conflict-free, four 16-byte stores per lane) and lane 0
 // stores the box with one tensor store (tO), which also clips rows and
-// columns outside the matrix.  The aux box arrives in `wbuf + 2048` by tensor
-// load (tX) on the warp's barrier `abar`, one chunk ahead: the caller issues
-// the tile's first chunk, each chunk issues the next.  `apar` is the
+// columns outside the matrix.  A bf16 aux box arrives in `wbuf + 2048` by
+// tensor load (tX) on the warp's barrier `abar`, one chunk ahead: the caller
+// issues the tile's first chunk, each chunk issues the next; an fp32 or split
+// aux is read directly, each lane its row's 32 values.  `apar` is the
 // barrier's phase; `pending` tracks a load in flight (drained before exit).
 // The caller runs it only for warps with rows inside the matrix (no tensor
 // access starts past the last row).  Returns this lane's sum of squares
@@ -700,7 +701,19 @@ SHP_DEV float epilogue_rows_tma(uint32_t tmem, const CUtensorMap* tO, const CUte
     float a[32];
     tmem_ld32(trow + static_cast<uint32_t>(c * 32), a);  // the whole warp
     float x[32];
-    if (need_aux) {
+    if (need_aux && ep.aux_fmt != OUT_BF16) {  // fp32 / split aux: the lane's row, direct
+      const int64_t abase = static_cast<int64_t>(b) * ep.bs_aux +
+                            static_cast<int64_t>(row) * ep.lda_aux + cb;
+      if (row < ep.M && cb + 32 <= ep.N) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) ld8(ep.aux_fmt, ep.aux_hi, ep.aux_lo, abase + 8 * g, x + 8 * g);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          x[j] = row < ep.M && cb + j < ep.N ? ld1(ep.aux_fmt, ep.aux_hi, ep.aux_lo, abase + j)
+                                             : 0.f;
+      }
+    } else if (need_aux) {
       if (!mbar_wait(abar, apar, abort_flag)) {
         stop = true;
         return nrm;
@@ -956,7 +969,8 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t* wbuf = reinterpret_cast<uint8_t*>(stage_epi) + (warp - 2) * 4096;
     uint64_t* abar = &auxb[warp - 2];
     const bool tma_epi = ep.vec == 2;
-    const bool aux_tma = tma_epi && (ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY);
+    const bool aux_tma =
+        tma_epi && (ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY) && ep.aux_fmt == OUT_BF16;
     uint32_t apar = 0;
     bool pending = false;
     int tl = 0;
@@ -1126,16 +1140,16 @@ cudaError_t launch_pp(const CUtensorMap& a, const CUtensorMap& al, const CUtenso
   EpiParams ep = ep_in;
   ep.vec = lane_rows_ok(ep) ? 1 : 0;
   // bf16 result boxes of 32 x 32 by tensor store (and bf16 aux boxes by
-  // tensor load) when there is no second output and no non-bf16 aux
+  // tensor load) when there is no second output
   CUtensorMap tO, tX;
   memset(&tO, 0, sizeof(tO));
   memset(&tX, 0, sizeof(tX));
   const bool need_aux = ep.kind == EPI_GPOLY || ep.kind == EPI_AXPY || ep.kind == EPI_MOMENTUM;
   if (ep.vec && ep.out2_hi == nullptr && ep.kind != EPI_MOMENTUM &&
-      (!need_aux || ep.aux_fmt == OUT_BF16) &&
       make_map(&tO, ep.out_hi, 2, N, M, batch, ep.ldo, ep.bso, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
-      (!need_aux || make_map(&tX, ep.aux_hi, 2, N, M, batch, ep.lda_aux, ep.bs_aux, 32, 32,
-                             CU_TENSOR_MAP_SWIZZLE_64B)))
+      (!need_aux || ep.aux_fmt != OUT_BF16 ||
+       make_map(&tX, ep.aux_hi, 2, N, M, batch, ep.lda_aux, ep.bs_aux, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_64B)))
     ep.vec = 2;
   constexpr int SMEM = 1024 + C::PP_STAGES * C::STAGE_BYTES + 8 * 32 * 33 * 4 + 320;
   static_assert(SMEM <= 232448, "persistent pair kernel exceeds shared memory");
