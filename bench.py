@@ -412,11 +412,14 @@ def small_only(args):
     opts = prism.make_opts(d=1, p=SB_P, lo=0.5, tol=1e-6, max_iter=SB_MAX_ITER, prec="3xtf32")
     X = torch.empty_like(A)
     rep = prism.make_report(batch, SB_MAX_ITER, dev)
-    for _ in range(max(args.warmup, 1) + args.steps):
+    for _ in range(max(args.warmup, 1)):
         prism.matfn_inv_root(A, "inv4", opts, S, out=X, report=rep)
-    torch.cuda.synchronize()
+    ms = _time(lambda: prism.matfn_inv_root(A, "inv4", opts, S, out=X, report=rep),
+               torch.cuda.current_stream(), args.steps)
     ok = int((rep["status"].cpu().numpy() == 0).sum())
-    print(json.dumps({"kernel": "small", "batch": batch, "status_ok": ok,
+    print(json.dumps({"kernel": "small", "batch": batch, "status_ok": ok, "ms_per_call": ms,
+                      "roots_per_s": batch / (ms / 1e3),
+                      "iters": rep["iters"].cpu().numpy()[0].tolist(),
                       "launches": args.steps + max(args.warmup, 1)}))
     return 0
 

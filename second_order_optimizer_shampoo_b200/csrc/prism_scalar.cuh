@@ -168,13 +168,16 @@ __device__ double argmin_quartic_warp(const double* c, double lo, double hi) {
     }
     if (fv == 0.0 || (fu < 0.0) == (fv < 0.0)) continue;
     for (int it = 0; it < 16 && v - u > 1e-15 * fmax(1.0, fabs(u)); ++it) {
-      const double w = v - u;
-      const double x = u + w * static_cast<double>(lane + 1) / 33.0;
+      // the 32 interior points u + h, u + 2h, .. u + 32h with h = (v - u) / 33
+      // (a multiply by the rounded 1/33: any partition of the bracket works,
+      // and a division per point is the round's longest dependency)
+      const double h = (v - u) * (1.0 / 33.0);
+      const double x = u + h * static_cast<double>(lane + 1);
       const double fx = dpoly4(c, x);
       const unsigned m = __ballot_sync(0xffffffffu, fx == 0.0 || (fx < 0.0) != (fu < 0.0));
       const int i = m != 0u ? __ffs(static_cast<int>(m)) - 1 : 32;  // first sign change
-      const double nu = i == 0 ? u : u + w * static_cast<double>(i) / 33.0;
-      const double nv = i == 32 ? v : u + w * static_cast<double>(i + 1) / 33.0;
+      const double nu = i == 0 ? u : u + h * static_cast<double>(i);
+      const double nv = i == 32 ? v : u + h * static_cast<double>(i + 1);
       if (i != 0) fu = dpoly4(c, nu);
       u = nu;
       v = nv;

@@ -11,11 +11,11 @@
 // path ("Sintesi Tecnica: PRISM", Parte I-II): residual, stop test, sketched
 // alpha fit, Delta = g - I, X + X Delta updates.
 //
-// Arithmetic: products on the CUDA cores in fp32 FMA (each thread owns a 4 x 4
-// output tile and streams float4 operands from shared memory), at least as
-// accurate as either fp32 storage mode of the batched path; the alpha fit and
-// the norms in fp64.  Four 64 x 68 fp32 buffers (68 KB) per CTA, three CTAs
-// per SM.
+// Arithmetic: products and sketch powers on the tensor cores (warp-level
+// mma.sync TF32 with the operands split into two TF32 parts, three products
+// per pair: the 3xTF32 split of the batched path) with fp32 iterates; the
+// alpha fit and the norms in fp64.  Four 64 x 68 fp32 buffers (68 KB) per
+// CTA, three CTAs per SM.
 #include <math.h>
 
 #include "internal.h"
@@ -55,121 +55,146 @@ SHP_DEV double block_sum(double v, double* red) {
   return s;
 }
 
-// A thread's 4 x 4 output tile: rows rb, rb + rs, rb + 2 rs, rb + 3 rs and
-// columns c0..c0+3.  Products with a row-major left factor use strided rows
-// (rs = 16): a warp covers 4 consecutive row indices x 8 column groups, so
-// each float4 operand read touches 4 rows (16 banks apart in total) of A and
-// 128 contiguous bytes of B, one wavefront each.  Products with a
-// transposed left factor read 4 consecutive rows of A^T as one float4 and
-// use consecutive rows (rs = 1).
-struct Tile {
-  int rb, rs, c0;
-  SHP_DEV int row(int i) const { return rb + rs * i; }
+// ---------------------------------------------------- products on the tensor cores
+// Every product of the iteration is one 64 x 64 (or smaller) matrix in shared
+// memory times another; each of the 8 warps computes a 16 x 32 block with
+// mma.sync m16n8k8 TF32 (the warp-level MMA: one CTA's whole product is
+// 0.26 MFLOP, too small for a tcgen05 issue / TMEM drain round trip per
+// product, and the iteration's products depend on each other).  Operands are
+// split in registers as x = hi + lo, hi = x rounded to TF32 and lo = the
+// remainder rounded to TF32, and each product is lo*hi + hi*lo + hi*hi in the
+// fp32 accumulator (the 3xTF32 split of the batched path).
+SHP_DEV uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+SHP_DEV void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = tf32_rna(x);
+  lo = tf32_rna(x - __uint_as_float(hi));
+}
+
+SHP_DEV void mma_16x8x8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// This warp's 16 x 32 block of a 64 x 64 product: warp w covers rows
+// 16 (w / 2) .. + 15 and columns 32 (w % 2) .. + 31; in the m16n8 accumulator
+// layout a lane holds rows lr and lr + 8 (lr = lane / 4) of its block and the
+// column pair lc, lc + 1 (lc = 2 (lane % 4)) of each of the four 8-column
+// tiles: acc[nt][q] sits at (row(q / 2), col(nt) + q % 2).
+struct WTile {
+  int r0, c0, lr, lc;
+  SHP_DEV int row(int h) const { return r0 + lr + 8 * h; }
+  SHP_DEV int col(int nt) const { return c0 + 8 * nt + lc; }
 };
 
-SHP_DEV Tile tile_rows_strided() {
+SHP_DEV WTile warp_tile() {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  return Tile{4 * (w >> 1) + (l >> 3), 16, 4 * (8 * (w & 1) + (l & 7))};
-}
-SHP_DEV Tile tile_rows_consecutive() {
-  const int t = static_cast<int>(threadIdx.x);
-  return Tile{4 * (t >> 4), 1, 4 * (t & 15)};
+  return WTile{16 * (w >> 1), 32 * (w & 1), l >> 2, 2 * (l & 3)};
 }
 
-// acc = op(A) B on tile t, K a multiple of 4.  op(A) = A (row-major M x K) or,
-// with AT, the transpose of the row-major K x M matrix A (t.rs must be 1).
+// acc = op(A) B on the warp's block, op(A) = A (row-major, rows x K) or, with
+// AT, the transpose of the row-major K x rows matrix A.  Terms with k >= K
+// are zero (K need not be a multiple of 8); rows and columns past the
+// operands' extents read in-buffer data whose results the callers do not
+// store.  The fragment reads of a row-major operand fall on 32 distinct banks
+// (row stride 68 floats); those of a transposed one on 16.
 template <bool AT>
-SHP_DEV void tile_mm(const float* A, const float* B, int K, const Tile& t, float acc[4][4]) {
+SHP_DEV void warp_mm(const float* A, const float* B, int K, const WTile& t, float acc[4][4]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  const int lane = threadIdx.x & 31, lk = lane & 3, lm = lane >> 2;
+  const int ra = t.r0 + lm, rb = ra + 8;
 #pragma unroll 2
-  for (int k = 0; k < K; k += 4) {
-    float a[4][4], b[4][4];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const float4 v = *reinterpret_cast<const float4*>(B + (k + kk) * SB_LD + t.c0);
-      b[kk][0] = v.x;
-      b[kk][1] = v.y;
-      b[kk][2] = v.z;
-      b[kk][3] = v.w;
-    }
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const int ka = k0 + lk, kb = ka + 4;
+    const bool va = ka < K, vb = kb < K;
+    float af[4];
     if (AT) {
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const float4 v = *reinterpret_cast<const float4*>(A + (k + kk) * SB_LD + t.rb);
-        a[0][kk] = v.x;
-        a[1][kk] = v.y;
-        a[2][kk] = v.z;
-        a[3][kk] = v.w;
-      }
+      af[0] = va ? A[ka * SB_LD + ra] : 0.f;
+      af[1] = va ? A[ka * SB_LD + rb] : 0.f;
+      af[2] = vb ? A[kb * SB_LD + ra] : 0.f;
+      af[3] = vb ? A[kb * SB_LD + rb] : 0.f;
     } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(A + t.row(i) * SB_LD + k);
-        a[i][0] = v.x;
-        a[i][1] = v.y;
-        a[i][2] = v.z;
-        a[i][3] = v.w;
-      }
+      af[0] = va ? A[ra * SB_LD + ka] : 0.f;
+      af[1] = va ? A[rb * SB_LD + ka] : 0.f;
+      af[2] = vb ? A[ra * SB_LD + kb] : 0.f;
+      af[3] = vb ? A[rb * SB_LD + kb] : 0.f;
     }
+    uint32_t ah[4], al[4];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
+    for (int i = 0; i < 4; ++i) split_tf32(af[i], ah[i], al[i]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i][kk], b[kk][j], acc[i][j]);
+    for (int nt = 0; nt < 4; ++nt) {
+      const int cn = t.c0 + 8 * nt + lm;
+      uint32_t bh0, bl0, bh1, bl1;
+      split_tf32(va ? B[ka * SB_LD + cn] : 0.f, bh0, bl0);
+      split_tf32(vb ? B[kb * SB_LD + cn] : 0.f, bh1, bl1);
+      mma_16x8x8(acc[nt], al, bh0, bh1);
+      mma_16x8x8(acc[nt], ah, bl0, bl1);
+      mma_16x8x8(acc[nt], ah, bh0, bh1);
+    }
   }
 }
 
-SHP_DEV void store_row4(float* C, int row, int c0, const float* v) {
-  *reinterpret_cast<float4*>(C + row * SB_LD + c0) = make_float4(v[0], v[1], v[2], v[3]);
+SHP_DEV void store2(float* C, int row, int col, float v0, float v1) {
+  *reinterpret_cast<float2*>(C + row * SB_LD + col) = make_float2(v0, v1);
 }
 
 // R = I - op(A) B on the n x n grid; returns this thread's sum of squares.
-// Rows of the tile past n are computed from in-buffer data and not stored.
+// (The condition on the warp's block origin is the same for all its lanes, as
+// mma.sync needs.)
 template <bool AT>
-SHP_DEV float residual(const float* A, const float* B, int K, int n, float* R, const Tile& t) {
+SHP_DEV float residual(const float* A, const float* B, int K, int n, float* R, const WTile& t) {
   float nrm = 0.f;
-  if (t.rb < n && t.c0 < n) {
+  if (t.r0 < n && t.c0 < n) {
     float acc[4][4];
-    tile_mm<AT>(A, B, K, t, acc);
+    warp_mm<AT>(A, B, K, t, acc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = t.row(i);
-      if (r >= n) break;
-      float v[4];
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[j] = (r == t.c0 + j ? 1.f : 0.f) - acc[i][j];
-        nrm += v[j] * v[j];
+      for (int h = 0; h < 2; ++h) {
+        const int r = t.row(h), c = t.col(nt);
+        if (r < n && c < n) {  // c even and n % 4 == 0: c + 1 < n too
+          const float v0 = (r == c ? 1.f : 0.f) - acc[nt][2 * h];
+          const float v1 = (r == c + 1 ? 1.f : 0.f) - acc[nt][2 * h + 1];
+          nrm += v0 * v0 + v1 * v1;
+          store2(R, r, c, v0, v1);
+        }
       }
-      store_row4(R, r, t.c0, v);
-    }
   }
   return nrm;
 }
 
 // C = X + A B (X may be A or B, C must be neither), rows x cols, inner K.
 SHP_DEV void axpy_mm(const float* A, const float* B, const float* X, int K, int rows, int cols,
-                     float* C, const Tile& t) {
-  if (t.rb >= rows || t.c0 >= cols) return;
+                     float* C, const WTile& t) {
+  if (t.r0 >= rows || t.c0 >= cols) return;
   float acc[4][4];
-  tile_mm<false>(A, B, K, t, acc);
+  warp_mm<false>(A, B, K, t, acc);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = t.row(i);
-    if (r >= rows) break;
-    const float4 x = *reinterpret_cast<const float4*>(X + r * SB_LD + t.c0);
-    const float v[4] = {x.x + acc[i][0], x.y + acc[i][1], x.z + acc[i][2], x.w + acc[i][3]};
-    store_row4(C, r, t.c0, v);
-  }
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = t.row(h), c = t.col(nt);
+      if (r < rows && c < cols) {
+        const float2 x = *reinterpret_cast<const float2*>(X + r * SB_LD + c);
+        store2(C, r, c, x.x + acc[nt][2 * h], x.y + acc[nt][2 * h + 1]);
+      }
+    }
 }
 
 // Delta = g - I: alpha R in place (d = 1), or W = R/2 + alpha R^2 (d = 2).
 // Returns the buffer that holds Delta.
-SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, const Tile& t) {
+SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, const WTile& t) {
   if (d == 1) {
     for (int e = threadIdx.x; e < n * n; e += SB_THREADS) {
       const int i = e / n, j = e - i * n;
@@ -178,39 +203,60 @@ SHP_DEV float* form_delta(int d, float alpha, float* R, float* W, int n, const T
     __syncthreads();
     return R;
   }
-  if (t.rb < n && t.c0 < n) {
+  if (t.r0 < n && t.c0 < n) {
     float acc[4][4];
-    tile_mm<false>(R, R, n, t, acc);
+    warp_mm<false>(R, R, n, t, acc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = t.row(i);
-      if (r >= n) break;
-      const float4 q = *reinterpret_cast<const float4*>(R + r * SB_LD + t.c0);
-      const float v[4] = {0.5f * q.x + alpha * acc[i][0], 0.5f * q.y + alpha * acc[i][1],
-                          0.5f * q.z + alpha * acc[i][2], 0.5f * q.w + alpha * acc[i][3]};
-      store_row4(W, r, t.c0, v);
-    }
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = t.row(h), c = t.col(nt);
+        if (r < n && c < n) {
+          const float2 q = *reinterpret_cast<const float2*>(R + r * SB_LD + c);
+          store2(W, r, c, 0.5f * q.x + alpha * acc[nt][2 * h], 0.5f * q.y + alpha * acc[nt][2 * h + 1]);
+        }
+      }
   }
   __syncthreads();
   return W;
 }
 
-// Vout = R Vin (n x p, row-major) by the whole CTA; each dot product runs as
-// four interleaved partial sums (k mod 4) so that its FMA chain is n/4 long.
+// Vout = R Vin (n x p, row-major with row stride p) on the tensor cores, the
+// same 3xTF32 split as the products: warp w computes rows 16 (w % 4) .. + 15
+// and sketch columns 8 (w / 4) .. + 7 (p <= 16; columns past p and terms past
+// n are zero, and rows past n are not stored).
 SHP_DEV void sketch_power(const float* R, const float* Vin, float* Vout, int n, int p) {
-  for (int e = threadIdx.x; e < n * p; e += SB_THREADS) {
-    const int row = e / p, col = e - row * p;
-    const float* Rr = R + row * SB_LD;
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < n; k += 4) {
-      const float4 r = *reinterpret_cast<const float4*>(Rr + k);
-      s0 = fmaf(r.x, Vin[k * p + col], s0);
-      s1 = fmaf(r.y, Vin[(k + 1) * p + col], s1);
-      s2 = fmaf(r.z, Vin[(k + 2) * p + col], s2);
-      s3 = fmaf(r.w, Vin[(k + 3) * p + col], s3);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, lk = lane & 3, lm = lane >> 2;
+  const int r0 = 16 * (w & 3), c0 = 8 * (w >> 2);
+  if (r0 < n && c0 < p) {  // the same for the whole warp, as mma.sync needs
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ra = r0 + lm, rb = ra + 8, cn = c0 + lm;
+    const bool vc = cn < p;
+#pragma unroll 2
+    for (int k0 = 0; k0 < n; k0 += 8) {
+      const int ka = k0 + lk, kb = ka + 4;
+      const bool va = ka < n, vb = kb < n;
+      const float af[4] = {va ? R[ra * SB_LD + ka] : 0.f, va ? R[rb * SB_LD + ka] : 0.f,
+                           vb ? R[ra * SB_LD + kb] : 0.f, vb ? R[rb * SB_LD + kb] : 0.f};
+      uint32_t ah[4], al[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) split_tf32(af[i], ah[i], al[i]);
+      uint32_t bh0, bl0, bh1, bl1;
+      split_tf32(va && vc ? Vin[ka * p + cn] : 0.f, bh0, bl0);
+      split_tf32(vb && vc ? Vin[kb * p + cn] : 0.f, bh1, bl1);
+      mma_16x8x8(acc, al, bh0, bh1);
+      mma_16x8x8(acc, ah, bl0, bl1);
+      mma_16x8x8(acc, ah, bh0, bh1);
     }
-    Vout[e] = (s0 + s1) + (s2 + s3);
+    const int cc = c0 + 2 * lk;  // the lane's column pair
+    if (ra < n) {
+      if (cc < p) Vout[ra * p + cc] = acc[0];
+      if (cc + 1 < p) Vout[ra * p + cc + 1] = acc[1];
+    }
+    if (rb < n) {
+      if (cc < p) Vout[rb * p + cc] = acc[2];
+      if (cc + 1 < p) Vout[rb * p + cc + 1] = acc[3];
+    }
   }
   __syncthreads();
 }
@@ -308,7 +354,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   __shared__ double red[SB_THREADS / 32][10];
   __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
-  const Tile ts = tile_rows_strided();
+  const WTile ts = warp_tile();
   const int64_t nn = static_cast<int64_t>(n) * n;
   const float* Ab = A + b * nn;
   float *Y = sm, *Z = sm + SB_MAT, *R = sm + 2 * SB_MAT, *W = sm + 3 * SB_MAT;
@@ -415,7 +461,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   __shared__ double red[SB_THREADS / 32][10];
   __shared__ float s_alpha, s_ratio;
   const int b = blockIdx.x, tid = threadIdx.x;
-  const Tile ts = tile_rows_strided(), tc = tile_rows_consecutive();
+  const WTile ts = warp_tile();
   int64_t boff = static_cast<int64_t>(b) * m * n;
   if (dims != nullptr) {  // blocks of different shapes, packed at offs[b]
     m = dims[2 * b];
@@ -455,7 +501,7 @@ __global__ void __launch_bounds__(SB_THREADS, 3)
   for (int k = 0;; ++k) {
     // R = I - X^T X (polar) or I - X X (sign of a symmetric X, m == n)
     const double n2 = block_sum(sign ? residual<false>(X, X, rows, k_n, R, ts)
-                                     : residual<true>(X, X, rows, k_n, R, tc),
+                                     : residual<true>(X, X, rows, k_n, R, ts),
                                 red[0]);
     const float r = sqrtf(static_cast<float>(n2) / static_cast<float>(k_n));
     const int st = stop_rule(r, k, mi, o.tol, prev, o.stall_below, o.stall_ratio);
