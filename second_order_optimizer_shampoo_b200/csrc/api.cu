@@ -66,6 +66,8 @@ Ctl carve_ctl(Arena& a, int64_t batch) {
   c.alpha = a.take<float>(batch);
   c.it = a.take<int>(1);
   c.flag = a.take<int>(1);
+  c.gram = a.take<double>(batch * 15);
+  c.gcnt = a.take<int>(batch);
   return c;
 }
 
@@ -239,12 +241,25 @@ int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass,
                      int* rep_degree = nullptr) {
   const int64_t np = n * o->p, nn = n * n;
   const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
+  // a fitted alpha at fixed degree is solved inside the last pass (no alpha launch)
+  const bool fuse = !o->fixed_alpha && !o->adaptive_degree && ctl.gram != nullptr;
   if (!o->fixed_alpha) {
     CK(sketch_pass(Rs, nullptr, n, nn, S_pass, 0, V + np, vbs, o->p, batch, ctl.active, ctl.it,
                    np, st, ctl.tmo));
-    for (int j = 2; j <= 2 * o->d + 1; ++j)
-      CK(sketch_pass(Rs, nullptr, n, nn, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
-                     ctl.active, nullptr, 0, st, ctl.tmo));
+    const int last = 2 * o->d + 1;
+    for (int j = 2; j <= last; ++j) {
+      if (fuse && j == last) {
+        bool fused = false;
+        CK(sketch_pass_alpha(Rs, n, nn, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
+                             ctl.active, st, ctl.tmo, V, o->d, o->lo, o->hi, ctl.alpha,
+                             rep_alpha, rep_stride, rep_slot_base, ctl.it, ctl.gram, ctl.gcnt,
+                             &fused));
+        if (fused) return SHP_OK;
+      } else {
+        CK(sketch_pass(Rs, nullptr, n, nn, V + (j - 1) * np, vbs, V + j * np, vbs, o->p, batch,
+                       ctl.active, nullptr, 0, st, ctl.tmo));
+      }
+    }
   }
   AdaptiveDeg ad{o->adaptive_degree, o->raise_above, ctl.deg, ctl.act1, ctl.act2, rep_degree};
   CK(alpha_solve(V, n, o->p, o->d, batch, o->lo, o->hi, o->fixed_alpha, ctl.active, ctl.alpha,

@@ -76,6 +76,10 @@ __global__ void k_reset(Ctl ctl, int batch, int first, int start_degree) {
   s.pass_status = ST_OK;
   ctl.active[b] = 1;
   ctl.alpha[b] = 0.f;
+  if (ctl.gram != nullptr) {  // the fused alpha's accumulators
+    for (int i = 0; i < 15; ++i) ctl.gram[b * 15 + i] = 0.0;
+    ctl.gcnt[b] = 0;
+  }
 }
 
 __global__ void __launch_bounds__(EW_THREADS)

@@ -149,6 +149,18 @@ struct AdaptiveDeg {
 // current degree, raising it by the rule of shp_prism_opts.adaptive_degree.
 // tmo (may be null): a block whose flag is set (a sketch wait ran out, so V
 // is incomplete) gets alpha = NaN and NaN coefficients instead of a fit.
+// The last sketch pass V_{2d+1} = R V_2d with the alpha fit folded in: each
+// consumer warp adds its rows' partial Gram of V_d .. V_{2d+1} (fp64) into
+// gram[b] and the warp that completes a block solves its alpha (fitted alpha
+// at fixed degree d; V is the moment stack [batch][2d+2][n][p]).  *fused
+// tells whether the fused kernel ran; when it did not (R not 16-byte aligned,
+// V too large for shared memory) the pass ran plain and the caller fits.
+cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, const float* Vin,
+                              int64_t vin_bstride, float* Vout, int64_t vout_bstride, int p,
+                              int batch, const int* active, cudaStream_t st, int* tmo,
+                              const float* V, int d, float lo, float hi, float* alpha,
+                              float* report_alpha, int64_t report_stride, int report_slot,
+                              const int* it, double* gram, int* gcnt, bool* fused);
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
@@ -178,6 +190,8 @@ struct Ctl {
   float* alpha;   // alpha_k per block
   int* it;        // iteration index k of the current pass (device-side loop)
   int* flag;      // loop condition for the host-driven diagnostic loop
+  double* gram;   // [batch][15] sketch Gram accumulated by the fused last pass
+  int* gcnt;      // [batch] items of the fused last pass seen so far
 };
 // Stop test of iteration k = *ctl.it for every active block.
 cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int max_iter, float tol,

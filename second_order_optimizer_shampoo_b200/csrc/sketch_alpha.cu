@@ -19,6 +19,8 @@
 #include <math.h>
 #include <stdlib.h>
 
+#include <string.h>
+
 #include "internal.h"
 #include "prism_scalar.cuh"
 #include "shp_common.cuh"
@@ -202,6 +204,156 @@ struct SkTma {
 
 // A wait that ran out: flag the block and leave (every other waiter then
 // runs out too, or sees the flag first).
+constexpr int AL_THREADS = 512;
+
+// Per-block alpha of one iteration.  Without adaptive degree: the Gram of
+// V_d..V_{2d+1}, the quartic and its minimiser on [lo, hi].  With adaptive
+// degree (d = 2): the Gram of V_1..V_5 at once; a block at degree 1 fits on
+// V_1..V_3 over [1/2, hi] and, when sqrt(J_1(alpha*)) / ||V_1||_F exceeds
+// raise_above, moves to degree 2 (V_2..V_5 over [3/8, hi]) for the rest of
+// the pass.  act1/act2 then mark the active blocks at each degree for the
+// masked launches that form Delta.
+struct AlphaArgs {
+  const float* V;
+  int64_t n, vbs;
+  int p, d, fixed;
+  float lo, hi;
+  const int* active;
+  float* alpha;
+  double* Jc;
+  float* rep;
+  int64_t rep_stride;
+  int rep_slot;
+  const int* it;
+  int adaptive;
+  float raise_above;
+  int* deg;
+  int* act1;
+  int* act2;
+  int* rep_deg;
+  const int* tmo;  // blocks whose sketch timed out: alpha = NaN
+};
+
+
+// alpha of block b from the Gram G[i][j] = <V_{first+i}, V_{first+j}> of its
+// sketch moments (first = d, or 1 with adaptive degree): the quartic J and its
+// minimiser on [lo, hi] by the calling warp (every lane takes part in the
+// bracketing), the degree rule, and lane 0 writes alpha, J's coefficients and
+// the report.  Shared by k_alpha and the fused last sketch pass.
+SHP_DEV void alpha_solve_warp(const AlphaArgs& g, int b, const double (&G)[5][5]) {
+  const int lane = threadIdx.x & 31;
+  const int rep_slot = g.rep_slot + (g.it != nullptr ? *g.it : 0);
+  const int first = g.adaptive ? 1 : g.d;  // V_first .. V_{first + nv - 1}
+  // fit at degree e on the Gram block starting at V_e (offset e - first)
+  auto fit = [&](int e, double lo, double* coef) {
+    double M[4][4];
+    const int o = e - first;
+    for (int i = 0; i < e + 2; ++i)
+      for (int j = 0; j < e + 2; ++j) M[i][j] = G[o + i][o + j];
+    quartic_from_gram(M, e, coef);
+    return argmin_quartic_warp(coef, lo, static_cast<double>(g.hi));
+  };
+  double coef[5];
+  int dcur = g.d;
+  double a;
+  if (!g.adaptive) {
+    a = fit(g.d, static_cast<double>(g.lo), coef);
+  } else {
+    dcur = g.deg[b];
+    if (dcur == 1) {
+      a = fit(1, 0.5, coef);
+      const double J = poly4(coef, a), base = G[0][0];  // ||V_1||^2 = ||R_k S_k||^2
+      if (base > 0.0 && sqrt(fmax(J, 0.0) / base) > static_cast<double>(g.raise_above))
+        dcur = 2;
+    }
+    if (dcur == 2) a = fit(2, 0.375, coef);
+  }
+  if (lane != 0) return;
+  g.alpha[b] = static_cast<float>(a);
+  if (g.Jc != nullptr)
+    for (int i = 0; i < 5; ++i) g.Jc[b * 5 + i] = coef[i];
+  if (g.rep != nullptr) g.rep[b * g.rep_stride + rep_slot] = static_cast<float>(a);
+  if (g.rep_deg != nullptr) g.rep_deg[b * g.rep_stride + rep_slot] = dcur;
+  if (g.adaptive) {
+    g.deg[b] = dcur;
+    g.act1[b] = dcur == 1;
+    g.act2[b] = dcur == 2;
+  }
+}
+
+// Fused alpha of the last sketch pass: a consumer warp's partial Gram of the
+// moments over the rows it produced, kept across the items of one block.
+struct GramPart {
+  double part[15];
+  int b, items;
+};
+
+SHP_DEV void gram_reset(GramPart& gp) {
+#pragma unroll
+  for (int i = 0; i < 15; ++i) gp.part[i] = 0.0;
+  gp.items = 0;
+}
+
+// Adds this warp's rows row0 .. row0 + rows - 1 of V_first .. V_{2d+1} (nv
+// vectors of block b, fp32, n x p each) to the partial Gram.
+SHP_DEV void gram_add(GramPart& gp, const AlphaArgs& g, int b, int64_t row0, int rows) {
+  const int lane = threadIdx.x & 31, nv = g.d + 2;
+  const int64_t len = g.n * g.p;
+  const float* Vb = g.V + b * g.vbs + static_cast<int64_t>(g.d) * len;
+  for (int e = lane; e < rows * g.p; e += 32) {
+    const int64_t row = row0 + e / g.p;
+    if (row >= g.n) continue;
+    const int64_t off = row * g.p + e % g.p;
+    double x[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) x[i] = i < nv ? static_cast<double>(Vb[i * len + off]) : 0.0;
+    int idx = 0;
+#pragma unroll
+    for (int i = 0; i < 5; ++i)
+#pragma unroll
+      for (int j = i; j < 5; ++j, ++idx) gp.part[idx] = fma(x[i], x[j], gp.part[idx]);
+  }
+  ++gp.items;
+}
+
+// Adds the warp's partial Gram of block gp.b into gram[b] and its item count
+// into gcnt[b]; the warp whose count completes the block (every item of the
+// pass seen by each consumer warp: total items x ST_CONS) solves alpha for it
+// and clears the block's accumulators for the next iteration.  A block whose
+// sketch timed out gets alpha = NaN.
+SHP_DEV void gram_flush(GramPart& gp, const AlphaArgs& g, double* gram, int* gcnt, int total,
+                        const int* tmo) {
+  const int lane = threadIdx.x & 31;
+  if (gp.b < 0 || gp.items == 0) return;
+  const int b = gp.b;
+#pragma unroll
+  for (int i = 0; i < 15; ++i) gp.part[i] = warp_sum(gp.part[i]);
+  int last = 0;
+  if (lane == 0) {
+    for (int i = 0; i < 15; ++i) atomicAdd(&gram[b * 15 + i], gp.part[i]);
+    __threadfence();
+    last = atomicAdd(&gcnt[b], gp.items) + gp.items == total;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (last) {
+    __threadfence();
+    double G[5][5];
+    int idx = 0;
+    for (int i = 0; i < 5; ++i)
+      for (int j = i; j < 5; ++j, ++idx) G[i][j] = G[j][i] = __ldcg(&gram[b * 15 + idx]);
+    if (tmo != nullptr && tmo[b] != 0) {
+      if (lane == 0) g.alpha[b] = __int_as_float(0x7fc00000);
+    } else {
+      alpha_solve_warp(g, b, G);
+    }
+    if (lane == 0) {
+      for (int i = 0; i < 15; ++i) gram[b * 15 + i] = 0.0;
+      gcnt[b] = 0;
+    }
+  }
+  gram_reset(gp);
+}
+
 SHP_DEV void sketch_give_up(volatile int* abort_flag, int* tmo, int b, int lane) {
   *abort_flag = 1;
   __threadfence_block();
@@ -213,7 +365,8 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
     k_sketch_tma(const __grid_constant__ CUtensorMap tR, int64_t n,
                  const float* __restrict__ Vin, int64_t vbs, float* __restrict__ Vout,
                  int64_t obs, int p, int batch, const int* __restrict__ active,
-                 const int* __restrict__ it, int64_t it_stride, int* tmo, int selftest) {
+                 const int* __restrict__ it, int64_t it_stride, int* tmo, int selftest,
+                 AlphaArgs fa, double* gram, int* gcnt) {
   count_kernel_run();
   using K = SkTma<P>;
   constexpr int ROWS = K::ROWS, RPI = K::RPI;
@@ -287,6 +440,10 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
   int kit = 0, ns = 0;  // stages consumed, V stagings
   int cur_b = -1, seen_b = -1;
   bool seen_on = true;
+  GramPart gp;  // fused alpha (gram != nullptr): this warp's partial Gram
+  gram_reset(gp);
+  gp.b = -1;
+  bool aborted = false;
   for (int64_t t = i0; t < i1; ++t) {
     if (*abort_flag) break;
     const int b = static_cast<int>(t / gpb);
@@ -300,6 +457,7 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
       // nothing completes, with the producer's copies already in flight
       if (selftest && !mbar_wait(never, 0, nullptr, SHP_SELFTEST_LIMIT)) {
         sketch_give_up(abort_flag, tmo, b, lane);
+        aborted = true;
         break;
       }
       __syncwarp();
@@ -372,40 +530,25 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
         for (int r = 0; r < ROWS; ++r) acc[r * P + j] = fmaf(x1[r].w, v1.w, acc[r * P + j]);
       }
     }
-    if (!ok) break;
+    if (!ok) {
+      aborted = true;
+      break;
+    }
     store_row_sums<ROWS, P>(acc, lane, r0 + warp * ROWS, n, p, Vout + b * obs);
+    if (gram != nullptr) {
+      if (b != gp.b) {
+        gram_flush(gp, fa, gram, gcnt, static_cast<int>(gpb) * ST_CONS, tmo);
+        gp.b = b;
+      }
+      __syncwarp();  // the rows this warp just stored are visible to all its lanes
+      gram_add(gp, fa, b, r0 + warp * ROWS, ROWS);
+    }
   }
+  // a pass that gave up leaves its blocks' counts short: no alpha is solved
+  // for them (it stays NaN from the stop test)
+  if (gram != nullptr && !aborted && !*abort_flag)
+    gram_flush(gp, fa, gram, gcnt, static_cast<int>(gpb) * ST_CONS, tmo);
 }
-
-constexpr int AL_THREADS = 512;
-
-// Per-block alpha of one iteration.  Without adaptive degree: the Gram of
-// V_d..V_{2d+1}, the quartic and its minimiser on [lo, hi].  With adaptive
-// degree (d = 2): the Gram of V_1..V_5 at once; a block at degree 1 fits on
-// V_1..V_3 over [1/2, hi] and, when sqrt(J_1(alpha*)) / ||V_1||_F exceeds
-// raise_above, moves to degree 2 (V_2..V_5 over [3/8, hi]) for the rest of
-// the pass.  act1/act2 then mark the active blocks at each degree for the
-// masked launches that form Delta.
-struct AlphaArgs {
-  const float* V;
-  int64_t n, vbs;
-  int p, d, fixed;
-  float lo, hi;
-  const int* active;
-  float* alpha;
-  double* Jc;
-  float* rep;
-  int64_t rep_stride;
-  int rep_slot;
-  const int* it;
-  int adaptive;
-  float raise_above;
-  int* deg;
-  int* act1;
-  int* act2;
-  int* rep_deg;
-  const int* tmo;  // blocks whose sketch timed out: alpha = NaN
-};
 
 // This thread's partial sums of <V_i, V_j> (i <= j < NV, packed row by row)
 // over elements threadIdx.x + k * AL_THREADS; NV is a compile-time constant so
@@ -506,50 +649,19 @@ __global__ void __launch_bounds__(AL_THREADS) k_alpha(AlphaArgs g) {
         ++idx;
       }
   }
-  // fit at degree e on the Gram block starting at V_e (offset e - first)
-  auto fit = [&](int e, double lo, double* coef) {
-    double M[4][4];
-    const int o = e - first;
-    for (int i = 0; i < e + 2; ++i)
-      for (int j = 0; j < e + 2; ++j) M[i][j] = G[o + i][o + j];
-    quartic_from_gram(M, e, coef);
-    return argmin_quartic_warp(coef, lo, static_cast<double>(g.hi));
-  };
-  double coef[5];
-  int dcur = g.d;
-  double a;
-  if (!g.adaptive) {
-    a = fit(g.d, static_cast<double>(g.lo), coef);
-  } else {
-    dcur = g.deg[b];
-    if (dcur == 1) {
-      a = fit(1, 0.5, coef);
-      const double J = poly4(coef, a), base = G[0][0];  // ||V_1||^2 = ||R_k S_k||^2
-      if (base > 0.0 && sqrt(fmax(J, 0.0) / base) > static_cast<double>(g.raise_above))
-        dcur = 2;
-    }
-    if (dcur == 2) a = fit(2, 0.375, coef);
-  }
-  if (threadIdx.x != 0) return;
-  g.alpha[b] = static_cast<float>(a);
-  if (g.Jc != nullptr)
-    for (int i = 0; i < 5; ++i) g.Jc[b * 5 + i] = coef[i];
-  if (g.rep != nullptr) g.rep[b * g.rep_stride + rep_slot] = static_cast<float>(a);
-  if (g.rep_deg != nullptr) g.rep_deg[b * g.rep_stride + rep_slot] = dcur;
-  if (g.adaptive) {
-    g.deg[b] = dcur;
-    g.act1[b] = dcur == 1;
-    g.act2[b] = dcur == 2;
-  }
+  alpha_solve_warp(g, b, G);
 }
 
 __global__ void k_control(BlockState* bs, int* active, const int* it, int batch, int64_t n,
                           int max_iter, float tol, float stall_below, float stall_ratio,
                           float* rep_res, int64_t res_stride, int res_slot, int* rep_iters,
-                          int iters_slot) {
+                          int iters_slot, float* alpha) {
   count_kernel_run();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch || active[b] == 0) return;
+  // this iteration's alpha is written by the fit; a fit that never completes
+  // (a sketch wait that gave up) leaves NaN, which stops the block
+  if (alpha != nullptr) alpha[b] = __int_as_float(0x7fc00000);
   const int k = *it;
   BlockState& s = bs[b];
   const float r = sqrtf(s.norm2 / static_cast<float>(n));
@@ -574,7 +686,8 @@ template <int P>
 bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin, int64_t vbs,
                        float* Vout, int64_t obs, int p, int batch, const int* active,
                        const int* it, int64_t it_stride, int* tmo, int selftest, cudaStream_t st,
-                       cudaError_t* err) {
+                       cudaError_t* err, const AlphaArgs* fa = nullptr, double* gram = nullptr,
+                       int* gcnt = nullptr) {
   const size_t smem = SkTma<P>::smem_bytes(n);
   if (smem > 200 * 1024) return false;  // V does not fit whole: the register kernel
   CUtensorMap tR;
@@ -594,8 +707,11 @@ bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin,
   if (dev >= 0) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t items = (n + SkTma<P>::RPI - 1) / SkTma<P>::RPI * batch;
   const int grid = static_cast<int>(items < sms ? items : sms);
+  AlphaArgs none;
+  memset(&none, 0, sizeof(none));
   kern<<<grid, 32 * (ST_CONS + 1), smem, st>>>(tR, n, Vin, vbs, Vout, obs, p, batch, active, it,
-                                                it_stride, tmo, selftest);
+                                                it_stride, tmo, selftest, fa ? *fa : none,
+                                                fa ? gram : nullptr, fa ? gcnt : nullptr);
   *err = cudaGetLastError();
   return true;
 }
@@ -640,6 +756,52 @@ cudaError_t sketch_pass(const float* Rhi, const float* Rlo, int64_t n, int64_t r
   return cudaGetLastError();
 }
 
+cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, const float* Vin,
+                              int64_t vin_bstride, float* Vout, int64_t vout_bstride, int p,
+                              int batch, const int* active, cudaStream_t st, int* tmo,
+                              const float* V, int d, float lo, float hi, float* alpha,
+                              float* report_alpha, int64_t report_stride, int report_slot,
+                              const int* it, double* gram, int* gcnt, bool* fused) {
+  *fused = false;
+  if (batch <= 0 || n <= 0) return cudaSuccess;
+  if (gram != nullptr && gcnt != nullptr && (reinterpret_cast<uintptr_t>(R) & 15) == 0 &&
+      n % 4 == 0 && r_bstride % 4 == 0) {
+    AlphaArgs g;
+    memset(&g, 0, sizeof(g));
+    g.tmo = tmo;
+    g.V = V;
+    g.n = n;
+    g.vbs = static_cast<int64_t>(2 * d + 2) * n * p;
+    g.p = p;
+    g.d = d;
+    g.lo = lo;
+    g.hi = hi;
+    g.active = active;
+    g.alpha = alpha;
+    g.rep = report_alpha;
+    g.rep_stride = report_stride;
+    g.rep_slot = report_slot;
+    g.it = it;
+    cudaError_t e = cudaSuccess;
+    bool done = false;
+    if (p <= 4)
+      done = launch_sketch_tma<4>(R, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p, batch,
+                                  active, nullptr, 0, tmo, 0, st, &e, &g, gram, gcnt);
+    else if (p <= 8)
+      done = launch_sketch_tma<8>(R, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p, batch,
+                                  active, nullptr, 0, tmo, 0, st, &e, &g, gram, gcnt);
+    else if (p <= 16)
+      done = launch_sketch_tma<16>(R, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
+                                   batch, active, nullptr, 0, tmo, 0, st, &e, &g, gram, gcnt);
+    if (done) {
+      *fused = e == cudaSuccess;
+      return e;
+    }
+  }
+  return sketch_pass(R, nullptr, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p, batch,
+                     active, nullptr, 0, st, tmo);
+}
+
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
@@ -680,7 +842,8 @@ cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int max_iter, flo
   if (batch <= 0) return cudaSuccess;
   k_control<<<(batch + 127) / 128, 128, 0, st>>>(ctl.bs, ctl.active, ctl.it, batch, n, max_iter,
                                                  tol, stall_below, stall_ratio, report_res,
-                                                 res_stride, res_slot, report_iters, iters_slot);
+                                                 res_stride, res_slot, report_iters, iters_slot,
+                                                 ctl.alpha);
   return cudaGetLastError();
 }
 
