@@ -346,16 +346,18 @@ def gemm_only(args):
 SB_N, SB_BATCH, SB_P, SB_MAX_ITER = 64, 16384, 4, 50
 FP32_LANES_PER_SM, SMS = 128, 148
 # dram__bytes_read.sum + dram__bytes_write.sum of one full-size small-block
-# launch: none from the current kernel (the strided-row tiles and the
-# symmetric start came after the last capture, whose 274.3 + 237.2 MB equal
-# the compulsory bytes), so the roofline reports no traffic
-SMALL_TRAFFIC_PER_LAUNCH = None
+# launch (16384 x 64^2, ncu capture of the current kernel)
+SMALL_TRAFFIC_PER_LAUNCH = 276.44e6 + 238.29e6
 
 
 def small_block_leg(args, dev, stream, sm_max_mhz):
     """Many small blocks: 16384 independent 64 x 64 SPD blocks (lambda
     log-uniform on [1e-3, 1]), A^(-1/4) by PRISM d = 1, p = 4, tol 1e-6, one
-    CTA per block iterating on chip (fp32 FMA products)."""
+    CTA per block iterating on chip (products and sketch powers on the
+    tensor cores, 3xTF32 warp-level MMA).  The block's iteration is a chain of
+    dependent steps and block barriers, so the figure is latency-bound; the
+    fraction is given against the 3xTF32 tensor rate and, for continuity, the
+    fp32 FMA rate."""
     import torch
 
     from second_order_optimizer_shampoo_b200 import _abi, prism, synth
@@ -388,16 +390,21 @@ def small_block_leg(args, dev, stream, sm_max_mhz):
     peaks, _ = load_peaks()
     tf = flops / (ms / 1e3) / 1e12
     fma_peak = SMS * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+    tf32 = peaks.get("tf32_tflops", peaks["bf16_tflops"] * TF32_OVER_BF16)
     return {"workload": "inv4_root_16384x64sq_spd_cond1e3_prism_d1_p4_tol1e-6_onchip",
             "ms_per_call": ms, "roots_per_s": SB_BATCH / (ms / 1e3), "value": tf,
             "unit": "TFLOP/s", "products": products, "status_ok": ok,
             "median_iters_per_pass": [int(x) for x in np.median(iters, axis=0)],
             "hbm_gbs": hbm_bytes / (ms / 1e3) / 1e9, "hbm_peak_gbs": peaks["hbm_gbs"],
-            "roofline": {"bound": "alu", "achieved": tf, "peak": fma_peak, "unit": "TFLOP/s",
-                         "frac": tf / fma_peak, "traffic": SMALL_TRAFFIC_PER_LAUNCH,
+            "fma_frac": tf / fma_peak,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": tf32 / 3, "unit": "TFLOP/s",
+                         "frac": tf / (tf32 / 3), "traffic": SMALL_TRAFFIC_PER_LAUNCH,
                          "traffic_unit": "bytes per launch", "algorithmic_bytes": hbm_bytes,
-                         "peak_note": f"fp32 FMA: {SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 "
-                                      f"flop x {sm_max_mhz:.0f} MHz (max SM clock)"}}
+                         "peak_note": "3xTF32 products: the measured TF32 peak / 3; the "
+                                      "iteration is latency-bound (a chain of dependent steps "
+                                      "per block), fma_frac against the fp32 FMA rate "
+                                      f"({SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 flop x "
+                                      f"{sm_max_mhz:.0f} MHz)"}}
 
 
 def small_only(args):
@@ -477,9 +484,13 @@ def shampoo_step_leg(args, dev, stream, host_loop=False, reps=10):
     def ema_steps():
         prism.shampoo_gram_ema_steps(Gst, LR[0:1], LR[1:2], beta, eps, "tf32", ws=ws_ema)
 
+    ws_one = torch.empty(max(prism.shp_workspace_bytes(_abi.SHP_OP_GRAM_EMA, n, n, 1,
+                                                       prism.make_opts(prec="tf32")), 16),
+                         dtype=torch.uint8, device=dev)
+
     def ema_one_step_calls():
         for G in Gs:
-            prism.shampoo_gram_ema(G, LR[0:1], LR[1:2], beta, eps, "tf32")
+            prism.shampoo_gram_ema(G, LR[0:1], LR[1:2], beta, eps, "tf32", ws=ws_one)
 
     def step():
         LR.copy_(eye.expand(2, n, n))
