@@ -361,14 +361,20 @@ int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const floa
  *   SHP_SELFTEST_SKETCH  TMA sketch: the consumers' first V hand-over, with
  *                        the producer's copies in flight (they are drained),
  *                        in the first pass of a whole alpha fit (d = 1)
+ *   SHP_SELFTEST_SKETCH_ALPHA  the last sketch pass with the alpha fit folded
+ *                        in (as inside the matrix-function loops): the same
+ *                        hand-over in that pass; no warp completes the block,
+ *                        so no alpha is solved
  * status: one device int32, set to SHP_ETIMEOUT by the kernel (cleared
- * first).  alpha_out: one device float (may be NULL), for SHP_SELFTEST_SKETCH
- * the fit's alpha, which must come out NaN (no fit on incomplete vectors).
+ * first).  alpha_out: one device float (may be NULL), for the sketch cases
+ * the fit's alpha, which must come out NaN (no fit on incomplete vectors; the
+ * folded case leaves the NaN it starts from, as the stop test sets it).
  * ws: at least SHP_SELFTEST_WS_BYTES of device scratch, 256-byte aligned
  * (zeroed by the call).  Returns SHP_OK once launched. */
 #define SHP_SELFTEST_GEMM 0
 #define SHP_SELFTEST_OZAKI 1
 #define SHP_SELFTEST_SKETCH 2
+#define SHP_SELFTEST_SKETCH_ALPHA 3
 #define SHP_SELFTEST_WS_BYTES (4u << 20)
 int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void* ws,
                               size_t ws_bytes, shp_stream stream);

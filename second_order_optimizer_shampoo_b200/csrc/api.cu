@@ -877,7 +877,8 @@ extern "C" {
 int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void* ws,
                               size_t ws_bytes, shp_stream stream) {
   if (status == nullptr || ws == nullptr || ws_bytes < SHP_SELFTEST_WS_BYTES) return SHP_EINVAL;
-  if (which != SHP_SELFTEST_GEMM && which != SHP_SELFTEST_OZAKI && which != SHP_SELFTEST_SKETCH)
+  if (which != SHP_SELFTEST_GEMM && which != SHP_SELFTEST_OZAKI && which != SHP_SELFTEST_SKETCH &&
+      which != SHP_SELFTEST_SKETCH_ALPHA)
     return SHP_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
@@ -911,6 +912,21 @@ int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void
     e.status = status;
     e.selftest = 1;
     CK(gemm_oz(sa.rows, sb.cols, n, n, n, 1, e, st));
+  } else if (which == SHP_SELFTEST_SKETCH_ALPHA) {
+    // the folded last pass of a d = 1 fit (V_3 = R V_2) times out; alpha starts
+    // as the stop test leaves it, NaN, and nothing may overwrite it
+    float* R = a.take<float>(n * n);
+    float* V = a.take<float>(4 * n * p);
+    double* gram = a.take<double>(15);
+    int* gcnt = a.take<int>(1);
+    float* alpha = alpha_out != nullptr ? alpha_out : a.take<float>(1);
+    const int64_t np = static_cast<int64_t>(n) * p;
+    CK(cudaMemsetAsync(alpha, 0xff, sizeof(float), st));  // a NaN pattern
+    bool fused = false;
+    CK(sketch_pass_alpha(R, n, n * n, V + 2 * np, 4 * np, V + 3 * np, 4 * np, p, 1, nullptr, st,
+                         status, V, 1, 0.5f, 1.f, alpha, nullptr, 0, 0, nullptr, gram, gcnt,
+                         &fused, 1));
+    if (!fused) return SHP_EUNSUPPORTED;  // the folded kernel is the TMA one (n p fits)
   } else {  // the alpha fit of one block (d = 1) whose first sketch pass times out
     float* R = a.take<float>(n * n);
     float* S = a.take<float>(n * p);

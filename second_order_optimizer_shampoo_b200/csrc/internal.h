@@ -160,7 +160,8 @@ cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, cons
                               int batch, const int* active, cudaStream_t st, int* tmo,
                               const float* V, int d, float lo, float hi, float* alpha,
                               float* report_alpha, int64_t report_stride, int report_slot,
-                              const int* it, double* gram, int* gcnt, bool* fused);
+                              const int* it, double* gram, int* gcnt, bool* fused,
+                              int selftest = 0);
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,

@@ -761,7 +761,8 @@ cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, cons
                               int batch, const int* active, cudaStream_t st, int* tmo,
                               const float* V, int d, float lo, float hi, float* alpha,
                               float* report_alpha, int64_t report_stride, int report_slot,
-                              const int* it, double* gram, int* gcnt, bool* fused) {
+                              const int* it, double* gram, int* gcnt, bool* fused,
+                              int selftest) {
   *fused = false;
   if (batch <= 0 || n <= 0) return cudaSuccess;
   if (gram != nullptr && gcnt != nullptr && (reinterpret_cast<uintptr_t>(R) & 15) == 0 &&
@@ -786,13 +787,14 @@ cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, cons
     bool done = false;
     if (p <= 4)
       done = launch_sketch_tma<4>(R, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p, batch,
-                                  active, nullptr, 0, tmo, 0, st, &e, &g, gram, gcnt);
+                                  active, nullptr, 0, tmo, selftest, st, &e, &g, gram, gcnt);
     else if (p <= 8)
       done = launch_sketch_tma<8>(R, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p, batch,
-                                  active, nullptr, 0, tmo, 0, st, &e, &g, gram, gcnt);
+                                  active, nullptr, 0, tmo, selftest, st, &e, &g, gram, gcnt);
     else if (p <= 16)
       done = launch_sketch_tma<16>(R, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p,
-                                   batch, active, nullptr, 0, tmo, 0, st, &e, &g, gram, gcnt);
+                                   batch, active, nullptr, 0, tmo, selftest, st, &e, &g, gram,
+                                   gcnt);
     if (done) {
       *fused = e == cudaSuccess;
       return e;
