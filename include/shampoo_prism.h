@@ -365,6 +365,11 @@ int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const floa
  *                        in (as inside the matrix-function loops): the same
  *                        hand-over in that pass; no warp completes the block,
  *                        so no alpha is solved
+ *   SHP_SELFTEST_SKETCH_CHAIN  the few-block sketch (every pass of an
+ *                        iteration and the fit in one cooperative launch, as
+ *                        the loops use it when the batch's R fits in shared
+ *                        memory): its first grid barrier, which CTA 0 never
+ *                        reaches; no alpha is solved
  * status: one device int32, set to SHP_ETIMEOUT by the kernel (cleared
  * first).  alpha_out: one device float (may be NULL), for the sketch cases
  * the fit's alpha, which must come out NaN (no fit on incomplete vectors; the
@@ -375,6 +380,7 @@ int prism_alpha_fit_noalloc(const float* R, int64_t n, int64_t batch, const floa
 #define SHP_SELFTEST_OZAKI 1
 #define SHP_SELFTEST_SKETCH 2
 #define SHP_SELFTEST_SKETCH_ALPHA 3
+#define SHP_SELFTEST_SKETCH_CHAIN 4
 #define SHP_SELFTEST_WS_BYTES (4u << 20)
 int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void* ws,
                               size_t ws_bytes, shp_stream stream);

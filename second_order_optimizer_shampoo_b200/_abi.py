@@ -26,7 +26,7 @@ SHP_OP_GRAM_EMA_STEPS = 5
 SHP_MATMUL_REUSE_A, SHP_MATMUL_REUSE_B, SHP_MATMUL_ACCUMULATE = 1, 2, 4
 # bounded-wait self-test
 SHP_SELFTEST_GEMM, SHP_SELFTEST_OZAKI, SHP_SELFTEST_SKETCH = 0, 1, 2
-SHP_SELFTEST_SKETCH_ALPHA = 3
+SHP_SELFTEST_SKETCH_ALPHA, SHP_SELFTEST_SKETCH_CHAIN = 3, 4
 SHP_SELFTEST_WS_BYTES = 4 << 20
 # fixed device scratch of prism_alpha_fit_noalloc
 SHP_NOALLOC_SCRATCH_BYTES = 4 << 20

@@ -68,6 +68,8 @@ Ctl carve_ctl(Arena& a, int64_t batch) {
   c.flag = a.take<int>(1);
   c.gram = a.take<double>(batch * 15);
   c.gcnt = a.take<int>(batch);
+  c.gbar = a.take<unsigned>(4);
+  c.gpart = a.take<double>(static_cast<size_t>(kChainMaxCtas) * 2 * 15);
   return c;
 }
 
@@ -243,7 +245,15 @@ int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass,
   const int64_t vbs = static_cast<int64_t>(2 * o->d + 2) * np;
   // a fitted alpha at fixed degree is solved inside the last pass (no alpha launch)
   const bool fuse = !o->fixed_alpha && !o->adaptive_degree && ctl.gram != nullptr;
+  bool chained = false;
   if (!o->fixed_alpha) {
+    // few blocks: every pass (and the fit) in one cooperative launch
+    CK(sketch_chain(Rs, n, nn, S_pass, np, ctl.it, V, o->p, o->d, batch, ctl.active, ctl.tmo,
+                    ctl.gbar, o->lo, o->hi, ctl.alpha, rep_alpha, rep_stride, rep_slot_base,
+                    fuse ? ctl.gpart : nullptr, fuse ? ctl.gcnt : nullptr, st, &chained));
+    if (chained && fuse) return SHP_OK;
+  }
+  if (!o->fixed_alpha && !chained) {
     CK(sketch_pass(Rs, nullptr, n, nn, S_pass, 0, V + np, vbs, o->p, batch, ctl.active, ctl.it,
                    np, st, ctl.tmo));
     const int last = 2 * o->d + 1;
@@ -878,7 +888,7 @@ int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void
                               size_t ws_bytes, shp_stream stream) {
   if (status == nullptr || ws == nullptr || ws_bytes < SHP_SELFTEST_WS_BYTES) return SHP_EINVAL;
   if (which != SHP_SELFTEST_GEMM && which != SHP_SELFTEST_OZAKI && which != SHP_SELFTEST_SKETCH &&
-      which != SHP_SELFTEST_SKETCH_ALPHA)
+      which != SHP_SELFTEST_SKETCH_ALPHA && which != SHP_SELFTEST_SKETCH_CHAIN)
     return SHP_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
@@ -927,6 +937,21 @@ int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void
                          status, V, 1, 0.5f, 1.f, alpha, nullptr, 0, 0, nullptr, gram, gcnt,
                          &fused, 1));
     if (!fused) return SHP_EUNSUPPORTED;  // the folded kernel is the TMA one (n p fits)
+  } else if (which == SHP_SELFTEST_SKETCH_CHAIN) {
+    // the few-block sketch of one block (d = 1, passes and fit in one
+    // cooperative launch) whose first grid barrier is never completed
+    float* R = a.take<float>(n * n);
+    float* S = a.take<float>(n * p);
+    float* V = a.take<float>(4 * n * p);
+    double* gpart = a.take<double>(static_cast<size_t>(kChainMaxCtas) * 2 * 15);
+    int* gcnt = a.take<int>(1);
+    unsigned* bar = a.take<unsigned>(4);
+    float* alpha = alpha_out != nullptr ? alpha_out : a.take<float>(1);
+    CK(cudaMemsetAsync(alpha, 0xff, sizeof(float), st));  // a NaN pattern
+    bool done = false;
+    CK(sketch_chain(R, n, n * n, S, 0, nullptr, V, p, 1, 1, nullptr, status, bar, 0.5f, 1.f,
+                    alpha, nullptr, 0, 0, gpart, gcnt, st, &done, 1));
+    if (!done) return SHP_EUNSUPPORTED;
   } else {  // the alpha fit of one block (d = 1) whose first sketch pass times out
     float* R = a.take<float>(n * n);
     float* S = a.take<float>(n * p);

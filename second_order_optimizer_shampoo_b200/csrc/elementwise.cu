@@ -80,6 +80,10 @@ __global__ void k_reset(Ctl ctl, int batch, int first, int start_degree) {
     for (int i = 0; i < 15; ++i) ctl.gram[b * 15 + i] = 0.0;
     ctl.gcnt[b] = 0;
   }
+  if (b == 0 && ctl.gbar != nullptr) {  // the few-block sketch's grid barrier
+    ctl.gbar[0] = 0u;
+    ctl.gbar[2] = 0u;
+  }
 }
 
 __global__ void __launch_bounds__(EW_THREADS)

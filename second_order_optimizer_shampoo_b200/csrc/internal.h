@@ -162,6 +162,26 @@ cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, cons
                               float* report_alpha, int64_t report_stride, int report_slot,
                               const int* it, double* gram, int* gcnt, bool* fused,
                               int selftest = 0);
+// Every pass V_1 = R S_k .. V_{2d+1} of one iteration in one cooperative
+// launch (S_k = S + (*it) * s_stride, shared by the batch; V as above), for a
+// batch whose rows of R fit in the CTAs' shared memory (no more blocks than
+// SMs).  With gpart/gcnt non-null the alpha fit of fixed degree d is folded
+// in: each CTA writes its partial Gram to its own slot of gpart
+// ([kChainMaxCtas][2][15] doubles) and the CTA that completes a block's count
+// in gcnt[b] (zero on entry; left zero) sums them and solves alpha.  bar:
+// three words of device scratch (arrivals, unused, abort) that reset_pass
+// clears; a grid barrier that runs out
+// sets tmo of every active block to ST_ETIMEOUT and the abort word, and
+// later launches then return at once.  selftest: CTA 0 skips the first
+// barrier, which the others wait out with the short limit.  *done = false:
+// not eligible, nothing launched (the caller runs the passes one by one).
+cudaError_t sketch_chain(const float* R, int64_t n, int64_t r_bstride, const float* S,
+                         int64_t s_stride, const int* it, float* V, int p, int d, int batch,
+                         const int* active, int* tmo, unsigned* bar, float lo, float hi,
+                         float* alpha, float* report_alpha, int64_t report_stride,
+                         int report_slot, double* gpart, int* gcnt, cudaStream_t st, bool* done,
+                         int selftest = 0);
+constexpr int kChainMaxCtas = 512;
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,
                         int fixed_alpha, const int* active, float* alpha, double* J_coef,
                         float* report_alpha, int64_t report_stride, int report_slot,
@@ -193,6 +213,8 @@ struct Ctl {
   int* flag;      // loop condition for the host-driven diagnostic loop
   double* gram;   // [batch][15] sketch Gram accumulated by the fused last pass
   int* gcnt;      // [batch] items of the fused last pass seen so far
+  unsigned* gbar;  // [4] grid barrier of the few-block sketch: arrivals, -, abort
+  double* gpart;   // [kChainMaxCtas][2][15] its CTAs' partial Grams
 };
 // Stop test of iteration k = *ctl.it for every active block.
 cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int max_iter, float tol,

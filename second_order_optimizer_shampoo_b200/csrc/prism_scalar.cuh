@@ -15,13 +15,23 @@
 namespace shp {
 namespace {
 
-// Coefficients of r_j(alpha) = T[j][0] + T[j][1] alpha + T[j][2] alpha^2 for
-// j = d..2d+1, written out from r(xi; alpha) = 1 - (1 - xi) g_d(xi; alpha)^2:
+// Coefficient of alpha^t in r_{d+j}(alpha) (j = 0 .. d+1), written out from
+// r(xi; alpha) = 1 - (1 - xi) g_d(xi; alpha)^2:
 //   d = 1 (f = 1):        r = (1-2a) xi + (2a - a^2) xi^2 + a^2 xi^3
 //   d = 2 (f = 1 + xi/2): r = (3/4 - 2a) xi^2 + (1/4 + a) xi^3 + (a - a^2) xi^4 + a^2 xi^5
-__device__ const double kRTab1[3][3] = {{1.0, -2.0, 0.0}, {0.0, 2.0, -1.0}, {0.0, 0.0, 1.0}};
-__device__ const double kRTab2[4][3] = {
-    {0.75, -2.0, 0.0}, {0.25, 1.0, 0.0}, {0.0, 1.0, -1.0}, {0.0, 0.0, 1.0}};
+// Called with compile-time arguments only, so every entry folds into the
+// arithmetic that uses it (the zeros vanish).
+template <int D>
+__device__ __forceinline__ constexpr double rtab(int j, int t) {
+  if constexpr (D == 1) {
+    constexpr double T[3][3] = {{1.0, -2.0, 0.0}, {0.0, 2.0, -1.0}, {0.0, 0.0, 1.0}};
+    return T[j][t];
+  } else {
+    constexpr double T[4][3] = {
+        {0.75, -2.0, 0.0}, {0.25, 1.0, 0.0}, {0.0, 1.0, -1.0}, {0.0, 0.0, 1.0}};
+    return T[j][t];
+  }
+}
 
 __device__ __forceinline__ double poly4(const double* c, double a) {
   return (((c[4] * a + c[3]) * a + c[2]) * a + c[1]) * a + c[0];
@@ -37,21 +47,24 @@ __device__ __forceinline__ double d2poly4(const double* c, double a) {
 // real roots of J'' (a quadratic), so each such piece holds at most one root
 // of J'; the root is bracketed, then polished by Newton.  The candidate with
 // the least J wins; values within 1e-12 (relative) of the best tie and go to
-// the smaller alpha; a constant or non-finite J gives lo.
+// the smaller alpha; a constant or non-finite J gives lo.  Everything below
+// works on named scalars and fully unrolled loops, so nothing leaves the
+// registers (indexed local arrays would go through local memory, and this
+// serial fp64 chain is on the critical path of every iteration).
 
-// Breakpoints lo < (roots of J'' inside) < hi; returns their count, or 0 when
-// J is constant or not finite (the minimiser is then lo).
-__device__ __forceinline__ int quartic_breaks(const double* c, double lo, double hi,
-                                              double* brk) {
+// The breakpoints lo = p0 <= p1 <= p2 <= p3 = hi: p1, p2 are the roots of J''
+// inside (lo, hi), an absent one repeating its left neighbour (an empty
+// piece).  False when J is constant or not finite (the minimiser is then lo).
+__device__ __forceinline__ bool quartic_breaks(const double* c, double lo, double hi,
+                                               double& p1, double& p2) {
   bool finite = true;
   double scale = 0.0;
+#pragma unroll
   for (int i = 0; i < 5; ++i) {
     if (!isfinite(c[i])) finite = false;
     if (i > 0) scale = fmax(scale, fabs(c[i]));
   }
-  if (!finite || scale == 0.0) return 0;
-  int nb = 0;
-  brk[nb++] = lo;
+  if (!finite || scale == 0.0) return false;
   const double qa = 12.0 * c[4], qb = 6.0 * c[3], qc = 2.0 * c[2];
   double r1 = NAN, r2 = NAN;
   if (qa != 0.0) {
@@ -74,139 +87,116 @@ __device__ __forceinline__ int quartic_breaks(const double* c, double lo, double
     r1 = r2;
     r2 = t;
   }
-  if (r1 > lo && r1 < hi) brk[nb++] = r1;
-  if (r2 > lo && r2 < hi && r2 != r1) brk[nb++] = r2;
-  brk[nb++] = hi;
-  return nb;
+  p1 = r1 > lo && r1 < hi ? r1 : lo;
+  p2 = r2 > lo && r2 < hi && r2 != r1 ? r2 : p1;
+  return true;
 }
 
-// Two Newton steps on J' from the bracket midpoint, kept inside [u0, v0].
-__device__ __forceinline__ double quartic_polish(const double* c, double u, double v, double u0,
-                                                 double v0) {
+// Newton on J' from the bracket midpoint, each step kept only while it stays
+// inside the bracket [u, v] (which holds the root).
+__device__ __forceinline__ double quartic_polish(const double* c, double u, double v) {
   double a = 0.5 * (u + v);
-  for (int it = 0; it < 2; ++it) {
+#pragma unroll
+  for (int it = 0; it < 3; ++it) {
     const double h = d2poly4(c, a);
-    if (h != 0.0) {
-      const double an = a - dpoly4(c, a) / h;
-      if (an >= u0 && an <= v0) a = an;
-    }
+    if (h == 0.0) break;
+    const double an = a - dpoly4(c, a) / h;
+    if (!(an >= u && an <= v)) break;
+    a = an;
   }
   return a;
 }
 
-// The candidate with the least J; ties (1e-12 relative) to the smaller alpha.
-__device__ __forceinline__ double quartic_pick(const double* c, const double* cand, int nc,
-                                               double hi) {
-  double best = poly4(c, cand[0]);
-  for (int i = 1; i < nc; ++i) best = fmin(best, poly4(c, cand[i]));
+// The root of J' on the piece [u, v] (J' monotone there) computed by a whole
+// warp (every lane returns it), or lo when J' keeps its sign: each round
+// evaluates J' at 32 interior points of the bracket at once and keeps the
+// 1/33 sub-interval where its sign first changes; four rounds narrow the
+// bracket a millionfold (relative), and the Newton polish then converges
+// quadratically from inside it.  All lanes run identical arithmetic, so they
+// agree on every decision.
+__device__ __forceinline__ double piece_root_warp(const double* c, double u, double v,
+                                                  double lo, double hi) {
+  const int lane = threadIdx.x & 31;
+  double fu = dpoly4(c, u);
+  const double fv = dpoly4(c, v);
+  if (fu == 0.0) return u;
+  if (fv == 0.0 || (fu < 0.0) == (fv < 0.0)) return lo;
+  const double u0 = u, v0 = v;
+  for (int it = 0; it < 16 && v - u > 1e-6 * fmax(1.0, fabs(u)); ++it) {
+    // the 32 interior points u + h, u + 2h, .. u + 32h with h = (v - u) / 33
+    // (a multiply by the rounded 1/33: any partition of the bracket works)
+    const double h = (v - u) * (1.0 / 33.0);
+    const double x = u + h * static_cast<double>(lane + 1);
+    const double fx = dpoly4(c, x);
+    const unsigned m = __ballot_sync(0xffffffffu, fx == 0.0 || (fx < 0.0) != (fu < 0.0));
+    const int i = m != 0u ? __ffs(static_cast<int>(m)) - 1 : 32;  // first sign change
+    const double nu = i == 0 ? u : u + h * static_cast<double>(i);
+    const double nv = i == 32 ? v : u + h * static_cast<double>(i + 1);
+    if (i != 0) fu = dpoly4(c, nu);
+    u = nu;
+    v = nv;
+    if (fu == 0.0) return u;
+  }
+  const double a = quartic_polish(c, fmax(u, u0), fmin(v, v0));
+  return a > lo && a < hi ? a : lo;
+}
+
+__device__ double argmin_quartic_warp(const double* c, double lo, double hi) {
+  double p1, p2;
+  if (!quartic_breaks(c, lo, hi, p1, p2)) return lo;
+  // candidates: the ends and one root of J' per piece (lo when none: a
+  // repeated candidate changes nothing)
+  const double a1 = piece_root_warp(c, lo, p1, lo, hi);
+  const double a2 = piece_root_warp(c, p1, p2, lo, hi);
+  const double a3 = piece_root_warp(c, p2, hi, lo, hi);
+  const double cand[5] = {lo, hi, a1, a2, a3};
+  double j[5];
+  double best = INFINITY;
+#pragma unroll
+  for (int i = 0; i < 5; ++i) {
+    j[i] = poly4(c, cand[i]);
+    best = fmin(best, j[i]);
+  }
   const double thr = best + 1e-12 * fmax(fabs(best), 1e-300);
   double pick = hi;
-  for (int i = 0; i < nc; ++i)
-    if (poly4(c, cand[i]) <= thr && cand[i] < pick) pick = cand[i];
+#pragma unroll
+  for (int i = 0; i < 5; ++i)
+    if (j[i] <= thr && cand[i] < pick) pick = cand[i];
   return pick;
 }
 
-// One thread: each monotone piece with a sign change of J' is bisected.
-__device__ double argmin_quartic(const double* c, double lo, double hi) {
-  double brk[4];
-  const int nb = quartic_breaks(c, lo, hi, brk);
-  if (nb == 0) return lo;
-  double cand[5];
-  int nc = 0;
-  cand[nc++] = lo;
-  cand[nc++] = hi;
-  for (int s = 0; s + 1 < nb; ++s) {
-    double u = brk[s], v = brk[s + 1];
-    double fu = dpoly4(c, u);
-    const double fv = dpoly4(c, v);
-    if (fu == 0.0) {
-      cand[nc++] = u;
-      continue;
-    }
-    if (fv == 0.0 || (fu < 0.0) == (fv < 0.0)) continue;
-    for (int it = 0; it < 200 && v - u > 1e-15 * fmax(1.0, fabs(u)); ++it) {
-      const double mid = 0.5 * (u + v);
-      const double fm = dpoly4(c, mid);
-      if (fm == 0.0) {
-        u = v = mid;
-        break;
-      }
-      if ((fm < 0.0) == (fu < 0.0)) {
-        u = mid;
-        fu = fm;
-      } else {
-        v = mid;
-      }
-    }
-    const double a = quartic_polish(c, u, v, brk[s], brk[s + 1]);
-    if (a > lo && a < hi) cand[nc++] = a;
-  }
-  return quartic_pick(c, cand, nc, hi);
-}
-
-// The same minimiser computed by a whole warp (every lane returns it): each
-// round evaluates J' at 32 interior points of the bracket at once and keeps
-// the 1/33 sub-interval where its sign first changes, so 10 rounds reach the
-// 1e-15 width that bisection needs 50 steps for.  All lanes run identical
-// arithmetic, so they agree on every decision.
-__device__ double argmin_quartic_warp(const double* c, double lo, double hi) {
-  const int lane = threadIdx.x & 31;
-  double brk[4];
-  const int nb = quartic_breaks(c, lo, hi, brk);
-  if (nb == 0) return lo;
-  double cand[5];
-  int nc = 0;
-  cand[nc++] = lo;
-  cand[nc++] = hi;
-  for (int s = 0; s + 1 < nb; ++s) {
-    double u = brk[s], v = brk[s + 1];
-    double fu = dpoly4(c, u);
-    const double fv = dpoly4(c, v);
-    if (fu == 0.0) {
-      cand[nc++] = u;
-      continue;
-    }
-    if (fv == 0.0 || (fu < 0.0) == (fv < 0.0)) continue;
-    for (int it = 0; it < 16 && v - u > 1e-15 * fmax(1.0, fabs(u)); ++it) {
-      // the 32 interior points u + h, u + 2h, .. u + 32h with h = (v - u) / 33
-      // (a multiply by the rounded 1/33: any partition of the bracket works,
-      // and a division per point is the round's longest dependency)
-      const double h = (v - u) * (1.0 / 33.0);
-      const double x = u + h * static_cast<double>(lane + 1);
-      const double fx = dpoly4(c, x);
-      const unsigned m = __ballot_sync(0xffffffffu, fx == 0.0 || (fx < 0.0) != (fu < 0.0));
-      const int i = m != 0u ? __ffs(static_cast<int>(m)) - 1 : 32;  // first sign change
-      const double nu = i == 0 ? u : u + h * static_cast<double>(i);
-      const double nv = i == 32 ? v : u + h * static_cast<double>(i + 1);
-      if (i != 0) fu = dpoly4(c, nu);
-      u = nu;
-      v = nv;
-      if (fu == 0.0) {
-        v = u;
-        break;
-      }
-    }
-    const double a = quartic_polish(c, u, v, brk[s], brk[s + 1]);
-    if (a > lo && a < hi) cand[nc++] = a;
-  }
-  return quartic_pick(c, cand, nc, hi);
-}
-
 // Coefficients (alpha^0 .. alpha^4) of J(alpha) = sum_ij r_i(alpha) r_j(alpha) M_ij
-// for the d + 2 sketch moments V_d .. V_{2d+1}; M is (d+2) x (d+2).
-__device__ void quartic_from_gram(const double (*M)[4], int d, double* coef) {
-  const int nv = d + 2;
-  double T[4][3];
-  for (int i = 0; i < nv; ++i)
-    for (int a = 0; a < 3; ++a) T[i][a] = d == 1 ? kRTab1[i][a] : kRTab2[i][a];
-  for (int i = 0; i < 5; ++i) coef[i] = 0.0;
-  for (int a = 0; a < 3; ++a)
-    for (int c = 0; c < 3; ++c) {
+// for the D + 2 sketch moments V_D .. V_{2D+1}; M is (D+2) x (D+2) (entries
+// past that unused).  U = M T first, then coef[a + c] += T[i][a] U[i][c].
+template <int D>
+__device__ __forceinline__ void quartic_from_gram_d(const double (&M)[4][4], double* coef) {
+  constexpr int NV = D + 2;
+  double U[NV][3];
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
       double s = 0.0;
-      for (int i = 0; i < nv; ++i)
-        for (int j = 0; j < nv; ++j) s += T[i][a] * M[i][j] * T[j][c];
-      coef[a + c] += s;
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        if (rtab<D>(j, t) != 0.0) s = fma(M[i][j], rtab<D>(j, t), s);
+      U[i][t] = s;
     }
+#pragma unroll
+  for (int k = 0; k < 5; ++k) coef[k] = 0.0;
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+#pragma unroll
+    for (int t = 0; t < 3; ++t)
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (rtab<D>(i, a) != 0.0) coef[a + t] = fma(rtab<D>(i, a), U[i][t], coef[a + t]);
+}
+__device__ __forceinline__ void quartic_from_gram(const double (&M)[4][4], int d, double* coef) {
+  if (d == 1)
+    quartic_from_gram_d<1>(M, coef);
+  else
+    quartic_from_gram_d<2>(M, coef);
 }
 
 // Stop rule of one pass at check k (k updates done), residual r = ||R_k||_F / sqrt(n):

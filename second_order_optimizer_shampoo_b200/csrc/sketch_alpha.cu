@@ -32,18 +32,14 @@ namespace {
 constexpr int SK_THREADS = 256;
 constexpr int SK_GROUPS = 2;  // row groups per warp in one CTA
 
-// Warp reduction of ROWS x P row sums (acc[r * P + j], one partial per lane)
-// by recursive halving: at the step with offset o each lane keeps the half of
-// its values selected by its lane bit o and adds the partner's copy of that
-// half, so 31 shuffles (for 32 values) leave lane l holding the total of
-// value l, where a shuffle tree per value would take 5 per value.  Stores
-// row0 + r, column j of Vb (rows >= n and columns >= p are not stored).
-template <int ROWS, int P>
-SHP_DEV void store_row_sums(float (&acc)[ROWS * P], int lane, int64_t row0, int64_t n, int p,
-                            float* Vb) {
-  constexpr int NV = ROWS * P;
-  static_assert(NV == 16 || NV == 32 || NV == 64, "16, 32 or 64 sums per warp");
-  constexpr int STEPS = NV >= 32 ? 5 : 4;
+// Warp reduction of NV per-lane partials by recursive halving: at the step
+// with offset o each lane keeps the half of its values selected by its lane
+// bit o and adds the partner's copy of that half, so 31 shuffles (for 32
+// values) leave lane l holding the total of value l, where a shuffle tree per
+// value would take 5 per value.  After 5 steps (NV >= 32) lane l holds the
+// totals of values l * (NV / 32) + k in acc[k], k < NV / 32.
+template <int NV, int STEPS>
+SHP_DEV void halve_lanes(float (&acc)[NV], int lane) {
 #pragma unroll
   for (int st = 0; st < STEPS; ++st) {
     const int o = 16 >> st;
@@ -56,6 +52,16 @@ SHP_DEV void store_row_sums(float (&acc)[ROWS * P], int lane, int64_t row0, int6
       acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
     }
   }
+}
+
+// Warp reduction of ROWS x P row sums (acc[r * P + j], one partial per lane);
+// stores row0 + r, column j of Vb (rows >= n and columns >= p are not stored).
+template <int ROWS, int P>
+SHP_DEV void store_row_sums(float (&acc)[ROWS * P], int lane, int64_t row0, int64_t n, int p,
+                            float* Vb) {
+  constexpr int NV = ROWS * P;
+  static_assert(NV == 16 || NV == 32 || NV == 64, "16, 32 or 64 sums per warp");
+  halve_lanes<NV, NV >= 32 ? 5 : 4>(acc, lane);
   if constexpr (NV == 16) {  // lanes l and l ^ 1 hold halves of value l >> 1
     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
     if ((lane & 1) == 0) {
@@ -235,6 +241,23 @@ struct AlphaArgs {
 };
 
 
+// G[i][j] (i, j < NV) from W rows of packed upper-triangle partial sums
+// red[w][idx] (idx running over i <= j row by row); unrolled, so G stays in
+// registers.
+template <int NV, int W>
+SHP_DEV void gram_unpack(const double (*red)[15], double (&G)[5][5]) {
+  int idx = 0;
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int j = i; j < NV; ++j, ++idx) {
+      double s = 0.0;
+#pragma unroll
+      for (int w = 0; w < W; ++w) s += red[w][idx];
+      G[i][j] = G[j][i] = s;
+    }
+}
+
 // alpha of block b from the Gram G[i][j] = <V_{first+i}, V_{first+j}> of its
 // sketch moments (first = d, or 1 with adaptive degree): the quartic J and its
 // minimiser on [lo, hi] by the calling warp (every lane takes part in the
@@ -247,9 +270,11 @@ SHP_DEV void alpha_solve_warp(const AlphaArgs& g, int b, const double (&G)[5][5]
   // fit at degree e on the Gram block starting at V_e (offset e - first)
   auto fit = [&](int e, double lo, double* coef) {
     double M[4][4];
-    const int o = e - first;
-    for (int i = 0; i < e + 2; ++i)
-      for (int j = 0; j < e + 2; ++j) M[i][j] = G[o + i][o + j];
+    const bool shift = e != first;  // first = 1 and e = 2: the block from V_2
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) M[i][j] = shift ? G[i + 1][j + 1] : G[i][j];
     quartic_from_gram(M, e, coef);
     return argmin_quartic_warp(coef, lo, static_cast<double>(g.hi));
   };
@@ -339,7 +364,9 @@ SHP_DEV void gram_flush(GramPart& gp, const AlphaArgs& g, double* gram, int* gcn
     __threadfence();
     double G[5][5];
     int idx = 0;
+#pragma unroll
     for (int i = 0; i < 5; ++i)
+#pragma unroll
       for (int j = i; j < 5; ++j, ++idx) G[i][j] = G[j][i] = __ldcg(&gram[b * 15 + idx]);
     if (tmo != nullptr && tmo[b] != 0) {
       if (lane == 0) g.alpha[b] = __int_as_float(0x7fc00000);
@@ -550,6 +577,321 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
     gram_flush(gp, fa, gram, gcnt, static_cast<int>(gpb) * ST_CONS, tmo);
 }
 
+// ---------------------------------------------------------------------------
+// Few blocks: every pass of one iteration in one cooperative launch.
+// With a handful of blocks a pass of the kernels above is a few microseconds
+// of work behind a launch and a pipeline ramp, five times per iteration.
+// Here each CTA keeps a contiguous range of the batch's rows of R (rows of at
+// most two blocks) in shared memory for the whole iteration; a pass stages
+// V_{j-1} of those blocks from global memory (L2), forms the CTA's rows of
+// V_j = R V_{j-1}, stores them, and a grid-wide barrier separates the passes.
+// The 8 warps split the columns (128 per step, a float4 per lane) and reduce
+// RC rows x P columns of partial sums at a time, across lanes by halving and
+// then across warps in shared memory.  The Gram of the fit needs only the
+// CTA's own rows of the moments, so the folded alpha of the last pass needs
+// no further barrier.  The barrier is bounded: one that runs out marks every
+// active block timed out and sets an abort word that ends the other CTAs'
+// waits, and later launches of the call return at once (the word is cleared
+// when a pass starts).
+constexpr int SC_THREADS = 256;
+constexpr int SC_WARPS = SC_THREADS / 32;
+
+template <int P>
+struct SkChain {
+  static constexpr int RC = P <= 8 ? 8 : 4;  // rows per chunk
+  static constexpr int NV = RC * P;          // partial sums per lane
+  // the warps' partial sums, later 16 x 15 doubles of the fit's reduction
+  static constexpr int RED_BYTES =
+      SC_WARPS * NV * 4 > 16 * 15 * 8 ? SC_WARPS * NV * 4 : 16 * 15 * 8;
+  static size_t smem_bytes(int64_t rpc, int64_t n) {
+    return static_cast<size_t>(rpc * n + 2 * P * (n + 4)) * 4 + RED_BYTES;
+  }
+};
+
+struct ChainArgs {
+  const float* R;
+  int64_t n, rbs;  // block size and block stride of R
+  const float* S;  // S_k = S + (*it) * s_stride, shared by the batch
+  int64_t s_stride;
+  const int* it;
+  float* V;  // V_j of block b at V + b * vbs + j * n * p
+  int64_t vbs;
+  int p, batch, last;  // passes j = 1 .. last
+  int vec;             // p == P and 16-byte aligned S and V: float4 staging
+  int64_t rpc;         // rows of the flattened batch per CTA (<= n)
+  const int* active;
+  int* tmo;
+  unsigned* bar;  // [0] arrivals, [1] generation, [2] abort
+  int selftest;   // CTA 0 skips the first barrier, which the others wait out
+};
+
+SHP_DEV unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier of a cooperative launch (every CTA resident) on a
+// counter that only grows within a pass (cleared when a pass starts): a CTA
+// arrives with one atomic add, which also tells it the count that completes
+// this barrier (the next multiple of the grid size), and waits until the
+// count reaches it, at most `limit` clock cycles or until the abort word is
+// set.  One round trip to arrive and one to see the last arrival.  False, in
+// every thread of the CTA, for a wait that gave up.
+SHP_DEV bool grid_barrier(unsigned* bar, long long limit, bool arrive) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned g = gridDim.x;
+    __threadfence();  // the CTA's stores (ordered by the block barrier) first
+    const unsigned seen = arrive ? atomicAdd(bar, 1u) : ld_acquire_gpu(bar);
+    const unsigned target = (seen / g + 1) * g;
+    if (seen + 1 != target || !arrive) {
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(bar) < target) {
+        if (ld_acquire_gpu(bar + 2) != 0 || clock64() - t0 > limit) {
+          ok = 0;
+          break;
+        }
+      }
+    }
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// The chain's alpha fit: for each of the CTA's segments (block segb[s], its
+// rows segr[s] .. segr[s] + rows[s] - 1) the CTA's partial Gram of V_d ..
+// V_{2d+1} goes to its own slot of gpart (15 doubles: no contended atomics);
+// the CTA that completes a block's count sums the partials of every CTA
+// holding rows of it (CTAs first .. last; in CTA i the block is segment 1
+// when i's first row lies in an earlier block) and solves alpha.  Half h of
+// the CTA reduces and solves segment h, so a CTA that completes two blocks
+// solves them side by side.  redd: 16 x 15 doubles of shared scratch.
+SHP_DEV void chain_fit(const AlphaArgs& fa, int nseg, const int (&segb)[2],
+                       const int64_t (&segr)[2], const int64_t (&rows)[2], const bool (&on)[2],
+                       double* gpart, int* gcnt, int64_t rpc, double* redd, const int* tmo) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n = fa.n;
+  __shared__ int last_s[2];
+  for (int s = 0; s < nseg; ++s) {
+    if (!on[s]) continue;
+    GramPart gp;
+    gram_reset(gp);
+    const int64_t w0 = rows[s] * warp / SC_WARPS, w1 = rows[s] * (warp + 1) / SC_WARPS;
+    gram_add(gp, fa, segb[s], segr[s] + w0, static_cast<int>(w1 - w0));
+#pragma unroll
+    for (int i = 0; i < 15; ++i) gp.part[i] = warp_sum(gp.part[i]);
+    if (lane == 0)
+#pragma unroll
+      for (int i = 0; i < 15; ++i) redd[warp * 15 + i] = gp.part[i];
+    __syncthreads();
+    if (threadIdx.x < 15) {
+      double t = 0.0;
+#pragma unroll
+      for (int w = 0; w < SC_WARPS; ++w) t += redd[w * 15 + threadIdx.x];
+      gpart[(blockIdx.x * 2 + s) * 15 + threadIdx.x] = t;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int b = segb[s];
+      const int64_t first = b * n / rpc, last = ((b + 1) * n - 1) / rpc;
+      __threadfence();  // the partial before the count
+      last_s[s] = atomicAdd(&gcnt[b], 1) == static_cast<int>(last - first);
+      if (last_s[s]) __threadfence();
+    }
+    __syncthreads();
+  }
+  // half h: 8 groups of 15 threads each sum every 8th CTA's partial of segment h
+  const int h = threadIdx.x / (SC_THREADS / 2), t = threadIdx.x % (SC_THREADS / 2);
+  const bool mine = h < nseg && on[h] && last_s[h] != 0;
+  if (mine && t < 8 * 15) {
+    const int b = segb[h], c = t % 15, grp = t / 15;
+    const int64_t first = b * n / rpc, last = ((b + 1) * n - 1) / rpc;
+    double acc = 0.0;
+#pragma unroll 4
+    for (int64_t i = first + grp; i <= last; i += 8) {
+      const int si = b * n > i * rpc ? 1 : 0;
+      acc += __ldcg(&gpart[(i * 2 + si) * 15 + c]);
+    }
+    redd[(h * 8 + grp) * 15 + c] = acc;
+  }
+  __syncthreads();
+  if (mine && t < 32) {  // the first warp of the half solves
+    const int b = segb[h];
+    double G[5][5] = {};
+    gram_unpack<5, 8>(reinterpret_cast<const double (*)[15]>(redd + h * 8 * 15), G);
+    if (tmo != nullptr && tmo[b] != 0) {
+      if (lane == 0) fa.alpha[b] = __int_as_float(0x7fc00000);
+    } else {
+      alpha_solve_warp(fa, b, G);
+    }
+    if (lane == 0) gcnt[b] = 0;
+  }
+}
+
+template <int P>
+__global__ void __launch_bounds__(SC_THREADS, 1)
+    k_sketch_chain(const ChainArgs c, const AlphaArgs fa, double* gpart, int* gcnt) {
+  count_kernel_run();
+  constexpr int RC = SkChain<P>::RC, NV = SkChain<P>::NV;
+  extern __shared__ __align__(16) float sc_smem[];
+  if (ld_acquire_gpu(c.bar + 2) != 0) return;  // an earlier launch of this pass gave up
+  const int64_t n = c.n, ldv = n + 4, np = n * c.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t total = static_cast<int64_t>(c.batch) * n;
+  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * c.rpc;
+  const int64_t g1 = g0 + c.rpc < total ? g0 + c.rpc : total;
+  float* Rs = sc_smem;               // the CTA's rows g0 .. g1 - 1, n floats each
+  float* Vs = Rs + c.rpc * n;        // [segment][P][ldv]: V_{j-1} transposed
+  float* red = Vs + 2 * P * ldv;     // [warp][NV]: the warps' partial sums (RED_BYTES)
+  // the CTA's rows as at most two segments, one block each: block, first row
+  // within the block, local rows [l0, l1)
+  int nseg = 0, segb[2] = {0, 0};
+  int64_t segr[2] = {0, 0}, segl0[2] = {0, 0}, segl1[2] = {0, 0};
+  bool on[2] = {false, false};
+  for (int64_t r = g0; r < g1 && nseg < 2;) {
+    const int b = static_cast<int>(r / n);
+    const int64_t end = (b + 1) * n < g1 ? (b + 1) * n : g1;
+    segb[nseg] = b;
+    segr[nseg] = r - b * n;
+    segl0[nseg] = r - g0;
+    segl1[nseg] = end - g0;
+    on[nseg] = c.active == nullptr || c.active[b] != 0;
+    ++nseg;
+    r = end;
+  }
+  const int k = c.it != nullptr ? *c.it : 0;
+
+  // R rows into shared memory (16-byte rows), eight loads in flight per thread
+  for (int s = 0; s < nseg; ++s) {
+    if (!on[s]) continue;
+    const float4* src = reinterpret_cast<const float4*>(c.R + segb[s] * c.rbs + segr[s] * n);
+    float4* dst = reinterpret_cast<float4*>(Rs + segl0[s] * n);
+    const int64_t cnt = (segl1[s] - segl0[s]) * n / 4;
+    for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
+      float4 t[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (i0 + u * SC_THREADS < cnt) t[u] = __ldg(src + i0 + u * SC_THREADS);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (i0 + u * SC_THREADS < cnt) dst[i0 + u * SC_THREADS] = t[u];
+    }
+  }
+
+  for (int j = 1; j <= c.last; ++j) {
+    if (j > 1) {
+      // V_{j-1} complete in every CTA; the self-test's CTA 0 never arrives
+      const bool test = c.selftest && j == 2;
+      if (!grid_barrier(c.bar, test ? SHP_SELFTEST_LIMIT : SHP_SPIN_LIMIT,
+                        !(test && blockIdx.x == 0))) {
+        if (threadIdx.x == 0) {
+          atomicExch(c.bar + 2, 1u);
+          if (c.tmo != nullptr)
+            for (int b = 0; b < c.batch; ++b)
+              if (c.active == nullptr || c.active[b] != 0) atomicExch(&c.tmo[b], ST_ETIMEOUT);
+        }
+        return;  // no copy is in flight: plain loads only
+      }
+    }
+    // stage V_{j-1} of the CTA's blocks (written by other CTAs: L2 loads)
+    for (int s = 0; s < nseg; ++s) {
+      if (!on[s]) continue;
+      const float* src = j == 1 ? c.S + static_cast<int64_t>(k) * c.s_stride
+                                : c.V + segb[s] * c.vbs + (j - 1) * np;
+      float* vs = Vs + s * P * ldv;
+      if (c.vec) {
+        const float4* s4 = reinterpret_cast<const float4*>(src);
+        const int64_t cnt = n * (P / 4);
+        for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
+          float4 t[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (i0 + u * SC_THREADS < cnt) t[u] = __ldcg(s4 + i0 + u * SC_THREADS);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int64_t i = i0 + u * SC_THREADS;
+            if (i >= cnt) break;
+            const int64_t col = i / (P / 4);
+            const int q = 4 * static_cast<int>(i % (P / 4));
+            vs[q * ldv + col] = t[u].x;
+            vs[(q + 1) * ldv + col] = t[u].y;
+            vs[(q + 2) * ldv + col] = t[u].z;
+            vs[(q + 3) * ldv + col] = t[u].w;
+          }
+        }
+      } else {
+        const int64_t cnt = n * P;
+        for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
+          float t[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int64_t i = i0 + u * SC_THREADS;
+            const int q = static_cast<int>(i % P);
+            t[u] = i < cnt && q < c.p ? __ldcg(src + (i / P) * c.p + q) : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int64_t i = i0 + u * SC_THREADS;
+            if (i < cnt) vs[(i % P) * ldv + i / P] = t[u];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    for (int s = 0; s < nseg; ++s) {
+      if (!on[s]) continue;
+      const float* vs = Vs + s * P * ldv;
+      float* out = c.V + segb[s] * c.vbs + j * np;
+      for (int64_t l0 = segl0[s]; l0 < segl1[s]; l0 += RC) {
+        float acc[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) acc[i] = 0.f;
+        for (int64_t col = warp * 128 + lane * 4; col < n; col += SC_WARPS * 128) {
+          float4 v[P];
+#pragma unroll
+          for (int q = 0; q < P; ++q) v[q] = *reinterpret_cast<const float4*>(vs + q * ldv + col);
+#pragma unroll
+          for (int r = 0; r < RC; ++r) {
+            const int64_t l = l0 + r < segl1[s] ? l0 + r : segl1[s] - 1;  // a spare row: not stored
+            const float4 x = *reinterpret_cast<const float4*>(Rs + l * n + col);
+#pragma unroll
+            for (int q = 0; q < P; ++q) {
+              float a = acc[r * P + q];
+              a = fmaf(x.x, v[q].x, a);
+              a = fmaf(x.y, v[q].y, a);
+              a = fmaf(x.z, v[q].z, a);
+              acc[r * P + q] = fmaf(x.w, v[q].w, a);
+            }
+          }
+        }
+        halve_lanes<NV, 5>(acc, lane);
+#pragma unroll
+        for (int i = 0; i < NV / 32; ++i) red[warp * NV + lane * (NV / 32) + i] = acc[i];
+        __syncthreads();
+        if (threadIdx.x < NV) {
+          float sum = 0.f;
+#pragma unroll
+          for (int w = 0; w < SC_WARPS; ++w) sum += red[w * NV + threadIdx.x];
+          const int r = threadIdx.x / P, q = threadIdx.x % P;
+          if (l0 + r < segl1[s] && q < c.p) out[(segr[s] + (l0 - segl0[s]) + r) * c.p + q] = sum;
+        }
+        __syncthreads();
+      }
+    }
+  }
+
+  // folded alpha: the Gram over the CTA's rows of V_d .. V_{2d+1}, stored by
+  // this CTA and ordered by the block barrier that ended the last chunk
+  if (gpart == nullptr) return;
+  const int64_t rows[2] = {segl1[0] - segl0[0], segl1[1] - segl0[1]};
+  chain_fit(fa, nseg, segb, segr, rows, on, gpart, gcnt, c.rpc, reinterpret_cast<double*>(red),
+            c.tmo);
+}
+
 // This thread's partial sums of <V_i, V_j> (i <= j < NV, packed row by row)
 // over elements threadIdx.x + k * AL_THREADS; NV is a compile-time constant so
 // that the 15 partials and the loaded values stay in registers.  Four
@@ -638,17 +980,13 @@ __global__ void __launch_bounds__(AL_THREADS) k_alpha(AlphaArgs g) {
   }
   __syncthreads();
   if (threadIdx.x >= 32) return;  // warp 0 forms J and finds its minimiser
-  double G[5][5];
-  {
-    int idx = 0;
-    for (int i = 0; i < nv; ++i)
-      for (int j = i; j < nv; ++j) {
-        double s = 0.0;
-        for (int w = 0; w < AL_THREADS / 32; ++w) s += red[w][idx];
-        G[i][j] = G[j][i] = s;
-        ++idx;
-      }
-  }
+  double G[5][5] = {};
+  if (nv == 3)
+    gram_unpack<3, AL_THREADS / 32>(red, G);
+  else if (nv == 4)
+    gram_unpack<4, AL_THREADS / 32>(red, G);
+  else
+    gram_unpack<5, AL_THREADS / 32>(red, G);
   alpha_solve_warp(g, b, G);
 }
 
@@ -713,6 +1051,56 @@ bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin,
                                                 it_stride, tmo, selftest, fa ? *fa : none,
                                                 fa ? gram : nullptr, fa ? gcnt : nullptr);
   *err = cudaGetLastError();
+  return true;
+}
+
+// The cooperative launch of k_sketch_chain: rows of the flattened batch are
+// spread evenly over at most one CTA per SM.  False (nothing launched) when
+// the batch has more blocks than SMs, the rows do not fit in shared memory,
+// or the device cannot launch the grid cooperatively.
+template <int P>
+bool launch_sketch_chain(ChainArgs c, const AlphaArgs* fa, double* gpart, int* gcnt,
+                         cudaStream_t st, cudaError_t* err) {
+  int dev = 0, sms = 0, coop = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+      sms <= 0 || coop == 0)
+    return false;
+  const int64_t total = static_cast<int64_t>(c.batch) * c.n;
+  c.rpc = (total + sms - 1) / sms;
+  if (c.rpc > c.n) return false;  // at most two blocks per CTA
+  const size_t smem = SkChain<P>::smem_bytes(c.rpc, c.n);
+  if (smem > 200 * 1024) return false;
+  auto kern = k_sketch_chain<P>;
+  static int set_for_dev[64];
+  if (set_for_dev[dev] == 0) {
+    *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (*err != cudaSuccess) return true;
+    set_for_dev[dev] = 1;
+  }
+  const int grid = static_cast<int>((total + c.rpc - 1) / c.rpc);
+  if (grid > kChainMaxCtas) return false;  // the partial-Gram slots
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, SC_THREADS, smem) !=
+          cudaSuccess ||
+      static_cast<int64_t>(per_sm) * sms < grid)
+    return false;
+  AlphaArgs none;
+  memset(&none, 0, sizeof(none));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(SC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  *err = cudaLaunchKernelEx(&cfg, kern, c, fa != nullptr ? *fa : none,
+                            fa != nullptr ? gpart : nullptr, fa != nullptr ? gcnt : nullptr);
   return true;
 }
 
@@ -802,6 +1190,67 @@ cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, cons
   }
   return sketch_pass(R, nullptr, n, r_bstride, Vin, vin_bstride, Vout, vout_bstride, p, batch,
                      active, nullptr, 0, st, tmo);
+}
+
+cudaError_t sketch_chain(const float* R, int64_t n, int64_t r_bstride, const float* S,
+                         int64_t s_stride, const int* it, float* V, int p, int d, int batch,
+                         const int* active, int* tmo, unsigned* bar, float lo, float hi,
+                         float* alpha, float* report_alpha, int64_t report_stride,
+                         int report_slot, double* gpart, int* gcnt, cudaStream_t st, bool* done,
+                         int selftest) {
+  *done = false;
+  if (batch <= 0 || n <= 0 || bar == nullptr || p < 1 || p > 16) return cudaSuccess;
+  if ((reinterpret_cast<uintptr_t>(R) & 15) != 0 || n % 4 != 0 || r_bstride % 4 != 0)
+    return cudaSuccess;
+  const int P = p <= 4 ? 4 : (p <= 8 ? 8 : 16);
+  ChainArgs c;
+  memset(&c, 0, sizeof(c));
+  c.R = R;
+  c.n = n;
+  c.rbs = r_bstride;
+  c.S = S;
+  c.s_stride = s_stride;
+  c.it = it;
+  c.V = V;
+  c.vbs = static_cast<int64_t>(2 * d + 2) * n * p;
+  c.p = p;
+  c.batch = batch;
+  c.last = 2 * d + 1;
+  c.vec = p == P && (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
+          (reinterpret_cast<uintptr_t>(V) & 15) == 0 && s_stride % 4 == 0;
+  c.active = active;
+  c.tmo = tmo;
+  c.bar = bar;
+  c.selftest = selftest;
+  AlphaArgs g;
+  memset(&g, 0, sizeof(g));
+  const bool fit = gpart != nullptr && gcnt != nullptr;
+  if (fit) {
+    g.tmo = tmo;
+    g.V = V;
+    g.n = n;
+    g.vbs = c.vbs;
+    g.p = p;
+    g.d = d;
+    g.lo = lo;
+    g.hi = hi;
+    g.active = active;
+    g.alpha = alpha;
+    g.rep = report_alpha;
+    g.rep_stride = report_stride;
+    g.rep_slot = report_slot;
+    g.it = it;
+  }
+  cudaError_t e = cudaSuccess;
+  bool launched = false;
+  if (P == 4)
+    launched = launch_sketch_chain<4>(c, fit ? &g : nullptr, gpart, gcnt, st, &e);
+  else if (P == 8)
+    launched = launch_sketch_chain<8>(c, fit ? &g : nullptr, gpart, gcnt, st, &e);
+  else
+    launched = launch_sketch_chain<16>(c, fit ? &g : nullptr, gpart, gcnt, st, &e);
+  *done = launched && e == cudaSuccess;
+  return e;
 }
 
 cudaError_t alpha_solve(const float* V, int64_t n, int p, int d, int batch, float lo, float hi,

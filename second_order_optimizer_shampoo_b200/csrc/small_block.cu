@@ -261,21 +261,28 @@ SHP_DEV void sketch_power(const float* R, const float* Vin, float* Vout, int n, 
   __syncthreads();
 }
 
-// alpha of degree e from V_e..V_{2e+1} (slot (j - 1) & 3 holds V_j): fp64
+// alpha of degree E from V_E..V_{2E+1} (slot (j - 1) & 3 holds V_j): fp64
 // Gram, quartic, minimiser on [lo, hi] by warp 0; every thread gets alpha and,
 // through *s_ratio, sqrt(J(alpha)) / ||V_1||_F (the predicted contraction).
-SHP_DEV float fit_degree(float* const* slot, int np, int e, double lo, double hi,
-                         double (*red)[10], float* s_alpha, float* s_ratio) {
-  const int tid = threadIdx.x, nv = e + 2;
+// E is a template argument so that every loop unrolls and the Gram stays in
+// registers.
+template <int E>
+SHP_DEV float fit_degree(float* const* slot, int np, double lo, double hi, double (*red)[10],
+                         float* s_alpha, float* s_ratio) {
+  constexpr int NV = E + 2;
+  const int tid = threadIdx.x;
   double part[10];
 #pragma unroll
   for (int i = 0; i < 10; ++i) part[i] = 0.0;
   for (int q = tid; q < np; q += SB_THREADS) {
-    double x[4];
-    for (int i = 0; i < nv; ++i) x[i] = static_cast<double>(slot[(e + i - 1) & 3][q]);
+    double x[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) x[i] = static_cast<double>(slot[(E + i - 1) & 3][q]);
     int idx = 0;
-    for (int i = 0; i < nv; ++i)
-      for (int j = i; j < nv; ++j) part[idx++] += x[i] * x[j];
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = i; j < NV; ++j) part[idx++] += x[i] * x[j];
   }
   const int warp = tid >> 5, lane = tid & 31;
 #pragma unroll
@@ -287,19 +294,22 @@ SHP_DEV float fit_degree(float* const* slot, int np, int e, double lo, double hi
   if (tid < 32) {  // warp 0: every lane forms J, the warp finds its minimiser
     double M[4][4];
     int idx = 0;
-    for (int i = 0; i < nv; ++i)
-      for (int j = i; j < nv; ++j) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = i; j < NV; ++j) {
         double s = 0.0;
+#pragma unroll
         for (int w = 0; w < SB_THREADS / 32; ++w) s += red[w][idx];
         M[i][j] = M[j][i] = s;
         ++idx;
       }
     double coef[5];
-    quartic_from_gram(M, e, coef);
+    quartic_from_gram_d<E>(M, coef);
     const double a = argmin_quartic_warp(coef, lo, hi);
     if (tid == 0) {
       *s_alpha = static_cast<float>(a);
-      const double base = M[0][0];  // ||V_1||^2 when e = 1
+      const double base = M[0][0];  // ||V_1||^2 when E = 1
       *s_ratio = base > 0.0 ? static_cast<float>(sqrt(fmax(poly4(coef, a), 0.0) / base)) : 0.f;
     }
   }
@@ -323,15 +333,15 @@ SHP_DEV float sketch_alpha(const float* R, int n, const SmallCfg& o, const float
   sketch_power(R, slot[1], slot[2], n, p);  // V_3
   float a = 0.f;
   if (*deg == 1) {
-    a = fit_degree(slot, np, 1, o.adaptive ? 0.5 : static_cast<double>(o.lo),
-                   static_cast<double>(o.hi), red, s_alpha, s_ratio);
+    a = fit_degree<1>(slot, np, o.adaptive ? 0.5 : static_cast<double>(o.lo),
+                      static_cast<double>(o.hi), red, s_alpha, s_ratio);
     if (!(o.adaptive && *s_ratio > o.raise_above)) return a;
     *deg = 2;
   }
   sketch_power(R, slot[2], slot[3], n, p);  // V_4
   sketch_power(R, slot[3], slot[0], n, p);  // V_5
-  return fit_degree(slot, np, 2, o.adaptive ? 0.375 : static_cast<double>(o.lo),
-                    static_cast<double>(o.hi), red, s_alpha, s_ratio);
+  return fit_degree<2>(slot, np, o.adaptive ? 0.375 : static_cast<double>(o.lo),
+                       static_cast<double>(o.hi), red, s_alpha, s_ratio);
 }
 
 // Report slots: resid[b][pass][k] (max_iter + 1 per pass), alpha[b][pass][k]

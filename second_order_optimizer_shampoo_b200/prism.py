@@ -330,11 +330,13 @@ def shp_matmul_f64(Amat, B, out=None, ws=None, reuse_a=False, reuse_b=False, acc
 
 def selftest_bounded_wait(which: str, device=None):
     """Make one bounded pipeline wait run out on purpose ("gemm", "ozaki",
-    "sketch" or "sketch_alpha", the last sketch pass with the fit folded in);
-    returns (status the kernel recorded, alpha of the sketch's fit) --
-    SHP_ETIMEOUT and, for the sketch cases, NaN are expected."""
+    "sketch", "sketch_alpha" -- the last sketch pass with the fit folded in --
+    or "sketch_chain", the few-block sketch's grid barrier); returns (status
+    the kernel recorded, alpha of the sketch's fit) -- SHP_ETIMEOUT and, for
+    the sketch cases, NaN are expected."""
     code = {"gemm": A.SHP_SELFTEST_GEMM, "ozaki": A.SHP_SELFTEST_OZAKI,
-            "sketch": A.SHP_SELFTEST_SKETCH, "sketch_alpha": A.SHP_SELFTEST_SKETCH_ALPHA}[which]
+            "sketch": A.SHP_SELFTEST_SKETCH, "sketch_alpha": A.SHP_SELFTEST_SKETCH_ALPHA,
+            "sketch_chain": A.SHP_SELFTEST_SKETCH_CHAIN}[which]
     device = device or torch.device("cuda", torch.cuda.current_device())
     status = torch.full((1,), -1, dtype=torch.int32, device=device)
     alpha = torch.zeros(1, dtype=torch.float32, device=device)

@@ -24,7 +24,7 @@ def prism():
     return p
 
 
-@pytest.mark.parametrize("which", ["gemm", "ozaki", "sketch", "sketch_alpha"])
+@pytest.mark.parametrize("which", ["gemm", "ozaki", "sketch", "sketch_alpha", "sketch_chain"])
 def test_bounded_wait_runs_out_and_the_context_survives(which):
     P = prism()
     status, alpha = P.selftest_bounded_wait(which)
