@@ -15,6 +15,8 @@ namespace {
 
 constexpr int EW_THREADS = 256;
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 dim3 ew_grid(int64_t count, int batch) {
   int64_t per = (count + EW_THREADS * 8 - 1) / (EW_THREADS * 8);
   if (per < 1) per = 1;
@@ -38,6 +40,26 @@ SHP_DEV float get(int fmt, const void* hi, const float* lo, int64_t off) {
   float v = static_cast<const float*>(hi)[off];
   if (fmt == OUT_SPLIT) v += lo[off];
   return v;
+}
+
+// Eight bf16 values of one 16-byte word, as fp32 (exact).
+SHP_DEV void unpack8(const uint4 u, float* x) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+// Eight fp32 values rounded to bf16 (nearest even) in one 16-byte word.
+SHP_DEV uint4 pack8(const float* x) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 t = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&t);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // Block-wide sum of a float partial into an fp32 atomic.
@@ -87,15 +109,36 @@ __global__ void k_reset(Ctl ctl, int batch, int first, int start_degree) {
 }
 
 __global__ void __launch_bounds__(EW_THREADS)
-    k_frob(const void* X, int bf16, int64_t count, double* dnorm) {
+    k_frob(const void* X, int bf16, int64_t count, double* dnorm, int vec) {
   count_kernel_run();
   const int b = blockIdx.y;
   double acc = 0.0;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
-       e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
-    const float v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(X)[b * count + e])
-                         : static_cast<const float*>(X)[b * count + e];
-    acc += static_cast<double>(v) * v;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * EW_THREADS;
+  const int64_t e0 = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x;
+  if (vec) {  // 16 bytes per load: 8 bf16 or 4 fp32 values (aligned, count a multiple)
+    const uint4* p = reinterpret_cast<const uint4*>(
+        static_cast<const uint8_t*>(X) + b * count * (bf16 ? 2 : 4));
+    const int64_t nv = count / (bf16 ? 8 : 4);
+    for (int64_t e = e0; e < nv; e += stride) {
+      const uint4 u = p[e];
+      if (bf16) {
+        float x[8];
+        unpack8(u, x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc += static_cast<double>(x[i]) * x[i];
+      } else {
+        const float x[4] = {__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                            __uint_as_float(u.w)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc += static_cast<double>(x[i]) * x[i];
+      }
+    }
+  } else {
+    for (int64_t e = e0; e < count; e += stride) {
+      const float v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(X)[b * count + e])
+                           : static_cast<const float*>(X)[b * count + e];
+      acc += static_cast<double>(v) * v;
+    }
   }
   __shared__ double red[EW_THREADS / 32];
   acc = warp_sum(acc);
@@ -288,13 +331,27 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_polar_init(const void* G, int gbf16, int64_t count, Ctl ctl, int fmt, void* Xhi,
-                 float* Xlo) {
+                 float* Xlo, int vec) {
   count_kernel_run();
   const int b = blockIdx.y;
   const float c = static_cast<float>(sqrt(ctl.dnorm[b]));
   if (blockIdx.x == 0 && threadIdx.x == 0) ctl.bs[b].c = c;
   // X_0 = G / ||G||_F as written: a zero block gives 0/0 and stops with
   // SHP_ENONFINITE at its first residual
+  if (vec) {  // bf16 to bf16, 8 values per 16-byte load and store
+    const uint4* g =
+        reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(G) + b * count);
+    uint4* x = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(Xhi) + b * count);
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count / 8;
+         e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
+      float v[8];
+      unpack8(g[e], v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = v[i] / c;
+      x[e] = pack8(v);
+    }
+    return;
+  }
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
        e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
     const int64_t off = b * count + e;
@@ -306,12 +363,21 @@ __global__ void __launch_bounds__(EW_THREADS)
 
 __global__ void __launch_bounds__(EW_THREADS)
     k_polar_finish(int64_t count, Ctl ctl, int fmt, const void* S0hi, const float* S0lo,
-                   const void* S1hi, const float* S1lo, void* X, int out_bf16) {
+                   const void* S1hi, const float* S1lo, void* X, int out_bf16, int vec) {
   count_kernel_run();
   const int b = blockIdx.y;
   const bool one = (ctl.bs[b].iters & 1) != 0;
   const void* hi = one ? S1hi : S0hi;
   const float* lo = one ? S1lo : S0lo;
+  if (vec) {  // bf16 to bf16: a 16-byte copy per thread and step
+    const uint4* src =
+        reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(hi) + b * count);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(X) + b * count);
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count / 8;
+         e += static_cast<int64_t>(gridDim.x) * EW_THREADS)
+      dst[e] = src[e];
+    return;
+  }
   for (int64_t e = blockIdx.x * static_cast<int64_t>(EW_THREADS) + threadIdx.x; e < count;
        e += static_cast<int64_t>(gridDim.x) * EW_THREADS) {
     const int64_t off = b * count + e;
@@ -354,7 +420,8 @@ cudaError_t reset_pass(const Ctl& ctl, int batch, int first_pass, cudaStream_t s
 
 cudaError_t frob_norm2(const void* X, int is_bf16, int64_t count, int batch, const Ctl& ctl,
                        cudaStream_t st) {
-  k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(X, is_bf16, count, ctl.dnorm);
+  const int vec = aligned16(X) && count % (is_bf16 ? 8 : 4) == 0;
+  k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(X, is_bf16, count, ctl.dnorm, vec);
   return cudaGetLastError();
 }
 
@@ -409,16 +476,19 @@ cudaError_t ema_replay(float* L, const float* P, int64_t n, int count, int batch
 
 cudaError_t polar_init(const void* G, int g_bf16, int64_t count, int batch, const Ctl& ctl,
                        int fmt, void* Xhi, float* Xlo, cudaStream_t st) {
+  const int vec = g_bf16 && fmt == OUT_BF16 && aligned16(G) && aligned16(Xhi) && count % 8 == 0;
   k_polar_init<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, g_bf16, count, ctl, fmt, Xhi,
-                                                             Xlo);
+                                                             Xlo, vec);
   return cudaGetLastError();
 }
 
 cudaError_t polar_finish(int64_t count, int batch, const Ctl& ctl, int fmt,
                          const void* const* Shi, const float* const* Slo, void* X_out,
                          int out_bf16, cudaStream_t st) {
-  k_polar_finish<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(count, ctl, fmt, Shi[0], Slo[0],
-                                                               Shi[1], Slo[1], X_out, out_bf16);
+  const int vec = out_bf16 && fmt == OUT_BF16 && aligned16(Shi[0]) && aligned16(Shi[1]) &&
+                  aligned16(X_out) && count % 8 == 0;
+  k_polar_finish<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(
+      count, ctl, fmt, Shi[0], Slo[0], Shi[1], Slo[1], X_out, out_bf16, vec);
   return cudaGetLastError();
 }
 
@@ -426,7 +496,8 @@ cudaError_t adaptive_step(const float* G, int64_t count, int batch, double* dn, 
                           float lr, float* eta, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(dn, 0, sizeof(double) * batch, st);
   if (e != cudaSuccess) return e;
-  k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, 0, count, dn);
+  k_frob<<<ew_grid(count, batch), EW_THREADS, 0, st>>>(G, 0, count, dn,
+                                                       aligned16(G) && count % 4 == 0);
   k_adaptive_eta<<<(batch + 127) / 128, 128, 0, st>>>(dn, acc, lr, eta, batch);
   return cudaGetLastError();
 }
