@@ -69,7 +69,7 @@ Ctl carve_ctl(Arena& a, int64_t batch) {
   c.gram = a.take<double>(batch * 15);
   c.gcnt = a.take<int>(batch);
   c.gbar = a.take<unsigned>(4);
-  c.gpart = a.take<double>(static_cast<size_t>(kChainMaxCtas) * 2 * 15);
+  c.gpart = a.take<double>(static_cast<size_t>(kChainMaxCtas) * 15);
   return c;
 }
 
@@ -943,7 +943,7 @@ int shp_selftest_bounded_wait(int which, int32_t* status, float* alpha_out, void
     float* R = a.take<float>(n * n);
     float* S = a.take<float>(n * p);
     float* V = a.take<float>(4 * n * p);
-    double* gpart = a.take<double>(static_cast<size_t>(kChainMaxCtas) * 2 * 15);
+    double* gpart = a.take<double>(static_cast<size_t>(kChainMaxCtas) * 15);
     int* gcnt = a.take<int>(1);
     unsigned* bar = a.take<unsigned>(4);
     float* alpha = alpha_out != nullptr ? alpha_out : a.take<float>(1);

@@ -167,7 +167,7 @@ cudaError_t sketch_pass_alpha(const float* R, int64_t n, int64_t r_bstride, cons
 // batch whose rows of R fit in the CTAs' shared memory (no more blocks than
 // SMs).  With gpart/gcnt non-null the alpha fit of fixed degree d is folded
 // in: each CTA writes its partial Gram to its own slot of gpart
-// ([kChainMaxCtas][2][15] doubles) and the CTA that completes a block's count
+// ([kChainMaxCtas][15] doubles) and the CTA that completes a block's count
 // in gcnt[b] (zero on entry; left zero) sums them and solves alpha.  bar:
 // three words of device scratch (arrivals, unused, abort) that reset_pass
 // clears; a grid barrier that runs out
@@ -214,7 +214,7 @@ struct Ctl {
   double* gram;   // [batch][15] sketch Gram accumulated by the fused last pass
   int* gcnt;      // [batch] items of the fused last pass seen so far
   unsigned* gbar;  // [4] grid barrier of the few-block sketch: arrivals, -, abort
-  double* gpart;   // [kChainMaxCtas][2][15] its CTAs' partial Grams
+  double* gpart;   // [kChainMaxCtas][15] its CTAs' partial Grams
 };
 // Stop test of iteration k = *ctl.it for every active block.
 cudaError_t control_step(const Ctl& ctl, int batch, int64_t n, int max_iter, float tol,

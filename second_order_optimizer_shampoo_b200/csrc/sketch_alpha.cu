@@ -581,18 +581,19 @@ __global__ void __launch_bounds__(32 * (ST_CONS + 1), 1)
 // Few blocks: every pass of one iteration in one cooperative launch.
 // With a handful of blocks a pass of the kernels above is a few microseconds
 // of work behind a launch and a pipeline ramp, five times per iteration.
-// Here each CTA keeps a contiguous range of the batch's rows of R (rows of at
-// most two blocks) in shared memory for the whole iteration; a pass stages
-// V_{j-1} of those blocks from global memory (L2), forms the CTA's rows of
-// V_j = R V_{j-1}, stores them, and a grid-wide barrier separates the passes.
-// The 8 warps split the columns (128 per step, a float4 per lane) and reduce
-// RC rows x P columns of partial sums at a time, across lanes by halving and
-// then across warps in shared memory.  The Gram of the fit needs only the
-// CTA's own rows of the moments, so the folded alpha of the last pass needs
-// no further barrier.  The barrier is bounded: one that runs out marks every
-// active block timed out and sets an abort word that ends the other CTAs'
-// waits, and later launches of the call return at once (the word is cleared
-// when a pass starts).
+// Here the SMs are shared out evenly among the blocks (cpb CTAs per block),
+// and each CTA keeps a contiguous range of rpc rows of one block's R in
+// shared memory for the whole iteration; a pass stages V_{j-1} of the block
+// from global memory (L2), forms the CTA's rows of V_j = R V_{j-1}, stores
+// them, and a grid-wide barrier separates the passes.  The 8 warps split the
+// columns (128 per step, a float4 per lane) and reduce RC rows x P columns
+// of partial sums at a time, across lanes by halving and then across warps
+// in shared memory.  The Gram of the fit needs only the CTA's own rows of
+// the moments, so the folded alpha of the last pass needs no further
+// barrier.  The barrier is bounded: one that runs out marks every active
+// block timed out and sets an abort word that ends the other CTAs' waits,
+// and later launches of the call return at once (the word is cleared when a
+// pass starts).
 constexpr int SC_THREADS = 256;
 constexpr int SC_WARPS = SC_THREADS / 32;
 
@@ -600,11 +601,11 @@ template <int P>
 struct SkChain {
   static constexpr int RC = P <= 8 ? 8 : 4;  // rows per chunk
   static constexpr int NV = RC * P;          // partial sums per lane
-  // the warps' partial sums, later 16 x 15 doubles of the fit's reduction
+  // the warps' partial sums, later 8 x 15 doubles of the fit's reduction
   static constexpr int RED_BYTES =
-      SC_WARPS * NV * 4 > 16 * 15 * 8 ? SC_WARPS * NV * 4 : 16 * 15 * 8;
+      SC_WARPS * NV * 4 > 8 * 15 * 8 ? SC_WARPS * NV * 4 : 8 * 15 * 8;
   static size_t smem_bytes(int64_t rpc, int64_t n) {
-    return static_cast<size_t>(rpc * n + 2 * P * (n + 4)) * 4 + RED_BYTES;
+    return static_cast<size_t>(rpc * n + P * (n + 4)) * 4 + RED_BYTES;
   }
 };
 
@@ -618,10 +619,11 @@ struct ChainArgs {
   int64_t vbs;
   int p, batch, last;  // passes j = 1 .. last
   int vec;             // p == P and 16-byte aligned S and V: float4 staging
-  int64_t rpc;         // rows of the flattened batch per CTA (<= n)
+  int cpb;             // CTAs per block: CTA c serves block c / cpb
+  int64_t rpc;         // rows per CTA (cpb * rpc >= n)
   const int* active;
   int* tmo;
-  unsigned* bar;  // [0] arrivals, [1] generation, [2] abort
+  unsigned* bar;  // [0] arrivals, [2] abort
   int selftest;   // CTA 0 skips the first barrier, which the others wait out
 };
 
@@ -662,67 +664,51 @@ SHP_DEV bool grid_barrier(unsigned* bar, long long limit, bool arrive) {
   return ok_s != 0;
 }
 
-// The chain's alpha fit: for each of the CTA's segments (block segb[s], its
-// rows segr[s] .. segr[s] + rows[s] - 1) the CTA's partial Gram of V_d ..
-// V_{2d+1} goes to its own slot of gpart (15 doubles: no contended atomics);
-// the CTA that completes a block's count sums the partials of every CTA
-// holding rows of it (CTAs first .. last; in CTA i the block is segment 1
-// when i's first row lies in an earlier block) and solves alpha.  Half h of
-// the CTA reduces and solves segment h, so a CTA that completes two blocks
-// solves them side by side.  redd: 16 x 15 doubles of shared scratch.
-SHP_DEV void chain_fit(const AlphaArgs& fa, int nseg, const int (&segb)[2],
-                       const int64_t (&segr)[2], const int64_t (&rows)[2], const bool (&on)[2],
-                       double* gpart, int* gcnt, int64_t rpc, double* redd, const int* tmo) {
+// The chain's alpha fit for block b: this CTA's partial Gram of V_d ..
+// V_{2d+1} over its rows [row0, row0 + rows) goes to its own slot of gpart
+// (15 doubles: no contended atomics); the CTA that completes the block's
+// count sums the partials of the block's cpb CTAs and solves alpha.
+// redd: 8 x 15 doubles of shared scratch.
+SHP_DEV void chain_fit(const AlphaArgs& fa, int b, int64_t row0, int64_t rows, double* gpart,
+                       int* gcnt, int cpb, double* redd, const int* tmo) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n = fa.n;
-  __shared__ int last_s[2];
-  for (int s = 0; s < nseg; ++s) {
-    if (!on[s]) continue;
-    GramPart gp;
-    gram_reset(gp);
-    const int64_t w0 = rows[s] * warp / SC_WARPS, w1 = rows[s] * (warp + 1) / SC_WARPS;
-    gram_add(gp, fa, segb[s], segr[s] + w0, static_cast<int>(w1 - w0));
+  __shared__ int last_s;
+  GramPart gp;
+  gram_reset(gp);
+  const int64_t w0 = rows * warp / SC_WARPS, w1 = rows * (warp + 1) / SC_WARPS;
+  gram_add(gp, fa, b, row0 + w0, static_cast<int>(w1 - w0));
 #pragma unroll
-    for (int i = 0; i < 15; ++i) gp.part[i] = warp_sum(gp.part[i]);
-    if (lane == 0)
+  for (int i = 0; i < 15; ++i) gp.part[i] = warp_sum(gp.part[i]);
+  if (lane == 0)
 #pragma unroll
-      for (int i = 0; i < 15; ++i) redd[warp * 15 + i] = gp.part[i];
-    __syncthreads();
-    if (threadIdx.x < 15) {
-      double t = 0.0;
+    for (int i = 0; i < 15; ++i) redd[warp * 15 + i] = gp.part[i];
+  __syncthreads();
+  if (threadIdx.x < 15) {
+    double t = 0.0;
 #pragma unroll
-      for (int w = 0; w < SC_WARPS; ++w) t += redd[w * 15 + threadIdx.x];
-      gpart[(blockIdx.x * 2 + s) * 15 + threadIdx.x] = t;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const int b = segb[s];
-      const int64_t first = b * n / rpc, last = ((b + 1) * n - 1) / rpc;
-      __threadfence();  // the partial before the count
-      last_s[s] = atomicAdd(&gcnt[b], 1) == static_cast<int>(last - first);
-      if (last_s[s]) __threadfence();
-    }
-    __syncthreads();
-  }
-  // half h: 8 groups of 15 threads each sum every 8th CTA's partial of segment h
-  const int h = threadIdx.x / (SC_THREADS / 2), t = threadIdx.x % (SC_THREADS / 2);
-  const bool mine = h < nseg && on[h] && last_s[h] != 0;
-  if (mine && t < 8 * 15) {
-    const int b = segb[h], c = t % 15, grp = t / 15;
-    const int64_t first = b * n / rpc, last = ((b + 1) * n - 1) / rpc;
-    double acc = 0.0;
-#pragma unroll 4
-    for (int64_t i = first + grp; i <= last; i += 8) {
-      const int si = b * n > i * rpc ? 1 : 0;
-      acc += __ldcg(&gpart[(i * 2 + si) * 15 + c]);
-    }
-    redd[(h * 8 + grp) * 15 + c] = acc;
+    for (int w = 0; w < SC_WARPS; ++w) t += redd[w * 15 + threadIdx.x];
+    gpart[blockIdx.x * 15 + threadIdx.x] = t;
   }
   __syncthreads();
-  if (mine && t < 32) {  // the first warp of the half solves
-    const int b = segb[h];
+  if (threadIdx.x == 0) {
+    __threadfence();  // the partial before the count
+    last_s = atomicAdd(&gcnt[b], 1) == cpb - 1;
+    if (last_s) __threadfence();
+  }
+  __syncthreads();
+  if (!last_s) return;
+  // the last CTA of block b: 8 groups of 15 threads each sum every 8th CTA
+  if (threadIdx.x < 8 * 15) {
+    const int c = threadIdx.x % 15, grp = threadIdx.x / 15;
+    double acc = 0.0;
+#pragma unroll 4
+    for (int i = grp; i < cpb; i += 8) acc += __ldcg(&gpart[(b * cpb + i) * 15 + c]);
+    redd[grp * 15 + c] = acc;
+  }
+  __syncthreads();
+  if (warp == 0) {
     double G[5][5] = {};
-    gram_unpack<5, 8>(reinterpret_cast<const double (*)[15]>(redd + h * 8 * 15), G);
+    gram_unpack<5, 8>(reinterpret_cast<const double (*)[15]>(redd), G);
     if (tmo != nullptr && tmo[b] != 0) {
       if (lane == 0) fa.alpha[b] = __int_as_float(0x7fc00000);
     } else {
@@ -741,36 +727,20 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
   if (ld_acquire_gpu(c.bar + 2) != 0) return;  // an earlier launch of this pass gave up
   const int64_t n = c.n, ldv = n + 4, np = n * c.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t total = static_cast<int64_t>(c.batch) * n;
-  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * c.rpc;
-  const int64_t g1 = g0 + c.rpc < total ? g0 + c.rpc : total;
-  float* Rs = sc_smem;               // the CTA's rows g0 .. g1 - 1, n floats each
-  float* Vs = Rs + c.rpc * n;        // [segment][P][ldv]: V_{j-1} transposed
-  float* red = Vs + 2 * P * ldv;     // [warp][NV]: the warps' partial sums (RED_BYTES)
-  // the CTA's rows as at most two segments, one block each: block, first row
-  // within the block, local rows [l0, l1)
-  int nseg = 0, segb[2] = {0, 0};
-  int64_t segr[2] = {0, 0}, segl0[2] = {0, 0}, segl1[2] = {0, 0};
-  bool on[2] = {false, false};
-  for (int64_t r = g0; r < g1 && nseg < 2;) {
-    const int b = static_cast<int>(r / n);
-    const int64_t end = (b + 1) * n < g1 ? (b + 1) * n : g1;
-    segb[nseg] = b;
-    segr[nseg] = r - b * n;
-    segl0[nseg] = r - g0;
-    segl1[nseg] = end - g0;
-    on[nseg] = c.active == nullptr || c.active[b] != 0;
-    ++nseg;
-    r = end;
-  }
+  const int b = static_cast<int>(blockIdx.x) / c.cpb;
+  const int64_t r0 = (static_cast<int64_t>(blockIdx.x) % c.cpb) * c.rpc;
+  const int64_t rows = n - r0 < c.rpc ? (n - r0 > 0 ? n - r0 : 0) : c.rpc;
+  const bool on = rows > 0 && (c.active == nullptr || c.active[b] != 0);
+  float* Rs = sc_smem;           // the CTA's rows r0 .. r0 + rows - 1, n floats each
+  float* Vs = Rs + c.rpc * n;    // [P][ldv]: V_{j-1} transposed
+  float* red = Vs + P * ldv;     // [warp][NV]: the warps' partial sums (RED_BYTES)
   const int k = c.it != nullptr ? *c.it : 0;
 
   // R rows into shared memory (16-byte rows), eight loads in flight per thread
-  for (int s = 0; s < nseg; ++s) {
-    if (!on[s]) continue;
-    const float4* src = reinterpret_cast<const float4*>(c.R + segb[s] * c.rbs + segr[s] * n);
-    float4* dst = reinterpret_cast<float4*>(Rs + segl0[s] * n);
-    const int64_t cnt = (segl1[s] - segl0[s]) * n / 4;
+  if (on) {
+    const float4* src = reinterpret_cast<const float4*>(c.R + b * c.rbs + r0 * n);
+    float4* dst = reinterpret_cast<float4*>(Rs);
+    const int64_t cnt = rows * n / 4;
     for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
       float4 t[8];
 #pragma unroll
@@ -791,105 +761,96 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
         if (threadIdx.x == 0) {
           atomicExch(c.bar + 2, 1u);
           if (c.tmo != nullptr)
-            for (int b = 0; b < c.batch; ++b)
-              if (c.active == nullptr || c.active[b] != 0) atomicExch(&c.tmo[b], ST_ETIMEOUT);
+            for (int bb = 0; bb < c.batch; ++bb)
+              if (c.active == nullptr || c.active[bb] != 0) atomicExch(&c.tmo[bb], ST_ETIMEOUT);
         }
         return;  // no copy is in flight: plain loads only
       }
     }
-    // stage V_{j-1} of the CTA's blocks (written by other CTAs: L2 loads)
-    for (int s = 0; s < nseg; ++s) {
-      if (!on[s]) continue;
-      const float* src = j == 1 ? c.S + static_cast<int64_t>(k) * c.s_stride
-                                : c.V + segb[s] * c.vbs + (j - 1) * np;
-      float* vs = Vs + s * P * ldv;
-      if (c.vec) {
-        const float4* s4 = reinterpret_cast<const float4*>(src);
-        const int64_t cnt = n * (P / 4);
-        for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
-          float4 t[8];
+    if (!on) continue;  // the barriers are still taken
+    // stage V_{j-1} of the block (written by other CTAs: L2 loads)
+    const float* src = j == 1 ? c.S + static_cast<int64_t>(k) * c.s_stride
+                              : c.V + b * c.vbs + (j - 1) * np;
+    if (c.vec) {
+      const float4* s4 = reinterpret_cast<const float4*>(src);
+      const int64_t cnt = n * (P / 4);
+      for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
+        float4 t[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (i0 + u * SC_THREADS < cnt) t[u] = __ldcg(s4 + i0 + u * SC_THREADS);
+        for (int u = 0; u < 8; ++u)
+          if (i0 + u * SC_THREADS < cnt) t[u] = __ldcg(s4 + i0 + u * SC_THREADS);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int64_t i = i0 + u * SC_THREADS;
-            if (i >= cnt) break;
-            const int64_t col = i / (P / 4);
-            const int q = 4 * static_cast<int>(i % (P / 4));
-            vs[q * ldv + col] = t[u].x;
-            vs[(q + 1) * ldv + col] = t[u].y;
-            vs[(q + 2) * ldv + col] = t[u].z;
-            vs[(q + 3) * ldv + col] = t[u].w;
-          }
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + u * SC_THREADS;
+          if (i >= cnt) break;
+          const int64_t col = i / (P / 4);
+          const int q = 4 * static_cast<int>(i % (P / 4));
+          Vs[q * ldv + col] = t[u].x;
+          Vs[(q + 1) * ldv + col] = t[u].y;
+          Vs[(q + 2) * ldv + col] = t[u].z;
+          Vs[(q + 3) * ldv + col] = t[u].w;
         }
-      } else {
-        const int64_t cnt = n * P;
-        for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
-          float t[8];
+      }
+    } else {
+      const int64_t cnt = n * P;
+      for (int64_t i0 = threadIdx.x; i0 < cnt; i0 += 8 * SC_THREADS) {
+        float t[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int64_t i = i0 + u * SC_THREADS;
-            const int q = static_cast<int>(i % P);
-            t[u] = i < cnt && q < c.p ? __ldcg(src + (i / P) * c.p + q) : 0.f;
-          }
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + u * SC_THREADS;
+          const int q = static_cast<int>(i % P);
+          t[u] = i < cnt && q < c.p ? __ldcg(src + (i / P) * c.p + q) : 0.f;
+        }
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int64_t i = i0 + u * SC_THREADS;
-            if (i < cnt) vs[(i % P) * ldv + i / P] = t[u];
-          }
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + u * SC_THREADS;
+          if (i < cnt) Vs[(i % P) * ldv + i / P] = t[u];
         }
       }
     }
     __syncthreads();
-    for (int s = 0; s < nseg; ++s) {
-      if (!on[s]) continue;
-      const float* vs = Vs + s * P * ldv;
-      float* out = c.V + segb[s] * c.vbs + j * np;
-      for (int64_t l0 = segl0[s]; l0 < segl1[s]; l0 += RC) {
-        float acc[NV];
+    float* out = c.V + b * c.vbs + j * np;
+    for (int64_t l0 = 0; l0 < rows; l0 += RC) {
+      float acc[NV];
 #pragma unroll
-        for (int i = 0; i < NV; ++i) acc[i] = 0.f;
-        for (int64_t col = warp * 128 + lane * 4; col < n; col += SC_WARPS * 128) {
-          float4 v[P];
+      for (int i = 0; i < NV; ++i) acc[i] = 0.f;
+      for (int64_t col = warp * 128 + lane * 4; col < n; col += SC_WARPS * 128) {
+        float4 v[P];
 #pragma unroll
-          for (int q = 0; q < P; ++q) v[q] = *reinterpret_cast<const float4*>(vs + q * ldv + col);
+        for (int q = 0; q < P; ++q) v[q] = *reinterpret_cast<const float4*>(Vs + q * ldv + col);
 #pragma unroll
-          for (int r = 0; r < RC; ++r) {
-            const int64_t l = l0 + r < segl1[s] ? l0 + r : segl1[s] - 1;  // a spare row: not stored
-            const float4 x = *reinterpret_cast<const float4*>(Rs + l * n + col);
+        for (int r = 0; r < RC; ++r) {
+          const int64_t l = l0 + r < rows ? l0 + r : rows - 1;  // a spare row: not stored
+          const float4 x = *reinterpret_cast<const float4*>(Rs + l * n + col);
 #pragma unroll
-            for (int q = 0; q < P; ++q) {
-              float a = acc[r * P + q];
-              a = fmaf(x.x, v[q].x, a);
-              a = fmaf(x.y, v[q].y, a);
-              a = fmaf(x.z, v[q].z, a);
-              acc[r * P + q] = fmaf(x.w, v[q].w, a);
-            }
+          for (int q = 0; q < P; ++q) {
+            float a = acc[r * P + q];
+            a = fmaf(x.x, v[q].x, a);
+            a = fmaf(x.y, v[q].y, a);
+            a = fmaf(x.z, v[q].z, a);
+            acc[r * P + q] = fmaf(x.w, v[q].w, a);
           }
         }
-        halve_lanes<NV, 5>(acc, lane);
-#pragma unroll
-        for (int i = 0; i < NV / 32; ++i) red[warp * NV + lane * (NV / 32) + i] = acc[i];
-        __syncthreads();
-        if (threadIdx.x < NV) {
-          float sum = 0.f;
-#pragma unroll
-          for (int w = 0; w < SC_WARPS; ++w) sum += red[w * NV + threadIdx.x];
-          const int r = threadIdx.x / P, q = threadIdx.x % P;
-          if (l0 + r < segl1[s] && q < c.p) out[(segr[s] + (l0 - segl0[s]) + r) * c.p + q] = sum;
-        }
-        __syncthreads();
       }
+      halve_lanes<NV, 5>(acc, lane);
+#pragma unroll
+      for (int i = 0; i < NV / 32; ++i) red[warp * NV + lane * (NV / 32) + i] = acc[i];
+      __syncthreads();
+      if (threadIdx.x < NV) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < SC_WARPS; ++w) sum += red[w * NV + threadIdx.x];
+        const int r = threadIdx.x / P, q = threadIdx.x % P;
+        if (l0 + r < rows && q < c.p) out[(r0 + l0 + r) * c.p + q] = sum;
+      }
+      __syncthreads();
     }
   }
 
   // folded alpha: the Gram over the CTA's rows of V_d .. V_{2d+1}, stored by
   // this CTA and ordered by the block barrier that ended the last chunk
-  if (gpart == nullptr) return;
-  const int64_t rows[2] = {segl1[0] - segl0[0], segl1[1] - segl0[1]};
-  chain_fit(fa, nseg, segb, segr, rows, on, gpart, gcnt, c.rpc, reinterpret_cast<double*>(red),
-            c.tmo);
+  if (gpart == nullptr || !on) return;
+  chain_fit(fa, b, r0, rows, gpart, gcnt, c.cpb, reinterpret_cast<double*>(red), c.tmo);
 }
 
 // This thread's partial sums of <V_i, V_j> (i <= j < NV, packed row by row)
@@ -1054,10 +1015,10 @@ bool launch_sketch_tma(const float* R, int64_t n, int64_t rbs, const float* Vin,
   return true;
 }
 
-// The cooperative launch of k_sketch_chain: rows of the flattened batch are
-// spread evenly over at most one CTA per SM.  False (nothing launched) when
-// the batch has more blocks than SMs, the rows do not fit in shared memory,
-// or the device cannot launch the grid cooperatively.
+// The cooperative launch of k_sketch_chain: the SMs are shared out evenly
+// among the blocks (cpb CTAs of rpc rows each per block).  False (nothing
+// launched) when the batch has more blocks than SMs, a CTA's rows do not fit
+// in shared memory, or the device cannot launch the grid cooperatively.
 template <int P>
 bool launch_sketch_chain(ChainArgs c, const AlphaArgs* fa, double* gpart, int* gcnt,
                          cudaStream_t st, cudaError_t* err) {
@@ -1065,11 +1026,11 @@ bool launch_sketch_chain(ChainArgs c, const AlphaArgs* fa, double* gpart, int* g
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
-      sms <= 0 || coop == 0)
+      sms <= 0 || coop == 0 || c.batch > sms)
     return false;
-  const int64_t total = static_cast<int64_t>(c.batch) * c.n;
-  c.rpc = (total + sms - 1) / sms;
-  if (c.rpc > c.n) return false;  // at most two blocks per CTA
+  const int64_t cpb_max = sms / c.batch;
+  c.rpc = (c.n + cpb_max - 1) / cpb_max;
+  c.cpb = static_cast<int>((c.n + c.rpc - 1) / c.rpc);  // every CTA has rows
   const size_t smem = SkChain<P>::smem_bytes(c.rpc, c.n);
   if (smem > 200 * 1024) return false;
   auto kern = k_sketch_chain<P>;
@@ -1079,7 +1040,7 @@ bool launch_sketch_chain(ChainArgs c, const AlphaArgs* fa, double* gpart, int* g
     if (*err != cudaSuccess) return true;
     set_for_dev[dev] = 1;
   }
-  const int grid = static_cast<int>((total + c.rpc - 1) / c.rpc);
+  const int grid = c.cpb * c.batch;
   if (grid > kChainMaxCtas) return false;  // the partial-Gram slots
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, SC_THREADS, smem) !=
