@@ -100,7 +100,7 @@ typedef enum { SHP_OP_INV_ROOT = 0, SHP_OP_POLAR = 1, SHP_OP_ALPHA_FIT = 2, SHP_
  *               degree e is then [c_e, hi] with c_e its Taylor coefficient
  *               (1/2, 3/8) and lo is not used; needs fixed_alpha = 0
  *   host_loop   0 (default): the iteration loop runs on the device inside a
- *               cached CUDA graph (conditional WHILE/IF nodes), with no host
+ *               cached CUDA graph (a conditional WHILE node), with no host
  *               synchronisation; 1: the same kernels are launched from a host
  *               loop that synchronises the stream once per iteration to read
  *               the loop condition (for profilers and launch tracers that do

@@ -280,11 +280,13 @@ int sketch_and_alpha(const float* Rs, int64_t n, int batch, const float* S_pass,
 // ------------------------------------------------------------------------
 // Device-side iteration loop.  Each Newton-Schulz pass is recorded into a CUDA
 // graph: the k = 0 step, then a conditional WHILE node whose body runs two
-// steps (odd k on ping-pong slot 1, then, behind a conditional IF, even k on
-// slot 0).  After every step a one-CTA kernel advances the device iteration
-// counter and sets the condition to "some block still active"; blocks stop
-// independently in k_control.  No host synchronisation, and no launches for
-// steps after the last block has stopped.  Graphs are cached by the call's
+// steps (odd k on ping-pong slot 1, then even k on slot 0).  After every step
+// a one-CTA kernel advances the device iteration counter; the one after the
+// even step sets the condition to "some block still active".  Blocks stop
+// independently in k_control, and every kernel of a step returns at once for
+// a stopped block, so the even step of the body pass in which the last block
+// stopped is a few empty launches (an IF node around it measured costlier
+// than that).  No host synchronisation.  Graphs are cached by the call's
 // pointers and sizes.
 
 struct CallKey {
@@ -358,29 +360,19 @@ int record_loop(cudaStream_t const* cs, cudaGraph_t g, const Ctl& ctl, int batch
   const cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
   int r = iter(0, true, cs[0]);
   if (r != SHP_OK) return r;
-  cudaGraphConditionalHandle hw, hif;
+  cudaGraphConditionalHandle hw;
   CK(cudaGraphConditionalHandleCreate(&hw, g, 0, cudaGraphCondAssignDefault));
   CK(loop_step(ctl, batch, 1, max_iter, hw, cs[0]));
-  cudaGraph_t body = nullptr, body2 = nullptr;
+  cudaGraph_t body = nullptr;
   CK(add_conditional(cs[0], hw, cudaGraphCondTypeWhile, &body));
-  CK(cudaGraphConditionalHandleCreate(&hif, body, 0, cudaGraphCondAssignDefault));
   CK(cudaStreamBeginCaptureToGraph(cs[1], body, nullptr, nullptr, 0, mode));
+  // two steps per pass of the body, the second without a conditional of its
+  // own: an IF node costs more than the step it would skip, which (all blocks
+  // stopped) is a few launches that return at once
   r = iter(1, false, cs[1]);
-  if (r == SHP_OK && loop_step(ctl, batch, 1, max_iter, hif, cs[1]) != cudaSuccess) r = SHP_ECUDA;
-  if (r == SHP_OK && add_conditional(cs[1], hif, cudaGraphCondTypeIf, &body2) != cudaSuccess)
-    r = SHP_ECUDA;
-  if (r == SHP_OK) {
-    if (cudaStreamBeginCaptureToGraph(cs[2], body2, nullptr, nullptr, 0, mode) != cudaSuccess) {
-      r = SHP_ECUDA;
-    } else {
-      r = iter(0, false, cs[2]);
-      if (r == SHP_OK && loop_step(ctl, batch, 1, max_iter, hif, cs[2]) != cudaSuccess)
-        r = SHP_ECUDA;
-      cudaGraph_t g2 = nullptr;
-      if (cudaStreamEndCapture(cs[2], &g2) != cudaSuccess && r == SHP_OK) r = SHP_ECUDA;
-    }
-  }
-  if (r == SHP_OK && loop_step(ctl, batch, 0, max_iter, hw, cs[1]) != cudaSuccess) r = SHP_ECUDA;
+  if (r == SHP_OK && loop_step(ctl, batch, 1, max_iter, 0, cs[1]) != cudaSuccess) r = SHP_ECUDA;
+  if (r == SHP_OK) r = iter(0, false, cs[1]);
+  if (r == SHP_OK && loop_step(ctl, batch, 1, max_iter, hw, cs[1]) != cudaSuccess) r = SHP_ECUDA;
   cudaGraph_t g1 = nullptr;
   if (cudaStreamEndCapture(cs[1], &g1) != cudaSuccess && r == SHP_OK) r = SHP_ECUDA;
   return r;
