@@ -113,6 +113,25 @@ def test_inv_root_powers_ragged_batch(power, d):
         assert relerr(X[b], o.spd_power_eigh(A[b], q)) <= 1e-5
 
 
+@pytest.mark.parametrize("p", [3, 4, 6, 12, 16])
+def test_sketch_sizes_few_blocks(p):
+    """Two blocks (n = 256) take the cooperative few-block sketch for every p it
+    serves: p = 4, 16 stage V with 16-byte loads, p = 3, 6, 12 element by
+    element with the unused columns of the widest staging zeroed.  alpha
+    trajectories within 1e-4 and the roots within 1e-5 of the oracle."""
+    n, batch = 256, 2
+    A = synth.spd_batch(n, batch, 1e-2, 1.0, 143)
+    S = synth.sketch_stack(60, n, p, 1043)
+    X, rep, opts = run_inv_root(A, "inv4", 2, p, 1e-6, 30, "3xtf32", S)
+    for b in range(batch):
+        assert rep["status"][b] == o.OK
+        it = rep["iters"][b]
+        Xo, infos = o.inv_root_ref(A[b], o.POW_INV4, oracle_opts(opts), S, force_iters=it)
+        for ps, info in enumerate(infos):
+            np.testing.assert_allclose(rep["alpha"][b, ps, :it[ps]], info.alpha, atol=1e-4)
+        assert relerr(X[b], Xo) <= 1e-5
+
+
 # Few blocks run one CTA per 128 x 128 tile; from about 74 tiles of 256 x 256
 # on (the SM pairs of a B200), the persistent CTA-pair kernel.  The ragged and
 # edge-case tests run both: a batch of 2 and a batch large enough for the pairs.
