@@ -1260,6 +1260,11 @@ cudaError_t gemm_tc(int mode, const Operand& A, const Operand& B, int M, int N, 
     if (2 * tiles < sms) {
       pair = false;
       BN = 128;
+      // a single block's product still leaves half the SMs idle at 128 x 128:
+      // 128 x 64 tiles (a symmetric result keeps 128 x 128 and its upper
+      // triangle)
+      const int64_t t128 = static_cast<int64_t>((N + 127) / 128) * ((M + 127) / 128) * batch;
+      if (!(ep.sym && M == N) && 2 * t128 <= sms) BN = 64;
     }
   }
   const int bn_cta = pair ? BN / 2 : BN;
