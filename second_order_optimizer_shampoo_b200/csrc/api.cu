@@ -311,7 +311,7 @@ std::mutex g_graph_mu;
 std::vector<CachedGraph> g_graphs;
 constexpr size_t kGraphCacheMax = 16;
 constexpr int kMaxDev = 64;
-cudaStream_t g_cap[kMaxDev][3] = {};
+cudaStream_t g_cap[kMaxDev][2] = {};  // the pass and its WHILE body
 
 // Adds a conditional node after the current capture frontier of `st`, makes
 // it the new frontier and returns its body graph.
@@ -391,7 +391,7 @@ int run_graph(CallKey key, Rec rec, cudaStream_t user) {
       return SHP_OK;
     }
   cudaStream_t* cs = g_cap[key.device];
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < 2; ++i)
     if (cs[i] == nullptr) CK(cudaStreamCreateWithFlags(&cs[i], cudaStreamNonBlocking));
   cudaGraph_t g = nullptr;
   CK(cudaGraphCreate(&g, 0));
