@@ -30,6 +30,7 @@ def test_header_constants_match_the_binding():
     the Python binding (the binding restates them, so drift would go silent)."""
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     found = dict(re.findall(r"\b(SHP_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    found.update(re.findall(r"#define\s+(SHP_[A-Z0-9_]+)\s+(\d+)\s*$", text, flags=re.M))
     m = re.search(r"#define\s+SHP_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
     assert m, "SHP_NOALLOC_SCRATCH_BYTES"
     found["SHP_NOALLOC_SCRATCH_BYTES"] = str(int(m.group(1)) << int(m.group(2)))
